@@ -1,0 +1,214 @@
+"""CPU oracle for the fused smooth-rotate-MXFP4 path -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline /
+reference legs may import this package.  The product path (the CUDA library
+and its Python binding) never imports or calls it, and the two share no code.
+
+The arithmetic lives in ``mxq_oracle.c`` (plain double-precision C, built with
+gcc, no fast-math, no FMA contraction); this module only marshals numpy arrays
+into it.  What each function computes, and the page passages it follows, is
+stated in the C file's header.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "mxq_oracle.c")
+_LIB = os.path.join(_HERE, "libmxq_oracle.so")
+
+GROUP = 32
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into ``oracle/libmxq_oracle.so`` (gcc, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=c11", "-fno-fast-math", "-ffp-contract=off", "-fopenmp",
+               "-shared", "-fPIC", "-o", _LIB + ".tmp", _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(_LIB + ".tmp", _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        I64 = ctypes.c_int64
+        I = ctypes.c_int
+        L.mxq_oracle_e2m1_code.argtypes = [ctypes.c_double]
+        L.mxq_oracle_e2m1_code.restype = I
+        L.mxq_oracle_e2m1_value.argtypes = [I]
+        L.mxq_oracle_e2m1_value.restype = ctypes.c_double
+        L.mxq_oracle_e8m0_byte.argtypes = [ctypes.c_double]
+        L.mxq_oracle_e8m0_byte.restype = I
+        L.mxq_oracle_e8m0_value.argtypes = [I]
+        L.mxq_oracle_e8m0_value.restype = ctypes.c_double
+        L.mxq_oracle_quantize_group_at.argtypes = [P, I, P, P, P]
+        L.mxq_oracle_quantize_group_at.restype = I
+        L.mxq_oracle_rotate_f64.argtypes = [P, I64, I64, P, P, P, I]
+        L.mxq_oracle_rotate_f64.restype = I
+        L.mxq_oracle_quantize.argtypes = [P, I64, I64, P, P, P, P, P, P, I]
+        L.mxq_oracle_quantize.restype = I
+        L.mxq_oracle_smooth_rotate_quantize.argtypes = [P, I64, I64, P, P, P, P, P, P, P, P, P, I]
+        L.mxq_oracle_smooth_rotate_quantize.restype = I
+        L.mxq_oracle_dequantize.argtypes = [P, P, I64, I64, P, P, P, P, I]
+        L.mxq_oracle_dequantize.restype = I
+        L.mxq_oracle_bf16_to_double.argtypes = [P, P, I64]
+        L.mxq_oracle_bf16_to_double.restype = None
+        L.mxq_oracle_double_to_bf16.argtypes = [P, P, I64]
+        L.mxq_oracle_double_to_bf16.restype = None
+        _lib = L
+    return _lib
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def default_threads() -> int:
+    return max(1, len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count() or 1)
+
+
+# ------------------------------------------------------------------ scalar rules
+
+def e2m1_code(u: float) -> int:
+    return int(lib().mxq_oracle_e2m1_code(float(u)))
+
+
+def e2m1_value(code: int) -> float:
+    return float(lib().mxq_oracle_e2m1_value(int(code)))
+
+
+def e8m0_byte(amax: float) -> int:
+    return int(lib().mxq_oracle_e8m0_byte(float(amax)))
+
+
+def e8m0_value(byte: int) -> float:
+    return float(lib().mxq_oracle_e8m0_value(int(byte)))
+
+
+def quantize_group_at(y, byte: int):
+    """Codes (unpacked, 32), element flags and alternative codes for one group at a given scale byte."""
+    y = _c(y, np.float64)
+    assert y.shape == (GROUP,)
+    codes = np.zeros(GROUP, np.uint8)
+    flags = np.zeros(GROUP, np.uint8)
+    alt = np.zeros(GROUP, np.uint8)
+    lib().mxq_oracle_quantize_group_at(_ptr(y), int(byte), _ptr(codes), _ptr(flags), _ptr(alt))
+    return codes, flags, alt
+
+
+# ------------------------------------------------------------------ matrices
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    bits = _c(bits, np.uint16)
+    out = np.empty(bits.shape, np.float64)
+    lib().mxq_oracle_bf16_to_double(_ptr(bits), _ptr(out), bits.size)
+    return out
+
+
+def f64_to_bf16_bits(v: np.ndarray) -> np.ndarray:
+    v = _c(v, np.float64)
+    out = np.empty(v.shape, np.uint16)
+    lib().mxq_oracle_double_to_bf16(_ptr(v), _ptr(out), v.size)
+    return out
+
+
+def rotate_f64(x: np.ndarray, r: np.ndarray, lam: Optional[np.ndarray] = None,
+               threads: int = 1) -> np.ndarray:
+    """Y = (X / lam) * R^, group by group, in double.  x: [rows, cols] float64, r: [32,32] [k][n]."""
+    x = _c(x, np.float64)
+    r = _c(r, np.float64)
+    rows, cols = x.shape
+    lam64 = None if lam is None else _c(lam, np.float64)
+    y = np.empty_like(x)
+    rc = lib().mxq_oracle_rotate_f64(_ptr(x), rows, cols, _ptr(r), _ptr(lam64), _ptr(y), threads)
+    if rc:
+        raise ValueError("oracle rotate: bad shape")
+    return y
+
+
+def quantize(y: np.ndarray, flags: bool = False, threads: int = 1) -> dict:
+    """Steps 4-8 on a [rows, cols] float64 matrix of rotated values."""
+    y = _c(y, np.float64)
+    rows, cols = y.shape
+    G = cols // GROUP
+    out = {"codes": np.zeros((rows, cols // 2), np.uint8), "scales": np.zeros((rows, G), np.uint8)}
+    if flags:
+        out.update(eflags=np.zeros((rows, cols), np.uint8), alt=np.zeros((rows, cols), np.uint8),
+                   gflags=np.zeros((rows, G), np.uint8), alt_scales=np.zeros((rows, G), np.uint8))
+    g = out.get
+    rc = lib().mxq_oracle_quantize(_ptr(y), rows, cols, _ptr(out["codes"]), _ptr(out["scales"]),
+                                   _ptr(g("eflags")), _ptr(g("alt")), _ptr(g("gflags")),
+                                   _ptr(g("alt_scales")), threads)
+    if rc:
+        raise ValueError("oracle quantize: bad shape")
+    return out
+
+
+def smooth_rotate_quantize(x_bits: np.ndarray, rhat_bits: np.ndarray, lam: Optional[np.ndarray] = None,
+                           want_y: bool = False, flags: bool = False, threads: int = 1) -> dict:
+    """The whole path from bf16 bit patterns: returns codes, scales (+ y, flags)."""
+    x_bits = _c(x_bits, np.uint16)
+    rhat_bits = _c(rhat_bits, np.uint16)
+    assert rhat_bits.shape == (GROUP, GROUP)
+    rows, cols = x_bits.shape
+    if cols % GROUP:
+        raise ValueError("cols must be a multiple of 32")
+    G = cols // GROUP
+    lam32 = None if lam is None else _c(lam, np.float32)
+    out = {"codes": np.zeros((rows, cols // 2), np.uint8), "scales": np.zeros((rows, G), np.uint8)}
+    if want_y:
+        out["y"] = np.zeros((rows, cols), np.float64)
+    if flags:
+        out.update(eflags=np.zeros((rows, cols), np.uint8), alt=np.zeros((rows, cols), np.uint8),
+                   gflags=np.zeros((rows, G), np.uint8), alt_scales=np.zeros((rows, G), np.uint8))
+    g = out.get
+    rc = lib().mxq_oracle_smooth_rotate_quantize(
+        _ptr(x_bits), rows, cols, _ptr(rhat_bits), _ptr(lam32), _ptr(out["codes"]), _ptr(out["scales"]),
+        _ptr(g("y")), _ptr(g("eflags")), _ptr(g("alt")), _ptr(g("gflags")), _ptr(g("alt_scales")), threads)
+    if rc:
+        raise ValueError("oracle: bad shape")
+    return out
+
+
+def dequantize(codes: np.ndarray, scales: np.ndarray, cols: int, rhat_bits: Optional[np.ndarray] = None,
+               lam: Optional[np.ndarray] = None, want_f64: bool = False, threads: int = 1):
+    """bf16 bit patterns of the dequantised matrix (and optionally the double before rounding)."""
+    codes = _c(codes, np.uint8)
+    scales = _c(scales, np.uint8)
+    rows = codes.shape[0]
+    assert codes.shape == (rows, cols // 2) and scales.shape == (rows, cols // GROUP)
+    rb = None if rhat_bits is None else _c(rhat_bits, np.uint16)
+    lam32 = None if lam is None else _c(lam, np.float32)
+    out = np.zeros((rows, cols), np.uint16)
+    f64 = np.zeros((rows, cols), np.float64) if want_f64 else None
+    rc = lib().mxq_oracle_dequantize(_ptr(codes), _ptr(scales), rows, cols, _ptr(rb), _ptr(lam32),
+                                     _ptr(out), _ptr(f64), threads)
+    if rc:
+        raise ValueError("oracle dequantize: bad shape")
+    return (out, f64) if want_f64 else out
+
+
+def unpack_codes(codes: np.ndarray) -> np.ndarray:
+    """[rows, cols/2] packed bytes -> [rows, cols] 4-bit codes (even column = low nibble)."""
+    codes = np.asarray(codes, np.uint8)
+    out = np.empty(codes.shape[:-1] + (codes.shape[-1] * 2,), np.uint8)
+    out[..., 0::2] = codes & 15
+    out[..., 1::2] = codes >> 4
+    return out

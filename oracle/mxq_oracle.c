@@ -1,0 +1,358 @@
+/*
+ * mxq_oracle.c -- CPU oracle for the DuQuant++ online smooth-rotate-MXFP4 step.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the
+ * benchmark's CPU-baseline leg may load this.  The CUDA path never calls it,
+ * and the two share no code, headers or tables.
+ *
+ * It is a plain, slow statement of what the path computes, in double
+ * precision.  It follows the DuQuant++ write-up "DuQuant++: block-aligned
+ * rotation quantisation for MXFP4 activation outliers" (jsqmd.com/news/928156):
+ *
+ *   smoothing  X -> X * Lambda^-1, a per-channel division          (§3.1, §3.3)
+ *   rotation   each 32-element group times one shared 32x32 R^ (X -> X * R^);
+ *              the block-diagonal operator is never formed          (§2.3, §3.2, §3.3)
+ *   MXFP4      absmax of the group -> shared power-of-two scale s_j ->
+ *              divide -> round to the nearest 4-bit float           (§2.1, §5.1 item 5)
+ *
+ * The write-up leaves the exact MXFP4 rule open.  This file takes the OCP
+ * Microscaling (MX) v1.0 reading:
+ *   - E8M0 exponent e = floor(log2(amax)) - 2, clamped to [-127, 127];
+ *   - code = E2M1 round-to-nearest with ties to the even code, |u| > 6 -> 6,
+ *     sign kept (so -0 and tiny negatives give code 0x8);
+ *   - amax NaN/Inf -> scale byte 0xFF and all codes 0;
+ *   - two codes per byte, the even column in the low nibble.
+ * The rotated values are rounded to fp32 before the scale and code decisions,
+ * the precision the CUDA kernel decides them in (the pages name none).
+ *
+ * Boundary flags (used by the parity tests to tell unique results from
+ * rounding-order ties):
+ *   element flag  ||u| - m| < 1e-3 * step(m) for a code midpoint m in
+ *                 {0, .25, .75, 1.25, 1.75, 2.5, 3.5, 5} (steps .5,.5,.5,.5,.5,1,1,2);
+ *                 the midpoint 0 separates +0 from -0;
+ *   group flag    |amax - 2^k| < 2.5e-4 * 2^k for the nearest power of two.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define GROUP 32
+
+/* ---------------------------------------------------------------- formats */
+
+/* bf16 bit pattern -> double (exact: bf16 is the top half of an IEEE single). */
+static double bf16_to_double(uint16_t b)
+{
+    uint32_t u = ((uint32_t)b) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* double -> bf16 bit pattern, one round-to-nearest-even step, overflow to Inf. */
+static uint16_t double_to_bf16(double v)
+{
+    if (isnan(v)) return 0x7FC0;
+    uint16_t sign = signbit(v) ? 0x8000 : 0;
+    double a = fabs(v);
+    if (a == 0.0) return sign;
+    if (isinf(a)) return sign | 0x7F80;
+    int ex;
+    frexp(a, &ex);                          /* a = f * 2^ex, f in [0.5, 1) */
+    int lead = ex - 1;                      /* a in [2^lead, 2^(lead+1)) */
+    if (lead < -126) lead = -126;           /* bf16 subnormals share fp32's floor */
+    double quantum = ldexp(1.0, lead - 7);  /* 8 significant bits */
+    double q = nearbyint(a / quantum) * quantum;   /* default mode: ties to even */
+    if (q >= ldexp(1.0, 128)) return sign | 0x7F80;
+    float f = (float)q;                     /* exact: q has <= 8 significant bits */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)(sign | ((u >> 16) & 0x7FFF));
+}
+
+/* E2M1 magnitudes of codes 0..7 (1 sign, 2 exponent, 1 mantissa bit; bias 1). */
+static const double E2M1_MAG[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+/* Midpoints between neighbouring magnitudes, the grid step there, and the two
+ * codes on either side.  Midpoint 0 separates +0 and -0. */
+static const double MID[8]  = {0.0, 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0};
+static const double STEP[8] = {0.5, 0.5, 0.5, 0.5, 0.5, 1.0, 1.0, 2.0};
+
+/* Round u to the nearest E2M1 value: nearest magnitude, ties to the even code,
+ * saturate above 6, keep the sign.  Returns the 4-bit code. */
+int mxq_oracle_e2m1_code(double u)
+{
+    int neg = signbit(u) ? 1 : 0;
+    double a = fabs(u);
+    int best = 0;
+    if (isnan(u)) return 0;
+    if (a >= E2M1_MAG[7]) {
+        best = 7;
+    } else {
+        double bestd = a;                   /* distance to magnitude 0 */
+        for (int c = 1; c < 8; ++c) {
+            double d = fabs(a - E2M1_MAG[c]);
+            /* strictly nearer wins; an exact tie goes to the even code */
+            if (d < bestd || (d == bestd && (c & 1) == 0)) {
+                best = c;
+                bestd = d;
+            }
+        }
+    }
+    return (neg << 3) | best;
+}
+
+/* Value of a 4-bit code. */
+double mxq_oracle_e2m1_value(int code)
+{
+    double m = E2M1_MAG[code & 7];
+    return (code & 8) ? -m : m;
+}
+
+/* Shared E8M0 byte for a group absmax (finite, >= 0): e = floor(log2 amax) - 2,
+ * clamped to [-127, 127]; byte = e + 127.  amax == 0 -> byte 0.  NaN/Inf -> 0xFF. */
+int mxq_oracle_e8m0_byte(double amax)
+{
+    if (isnan(amax) || isinf(amax)) return 0xFF;
+    if (amax == 0.0) return 0;
+    int ex;
+    frexp(amax, &ex);                       /* floor(log2 amax) = ex - 1 */
+    int e = (ex - 1) - 2;
+    if (e < -127) e = -127;
+    if (e > 127) e = 127;
+    return e + 127;
+}
+
+/* Value 2^(byte - 127) of a scale byte (byte 0xFF is NaN). */
+double mxq_oracle_e8m0_value(int byte)
+{
+    if (byte == 0xFF) return NAN;
+    return ldexp(1.0, byte - 127);
+}
+
+/* ------------------------------------------------------ one group, step by step */
+
+/* Quantise 32 rotated values y (already rounded to fp32) with a given scale
+ * byte.  Writes 32 unpacked codes and, if requested, the element boundary flag
+ * and the code on the other side of the flagged midpoint. */
+int mxq_oracle_quantize_group_at(const double *y, int byte, uint8_t *codes,
+                                 uint8_t *flags, uint8_t *alt)
+{
+    if (byte == 0xFF) {
+        for (int n = 0; n < GROUP; ++n) {
+            codes[n] = 0;
+            if (flags) flags[n] = 0;
+            if (alt) alt[n] = 0;
+        }
+        return 0;
+    }
+    int e = byte - 127;
+    for (int n = 0; n < GROUP; ++n) {
+        double u = ldexp(y[n], -e);         /* exact power-of-two scaling */
+        int c = mxq_oracle_e2m1_code(u);
+        codes[n] = (uint8_t)c;
+        if (flags || alt) {
+            double a = fabs(u);
+            int f = 0, other = c;
+            for (int m = 0; m < 8; ++m) {
+                if (fabs(a - MID[m]) < 1e-3 * STEP[m]) {
+                    f = 1;
+                    if (m == 0) {
+                        other = c ^ 8;      /* +0 <-> -0 */
+                    } else {
+                        int lo = m - 1, hi = m;   /* magnitudes either side */
+                        int mag = c & 7;
+                        other = (c & 8) | (mag == lo ? hi : lo);
+                    }
+                }
+            }
+            if (flags) flags[n] = (uint8_t)f;
+            if (alt) alt[n] = (uint8_t)other;
+        }
+    }
+    return 0;
+}
+
+/* Steps 4-8 for one group of double y: round to fp32, absmax, E8M0, codes,
+ * plus the boundary information. */
+static void quantize_group(const double *yin, uint8_t *codes_unpacked, uint8_t *byte_out,
+                           uint8_t *eflags, uint8_t *alt, uint8_t *gflag, uint8_t *alt_byte)
+{
+    double y[GROUP];
+    double amax = 0.0;
+    int bad = 0;
+    for (int n = 0; n < GROUP; ++n) {
+        y[n] = (double)(float)yin[n];       /* the decision precision: fp32 */
+        if (isnan(y[n]) || isinf(y[n])) bad = 1;
+        double a = fabs(y[n]);
+        if (a > amax) amax = a;
+    }
+    int byte = bad ? 0xFF : mxq_oracle_e8m0_byte(amax);
+    *byte_out = (uint8_t)byte;
+    mxq_oracle_quantize_group_at(y, byte, codes_unpacked, eflags, alt);
+
+    if (gflag || alt_byte) {
+        int f = 0, other = byte;
+        if (!bad && amax > 0.0) {
+            int ex;
+            frexp(amax, &ex);
+            double below = ldexp(1.0, ex - 1);      /* 2^floor(log2 amax) <= amax */
+            double above = ldexp(1.0, ex);          /* > amax */
+            if (amax - below < 2.5e-4 * below) {
+                f = 1;
+                other = mxq_oracle_e8m0_byte(below * (1.0 - 1e-9));
+            } else if (above - amax < 2.5e-4 * above) {
+                f = 1;
+                other = mxq_oracle_e8m0_byte(above);
+            }
+        }
+        if (gflag) *gflag = (uint8_t)f;
+        if (alt_byte) *alt_byte = (uint8_t)other;
+    }
+}
+
+/* ------------------------------------------------------------ whole matrices */
+
+/* Steps 2-3 on doubles: Y[r, 32g+n] = sum_k (X[r, 32g+k] / lam[32g+k]) * R[k][n].
+ * lam may be NULL (no smoothing).  R is row-major [k][n]. */
+int mxq_oracle_rotate_f64(const double *X, int64_t rows, int64_t cols, const double *R,
+                          const double *lam, double *Y, int nthreads)
+{
+    if (rows < 0 || cols < 0 || cols % GROUP) return 1;
+    int64_t G = cols / GROUP;
+#pragma omp parallel for schedule(static) num_threads(nthreads > 0 ? nthreads : 1)
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t g = 0; g < G; ++g) {
+            double x[GROUP];
+            for (int k = 0; k < GROUP; ++k) {
+                x[k] = X[r * cols + g * GROUP + k];
+                if (lam) x[k] = x[k] / lam[g * GROUP + k];
+            }
+            for (int n = 0; n < GROUP; ++n) {
+                double acc = 0.0;
+                for (int k = 0; k < GROUP; ++k) acc += x[k] * R[k * GROUP + n];
+                Y[r * cols + g * GROUP + n] = acc;
+            }
+        }
+    }
+    return 0;
+}
+
+/* Steps 4-8 for a whole matrix of rotated values.  Every output except codes
+ * and scales may be NULL.  codes: [rows, cols/2] packed (even column in the low
+ * nibble); scales: [rows, cols/32]; eflags/alt: [rows, cols] unpacked;
+ * gflags/alt_scales: [rows, cols/32]. */
+int mxq_oracle_quantize(const double *Y, int64_t rows, int64_t cols, uint8_t *codes,
+                        uint8_t *scales, uint8_t *eflags, uint8_t *alt, uint8_t *gflags,
+                        uint8_t *alt_scales, int nthreads)
+{
+    if (rows < 0 || cols < 0 || cols % GROUP) return 1;
+    int64_t G = cols / GROUP;
+#pragma omp parallel for schedule(static) num_threads(nthreads > 0 ? nthreads : 1)
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t g = 0; g < G; ++g) {
+            int64_t e0 = r * cols + g * GROUP;
+            uint8_t c[GROUP];
+            quantize_group(Y + e0, c, scales + r * G + g, eflags ? eflags + e0 : NULL,
+                           alt ? alt + e0 : NULL, gflags ? gflags + r * G + g : NULL,
+                           alt_scales ? alt_scales + r * G + g : NULL);
+            for (int i = 0; i < GROUP / 2; ++i)
+                codes[e0 / 2 + i] = (uint8_t)(c[2 * i] | (c[2 * i + 1] << 4));
+        }
+    }
+    return 0;
+}
+
+/* The whole path from bf16 inputs, one row at a time (no full-size double
+ * buffers): X bf16 [rows, cols], R bf16 [32][32] row-major [k][n], lam fp32
+ * [cols] or NULL.  Y (double [rows, cols]) and the flag outputs may be NULL. */
+int mxq_oracle_smooth_rotate_quantize(const uint16_t *X, int64_t rows, int64_t cols,
+                                      const uint16_t *Rb, const float *lam, uint8_t *codes,
+                                      uint8_t *scales, double *Y, uint8_t *eflags, uint8_t *alt,
+                                      uint8_t *gflags, uint8_t *alt_scales, int nthreads)
+{
+    if (rows < 0 || cols < 0 || cols % GROUP) return 1;
+    int64_t G = cols / GROUP;
+    double R[GROUP * GROUP];
+    for (int i = 0; i < GROUP * GROUP; ++i) R[i] = bf16_to_double(Rb[i]);
+#pragma omp parallel for schedule(dynamic, 4) num_threads(nthreads > 0 ? nthreads : 1)
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t g = 0; g < G; ++g) {
+            double x[GROUP], y[GROUP];
+            uint8_t c[GROUP];
+            int64_t e0 = r * cols + g * GROUP;
+            /* step 1-2: exact bf16 -> double, then the per-channel division */
+            for (int k = 0; k < GROUP; ++k) {
+                x[k] = bf16_to_double(X[e0 + k]);
+                if (lam) x[k] = x[k] / (double)lam[g * GROUP + k];
+            }
+            /* step 3: y = x * R^ */
+            for (int n = 0; n < GROUP; ++n) {
+                double acc = 0.0;
+                for (int k = 0; k < GROUP; ++k) acc += x[k] * R[k * GROUP + n];
+                y[n] = acc;
+                if (Y) Y[e0 + n] = acc;
+            }
+            /* steps 4-8 */
+            quantize_group(y, c, scales + r * G + g, eflags ? eflags + e0 : NULL,
+                           alt ? alt + e0 : NULL, gflags ? gflags + r * G + g : NULL,
+                           alt_scales ? alt_scales + r * G + g : NULL);
+            for (int i = 0; i < GROUP / 2; ++i)
+                codes[e0 / 2 + i] = (uint8_t)(c[2 * i] | (c[2 * i + 1] << 4));
+        }
+    }
+    return 0;
+}
+
+/* Dequantise: v = E2M1(code) * 2^(byte-127).  With R (bf16 [k][n]) the
+ * rotation is undone, x_k = sum_n v_n R[k][n], and with lam the smoothing too,
+ * x_k *= lam[k].  The exact double result is rounded once to bf16.  out_f64
+ * (optional) receives the double before rounding. */
+int mxq_oracle_dequantize(const uint8_t *codes, const uint8_t *scales, int64_t rows,
+                          int64_t cols, const uint16_t *Rb, const float *lam, uint16_t *out,
+                          double *out_f64, int nthreads)
+{
+    if (rows < 0 || cols < 0 || cols % GROUP) return 1;
+    int64_t G = cols / GROUP;
+    double R[GROUP * GROUP];
+    if (Rb)
+        for (int i = 0; i < GROUP * GROUP; ++i) R[i] = bf16_to_double(Rb[i]);
+#pragma omp parallel for schedule(static) num_threads(nthreads > 0 ? nthreads : 1)
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t g = 0; g < G; ++g) {
+            int64_t e0 = r * cols + g * GROUP;
+            double s = mxq_oracle_e8m0_value(scales[r * G + g]);
+            double v[GROUP], x[GROUP];
+            for (int n = 0; n < GROUP; ++n) {
+                int byte = codes[(e0 + n) / 2];
+                int code = (n & 1) ? (byte >> 4) : (byte & 15);
+                v[n] = mxq_oracle_e2m1_value(code) * s;
+            }
+            for (int k = 0; k < GROUP; ++k) {
+                if (Rb) {
+                    double acc = 0.0;
+                    for (int n = 0; n < GROUP; ++n) acc += v[n] * R[k * GROUP + n];
+                    x[k] = acc;
+                } else {
+                    x[k] = v[k];
+                }
+                if (lam) x[k] = x[k] * (double)lam[g * GROUP + k];
+                out[e0 + k] = double_to_bf16(x[k]);
+                if (out_f64) out_f64[e0 + k] = x[k];
+            }
+        }
+    }
+    return 0;
+}
+
+/* Exposed for the pins: exact bf16 <-> double conversions. */
+void mxq_oracle_bf16_to_double(const uint16_t *b, double *d, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) d[i] = bf16_to_double(b[i]);
+}
+
+void mxq_oracle_double_to_bf16(const double *d, uint16_t *b, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) b[i] = double_to_bf16(d[i]);
+}
