@@ -1,0 +1,376 @@
+#!/usr/bin/env python3
+"""Benchmark of the fused smooth-rotate-MXFP4 path on B200.
+
+One step = one pass of the whole hot path over one batch: a single launch of
+the fused kernel.  That launch loads X, applies the optional smoothing, the
+32x32 rotation on the tensor cores, the absmax, the E8M0 scale, the E2M1
+rounding and the packed stores.  The workload is the down-projection input,
+8192 x 14336 bf16: Student-t(3) entries, 8 tokens carrying 1e3-1e4 outliers in
+4 channels, a random orthogonal R̂, no smoothing.
+
+Metric: GB/s of algorithmic traffic per step.  That is 2 B of bf16 read plus
+0.5 B of codes and 1/32 B of scale written, per element: 2.53125 B/elem.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mine|reference]
+
+With N > 1, launch it under torch.distributed.run, one rank per GPU.  Each rank
+quantises its own batch of the same shape (weak scaling, no collective on the
+data path).  The timing is the max over ranks.  ``--impl reference`` times the
+CPU oracle on the host cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import synth  # noqa: E402
+
+CFG = 3
+ROWS, COLS = synth.CONFIG_SHAPES[CFG]
+BYTES_PER_ELEM = 2.0 + 0.5 + 1.0 / 32.0
+METRIC = "rotate+MXFP4-quantize GB/s and % of HBM roofline, 1×B200, down-proj shape"
+UNIT = "GB/s"
+WORKLOAD = ("down-proj input 8192x14336 bf16 (Student-t(3), 8 tokens x 4 channels of 1e3-1e4 outliers), "
+            "random orthogonal 32x32 R, no smoothing -> MXFP4 codes + E8M0 scales")
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = ["mxfp4_block_rotation_b200/csrc/rotquant_sm100.cu",
+                  "mxfp4_block_rotation_b200/csrc/sm100_ptx.cuh"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "rotate_kernel_downproj_traffic.json")
+
+
+def algorithmic_bytes(rows: int, cols: int) -> float:
+    return rows * cols * BYTES_PER_ELEM
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def recorded_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if the kernel source is unchanged."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if rec.get("kernel_source_sha256") != kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sms, maxes, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sms.append(float(parts[1]))
+                    maxes.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for name, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(name)
+        os.unlink(self.path)
+        if not sms:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        busy = [s for s in sms if s > 0.5 * max(sms)] or sms
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": max(maxes), "reasons": sorted(reasons),
+                "samples": len(sms)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle leg
+
+def oracle_rate(x_bits: np.ndarray, rhat_bits: np.ndarray, target_s: float, threads: int):
+    """Time the oracle on a row sample sized for about target_s seconds (whole passes over the
+    workload are repeated if one pass is shorter); returns (GB/s, elements processed, seconds)."""
+    import oracle
+    probe = min(x_bits.shape[0], max(8, threads * 2))
+    t0 = time.perf_counter()
+    oracle.smooth_rotate_quantize(x_bits[:probe], rhat_bits, None, threads=threads)
+    dt = max(time.perf_counter() - t0, 1e-6)
+    n = int(min(x_bits.shape[0], max(probe, probe * target_s / dt)))
+    done, t0 = 0, time.perf_counter()
+    while True:
+        oracle.smooth_rotate_quantize(x_bits[:n], rhat_bits, None, threads=threads)
+        done += n
+        dt = time.perf_counter() - t0
+        if dt >= 0.5 * target_s:
+            break
+    return algorithmic_bytes(done, x_bits.shape[1]) / dt / 1e9, done * x_bits.shape[1], dt
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    w = synth.make_config(CFG)
+    xb = synth.bf16_bits(w.x)
+    rb = synth.bf16_bits(w.rhat)
+    threads = host_cores()
+    per_step_s = max(1.0, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+    probe = min(ROWS, max(8, threads * 2))
+    t0 = time.perf_counter()
+    oracle.smooth_rotate_quantize(xb[:probe], rb, None, threads=threads)
+    n_rows = int(min(ROWS, max(probe, probe * per_step_s / max(time.perf_counter() - t0, 1e-6))))
+    times = []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        oracle.smooth_rotate_quantize(xb[:n_rows], rb, None, threads=threads)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    sec = sum(times) / len(times)
+    value = algorithmic_bytes(n_rows, COLS) / sec / 1e9
+    sample = f"first {n_rows} of {ROWS} rows of the workload per step ({n_rows * COLS} elements)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "rows": ROWS, "cols": COLS, "lambda": None},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU leg
+
+def run_mine(args):
+    import mxfp4_block_rotation_b200 as mxq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}; launch N>1 under torch.distributed.run")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    w = synth.make_config(CFG)
+    rows, cols = w.rows, w.cols
+    n_bytes = algorithmic_bytes(rows, cols)
+    # two input/output sets alternated: each X (235 MB) already exceeds the 126 MB L2
+    xs = [w.x.to(dev), w.x.to(dev)]
+    rhat = w.rhat.to(dev)
+    outs = [(torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev),
+             torch.empty((rows, cols // 32), dtype=torch.uint8, device=dev)) for _ in range(2)]
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        c, s = outs[i & 1]
+        mxq.smooth_rotate_quantize(xs[i & 1], rhat, None, codes=c, scales=s, stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    mxq.sync_check()
+
+    k = args.steps
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(k)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(k)]
+    t_begin = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        t_begin.record(stream)
+        for i in range(k):
+            ev_s[i].record(stream)
+            step(i)
+            ev_e[i].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+        if dist is not None:
+            dist.barrier()
+    mxq.sync_check()
+    total_ms = t_begin.elapsed_time(t_end)
+    kern_ms = [a.elapsed_time(b) for a, b in zip(ev_s, ev_e)]
+    t = torch.tensor([total_ms, sum(kern_ms) / k], dtype=torch.float64, device=dev)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, kern_avg_ms = float(t[0]), float(t[1])
+    ms_per_step = total_ms / k
+    value = world * n_bytes / (ms_per_step * 1e-3) / 1e9
+
+    # end to end through the public API: pinned host X -> device -> kernel -> codes/scales back to host
+    e2e = run_e2e(mxq, w, rhat, dev, stream, args, dist)
+
+    if rank == 0:
+        peak, peak_kind = hbm_peak()
+        achieved = n_bytes / (kern_avg_ms * 1e-3) / 1e9
+        traffic = recorded_traffic()
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": k, "warmup": args.warmup,
+            "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "rows": rows, "cols": cols, "lambda": None,
+                       "elements_per_gpu": rows * cols, "bytes_per_step_per_gpu": n_bytes,
+                       "l2": "inputs larger than L2: two 235 MB X buffers alternated (L2 126 MB)",
+                       "parallelism": f"dp{world} (independent row batches, no collective)"},
+            "elements_per_s": world * rows * cols / (ms_per_step * 1e-3),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+                         if peak_kind == "measured" else "fallback 6.65 TB/s",
+                         "kernel": "rotate_kernel<no smoothing, quantize>", "kernel_ms": kern_avg_ms},
+            "e2e": e2e,
+            "gpu_launches": k,
+            "clocks": clocks.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            import oracle
+            oracle.build()
+            threads = host_cores()
+            gbs, n_el, sec = oracle_rate(synth.bf16_bits(w.x), synth.bf16_bits(w.rhat), args.cpu_seconds,
+                                         threads)
+            line["cpu_baseline"] = {"value": gbs, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                    "sample": f"{n_el} elements (leading rows of the workload, whole "
+                                              f"passes repeated) in {sec:.1f} s of oracle time"}
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def run_e2e(mxq, w, rhat, dev, stream, args, dist):
+    rows, cols = w.rows, w.cols
+    x_host = w.x.pin_memory()
+    c_host = torch.empty((rows, cols // 2), dtype=torch.uint8).pin_memory()
+    s_host = torch.empty((rows, cols // 32), dtype=torch.uint8).pin_memory()
+    x_dev = torch.empty_like(x_host, device=dev)
+    c_dev = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+    s_dev = torch.empty((rows, cols // 32), dtype=torch.uint8, device=dev)
+
+    def step():
+        x_dev.copy_(x_host, non_blocking=True)
+        mxq.smooth_rotate_quantize(x_dev, rhat, None, codes=c_dev, scales=s_dev, stream=stream)
+        c_host.copy_(c_dev, non_blocking=True)
+        s_host.copy_(s_dev, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    k = max(3, args.steps // 2)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    a.record(stream)
+    for _ in range(k):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = a.elapsed_time(b) / k
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    world = 1
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        world = dist.get_world_size()
+    ms = float(t[0])
+    return {"value": world * algorithmic_bytes(rows, cols) / (ms * 1e-3) / 1e9, "unit": UNIT,
+            "h2d_bytes_per_step": x_host.numel() * 2,
+            "d2h_bytes_per_step": c_host.numel() + s_host.numel(), "ms_per_step": ms, "steps": k}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["mine", "reference"], default="mine")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="oracle time for the cpu_baseline sample (rank 0, N=1 only)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_mine(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,161 @@
+/*
+ * mxq.h -- C ABI of the B200 (sm_100a) fused smooth-rotate-MXFP4 library, libmxq.so.
+ *
+ * The operation is the online step of DuQuant++ as the write-up "DuQuant++:
+ * block-aligned rotation quantisation for MXFP4 activation outliers"
+ * (jsqmd.com/news/928156) describes it.
+ *   - Each activation row is cut into 32-element MXFP4 groups (§2.1, §2.3).
+ *   - Every group is divided per channel by the SmoothQuant scale Lambda
+ *     (§3.1; online it is X * Lambda^-1, §3.3).
+ *   - It is then multiplied by one shared, outlier-aware 32x32 orthogonal
+ *     matrix R^, i.e. X -> X * R^ (§2.3, §3.2 step 4, §3.3).  No permutation
+ *     and no second rotation.
+ *   - Last, the group is quantised to MXFP4 (§2.1, §5.1 item 5).  One shared
+ *     power-of-two scale per group comes from its absmax, and each element is
+ *     rounded to the nearest 4-bit float.
+ * §5.2 item 1 and §5.4 item 3 ask for the smoothing and the rotation to be
+ * fused into one kernel ahead of the MXFP4 linear layer.  Here the
+ * quantisation is fused in as well.
+ *
+ * MXFP4 rule (the OCP Microscaling v1.0 reading of §2.1; the page gives none):
+ *   amax  = max_n |y_n| over the group's 32 rotated fp32 values
+ *   e     = clamp(floor(log2 amax) - 2, -127, 127); amax == 0 gives e = -127
+ *   scale byte (E8M0) = e + 127; a NaN/Inf amax gives byte 0xFF and all codes 0
+ *   code_n = E2M1(y_n * 2^-e): round to nearest, ties to the even code,
+ *            |.| > 6 saturates to 6, sign kept (-0 and tiny negatives -> 0x8)
+ *   E2M1 codes 0..7 = magnitudes {0, 0.5, 1, 1.5, 2, 3, 4, 6}; bit 3 = sign.
+ *
+ * Layouts (all row-major, no padding between rows):
+ *   X       bf16  [rows, cols]           cols % 32 == 0
+ *   R^      bf16  [32, 32]               R^[k][n]: y_n = sum_k x_k * R^[k][n]
+ *   Lambda  fp32  [cols] or NULL         strictly positive and finite; NULL = no smoothing
+ *   codes   uint8 [rows, cols/2]         byte i of a row holds column 2i in its low
+ *                                        nibble and column 2i+1 in its high nibble
+ *   scales  uint8 [rows, cols/32]        one E8M0 byte per group
+ *
+ * Common rules for every entry point below.
+ *   Memory.  All pointers are device memory owned by the caller (for example
+ *     from PyTorch).  The library allocates nothing, keeps no per-call state
+ *     and may be called from several host threads.
+ *   Streams.  `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is queued on it asynchronously; the call returns right
+ *     after the launch.
+ *   Errors.  Bad arguments return MXQ_ERR_INVALID_ARG before anything is
+ *     launched.  That covers NULL pointers where one is required, negative
+ *     sizes, cols % 32 != 0, misaligned pointers, pointers that are not device
+ *     memory of the current device, and outputs that overlap inputs.
+ *     rows == 0 or cols == 0 is a valid no-op (pointers are then not looked at).
+ *     Launch failures return MXQ_ERR_CUDA.
+ *     Faults during execution surface at the caller's next synchronisation.
+ *   Bounded waits.  The kernels' internal pipeline waits are bounded.  If one
+ *     runs out, the kernel records MXQ_ERR_TIMEOUT in a device status word and
+ *     returns early; its outputs are then undefined.  mxq_sync_check() reads
+ *     and clears that word.
+ *   Contract on values.  Results are defined for finite inputs whose rotated
+ *     values are finite in fp32.  Inf/NaN inputs give scale byte 0xFF for the
+ *     groups they reach.
+ */
+#ifndef MXQ_H
+#define MXQ_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MXQ_OK = 0,
+    MXQ_ERR_INVALID_ARG = 1,   /* rejected before launch; nothing was queued */
+    MXQ_ERR_UNSUPPORTED = 2,   /* device is not sm_100 or lacks the needed shared memory */
+    MXQ_ERR_CUDA = 3,          /* a CUDA runtime/driver call or the launch failed */
+    MXQ_ERR_TIMEOUT = 4        /* a kernel's bounded pipeline wait ran out (see mxq_sync_check) */
+} mxq_status;
+
+/*
+ * Fused smooth -> rotate -> MXFP4 quantise (DuQuant++ write-up §3.3 online
+ * step X * Lambda^-1 * R^, followed by §2.1's MXFP4 quantiser).
+ *
+ *   X_bf16              in   bf16 [rows, cols], 16-byte aligned
+ *   rows, cols          in   rows >= 0; cols >= 0 and cols % 32 == 0
+ *   Rhat_bf16           in   bf16 [32, 32] row-major [k][n], 2-byte aligned
+ *   Lambda_or_null      in   fp32 [cols], 4-byte aligned, or NULL for no smoothing
+ *   out_codes_u8_packed out  uint8 [rows, cols/2], 16-byte aligned
+ *   out_scales_e8m0     out  uint8 [rows, cols/32], any alignment
+ *   stream              in   cudaStream_t
+ *
+ * The rotation runs on the tensor cores.  X is the exact bf16 A operand and
+ * R^ (or, with Lambda, diag(1/Lambda)·R^ split into a bf16 high part and a
+ * bf16 low part) is the B operand, with fp32 accumulation.  The scale and the
+ * codes are then decided on those fp32 values.
+ */
+mxq_status mxq_smooth_rotate_quantize(const void *X_bf16, int64_t rows, int64_t cols,
+                                      const void *Rhat_bf16, const float *Lambda_or_null,
+                                      uint8_t *out_codes_u8_packed, uint8_t *out_scales_e8m0,
+                                      void *stream);
+
+/*
+ * Same inputs as mxq_smooth_rotate_quantize.  Writes the rotated fp32 values
+ * Y = X * Lambda^-1 * R^ (§3.3) instead of quantising them.  It checks the
+ * intermediate precision; the quantiser decides on these same values.
+ *
+ *   out_f32             out  fp32 [rows, cols], 16-byte aligned
+ */
+mxq_status mxq_smooth_rotate_f32(const void *X_bf16, int64_t rows, int64_t cols,
+                                 const void *Rhat_bf16, const float *Lambda_or_null,
+                                 float *out_f32, void *stream);
+
+/*
+ * MXFP4 dequantise: the fake-quant "simulator" of the write-up's §5.1 item 5.
+ * Each value is v = E2M1(code) * 2^(byte - 127), with byte 0xFF giving NaN.
+ *
+ *   codes, scales       in   as produced above; codes 16-byte aligned
+ *   rows, cols          in   as above
+ *   Rhat_bf16_or_null   in   NULL: write v itself.  It is exactly representable
+ *                            in bf16, so the output is bit-exact (overflow
+ *                            gives +-Inf).
+ *                            non-NULL: undo the rotation, x_k = sum_n v_n R^[k][n]
+ *                            (v * R^T), with fp32 accumulation.
+ *   Lambda_or_null      in   non-NULL: undo the smoothing too, x_k *= Lambda[k]
+ *                            (allowed only together with R^)
+ *   out_bf16            out  bf16 [rows, cols], 16-byte aligned; the fp32 result
+ *                            rounded to nearest even
+ */
+mxq_status mxq_dequantize(const uint8_t *codes, const uint8_t *scales, int64_t rows,
+                          int64_t cols, const void *Rhat_bf16_or_null,
+                          const float *Lambda_or_null, void *out_bf16, void *stream);
+
+/*
+ * Synchronise `stream` and then read and clear the device status word.
+ * Returns MXQ_ERR_CUDA if the stream reported an error and MXQ_ERR_TIMEOUT if
+ * a kernel's bounded wait ran out since the last check; otherwise MXQ_OK.
+ */
+mxq_status mxq_sync_check(void *stream);
+
+/*
+ * Diagnostic for the failure-detection path (no counterpart on the pages).
+ * Queues one single-thread kernel on `stream`.  It waits on a shared-memory
+ * barrier that nothing ever completes, using the same bounded wait as the
+ * fused kernel's pipeline.  After `timeout_ms` (1..10000) the wait gives up: it
+ * sets MXQ_ERR_TIMEOUT in the device status word and writes 2 to
+ * *result_device.  A following mxq_sync_check() then returns MXQ_ERR_TIMEOUT
+ * and clears the word.  No GPU fault, trap or hang is involved.
+ *
+ *   result_device   out  one int of device memory, 4-byte aligned
+ */
+mxq_status mxq_selftest_bounded_wait(uint32_t timeout_ms, int *result_device, void *stream);
+
+/* A static, human-readable string for a status code (never NULL). */
+const char *mxq_status_string(mxq_status status);
+
+/* The text of the last CUDA error this thread saw inside the library (static storage). */
+const char *mxq_last_cuda_error(void);
+
+/* Library ABI version: major * 10000 + minor * 100 + patch. */
+int mxq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MXQ_H */

@@ -1,0 +1,208 @@
+"""Fused smooth-rotate-MXFP4 quantisation for B200 (sm_100a): Python binding.
+
+This module only marshals arguments into the C ABI of ``libmxq.so`` (declared in
+``include/mxq.h``).  Every step of the path runs in the library's CUDA kernels:
+the per-channel smoothing, the 32x32 block rotation, the scale and code
+decisions and the packing.  There is no CPU or PyTorch fallback.  If the
+library is missing or the device is not supported, the calls raise.
+
+The method is the online step of DuQuant++ (jsqmd.com/news/928156, §2.1, §2.3,
+§3.3).  Each 32-element group of an activation row is divided per channel by Λ,
+multiplied by one shared orthogonal 32x32 matrix R̂, and quantised to MXFP4.
+MXFP4 here means one E8M0 scale per group and E2M1 codes, two per byte, the
+even column in the low nibble.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional, Tuple
+
+import torch
+
+__all__ = [
+    "MxqError", "smooth_rotate_quantize", "smooth_rotate_f32", "dequantize", "sync_check",
+    "selftest_bounded_wait",
+    "status_string", "version", "lib", "LIB_PATH", "HEADER_PATH", "declared_symbols",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmxq.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "mxq.h")
+
+MXQ_OK = 0
+_STATUS_NAMES = {0: "MXQ_OK", 1: "MXQ_ERR_INVALID_ARG", 2: "MXQ_ERR_UNSUPPORTED", 3: "MXQ_ERR_CUDA",
+                 4: "MXQ_ERR_TIMEOUT"}
+
+
+class MxqError(RuntimeError):
+    """A libmxq call returned a status other than MXQ_OK."""
+
+    def __init__(self, status: int, where: str, detail: str = ""):
+        self.status = status
+        super().__init__(f"{where}: {_STATUS_NAMES.get(status, status)}" + (f" ({detail})" if detail else ""))
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmxq.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise MxqError(3, "load", f"{LIB_PATH} is missing; build it with "
+                                      "`python -m mxfp4_block_rotation_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+        L.mxq_smooth_rotate_quantize.argtypes = [P, I64, I64, P, P, P, P, P]
+        L.mxq_smooth_rotate_quantize.restype = I
+        L.mxq_smooth_rotate_f32.argtypes = [P, I64, I64, P, P, P, P]
+        L.mxq_smooth_rotate_f32.restype = I
+        L.mxq_dequantize.argtypes = [P, P, I64, I64, P, P, P, P]
+        L.mxq_dequantize.restype = I
+        L.mxq_selftest_bounded_wait.argtypes = [ctypes.c_uint32, P, P]
+        L.mxq_selftest_bounded_wait.restype = I
+        L.mxq_sync_check.argtypes = [P]
+        L.mxq_sync_check.restype = I
+        L.mxq_status_string.argtypes = [I]
+        L.mxq_status_string.restype = ctypes.c_char_p
+        L.mxq_last_cuda_error.argtypes = []
+        L.mxq_last_cuda_error.restype = ctypes.c_char_p
+        L.mxq_version.argtypes = []
+        L.mxq_version.restype = I
+        _lib = L
+    return _lib
+
+
+def declared_symbols() -> list[str]:
+    """Names of the functions include/mxq.h declares."""
+    with open(HEADER_PATH) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mxq_[a-z0-9_]+)\s*\(", text)))
+
+
+def status_string(status: int) -> str:
+    return lib().mxq_status_string(int(status)).decode()
+
+
+def version() -> int:
+    return int(lib().mxq_version())
+
+
+def _check(status: int, where: str) -> None:
+    if status != MXQ_OK:
+        raise MxqError(status, where, lib().mxq_last_cuda_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device: torch.device, stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, device: torch.device) -> None:
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _inputs(x, rhat, lam):
+    if x.dim() != 2:
+        raise ValueError("x must be 2-D [rows, cols]")
+    dev = x.device
+    if dev.type != "cuda":
+        raise ValueError("x must be a CUDA tensor (this library has no CPU path)")
+    _need(x, "x", torch.bfloat16, dev)
+    _need(rhat, "rhat", torch.bfloat16, dev)
+    if tuple(rhat.shape) != (32, 32):
+        raise ValueError("rhat must be [32, 32]")
+    if lam is not None:
+        _need(lam, "lam", torch.float32, dev)
+        if tuple(lam.shape) != (x.shape[1],):
+            raise ValueError("lam must be [cols]")
+    return dev
+
+
+def smooth_rotate_quantize(x: torch.Tensor, rhat: torch.Tensor, lam: Optional[torch.Tensor] = None, *,
+                           codes: Optional[torch.Tensor] = None, scales: Optional[torch.Tensor] = None,
+                           stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """MXFP4(X · Λ⁻¹ · R̂) -> (codes uint8 [rows, cols/2], scales uint8 [rows, cols/32])."""
+    dev = _inputs(x, rhat, lam)
+    rows, cols = x.shape
+    if codes is None:
+        codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+    if scales is None:
+        scales = torch.empty((rows, cols // 32), dtype=torch.uint8, device=dev)
+    _need(codes, "codes", torch.uint8, dev)
+    _need(scales, "scales", torch.uint8, dev)
+    st = lib().mxq_smooth_rotate_quantize(_ptr(x), rows, cols, _ptr(rhat), _ptr(lam), _ptr(codes),
+                                          _ptr(scales), _stream(dev, stream))
+    _check(st, "mxq_smooth_rotate_quantize")
+    return codes, scales
+
+
+def smooth_rotate_f32(x: torch.Tensor, rhat: torch.Tensor, lam: Optional[torch.Tensor] = None, *,
+                      out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """X · Λ⁻¹ · R̂ in fp32 [rows, cols] (the values the quantiser decides on)."""
+    dev = _inputs(x, rhat, lam)
+    rows, cols = x.shape
+    if out is None:
+        out = torch.empty((rows, cols), dtype=torch.float32, device=dev)
+    _need(out, "out", torch.float32, dev)
+    st = lib().mxq_smooth_rotate_f32(_ptr(x), rows, cols, _ptr(rhat), _ptr(lam), _ptr(out),
+                                     _stream(dev, stream))
+    _check(st, "mxq_smooth_rotate_f32")
+    return out
+
+
+def dequantize(codes: torch.Tensor, scales: torch.Tensor, rhat: Optional[torch.Tensor] = None,
+               lam: Optional[torch.Tensor] = None, *, out: Optional[torch.Tensor] = None,
+               stream=None) -> torch.Tensor:
+    """bf16 [rows, cols] from MXFP4 codes/scales; with rhat (and lam) the transform is undone."""
+    if codes.dim() != 2 or scales.dim() != 2:
+        raise ValueError("codes and scales must be 2-D")
+    dev = codes.device
+    if dev.type != "cuda":
+        raise ValueError("codes must be a CUDA tensor (this library has no CPU path)")
+    rows, half = codes.shape
+    cols = half * 2
+    _need(codes, "codes", torch.uint8, dev)
+    _need(scales, "scales", torch.uint8, dev)
+    if tuple(scales.shape) != (rows, cols // 32):
+        raise ValueError("scales must be [rows, cols/32]")
+    if rhat is not None:
+        _need(rhat, "rhat", torch.bfloat16, dev)
+    if lam is not None:
+        _need(lam, "lam", torch.float32, dev)
+    if out is None:
+        out = torch.empty((rows, cols), dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, dev)
+    st = lib().mxq_dequantize(_ptr(codes), _ptr(scales), rows, cols, _ptr(rhat), _ptr(lam), _ptr(out),
+                              _stream(dev, stream))
+    _check(st, "mxq_dequantize")
+    return out
+
+
+def selftest_bounded_wait(timeout_ms: int = 50, device=None, stream=None) -> int:
+    """Run the bounded-wait diagnostic kernel; returns its result code (2 = wait ran out as designed)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    res = torch.zeros(1, dtype=torch.int32, device=dev)
+    _check(lib().mxq_selftest_bounded_wait(int(timeout_ms), _ptr(res), _stream(dev, stream)),
+           "mxq_selftest_bounded_wait")
+    return int(res.item())
+
+
+def sync_check(stream=None, device=None) -> None:
+    """Synchronise the stream and raise if a kernel's bounded wait ran out or the stream failed."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    _check(lib().mxq_sync_check(_stream(dev, stream)), "mxq_sync_check")

@@ -1,0 +1,327 @@
+// mxq_api.cu -- the C ABI of libmxq.so (declared in include/mxq.h).
+//
+// Host-side layer only.  It validates arguments so that a bad call cannot reach
+// the GPU: sizes, alignment, device residency and extent of every buffer,
+// overlap of outputs with inputs.  It then builds the TMA descriptor over X
+// and launches the kernels on the caller's stream.  It allocates no device
+// memory and keeps no per-call state.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/mxq.h"
+#include "mxq_internal.h"
+
+namespace {
+
+thread_local char g_last_error[256] = "no error";
+
+void note_cuda(cudaError_t e, const char *where)
+{
+    std::snprintf(g_last_error, sizeof g_last_error, "%s: %s (%d)", where, cudaGetErrorString(e),
+                  static_cast<int>(e));
+}
+
+void note_cu(CUresult r, const char *where)
+{
+    std::snprintf(g_last_error, sizeof g_last_error, "%s: CUresult %d", where, static_cast<int>(r));
+}
+
+// Driver entry points, fetched through the runtime (no link against libcuda).
+struct Driver {
+    PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    PFN_cuPointerGetAttributes_v7000 ptr_attrs = nullptr;
+    bool ok = false;
+};
+
+const Driver &driver()
+{
+    static Driver d;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q1, q2;
+        void *p1 = nullptr, *p2 = nullptr;
+        cudaError_t e1 = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p1, 12000,
+                                                          cudaEnableDefault, &q1);
+        cudaError_t e2 = cudaGetDriverEntryPointByVersion("cuPointerGetAttributes", &p2, 7000,
+                                                          cudaEnableDefault, &q2);
+        if (e1 == cudaSuccess && e2 == cudaSuccess && q1 == cudaDriverEntryPointSuccess &&
+            q2 == cudaDriverEntryPointSuccess) {
+            d.encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p1);
+            d.ptr_attrs = reinterpret_cast<PFN_cuPointerGetAttributes_v7000>(p2);
+            d.ok = true;
+        }
+    });
+    return d;
+}
+
+struct DeviceInfo {
+    std::atomic<int> state{0};   // 0 unknown, 1 supported, 2 unsupported
+    int num_sms = 0;
+};
+DeviceInfo g_dev[64];
+
+// Resolve the current device and check it is an sm_100 part.
+mxq_status current_device(int *dev_out, int *sms_out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        note_cuda(e, "cudaGetDevice");
+        return MXQ_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= 64) return MXQ_ERR_UNSUPPORTED;
+    DeviceInfo &info = g_dev[dev];
+    if (info.state.load(std::memory_order_acquire) == 0) {
+        int major = 0, sms = 0, optin = 0;
+        if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) {
+            note_cuda(e, "cudaDeviceGetAttribute");
+            return MXQ_ERR_CUDA;
+        }
+        info.num_sms = sms;
+        info.state.store((major == 10 && optin >= 210 * 1024) ? 1 : 2, std::memory_order_release);
+    }
+    if (info.state.load(std::memory_order_acquire) != 1) return MXQ_ERR_UNSUPPORTED;
+    *dev_out = dev;
+    *sms_out = info.num_sms;
+    return MXQ_OK;
+}
+
+// [p, p + bytes) must be device (or managed) memory of `dev`, inside one allocation.
+mxq_status check_buffer(const void *p, uint64_t bytes, int dev)
+{
+    const Driver &d = driver();
+    if (!d.ok) {
+        std::snprintf(g_last_error, sizeof g_last_error, "driver entry points unavailable");
+        return MXQ_ERR_CUDA;
+    }
+    unsigned int mem_type = 0;
+    int ordinal = -1;
+    CUdeviceptr start = 0;
+    size_t size = 0;
+    CUpointer_attribute attrs[4] = {CU_POINTER_ATTRIBUTE_MEMORY_TYPE, CU_POINTER_ATTRIBUTE_DEVICE_ORDINAL,
+                                    CU_POINTER_ATTRIBUTE_RANGE_START_ADDR, CU_POINTER_ATTRIBUTE_RANGE_SIZE};
+    void *data[4] = {&mem_type, &ordinal, &start, &size};
+    CUresult r = d.ptr_attrs(4, attrs, data, reinterpret_cast<CUdeviceptr>(p));
+    if (r != CUDA_SUCCESS) {
+        note_cu(r, "cuPointerGetAttributes");
+        return MXQ_ERR_INVALID_ARG;
+    }
+    if (mem_type != CU_MEMORYTYPE_DEVICE || ordinal != dev) {
+        std::snprintf(g_last_error, sizeof g_last_error, "pointer %p is not device memory of device %d", p, dev);
+        return MXQ_ERR_INVALID_ARG;
+    }
+    const uint64_t a = reinterpret_cast<uint64_t>(p);
+    if (start != 0 && size != 0 && (a < start || a + bytes > start + size)) {
+        std::snprintf(g_last_error, sizeof g_last_error, "buffer %p + %llu B overruns its allocation", p,
+                      static_cast<unsigned long long>(bytes));
+        return MXQ_ERR_INVALID_ARG;
+    }
+    return MXQ_OK;
+}
+
+bool overlaps(const void *a, uint64_t na, const void *b, uint64_t nb)
+{
+    const uint64_t x = reinterpret_cast<uint64_t>(a), y = reinterpret_cast<uint64_t>(b);
+    return na && nb && x < y + nb && y < x + na;
+}
+
+bool aligned(const void *p, uint64_t n) { return (reinterpret_cast<uint64_t>(p) % n) == 0; }
+
+mxq_status bad(const char *why)
+{
+    std::snprintf(g_last_error, sizeof g_last_error, "invalid argument: %s", why);
+    return MXQ_ERR_INVALID_ARG;
+}
+
+// Shape checks common to every entry point (pure host logic, no CUDA calls).
+mxq_status check_shape(int64_t rows, int64_t cols)
+{
+    if (rows < 0 || cols < 0) return bad("negative size");
+    if (cols % 32) return bad("cols must be a multiple of 32");
+    if (rows >= (int64_t(1) << 31) || cols >= (int64_t(1) << 31)) return bad("rows/cols must be < 2^31");
+    if (rows > 0 && cols > 0 && ((rows + 127) / 128) * ((cols + 127) / 128) >= (int64_t(1) << 31))
+        return bad("too many tiles");
+    return MXQ_OK;
+}
+
+mxq_status make_tmap_x(CUtensorMap *map, const void *X, int64_t rows, int64_t cols)
+{
+    const Driver &d = driver();
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+    cuuint32_t box[2] = {64, static_cast<cuuint32_t>(mxq::kTileM)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = d.encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(X), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        note_cu(r, "cuTensorMapEncodeTiled");
+        return MXQ_ERR_CUDA;
+    }
+    return MXQ_OK;
+}
+
+// Common front half of the two rotate entry points.
+mxq_status rotate_common(const void *X, int64_t rows, int64_t cols, const void *R, const float *lam,
+                         void *out0, uint64_t out0_bytes, uint64_t out0_align, void *out1,
+                         uint64_t out1_bytes, mxq::RotOut mode, void *stream)
+{
+    mxq_status st = check_shape(rows, cols);
+    if (st != MXQ_OK) return st;
+    if (rows == 0 || cols == 0) return MXQ_OK;   // nothing is read or written
+    if (!X || !R || !out0 || (mode == mxq::RotOut::Quant && !out1)) return bad("null pointer");
+    if (!aligned(X, 16)) return bad("X must be 16-byte aligned");
+    if (!aligned(R, 2)) return bad("Rhat must be 2-byte aligned");
+    if (lam && !aligned(lam, 4)) return bad("Lambda must be 4-byte aligned");
+    if (!aligned(out0, out0_align)) return bad("output must be 16-byte aligned");
+    const uint64_t nx = static_cast<uint64_t>(rows) * cols * 2, nl = lam ? static_cast<uint64_t>(cols) * 4 : 0;
+    const void *ins[3] = {X, R, lam};
+    const uint64_t nins[3] = {nx, 32 * 32 * 2, nl};
+    for (int i = 0; i < 3; ++i) {
+        if (overlaps(out0, out0_bytes, ins[i], nins[i]) || (out1 && overlaps(out1, out1_bytes, ins[i], nins[i])))
+            return bad("an output overlaps an input");
+    }
+    if (out1 && overlaps(out0, out0_bytes, out1, out1_bytes)) return bad("outputs overlap");
+
+    int dev = 0, sms = 0;
+    if ((st = current_device(&dev, &sms)) != MXQ_OK) return st;
+    if ((st = check_buffer(X, nx, dev)) != MXQ_OK) return st;
+    if ((st = check_buffer(R, 32 * 32 * 2, dev)) != MXQ_OK) return st;
+    if (lam && (st = check_buffer(lam, nl, dev)) != MXQ_OK) return st;
+    if ((st = check_buffer(out0, out0_bytes, dev)) != MXQ_OK) return st;
+    if (out1 && (st = check_buffer(out1, out1_bytes, dev)) != MXQ_OK) return st;
+
+    alignas(64) CUtensorMap map;
+    if ((st = make_tmap_x(&map, X, rows, cols)) != MXQ_OK) return st;
+    mxq::RotArgs args{};
+    args.rhat = static_cast<const uint16_t *>(R);
+    args.lambda = lam;
+    args.rows = rows;
+    args.cols = cols;
+    if (mode == mxq::RotOut::Quant) {
+        args.codes = static_cast<uint8_t *>(out0);
+        args.scales = static_cast<uint8_t *>(out1);
+    } else {
+        args.y = static_cast<float *>(out0);
+    }
+    cudaError_t e = mxq::launch_rotate(map, args, mode, sms, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) {
+        note_cuda(e, "launch rotate kernel");
+        return MXQ_ERR_CUDA;
+    }
+    return MXQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+mxq_status mxq_smooth_rotate_quantize(const void *X_bf16, int64_t rows, int64_t cols, const void *Rhat_bf16,
+                                      const float *Lambda_or_null, uint8_t *out_codes_u8_packed,
+                                      uint8_t *out_scales_e8m0, void *stream)
+{
+    const uint64_t nc = rows > 0 && cols > 0 ? static_cast<uint64_t>(rows) * cols / 2 : 0;
+    const uint64_t ns = rows > 0 && cols > 0 ? static_cast<uint64_t>(rows) * (cols / 32) : 0;
+    return rotate_common(X_bf16, rows, cols, Rhat_bf16, Lambda_or_null, out_codes_u8_packed, nc, 16,
+                         out_scales_e8m0, ns, mxq::RotOut::Quant, stream);
+}
+
+mxq_status mxq_smooth_rotate_f32(const void *X_bf16, int64_t rows, int64_t cols, const void *Rhat_bf16,
+                                 const float *Lambda_or_null, float *out_f32, void *stream)
+{
+    const uint64_t ny = rows > 0 && cols > 0 ? static_cast<uint64_t>(rows) * cols * 4 : 0;
+    return rotate_common(X_bf16, rows, cols, Rhat_bf16, Lambda_or_null, out_f32, ny, 16, nullptr, 0,
+                         mxq::RotOut::F32, stream);
+}
+
+mxq_status mxq_dequantize(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t cols,
+                          const void *Rhat_bf16_or_null, const float *Lambda_or_null, void *out_bf16,
+                          void *stream)
+{
+    mxq_status st = check_shape(rows, cols);
+    if (st != MXQ_OK) return st;
+    if (rows == 0 || cols == 0) return MXQ_OK;   // nothing is read or written
+    if (!codes || !scales || !out_bf16) return bad("null pointer");
+    if (Lambda_or_null && !Rhat_bf16_or_null) return bad("Lambda requires Rhat");
+    if (!aligned(codes, 16) || !aligned(out_bf16, 16)) return bad("codes and output must be 16-byte aligned");
+    if (Rhat_bf16_or_null && !aligned(Rhat_bf16_or_null, 2)) return bad("Rhat must be 2-byte aligned");
+    if (Lambda_or_null && !aligned(Lambda_or_null, 4)) return bad("Lambda must be 4-byte aligned");
+    const uint64_t nc = static_cast<uint64_t>(rows) * cols / 2, ns = static_cast<uint64_t>(rows) * (cols / 32);
+    const uint64_t no = static_cast<uint64_t>(rows) * cols * 2;
+    const uint64_t nl = Lambda_or_null ? static_cast<uint64_t>(cols) * 4 : 0;
+    const uint64_t nr = Rhat_bf16_or_null ? 32 * 32 * 2 : 0;
+    if (overlaps(out_bf16, no, codes, nc) || overlaps(out_bf16, no, scales, ns) ||
+        overlaps(out_bf16, no, Rhat_bf16_or_null, nr) || overlaps(out_bf16, no, Lambda_or_null, nl))
+        return bad("the output overlaps an input");
+    int dev = 0, sms = 0;
+    if ((st = current_device(&dev, &sms)) != MXQ_OK) return st;
+    if ((st = check_buffer(codes, nc, dev)) != MXQ_OK) return st;
+    if ((st = check_buffer(scales, ns, dev)) != MXQ_OK) return st;
+    if ((st = check_buffer(out_bf16, no, dev)) != MXQ_OK) return st;
+    if (Rhat_bf16_or_null && (st = check_buffer(Rhat_bf16_or_null, nr, dev)) != MXQ_OK) return st;
+    if (Lambda_or_null && (st = check_buffer(Lambda_or_null, nl, dev)) != MXQ_OK) return st;
+    cudaError_t e = mxq::launch_dequant(codes, scales, rows, cols, static_cast<const uint16_t *>(Rhat_bf16_or_null),
+                                        Lambda_or_null, static_cast<uint16_t *>(out_bf16), sms,
+                                        static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) {
+        note_cuda(e, "launch dequantize kernel");
+        return MXQ_ERR_CUDA;
+    }
+    return MXQ_OK;
+}
+
+mxq_status mxq_sync_check(void *stream)
+{
+    unsigned int status = 0;
+    cudaError_t e = mxq::read_and_clear_status(&status, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) {
+        note_cuda(e, "mxq_sync_check");
+        return MXQ_ERR_CUDA;
+    }
+    if (status & mxq::kStatusTimeout) {
+        std::snprintf(g_last_error, sizeof g_last_error, "a kernel's bounded wait ran out");
+        return MXQ_ERR_TIMEOUT;
+    }
+    return MXQ_OK;
+}
+
+mxq_status mxq_selftest_bounded_wait(uint32_t timeout_ms, int *result_device, void *stream)
+{
+    if (!result_device || !aligned(result_device, 4)) return bad("result must be a 4-byte aligned device int");
+    if (timeout_ms == 0 || timeout_ms > 10000) return bad("timeout_ms must be in 1..10000");
+    int dev = 0, sms = 0;
+    mxq_status st = current_device(&dev, &sms);
+    if (st != MXQ_OK) return st;
+    if ((st = check_buffer(result_device, 4, dev)) != MXQ_OK) return st;
+    cudaError_t e = mxq::launch_wait_selftest(static_cast<uint64_t>(timeout_ms) * 1000000ull, result_device,
+                                              static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) {
+        note_cuda(e, "launch wait self-test");
+        return MXQ_ERR_CUDA;
+    }
+    return MXQ_OK;
+}
+
+const char *mxq_status_string(mxq_status status)
+{
+    switch (status) {
+    case MXQ_OK: return "MXQ_OK";
+    case MXQ_ERR_INVALID_ARG: return "MXQ_ERR_INVALID_ARG: argument rejected before launch";
+    case MXQ_ERR_UNSUPPORTED: return "MXQ_ERR_UNSUPPORTED: device is not an sm_100 part";
+    case MXQ_ERR_CUDA: return "MXQ_ERR_CUDA: a CUDA call or kernel launch failed";
+    case MXQ_ERR_TIMEOUT: return "MXQ_ERR_TIMEOUT: a kernel's bounded wait ran out";
+    }
+    return "unknown mxq_status";
+}
+
+const char *mxq_last_cuda_error(void) { return g_last_error; }
+
+int mxq_version(void) { return 1 * 10000 + 0 * 100 + 0; }
+
+}  // extern "C"

@@ -1,0 +1,50 @@
+// mxq_internal.h -- declarations shared by the library's translation units
+// (kernel launchers and the C ABI layer).  Not part of the public ABI.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace mxq {
+
+// Device status word bits (written by kernels, read by mxq_sync_check).
+enum : unsigned int {
+    kStatusTimeout = 1u,   // a bounded pipeline wait ran out
+};
+
+// Output mode of the fused rotate kernel.
+enum class RotOut { Quant, F32 };
+
+struct RotArgs {
+    const uint16_t *rhat;      // bf16 [32][32], row-major [k][n]
+    const float *lambda;       // fp32 [cols] or nullptr
+    uint8_t *codes;            // [rows, cols/2]   (Quant)
+    uint8_t *scales;           // [rows, cols/32]  (Quant)
+    float *y;                  // [rows, cols]     (F32)
+    int64_t rows;
+    int64_t cols;
+};
+
+// Launch the fused smooth-rotate(-quantize) kernel.  `tmap_x` is a 2-D tensor
+// map over X (bf16, dims {cols, rows}, box {64, 128}, 128-byte swizzle).
+cudaError_t launch_rotate(const CUtensorMap &tmap_x, const RotArgs &args, RotOut mode, int num_sms,
+                          cudaStream_t stream);
+
+// Dequantise (plain, or undoing rotation and smoothing).
+cudaError_t launch_dequant(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t cols,
+                           const uint16_t *rhat, const float *lambda, uint16_t *out, int num_sms,
+                           cudaStream_t stream);
+
+// Diagnostic kernel: a bounded wait on a barrier nothing completes (writes 2 to
+// *result once the wait ran out and the abort flag was raised).
+cudaError_t launch_wait_selftest(uint64_t timeout_ns, int *result, cudaStream_t stream);
+
+// Read-and-clear of the device status word, stream ordered.
+cudaError_t read_and_clear_status(unsigned int *host_status, cudaStream_t stream);
+
+// Rows per tile and columns per tile of the fused kernel (for host-side sizing).
+constexpr int kTileM = 128;
+constexpr int kTileCols = 128;
+
+}  // namespace mxq

@@ -1,0 +1,92 @@
+"""Host-only checks of the C ABI: the library loads, exports what the header
+declares, and rejects bad arguments before touching the GPU (no device needed)."""
+import ctypes
+import subprocess
+
+import pytest
+
+import mxfp4_block_rotation_b200 as mxq
+from mxfp4_block_rotation_b200 import build as mxq_build
+
+INVALID = 1
+
+
+@pytest.fixture(scope="module")
+def L():
+    mxq_build.build()
+    return mxq.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = mxq.declared_symbols()
+    assert {"mxq_smooth_rotate_quantize", "mxq_dequantize", "mxq_smooth_rotate_f32", "mxq_sync_check",
+            "mxq_status_string", "mxq_last_cuda_error", "mxq_version"} <= set(names)
+    out = subprocess.run(["nm", "-D", "--defined-only", mxq.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for n in names:
+        assert n in exported, n
+        assert hasattr(L, n)
+
+
+def test_status_strings_and_version(L):
+    for s in range(5):
+        assert mxq.status_string(s).startswith(("MXQ_OK", "MXQ_ERR"))
+    assert mxq.status_string(99) == "unknown mxq_status"
+    assert mxq.version() >= 10000
+
+
+P = ctypes.c_void_p
+
+
+def _q(L, x, rows, cols, r, lam, c, s):
+    return L.mxq_smooth_rotate_quantize(P(x), rows, cols, P(r), P(lam), P(c), P(s), None)
+
+
+def test_rejects_bad_shapes_before_launch(L):
+    good = 0x100000
+    assert _q(L, good, -1, 32, good, None, good * 2, good * 3) == INVALID
+    assert _q(L, good, 4, 33, good, None, good * 2, good * 3) == INVALID
+    assert _q(L, good, 4, -32, good, None, good * 2, good * 3) == INVALID
+    assert _q(L, good, 1 << 31, 32, good, None, good * 2, good * 3) == INVALID
+    assert L.mxq_last_cuda_error().startswith(b"invalid argument")
+
+
+def test_rejects_null_and_misaligned(L):
+    a = 0x100000
+    assert _q(L, None, 4, 64, a, None, a * 2, a * 3) == INVALID
+    assert _q(L, a, 4, 64, None, None, a * 2, a * 3) == INVALID
+    assert _q(L, a, 4, 64, a * 5, None, None, a * 3) == INVALID
+    assert _q(L, a + 8, 4, 64, a * 5, None, a * 2, a * 3) == INVALID        # X not 16-B aligned
+    assert _q(L, a, 4, 64, a * 5 + 1, None, a * 2, a * 3) == INVALID        # R^ odd address
+    assert _q(L, a, 4, 64, a * 5, a * 7 + 2, a * 2, a * 3) == INVALID       # Lambda not 4-B aligned
+    assert _q(L, a, 4, 64, a * 5, None, a * 2 + 4, a * 3) == INVALID        # codes not 16-B aligned
+    assert L.mxq_smooth_rotate_f32(P(a), 4, 64, P(a * 5), None, P(a * 2 + 8), None) == INVALID
+    # dequantize: Lambda without R^, misaligned output
+    assert L.mxq_dequantize(P(a), P(a * 2), 4, 64, None, P(a * 3), P(a * 4), None) == INVALID
+    assert L.mxq_dequantize(P(a), P(a * 2), 4, 64, None, None, P(a * 4 + 2), None) == INVALID
+
+
+def test_rejects_overlapping_outputs(L):
+    a = 0x100000
+    # codes overlap X
+    assert _q(L, a, 4, 64, a * 5, None, a + 16, a * 3) == INVALID
+    # scales overlap codes
+    assert _q(L, a, 4, 64, a * 5, None, a * 2, a * 2 + 16) == INVALID
+    # dequant output overlaps the codes
+    assert L.mxq_dequantize(P(a), P(a * 2), 4, 64, None, None, P(a), None) == INVALID
+
+
+def test_empty_is_a_noop(L):
+    a = 0x100000
+    assert _q(L, a, 0, 64, a * 5, None, a * 2, a * 3) == 0
+    assert _q(L, a, 4, 0, a * 5, None, a * 2, a * 3) == 0
+    assert L.mxq_dequantize(P(a), P(a * 2), 0, 64, None, None, P(a * 4), None) == 0
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(4, 32, dtype=torch.bfloat16)
+    r = torch.eye(32, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        mxq.smooth_rotate_quantize(x, r)
