@@ -16,10 +16,11 @@
 //     row-major), D = 128 lanes x 32 fp32 columns of tensor memory.  Four
 //     accumulator stages of 128 columns fill the 512 TMEM columns.
 //   * With Lambda, the B operand of group g is diag(1/Lambda_g)·R^.  It is built
-//     per tile in fp32 and split into a bf16 high and a bf16 low part (two MMAs
-//     into the same accumulator), so X stays the exact bf16 A operand and the
-//     smoothing costs no precision beyond ~2^-17 relative.  Two builder warps
-//     make these matrices into a double-buffered slot.
+//     per tile in fp32 and split into three bf16 parts, high + middle + low
+//     (three MMAs into the same accumulator, ~24 bits of B).  X stays the exact
+//     bf16 A operand, and the smoothing adds only ~2^-25 relative error on top
+//     of fp32 accumulation.  Two builder warps make these matrices into a
+//     double-buffered slot.
 //   * Eight epilogue warps (two groups of four; each group takes every other
 //     tile).  tcgen05.ld 32x32b.x32 gives each thread one row's whole 32-value
 //     group, so absmax, E8M0, scaling and the E2M1 conversion are thread-local.
@@ -50,8 +51,11 @@ constexpr int kMmaWarp = 9;
 constexpr int kBuildWarp0 = 10;
 constexpr int kBuildWarps = 2;
 constexpr int kThreads = (kEpiWarps + 2 + kBuildWarps) * 32;   // 384
-constexpr int kBMatBytes = 32 * 128;                   // one B: 32 rows (n) x 128 B (hi k | lo k)
-constexpr int kBSlotBytes = kTileG * kBMatBytes;       // 16 KB: one tile's four B matrices
+constexpr int kBMatBytes = 32 * 128;                   // one B atom: 32 rows (n) x 128 B
+// With Lambda a tile's B slot holds, per group j, an atom [hi | mid] at j*4 KB and
+// the low parts of groups 2p and 2p+1 side by side in the atom at 16 KB + p*4 KB.
+constexpr int kBLoOffset = kTileG * kBMatBytes;
+constexpr int kBSlotBytes = kBLoOffset + (kTileG / 2) * kBMatBytes;   // 24 KB
 constexpr uint64_t kTimeoutNs = 2000000000ull;         // 2 s per wait
 
 template <bool kLambda>
@@ -108,6 +112,37 @@ __device__ __forceinline__ uint32_t pack_bf16x2(__nv_bfloat16 lo, __nv_bfloat16 
 {
     return static_cast<uint32_t>(__bfloat16_as_ushort(lo)) |
            (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
+}
+
+// MXFP4 of one 32-value group (fp32 bit patterns): returns the E8M0 byte and
+// writes the 32 E2M1 codes packed into four words (value 2i in the low nibble
+// of byte i).  E8M0 = floor(log2 amax) - 2 + 127 comes straight from amax's
+// exponent field (clamped at 0); 2^-e is built from bits, so the scaling is exact.
+__device__ __forceinline__ uint32_t quantize_group(const uint32_t (&r)[32], uint32_t (&w)[4])
+{
+    float m[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        m[i] = ptx::fmax_nan(fabsf(__uint_as_float(r[2 * i])), fabsf(__uint_as_float(r[2 * i + 1])));
+#pragma unroll
+    for (int step = 8; step >= 1; step >>= 1)
+#pragma unroll
+        for (int i = 0; i < step; ++i) m[i] = ptx::fmax_nan(m[i], m[i + step]);
+    const uint32_t E = (__float_as_uint(m[0]) >> 23) & 0xFFu;
+    if (E == 0xFFu) {   // NaN/Inf group: scale byte 0xFF, codes 0
+        w[0] = w[1] = w[2] = w[3] = 0u;
+        return 0xFFu;
+    }
+    const uint32_t byte = E > 2u ? E - 2u : 0u;
+    const float s = __uint_as_float((254u - byte) << 23);   // 2^-e
+    float u[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) u[i] = __fmul_rn(__uint_as_float(r[i]), s);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        w[q] = ptx::cvt_e2m1x8(u[8 * q], u[8 * q + 1], u[8 * q + 2], u[8 * q + 3], u[8 * q + 4], u[8 * q + 5],
+                               u[8 * q + 6], u[8 * q + 7]);
+    return byte;
 }
 
 template <bool kLambda, RotOut kMode>
@@ -224,15 +259,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int j = 0; j < kTileG; ++j) {
                     const uint32_t a_j = a_base + (j >> 1) * kBoxBytes + (j & 1) * 64;
-                    const uint32_t b_j = b_base + (kLambda ? j * kBMatBytes : 0);
+                    const uint32_t d_j = d_base + j * 32;
 #pragma unroll
                     for (int kh = 0; kh < 2; ++kh) {
                         const uint64_t ad = ptx::smem_desc_sw128(a_j + kh * 32);
-                        ptx::mma_bf16(d_base + j * 32, ad, ptx::smem_desc_sw128(b_j + kh * 32), idesc,
-                                      kh);
-                        if constexpr (kLambda)
-                            ptx::mma_bf16(d_base + j * 32, ad, ptx::smem_desc_sw128(b_j + 64 + kh * 32),
-                                          idesc, 1);
+                        if constexpr (kLambda) {
+                            // smallest part first; the first MMA of the group overwrites D
+                            const uint32_t b_hi = b_base + j * kBMatBytes + kh * 32;
+                            const uint32_t b_lo =
+                                b_base + kBLoOffset + (j >> 1) * kBMatBytes + (j & 1) * 64 + kh * 32;
+                            ptx::mma_bf16(d_j, ad, ptx::smem_desc_sw128(b_lo), idesc, kh);
+                            ptx::mma_bf16(d_j, ad, ptx::smem_desc_sw128(b_hi + 64), idesc, 1);
+                            ptx::mma_bf16(d_j, ad, ptx::smem_desc_sw128(b_hi), idesc, 1);
+                        } else {
+                            ptx::mma_bf16(d_j, ad, ptx::smem_desc_sw128(b_base + kh * 32), idesc, kh);
+                        }
                     }
                 }
                 ptx::mma_commit(ptx::smem_addr(&bars->empty[s]));
@@ -256,25 +297,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int task = bt; task < kTileG * 32 * 4; task += kBuildWarps * 32) {
                     const int j = task >> 7, n = (task >> 2) & 31, c = task & 3;
                     const int64_t ch0 = ch_tile + j * 32 + c * 8;
-                    uint32_t hw[4], lw[4];
+                    uint32_t hw[4], mw[4], lw[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        __nv_bfloat16 h[2], l[2];
+                        __nv_bfloat16 h[2], m[2], l[2];
 #pragma unroll
                         for (int u = 0; u < 2; ++u) {
                             const int k = c * 8 + 2 * e + u;
                             const int64_t ch = ch0 + 2 * e + u;
                             const float val =
                                 ch < cols ? __fdiv_rn(rt[n * 32 + k], args.lambda[ch]) : 0.0f;
+                            // val = hi + mid + lo to ~24 bits; each residual is exact in fp32
                             h[u] = __float2bfloat16_rn(val);
-                            l[u] = __float2bfloat16_rn(val - __bfloat162float(h[u]));
+                            const float r1 = val - __bfloat162float(h[u]);
+                            m[u] = __float2bfloat16_rn(r1);
+                            l[u] = __float2bfloat16_rn(r1 - __bfloat162float(m[u]));
                         }
                         hw[e] = pack_bf16x2(h[0], h[1]);
+                        mw[e] = pack_bf16x2(m[0], m[1]);
                         lw[e] = pack_bf16x2(l[0], l[1]);
                     }
                     uint8_t *bm = bs + j * kBMatBytes;
+                    uint8_t *bl = bs + kBLoOffset + (j >> 1) * kBMatBytes;
                     *reinterpret_cast<uint4 *>(bm + sw128(n, c)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
                     *reinterpret_cast<uint4 *>(bm + sw128(n, c + 4)) =
+                        make_uint4(mw[0], mw[1], mw[2], mw[3]);
+                    *reinterpret_cast<uint4 *>(bl + sw128(n, c + 4 * (j & 1))) =
                         make_uint4(lw[0], lw[1], lw[2], lw[3]);
                 }
                 ptx::fence_proxy_async_smem();
@@ -299,43 +347,35 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                    static_cast<uint32_t>(a * kTileCols);
             uint32_t sc_word = 0;
-#pragma unroll 1
+            // Two register buffers: the TMEM load of group j+1 is in flight while group j
+            // is quantised.  Fully unrolled so both buffers stay in fixed registers.
+            uint32_t ra[32], rb[32];
+            ptx::tmem_ld_32cols(t_row, ra);
+            ptx::tmem_wait_ld();
+#pragma unroll
             for (int j = 0; j < kTileG; ++j) {
-                float v[32];
-                ptx::tmem_ld_32cols(t_row + j * 32, v);
+                uint32_t(&cur)[32] = (j & 1) ? rb : ra;
+                uint32_t(&nxt)[32] = (j & 1) ? ra : rb;
+                if (j + 1 < kTileG) ptx::tmem_ld_32cols(t_row + (j + 1) * 32, nxt);
                 const int64_t g = static_cast<int64_t>(ctile) * kTileG + j;
-                if (g >= G || !row_ok) continue;
-                if constexpr (kMode == RotOut::F32) {
-                    float *dst = args.y + row * cols + g * 32;
+                if (g < G && row_ok) {
+                    if constexpr (kMode == RotOut::F32) {
+                        float *dst = args.y + row * cols + g * 32;
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        ptx::st_global_v4(dst + 4 * i, __float_as_uint(v[4 * i]),
-                                          __float_as_uint(v[4 * i + 1]), __float_as_uint(v[4 * i + 2]),
-                                          __float_as_uint(v[4 * i + 3]));
-                } else {
-                    float amax = 0.0f;
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) amax = ptx::fmax_nan(amax, fabsf(v[i]));
-                    const uint32_t E = (__float_as_uint(amax) >> 23) & 0xFFu;
-                    uint32_t byte, w0 = 0, w1 = 0, w2 = 0, w3 = 0;
-                    if (E == 0xFFu) {
-                        byte = 0xFFu;   // NaN/Inf group: scale NaN, codes 0
+                        for (int i = 0; i < 8; ++i)
+                            ptx::st_global_v4(dst + 4 * i, cur[4 * i], cur[4 * i + 1], cur[4 * i + 2],
+                                              cur[4 * i + 3]);
                     } else {
-                        byte = E > 2u ? E - 2u : 0u;   // floor(log2 amax) - 2 + 127, clamped
-                        const float s = __uint_as_float((254u - byte) << 23);   // 2^-e, exact
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], s);
-                        w0 = ptx::cvt_e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
-                        w1 = ptx::cvt_e2m1x8(v[8], v[9], v[10], v[11], v[12], v[13], v[14], v[15]);
-                        w2 = ptx::cvt_e2m1x8(v[16], v[17], v[18], v[19], v[20], v[21], v[22], v[23]);
-                        w3 = ptx::cvt_e2m1x8(v[24], v[25], v[26], v[27], v[28], v[29], v[30], v[31]);
+                        uint32_t w[4];
+                        const uint32_t byte = quantize_group(cur, w);
+                        ptx::st_global_v4(args.codes + row * (cols / 2) + g * 16, w[0], w[1], w[2], w[3]);
+                        if (scale_vec)
+                            sc_word |= byte << (8 * j);
+                        else
+                            args.scales[row * G + g] = static_cast<uint8_t>(byte);
                     }
-                    ptx::st_global_v4(args.codes + row * (cols / 2) + g * 16, w0, w1, w2, w3);
-                    if (scale_vec)
-                        sc_word |= byte << (8 * j);
-                    else
-                        args.scales[row * G + g] = static_cast<uint8_t>(byte);
                 }
+                if (j + 1 < kTileG) ptx::tmem_wait_ld();
             }
             ptx::tc_fence_before();
             __syncwarp();

@@ -148,10 +148,10 @@ __device__ __forceinline__ void mma_commit(uint32_t bar)
                  : "memory");
 }
 
-// Each thread of the warp reads 32 consecutive fp32 columns of its own TMEM lane.
-__device__ __forceinline__ void tmem_ld_32cols(uint32_t taddr, float (&v)[32])
+// Each thread of the warp reads 32 consecutive 32-bit columns of its own TMEM
+// lane.  The registers are valid only after tmem_wait_ld().
+__device__ __forceinline__ void tmem_ld_32cols(uint32_t taddr, uint32_t (&r)[32])
 {
-    uint32_t r[32];
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
         "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
@@ -163,9 +163,11 @@ __device__ __forceinline__ void tmem_ld_32cols(uint32_t taddr, float (&v)[32])
           "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr)
         : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld()
+{
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 // Shared-memory matrix descriptor for a K-major operand in the 128-byte swizzle
