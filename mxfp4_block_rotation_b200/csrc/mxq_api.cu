@@ -150,6 +150,23 @@ mxq_status check_shape(int64_t rows, int64_t cols)
     return MXQ_OK;
 }
 
+mxq_status make_tmap_codes(CUtensorMap *map, void *codes, int64_t rows, int64_t cols)
+{
+    const Driver &d = driver();
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols / 2), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols / 2)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(mxq::kTileCols / 2), static_cast<cuuint32_t>(mxq::kTileM)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = d.encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, codes, dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                          CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        note_cu(r, "cuTensorMapEncodeTiled(codes)");
+        return MXQ_ERR_CUDA;
+    }
+    return MXQ_OK;
+}
+
 mxq_status make_tmap_x(CUtensorMap *map, const void *X, int64_t rows, int64_t cols)
 {
     const Driver &d = driver();
@@ -198,7 +215,13 @@ mxq_status rotate_common(const void *X, int64_t rows, int64_t cols, const void *
     if (out1 && (st = check_buffer(out1, out1_bytes, dev)) != MXQ_OK) return st;
 
     alignas(64) CUtensorMap map;
+    alignas(64) CUtensorMap map_codes;
     if ((st = make_tmap_x(&map, X, rows, cols)) != MXQ_OK) return st;
+    if (mode == mxq::RotOut::Quant) {
+        if ((st = make_tmap_codes(&map_codes, out0, rows, cols)) != MXQ_OK) return st;
+    } else {
+        map_codes = map;   // unused by the fp32 variant
+    }
     mxq::RotArgs args{};
     args.rhat = static_cast<const uint16_t *>(R);
     args.lambda = lam;
@@ -210,7 +233,7 @@ mxq_status rotate_common(const void *X, int64_t rows, int64_t cols, const void *
     } else {
         args.y = static_cast<float *>(out0);
     }
-    cudaError_t e = mxq::launch_rotate(map, args, mode, sms, static_cast<cudaStream_t>(stream));
+    cudaError_t e = mxq::launch_rotate(map, map_codes, args, mode, sms, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) {
         note_cuda(e, "launch rotate kernel");
         return MXQ_ERR_CUDA;

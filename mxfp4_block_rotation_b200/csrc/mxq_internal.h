@@ -27,9 +27,11 @@ struct RotArgs {
 };
 
 // Launch the fused smooth-rotate(-quantize) kernel.  `tmap_x` is a 2-D tensor
-// map over X (bf16, dims {cols, rows}, box {64, 128}, 128-byte swizzle).
-cudaError_t launch_rotate(const CUtensorMap &tmap_x, const RotArgs &args, RotOut mode, int num_sms,
-                          cudaStream_t stream);
+// map over X (bf16, dims {cols, rows}, box {64, 128}, 128-byte swizzle);
+// `tmap_codes` one over the packed codes (uint8, dims {cols/2, rows}, box
+// {64, 128}, 64-byte swizzle), used in Quant mode only.
+cudaError_t launch_rotate(const CUtensorMap &tmap_x, const CUtensorMap &tmap_codes, const RotArgs &args,
+                          RotOut mode, int num_sms, cudaStream_t stream);
 
 // Dequantise (plain, or undoing rotation and smoothing).
 cudaError_t launch_dequant(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t cols,

@@ -24,8 +24,12 @@
 //   * Eight epilogue warps (two groups of four; each group takes every other
 //     tile).  tcgen05.ld 32x32b.x32 gives each thread one row's whole 32-value
 //     group, so absmax, E8M0, scaling and the E2M1 conversion are thread-local.
-//     The thread writes 16 code bytes with one vector store and the four scale
-//     bytes of its row with one 32-bit store.
+//     The thread puts the 16 code bytes of each group into a shared-memory
+//     staging tile (128 rows x 64 B, 64-byte swizzle).  One thread then writes
+//     the tile with a single TMA bulk tensor store: 64 contiguous bytes per
+//     row, instead of 32 scattered 16-byte pieces per warp instruction.  The
+//     scattered form flooded the L2 with partial-sector writes.  The four
+//     scale bytes of a row go out with one 32-bit store.
 //   * Every mbarrier wait is bounded in time.  If one runs out, the kernel sets
 //     the device status word, lets every role leave its loop, drains its own
 //     copies and MMAs (again bounded), frees TMEM and returns.
@@ -58,11 +62,15 @@ constexpr int kBLoOffset = kTileG * kBMatBytes;
 constexpr int kBSlotBytes = kBLoOffset + (kTileG / 2) * kBMatBytes;   // 24 KB
 constexpr uint64_t kTimeoutNs = 2000000000ull;         // 2 s per wait
 
+constexpr int kCodeTileBytes = kTileM * kTileG * 16;    // 128 rows x 64 B of packed codes
+
 template <bool kLambda>
 struct Cfg {
-    static constexpr int kStages = kLambda ? 5 : 6;
+    static constexpr int kStages = kLambda ? 4 : 6;
     static constexpr int kBBytes = kLambda ? 2 * kBSlotBytes : kBMatBytes;
-    static constexpr int kRtOffset = kStages * kStageBytes + kBBytes;
+    static constexpr int kStageOffset = 2 * kCodeTileBytes;   // code staging tiles first (1 KB aligned)
+    static constexpr int kBOffset = kStageOffset + kStages * kStageBytes;
+    static constexpr int kRtOffset = kBOffset + kBBytes;
     static constexpr int kBarOffset = kRtOffset + 32 * 32 * 4;
     static constexpr int kSmemBytes = kBarOffset + 256 + 1024;   // + barrier block + alignment slack
 };
@@ -77,6 +85,7 @@ struct Bars {
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
+    int eg_ok[2][2];   // per epilogue warp group, per tile parity: the leader's wait result
 };
 static_assert(sizeof(Bars) <= 256, "barrier block");
 
@@ -147,14 +156,16 @@ __device__ __forceinline__ uint32_t quantize_group(const uint32_t (&r)[32], uint
 
 template <bool kLambda, RotOut kMode>
 __global__ void __launch_bounds__(kThreads, 1)
-    rotate_kernel(const __grid_constant__ CUtensorMap tmap_x, const RotArgs args)
+    rotate_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_codes,
+                  const RotArgs args)
 {
     using C = Cfg<kLambda>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
-    uint8_t *stages = smem;
-    uint8_t *bmat = smem + C::kStages * kStageBytes;
+    uint8_t *code_tiles = smem;                       // one staging tile per epilogue warp group
+    uint8_t *stages = smem + C::kStageOffset;
+    uint8_t *bmat = smem + C::kBOffset;
     float *rt = reinterpret_cast<float *>(smem + C::kRtOffset);   // R^ as fp32, [n][k]
     Bars *bars = reinterpret_cast<Bars *>(smem + C::kBarOffset);
     volatile int *abort = &bars->abort;
@@ -186,7 +197,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         bars->abort = 0;
         ptx::fence_mbar_init();
     }
-    if (warp == kTmaWarp && lane == 0) ptx::prefetch_tmap(&tmap_x);
+    if (warp == kTmaWarp && lane == 0) {
+        ptx::prefetch_tmap(&tmap_x);
+        if constexpr (kMode == RotOut::Quant) ptx::prefetch_tmap(&tmap_codes);
+    }
     if (warp == kMmaWarp) {
         ptx::tmem_alloc(ptx::smem_addr(&bars->tmem_base), kTmemCols);
         ptx::tmem_relinquish();
@@ -334,15 +348,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q = warp & 3;       // TMEM lane quarter this warp may access
         const int ewg = warp >> 2;    // which half of the tiles this warp group takes
         const bool scale_vec = (G % 4 == 0) && ((reinterpret_cast<uintptr_t>(args.scales) & 3) == 0);
+        const uint32_t ctile_smem = ptx::smem_addr(code_tiles + ewg * kCodeTileBytes);
+        const bool leader = (warp & 3) == 0 && lane == 0;   // issues this warp group's code stores
         int it = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
             if ((it & 1) != ewg) continue;
             const int a = it % kAccStages;
-            const int ok = wait_bar(&bars->acc_full[a], (it / kAccStages) & 1, abort);
-            if (!__all_sync(0xffffffffu, ok)) break;
+            // The leader alone waits (bounded) and hands the verdict to its warp group through a
+            // named barrier, so the four warps leave the loop together or not at all.
+            volatile int *ok_slot = &bars->eg_ok[ewg][(it >> 1) & 1];
+            if (leader) {
+                int ok = wait_bar(&bars->acc_full[a], (it / kAccStages) & 1, abort);
+                // the staging tile must have been read by this group's previous store
+                if constexpr (kMode == RotOut::Quant) ptx::bulk_wait_group_read0();
+                *ok_slot = ok;
+            }
+            __syncwarp();
+            ptx::named_bar_sync(1 + ewg, 128);
+            if (!*ok_slot) break;
             ptx::tc_fence_after();
             const int rtile = tile / n_ct, ctile = tile % n_ct;
-            const int64_t row = static_cast<int64_t>(rtile) * kTileM + q * 32 + lane;
+            const int r_local = q * 32 + lane;
+            const int64_t row = static_cast<int64_t>(rtile) * kTileM + r_local;
             const bool row_ok = row < rows;
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                    static_cast<uint32_t>(a * kTileCols);
@@ -358,22 +385,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint32_t(&nxt)[32] = (j & 1) ? ra : rb;
                 if (j + 1 < kTileG) ptx::tmem_ld_32cols(t_row + (j + 1) * 32, nxt);
                 const int64_t g = static_cast<int64_t>(ctile) * kTileG + j;
-                if (g < G && row_ok) {
-                    if constexpr (kMode == RotOut::F32) {
+                if constexpr (kMode == RotOut::F32) {
+                    if (g < G && row_ok) {
                         float *dst = args.y + row * cols + g * 32;
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
                             ptx::st_global_v4(dst + 4 * i, cur[4 * i], cur[4 * i + 1], cur[4 * i + 2],
                                               cur[4 * i + 3]);
-                    } else {
-                        uint32_t w[4];
-                        const uint32_t byte = quantize_group(cur, w);
-                        ptx::st_global_v4(args.codes + row * (cols / 2) + g * 16, w[0], w[1], w[2], w[3]);
-                        if (scale_vec)
-                            sc_word |= byte << (8 * j);
-                        else
-                            args.scales[row * G + g] = static_cast<uint8_t>(byte);
                     }
+                } else {
+                    uint32_t w[4];
+                    const uint32_t byte = quantize_group(cur, w);
+                    // 64-byte swizzle: 16-byte chunk j of row r sits at chunk j ^ ((r >> 1) & 3)
+                    const uint32_t chunk = static_cast<uint32_t>(j) ^ ((static_cast<uint32_t>(r_local) >> 1) & 3u);
+                    ptx::st_shared_v4(ctile_smem + r_local * 64 + chunk * 16, w[0], w[1], w[2], w[3]);
+                    if (scale_vec)
+                        sc_word |= byte << (8 * j);
+                    else if (g < G && row_ok)
+                        args.scales[row * G + g] = static_cast<uint8_t>(byte);
                 }
                 if (j + 1 < kTileG) ptx::tmem_wait_ld();
             }
@@ -384,7 +413,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (scale_vec && row_ok)
                     *reinterpret_cast<uint32_t *>(args.scales + row * G +
                                                   static_cast<int64_t>(ctile) * kTileG) = sc_word;
+                // staging tile complete -> one bulk store (rows/columns past the tensor are clipped)
+                ptx::fence_proxy_async_smem();
+                __syncwarp();
+                ptx::named_bar_sync(1 + ewg, 128);
+                if (leader) {
+                    ptx::tma_store_2d(&tmap_codes, ctile * (kTileCols / 2), rtile * kTileM, ctile_smem);
+                    ptx::bulk_commit_group();
+                }
             }
+        }
+        if constexpr (kMode == RotOut::Quant) {
+            if (leader) ptx::bulk_wait_group0();   // stores done before the CTA's shared memory goes
         }
     }
 
@@ -416,30 +456,32 @@ __global__ void bounded_wait_selftest(uint64_t timeout_ns, int *result)
 }
 
 template <bool kLambda, RotOut kMode>
-cudaError_t launch_one(const CUtensorMap &tmap, const RotArgs &args, int grid, cudaStream_t stream)
+cudaError_t launch_one(const CUtensorMap &tmap, const CUtensorMap &tmap_codes, const RotArgs &args, int grid,
+                       cudaStream_t stream)
 {
     auto kern = rotate_kernel<kLambda, kMode>;
     constexpr int smem = Cfg<kLambda>::kSmemBytes;
+    static_assert(smem <= 232448, "shared memory budget");
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads, smem, stream>>>(tmap, args);
+    kern<<<grid, kThreads, smem, stream>>>(tmap, tmap_codes, args);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_rotate(const CUtensorMap &tmap_x, const RotArgs &args, RotOut mode, int num_sms,
-                          cudaStream_t stream)
+cudaError_t launch_rotate(const CUtensorMap &tmap_x, const CUtensorMap &tmap_codes, const RotArgs &args,
+                          RotOut mode, int num_sms, cudaStream_t stream)
 {
     const int64_t n_tiles = ((args.rows + kTileM - 1) / kTileM) * ((args.cols + kTileCols - 1) / kTileCols);
     if (n_tiles <= 0) return cudaSuccess;
     const int grid = static_cast<int>(n_tiles < num_sms ? n_tiles : num_sms);
     const bool lam = args.lambda != nullptr;
     if (mode == RotOut::Quant)
-        return lam ? launch_one<true, RotOut::Quant>(tmap_x, args, grid, stream)
-                   : launch_one<false, RotOut::Quant>(tmap_x, args, grid, stream);
-    return lam ? launch_one<true, RotOut::F32>(tmap_x, args, grid, stream)
-               : launch_one<false, RotOut::F32>(tmap_x, args, grid, stream);
+        return lam ? launch_one<true, RotOut::Quant>(tmap_x, tmap_codes, args, grid, stream)
+                   : launch_one<false, RotOut::Quant>(tmap_x, tmap_codes, args, grid, stream);
+    return lam ? launch_one<true, RotOut::F32>(tmap_x, tmap_codes, args, grid, stream)
+               : launch_one<false, RotOut::F32>(tmap_x, tmap_codes, args, grid, stream);
 }
 
 cudaError_t launch_wait_selftest(uint64_t timeout_ns, int *result, cudaStream_t stream)
