@@ -205,29 +205,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tmem_alloc(ptx::smem_addr(&bars->tmem_base), kTmemCols);
         ptx::tmem_relinquish();
     }
-    for (int i = threadIdx.x; i < 32 * 32; i += kThreads) {
-        const int k = i >> 5, n = i & 31;
-        rt[n * 32 + k] = __bfloat162float(__ushort_as_bfloat16(args.rhat[i]));
-    }
-    if constexpr (!kLambda) {
-        // B = R^ in K-major form (row n holds R^[0..31][n]); high part only.
-        for (int t = threadIdx.x; t < 32 * 4; t += kThreads) {
-            const int n = t >> 2, c = t & 3;
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int k = c * 8 + 2 * e;
-                w[e] = static_cast<uint32_t>(args.rhat[k * 32 + n]) |
-                       (static_cast<uint32_t>(args.rhat[(k + 1) * 32 + n]) << 16);
-            }
-            *reinterpret_cast<uint4 *>(bmat + sw128(n, c)) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-        ptx::fence_proxy_async_smem();
-    }
+    // Nothing above touches global memory, so the next kernel in the stream may start
+    // its own set-up now; every global access below waits for the previous kernel.
+    ptx::griddep_launch_dependents();
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem_base = bars->tmem_base;
+    ptx::griddep_wait();
 
     // ---------------------------------------------------------------- roles
     if (warp == kTmaWarp) {
@@ -256,8 +241,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             constexpr uint32_t idesc = ptx::idesc_bf16_f32(128, 32);
             const uint32_t b_base0 = ptx::smem_addr(bmat);
+            // without smoothing, B is built once by the builder warps
+            const bool b_ok = kLambda || wait_bar(&bars->b_full[0], 0, abort);
             int it = 0;
-            for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+            for (int tile = blockIdx.x; b_ok && tile < num_tiles; tile += gridDim.x, ++it) {
                 const int s = it % C::kStages;
                 const int a = it % kAccStages;
                 const int slot = it & 1;
@@ -299,8 +286,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             wait_bar(&bars->drain, 0, nullptr);
         }
     } else if (warp >= kBuildWarp0) {
-        if constexpr (kLambda) {
-            const int bt = threadIdx.x - kBuildWarp0 * 32;
+        // Builders: R^ in fp32, transposed to [n][k], then the B operand(s) of the MMA.
+        const int bt = threadIdx.x - kBuildWarp0 * 32;
+        for (int i = bt; i < 32 * 32; i += kBuildWarps * 32) {
+            const int k = i >> 5, n = i & 31;
+            rt[n * 32 + k] = __bfloat162float(__ushort_as_bfloat16(args.rhat[i]));
+        }
+        ptx::named_bar_sync(3, kBuildWarps * 32);
+        if constexpr (!kLambda) {
+            // B = R^ in K-major form (row n holds R^[0..31][n]), bf16, built once; signalled
+            // through phase 0 of b_full[0].
+            for (int t = bt; t < 32 * 4; t += kBuildWarps * 32) {
+                const int n = t >> 2, c = t & 3;
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int k = c * 8 + 2 * e;
+                    w[e] = static_cast<uint32_t>(args.rhat[k * 32 + n]) |
+                           (static_cast<uint32_t>(args.rhat[(k + 1) * 32 + n]) << 16);
+                }
+                *reinterpret_cast<uint4 *>(bmat + sw128(n, c)) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::mbar_arrive(ptx::smem_addr(&bars->b_full[0]));
+        } else {
             int it = 0;
             for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
                 const int slot = it & 1;
@@ -464,8 +473,19 @@ cudaError_t launch_one(const CUtensorMap &tmap, const CUtensorMap &tmap_codes, c
     static_assert(smem <= 232448, "shared memory budget");
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads, smem, stream>>>(tmap, tmap_codes, args);
-    return cudaGetLastError();
+    // Programmatic dependent launch: this grid may start while the previous kernel in the
+    // stream drains; the kernel orders its global accesses with griddepcontrol.wait.
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, tmap, tmap_codes, args);
 }
 
 }  // namespace

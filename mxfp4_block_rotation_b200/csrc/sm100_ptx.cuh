@@ -29,6 +29,22 @@ __device__ __forceinline__ uint64_t globaltimer_ns()
     return t;
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+
+// Block until the grid this one depends on (the previous kernel in the stream)
+// has completed and its memory is visible.  A no-op without a dependency.
+__device__ __forceinline__ void griddep_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Let the next kernel in the stream begin launching (its CTAs still wait in
+// griddep_wait before touching memory this grid writes).
+__device__ __forceinline__ void griddep_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ mbarrier
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
