@@ -145,8 +145,8 @@ mxq_status check_shape(int64_t rows, int64_t cols)
     if (rows < 0 || cols < 0) return bad("negative size");
     if (cols % 32) return bad("cols must be a multiple of 32");
     if (rows >= (int64_t(1) << 31) || cols >= (int64_t(1) << 31)) return bad("rows/cols must be < 2^31");
-    if (rows > 0 && cols > 0 && ((rows + 127) / 128) * ((cols + 127) / 128) >= (int64_t(1) << 31))
-        return bad("too many tiles");
+    if (rows > 0 && cols > 0 && rows * (cols / 32) >= (int64_t(1) << 31) - 512)
+        return bad("rows * cols / 32 must be < 2^31 - 512");
     return MXQ_OK;
 }
 
@@ -162,6 +162,23 @@ mxq_status make_tmap_codes(CUtensorMap *map, void *codes, int64_t rows, int64_t 
                           CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
         note_cu(r, "cuTensorMapEncodeTiled(codes)");
+        return MXQ_ERR_CUDA;
+    }
+    return MXQ_OK;
+}
+
+mxq_status make_tmap_groups(CUtensorMap *map, const void *X, int64_t rows, int64_t cols)
+{
+    const Driver &d = driver();
+    cuuint64_t dims[2] = {32, static_cast<cuuint64_t>(rows) * static_cast<cuuint64_t>(cols / 32)};
+    cuuint64_t strides[1] = {64};
+    cuuint32_t box[2] = {32, 256};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = d.encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(X), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        note_cu(r, "cuTensorMapEncodeTiled(groups)");
         return MXQ_ERR_CUDA;
     }
     return MXQ_OK;
@@ -214,13 +231,12 @@ mxq_status rotate_common(const void *X, int64_t rows, int64_t cols, const void *
     if ((st = check_buffer(out0, out0_bytes, dev)) != MXQ_OK) return st;
     if (out1 && (st = check_buffer(out1, out1_bytes, dev)) != MXQ_OK) return st;
 
-    alignas(64) CUtensorMap map;
-    alignas(64) CUtensorMap map_codes;
-    if ((st = make_tmap_x(&map, X, rows, cols)) != MXQ_OK) return st;
-    if (mode == mxq::RotOut::Quant) {
-        if ((st = make_tmap_codes(&map_codes, out0, rows, cols)) != MXQ_OK) return st;
+    mxq::RotMaps maps;
+    if (lam == nullptr) {
+        if ((st = make_tmap_groups(&maps.groups, X, rows, cols)) != MXQ_OK) return st;
     } else {
-        map_codes = map;   // unused by the fp32 variant
+        if ((st = make_tmap_x(&maps.x, X, rows, cols)) != MXQ_OK) return st;
+        if (mode == mxq::RotOut::Quant && (st = make_tmap_codes(&maps.codes, out0, rows, cols)) != MXQ_OK) return st;
     }
     mxq::RotArgs args{};
     args.rhat = static_cast<const uint16_t *>(R);
@@ -233,7 +249,7 @@ mxq_status rotate_common(const void *X, int64_t rows, int64_t cols, const void *
     } else {
         args.y = static_cast<float *>(out0);
     }
-    cudaError_t e = mxq::launch_rotate(map, map_codes, args, mode, sms, static_cast<cudaStream_t>(stream));
+    cudaError_t e = mxq::launch_rotate(maps, args, mode, sms, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) {
         note_cuda(e, "launch rotate kernel");
         return MXQ_ERR_CUDA;

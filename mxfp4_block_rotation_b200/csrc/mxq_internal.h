@@ -26,12 +26,19 @@ struct RotArgs {
     int64_t cols;
 };
 
-// Launch the fused smooth-rotate(-quantize) kernel.  `tmap_x` is a 2-D tensor
-// map over X (bf16, dims {cols, rows}, box {64, 128}, 128-byte swizzle);
-// `tmap_codes` one over the packed codes (uint8, dims {cols/2, rows}, box
-// {64, 128}, 64-byte swizzle), used in Quant mode only.
-cudaError_t launch_rotate(const CUtensorMap &tmap_x, const CUtensorMap &tmap_codes, const RotArgs &args,
-                          RotOut mode, int num_sms, cudaStream_t stream);
+// TMA descriptors the rotate kernels read.  Without Lambda only `groups` is used:
+// X as a dense [rows*cols/32, 32] bf16 matrix (box {32, 256}, 64-byte swizzle).
+// With Lambda, `x` is X as [rows, cols] bf16 (box {64, 128}, 128-byte swizzle)
+// and `codes` the packed codes as [rows, cols/2] uint8 (box {64, 128}, 64-byte
+// swizzle; Quant mode only).
+struct RotMaps {
+    alignas(64) CUtensorMap groups;
+    alignas(64) CUtensorMap x;
+    alignas(64) CUtensorMap codes;
+};
+
+// Launch the fused smooth-rotate(-quantize) kernel for `args`.
+cudaError_t launch_rotate(const RotMaps &maps, const RotArgs &args, RotOut mode, int num_sms, cudaStream_t stream);
 
 // Dequantise (plain, or undoing rotation and smoothing).
 cudaError_t launch_dequant(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t cols,

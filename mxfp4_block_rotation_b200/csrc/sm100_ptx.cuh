@@ -234,6 +234,18 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr)
     return d;
 }
 
+// Same for the 64-byte swizzle layout: rows of 64 B, 8-row atoms 512 B apart.
+__device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t saddr)
+{
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFF);   // start address, 16-B units
+    d |= static_cast<uint64_t>(1) << 16;                  // leading byte offset (unused when swizzled)
+    d |= static_cast<uint64_t>(512 >> 4) << 32;          // stride byte offset: next 8-row atom
+    d |= static_cast<uint64_t>(1) << 46;                  // descriptor version (sm100)
+    d |= static_cast<uint64_t>(4) << 61;                  // layout: 64-byte swizzle
+    return d;
+}
+
 // Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both K-major.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n)
 {
