@@ -15,15 +15,15 @@
 // The rotation is a dense bf16 contraction on the tensor cores: tcgen05.mma
 // M=128, N=32, K=16, fp32 accumulate.  A is 128 groups of X staged by TMA in
 // shared memory, B = R^ in K-major form (R^T row-major), and D is 128 TMEM
-// lanes x 32 columns.  Four accumulator stages of 128 columns fill TMEM's 512
+// lanes x 32 columns.  Accumulator stages (32 columns per MMA) fill TMEM's 512
 // columns.  The epilogue reads TMEM with tcgen05.ld 32x32b.x32, so each thread
 // holds one group's 32 rotated values.  Absmax, E8M0, scaling and the E2M1
 // conversion are therefore thread-local.
 //
 // Without Lambda (rotate_flat_kernel): X is a dense [rows*cols/32, 32] matrix,
 // the reshape-and-bmm form of §3.3's implementation tips.  An MMA takes 128
-// consecutive groups; a stage is 512 groups, two TMA boxes of 16 contiguous KB
-// each.  A warp's 32 lanes quantise 32 consecutive groups, so its code store
+// consecutive groups; a stage is kFlatMmas MMAs' worth, loaded as TMA boxes of
+// 16 contiguous KB.  A warp's 32 lanes quantise 32 consecutive groups, so its code store
 // covers 512 contiguous bytes and its scale store 32.  Loads and stores all
 // stream through HBM in address order.
 //
@@ -52,9 +52,8 @@ __device__ unsigned int g_status;
 
 namespace {
 
-constexpr int kAccStages = 4;
-constexpr uint32_t kTmemCols = 512;      // 4 accumulator stages x 128 fp32 columns
-constexpr int kAccCols = 128;
+constexpr uint32_t kTmemCols = 512;      // all of TMEM: accumulator stages of 32 columns per MMA
+constexpr int kMaxAcc = 8;
 constexpr int kEpiWarps = 8;
 constexpr int kTmaWarp = 8;
 constexpr int kMmaWarp = 9;
@@ -68,8 +67,8 @@ constexpr int kMaxStages = 8;
 struct Bars {
     uint64_t full[kMaxStages];
     uint64_t empty[kMaxStages];
-    uint64_t acc_full[kAccStages];
-    uint64_t acc_empty[kAccStages];
+    uint64_t acc_full[kMaxAcc];
+    uint64_t acc_empty[kMaxAcc];
     uint64_t b_full[2];
     uint64_t b_empty[2];
     uint64_t drain;
@@ -77,7 +76,7 @@ struct Bars {
     int abort;
     int eg_ok[2][2];   // per epilogue warp group, per tile parity: the leader's wait result
 };
-static_assert(sizeof(Bars) <= 256, "barrier block");
+static_assert(sizeof(Bars) <= 512, "barrier block");
 
 // Bounded wait on an mbarrier phase.  False if the wait ran out or (when abort
 // is non-null) another role has already aborted.  Drains at exit pass a null
@@ -151,7 +150,7 @@ __device__ __forceinline__ uint32_t quantize_group(const uint32_t (&r)[32], uint
 
 // Barrier initialisation, TMEM allocation and the programmatic-dependent-launch
 // handshake shared by both kernels.  Returns the TMEM base address.
-__device__ __forceinline__ uint32_t kernel_setup(Bars *bars, int n_stages, const CUtensorMap *map0,
+__device__ __forceinline__ uint32_t kernel_setup(Bars *bars, int n_stages, int n_acc, const CUtensorMap *map0,
                                                  const CUtensorMap *map1)
 {
     const int warp = threadIdx.x >> 5;
@@ -161,7 +160,7 @@ __device__ __forceinline__ uint32_t kernel_setup(Bars *bars, int n_stages, const
             ptx::mbar_init(ptx::smem_addr(&bars->full[s]), 1);
             ptx::mbar_init(ptx::smem_addr(&bars->empty[s]), 1);
         }
-        for (int a = 0; a < kAccStages; ++a) {
+        for (int a = 0; a < n_acc; ++a) {
             ptx::mbar_init(ptx::smem_addr(&bars->acc_full[a]), 1);
             ptx::mbar_init(ptx::smem_addr(&bars->acc_empty[a]), kEpiWarps / 2);
         }
@@ -224,10 +223,15 @@ __device__ __forceinline__ void kernel_teardown(uint32_t tmem_base)
 // =====================================================================================
 
 constexpr int kFlatBoxGroups = 256;                        // one TMA box: 256 groups x 64 B = 16 KB
-constexpr int kFlatStageGroups = 512;                      // one stage: 4 MMAs of 128 groups
-constexpr int kFlatStageBytes = kFlatStageGroups * 64;     // 32 KB
-constexpr int kFlatStages = 4;
-constexpr int kFlatSmemBytes = kFlatStages * kFlatStageBytes + kBMatBytes + 256 + 1024;
+constexpr int kFlatMmas = 4;                               // MMAs (of 128 groups) per stage
+constexpr int kFlatStageGroups = 128 * kFlatMmas;
+constexpr int kFlatBoxes = kFlatStageGroups / kFlatBoxGroups;
+constexpr int kFlatStageBytes = kFlatStageGroups * 64;
+constexpr int kFlatStages = 3;                             // ~96 KB in flight per SM measured best
+constexpr int kFlatAccCols = 32 * kFlatMmas;               // TMEM columns per accumulator stage
+constexpr int kFlatAcc = (512 / kFlatAccCols) < kMaxAcc ? (512 / kFlatAccCols) : kMaxAcc;
+constexpr int kFlatSmemBytes = kFlatStages * kFlatStageBytes + kBMatBytes + 512 + 1024;
+static_assert(kFlatBoxes >= 1 && kFlatStageGroups % kFlatBoxGroups == 0 && kFlatStages <= kMaxStages, "flat tiling");
 
 template <RotOut kMode>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -243,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t n_groups = args.rows * (args.cols / 32);
     const int n_chunks = static_cast<int>((n_groups + kFlatStageGroups - 1) / kFlatStageGroups);
 
-    const uint32_t tmem_base = kernel_setup(bars, kFlatStages, &tmap_g, nullptr);
+    const uint32_t tmem_base = kernel_setup(bars, kFlatStages, kFlatAcc, &tmap_g, nullptr);
 
     if (warp == kTmaWarp) {
         if (lane == 0) {
@@ -256,8 +260,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t dst = ptx::smem_addr(stages + s * kFlatStageBytes);
                 const int g0 = c * kFlatStageGroups;
                 ptx::mbar_arrive_expect_tx(full, kFlatStageBytes);
-                ptx::tma_load_2d(dst, &tmap_g, 0, g0, full, pol);
-                ptx::tma_load_2d(dst + kFlatBoxGroups * 64, &tmap_g, 0, g0 + kFlatBoxGroups, full, pol);
+#pragma unroll
+                for (int b = 0; b < kFlatBoxes; ++b)
+                    ptx::tma_load_2d(dst + b * kFlatBoxGroups * 64, &tmap_g, 0, g0 + b * kFlatBoxGroups, full, pol);
             }
             drain_loads(bars, kFlatStages, it);
         }
@@ -269,14 +274,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             int it = 0;
             for (int c = blockIdx.x; b_ok && c < n_chunks; c += gridDim.x, ++it) {
                 const int s = it % kFlatStages;
-                const int a = it % kAccStages;
+                const int a = it % kFlatAcc;
                 if (!wait_bar(&bars->full[s], (it / kFlatStages) & 1, abort)) break;
-                if (!wait_bar(&bars->acc_empty[a], ((it / kAccStages) & 1) ^ 1, abort)) break;
+                if (!wait_bar(&bars->acc_empty[a], ((it / kFlatAcc) & 1) ^ 1, abort)) break;
                 ptx::tc_fence_after();
                 const uint32_t a_base = ptx::smem_addr(stages + s * kFlatStageBytes);
-                const uint32_t d_base = tmem_base + static_cast<uint32_t>(a * kAccCols);
+                const uint32_t d_base = tmem_base + static_cast<uint32_t>(a * kFlatAccCols);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
+                for (int j = 0; j < kFlatMmas; ++j) {
 #pragma unroll
                     for (int kh = 0; kh < 2; ++kh)
                         ptx::mma_bf16(d_base + j * 32, ptx::smem_desc_sw64(a_base + j * 128 * 64 + kh * 32),
@@ -309,12 +314,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         int it = 0;
         for (int c = blockIdx.x; c < n_chunks; c += gridDim.x, ++it) {
             if ((it & 1) != ewg) continue;
-            const int a = it % kAccStages;
+            const int a = it % kFlatAcc;
             int ok = 0;
-            if (lane == 0) ok = wait_bar(&bars->acc_full[a], (it / kAccStages) & 1, abort);
+            if (lane == 0) ok = wait_bar(&bars->acc_full[a], (it / kFlatAcc) & 1, abort);
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
             ptx::tc_fence_after();
-            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * kAccCols;
+            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * kFlatAccCols;
             const int64_t g_lane = static_cast<int64_t>(c) * kFlatStageGroups + q * 32 + lane;
             // The TMEM load of MMA j+1 is in flight while group j is quantised; fully
             // unrolled so both register buffers stay put.
@@ -322,10 +327,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tmem_ld_32cols(t_row, ra);
             ptx::tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int j = 0; j < kFlatMmas; ++j) {
                 uint32_t(&cur)[32] = (j & 1) ? rb : ra;
                 uint32_t(&nxt)[32] = (j & 1) ? ra : rb;
-                if (j + 1 < 4) ptx::tmem_ld_32cols(t_row + (j + 1) * 32, nxt);
+                if (j + 1 < kFlatMmas) ptx::tmem_ld_32cols(t_row + (j + 1) * 32, nxt);
                 const int64_t g = g_lane + j * 128;
                 if (g < n_groups) {
                     if constexpr (kMode == RotOut::F32) {
@@ -341,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         args.scales[g] = static_cast<uint8_t>(byte);
                     }
                 }
-                if (j + 1 < 4) ptx::tmem_wait_ld();
+                if (j + 1 < kFlatMmas) ptx::tmem_wait_ld();
             }
             ptx::tc_fence_before();
             __syncwarp();
@@ -356,6 +361,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // =====================================================================================
 
 constexpr int kColTileG = 4;                                  // groups per tile
+constexpr int kColAcc = 4;                                    // accumulator stages of 128 columns
+constexpr int kColAccCols = 128;
 constexpr int kColStageBytes = kTileM * kTileCols * 2;        // 32 KB of bf16 per stage
 constexpr int kColBoxBytes = kColStageBytes / 2;              // one TMA box: 128 rows x 128 B
 constexpr int kCodeTileBytes = kTileM * kColTileG * 16;       // 128 rows x 64 B of packed codes
@@ -368,7 +375,7 @@ constexpr int kColStageOffset = 2 * kCodeTileBytes;           // code staging ti
 constexpr int kColBOffset = kColStageOffset + kColStages * kColStageBytes;
 constexpr int kColRtOffset = kColBOffset + 2 * kBSlotBytes;
 constexpr int kColBarOffset = kColRtOffset + 32 * 32 * 4;
-constexpr int kColSmemBytes = kColBarOffset + 256 + 1024;
+constexpr int kColSmemBytes = kColBarOffset + 512 + 1024;
 
 template <RotOut kMode>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -394,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int num_tiles = n_ct * n_rt;
 
     const uint32_t tmem_base =
-        kernel_setup(bars, kColStages, &tmap_x, kMode == RotOut::Quant ? &tmap_codes : nullptr);
+        kernel_setup(bars, kColStages, kColAcc, &tmap_x, kMode == RotOut::Quant ? &tmap_codes : nullptr);
 
     if (warp == kTmaWarp) {
         if (lane == 0) {
@@ -419,15 +426,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             int it = 0;
             for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
                 const int s = it % kColStages;
-                const int a = it % kAccStages;
+                const int a = it % kColAcc;
                 const int slot = it & 1;
                 if (!wait_bar(&bars->full[s], (it / kColStages) & 1, abort)) break;
-                if (!wait_bar(&bars->acc_empty[a], ((it / kAccStages) & 1) ^ 1, abort)) break;
+                if (!wait_bar(&bars->acc_empty[a], ((it / kColAcc) & 1) ^ 1, abort)) break;
                 if (!wait_bar(&bars->b_full[slot], (it >> 1) & 1, abort)) break;
                 ptx::tc_fence_after();
                 const uint32_t a_base = ptx::smem_addr(stages + s * kColStageBytes);
                 const uint32_t b_base = b_base0 + slot * kBSlotBytes;
-                const uint32_t d_base = tmem_base + static_cast<uint32_t>(a * kAccCols);
+                const uint32_t d_base = tmem_base + static_cast<uint32_t>(a * kColAccCols);
 #pragma unroll
                 for (int j = 0; j < kColTileG; ++j) {
                     const uint32_t a_j = a_base + (j >> 1) * kColBoxBytes + (j & 1) * 64;
@@ -504,12 +511,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         int it = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
             if ((it & 1) != ewg) continue;
-            const int a = it % kAccStages;
+            const int a = it % kColAcc;
             // The leader alone waits (bounded) and hands the verdict to its warp group through a
             // named barrier, so the four warps leave the loop together or not at all.
             volatile int *ok_slot = &bars->eg_ok[ewg][(it >> 1) & 1];
             if (leader) {
-                int ok = wait_bar(&bars->acc_full[a], (it / kAccStages) & 1, abort);
+                int ok = wait_bar(&bars->acc_full[a], (it / kColAcc) & 1, abort);
                 // the staging tile must have been read by this group's previous store
                 if constexpr (kMode == RotOut::Quant) ptx::bulk_wait_group_read0();
                 *ok_slot = ok;
@@ -522,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int r_local = q * 32 + lane;
             const int64_t row = static_cast<int64_t>(rtile) * kTileM + r_local;
             const bool row_ok = row < rows;
-            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * kAccCols;
+            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * kColAccCols;
             uint32_t sc_word = 0;
             uint32_t ra[32], rb[32];
             ptx::tmem_ld_32cols(t_row, ra);
