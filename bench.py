@@ -275,6 +275,7 @@ def run_mine(args):
 
     # end to end through the public API: pinned host X -> device -> kernel -> codes/scales back to host
     e2e = None if args.no_e2e else run_e2e(mxq, w, rhat, dev, stream, args, dist)
+    extras = None if (args.no_extras or world > 1) else run_extras(mxq, w, xs, rhat, outs, dev, stream)
 
     if rank == 0:
         peak, peak_kind = hbm_peak()
@@ -298,6 +299,8 @@ def run_mine(args):
             "gpu_launches": k,
             "clocks": clocks.summary(),
         }
+        if extras is not None:
+            line["other_rows"] = extras
         if world == 1 and not args.no_cpu_baseline:
             import oracle
             oracle.build()
@@ -312,6 +315,55 @@ def run_mine(args):
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def _timed(fn, k, stream, dev):
+    for i in range(5):
+        fn(i)
+    torch.cuda.synchronize(dev)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(k):
+        fn(i)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    return a.elapsed_time(b) / k
+
+
+def run_extras(mxq, w, xs, rhat, outs, dev, stream, k=300):
+    """The other rows of the path on the same workload, each timed back to back."""
+    rows, cols = w.rows, w.cols
+    peak, _ = hbm_peak()
+    lam = synth.smoothing_scale(w.x).to(dev)   # the smoothing recipe: clip(max|X_j|^0.5, 1e-2, 1e2)
+    res = {}
+
+    def row(name, ms, nbytes, what):
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        res[name] = {"what": what, "ms": ms, "GB/s": gbs, "frac_of_hbm_peak": gbs / peak,
+                     "bytes_per_launch": nbytes}
+
+    def quant_lam(i):
+        c, s = outs[i & 1]
+        mxq.smooth_rotate_quantize(xs[i & 1], rhat, lam, codes=c, scales=s, stream=stream)
+    row("smooth_rotate_quantize_with_lambda", _timed(quant_lam, k, stream, dev),
+        algorithmic_bytes(rows, cols) + 4 * cols,
+        "same X, Lambda_j = clip(max_t|X_tj|^0.5, 1e-2, 1e2) (rotate_cols_kernel)")
+    deq = [torch.empty((rows, cols), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    deq_bytes = rows * cols * (0.5 + 1.0 / 32.0 + 2.0)
+
+    def dq_plain(i):
+        c, s = outs[i & 1]
+        mxq.dequantize(c, s, out=deq[i & 1], stream=stream)
+    row("dequantize", _timed(dq_plain, k, stream, dev), deq_bytes, "codes + scales -> bf16 (rotated domain)")
+
+    def dq_inv(i):
+        c, s = outs[i & 1]
+        mxq.dequantize(c, s, rhat, lam, out=deq[i & 1], stream=stream)
+    row("dequantize_inverse_rotation_and_smoothing", _timed(dq_inv, k, stream, dev), deq_bytes + 4 * cols,
+        "codes + scales -> (v * R^T) * Lambda -> bf16")
+    mxq.sync_check()
+    return res
 
 
 def run_e2e(mxq, w, rhat, dev, stream, args, dist):
@@ -358,13 +410,14 @@ def run_e2e(mxq, w, rhat, dev, stream, args, dist):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=10000)
+    ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["mine", "reference"], default="mine")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="oracle time for the cpu_baseline sample (rank 0, N=1 only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg (profiling runs)")
+    ap.add_argument("--no-extras", action="store_true", help="skip timing the smoothing and dequantize rows")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
