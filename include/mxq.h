@@ -111,11 +111,12 @@ mxq_status mxq_smooth_rotate_f32(const void *X_bf16, int64_t rows, int64_t cols,
  *
  *   codes, scales       in   as produced above; codes 16-byte aligned
  *   rows, cols          in   as above
- *   Rhat_bf16_or_null   in   NULL: write v itself.  It is exactly representable
+ *   Rhat_bf16_or_null   in   16-byte aligned.  NULL: write v itself.  It is exactly representable
  *                            in bf16, so the output is bit-exact (overflow
  *                            gives +-Inf).
  *                            non-NULL: undo the rotation, x_k = sum_n v_n R^[k][n]
- *                            (v * R^T), with fp32 accumulation.
+ *                            (v * R^T), on the tensor cores: v is the exact bf16
+ *                            A operand, fp32 accumulation.
  *   Lambda_or_null      in   non-NULL: undo the smoothing too, x_k *= Lambda[k]
  *                            (allowed only together with R^)
  *   out_bf16            out  bf16 [rows, cols], 16-byte aligned; the fp32 result

@@ -289,7 +289,7 @@ mxq_status mxq_dequantize(const uint8_t *codes, const uint8_t *scales, int64_t r
     if (!codes || !scales || !out_bf16) return bad("null pointer");
     if (Lambda_or_null && !Rhat_bf16_or_null) return bad("Lambda requires Rhat");
     if (!aligned(codes, 16) || !aligned(out_bf16, 16)) return bad("codes and output must be 16-byte aligned");
-    if (Rhat_bf16_or_null && !aligned(Rhat_bf16_or_null, 2)) return bad("Rhat must be 2-byte aligned");
+    if (Rhat_bf16_or_null && !aligned(Rhat_bf16_or_null, 16)) return bad("Rhat must be 16-byte aligned for dequantize");
     if (Lambda_or_null && !aligned(Lambda_or_null, 4)) return bad("Lambda must be 4-byte aligned");
     const uint64_t nc = static_cast<uint64_t>(rows) * cols / 2, ns = static_cast<uint64_t>(rows) * (cols / 32);
     const uint64_t no = static_cast<uint64_t>(rows) * cols * 2;
@@ -305,8 +305,12 @@ mxq_status mxq_dequantize(const uint8_t *codes, const uint8_t *scales, int64_t r
     if ((st = check_buffer(out_bf16, no, dev)) != MXQ_OK) return st;
     if (Rhat_bf16_or_null && (st = check_buffer(Rhat_bf16_or_null, nr, dev)) != MXQ_OK) return st;
     if (Lambda_or_null && (st = check_buffer(Lambda_or_null, nl, dev)) != MXQ_OK) return st;
-    cudaError_t e = mxq::launch_dequant(codes, scales, rows, cols, static_cast<const uint16_t *>(Rhat_bf16_or_null),
-                                        Lambda_or_null, static_cast<uint16_t *>(out_bf16), sms,
+    cudaError_t e =
+        Rhat_bf16_or_null
+            ? mxq::launch_dequant_rot(codes, scales, rows, cols, static_cast<const uint16_t *>(Rhat_bf16_or_null),
+                                      Lambda_or_null, static_cast<uint16_t *>(out_bf16), sms,
+                                      static_cast<cudaStream_t>(stream))
+            : mxq::launch_dequant_plain(codes, scales, rows, cols, static_cast<uint16_t *>(out_bf16), sms,
                                         static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) {
         note_cuda(e, "launch dequantize kernel");

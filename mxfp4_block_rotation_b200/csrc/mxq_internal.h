@@ -40,10 +40,14 @@ struct RotMaps {
 // Launch the fused smooth-rotate(-quantize) kernel for `args`.
 cudaError_t launch_rotate(const RotMaps &maps, const RotArgs &args, RotOut mode, int num_sms, cudaStream_t stream);
 
-// Dequantise (plain, or undoing rotation and smoothing).
-cudaError_t launch_dequant(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t cols,
-                           const uint16_t *rhat, const float *lambda, uint16_t *out, int num_sms,
-                           cudaStream_t stream);
+// Dequantise to bf16 in the rotated domain (codes 16-byte aligned, out 16-byte aligned).
+cudaError_t launch_dequant_plain(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t cols,
+                                 uint16_t *out, int num_sms, cudaStream_t stream);
+
+// Dequantise and undo the rotation (rhat non-null) and the smoothing (lambda, may be null).
+cudaError_t launch_dequant_rot(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t cols,
+                               const uint16_t *rhat, const float *lambda, uint16_t *out, int num_sms,
+                               cudaStream_t stream);
 
 // Diagnostic kernel: a bounded wait on a barrier nothing completes (writes 2 to
 // *result once the wait ran out and the abort flag was raised).

@@ -148,35 +148,41 @@ __device__ __forceinline__ uint32_t quantize_group(const uint32_t (&r)[32], uint
     return byte;
 }
 
+// Per-kernel numbers the shared set-up needs.
+struct SetupCfg {
+    int n_stages;     // shared-memory stages (full/empty barrier pairs)
+    int n_acc;        // TMEM accumulator stages
+    int full_count;   // arrivals that complete a stage's full barrier (1 for a TMA producer)
+    int b_count;      // arrivals that complete b_full (the B builders' threads)
+    int mma_warp;     // the warp that owns TMEM
+};
+
 // Barrier initialisation, TMEM allocation and the programmatic-dependent-launch
-// handshake shared by both kernels.  Returns the TMEM base address.
-__device__ __forceinline__ uint32_t kernel_setup(Bars *bars, int n_stages, int n_acc, const CUtensorMap *map0,
+// handshake shared by the kernels.  Returns the TMEM base address.
+__device__ __forceinline__ uint32_t kernel_setup(Bars *bars, const SetupCfg &cfg, const CUtensorMap *map0,
                                                  const CUtensorMap *map1)
 {
     const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < n_stages; ++s) {
-            ptx::mbar_init(ptx::smem_addr(&bars->full[s]), 1);
+        for (int s = 0; s < cfg.n_stages; ++s) {
+            ptx::mbar_init(ptx::smem_addr(&bars->full[s]), cfg.full_count);
             ptx::mbar_init(ptx::smem_addr(&bars->empty[s]), 1);
         }
-        for (int a = 0; a < n_acc; ++a) {
+        for (int a = 0; a < cfg.n_acc; ++a) {
             ptx::mbar_init(ptx::smem_addr(&bars->acc_full[a]), 1);
             ptx::mbar_init(ptx::smem_addr(&bars->acc_empty[a]), kEpiWarps / 2);
         }
         for (int s = 0; s < 2; ++s) {
-            ptx::mbar_init(ptx::smem_addr(&bars->b_full[s]), kBuildWarps * 32);
+            ptx::mbar_init(ptx::smem_addr(&bars->b_full[s]), cfg.b_count);
             ptx::mbar_init(ptx::smem_addr(&bars->b_empty[s]), 1);
         }
         ptx::mbar_init(ptx::smem_addr(&bars->drain), 1);
         bars->abort = 0;
         ptx::fence_mbar_init();
-    }
-    if (warp == kTmaWarp && lane == 0) {
-        ptx::prefetch_tmap(map0);
+        if (map0) ptx::prefetch_tmap(map0);
         if (map1) ptx::prefetch_tmap(map1);
     }
-    if (warp == kMmaWarp) {
+    if (warp == cfg.mma_warp) {
         ptx::tmem_alloc(ptx::smem_addr(&bars->tmem_base), kTmemCols);
         ptx::tmem_relinquish();
     }
@@ -207,11 +213,11 @@ __device__ __forceinline__ void drain_mmas(Bars *bars)
     wait_bar(&bars->drain, 0, nullptr);
 }
 
-__device__ __forceinline__ void kernel_teardown(uint32_t tmem_base)
+__device__ __forceinline__ void kernel_teardown(uint32_t tmem_base, int mma_warp)
 {
     ptx::tc_fence_before();
     __syncthreads();
-    if ((threadIdx.x >> 5) == kMmaWarp) {
+    if ((threadIdx.x >> 5) == mma_warp) {
         __syncwarp();
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem_base, kTmemCols);
@@ -247,7 +253,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t n_groups = args.rows * (args.cols / 32);
     const int n_chunks = static_cast<int>((n_groups + kFlatStageGroups - 1) / kFlatStageGroups);
 
-    const uint32_t tmem_base = kernel_setup(bars, kFlatStages, kFlatAcc, &tmap_g, nullptr);
+    const uint32_t tmem_base =
+        kernel_setup(bars, SetupCfg{kFlatStages, kFlatAcc, 1, kBuildWarps * 32, kMmaWarp}, &tmap_g, nullptr);
 
     if (warp == kTmaWarp) {
         if (lane == 0) {
@@ -353,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) ptx::mbar_arrive(ptx::smem_addr(&bars->acc_empty[a]));
         }
     }
-    kernel_teardown(tmem_base);
+    kernel_teardown(tmem_base, kMmaWarp);
 }
 
 // =====================================================================================
@@ -377,6 +384,44 @@ constexpr int kColRtOffset = kColBOffset + 2 * kBSlotBytes;
 constexpr int kColBarOffset = kColRtOffset + 32 * 32 * 4;
 constexpr int kColSmemBytes = kColBarOffset + 512 + 1024;
 
+// Tile order of the smoothing kernel.  B_g depends only on the column group, so
+// each CTA walks whole column strips top to bottom and builds a strip's B_g
+// once.  With no more strips than CTAs, the grid is k CTAs per strip, each
+// taking every k-th row block.  Otherwise each CTA takes every grid-th strip in
+// turn.  At any moment the CTAs sit at about the same row block, so together
+// they still read whole rows of X.
+struct StripSched {
+    int ct0, ct_step, rt0, rt_step, per_strip, n_tiles;
+    __device__ StripSched(int n_ct, int n_rt, int cta, int grid)
+    {
+        if (n_ct <= grid) {
+            ct0 = cta % n_ct;
+            ct_step = n_ct;
+            rt0 = cta / n_ct;
+            rt_step = grid / n_ct;
+        } else {
+            ct0 = cta;
+            ct_step = grid;
+            rt0 = 0;
+            rt_step = 1;
+        }
+        per_strip = rt0 < n_rt ? (n_rt - rt0 + rt_step - 1) / rt_step : 0;
+        const int strips = ct0 < n_ct ? (n_ct - ct0 + ct_step - 1) / ct_step : 0;
+        n_tiles = strips * per_strip;
+    }
+    __device__ int ct(int it) const { return ct0 + (it / per_strip) * ct_step; }
+    __device__ int rt(int it) const { return rt0 + (it % per_strip) * rt_step; }
+};
+
+__host__ int strip_grid(int n_ct, int n_rt, int num_sms)
+{
+    if (n_ct > num_sms) return num_sms;
+    int k = num_sms / n_ct;
+    if (k > n_rt) k = n_rt;
+    if (k < 1) k = 1;
+    return n_ct * k;
+}
+
 template <RotOut kMode>
 __global__ void __launch_bounds__(kThreads, 1)
     rotate_cols_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_codes,
@@ -398,19 +443,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t G = cols / 32;
     const int n_ct = static_cast<int>((cols + kTileCols - 1) / kTileCols);
     const int n_rt = static_cast<int>((rows + kTileM - 1) / kTileM);
-    const int num_tiles = n_ct * n_rt;
+    const StripSched sched(n_ct, n_rt, blockIdx.x, gridDim.x);
 
     const uint32_t tmem_base =
-        kernel_setup(bars, kColStages, kColAcc, &tmap_x, kMode == RotOut::Quant ? &tmap_codes : nullptr);
+        kernel_setup(bars, SetupCfg{kColStages, kColAcc, 1, kBuildWarps * 32, kMmaWarp}, &tmap_x,
+                     kMode == RotOut::Quant ? &tmap_codes : nullptr);
 
     if (warp == kTmaWarp) {
         if (lane == 0) {
             const uint64_t pol = ptx::policy_evict_first();
             int it = 0;
-            for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+            for (; it < sched.n_tiles; ++it) {
                 const int s = it % kColStages;
                 if (!wait_bar(&bars->empty[s], ((it / kColStages) & 1) ^ 1, abort)) break;
-                const int rtile = tile / n_ct, ctile = tile % n_ct;
+                const int rtile = sched.rt(it), ctile = sched.ct(it);
                 const uint32_t full = ptx::smem_addr(&bars->full[s]);
                 const uint32_t dst = ptx::smem_addr(stages + s * kColStageBytes);
                 ptx::mbar_arrive_expect_tx(full, kColStageBytes);
@@ -423,8 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             constexpr uint32_t idesc = ptx::idesc_bf16_f32(128, 32);
             const uint32_t b_base0 = ptx::smem_addr(bmat);
-            int it = 0;
-            for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+            for (int it = 0; it < sched.n_tiles; ++it) {
                 const int s = it % kColStages;
                 const int a = it % kColAcc;
                 const int slot = it & 1;
@@ -464,11 +509,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             rt[n * 32 + k] = __bfloat162float(__ushort_as_bfloat16(args.rhat[i]));
         }
         ptx::named_bar_sync(3, kBuildWarps * 32);
-        int it = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+        int built0 = -1, built1 = -1;   // column strip whose B_g each slot holds
+        for (int it = 0; it < sched.n_tiles; ++it) {
             const int slot = it & 1;
             if (!wait_bar(&bars->b_empty[slot], ((it >> 1) & 1) ^ 1, abort)) break;
-            const int64_t ch_tile = static_cast<int64_t>(tile % n_ct) * kTileCols;
+            const int ct = sched.ct(it);
+            if ((slot ? built1 : built0) == ct) {   // same strip: the slot's matrices are still right
+                ptx::mbar_arrive(ptx::smem_addr(&bars->b_full[slot]));
+                continue;
+            }
+            if (slot)
+                built1 = ct;
+            else
+                built0 = ct;
+            const int64_t ch_tile = static_cast<int64_t>(ct) * kTileCols;
             uint8_t *bs = bmat + slot * kBSlotBytes;
             // 4 groups x 32 rows (n) x 4 chunks of 8 k = 512 chunk tasks.
             for (int task = bt; task < kColTileG * 32 * 4; task += kBuildWarps * 32) {
@@ -508,9 +562,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool scale_vec = (G % 4 == 0) && ((reinterpret_cast<uintptr_t>(args.scales) & 3) == 0);
         const uint32_t ctile_smem = ptx::smem_addr(code_tiles + ewg * kCodeTileBytes);
         const bool leader = q == 0 && lane == 0;   // issues this warp group's code stores
-        int it = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
-            if ((it & 1) != ewg) continue;
+        for (int it = ewg; it < sched.n_tiles; it += 2) {
             const int a = it % kColAcc;
             // The leader alone waits (bounded) and hands the verdict to its warp group through a
             // named barrier, so the four warps leave the loop together or not at all.
@@ -525,7 +577,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::named_bar_sync(1 + ewg, 128);
             if (!*ok_slot) break;
             ptx::tc_fence_after();
-            const int rtile = tile / n_ct, ctile = tile % n_ct;
+            const int rtile = sched.rt(it), ctile = sched.ct(it);
             const int r_local = q * 32 + lane;
             const int64_t row = static_cast<int64_t>(rtile) * kTileM + r_local;
             const bool row_ok = row < rows;
@@ -582,16 +634,213 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (leader) ptx::bulk_wait_group0();   // stores done before the CTA's shared memory goes
         }
     }
-    kernel_teardown(tmem_base);
+    kernel_teardown(tmem_base, kMmaWarp);
 }
 
-static_assert(kFlatSmemBytes <= 232448 && kColSmemBytes <= 232448, "shared memory budget");
+// =====================================================================================
+// Dequantise and undo the transform: out = (v * R^T) * Lambda, v = E2M1(code) * 2^e.
+// =====================================================================================
+//
+// The same flat group-major pipeline as rotate_flat_kernel, run backwards.  Four
+// decoder warps turn each stage's 512 groups of codes into bf16 values in
+// shared memory: the MMA's A tile, 64-byte swizzle.  The values are exact in
+// bf16: two significant bits times a power of two.  The MMA computes
+// D[g][k] = sum_n v[g][n] * R^[k][n], so B is R^ as stored (row k, contiguous n
+// = K-major).  The epilogue multiplies by Lambda_k and rounds to bf16.
+
+constexpr int kDqDecWarp0 = 8;
+constexpr int kDqDecWarps = 4;
+constexpr int kDqMmaWarp = 12;
+constexpr int kDqThreads = (kDqMmaWarp + 1) * 32;   // 416
+constexpr int kDqStages = 3;
+constexpr int kDqStageGroups = 512;                 // 4 MMAs of 128 groups
+constexpr int kDqStageBytes = kDqStageGroups * 64;
+constexpr int kDqAcc = 4;
+constexpr int kDqAccCols = 128;
+constexpr int kDqSmemBytes = kDqStages * kDqStageBytes + kBMatBytes + 1024 + 512 + 1024;
+
+__device__ __forceinline__ uint32_t e2m1_bf16(uint32_t code)
+{
+    // magnitudes {0, 0.5, 1, 1.5, 2, 3, 4, 6}: code 1 is E2M1's subnormal 0.5; codes
+    // 2..7 are 2^(e-1) * (1 + m/2) with e = code >> 1, m = code & 1
+    const uint32_t m = code & 7u;
+    const uint32_t mag = m == 0u ? 0u : (m == 1u ? 0x3F00u : ((126u + (m >> 1)) << 7) | ((m & 1u) << 6));
+    return mag | ((code & 8u) << 12);
+}
+
+__device__ __forceinline__ uint32_t hmul2_bits(uint32_t a, __nv_bfloat162 s)
+{
+    const __nv_bfloat162 v = __halves2bfloat162(__ushort_as_bfloat16(static_cast<unsigned short>(a & 0xFFFFu)),
+                                                __ushort_as_bfloat16(static_cast<unsigned short>(a >> 16)));
+    const __nv_bfloat162 r = __hmul2(v, s);
+    return static_cast<uint32_t>(__bfloat16_as_ushort(__low2bfloat16(r))) |
+           (static_cast<uint32_t>(__bfloat16_as_ushort(__high2bfloat16(r))) << 16);
+}
+
+template <bool kLambda>
+__global__ void __launch_bounds__(kDqThreads, 1)
+    dequant_rot_kernel(const uint4 *__restrict__ codes, const uint8_t *__restrict__ scales, int64_t n_groups,
+                       int64_t G, const uint16_t *__restrict__ rhat, const float *__restrict__ lambda,
+                       uint16_t *__restrict__ out)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *stages = align_1k(smem_raw);
+    uint8_t *bmat = stages + kDqStages * kDqStageBytes;
+    uint32_t *lut = reinterpret_cast<uint32_t *>(bmat + kBMatBytes);   // code byte -> bf16x2
+    Bars *bars = reinterpret_cast<Bars *>(bmat + kBMatBytes + 1024);
+    volatile int *abort = &bars->abort;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int n_chunks = static_cast<int>((n_groups + kDqStageGroups - 1) / kDqStageGroups);
+
+    const uint32_t tmem_base = kernel_setup(
+        bars, SetupCfg{kDqStages, kDqAcc, kDqDecWarps * 32, kDqDecWarps * 32, kDqMmaWarp}, nullptr, nullptr);
+
+    if (warp >= kDqDecWarp0 && warp < kDqDecWarp0 + kDqDecWarps) {
+        const int dt = threadIdx.x - kDqDecWarp0 * 32;   // 0..127
+        for (int i = dt; i < 256; i += kDqDecWarps * 32)
+            lut[i] = e2m1_bf16(static_cast<uint32_t>(i) & 15u) | (e2m1_bf16(static_cast<uint32_t>(i) >> 4) << 16);
+        // B: row k holds R^[k][0..31] (bf16) in the first 64 B of a 128-byte-swizzled row
+        if (dt < 32 * 4) {
+            const int k = dt >> 2, c = dt & 3;
+            const uint4 v = *reinterpret_cast<const uint4 *>(rhat + k * 32 + c * 8);
+            *reinterpret_cast<uint4 *>(bmat + sw128(k, c)) = v;
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::mbar_arrive(ptx::smem_addr(&bars->b_full[0]));
+        ptx::named_bar_sync(3, kDqDecWarps * 32);   // the table is complete
+        int it = 0;
+        for (int c = blockIdx.x; c < n_chunks; c += gridDim.x, ++it) {
+            const int s = it % kDqStages;
+            int ok = 0;
+            if (lane == 0) ok = wait_bar(&bars->empty[s], ((it / kDqStages) & 1) ^ 1, abort);
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            const uint32_t st = ptx::smem_addr(stages + s * kDqStageBytes);
+#pragma unroll
+            for (int i = 0; i < kDqStageGroups / (kDqDecWarps * 32); ++i) {
+                const int r = dt + i * kDqDecWarps * 32;   // group row within the stage
+                const int64_t g = static_cast<int64_t>(c) * kDqStageGroups + r;
+                uint32_t w[16];
+                if (g < n_groups) {
+                    const uint4 cw = __ldcs(codes + g);
+                    const uint32_t byte = __ldg(scales + g);
+                    const uint32_t sb = byte == 0xFFu ? 0x7FC0u : (byte == 0u ? 0x0040u : (byte << 7));
+                    const __nv_bfloat162 s2 = __halves2bfloat162(__ushort_as_bfloat16(static_cast<unsigned short>(sb)),
+                                                                 __ushort_as_bfloat16(static_cast<unsigned short>(sb)));
+                    const uint32_t cws[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+                    for (int b = 0; b < 16; ++b) w[b] = hmul2_bits(lut[(cws[b >> 2] >> (8 * (b & 3))) & 0xFFu], s2);
+                } else {
+#pragma unroll
+                    for (int b = 0; b < 16; ++b) w[b] = 0u;
+                }
+                // 64-byte swizzle: 16-byte chunk q of row r sits at chunk q ^ ((r >> 1) & 3)
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    ptx::st_shared_v4(st + r * 64 + ((q ^ ((r >> 1) & 3)) << 4), w[4 * q], w[4 * q + 1],
+                                      w[4 * q + 2], w[4 * q + 3]);
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::mbar_arrive(ptx::smem_addr(&bars->full[s]));
+        }
+    } else if (warp == kDqMmaWarp) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = ptx::idesc_bf16_f32(128, 32);
+            const uint32_t b_base = ptx::smem_addr(bmat);
+            const bool b_ok = wait_bar(&bars->b_full[0], 0, abort);
+            int it = 0;
+            for (int c = blockIdx.x; b_ok && c < n_chunks; c += gridDim.x, ++it) {
+                const int s = it % kDqStages;
+                const int a = it % kDqAcc;
+                if (!wait_bar(&bars->full[s], (it / kDqStages) & 1, abort)) break;
+                if (!wait_bar(&bars->acc_empty[a], ((it / kDqAcc) & 1) ^ 1, abort)) break;
+                ptx::tc_fence_after();
+                const uint32_t a_base = ptx::smem_addr(stages + s * kDqStageBytes);
+                const uint32_t d_base = tmem_base + static_cast<uint32_t>(a * kDqAccCols);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+#pragma unroll
+                    for (int kh = 0; kh < 2; ++kh)
+                        ptx::mma_bf16(d_base + j * 32, ptx::smem_desc_sw64(a_base + j * 128 * 64 + kh * 32),
+                                      ptx::smem_desc_sw128(b_base + kh * 32), idesc, kh);
+                }
+                ptx::mma_commit(ptx::smem_addr(&bars->empty[s]));
+                ptx::mma_commit(ptx::smem_addr(&bars->acc_full[a]));
+            }
+            drain_mmas(bars);
+        }
+    } else if (warp < kEpiWarps) {
+        const int q = warp & 3;
+        const int ewg = warp >> 2;
+        const bool lam_vec = kLambda && ((reinterpret_cast<uintptr_t>(lambda) & 15) == 0);
+        int it = 0;
+        for (int c = blockIdx.x; c < n_chunks; c += gridDim.x, ++it) {
+            if ((it & 1) != ewg) continue;
+            const int a = it % kDqAcc;
+            int ok = 0;
+            if (lane == 0) ok = wait_bar(&bars->acc_full[a], (it / kDqAcc) & 1, abort);
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            ptx::tc_fence_after();
+            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * kDqAccCols;
+            const int64_t g_lane = static_cast<int64_t>(c) * kDqStageGroups + q * 32 + lane;
+            uint32_t ra[32], rb[32];
+            ptx::tmem_ld_32cols(t_row, ra);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                uint32_t(&cur)[32] = (j & 1) ? rb : ra;
+                uint32_t(&nxt)[32] = (j & 1) ? ra : rb;
+                if (j + 1 < 4) ptx::tmem_ld_32cols(t_row + (j + 1) * 32, nxt);
+                const int64_t g = g_lane + j * 128;
+                if (g < n_groups) {
+                    float x[32];
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) x[k] = __uint_as_float(cur[k]);
+                    if constexpr (kLambda) {
+                        const float *lg = lambda + (g % G) * 32;
+                        if (lam_vec) {
+#pragma unroll
+                            for (int k4 = 0; k4 < 8; ++k4) {
+                                const float4 l4 = __ldg(reinterpret_cast<const float4 *>(lg) + k4);
+                                x[4 * k4] = __fmul_rn(x[4 * k4], l4.x);
+                                x[4 * k4 + 1] = __fmul_rn(x[4 * k4 + 1], l4.y);
+                                x[4 * k4 + 2] = __fmul_rn(x[4 * k4 + 2], l4.z);
+                                x[4 * k4 + 3] = __fmul_rn(x[4 * k4 + 3], l4.w);
+                            }
+                        } else {
+#pragma unroll
+                            for (int k = 0; k < 32; ++k) x[k] = __fmul_rn(x[k], __ldg(lg + k));
+                        }
+                    }
+                    uint32_t o[16];
+#pragma unroll
+                    for (int k2 = 0; k2 < 16; ++k2) {
+                        const __nv_bfloat162 p = __floats2bfloat162_rn(x[2 * k2], x[2 * k2 + 1]);
+                        o[k2] = static_cast<uint32_t>(__bfloat16_as_ushort(__low2bfloat16(p))) |
+                                (static_cast<uint32_t>(__bfloat16_as_ushort(__high2bfloat16(p))) << 16);
+                    }
+                    uint16_t *dst = out + g * 32;
+#pragma unroll
+                    for (int v = 0; v < 4; ++v)
+                        ptx::st_global_v4(dst + 8 * v, o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+                }
+                if (j + 1 < 4) ptx::tmem_wait_ld();
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(ptx::smem_addr(&bars->acc_empty[a]));
+        }
+    }
+    kernel_teardown(tmem_base, kDqMmaWarp);
+}
+
+static_assert(kFlatSmemBytes <= 232448 && kColSmemBytes <= 232448 && kDqSmemBytes <= 232448, "shared memory budget");
 
 // Launch with programmatic stream serialisation: the grid may start while the
 // previous kernel in the stream drains (the kernels order their global accesses
 // with griddepcontrol.wait).
 template <typename Kern, typename... Args>
-cudaError_t launch_pdl(Kern kern, int grid, int smem, cudaStream_t stream, Args... args)
+cudaError_t launch_pdl(Kern kern, int grid, int block, int smem, cudaStream_t stream, Args... args)
 {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
@@ -600,7 +849,7 @@ cudaError_t launch_pdl(Kern kern, int grid, int smem, cudaStream_t stream, Args.
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(block);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cfg.attrs = attr;
@@ -634,14 +883,34 @@ cudaError_t launch_rotate(const RotMaps &maps, const RotArgs &args, RotOut mode,
         const int64_t n_chunks = (n_groups + kFlatStageGroups - 1) / kFlatStageGroups;
         const int grid = static_cast<int>(n_chunks < num_sms ? n_chunks : num_sms);
         return mode == RotOut::Quant
-                   ? launch_pdl(rotate_flat_kernel<RotOut::Quant>, grid, kFlatSmemBytes, stream, maps.groups, args)
-                   : launch_pdl(rotate_flat_kernel<RotOut::F32>, grid, kFlatSmemBytes, stream, maps.groups, args);
+                   ? launch_pdl(rotate_flat_kernel<RotOut::Quant>, grid, kThreads, kFlatSmemBytes, stream, maps.groups,
+                                args)
+                   : launch_pdl(rotate_flat_kernel<RotOut::F32>, grid, kThreads, kFlatSmemBytes, stream, maps.groups,
+                                args);
     }
-    const int64_t n_tiles = ((args.rows + kTileM - 1) / kTileM) * ((args.cols + kTileCols - 1) / kTileCols);
-    const int grid = static_cast<int>(n_tiles < num_sms ? n_tiles : num_sms);
+    const int grid = strip_grid(static_cast<int>((args.cols + kTileCols - 1) / kTileCols),
+                                static_cast<int>((args.rows + kTileM - 1) / kTileM), num_sms);
     return mode == RotOut::Quant
-               ? launch_pdl(rotate_cols_kernel<RotOut::Quant>, grid, kColSmemBytes, stream, maps.x, maps.codes, args)
-               : launch_pdl(rotate_cols_kernel<RotOut::F32>, grid, kColSmemBytes, stream, maps.x, maps.codes, args);
+               ? launch_pdl(rotate_cols_kernel<RotOut::Quant>, grid, kThreads, kColSmemBytes, stream, maps.x,
+                            maps.codes, args)
+               : launch_pdl(rotate_cols_kernel<RotOut::F32>, grid, kThreads, kColSmemBytes, stream, maps.x,
+                            maps.codes, args);
+}
+
+cudaError_t launch_dequant_rot(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t cols,
+                               const uint16_t *rhat, const float *lambda, uint16_t *out, int num_sms,
+                               cudaStream_t stream)
+{
+    const int64_t G = cols / 32;
+    const int64_t n_groups = rows * G;
+    if (n_groups <= 0) return cudaSuccess;
+    const int64_t n_chunks = (n_groups + kDqStageGroups - 1) / kDqStageGroups;
+    const int grid = static_cast<int>(n_chunks < num_sms ? n_chunks : num_sms);
+    const uint4 *c4 = reinterpret_cast<const uint4 *>(codes);
+    return lambda ? launch_pdl(dequant_rot_kernel<true>, grid, kDqThreads, kDqSmemBytes, stream, c4, scales, n_groups,
+                               G, rhat, lambda, out)
+                  : launch_pdl(dequant_rot_kernel<false>, grid, kDqThreads, kDqSmemBytes, stream, c4, scales, n_groups,
+                               G, rhat, lambda, out);
 }
 
 cudaError_t launch_wait_selftest(uint64_t timeout_ns, int *result, cudaStream_t stream)
