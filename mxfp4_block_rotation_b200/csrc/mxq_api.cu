@@ -167,12 +167,13 @@ mxq_status make_tmap_codes(CUtensorMap *map, void *codes, int64_t rows, int64_t 
     return MXQ_OK;
 }
 
-mxq_status make_tmap_groups(CUtensorMap *map, const void *X, int64_t rows, int64_t cols)
+// A bf16 [rows, cols] matrix viewed as [rows*cols/32, 32]: one 64-byte row per group.
+mxq_status make_tmap_groups(CUtensorMap *map, const void *X, int64_t rows, int64_t cols, uint32_t box_rows = 256)
 {
     const Driver &d = driver();
     cuuint64_t dims[2] = {32, static_cast<cuuint64_t>(rows) * static_cast<cuuint64_t>(cols / 32)};
     cuuint64_t strides[1] = {64};
-    cuuint32_t box[2] = {32, 256};
+    cuuint32_t box[2] = {32, box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = d.encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(X), dims, strides, box,
                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
@@ -305,13 +306,16 @@ mxq_status mxq_dequantize(const uint8_t *codes, const uint8_t *scales, int64_t r
     if ((st = check_buffer(out_bf16, no, dev)) != MXQ_OK) return st;
     if (Rhat_bf16_or_null && (st = check_buffer(Rhat_bf16_or_null, nr, dev)) != MXQ_OK) return st;
     if (Lambda_or_null && (st = check_buffer(Lambda_or_null, nl, dev)) != MXQ_OK) return st;
-    cudaError_t e =
-        Rhat_bf16_or_null
-            ? mxq::launch_dequant_rot(codes, scales, rows, cols, static_cast<const uint16_t *>(Rhat_bf16_or_null),
-                                      Lambda_or_null, static_cast<uint16_t *>(out_bf16), sms,
-                                      static_cast<cudaStream_t>(stream))
-            : mxq::launch_dequant_plain(codes, scales, rows, cols, static_cast<uint16_t *>(out_bf16), sms,
-                                        static_cast<cudaStream_t>(stream));
+    cudaError_t e;
+    if (Rhat_bf16_or_null) {
+        alignas(64) CUtensorMap map_out;
+        if ((st = make_tmap_groups(&map_out, out_bf16, rows, cols, 32)) != MXQ_OK) return st;
+        e = mxq::launch_dequant_rot(map_out, codes, scales, rows, cols, static_cast<const uint16_t *>(Rhat_bf16_or_null),
+                                    Lambda_or_null, sms, static_cast<cudaStream_t>(stream));
+    } else {
+        e = mxq::launch_dequant_plain(codes, scales, rows, cols, static_cast<uint16_t *>(out_bf16), sms,
+                                      static_cast<cudaStream_t>(stream));
+    }
     if (e != cudaSuccess) {
         note_cuda(e, "launch dequantize kernel");
         return MXQ_ERR_CUDA;

@@ -44,9 +44,11 @@ cudaError_t launch_rotate(const RotMaps &maps, const RotArgs &args, RotOut mode,
 cudaError_t launch_dequant_plain(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t cols,
                                  uint16_t *out, int num_sms, cudaStream_t stream);
 
-// Dequantise and undo the rotation (rhat non-null) and the smoothing (lambda, may be null).
-cudaError_t launch_dequant_rot(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t cols,
-                               const uint16_t *rhat, const float *lambda, uint16_t *out, int num_sms,
+// Dequantise and undo the rotation (rhat non-null) and the smoothing (lambda, may be
+// null).  `tmap_out` views the bf16 output as [rows*cols/32, 32] (box {32, 32},
+// 64-byte swizzle).
+cudaError_t launch_dequant_rot(const CUtensorMap &tmap_out, const uint8_t *codes, const uint8_t *scales, int64_t rows,
+                               int64_t cols, const uint16_t *rhat, const float *lambda, int num_sms,
                                cudaStream_t stream);
 
 // Diagnostic kernel: a bounded wait on a barrier nothing completes (writes 2 to

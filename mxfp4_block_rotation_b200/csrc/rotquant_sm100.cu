@@ -657,7 +657,9 @@ constexpr int kDqStageGroups = 512;                 // 4 MMAs of 128 groups
 constexpr int kDqStageBytes = kDqStageGroups * 64;
 constexpr int kDqAcc = 4;
 constexpr int kDqAccCols = 128;
-constexpr int kDqSmemBytes = kDqStages * kDqStageBytes + kBMatBytes + 1024 + 512 + 1024;
+constexpr int kDqOutBuf = 32 * 64;                 // one epilogue warp's 32 output groups (2 KB)
+constexpr int kDqOutBytes = kEpiWarps * 2 * kDqOutBuf;   // double-buffered per epilogue warp
+constexpr int kDqSmemBytes = kDqStages * kDqStageBytes + kBMatBytes + 1024 + kDqOutBytes + 512 + 1024;
 
 __device__ __forceinline__ uint32_t e2m1_bf16(uint32_t code)
 {
@@ -679,22 +681,23 @@ __device__ __forceinline__ uint32_t hmul2_bits(uint32_t a, __nv_bfloat162 s)
 
 template <bool kLambda>
 __global__ void __launch_bounds__(kDqThreads, 1)
-    dequant_rot_kernel(const uint4 *__restrict__ codes, const uint8_t *__restrict__ scales, int64_t n_groups,
-                       int64_t G, const uint16_t *__restrict__ rhat, const float *__restrict__ lambda,
-                       uint16_t *__restrict__ out)
+    dequant_rot_kernel(const __grid_constant__ CUtensorMap tmap_out, const uint4 *__restrict__ codes,
+                       const uint8_t *__restrict__ scales, int64_t n_groups, int64_t G,
+                       const uint16_t *__restrict__ rhat, const float *__restrict__ lambda)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *stages = align_1k(smem_raw);
     uint8_t *bmat = stages + kDqStages * kDqStageBytes;
     uint32_t *lut = reinterpret_cast<uint32_t *>(bmat + kBMatBytes);   // code byte -> bf16x2
-    Bars *bars = reinterpret_cast<Bars *>(bmat + kBMatBytes + 1024);
+    uint8_t *outbuf = bmat + kBMatBytes + 1024;                          // epilogue staging
+    Bars *bars = reinterpret_cast<Bars *>(outbuf + kDqOutBytes);
     volatile int *abort = &bars->abort;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int n_chunks = static_cast<int>((n_groups + kDqStageGroups - 1) / kDqStageGroups);
 
     const uint32_t tmem_base = kernel_setup(
-        bars, SetupCfg{kDqStages, kDqAcc, kDqDecWarps * 32, kDqDecWarps * 32, kDqMmaWarp}, nullptr, nullptr);
+        bars, SetupCfg{kDqStages, kDqAcc, kDqDecWarps * 32, kDqDecWarps * 32, kDqMmaWarp}, &tmap_out, nullptr);
 
     if (warp >= kDqDecWarp0 && warp < kDqDecWarp0 + kDqDecWarps) {
         const int dt = threadIdx.x - kDqDecWarp0 * 32;   // 0..127
@@ -770,10 +773,13 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             drain_mmas(bars);
         }
     } else if (warp < kEpiWarps) {
+        // Each warp stages its 32 groups' outputs (2 KB, 64-byte swizzle) and writes them
+        // with one TMA bulk tensor store: 2 KB contiguous instead of 16-byte pieces.
         const int q = warp & 3;
         const int ewg = warp >> 2;
         const bool lam_vec = kLambda && ((reinterpret_cast<uintptr_t>(lambda) & 15) == 0);
-        int it = 0;
+        const uint32_t obuf0 = ptx::smem_addr(outbuf + warp * 2 * kDqOutBuf);
+        int it = 0, nstore = 0;
         for (int c = blockIdx.x; c < n_chunks; c += gridDim.x, ++it) {
             if ((it & 1) != ewg) continue;
             const int a = it % kDqAcc;
@@ -782,7 +788,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
             ptx::tc_fence_after();
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * kDqAccCols;
-            const int64_t g_lane = static_cast<int64_t>(c) * kDqStageGroups + q * 32 + lane;
+            const int64_t g_warp = static_cast<int64_t>(c) * kDqStageGroups + q * 32;
             uint32_t ra[32], rb[32];
             ptx::tmem_ld_32cols(t_row, ra);
             ptx::tmem_wait_ld();
@@ -791,45 +797,55 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                 uint32_t(&cur)[32] = (j & 1) ? rb : ra;
                 uint32_t(&nxt)[32] = (j & 1) ? ra : rb;
                 if (j + 1 < 4) ptx::tmem_ld_32cols(t_row + (j + 1) * 32, nxt);
-                const int64_t g = g_lane + j * 128;
-                if (g < n_groups) {
-                    float x[32];
+                const int64_t g0 = g_warp + j * 128;   // this warp's first group of MMA j
+                const int64_t g = g0 + lane;
+                // times Lambda_k (channels of this group), then round to bf16 pairs
+                uint32_t o[16];
+                const float *lg = kLambda ? lambda + (g < n_groups ? g % G : 0) * 32 : nullptr;
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) x[k] = __uint_as_float(cur[k]);
+                for (int k4 = 0; k4 < 8; ++k4) {
+                    float4 l4 = make_float4(1.0f, 1.0f, 1.0f, 1.0f);
                     if constexpr (kLambda) {
-                        const float *lg = lambda + (g % G) * 32;
                         if (lam_vec) {
-#pragma unroll
-                            for (int k4 = 0; k4 < 8; ++k4) {
-                                const float4 l4 = __ldg(reinterpret_cast<const float4 *>(lg) + k4);
-                                x[4 * k4] = __fmul_rn(x[4 * k4], l4.x);
-                                x[4 * k4 + 1] = __fmul_rn(x[4 * k4 + 1], l4.y);
-                                x[4 * k4 + 2] = __fmul_rn(x[4 * k4 + 2], l4.z);
-                                x[4 * k4 + 3] = __fmul_rn(x[4 * k4 + 3], l4.w);
-                            }
+                            l4 = __ldg(reinterpret_cast<const float4 *>(lg) + k4);
                         } else {
-#pragma unroll
-                            for (int k = 0; k < 32; ++k) x[k] = __fmul_rn(x[k], __ldg(lg + k));
+                            l4.x = __ldg(lg + 4 * k4);
+                            l4.y = __ldg(lg + 4 * k4 + 1);
+                            l4.z = __ldg(lg + 4 * k4 + 2);
+                            l4.w = __ldg(lg + 4 * k4 + 3);
                         }
                     }
-                    uint32_t o[16];
-#pragma unroll
-                    for (int k2 = 0; k2 < 16; ++k2) {
-                        const __nv_bfloat162 p = __floats2bfloat162_rn(x[2 * k2], x[2 * k2 + 1]);
-                        o[k2] = static_cast<uint32_t>(__bfloat16_as_ushort(__low2bfloat16(p))) |
-                                (static_cast<uint32_t>(__bfloat16_as_ushort(__high2bfloat16(p))) << 16);
-                    }
-                    uint16_t *dst = out + g * 32;
-#pragma unroll
-                    for (int v = 0; v < 4; ++v)
-                        ptx::st_global_v4(dst + 8 * v, o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+                    const __nv_bfloat162 p0 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(cur[4 * k4]), l4.x),
+                                                                    __fmul_rn(__uint_as_float(cur[4 * k4 + 1]), l4.y));
+                    const __nv_bfloat162 p1 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(cur[4 * k4 + 2]), l4.z),
+                                                                    __fmul_rn(__uint_as_float(cur[4 * k4 + 3]), l4.w));
+                    o[2 * k4] = static_cast<uint32_t>(__bfloat16_as_ushort(__low2bfloat16(p0))) |
+                                (static_cast<uint32_t>(__bfloat16_as_ushort(__high2bfloat16(p0))) << 16);
+                    o[2 * k4 + 1] = static_cast<uint32_t>(__bfloat16_as_ushort(__low2bfloat16(p1))) |
+                                    (static_cast<uint32_t>(__bfloat16_as_ushort(__high2bfloat16(p1))) << 16);
                 }
+                const uint32_t buf = obuf0 + (nstore & 1) * kDqOutBuf;
+                // the buffer's previous store (two stores ago) must have been read
+                if (lane == 0) ptx::bulk_wait_group_read1();
+                __syncwarp();
+#pragma unroll
+                for (int v = 0; v < 4; ++v)
+                    ptx::st_shared_v4(buf + lane * 64 + ((v ^ ((lane >> 1) & 3)) << 4), o[4 * v], o[4 * v + 1],
+                                      o[4 * v + 2], o[4 * v + 3]);
+                ptx::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0 && g0 < n_groups) {   // rows past n_groups are clipped by the tensor map
+                    ptx::tma_store_2d(&tmap_out, 0, static_cast<int32_t>(g0), buf);
+                    ptx::bulk_commit_group();
+                }
+                ++nstore;
                 if (j + 1 < 4) ptx::tmem_wait_ld();
             }
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(ptx::smem_addr(&bars->acc_empty[a]));
         }
+        if (lane == 0) ptx::bulk_wait_group0();   // stores done before the CTA's shared memory goes
     }
     kernel_teardown(tmem_base, kDqMmaWarp);
 }
@@ -897,8 +913,8 @@ cudaError_t launch_rotate(const RotMaps &maps, const RotArgs &args, RotOut mode,
                             maps.codes, args);
 }
 
-cudaError_t launch_dequant_rot(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t cols,
-                               const uint16_t *rhat, const float *lambda, uint16_t *out, int num_sms,
+cudaError_t launch_dequant_rot(const CUtensorMap &tmap_out, const uint8_t *codes, const uint8_t *scales, int64_t rows,
+                               int64_t cols, const uint16_t *rhat, const float *lambda, int num_sms,
                                cudaStream_t stream)
 {
     const int64_t G = cols / 32;
@@ -907,10 +923,10 @@ cudaError_t launch_dequant_rot(const uint8_t *codes, const uint8_t *scales, int6
     const int64_t n_chunks = (n_groups + kDqStageGroups - 1) / kDqStageGroups;
     const int grid = static_cast<int>(n_chunks < num_sms ? n_chunks : num_sms);
     const uint4 *c4 = reinterpret_cast<const uint4 *>(codes);
-    return lambda ? launch_pdl(dequant_rot_kernel<true>, grid, kDqThreads, kDqSmemBytes, stream, c4, scales, n_groups,
-                               G, rhat, lambda, out)
-                  : launch_pdl(dequant_rot_kernel<false>, grid, kDqThreads, kDqSmemBytes, stream, c4, scales, n_groups,
-                               G, rhat, lambda, out);
+    return lambda ? launch_pdl(dequant_rot_kernel<true>, grid, kDqThreads, kDqSmemBytes, stream, tmap_out, c4, scales,
+                               n_groups, G, rhat, lambda)
+                  : launch_pdl(dequant_rot_kernel<false>, grid, kDqThreads, kDqSmemBytes, stream, tmap_out, c4, scales,
+                               n_groups, G, rhat, lambda);
 }
 
 cudaError_t launch_wait_selftest(uint64_t timeout_ns, int *result, cudaStream_t stream)

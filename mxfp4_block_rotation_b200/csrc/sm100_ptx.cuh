@@ -129,6 +129,12 @@ __device__ __forceinline__ void bulk_wait_group_read0()
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
+// Same, but allow the most recent group to still be reading.
+__device__ __forceinline__ void bulk_wait_group_read1()
+{
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
 // Wait until every bulk store this thread committed has completed.
 __device__ __forceinline__ void bulk_wait_group0()
 {
