@@ -11,7 +11,7 @@
 //   warps 0-7   epilogue, two groups of four, each group taking every other stage
 //   warp 8      TMA producer (one thread)
 //   warp 9      TMEM allocator + MMA issuer (one thread)
-//   warps 10-11 builders of the MMA's B operand
+//   warps 10-11 builders of the MMA's B operand (10-13 in the smoothing kernel)
 // The rotation is a dense bf16 contraction on the tensor cores: tcgen05.mma
 // M=128, N=32, K=16, fp32 accumulate.  A is 128 groups of X staged by TMA in
 // shared memory, B = R^ in K-major form (R^T row-major), and D is 128 TMEM
@@ -29,9 +29,11 @@
 //
 // With Lambda (rotate_cols_kernel): the B operand depends on the channel
 // group, B_g = diag(1/Lambda_g)·R^, so an MMA must hold one column group over
-// 128 token rows.  A tile is 128 rows x 128 columns (4 groups).  The builder
-// warps make each tile's four B_g in fp32 and split them three ways into bf16,
-// high + middle + low (three MMAs into one accumulator, ~24 bits of B).  X stays
+// 128 token rows.  A tile is 128 rows x 128 columns (4 groups); tiles go round
+// robin over the row-major tile list, so the CTAs together read whole rows.
+// The builder warps make each tile's four B_g in fp32 and split them three
+// ways into bf16, high + middle + low (three MMAs into one accumulator, ~24
+// bits of B).  X stays
 // the exact bf16 A operand, so the smoothing adds only ~2^-25 relative error on
 // top of fp32 accumulation.  Codes go through a shared-memory staging tile and
 // one TMA bulk tensor store per tile (64 contiguous bytes per row).
@@ -75,6 +77,7 @@ struct Bars {
     uint32_t tmem_base;
     int abort;
     int eg_ok[2][2];   // per epilogue warp group, per tile parity: the leader's wait result
+    int bl_ok[2];      // per tile parity: the B builders' leader's wait result
 };
 static_assert(sizeof(Bars) <= 512, "barrier block");
 
@@ -381,49 +384,28 @@ constexpr int kColStages = 4;
 constexpr int kColStageOffset = 2 * kCodeTileBytes;           // code staging tiles first
 constexpr int kColBOffset = kColStageOffset + kColStages * kColStageBytes;
 constexpr int kColRtOffset = kColBOffset + 2 * kBSlotBytes;
-constexpr int kColBarOffset = kColRtOffset + 32 * 32 * 4;
+constexpr int kColInvOffset = kColRtOffset + 32 * 32 * 4;     // per slot: 1/Lambda of the tile's 128 channels
+constexpr int kColBarOffset = kColInvOffset + 2 * kTileCols * 8;
 constexpr int kColSmemBytes = kColBarOffset + 512 + 1024;
+constexpr int kColBuildWarps = 4;                             // warps 10-13
+constexpr int kColThreads = (kEpiWarps + 2 + kColBuildWarps) * 32;   // 448
 
-// Tile order of the smoothing kernel.  B_g depends only on the column group, so
-// each CTA walks whole column strips top to bottom and builds a strip's B_g
-// once.  With no more strips than CTAs, the grid is k CTAs per strip, each
-// taking every k-th row block.  Otherwise each CTA takes every grid-th strip in
-// turn.  At any moment the CTAs sit at about the same row block, so together
-// they still read whole rows of X.
-struct StripSched {
-    int ct0, ct_step, rt0, rt_step, per_strip, n_tiles;
-    __device__ StripSched(int n_ct, int n_rt, int cta, int grid)
+// Tile order of the smoothing kernel: round robin over the row-major tile list,
+// so at any moment the CTAs' tiles cover a few consecutive row blocks of X,
+// whole rows that DRAM reads well.
+struct TileSched {
+    int n_ct, first, step, n_tiles;
+    __device__ TileSched(int n_ct_, int n_rt, int cta, int grid) : n_ct(n_ct_), first(cta), step(grid)
     {
-        if (n_ct <= grid) {
-            ct0 = cta % n_ct;
-            ct_step = n_ct;
-            rt0 = cta / n_ct;
-            rt_step = grid / n_ct;
-        } else {
-            ct0 = cta;
-            ct_step = grid;
-            rt0 = 0;
-            rt_step = 1;
-        }
-        per_strip = rt0 < n_rt ? (n_rt - rt0 + rt_step - 1) / rt_step : 0;
-        const int strips = ct0 < n_ct ? (n_ct - ct0 + ct_step - 1) / ct_step : 0;
-        n_tiles = strips * per_strip;
+        const int total = n_ct * n_rt;
+        n_tiles = cta < total ? (total - cta + grid - 1) / grid : 0;
     }
-    __device__ int ct(int it) const { return ct0 + (it / per_strip) * ct_step; }
-    __device__ int rt(int it) const { return rt0 + (it % per_strip) * rt_step; }
+    __device__ int ct(int it) const { return (first + it * step) % n_ct; }
+    __device__ int rt(int it) const { return (first + it * step) / n_ct; }
 };
 
-__host__ int strip_grid(int n_ct, int n_rt, int num_sms)
-{
-    if (n_ct > num_sms) return num_sms;
-    int k = num_sms / n_ct;
-    if (k > n_rt) k = n_rt;
-    if (k < 1) k = 1;
-    return n_ct * k;
-}
-
 template <RotOut kMode>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kColThreads, 1)
     rotate_cols_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_codes,
                        const RotArgs args)
 {
@@ -433,6 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *stages = smem + kColStageOffset;
     uint8_t *bmat = smem + kColBOffset;
     float *rt = reinterpret_cast<float *>(smem + kColRtOffset);   // R^ as fp32, [n][k]
+    float2 *inv_tab = reinterpret_cast<float2 *>(smem + kColInvOffset);   // [slot][channel] (1/L, residual)
     Bars *bars = reinterpret_cast<Bars *>(smem + kColBarOffset);
     volatile int *abort = &bars->abort;
 
@@ -443,10 +426,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t G = cols / 32;
     const int n_ct = static_cast<int>((cols + kTileCols - 1) / kTileCols);
     const int n_rt = static_cast<int>((rows + kTileM - 1) / kTileM);
-    const StripSched sched(n_ct, n_rt, blockIdx.x, gridDim.x);
+    const TileSched sched(n_ct, n_rt, blockIdx.x, gridDim.x);
 
     const uint32_t tmem_base =
-        kernel_setup(bars, SetupCfg{kColStages, kColAcc, 1, kBuildWarps * 32, kMmaWarp}, &tmap_x,
+        kernel_setup(bars, SetupCfg{kColStages, kColAcc, 1, kColBuildWarps * 32, kMmaWarp}, &tmap_x,
                      kMode == RotOut::Quant ? &tmap_codes : nullptr);
 
     if (warp == kTmaWarp) {
@@ -502,58 +485,77 @@ __global__ void __launch_bounds__(kThreads, 1)
             drain_mmas(bars);
         }
     } else if (warp >= kBuildWarp0) {
-        // Builders: R^ in fp32, transposed to [n][k], then each tile's B_g split three ways.
-        const int bt = threadIdx.x - kBuildWarp0 * 32;
-        for (int i = bt; i < 32 * 32; i += kBuildWarps * 32) {
+        // Builders: R^ in fp32, transposed to [n][k]; then per tile 1/Lambda of its 128
+        // channels (a reciprocal plus its FMA residual, so R*(1/Lambda) is good to about
+        // an ulp), then the four B_g = diag(1/Lambda_g) R^ split three ways into bf16.
+        const int bt = threadIdx.x - kBuildWarp0 * 32;   // 0..127
+        constexpr int kB = kColBuildWarps * 32;
+        for (int i = bt; i < 32 * 32; i += kB) {
             const int k = i >> 5, n = i & 31;
             rt[n * 32 + k] = __bfloat162float(__ushort_as_bfloat16(args.rhat[i]));
         }
-        ptx::named_bar_sync(3, kBuildWarps * 32);
-        int built0 = -1, built1 = -1;   // column strip whose B_g each slot holds
+        ptx::named_bar_sync(3, kB);
+        int built0 = -1, built1 = -1;   // column tile whose B_g each slot holds
         for (int it = 0; it < sched.n_tiles; ++it) {
             const int slot = it & 1;
-            if (!wait_bar(&bars->b_empty[slot], ((it >> 1) & 1) ^ 1, abort)) break;
+            // one thread waits (bounded) for the slot; the verdict goes to all builders
+            // (the flag alternates per tile, so a slow reader never sees the next tile's value)
+            if (bt == 0) bars->bl_ok[it & 1] = wait_bar(&bars->b_empty[slot], ((it >> 1) & 1) ^ 1, abort);
+            __syncwarp();
+            ptx::named_bar_sync(3, kB);
+            if (!*reinterpret_cast<volatile int *>(&bars->bl_ok[it & 1])) break;
             const int ct = sched.ct(it);
-            if ((slot ? built1 : built0) == ct) {   // same strip: the slot's matrices are still right
-                ptx::mbar_arrive(ptx::smem_addr(&bars->b_full[slot]));
-                continue;
-            }
-            if (slot)
-                built1 = ct;
-            else
-                built0 = ct;
-            const int64_t ch_tile = static_cast<int64_t>(ct) * kTileCols;
-            uint8_t *bs = bmat + slot * kBSlotBytes;
-            // 4 groups x 32 rows (n) x 4 chunks of 8 k = 512 chunk tasks.
-            for (int task = bt; task < kColTileG * 32 * 4; task += kBuildWarps * 32) {
-                const int j = task >> 7, n = (task >> 2) & 31, c = task & 3;
-                const int64_t ch0 = ch_tile + j * 32 + c * 8;
-                uint32_t hw[4], mw[4], lw[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    __nv_bfloat16 h[2], m[2], l[2];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int k = c * 8 + 2 * e + u;
-                        const int64_t ch = ch0 + 2 * e + u;
-                        const float val = ch < cols ? __fdiv_rn(rt[n * 32 + k], args.lambda[ch]) : 0.0f;
-                        // val = hi + mid + lo to ~24 bits; each residual is exact in fp32
-                        h[u] = __float2bfloat16_rn(val);
-                        const float r1 = val - __bfloat162float(h[u]);
-                        m[u] = __float2bfloat16_rn(r1);
-                        l[u] = __float2bfloat16_rn(r1 - __bfloat162float(m[u]));
+            if ((slot ? built1 : built0) != ct) {
+                if (slot)
+                    built1 = ct;
+                else
+                    built0 = ct;
+                const int64_t ch_tile = static_cast<int64_t>(ct) * kTileCols;
+                float2 *inv = inv_tab + slot * kTileCols;
+                {
+                    const int64_t ch = ch_tile + bt;
+                    float ih = 0.0f, il = 0.0f;
+                    if (ch < cols) {
+                        const float lam = args.lambda[ch];
+                        ih = __frcp_rn(lam);
+                        il = __fmul_rn(__fmaf_rn(-lam, ih, 1.0f), ih);   // 1/lam - ih, to working precision
                     }
-                    hw[e] = pack_bf16x2(h[0], h[1]);
-                    mw[e] = pack_bf16x2(m[0], m[1]);
-                    lw[e] = pack_bf16x2(l[0], l[1]);
+                    inv[bt] = make_float2(ih, il);
                 }
-                uint8_t *bm = bs + j * kBMatBytes;
-                uint8_t *bl = bs + kBLoOffset + (j >> 1) * kBMatBytes;
-                *reinterpret_cast<uint4 *>(bm + sw128(n, c)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-                *reinterpret_cast<uint4 *>(bm + sw128(n, c + 4)) = make_uint4(mw[0], mw[1], mw[2], mw[3]);
-                *reinterpret_cast<uint4 *>(bl + sw128(n, c + 4 * (j & 1))) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                ptx::named_bar_sync(3, kB);
+                uint8_t *bs = bmat + slot * kBSlotBytes;
+                // 4 groups x 32 rows (n) x 4 chunks of 8 k = 512 chunk tasks.
+                for (int task = bt; task < kColTileG * 32 * 4; task += kB) {
+                    const int j = task >> 7, n = (task >> 2) & 31, c = task & 3;
+                    uint32_t hw[4], mw[4], lw[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        __nv_bfloat16 h[2], m[2], l[2];
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            const int k = c * 8 + 2 * e + u;
+                            const float2 iv = inv[j * 32 + k];
+                            const float r = rt[n * 32 + k];
+                            const float val = __fmaf_rn(r, iv.x, __fmul_rn(r, iv.y));   // R / Lambda
+                            // val = hi + mid + lo to ~24 bits; each residual is exact in fp32
+                            h[u] = __float2bfloat16_rn(val);
+                            const float r1 = val - __bfloat162float(h[u]);
+                            m[u] = __float2bfloat16_rn(r1);
+                            l[u] = __float2bfloat16_rn(r1 - __bfloat162float(m[u]));
+                        }
+                        hw[e] = pack_bf16x2(h[0], h[1]);
+                        mw[e] = pack_bf16x2(m[0], m[1]);
+                        lw[e] = pack_bf16x2(l[0], l[1]);
+                    }
+                    uint8_t *bm = bs + j * kBMatBytes;
+                    uint8_t *bl = bs + kBLoOffset + (j >> 1) * kBMatBytes;
+                    *reinterpret_cast<uint4 *>(bm + sw128(n, c)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                    *reinterpret_cast<uint4 *>(bm + sw128(n, c + 4)) = make_uint4(mw[0], mw[1], mw[2], mw[3]);
+                    *reinterpret_cast<uint4 *>(bl + sw128(n, c + 4 * (j & 1))) =
+                        make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                }
+                ptx::fence_proxy_async_smem();
             }
-            ptx::fence_proxy_async_smem();
             ptx::mbar_arrive(ptx::smem_addr(&bars->b_full[slot]));
         }
     } else {
@@ -659,7 +661,8 @@ constexpr int kDqAcc = 4;
 constexpr int kDqAccCols = 128;
 constexpr int kDqOutBuf = 32 * 64;                 // one epilogue warp's 32 output groups (2 KB)
 constexpr int kDqOutBytes = kEpiWarps * 2 * kDqOutBuf;   // double-buffered per epilogue warp
-constexpr int kDqSmemBytes = kDqStages * kDqStageBytes + kBMatBytes + 1024 + kDqOutBytes + 512 + 1024;
+constexpr int kDqLamBytes = kEpiWarps * 32 * 128;   // per epilogue warp: Lambda of its 32 groups
+constexpr int kDqSmemBytes = kDqStages * kDqStageBytes + kBMatBytes + 1024 + kDqOutBytes + kDqLamBytes + 512 + 1024;
 
 __device__ __forceinline__ uint32_t e2m1_bf16(uint32_t code)
 {
@@ -690,7 +693,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     uint8_t *bmat = stages + kDqStages * kDqStageBytes;
     uint32_t *lut = reinterpret_cast<uint32_t *>(bmat + kBMatBytes);   // code byte -> bf16x2
     uint8_t *outbuf = bmat + kBMatBytes + 1024;                          // epilogue staging
-    Bars *bars = reinterpret_cast<Bars *>(outbuf + kDqOutBytes);
+    uint8_t *lambuf = outbuf + kDqOutBytes;                              // epilogue Lambda rows
+    Bars *bars = reinterpret_cast<Bars *>(lambuf + kDqLamBytes);
     volatile int *abort = &bars->abort;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -777,8 +781,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         // with one TMA bulk tensor store: 2 KB contiguous instead of 16-byte pieces.
         const int q = warp & 3;
         const int ewg = warp >> 2;
-        const bool lam_vec = kLambda && ((reinterpret_cast<uintptr_t>(lambda) & 15) == 0);
         const uint32_t obuf0 = ptx::smem_addr(outbuf + warp * 2 * kDqOutBuf);
+        float *lrows = reinterpret_cast<float *>(lambuf + warp * 32 * 128);   // 32 rows x 32 channels
         int it = 0, nstore = 0;
         for (int c = blockIdx.x; c < n_chunks; c += gridDim.x, ++it) {
             if ((it & 1) != ewg) continue;
@@ -789,32 +793,38 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             ptx::tc_fence_after();
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * kDqAccCols;
             const int64_t g_warp = static_cast<int64_t>(c) * kDqStageGroups + q * 32;
-            uint32_t ra[32], rb[32];
-            ptx::tmem_ld_32cols(t_row, ra);
-            ptx::tmem_wait_ld();
-#pragma unroll
+            // (one register buffer: with 13 warps an SMSP holds four, so 128 registers a thread)
+#pragma unroll 1
             for (int j = 0; j < 4; ++j) {
-                uint32_t(&cur)[32] = (j & 1) ? rb : ra;
-                uint32_t(&nxt)[32] = (j & 1) ? ra : rb;
-                if (j + 1 < 4) ptx::tmem_ld_32cols(t_row + (j + 1) * 32, nxt);
+                uint32_t cur[32];
+                ptx::tmem_ld_32cols(t_row + j * 32, cur);
+                ptx::tmem_wait_ld();
                 const int64_t g0 = g_warp + j * 128;   // this warp's first group of MMA j
                 const int64_t g = g0 + lane;
+                // Lambda of the 32 groups' channels: fetched with coalesced loads (8 lanes per
+                // 128-byte row) into this warp's rows, 16-byte chunks XOR-swizzled by row.
+                if constexpr (kLambda) {
+                    __syncwarp();
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int r = 4 * i + (lane >> 3), cc = lane & 7;
+                        const float *src = lambda + ((g0 + r) % G) * 32 + cc * 4;
+                        float4 l4;
+                        l4.x = __ldg(src);
+                        l4.y = __ldg(src + 1);
+                        l4.z = __ldg(src + 2);
+                        l4.w = __ldg(src + 3);
+                        *reinterpret_cast<float4 *>(lrows + r * 32 + ((cc ^ (r & 7)) << 2)) = l4;
+                    }
+                    __syncwarp();
+                }
                 // times Lambda_k (channels of this group), then round to bf16 pairs
                 uint32_t o[16];
-                const float *lg = kLambda ? lambda + (g < n_groups ? g % G : 0) * 32 : nullptr;
 #pragma unroll
                 for (int k4 = 0; k4 < 8; ++k4) {
                     float4 l4 = make_float4(1.0f, 1.0f, 1.0f, 1.0f);
-                    if constexpr (kLambda) {
-                        if (lam_vec) {
-                            l4 = __ldg(reinterpret_cast<const float4 *>(lg) + k4);
-                        } else {
-                            l4.x = __ldg(lg + 4 * k4);
-                            l4.y = __ldg(lg + 4 * k4 + 1);
-                            l4.z = __ldg(lg + 4 * k4 + 2);
-                            l4.w = __ldg(lg + 4 * k4 + 3);
-                        }
-                    }
+                    if constexpr (kLambda)
+                        l4 = *reinterpret_cast<const float4 *>(lrows + lane * 32 + ((k4 ^ (lane & 7)) << 2));
                     const __nv_bfloat162 p0 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(cur[4 * k4]), l4.x),
                                                                     __fmul_rn(__uint_as_float(cur[4 * k4 + 1]), l4.y));
                     const __nv_bfloat162 p1 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(cur[4 * k4 + 2]), l4.z),
@@ -839,7 +849,6 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                     ptx::bulk_commit_group();
                 }
                 ++nstore;
-                if (j + 1 < 4) ptx::tmem_wait_ld();
             }
             ptx::tc_fence_before();
             __syncwarp();
@@ -904,12 +913,12 @@ cudaError_t launch_rotate(const RotMaps &maps, const RotArgs &args, RotOut mode,
                    : launch_pdl(rotate_flat_kernel<RotOut::F32>, grid, kThreads, kFlatSmemBytes, stream, maps.groups,
                                 args);
     }
-    const int grid = strip_grid(static_cast<int>((args.cols + kTileCols - 1) / kTileCols),
-                                static_cast<int>((args.rows + kTileM - 1) / kTileM), num_sms);
+    const int64_t n_tiles = ((args.rows + kTileM - 1) / kTileM) * ((args.cols + kTileCols - 1) / kTileCols);
+    const int grid = static_cast<int>(n_tiles < num_sms ? n_tiles : num_sms);
     return mode == RotOut::Quant
-               ? launch_pdl(rotate_cols_kernel<RotOut::Quant>, grid, kThreads, kColSmemBytes, stream, maps.x,
+               ? launch_pdl(rotate_cols_kernel<RotOut::Quant>, grid, kColThreads, kColSmemBytes, stream, maps.x,
                             maps.codes, args)
-               : launch_pdl(rotate_cols_kernel<RotOut::F32>, grid, kThreads, kColSmemBytes, stream, maps.x,
+               : launch_pdl(rotate_cols_kernel<RotOut::F32>, grid, kColThreads, kColSmemBytes, stream, maps.x,
                             maps.codes, args);
 }
 
