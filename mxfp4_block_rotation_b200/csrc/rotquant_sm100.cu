@@ -390,18 +390,44 @@ constexpr int kColSmemBytes = kColBarOffset + 512 + 1024;
 constexpr int kColBuildWarps = 4;                             // warps 10-13
 constexpr int kColThreads = (kEpiWarps + 2 + kColBuildWarps) * 32;   // 448
 
-// Tile order of the smoothing kernel: round robin over the row-major tile list,
-// so at any moment the CTAs' tiles cover a few consecutive row blocks of X,
-// whole rows that DRAM reads well.
-struct TileSched {
-    int n_ct, first, step, n_tiles;
-    __device__ TileSched(int n_ct_, int n_rt, int cta, int grid) : n_ct(n_ct_), first(cta), step(grid)
+// Tile order of the smoothing kernel.  A unit is kUnitRows consecutive row
+// blocks of one column tile, so one B_g build serves kUnitRows tiles.  Units are
+// numbered band-major (u = band * n_ct + ct) and dealt round robin to the CTAs.
+// At any moment the CTAs' units therefore cover whole rows of a couple of row
+// bands, which DRAM reads well.  Only the last band can be shorter than
+// kUnitRows, and a CTA meets it only in its last units, so a CTA's it-th tile
+// has a closed form.
+constexpr int kUnitRows = 2;
+
+struct UnitSched {
+    int n_ct, cta, grid, r_last, k_full, n_units_cta, n_tiles;
+    __device__ UnitSched(int n_ct_, int n_rt, int cta_, int grid_) : n_ct(n_ct_), cta(cta_), grid(grid_)
     {
-        const int total = n_ct * n_rt;
-        n_tiles = cta < total ? (total - cta + grid - 1) / grid : 0;
+        const int n_bands = (n_rt + kUnitRows - 1) / kUnitRows;
+        r_last = n_rt - (n_bands - 1) * kUnitRows;
+        const int n_units = n_ct * n_bands;
+        n_units_cta = cta < n_units ? (n_units - cta + grid - 1) / grid : 0;
+        const int before_last = (n_bands - 1) * n_ct;   // units in full bands
+        const int k = cta < before_last ? (before_last - cta + grid - 1) / grid : 0;
+        k_full = k < n_units_cta ? k : n_units_cta;
+        n_tiles = k_full * kUnitRows + (n_units_cta - k_full) * r_last;
     }
-    __device__ int ct(int it) const { return (first + it * step) % n_ct; }
-    __device__ int rt(int it) const { return (first + it * step) / n_ct; }
+    // The it-th tile of this CTA: its unit's ordinal ui, the position in the unit and the unit's length.
+    __device__ void at(int it, int &ui, int &sub, int &len) const
+    {
+        if (it < k_full * kUnitRows) {
+            ui = it / kUnitRows;
+            sub = it % kUnitRows;
+            len = kUnitRows;
+        } else {
+            const int t = it - k_full * kUnitRows;
+            ui = k_full + t / r_last;
+            sub = t % r_last;
+            len = r_last;
+        }
+    }
+    __device__ int ct_of_unit(int ui) const { return (cta + ui * grid) % n_ct; }
+    __device__ int rt0_of_unit(int ui) const { return ((cta + ui * grid) / n_ct) * kUnitRows; }
 };
 
 template <RotOut kMode>
@@ -426,7 +452,7 @@ __global__ void __launch_bounds__(kColThreads, 1)
     const int64_t G = cols / 32;
     const int n_ct = static_cast<int>((cols + kTileCols - 1) / kTileCols);
     const int n_rt = static_cast<int>((rows + kTileM - 1) / kTileM);
-    const TileSched sched(n_ct, n_rt, blockIdx.x, gridDim.x);
+    const UnitSched sched(n_ct, n_rt, blockIdx.x, gridDim.x);
 
     const uint32_t tmem_base =
         kernel_setup(bars, SetupCfg{kColStages, kColAcc, 1, kColBuildWarps * 32, kMmaWarp}, &tmap_x,
@@ -439,7 +465,9 @@ __global__ void __launch_bounds__(kColThreads, 1)
             for (; it < sched.n_tiles; ++it) {
                 const int s = it % kColStages;
                 if (!wait_bar(&bars->empty[s], ((it / kColStages) & 1) ^ 1, abort)) break;
-                const int rtile = sched.rt(it), ctile = sched.ct(it);
+                int ui, sub, len;
+                sched.at(it, ui, sub, len);
+                const int ctile = sched.ct_of_unit(ui), rtile = sched.rt0_of_unit(ui) + sub;
                 const uint32_t full = ptx::smem_addr(&bars->full[s]);
                 const uint32_t dst = ptx::smem_addr(stages + s * kColStageBytes);
                 ptx::mbar_arrive_expect_tx(full, kColStageBytes);
@@ -455,10 +483,12 @@ __global__ void __launch_bounds__(kColThreads, 1)
             for (int it = 0; it < sched.n_tiles; ++it) {
                 const int s = it % kColStages;
                 const int a = it % kColAcc;
-                const int slot = it & 1;
+                int ui, sub, len;
+                sched.at(it, ui, sub, len);
+                const int slot = ui & 1;
                 if (!wait_bar(&bars->full[s], (it / kColStages) & 1, abort)) break;
                 if (!wait_bar(&bars->acc_empty[a], ((it / kColAcc) & 1) ^ 1, abort)) break;
-                if (!wait_bar(&bars->b_full[slot], (it >> 1) & 1, abort)) break;
+                if (sub == 0 && !wait_bar(&bars->b_full[slot], (ui >> 1) & 1, abort)) break;
                 ptx::tc_fence_after();
                 const uint32_t a_base = ptx::smem_addr(stages + s * kColStageBytes);
                 const uint32_t b_base = b_base0 + slot * kBSlotBytes;
@@ -480,7 +510,7 @@ __global__ void __launch_bounds__(kColThreads, 1)
                 }
                 ptx::mma_commit(ptx::smem_addr(&bars->empty[s]));
                 ptx::mma_commit(ptx::smem_addr(&bars->acc_full[a]));
-                ptx::mma_commit(ptx::smem_addr(&bars->b_empty[slot]));
+                if (sub == len - 1) ptx::mma_commit(ptx::smem_addr(&bars->b_empty[slot]));
             }
             drain_mmas(bars);
         }
@@ -496,15 +526,15 @@ __global__ void __launch_bounds__(kColThreads, 1)
         }
         ptx::named_bar_sync(3, kB);
         int built0 = -1, built1 = -1;   // column tile whose B_g each slot holds
-        for (int it = 0; it < sched.n_tiles; ++it) {
-            const int slot = it & 1;
+        for (int ui = 0; ui < sched.n_units_cta; ++ui) {
+            const int slot = ui & 1;
             // one thread waits (bounded) for the slot; the verdict goes to all builders
-            // (the flag alternates per tile, so a slow reader never sees the next tile's value)
-            if (bt == 0) bars->bl_ok[it & 1] = wait_bar(&bars->b_empty[slot], ((it >> 1) & 1) ^ 1, abort);
+            // (the flag alternates per unit, so a slow reader never sees the next unit's value)
+            if (bt == 0) bars->bl_ok[ui & 1] = wait_bar(&bars->b_empty[slot], ((ui >> 1) & 1) ^ 1, abort);
             __syncwarp();
             ptx::named_bar_sync(3, kB);
-            if (!*reinterpret_cast<volatile int *>(&bars->bl_ok[it & 1])) break;
-            const int ct = sched.ct(it);
+            if (!*reinterpret_cast<volatile int *>(&bars->bl_ok[ui & 1])) break;
+            const int ct = sched.ct_of_unit(ui);
             if ((slot ? built1 : built0) != ct) {
                 if (slot)
                     built1 = ct;
@@ -579,7 +609,9 @@ __global__ void __launch_bounds__(kColThreads, 1)
             ptx::named_bar_sync(1 + ewg, 128);
             if (!*ok_slot) break;
             ptx::tc_fence_after();
-            const int rtile = sched.rt(it), ctile = sched.ct(it);
+            int ui, sub, len;
+            sched.at(it, ui, sub, len);
+            const int ctile = sched.ct_of_unit(ui), rtile = sched.rt0_of_unit(ui) + sub;
             const int r_local = q * 32 + lane;
             const int64_t row = static_cast<int64_t>(rtile) * kTileM + r_local;
             const bool row_ok = row < rows;
@@ -782,6 +814,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         const int q = warp & 3;
         const int ewg = warp >> 2;
         const uint32_t obuf0 = ptx::smem_addr(outbuf + warp * 2 * kDqOutBuf);
+        const bool lam_vec = kLambda && ((reinterpret_cast<uintptr_t>(lambda) & 15) == 0);
         float *lrows = reinterpret_cast<float *>(lambuf + warp * 32 * 128);   // 32 rows x 32 channels
         int it = 0, nstore = 0;
         for (int c = blockIdx.x; c < n_chunks; c += gridDim.x, ++it) {
@@ -800,20 +833,24 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                 ptx::tmem_ld_32cols(t_row + j * 32, cur);
                 ptx::tmem_wait_ld();
                 const int64_t g0 = g_warp + j * 128;   // this warp's first group of MMA j
-                const int64_t g = g0 + lane;
                 // Lambda of the 32 groups' channels: fetched with coalesced loads (8 lanes per
                 // 128-byte row) into this warp's rows, 16-byte chunks XOR-swizzled by row.
                 if constexpr (kLambda) {
                     __syncwarp();
+                    const int col0 = static_cast<int>(g0 % G);   // column group of this warp's first group
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         const int r = 4 * i + (lane >> 3), cc = lane & 7;
-                        const float *src = lambda + ((g0 + r) % G) * 32 + cc * 4;
+                        const float *src = lambda + static_cast<int64_t>((col0 + r) % static_cast<int>(G)) * 32 + cc * 4;
                         float4 l4;
-                        l4.x = __ldg(src);
-                        l4.y = __ldg(src + 1);
-                        l4.z = __ldg(src + 2);
-                        l4.w = __ldg(src + 3);
+                        if (lam_vec) {
+                            l4 = __ldg(reinterpret_cast<const float4 *>(src));
+                        } else {
+                            l4.x = __ldg(src);
+                            l4.y = __ldg(src + 1);
+                            l4.z = __ldg(src + 2);
+                            l4.w = __ldg(src + 3);
+                        }
                         *reinterpret_cast<float4 *>(lrows + r * 32 + ((cc ^ (r & 7)) << 2)) = l4;
                     }
                     __syncwarp();
