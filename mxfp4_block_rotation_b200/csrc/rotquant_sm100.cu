@@ -397,7 +397,7 @@ constexpr int kColThreads = (kEpiWarps + 2 + kColBuildWarps) * 32;   // 448
 // bands, which DRAM reads well.  Only the last band can be shorter than
 // kUnitRows, and a CTA meets it only in its last units, so a CTA's it-th tile
 // has a closed form.
-constexpr int kUnitRows = 2;
+constexpr int kUnitRows = 4;
 
 struct UnitSched {
     int n_ct, cta, grid, r_last, k_full, n_units_cta, n_tiles;
