@@ -46,7 +46,8 @@ UNIT = "GB/s"
 WORKLOAD = ("down-proj input 8192x14336 bf16 (Student-t(3), 8 tokens x 4 channels of 1e3-1e4 outliers), "
             "random orthogonal 32x32 R, no smoothing -> MXFP4 codes + E8M0 scales")
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_SOURCES = ["mxfp4_block_rotation_b200/csrc/rotquant_sm100.cu",
+KERNEL_SOURCES = ["mxfp4_block_rotation_b200/csrc/rotate_flat_sm100.cu",
+                  "mxfp4_block_rotation_b200/csrc/pipeline_sm100.cuh",
                   "mxfp4_block_rotation_b200/csrc/sm100_ptx.cuh"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "rotate_kernel_downproj_traffic.json")
 

@@ -232,12 +232,17 @@ mxq_status rotate_common(const void *X, int64_t rows, int64_t cols, const void *
     if ((st = check_buffer(out0, out0_bytes, dev)) != MXQ_OK) return st;
     if (out1 && (st = check_buffer(out1, out1_bytes, dev)) != MXQ_OK) return st;
 
-    mxq::RotMaps maps;
+    alignas(64) CUtensorMap map_a;   // X as [n_groups, 32] (no smoothing) or [rows, cols]
+    alignas(64) CUtensorMap map_c;   // the packed codes (smoothing, quantise mode)
     if (lam == nullptr) {
-        if ((st = make_tmap_groups(&maps.groups, X, rows, cols)) != MXQ_OK) return st;
+        if ((st = make_tmap_groups(&map_a, X, rows, cols)) != MXQ_OK) return st;
     } else {
-        if ((st = make_tmap_x(&maps.x, X, rows, cols)) != MXQ_OK) return st;
-        if (mode == mxq::RotOut::Quant && (st = make_tmap_codes(&maps.codes, out0, rows, cols)) != MXQ_OK) return st;
+        if ((st = make_tmap_x(&map_a, X, rows, cols)) != MXQ_OK) return st;
+        if (mode == mxq::RotOut::Quant) {
+            if ((st = make_tmap_codes(&map_c, out0, rows, cols)) != MXQ_OK) return st;
+        } else {
+            map_c = map_a;   // unused by the fp32 variant
+        }
     }
     mxq::RotArgs args{};
     args.rhat = static_cast<const uint16_t *>(R);
@@ -250,7 +255,9 @@ mxq_status rotate_common(const void *X, int64_t rows, int64_t cols, const void *
     } else {
         args.y = static_cast<float *>(out0);
     }
-    cudaError_t e = mxq::launch_rotate(maps, args, mode, sms, static_cast<cudaStream_t>(stream));
+    cudaError_t e = lam == nullptr
+                        ? mxq::launch_rotate_flat(map_a, args, mode, sms, static_cast<cudaStream_t>(stream))
+                        : mxq::launch_rotate_cols(map_a, map_c, args, mode, sms, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) {
         note_cuda(e, "launch rotate kernel");
         return MXQ_ERR_CUDA;

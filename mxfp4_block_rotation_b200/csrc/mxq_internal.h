@@ -26,19 +26,16 @@ struct RotArgs {
     int64_t cols;
 };
 
-// TMA descriptors the rotate kernels read.  Without Lambda only `groups` is used:
-// X as a dense [rows*cols/32, 32] bf16 matrix (box {32, 256}, 64-byte swizzle).
-// With Lambda, `x` is X as [rows, cols] bf16 (box {64, 128}, 128-byte swizzle)
-// and `codes` the packed codes as [rows, cols/2] uint8 (box {64, 128}, 64-byte
-// swizzle; Quant mode only).
-struct RotMaps {
-    alignas(64) CUtensorMap groups;
-    alignas(64) CUtensorMap x;
-    alignas(64) CUtensorMap codes;
-};
+// Fused rotate -> MXFP4 without smoothing.  `tmap_groups` views X as a dense
+// [rows*cols/32, 32] bf16 matrix (box {32, 256}, 64-byte swizzle).
+cudaError_t launch_rotate_flat(const CUtensorMap &tmap_groups, const RotArgs &args, RotOut mode, int num_sms,
+                               cudaStream_t stream);
 
-// Launch the fused smooth-rotate(-quantize) kernel for `args`.
-cudaError_t launch_rotate(const RotMaps &maps, const RotArgs &args, RotOut mode, int num_sms, cudaStream_t stream);
+// Fused smooth -> rotate -> MXFP4 (args.lambda non-null).  `tmap_x` views X as
+// [rows, cols] bf16 (box {64, 128}, 128-byte swizzle); `tmap_codes` the packed
+// codes as [rows, cols/2] uint8 (box {64, 128}, 64-byte swizzle; Quant mode only).
+cudaError_t launch_rotate_cols(const CUtensorMap &tmap_x, const CUtensorMap &tmap_codes, const RotArgs &args,
+                               RotOut mode, int num_sms, cudaStream_t stream);
 
 // Dequantise to bf16 in the rotated domain (codes 16-byte aligned, out 16-byte aligned).
 cudaError_t launch_dequant_plain(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t cols,
@@ -54,6 +51,9 @@ cudaError_t launch_dequant_rot(const CUtensorMap &tmap_out, const uint8_t *codes
 // Diagnostic kernel: a bounded wait on a barrier nothing completes (writes 2 to
 // *result once the wait ran out and the abort flag was raised).
 cudaError_t launch_wait_selftest(uint64_t timeout_ns, int *result, cudaStream_t stream);
+
+// Device address of the status word on the current device (nullptr on failure).
+unsigned int *status_word();
 
 // Read-and-clear of the device status word, stream ordered.
 cudaError_t read_and_clear_status(unsigned int *host_status, cudaStream_t stream);

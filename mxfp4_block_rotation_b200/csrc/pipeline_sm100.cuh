@@ -1,0 +1,210 @@
+// pipeline_sm100.cuh -- pieces shared by the warp-specialised tcgen05 kernels
+// (rotate_flat_sm100.cu, rotate_cols_sm100.cu, dequant_sm100.cu): warp roles,
+// the shared-memory barrier block, the bounded mbarrier wait, the MXFP4 group
+// quantiser, kernel set-up / tear-down and the programmatic-dependent launch.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "mxq_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace mxq {
+namespace pipe {
+
+constexpr uint32_t kTmemCols = 512;      // all of TMEM: accumulator stages of 32 columns per MMA
+constexpr int kMaxAcc = 8;
+constexpr int kEpiWarps = 8;
+constexpr int kTmaWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kBuildWarp0 = 10;
+constexpr int kBuildWarps = 2;
+constexpr int kThreads = (kEpiWarps + 2 + kBuildWarps) * 32;   // 384, the flat rotate kernel
+constexpr int kBMatBytes = 32 * 128;     // one B atom: 32 rows (n) x 128 B, 128-byte swizzle
+constexpr uint64_t kTimeoutNs = 2000000000ull;   // 2 s per wait
+constexpr int kMaxStages = 8;
+
+struct Bars {
+    uint64_t full[kMaxStages];
+    uint64_t empty[kMaxStages];
+    uint64_t acc_full[kMaxAcc];
+    uint64_t acc_empty[kMaxAcc];
+    uint64_t b_full[2];
+    uint64_t b_empty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+    int eg_ok[2][2];   // per epilogue warp group, per tile parity: the leader's wait result
+    int bl_ok[2];      // per tile parity: the B builders' leader's wait result
+};
+static_assert(sizeof(Bars) <= 512, "barrier block");
+
+// Bounded wait on an mbarrier phase.  False if the wait ran out or (when abort
+// is non-null) another role has already aborted.  Drains at exit pass a null
+// abort so they keep waiting, within the time bound, for work already in flight.
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned int *status,
+                                         uint64_t timeout_ns = kTimeoutNs)
+{
+    const uint32_t b = ptx::smem_addr(bar);
+    if (ptx::mbar_try_wait(b, parity)) return true;
+    const uint64_t t0 = ptx::globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (ptx::mbar_try_wait(b, parity)) return true;
+        if ((i & 63) == 0) {
+            if (abort && *abort) return false;
+            if (ptx::globaltimer_ns() - t0 > timeout_ns || i > (1u << 30)) {
+                if (abort) *abort = 1;
+                atomicOr(status, kStatusTimeout);
+                return false;
+            }
+        }
+    }
+}
+
+// Byte offset of 16-byte chunk c of row r inside a 128-byte-swizzled atom.
+__device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t c)
+{
+    return r * 128u + ((c ^ (r & 7u)) << 4);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(__nv_bfloat16 lo, __nv_bfloat16 hi)
+{
+    return static_cast<uint32_t>(__bfloat16_as_ushort(lo)) |
+           (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
+}
+
+__device__ __forceinline__ uint8_t *align_1k(uint8_t *p)
+{
+    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~static_cast<uintptr_t>(1023));
+}
+
+// MXFP4 of one 32-value group (fp32 bit patterns): returns the E8M0 byte and
+// writes the 32 E2M1 codes packed into four words (value 2i in the low nibble
+// of byte i).  E8M0 = floor(log2 amax) - 2 + 127 comes straight from amax's
+// exponent field (clamped at 0); 2^-e is built from bits, so the scaling is exact.
+__device__ __forceinline__ uint32_t quantize_group(const uint32_t (&r)[32], uint32_t (&w)[4])
+{
+    float m[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        m[i] = ptx::fmax_nan(fabsf(__uint_as_float(r[2 * i])), fabsf(__uint_as_float(r[2 * i + 1])));
+#pragma unroll
+    for (int step = 8; step >= 1; step >>= 1)
+#pragma unroll
+        for (int i = 0; i < step; ++i) m[i] = ptx::fmax_nan(m[i], m[i + step]);
+    const uint32_t E = (__float_as_uint(m[0]) >> 23) & 0xFFu;
+    if (E == 0xFFu) {   // NaN/Inf group: scale byte 0xFF, codes 0
+        w[0] = w[1] = w[2] = w[3] = 0u;
+        return 0xFFu;
+    }
+    const uint32_t byte = E > 2u ? E - 2u : 0u;
+    const float s = __uint_as_float((254u - byte) << 23);   // 2^-e
+    float u[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) u[i] = __fmul_rn(__uint_as_float(r[i]), s);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        w[q] = ptx::cvt_e2m1x8(u[8 * q], u[8 * q + 1], u[8 * q + 2], u[8 * q + 3], u[8 * q + 4], u[8 * q + 5],
+                               u[8 * q + 6], u[8 * q + 7]);
+    return byte;
+}
+
+// Per-kernel numbers the shared set-up needs.
+struct SetupCfg {
+    int n_stages;     // shared-memory stages (full/empty barrier pairs)
+    int n_acc;        // TMEM accumulator stages
+    int full_count;   // arrivals that complete a stage's full barrier (1 for a TMA producer)
+    int b_count;      // arrivals that complete b_full (the B builders' threads)
+    int mma_warp;     // the warp that owns TMEM
+};
+
+// Barrier initialisation, TMEM allocation and the programmatic-dependent-launch
+// handshake shared by the kernels.  Returns the TMEM base address.
+__device__ __forceinline__ uint32_t kernel_setup(Bars *bars, const SetupCfg &cfg, const CUtensorMap *map0,
+                                                 const CUtensorMap *map1)
+{
+    const int warp = threadIdx.x >> 5;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < cfg.n_stages; ++s) {
+            ptx::mbar_init(ptx::smem_addr(&bars->full[s]), cfg.full_count);
+            ptx::mbar_init(ptx::smem_addr(&bars->empty[s]), 1);
+        }
+        for (int a = 0; a < cfg.n_acc; ++a) {
+            ptx::mbar_init(ptx::smem_addr(&bars->acc_full[a]), 1);
+            ptx::mbar_init(ptx::smem_addr(&bars->acc_empty[a]), kEpiWarps / 2);
+        }
+        for (int s = 0; s < 2; ++s) {
+            ptx::mbar_init(ptx::smem_addr(&bars->b_full[s]), cfg.b_count);
+            ptx::mbar_init(ptx::smem_addr(&bars->b_empty[s]), 1);
+        }
+        ptx::mbar_init(ptx::smem_addr(&bars->drain), 1);
+        bars->abort = 0;
+        ptx::fence_mbar_init();
+        if (map0) ptx::prefetch_tmap(map0);
+        if (map1) ptx::prefetch_tmap(map1);
+    }
+    if (warp == cfg.mma_warp) {
+        ptx::tmem_alloc(ptx::smem_addr(&bars->tmem_base), kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    // Nothing above touches global memory, so the next kernel in the stream may start
+    // its own set-up now; every global access below waits for the previous kernel.
+    ptx::griddep_launch_dependents();
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = bars->tmem_base;
+    ptx::griddep_wait();
+    return tmem_base;
+}
+
+// Producer epilogue: let the last copy into each stage land before the CTA can exit.
+__device__ __forceinline__ void drain_loads(Bars *bars, int n_stages, int issued, unsigned int *status)
+{
+    for (int s = 0; s < n_stages && s < issued; ++s) {
+        const int last = issued - 1 - ((issued - 1 - s) % n_stages);
+        wait_bar(&bars->full[s], (last / n_stages) & 1, nullptr, status);
+    }
+}
+
+// MMA epilogue: every MMA this thread issued must finish before TMEM is freed.
+__device__ __forceinline__ void drain_mmas(Bars *bars, unsigned int *status)
+{
+    ptx::mma_commit(ptx::smem_addr(&bars->drain));
+    wait_bar(&bars->drain, 0, nullptr, status);
+}
+
+__device__ __forceinline__ void kernel_teardown(uint32_t tmem_base, int mma_warp)
+{
+    ptx::tc_fence_before();
+    __syncthreads();
+    if ((threadIdx.x >> 5) == mma_warp) {
+        __syncwarp();
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+// Launch with programmatic stream serialisation: the grid may start while the
+// previous kernel in the stream drains (the kernels order their global accesses
+// with griddepcontrol.wait).
+template <typename Kern, typename... Args>
+cudaError_t launch_pdl(Kern kern, int grid, int block, int smem, cudaStream_t stream, Args... args)
+{
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+}  // namespace pipe
+}  // namespace mxq

@@ -1,0 +1,344 @@
+// rotate_cols_sm100.cu -- fused smooth -> rotate -> MXFP4-quantise kernel (B200, sm_100a).
+//
+// The online step of the DuQuant++ write-up (jsqmd.com/news/928156) with the
+// SmoothQuant scale: X_hat = X * Lambda^-1 * R^ (§3.1, §3.3), quantised to MXFP4 as
+// in §2.1.  The B operand depends on the channel group, B_g = diag(1/Lambda_g)·R^,
+// so an MMA must hold one column group over 128 token rows.  A tile is 128 rows x
+// 128 columns (4 groups), loaded as two 128-byte-swizzled TMA boxes.
+//
+// Warp roles as in the flat kernel, with four builder warps (10-13).  Per unit
+// (4 row blocks of one column tile) they make the tile's four B_g in fp32: a
+// reciprocal per channel plus its FMA residual, so R*(1/Lambda) is good to about
+// an ulp.  Each B_g is then split three ways into bf16, high + middle + low
+// (three MMAs into one accumulator, ~24 bits of B).  X stays the exact bf16 A
+// operand, so the smoothing adds only ~2^-25 relative error on top of fp32
+// accumulation.  Codes go through a shared-memory staging tile (64-byte swizzle)
+// and one TMA bulk tensor store per tile (64 contiguous bytes per row).
+#include "pipeline_sm100.cuh"
+
+namespace mxq {
+namespace {
+
+using namespace pipe;
+
+constexpr int kColTileG = 4;                                  // groups per tile
+constexpr int kColAcc = 4;                                    // accumulator stages of 128 columns
+constexpr int kColAccCols = 128;
+constexpr int kColStageBytes = kTileM * kTileCols * 2;        // 32 KB of bf16 per stage
+constexpr int kColBoxBytes = kColStageBytes / 2;              // one TMA box: 128 rows x 128 B
+constexpr int kCodeTileBytes = kTileM * kColTileG * 16;       // 128 rows x 64 B of packed codes
+// A tile's B slot holds, per group j, an atom [hi | mid] at j*4 KB and the low
+// parts of groups 2p and 2p+1 side by side in the atom at 16 KB + p*4 KB.
+constexpr int kBLoOffset = kColTileG * kBMatBytes;
+constexpr int kBSlotBytes = kBLoOffset + (kColTileG / 2) * kBMatBytes;   // 24 KB
+constexpr int kColStages = 4;
+constexpr int kColStageOffset = 2 * kCodeTileBytes;           // code staging tiles first
+constexpr int kColBOffset = kColStageOffset + kColStages * kColStageBytes;
+constexpr int kColRtOffset = kColBOffset + 2 * kBSlotBytes;
+constexpr int kColInvOffset = kColRtOffset + 32 * 32 * 4;     // per slot: 1/Lambda of the tile's 128 channels
+constexpr int kColBarOffset = kColInvOffset + 2 * kTileCols * 8;
+constexpr int kColSmemBytes = kColBarOffset + 512 + 1024;
+constexpr int kColBuildWarps = 4;                             // warps 10-13
+constexpr int kColThreads = (kEpiWarps + 2 + kColBuildWarps) * 32;   // 448
+
+// Tile order of the smoothing kernel.  A unit is kUnitRows consecutive row
+// blocks of one column tile, so one B_g build serves kUnitRows tiles.  Units are
+// numbered band-major (u = band * n_ct + ct) and dealt round robin to the CTAs.
+// At any moment the CTAs' units therefore cover whole rows of a couple of row
+// bands, which DRAM reads well.  Only the last band can be shorter than
+// kUnitRows, and a CTA meets it only in its last units, so a CTA's it-th tile
+// has a closed form.
+constexpr int kUnitRows = 4;
+
+struct UnitSched {
+    int n_ct, cta, grid, r_last, k_full, n_units_cta, n_tiles;
+    __device__ UnitSched(int n_ct_, int n_rt, int cta_, int grid_) : n_ct(n_ct_), cta(cta_), grid(grid_)
+    {
+        const int n_bands = (n_rt + kUnitRows - 1) / kUnitRows;
+        r_last = n_rt - (n_bands - 1) * kUnitRows;
+        const int n_units = n_ct * n_bands;
+        n_units_cta = cta < n_units ? (n_units - cta + grid - 1) / grid : 0;
+        const int before_last = (n_bands - 1) * n_ct;   // units in full bands
+        const int k = cta < before_last ? (before_last - cta + grid - 1) / grid : 0;
+        k_full = k < n_units_cta ? k : n_units_cta;
+        n_tiles = k_full * kUnitRows + (n_units_cta - k_full) * r_last;
+    }
+    // The it-th tile of this CTA: its unit's ordinal ui, the position in the unit and the unit's length.
+    __device__ void at(int it, int &ui, int &sub, int &len) const
+    {
+        if (it < k_full * kUnitRows) {
+            ui = it / kUnitRows;
+            sub = it % kUnitRows;
+            len = kUnitRows;
+        } else {
+            const int t = it - k_full * kUnitRows;
+            ui = k_full + t / r_last;
+            sub = t % r_last;
+            len = r_last;
+        }
+    }
+    __device__ int ct_of_unit(int ui) const { return (cta + ui * grid) % n_ct; }
+    __device__ int rt0_of_unit(int ui) const { return ((cta + ui * grid) / n_ct) * kUnitRows; }
+};
+
+template <RotOut kMode>
+__global__ void __launch_bounds__(kColThreads, 1)
+    rotate_cols_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_codes,
+                       const RotArgs args, unsigned int *status)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = align_1k(smem_raw);
+    uint8_t *code_tiles = smem;                       // one staging tile per epilogue warp group
+    uint8_t *stages = smem + kColStageOffset;
+    uint8_t *bmat = smem + kColBOffset;
+    float *rt = reinterpret_cast<float *>(smem + kColRtOffset);   // R^ as fp32, [n][k]
+    float2 *inv_tab = reinterpret_cast<float2 *>(smem + kColInvOffset);   // [slot][channel] (1/L, residual)
+    Bars *bars = reinterpret_cast<Bars *>(smem + kColBarOffset);
+    volatile int *abort = &bars->abort;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t rows = args.rows;
+    const int64_t cols = args.cols;
+    const int64_t G = cols / 32;
+    const int n_ct = static_cast<int>((cols + kTileCols - 1) / kTileCols);
+    const int n_rt = static_cast<int>((rows + kTileM - 1) / kTileM);
+    const UnitSched sched(n_ct, n_rt, blockIdx.x, gridDim.x);
+
+    const uint32_t tmem_base =
+        kernel_setup(bars, SetupCfg{kColStages, kColAcc, 1, kColBuildWarps * 32, kMmaWarp}, &tmap_x,
+                     kMode == RotOut::Quant ? &tmap_codes : nullptr);
+
+    if (warp == kTmaWarp) {
+        if (lane == 0) {
+            const uint64_t pol = ptx::policy_evict_first();
+            int it = 0;
+            for (; it < sched.n_tiles; ++it) {
+                const int s = it % kColStages;
+                if (!wait_bar(&bars->empty[s], ((it / kColStages) & 1) ^ 1, abort, status)) break;
+                int ui, sub, len;
+                sched.at(it, ui, sub, len);
+                const int ctile = sched.ct_of_unit(ui), rtile = sched.rt0_of_unit(ui) + sub;
+                const uint32_t full = ptx::smem_addr(&bars->full[s]);
+                const uint32_t dst = ptx::smem_addr(stages + s * kColStageBytes);
+                ptx::mbar_arrive_expect_tx(full, kColStageBytes);
+                ptx::tma_load_2d(dst, &tmap_x, ctile * kTileCols, rtile * kTileM, full, pol);
+                ptx::tma_load_2d(dst + kColBoxBytes, &tmap_x, ctile * kTileCols + 64, rtile * kTileM, full, pol);
+            }
+            drain_loads(bars, kColStages, it, status);
+        }
+    } else if (warp == kMmaWarp) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = ptx::idesc_bf16_f32(128, 32);
+            const uint32_t b_base0 = ptx::smem_addr(bmat);
+            for (int it = 0; it < sched.n_tiles; ++it) {
+                const int s = it % kColStages;
+                const int a = it % kColAcc;
+                int ui, sub, len;
+                sched.at(it, ui, sub, len);
+                const int slot = ui & 1;
+                if (!wait_bar(&bars->full[s], (it / kColStages) & 1, abort, status)) break;
+                if (!wait_bar(&bars->acc_empty[a], ((it / kColAcc) & 1) ^ 1, abort, status)) break;
+                if (sub == 0 && !wait_bar(&bars->b_full[slot], (ui >> 1) & 1, abort, status)) break;
+                ptx::tc_fence_after();
+                const uint32_t a_base = ptx::smem_addr(stages + s * kColStageBytes);
+                const uint32_t b_base = b_base0 + slot * kBSlotBytes;
+                const uint32_t d_base = tmem_base + static_cast<uint32_t>(a * kColAccCols);
+#pragma unroll
+                for (int j = 0; j < kColTileG; ++j) {
+                    const uint32_t a_j = a_base + (j >> 1) * kColBoxBytes + (j & 1) * 64;
+                    const uint32_t d_j = d_base + j * 32;
+#pragma unroll
+                    for (int kh = 0; kh < 2; ++kh) {
+                        const uint64_t ad = ptx::smem_desc_sw128(a_j + kh * 32);
+                        // smallest part first; the first MMA of the group overwrites D
+                        const uint32_t b_hi = b_base + j * kBMatBytes + kh * 32;
+                        const uint32_t b_lo = b_base + kBLoOffset + (j >> 1) * kBMatBytes + (j & 1) * 64 + kh * 32;
+                        ptx::mma_bf16(d_j, ad, ptx::smem_desc_sw128(b_lo), idesc, kh);
+                        ptx::mma_bf16(d_j, ad, ptx::smem_desc_sw128(b_hi + 64), idesc, 1);
+                        ptx::mma_bf16(d_j, ad, ptx::smem_desc_sw128(b_hi), idesc, 1);
+                    }
+                }
+                ptx::mma_commit(ptx::smem_addr(&bars->empty[s]));
+                ptx::mma_commit(ptx::smem_addr(&bars->acc_full[a]));
+                if (sub == len - 1) ptx::mma_commit(ptx::smem_addr(&bars->b_empty[slot]));
+            }
+            drain_mmas(bars, status);
+        }
+    } else if (warp >= kBuildWarp0) {
+        // Builders: R^ in fp32, transposed to [n][k]; then per tile 1/Lambda of its 128
+        // channels (a reciprocal plus its FMA residual, so R*(1/Lambda) is good to about
+        // an ulp), then the four B_g = diag(1/Lambda_g) R^ split three ways into bf16.
+        const int bt = threadIdx.x - kBuildWarp0 * 32;   // 0..127
+        constexpr int kB = kColBuildWarps * 32;
+        for (int i = bt; i < 32 * 32; i += kB) {
+            const int k = i >> 5, n = i & 31;
+            rt[n * 32 + k] = __bfloat162float(__ushort_as_bfloat16(args.rhat[i]));
+        }
+        ptx::named_bar_sync(3, kB);
+        int built0 = -1, built1 = -1;   // column tile whose B_g each slot holds
+        for (int ui = 0; ui < sched.n_units_cta; ++ui) {
+            const int slot = ui & 1;
+            // one thread waits (bounded) for the slot; the verdict goes to all builders
+            // (the flag alternates per unit, so a slow reader never sees the next unit's value)
+            if (bt == 0) bars->bl_ok[ui & 1] = wait_bar(&bars->b_empty[slot], ((ui >> 1) & 1) ^ 1, abort, status);
+            __syncwarp();
+            ptx::named_bar_sync(3, kB);
+            if (!*reinterpret_cast<volatile int *>(&bars->bl_ok[ui & 1])) break;
+            const int ct = sched.ct_of_unit(ui);
+            if ((slot ? built1 : built0) != ct) {
+                if (slot)
+                    built1 = ct;
+                else
+                    built0 = ct;
+                const int64_t ch_tile = static_cast<int64_t>(ct) * kTileCols;
+                float2 *inv = inv_tab + slot * kTileCols;
+                {
+                    const int64_t ch = ch_tile + bt;
+                    float ih = 0.0f, il = 0.0f;
+                    if (ch < cols) {
+                        const float lam = args.lambda[ch];
+                        ih = __frcp_rn(lam);
+                        il = __fmul_rn(__fmaf_rn(-lam, ih, 1.0f), ih);   // 1/lam - ih, to working precision
+                    }
+                    inv[bt] = make_float2(ih, il);
+                }
+                ptx::named_bar_sync(3, kB);
+                uint8_t *bs = bmat + slot * kBSlotBytes;
+                // 4 groups x 32 rows (n) x 4 chunks of 8 k = 512 chunk tasks.
+                for (int task = bt; task < kColTileG * 32 * 4; task += kB) {
+                    const int j = task >> 7, n = (task >> 2) & 31, c = task & 3;
+                    uint32_t hw[4], mw[4], lw[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        __nv_bfloat16 h[2], m[2], l[2];
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            const int k = c * 8 + 2 * e + u;
+                            const float2 iv = inv[j * 32 + k];
+                            const float r = rt[n * 32 + k];
+                            const float val = __fmaf_rn(r, iv.x, __fmul_rn(r, iv.y));   // R / Lambda
+                            // val = hi + mid + lo to ~24 bits; each residual is exact in fp32
+                            h[u] = __float2bfloat16_rn(val);
+                            const float r1 = val - __bfloat162float(h[u]);
+                            m[u] = __float2bfloat16_rn(r1);
+                            l[u] = __float2bfloat16_rn(r1 - __bfloat162float(m[u]));
+                        }
+                        hw[e] = pack_bf16x2(h[0], h[1]);
+                        mw[e] = pack_bf16x2(m[0], m[1]);
+                        lw[e] = pack_bf16x2(l[0], l[1]);
+                    }
+                    uint8_t *bm = bs + j * kBMatBytes;
+                    uint8_t *bl = bs + kBLoOffset + (j >> 1) * kBMatBytes;
+                    *reinterpret_cast<uint4 *>(bm + sw128(n, c)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                    *reinterpret_cast<uint4 *>(bm + sw128(n, c + 4)) = make_uint4(mw[0], mw[1], mw[2], mw[3]);
+                    *reinterpret_cast<uint4 *>(bl + sw128(n, c + 4 * (j & 1))) =
+                        make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                }
+                ptx::fence_proxy_async_smem();
+            }
+            ptx::mbar_arrive(ptx::smem_addr(&bars->b_full[slot]));
+        }
+    } else {
+        const int q = warp & 3;
+        const int ewg = warp >> 2;
+        const bool scale_vec = (G % 4 == 0) && ((reinterpret_cast<uintptr_t>(args.scales) & 3) == 0);
+        const uint32_t ctile_smem = ptx::smem_addr(code_tiles + ewg * kCodeTileBytes);
+        const bool leader = q == 0 && lane == 0;   // issues this warp group's code stores
+        for (int it = ewg; it < sched.n_tiles; it += 2) {
+            const int a = it % kColAcc;
+            // The leader alone waits (bounded) and hands the verdict to its warp group through a
+            // named barrier, so the four warps leave the loop together or not at all.
+            volatile int *ok_slot = &bars->eg_ok[ewg][(it >> 1) & 1];
+            if (leader) {
+                int ok = wait_bar(&bars->acc_full[a], (it / kColAcc) & 1, abort, status);
+                // the staging tile must have been read by this group's previous store
+                if constexpr (kMode == RotOut::Quant) ptx::bulk_wait_group_read0();
+                *ok_slot = ok;
+            }
+            __syncwarp();
+            ptx::named_bar_sync(1 + ewg, 128);
+            if (!*ok_slot) break;
+            ptx::tc_fence_after();
+            int ui, sub, len;
+            sched.at(it, ui, sub, len);
+            const int ctile = sched.ct_of_unit(ui), rtile = sched.rt0_of_unit(ui) + sub;
+            const int r_local = q * 32 + lane;
+            const int64_t row = static_cast<int64_t>(rtile) * kTileM + r_local;
+            const bool row_ok = row < rows;
+            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * kColAccCols;
+            uint32_t sc_word = 0;
+            uint32_t ra[32], rb[32];
+            ptx::tmem_ld_32cols(t_row, ra);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < kColTileG; ++j) {
+                uint32_t(&cur)[32] = (j & 1) ? rb : ra;
+                uint32_t(&nxt)[32] = (j & 1) ? ra : rb;
+                if (j + 1 < kColTileG) ptx::tmem_ld_32cols(t_row + (j + 1) * 32, nxt);
+                const int64_t g = static_cast<int64_t>(ctile) * kColTileG + j;
+                if constexpr (kMode == RotOut::F32) {
+                    if (g < G && row_ok) {
+                        float *dst = args.y + row * cols + g * 32;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            ptx::st_global_v4(dst + 4 * i, cur[4 * i], cur[4 * i + 1], cur[4 * i + 2],
+                                              cur[4 * i + 3]);
+                    }
+                } else {
+                    uint32_t w[4];
+                    const uint32_t byte = quantize_group(cur, w);
+                    // 64-byte swizzle: 16-byte chunk j of row r sits at chunk j ^ ((r >> 1) & 3)
+                    const uint32_t chunk = static_cast<uint32_t>(j) ^ ((static_cast<uint32_t>(r_local) >> 1) & 3u);
+                    ptx::st_shared_v4(ctile_smem + r_local * 64 + chunk * 16, w[0], w[1], w[2], w[3]);
+                    if (scale_vec)
+                        sc_word |= byte << (8 * j);
+                    else if (g < G && row_ok)
+                        args.scales[row * G + g] = static_cast<uint8_t>(byte);
+                }
+                if (j + 1 < kColTileG) ptx::tmem_wait_ld();
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(ptx::smem_addr(&bars->acc_empty[a]));
+            if constexpr (kMode == RotOut::Quant) {
+                if (scale_vec && row_ok)
+                    *reinterpret_cast<uint32_t *>(args.scales + row * G + static_cast<int64_t>(ctile) * kColTileG) =
+                        sc_word;
+                // staging tile complete -> one bulk store (rows/columns past the tensor are clipped)
+                ptx::fence_proxy_async_smem();
+                __syncwarp();
+                ptx::named_bar_sync(1 + ewg, 128);
+                if (leader) {
+                    ptx::tma_store_2d(&tmap_codes, ctile * (kTileCols / 2), rtile * kTileM, ctile_smem);
+                    ptx::bulk_commit_group();
+                }
+            }
+        }
+        if constexpr (kMode == RotOut::Quant) {
+            if (leader) ptx::bulk_wait_group0();   // stores done before the CTA's shared memory goes
+        }
+    }
+    kernel_teardown(tmem_base, kMmaWarp);
+}
+
+static_assert(kColSmemBytes <= 232448, "shared memory budget");
+
+}  // namespace
+
+cudaError_t launch_rotate_cols(const CUtensorMap &tmap_x, const CUtensorMap &tmap_codes, const RotArgs &args,
+                               RotOut mode, int num_sms, cudaStream_t stream)
+{
+    const int64_t n_tiles = ((args.rows + kTileM - 1) / kTileM) * ((args.cols + kTileCols - 1) / kTileCols);
+    if (n_tiles <= 0) return cudaSuccess;
+    const int grid = static_cast<int>(n_tiles < num_sms ? n_tiles : num_sms);
+    unsigned int *status = status_word();
+    if (!status) return cudaErrorInvalidSymbol;
+    return mode == RotOut::Quant
+               ? launch_pdl(rotate_cols_kernel<RotOut::Quant>, grid, kColThreads, kColSmemBytes, stream, tmap_x,
+                            tmap_codes, args, status)
+               : launch_pdl(rotate_cols_kernel<RotOut::F32>, grid, kColThreads, kColSmemBytes, stream, tmap_x,
+                            tmap_codes, args, status);
+}
+
+}  // namespace mxq
