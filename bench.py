@@ -49,7 +49,7 @@ FALLBACK_HBM_GBS = 6650.0
 KERNEL_SOURCES = ["mxfp4_block_rotation_b200/csrc/rotate_flat_sm100.cu",
                   "mxfp4_block_rotation_b200/csrc/pipeline_sm100.cuh",
                   "mxfp4_block_rotation_b200/csrc/sm100_ptx.cuh"]
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "rotate_kernel_downproj_traffic.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "rotate_flat_kernel_downproj_traffic.json")
 
 
 def algorithmic_bytes(rows: int, cols: int) -> float:
@@ -83,6 +83,19 @@ def recorded_traffic():
     if rec.get("kernel_source_sha256") != kernel_source_hash():
         return None
     return rec.get("dram_bytes_per_launch")
+
+
+def max_over_ranks(values, dist=None, device=None):
+    """Element-wise max of a list of floats over all ranks (identity without a process group)."""
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
+def weak_scaling_value(world: int, bytes_per_rank: float, ms_per_step: float) -> float:
+    """Whole-job GB/s: every rank moves bytes_per_rank per step; the step time is the slowest rank's."""
+    return world * bytes_per_rank / (ms_per_step * 1e-3) / 1e9
 
 
 def host_cores() -> int:
@@ -183,7 +196,7 @@ def run_reference(args):
     xb = synth.bf16_bits(w.x)
     rb = synth.bf16_bits(w.rhat)
     threads = host_cores()
-    per_step_s = max(1.0, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+    per_step_s = max(0.05, min(args.cpu_seconds, 150.0 / max(1, args.steps + args.warmup)))
     probe = min(ROWS, max(8, threads * 2))
     t0 = time.perf_counter()
     oracle.smooth_rotate_quantize(xb[:probe], rb, None, threads=threads)
@@ -265,14 +278,10 @@ def run_mine(args):
         if dist is not None:
             dist.barrier()
     mxq.sync_check()
-    total_ms = t_begin.elapsed_time(t_end)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if dist is not None:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t[0])
+    total_ms = max_over_ranks([t_begin.elapsed_time(t_end)], dist, dev)[0]
     kern_avg_ms = total_ms / k
     ms_per_step = total_ms / k
-    value = world * n_bytes / (ms_per_step * 1e-3) / 1e9
+    value = weak_scaling_value(world, n_bytes, ms_per_step)
 
     # end to end through the public API: pinned host X -> device -> kernel -> codes/scales back to host
     e2e = None if args.no_e2e else run_e2e(mxq, w, rhat, dev, stream, args, dist)
@@ -396,14 +405,9 @@ def run_e2e(mxq, w, rhat, dev, stream, args, dist):
         step()
     b.record(stream)
     torch.cuda.synchronize(dev)
-    ms = a.elapsed_time(b) / k
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    world = 1
-    if dist is not None:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        world = dist.get_world_size()
-    ms = float(t[0])
-    return {"value": world * algorithmic_bytes(rows, cols) / (ms * 1e-3) / 1e9, "unit": UNIT,
+    ms = max_over_ranks([a.elapsed_time(b) / k], dist, dev)[0]
+    world = dist.get_world_size() if dist is not None else 1
+    return {"value": weak_scaling_value(world, algorithmic_bytes(rows, cols), ms), "unit": UNIT,
             "h2d_bytes_per_step": x_host.numel() * 2,
             "d2h_bytes_per_step": c_host.numel() + s_host.numel(), "ms_per_step": ms, "steps": k}
 
@@ -414,8 +418,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=10000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["mine", "reference"], default="mine")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0,
-                    help="oracle time for the cpu_baseline sample (rank 0, N=1 only)")
+    ap.add_argument("--cpu-seconds", type=float, default=8.0,
+                    help="oracle seconds: the cpu_baseline sample (rank 0, N=1) and each --impl reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg (profiling runs)")
     ap.add_argument("--no-extras", action="store_true", help="skip timing the smoothing and dequantize rows")
