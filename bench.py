@@ -372,6 +372,18 @@ def run_extras(mxq, w, xs, rhat, outs, dev, stream, k=300):
         mxq.dequantize(c, s, rhat, lam, out=deq[i & 1], stream=stream)
     row("dequantize_inverse_rotation_and_smoothing", _timed(dq_inv, k, stream, dev), deq_bytes + 4 * cols,
         "codes + scales -> (v * R^T) * Lambda -> bf16")
+    ws = torch.empty(mxq.lib().mxq_quant_error_workspace_bytes(rows, cols, 0), dtype=torch.uint8, device=dev)
+    errs = torch.empty((rows, cols // 32), dtype=torch.float32, device=dev)
+    mean = torch.empty((), dtype=torch.float64, device=dev)
+
+    def qerr(i):
+        import ctypes
+        st = mxq.lib().mxq_quant_error(ctypes.c_void_p(xs[i & 1].data_ptr()), rows, cols, ctypes.c_void_p(rhat.data_ptr()),
+                                       None, ctypes.c_void_p(errs.data_ptr()), ctypes.c_void_p(mean.data_ptr()),
+                                       ctypes.c_void_p(ws.data_ptr()), ws.numel(), ctypes.c_void_p(stream.cuda_stream))
+        assert st == 0
+    row("quant_error_per_group_and_mean", _timed(qerr, k, stream, dev), rows * cols * 2.0 + rows * (cols // 32) * 4.0,
+        "per-group ||Q(y)-y||/||y|| (fp32 out) and its mean: reads X, writes 4 B per group")
     mxq.sync_check()
     return res
 

@@ -58,6 +58,7 @@
 #ifndef MXQ_H
 #define MXQ_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -125,6 +126,30 @@ mxq_status mxq_smooth_rotate_f32(const void *X_bf16, int64_t rows, int64_t cols,
 mxq_status mxq_dequantize(const uint8_t *codes, const uint8_t *scales, int64_t rows,
                           int64_t cols, const void *Rhat_bf16_or_null,
                           const float *Lambda_or_null, void *out_bf16, void *stream);
+
+/*
+ * The per-group MXFP4 quantisation error: the write-up's §4.1, Figure 1, which
+ * compares the original activations, a random Hadamard block rotation and the
+ * outlier-aware rotation by this error inside each group.  Each group's 32
+ * values y = X * Lambda^-1 * R^ (fp32, as the quantiser sees them) are quantised
+ * exactly as mxq_smooth_rotate_quantize does, then dequantised to Q(y).  The
+ * error is
+ *     e_g = ||Q(y) - y||_2 / ||y||_2      (0 for an all-zero group, NaN for a NaN/Inf one)
+ * and the call also returns the mean of e_g over all rows * cols/32 groups.  The
+ * mean is summed in a fixed order, so it is the same on every run.
+ *
+ *   X_bf16, rows, cols, Rhat_bf16, Lambda_or_null   as for mxq_smooth_rotate_quantize
+ *                                                    (rows, cols > 0)
+ *   out_group_err_or_null   out  fp32 [rows, cols/32], 4-byte aligned, or NULL
+ *   out_mean                out  one double (device), 8-byte aligned
+ *   workspace               in/out  device scratch for per-warp partial sums, 8-byte
+ *                                aligned, at least mxq_quant_error_workspace_bytes()
+ *                                bytes; caller-owned, overwritten, no state kept
+ */
+size_t mxq_quant_error_workspace_bytes(int64_t rows, int64_t cols, int with_lambda);
+mxq_status mxq_quant_error(const void *X_bf16, int64_t rows, int64_t cols, const void *Rhat_bf16,
+                           const float *Lambda_or_null, float *out_group_err_or_null, double *out_mean,
+                           void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * Synchronise `stream` and then read and clear the device status word.

@@ -23,7 +23,7 @@ import torch
 
 __all__ = [
     "MxqError", "smooth_rotate_quantize", "smooth_rotate_f32", "dequantize", "sync_check",
-    "selftest_bounded_wait",
+    "selftest_bounded_wait", "quant_error",
     "status_string", "version", "lib", "LIB_PATH", "HEADER_PATH", "declared_symbols",
 ]
 
@@ -64,6 +64,10 @@ def lib() -> ctypes.CDLL:
         L.mxq_dequantize.restype = I
         L.mxq_selftest_bounded_wait.argtypes = [ctypes.c_uint32, P, P]
         L.mxq_selftest_bounded_wait.restype = I
+        L.mxq_quant_error_workspace_bytes.argtypes = [I64, I64, I]
+        L.mxq_quant_error_workspace_bytes.restype = ctypes.c_size_t
+        L.mxq_quant_error.argtypes = [P, I64, I64, P, P, P, P, P, ctypes.c_size_t, P]
+        L.mxq_quant_error.restype = I
         L.mxq_sync_check.argtypes = [P]
         L.mxq_sync_check.restype = I
         L.mxq_status_string.argtypes = [I]
@@ -191,6 +195,24 @@ def dequantize(codes: torch.Tensor, scales: torch.Tensor, rhat: Optional[torch.T
                               _stream(dev, stream))
     _check(st, "mxq_dequantize")
     return out
+
+
+def quant_error(x: torch.Tensor, rhat: torch.Tensor, lam: Optional[torch.Tensor] = None, *,
+                per_group: bool = True, workspace: Optional[torch.Tensor] = None, stream=None):
+    """Per-group MXFP4 error ||Q(y) - y|| / ||y|| (fp32 [rows, cols/32], or None) and its mean (a 0-d
+    float64 device tensor).  `workspace` (uint8, device) is allocated here when not given."""
+    dev = _inputs(x, rhat, lam)
+    rows, cols = x.shape
+    need = int(lib().mxq_quant_error_workspace_bytes(rows, cols, int(lam is not None)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 8), dtype=torch.uint8, device=dev)
+    _need(workspace, "workspace", torch.uint8, dev)
+    err = torch.empty((rows, cols // 32), dtype=torch.float32, device=dev) if per_group else None
+    mean = torch.empty((), dtype=torch.float64, device=dev)
+    st = lib().mxq_quant_error(_ptr(x), rows, cols, _ptr(rhat), _ptr(lam), _ptr(err), _ptr(mean),
+                               _ptr(workspace), workspace.numel(), _stream(dev, stream))
+    _check(st, "mxq_quant_error")
+    return err, mean
 
 
 def selftest_bounded_wait(timeout_ms: int = 50, device=None, stream=None) -> int:

@@ -330,6 +330,77 @@ mxq_status mxq_dequantize(const uint8_t *codes, const uint8_t *scales, int64_t r
     return MXQ_OK;
 }
 
+size_t mxq_quant_error_workspace_bytes(int64_t rows, int64_t cols, int with_lambda)
+{
+    if (check_shape(rows, cols) != MXQ_OK || rows == 0 || cols == 0) return 0;
+    const int64_t n = with_lambda ? mxq::rotate_cols_partials(rows, cols) : mxq::rotate_flat_partials(rows, cols);
+    return static_cast<size_t>(n) * sizeof(double);
+}
+
+mxq_status mxq_quant_error(const void *X_bf16, int64_t rows, int64_t cols, const void *Rhat_bf16,
+                           const float *Lambda_or_null, float *out_group_err_or_null, double *out_mean,
+                           void *workspace, size_t workspace_bytes, void *stream)
+{
+    mxq_status st = check_shape(rows, cols);
+    if (st != MXQ_OK) return st;
+    if (!out_mean || !aligned(out_mean, 8)) return bad("out_mean must be an 8-byte aligned device double");
+    if (rows == 0 || cols == 0) return bad("the mean of an empty matrix is undefined");
+    if (!X_bf16 || !Rhat_bf16) return bad("null pointer");
+    if (!aligned(X_bf16, 16)) return bad("X must be 16-byte aligned");
+    if (!aligned(Rhat_bf16, 2)) return bad("Rhat must be 2-byte aligned");
+    if (Lambda_or_null && !aligned(Lambda_or_null, 4)) return bad("Lambda must be 4-byte aligned");
+    if (out_group_err_or_null && !aligned(out_group_err_or_null, 4)) return bad("per-group errors must be 4-byte aligned");
+    const size_t need = mxq_quant_error_workspace_bytes(rows, cols, Lambda_or_null != nullptr);
+    if (!workspace || !aligned(workspace, 8) || workspace_bytes < need)
+        return bad("workspace missing, not 8-byte aligned or smaller than mxq_quant_error_workspace_bytes()");
+    const uint64_t nx = static_cast<uint64_t>(rows) * cols * 2, nl = Lambda_or_null ? static_cast<uint64_t>(cols) * 4 : 0;
+    const uint64_t ne = out_group_err_or_null ? static_cast<uint64_t>(rows) * (cols / 32) * 4 : 0;
+    const void *ins[3] = {X_bf16, Rhat_bf16, Lambda_or_null};
+    const uint64_t nins[3] = {nx, 32 * 32 * 2, nl};
+    void *outs[3] = {out_group_err_or_null, out_mean, workspace};
+    const uint64_t nouts[3] = {ne, 8, need};
+    for (int o = 0; o < 3; ++o) {
+        for (int i = 0; i < 3; ++i)
+            if (overlaps(outs[o], nouts[o], ins[i], nins[i])) return bad("an output overlaps an input");
+        for (int o2 = o + 1; o2 < 3; ++o2)
+            if (overlaps(outs[o], nouts[o], outs[o2], nouts[o2])) return bad("outputs overlap");
+    }
+    int dev = 0, sms = 0;
+    if ((st = current_device(&dev, &sms)) != MXQ_OK) return st;
+    if ((st = check_buffer(X_bf16, nx, dev)) != MXQ_OK) return st;
+    if ((st = check_buffer(Rhat_bf16, 32 * 32 * 2, dev)) != MXQ_OK) return st;
+    if (Lambda_or_null && (st = check_buffer(Lambda_or_null, nl, dev)) != MXQ_OK) return st;
+    if (out_group_err_or_null && (st = check_buffer(out_group_err_or_null, ne, dev)) != MXQ_OK) return st;
+    if ((st = check_buffer(out_mean, 8, dev)) != MXQ_OK) return st;
+    if ((st = check_buffer(workspace, need, dev)) != MXQ_OK) return st;
+
+    mxq::RotArgs args{};
+    args.rhat = static_cast<const uint16_t *>(Rhat_bf16);
+    args.lambda = Lambda_or_null;
+    args.rows = rows;
+    args.cols = cols;
+    args.err = out_group_err_or_null;
+    args.partials = static_cast<double *>(workspace);
+    alignas(64) CUtensorMap map_a;
+    cudaError_t e;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (Lambda_or_null == nullptr) {
+        if ((st = make_tmap_groups(&map_a, X_bf16, rows, cols)) != MXQ_OK) return st;
+        e = mxq::launch_rotate_flat(map_a, args, mxq::RotOut::Err, sms, s);
+    } else {
+        if ((st = make_tmap_x(&map_a, X_bf16, rows, cols)) != MXQ_OK) return st;
+        e = mxq::launch_rotate_cols(map_a, map_a, args, mxq::RotOut::Err, sms, s);
+    }
+    if (e == cudaSuccess)
+        e = mxq::launch_error_mean(args.partials, static_cast<int64_t>(need / sizeof(double)), rows * (cols / 32),
+                                   out_mean, s);
+    if (e != cudaSuccess) {
+        note_cuda(e, "launch quantisation-error kernels");
+        return MXQ_ERR_CUDA;
+    }
+    return MXQ_OK;
+}
+
 mxq_status mxq_sync_check(void *stream)
 {
     unsigned int status = 0;

@@ -13,8 +13,10 @@ enum : unsigned int {
     kStatusTimeout = 1u,   // a bounded pipeline wait ran out
 };
 
-// Output mode of the fused rotate kernel.
-enum class RotOut { Quant, F32 };
+// Output mode of the fused rotate kernels: packed codes + scales, the rotated
+// fp32 values, or the per-group MXFP4 quantisation error (plus per-warp partial
+// sums for its mean).
+enum class RotOut { Quant, F32, Err };
 
 struct RotArgs {
     const uint16_t *rhat;      // bf16 [32][32], row-major [k][n]
@@ -22,6 +24,8 @@ struct RotArgs {
     uint8_t *codes;            // [rows, cols/2]   (Quant)
     uint8_t *scales;           // [rows, cols/32]  (Quant)
     float *y;                  // [rows, cols]     (F32)
+    float *err;                // [rows, cols/32]  (Err; may be null)
+    double *partials;          // per-warp error sums (Err): see rotate_*_partials()
     int64_t rows;
     int64_t cols;
 };
@@ -36,6 +40,14 @@ cudaError_t launch_rotate_flat(const CUtensorMap &tmap_groups, const RotArgs &ar
 // codes as [rows, cols/2] uint8 (box {64, 128}, 64-byte swizzle; Quant mode only).
 cudaError_t launch_rotate_cols(const CUtensorMap &tmap_x, const CUtensorMap &tmap_codes, const RotArgs &args,
                                RotOut mode, int num_sms, cudaStream_t stream);
+
+// Number of per-warp partial sums the Err mode writes (one double each).
+int64_t rotate_flat_partials(int64_t rows, int64_t cols);
+int64_t rotate_cols_partials(int64_t rows, int64_t cols);
+
+// Mean of the per-group errors from the partial sums, in a fixed order: out = sum / n_groups.
+cudaError_t launch_error_mean(const double *partials, int64_t n_partials, int64_t n_groups, double *out,
+                              cudaStream_t stream);
 
 // Dequantise to bf16 in the rotated domain (codes 16-byte aligned, out 16-byte aligned).
 cudaError_t launch_dequant_plain(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t cols,

@@ -109,6 +109,44 @@ __device__ __forceinline__ uint32_t quantize_group(const uint32_t (&r)[32], uint
     return byte;
 }
 
+// E2M1 code (bit 3 = sign) -> its value as fp32.  Magnitudes {0, 0.5, 1, 1.5, 2,
+// 3, 4, 6}: code 1 is E2M1's subnormal 0.5, codes 2..7 are 2^(e-1) * (1 + m/2)
+// with e = code >> 1, m = code & 1.
+__device__ __forceinline__ float e2m1_f32(uint32_t code)
+{
+    const uint32_t m = code & 7u;
+    const uint32_t bits = m == 0u ? 0u : (m == 1u ? 0x3F000000u : (((126u + (m >> 1)) << 23) | ((m & 1u) << 22)));
+    return __uint_as_float(bits | ((code & 8u) << 28));
+}
+
+// Normalised MXFP4 quantisation error of one group: ||Q(y) - y||_2 / ||y||_2, where
+// Q(y) is the group dequantised from its codes `w` and scale `byte`.  An all-zero
+// group has error 0; a NaN/Inf group (byte 0xFF) gives NaN.
+__device__ __forceinline__ float group_error(const uint32_t (&r)[32], uint32_t byte, const uint32_t (&w)[4])
+{
+    const float s = byte == 0xFFu ? __uint_as_float(0x7FC00000u)
+                                  : (byte == 0u ? __uint_as_float(0x00400000u) : __uint_as_float(byte << 23));
+    float num = 0.0f, den = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const float y = __uint_as_float(r[i]);
+        const float v = __fmul_rn(e2m1_f32((w[i >> 3] >> (4 * (i & 7))) & 15u), s);
+        const float d = __fsub_rn(v, y);
+        num = __fmaf_rn(d, d, num);
+        den = __fmaf_rn(y, y, den);
+    }
+    if (byte == 0xFFu) return s;   // NaN
+    return den > 0.0f ? __fsqrt_rn(__fdiv_rn(num, den)) : 0.0f;
+}
+
+// Sum over the warp in a fixed shuffle order (deterministic); the result is in lane 0.
+__device__ __forceinline__ double warp_sum(double v)
+{
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) v += __shfl_down_sync(0xffffffffu, v, off);
+    return v;
+}
+
 // Per-kernel numbers the shared set-up needs.
 struct SetupCfg {
     int n_stages;     // shared-memory stages (full/empty barrier pairs)

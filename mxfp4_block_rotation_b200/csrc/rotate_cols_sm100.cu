@@ -268,6 +268,7 @@ __global__ void __launch_bounds__(kColThreads, 1)
             const bool row_ok = row < rows;
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * kColAccCols;
             uint32_t sc_word = 0;
+            double err_acc = 0.0;   // Err mode: this row's groups of the tile, in order
             uint32_t ra[32], rb[32];
             ptx::tmem_ld_32cols(t_row, ra);
             ptx::tmem_wait_ld();
@@ -285,6 +286,14 @@ __global__ void __launch_bounds__(kColThreads, 1)
                             ptx::st_global_v4(dst + 4 * i, cur[4 * i], cur[4 * i + 1], cur[4 * i + 2],
                                               cur[4 * i + 3]);
                     }
+                } else if constexpr (kMode == RotOut::Err) {
+                    if (g < G && row_ok) {
+                        uint32_t w[4];
+                        const uint32_t byte = quantize_group(cur, w);
+                        const float e = group_error(cur, byte, w);
+                        if (args.err) args.err[row * G + g] = e;
+                        err_acc += static_cast<double>(e);
+                    }
                 } else {
                     uint32_t w[4];
                     const uint32_t byte = quantize_group(cur, w);
@@ -301,6 +310,10 @@ __global__ void __launch_bounds__(kColThreads, 1)
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(ptx::smem_addr(&bars->acc_empty[a]));
+            if constexpr (kMode == RotOut::Err) {
+                const double sum = warp_sum(err_acc);
+                if (lane == 0) args.partials[(static_cast<int64_t>(rtile) * n_ct + ctile) * 4 + q] = sum;
+            }
             if constexpr (kMode == RotOut::Quant) {
                 if (scale_vec && row_ok)
                     *reinterpret_cast<uint32_t *>(args.scales + row * G + static_cast<int64_t>(ctile) * kColTileG) =
@@ -334,11 +347,19 @@ cudaError_t launch_rotate_cols(const CUtensorMap &tmap_x, const CUtensorMap &tma
     const int grid = static_cast<int>(n_tiles < num_sms ? n_tiles : num_sms);
     unsigned int *status = status_word();
     if (!status) return cudaErrorInvalidSymbol;
-    return mode == RotOut::Quant
-               ? launch_pdl(rotate_cols_kernel<RotOut::Quant>, grid, kColThreads, kColSmemBytes, stream, tmap_x,
-                            tmap_codes, args, status)
-               : launch_pdl(rotate_cols_kernel<RotOut::F32>, grid, kColThreads, kColSmemBytes, stream, tmap_x,
-                            tmap_codes, args, status);
+    if (mode == RotOut::Quant)
+        return launch_pdl(rotate_cols_kernel<RotOut::Quant>, grid, kColThreads, kColSmemBytes, stream, tmap_x,
+                          tmap_codes, args, status);
+    if (mode == RotOut::Err)
+        return launch_pdl(rotate_cols_kernel<RotOut::Err>, grid, kColThreads, kColSmemBytes, stream, tmap_x,
+                          tmap_codes, args, status);
+    return launch_pdl(rotate_cols_kernel<RotOut::F32>, grid, kColThreads, kColSmemBytes, stream, tmap_x, tmap_codes,
+                      args, status);
+}
+
+int64_t rotate_cols_partials(int64_t rows, int64_t cols)
+{
+    return ((rows + kTileM - 1) / kTileM) * ((cols + kTileCols - 1) / kTileCols) * 4;
 }
 
 }  // namespace mxq

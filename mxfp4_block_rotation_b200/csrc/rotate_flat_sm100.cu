@@ -128,6 +128,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tc_fence_after();
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * kFlatAccCols;
             const int64_t g_lane = static_cast<int64_t>(c) * kFlatStageGroups + q * 32 + lane;
+            double err_acc = 0.0;   // Err mode: this lane's groups, in order
             // The TMEM load of MMA j+1 is in flight while group j is quantised; fully
             // unrolled so both register buffers stay put.
             uint32_t ra[32], rb[32];
@@ -146,6 +147,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int i = 0; i < 8; ++i)
                             ptx::st_global_v4(dst + 4 * i, cur[4 * i], cur[4 * i + 1], cur[4 * i + 2],
                                               cur[4 * i + 3]);
+                    } else if constexpr (kMode == RotOut::Err) {
+                        uint32_t w[4];
+                        const uint32_t byte = quantize_group(cur, w);
+                        const float e = group_error(cur, byte, w);
+                        if (args.err) args.err[g] = e;
+                        err_acc += static_cast<double>(e);
                     } else {
                         uint32_t w[4];
                         const uint32_t byte = quantize_group(cur, w);
@@ -158,6 +165,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(ptx::smem_addr(&bars->acc_empty[a]));
+            if constexpr (kMode == RotOut::Err) {
+                const double sum = warp_sum(err_acc);
+                if (lane == 0) args.partials[static_cast<int64_t>(c) * 4 + q] = sum;   // one slot per warp and stage
+            }
         }
     }
     kernel_teardown(tmem_base, kMmaWarp);
@@ -176,11 +187,19 @@ cudaError_t launch_rotate_flat(const CUtensorMap &tmap_groups, const RotArgs &ar
     const int grid = static_cast<int>(n_chunks < num_sms ? n_chunks : num_sms);
     unsigned int *status = status_word();
     if (!status) return cudaErrorInvalidSymbol;
-    return mode == RotOut::Quant
-               ? launch_pdl(rotate_flat_kernel<RotOut::Quant>, grid, kThreads, kFlatSmemBytes, stream, tmap_groups, args,
-                            status)
-               : launch_pdl(rotate_flat_kernel<RotOut::F32>, grid, kThreads, kFlatSmemBytes, stream, tmap_groups, args,
-                            status);
+    if (mode == RotOut::Quant)
+        return launch_pdl(rotate_flat_kernel<RotOut::Quant>, grid, kThreads, kFlatSmemBytes, stream, tmap_groups,
+                          args, status);
+    if (mode == RotOut::Err)
+        return launch_pdl(rotate_flat_kernel<RotOut::Err>, grid, kThreads, kFlatSmemBytes, stream, tmap_groups, args,
+                          status);
+    return launch_pdl(rotate_flat_kernel<RotOut::F32>, grid, kThreads, kFlatSmemBytes, stream, tmap_groups, args,
+                      status);
+}
+
+int64_t rotate_flat_partials(int64_t rows, int64_t cols)
+{
+    return ((rows * (cols / 32) + kFlatStageGroups - 1) / kFlatStageGroups) * 4;
 }
 
 }  // namespace mxq

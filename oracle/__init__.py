@@ -64,6 +64,8 @@ def lib():
         L.mxq_oracle_smooth_rotate_quantize.restype = I
         L.mxq_oracle_dequantize.argtypes = [P, P, I64, I64, P, P, P, P, I]
         L.mxq_oracle_dequantize.restype = I
+        L.mxq_oracle_group_error.argtypes = [P, I64, I64, P, P, P, P, I]
+        L.mxq_oracle_group_error.restype = I
         L.mxq_oracle_bf16_to_double.argtypes = [P, P, I64]
         L.mxq_oracle_bf16_to_double.restype = None
         L.mxq_oracle_double_to_bf16.argtypes = [P, P, I64]
@@ -203,6 +205,22 @@ def dequantize(codes: np.ndarray, scales: np.ndarray, cols: int, rhat_bits: Opti
     if rc:
         raise ValueError("oracle dequantize: bad shape")
     return (out, f64) if want_f64 else out
+
+
+def group_error(x_bits: np.ndarray, rhat_bits: np.ndarray, lam: Optional[np.ndarray] = None,
+                threads: int = 1):
+    """Per-group MXFP4 error ||Q(y) - y|| / ||y|| [rows, cols/32] (float64) and its mean."""
+    x_bits = _c(x_bits, np.uint16)
+    rhat_bits = _c(rhat_bits, np.uint16)
+    rows, cols = x_bits.shape
+    lam32 = None if lam is None else _c(lam, np.float32)
+    err = np.zeros((rows, cols // GROUP), np.float64)
+    mean = np.zeros(1, np.float64)
+    rc = lib().mxq_oracle_group_error(_ptr(x_bits), rows, cols, _ptr(rhat_bits), _ptr(lam32), _ptr(err),
+                                      _ptr(mean), threads)
+    if rc:
+        raise ValueError("oracle group_error: bad shape")
+    return err, float(mean[0])
 
 
 def unpack_codes(codes: np.ndarray) -> np.ndarray:

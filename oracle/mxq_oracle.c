@@ -346,6 +346,57 @@ int mxq_oracle_dequantize(const uint8_t *codes, const uint8_t *scales, int64_t r
     return 0;
 }
 
+/* The per-group MXFP4 quantisation error of the write-up's §4.1 (Figure 1):
+ * e_g = ||Q(y) - y||_2 / ||y||_2, where y is the group's rotated values
+ * rounded to fp32 (the values the quantiser decides on) and Q(y) the group
+ * dequantised from its own codes and scale.  An all-zero group has error 0 and a
+ * NaN/Inf group NaN.  err [rows, cols/32] may be NULL; *mean gets the plain
+ * average over all groups, summed in row-major order. */
+int mxq_oracle_group_error(const uint16_t *X, int64_t rows, int64_t cols, const uint16_t *Rb,
+                           const float *lam, double *err, double *mean, int nthreads)
+{
+    if (rows <= 0 || cols <= 0 || cols % GROUP) return 1;
+    int64_t G = cols / GROUP;
+    double R[GROUP * GROUP];
+    for (int i = 0; i < GROUP * GROUP; ++i) R[i] = bf16_to_double(Rb[i]);
+    double *e_all = err ? err : (double *)malloc(sizeof(double) * (size_t)(rows * G));
+    if (!e_all) return 2;
+#pragma omp parallel for schedule(static) num_threads(nthreads > 0 ? nthreads : 1)
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t g = 0; g < G; ++g) {
+            double x[GROUP], y[GROUP];
+            uint8_t c[GROUP], byte;
+            int64_t e0 = r * cols + g * GROUP;
+            for (int k = 0; k < GROUP; ++k) {
+                x[k] = bf16_to_double(X[e0 + k]);
+                if (lam) x[k] = x[k] / (double)lam[g * GROUP + k];
+            }
+            for (int n = 0; n < GROUP; ++n) {
+                double acc = 0.0;
+                for (int k = 0; k < GROUP; ++k) acc += x[k] * R[k * GROUP + n];
+                y[n] = (double)(float)acc;          /* fp32, as in quantize_group */
+            }
+            quantize_group(y, c, &byte, NULL, NULL, NULL, NULL);
+            double num = 0.0, den = 0.0;
+            double s = mxq_oracle_e8m0_value(byte);
+            for (int n = 0; n < GROUP; ++n) {
+                double v = mxq_oracle_e2m1_value(c[n]) * s;
+                num += (v - y[n]) * (v - y[n]);
+                den += y[n] * y[n];
+            }
+            double e;
+            if (byte == 0xFF) e = NAN;
+            else e = den > 0.0 ? sqrt(num / den) : 0.0;
+            e_all[r * G + g] = e;
+        }
+    }
+    double total = 0.0;
+    for (int64_t i = 0; i < rows * G; ++i) total += e_all[i];
+    *mean = total / (double)(rows * G);
+    if (!err) free(e_all);
+    return 0;
+}
+
 /* Exposed for the pins: exact bf16 <-> double conversions. */
 void mxq_oracle_bf16_to_double(const uint16_t *b, double *d, int64_t n)
 {

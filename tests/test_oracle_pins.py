@@ -345,3 +345,52 @@ def test_dequant_with_rotation_inverts():
     ref = (deq.reshape(4, 4, 32) @ rr.T).reshape(4, 128) * lam[None, :]
     assert np.abs(back64 - ref).max() <= 1e-12 * np.abs(ref).max()
     assert np.array_equal(oracle.f64_to_bf16_bits(back64), back)
+
+
+# ---------------------------------------------------------------- the per-group error metric (§4.1, Figure 1)
+
+def test_group_error_worked_example_closed_form():
+    # §2.1's group: Q keeps only the 1024 outlier (code 0x6 at scale 2^8), so the error is
+    # ||x without the outlier|| / ||x|| exactly.
+    g = _read_golden("worked_example.txt")
+    x = synth.to_bf16(np.array([float(v) for v in g["input"]]).reshape(1, 32))
+    xv = x.to(torch.float64).numpy()[0]
+    err, mean = oracle.group_error(synth.bf16_bits(x), _eye_bits())
+    expect = math.sqrt((xv ** 2).sum() - 1024.0 ** 2) / math.sqrt((xv ** 2).sum())
+    assert abs(err[0, 0] - expect) < 1e-15 and mean == err[0, 0]
+
+
+def test_group_error_zero_on_grid_and_zero_groups():
+    y = np.zeros((2, 64))
+    y[0, :32] = [(-1) ** i * [0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0][i % 7] * 2.0 ** 5 for i in range(32)]
+    x = synth.to_bf16(y)
+    err, mean = oracle.group_error(synth.bf16_bits(x), _eye_bits())
+    assert (err == 0.0).all() and mean == 0.0
+
+
+def test_group_error_matches_bruteforce():
+    r = synth.haar_orthogonal(21)
+    rb = synth.bf16_bits(synth.rhat_tensor(r))
+    x = synth.make_config(3, rows=6, cols=128).x
+    err, mean = oracle.group_error(synth.bf16_bits(x), rb)
+    y = oracle.rotate_f64(oracle.bf16_bits_to_f64(synth.bf16_bits(x)), oracle.bf16_bits_to_f64(rb))
+    ref = np.zeros_like(err)
+    for i in range(6):
+        for g in range(4):
+            yy = _f32(y[i, 32 * g:32 * g + 32])
+            byte, codes = bf.quantize_group(yy)
+            v = np.array([bf.e2m1_decode(c) for c in codes]) * 2.0 ** (byte - 127)
+            ref[i, g] = np.linalg.norm(v - yy) / np.linalg.norm(yy)
+    assert np.abs(err - ref).max() < 1e-12
+    assert abs(mean - ref.mean()) < 1e-12
+
+
+def test_hadamard_lowers_error_on_outlier_activations():
+    # §4.1's Figure 1: a random Hadamard block rotation lowers the per-group MXFP4 error
+    # of outlier-heavy activations relative to the original ones.
+    w = synth.make_config(1, rows=64, cols=4096)
+    xb = synth.bf16_bits(w.x)
+    _, e_orig = oracle.group_error(xb, _eye_bits(), threads=oracle.default_threads())
+    _, e_had = oracle.group_error(xb, synth.bf16_bits(synth.rhat_tensor(synth.hadamard_rhat(5))),
+                                  threads=oracle.default_threads())
+    assert e_had < e_orig

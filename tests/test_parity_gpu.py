@@ -313,3 +313,37 @@ def test_full_config5_with_round_trip():
     rel = np.linalg.norm((got - x).reshape(len(rows_s), -1, 32), axis=2) / \
         np.maximum(np.linalg.norm(x.reshape(len(rows_s), -1, 32), axis=2), 1e-30)
     assert np.median(rel) < 0.2
+
+
+# ---------------------------------------------------------------- the per-group error metric
+
+@pytest.mark.parametrize("rows,cols,with_lam", [(300, 4096, False), (129, 1056, False), (257, 2048, True),
+                                                (3, 96, True), (1, 32, False)])
+def test_quant_error_matches_oracle(rows, cols, with_lam):
+    w = synth.make_config(3, rows=rows, cols=cols)
+    r = synth.rhat_tensor(synth.haar_orthogonal(rows + 1))
+    lam = synth.random_lambda(cols, seed=3) if with_lam else None
+    err, mean = mxq.quant_error(w.x.to(DEV), r.to(DEV), None if lam is None else lam.to(DEV))
+    mxq.sync_check()
+    err = err.cpu().numpy().astype(np.float64)
+    ref_err, ref_mean = oracle.group_error(_bits(w.x), _bits(r), None if lam is None else lam.numpy(),
+                                           threads=oracle.default_threads())
+    flags = oracle.smooth_rotate_quantize(_bits(w.x), _bits(r), None if lam is None else lam.numpy(), flags=True,
+                                          threads=oracle.default_threads())
+    boundary = flags["gflags"].astype(bool) | flags["eflags"].reshape(rows, cols // 32, 32).any(axis=2)
+    ok = np.abs(err - ref_err) <= 1e-5 + 1e-4 * ref_err
+    assert (ok | boundary).all()
+    assert (~ok).sum() <= max(1, 1e-5 * rows * cols)
+    assert abs(float(mean.item()) - ref_mean) <= 1e-4 * ref_mean + 1e-7
+
+
+def test_quant_error_deterministic_and_workspace_checked():
+    w = synth.make_config(2, rows=512, cols=4096)
+    x, r = w.x.to(DEV), w.rhat.to(DEV)
+    _, m1 = mxq.quant_error(x, r, per_group=False)
+    _, m2 = mxq.quant_error(x, r, per_group=False)
+    assert m1.item() == m2.item()
+    small = torch.empty(8, dtype=torch.uint8, device=DEV)
+    with pytest.raises(mxq.MxqError) as ei:
+        mxq.quant_error(x, r, workspace=small)
+    assert ei.value.status == 1
