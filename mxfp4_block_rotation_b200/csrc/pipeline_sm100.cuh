@@ -5,6 +5,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "mxq_internal.h"
 #include "sm100_ptx.cuh"
@@ -109,34 +110,52 @@ __device__ __forceinline__ uint32_t quantize_group(const uint32_t (&r)[32], uint
     return byte;
 }
 
-// E2M1 code (bit 3 = sign) -> its value as fp32.  Magnitudes {0, 0.5, 1, 1.5, 2,
-// 3, 4, 6}: code 1 is E2M1's subnormal 0.5, codes 2..7 are 2^(e-1) * (1 + m/2)
-// with e = code >> 1, m = code & 1.
-__device__ __forceinline__ float e2m1_f32(uint32_t code)
+// MXFP4 of one group as in quantize_group, plus its normalised quantisation error
+// ||Q(y) - y||_2 / ||y||_2.  With u = y * 2^-e the power of two cancels:
+// error = ||Q(u) - u|| / ||u||, where Q(u) is u's E2M1 value.  The hardware
+// decodes the codes back exactly (E2M1 -> f16).  An all-zero group has error 0, a
+// NaN/Inf group NaN.
+__device__ __forceinline__ uint32_t quantize_group_err(const uint32_t (&r)[32], uint32_t (&w)[4], float &err)
 {
-    const uint32_t m = code & 7u;
-    const uint32_t bits = m == 0u ? 0u : (m == 1u ? 0x3F000000u : (((126u + (m >> 1)) << 23) | ((m & 1u) << 22)));
-    return __uint_as_float(bits | ((code & 8u) << 28));
-}
-
-// Normalised MXFP4 quantisation error of one group: ||Q(y) - y||_2 / ||y||_2, where
-// Q(y) is the group dequantised from its codes `w` and scale `byte`.  An all-zero
-// group has error 0; a NaN/Inf group (byte 0xFF) gives NaN.
-__device__ __forceinline__ float group_error(const uint32_t (&r)[32], uint32_t byte, const uint32_t (&w)[4])
-{
-    const float s = byte == 0xFFu ? __uint_as_float(0x7FC00000u)
-                                  : (byte == 0u ? __uint_as_float(0x00400000u) : __uint_as_float(byte << 23));
-    float num = 0.0f, den = 0.0f;
+    float m[16];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        const float y = __uint_as_float(r[i]);
-        const float v = __fmul_rn(e2m1_f32((w[i >> 3] >> (4 * (i & 7))) & 15u), s);
-        const float d = __fsub_rn(v, y);
-        num = __fmaf_rn(d, d, num);
-        den = __fmaf_rn(y, y, den);
+    for (int i = 0; i < 16; ++i)
+        m[i] = ptx::fmax_nan(fabsf(__uint_as_float(r[2 * i])), fabsf(__uint_as_float(r[2 * i + 1])));
+#pragma unroll
+    for (int step = 8; step >= 1; step >>= 1)
+#pragma unroll
+        for (int i = 0; i < step; ++i) m[i] = ptx::fmax_nan(m[i], m[i + step]);
+    const uint32_t E = (__float_as_uint(m[0]) >> 23) & 0xFFu;
+    if (E == 0xFFu) {
+        w[0] = w[1] = w[2] = w[3] = 0u;
+        err = __uint_as_float(0x7FC00000u);
+        return 0xFFu;
     }
-    if (byte == 0xFFu) return s;   // NaN
-    return den > 0.0f ? __fsqrt_rn(__fdiv_rn(num, den)) : 0.0f;
+    const uint32_t byte = E > 2u ? E - 2u : 0u;
+    const float s = __uint_as_float((254u - byte) << 23);   // 2^-e
+    float u[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) u[i] = __fmul_rn(__uint_as_float(r[i]), s);
+    float num[4] = {0.0f, 0.0f, 0.0f, 0.0f}, den[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        w[q] = ptx::cvt_e2m1x8(u[8 * q], u[8 * q + 1], u[8 * q + 2], u[8 * q + 3], u[8 * q + 4], u[8 * q + 5],
+                               u[8 * q + 6], u[8 * q + 7]);
+        uint32_t h[4];
+        ptx::cvt_e2m1x8_to_f16x2(w[q], h);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 v = __half22float2(*reinterpret_cast<const __half2 *>(&h[k]));
+            const float a = u[8 * q + 2 * k], b = u[8 * q + 2 * k + 1];
+            const float da = __fsub_rn(v.x, a), db = __fsub_rn(v.y, b);
+            num[k] = __fmaf_rn(db, db, __fmaf_rn(da, da, num[k]));
+            den[k] = __fmaf_rn(b, b, __fmaf_rn(a, a, den[k]));
+        }
+    }
+    const float n = (num[0] + num[1]) + (num[2] + num[3]);
+    const float d = (den[0] + den[1]) + (den[2] + den[3]);
+    err = d > 0.0f ? __fsqrt_rn(__fdiv_rn(n, d)) : 0.0f;
+    return byte;
 }
 
 // Sum over the warp in a fixed shuffle order (deterministic); the result is in lane 0.

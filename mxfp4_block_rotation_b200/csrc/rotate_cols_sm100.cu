@@ -289,8 +289,8 @@ __global__ void __launch_bounds__(kColThreads, 1)
                 } else if constexpr (kMode == RotOut::Err) {
                     if (g < G && row_ok) {
                         uint32_t w[4];
-                        const uint32_t byte = quantize_group(cur, w);
-                        const float e = group_error(cur, byte, w);
+                        float e;
+                        quantize_group_err(cur, w, e);
                         if (args.err) args.err[row * G + g] = e;
                         err_acc += static_cast<double>(e);
                     }

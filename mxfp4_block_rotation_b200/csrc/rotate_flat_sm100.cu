@@ -149,8 +149,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                               cur[4 * i + 3]);
                     } else if constexpr (kMode == RotOut::Err) {
                         uint32_t w[4];
-                        const uint32_t byte = quantize_group(cur, w);
-                        const float e = group_error(cur, byte, w);
+                        float e;
+                        quantize_group_err(cur, w, e);
                         if (args.err) args.err[g] = e;
                         err_acc += static_cast<double>(e);
                     } else {
