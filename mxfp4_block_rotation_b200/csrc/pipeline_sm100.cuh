@@ -5,7 +5,6 @@
 #pragma once
 
 #include <cuda_bf16.h>
-#include <cuda_fp16.h>
 
 #include "mxq_internal.h"
 #include "sm100_ptx.cuh"
@@ -110,11 +109,23 @@ __device__ __forceinline__ uint32_t quantize_group(const uint32_t (&r)[32], uint
     return byte;
 }
 
+// E2M1 value of u (|u| < 8): round to nearest, ties to the even code, saturate at
+// 6, sign kept.  The grid step is 0.5 below 2, 1 below 4 and 2 above, and on each
+// stretch "even code" is "even multiple of the step", so rint (ties to even)
+// applied to u/step gives the same value the E2M1 conversion encodes.
+__device__ __forceinline__ float e2m1_round(float u)
+{
+    const float a = fabsf(u);
+    const float step = a < 2.0f ? 0.5f : (a < 4.0f ? 1.0f : 2.0f);
+    const float inv = a < 2.0f ? 2.0f : (a < 4.0f ? 1.0f : 0.5f);
+    const float q = fminf(__fmul_rn(rintf(__fmul_rn(a, inv)), step), 6.0f);
+    return copysignf(q, u);
+}
+
 // MXFP4 of one group as in quantize_group, plus its normalised quantisation error
 // ||Q(y) - y||_2 / ||y||_2.  With u = y * 2^-e the power of two cancels:
-// error = ||Q(u) - u|| / ||u||, where Q(u) is u's E2M1 value.  The hardware
-// decodes the codes back exactly (E2M1 -> f16).  An all-zero group has error 0, a
-// NaN/Inf group NaN.
+// error = ||Q(u) - u|| / ||u||, where Q(u) is u's E2M1 value.  An all-zero group
+// has error 0, a NaN/Inf group NaN.
 __device__ __forceinline__ uint32_t quantize_group_err(const uint32_t (&r)[32], uint32_t (&w)[4], float &err)
 {
     float m[16];
@@ -136,21 +147,16 @@ __device__ __forceinline__ uint32_t quantize_group_err(const uint32_t (&r)[32], 
     float u[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) u[i] = __fmul_rn(__uint_as_float(r[i]), s);
-    float num[4] = {0.0f, 0.0f, 0.0f, 0.0f}, den[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < 4; ++q)
         w[q] = ptx::cvt_e2m1x8(u[8 * q], u[8 * q + 1], u[8 * q + 2], u[8 * q + 3], u[8 * q + 4], u[8 * q + 5],
                                u[8 * q + 6], u[8 * q + 7]);
-        uint32_t h[4];
-        ptx::cvt_e2m1x8_to_f16x2(w[q], h);
+    float num[4] = {0.0f, 0.0f, 0.0f, 0.0f}, den[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float2 v = __half22float2(*reinterpret_cast<const __half2 *>(&h[k]));
-            const float a = u[8 * q + 2 * k], b = u[8 * q + 2 * k + 1];
-            const float da = __fsub_rn(v.x, a), db = __fsub_rn(v.y, b);
-            num[k] = __fmaf_rn(db, db, __fmaf_rn(da, da, num[k]));
-            den[k] = __fmaf_rn(b, b, __fmaf_rn(a, a, den[k]));
-        }
+    for (int i = 0; i < 32; ++i) {
+        const float d = __fsub_rn(e2m1_round(u[i]), u[i]);
+        num[i & 3] = __fmaf_rn(d, d, num[i & 3]);
+        den[i & 3] = __fmaf_rn(u[i], u[i], den[i & 3]);
     }
     const float n = (num[0] + num[1]) + (num[2] + num[3]);
     const float d = (den[0] + den[1]) + (den[2] + den[3]);

@@ -282,21 +282,6 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(float a0, float a1, float a2, flo
     return out;
 }
 
-// Four E2M1 byte pairs (a word of 8 codes) -> four f16x2: byte i's low nibble goes
-// to the low half of out[i].  Exact: every E2M1 value is an f16.
-__device__ __forceinline__ void cvt_e2m1x8_to_f16x2(uint32_t w, uint32_t (&out)[4])
-{
-    asm volatile(
-        "{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
-        "mov.b32 {q0, q1, q2, q3}, %4;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %0, q0;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %1, q1;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %2, q2;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %3, q3;\n\t}"
-        : "=r"(out[0]), "=r"(out[1]), "=r"(out[2]), "=r"(out[3])
-        : "r"(w));
-}
-
 // max that propagates NaN (so a NaN anywhere in a group makes its absmax NaN).
 __device__ __forceinline__ float fmax_nan(float a, float b)
 {
