@@ -152,6 +152,33 @@ mxq_status mxq_quant_error(const void *X_bf16, int64_t rows, int64_t cols, const
                            void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * mxq_quant_error without a workspace, for callers that cannot allocate device
+ * memory (no counterpart in the paper; it only changes where scratch lives).
+ * Such callers include a plug-in handed only input and output pointers, a
+ * process whose framework already holds the GPU's free memory (cudaMalloc
+ * would fail), and a latency-critical path that cannot take cudaMalloc's
+ * implicit synchronisation.  The partial sums mxq_quant_error keeps in its
+ * workspace live instead in a fixed 1 MiB array of device memory inside the
+ * library.  Every GPU that loads the library holds it until the process exits.
+ * The function itself allocates nothing.
+ *
+ *   arguments        as mxq_quant_error, without workspace/workspace_bytes
+ *   limit            131072 partial sums: at most 16,777,216 groups of 32
+ *                    (rows * cols <= 536,870,912; with Lambda, rows and cols
+ *                    count as rounded up to multiples of 128).  Larger inputs
+ *                    return MXQ_ERR_INVALID_ARG and mxq_last_cuda_error() says why
+ *   first call       on each device, the first call looks up the array's device
+ *                    address (cudaGetSymbolAddress) with that device current;
+ *                    make that first call before any stream capture
+ *   sharing          all calls use the same array; each call writes every slot
+ *                    it reads, so nothing carries over.  Calls whose GPU work
+ *                    overlaps (different streams, no ordering) race on it.
+ */
+mxq_status mxq_quant_error_noalloc(const void *X_bf16, int64_t rows, int64_t cols, const void *Rhat_bf16,
+                                   const float *Lambda_or_null, float *out_group_err_or_null, double *out_mean,
+                                   void *stream);
+
+/*
  * Synchronise `stream` and then read and clear the device status word.
  * Returns MXQ_ERR_CUDA if the stream reported an error and MXQ_ERR_TIMEOUT if
  * a kernel's bounded wait ran out since the last check; otherwise MXQ_OK.

@@ -68,6 +68,8 @@ def lib() -> ctypes.CDLL:
         L.mxq_quant_error_workspace_bytes.restype = ctypes.c_size_t
         L.mxq_quant_error.argtypes = [P, I64, I64, P, P, P, P, P, ctypes.c_size_t, P]
         L.mxq_quant_error.restype = I
+        L.mxq_quant_error_noalloc.argtypes = [P, I64, I64, P, P, P, P, P]
+        L.mxq_quant_error_noalloc.restype = I
         L.mxq_sync_check.argtypes = [P]
         L.mxq_sync_check.restype = I
         L.mxq_status_string.argtypes = [I]

@@ -267,6 +267,10 @@ mxq_status rotate_common(const void *X, int64_t rows, int64_t cols, const void *
 
 }  // namespace
 
+namespace mxq {
+void set_last_error(const char *msg) { std::snprintf(g_last_error, sizeof g_last_error, "%s", msg); }
+}  // namespace mxq
+
 extern "C" {
 
 mxq_status mxq_smooth_rotate_quantize(const void *X_bf16, int64_t rows, int64_t cols, const void *Rhat_bf16,

@@ -64,6 +64,9 @@ cudaError_t launch_dequant_rot(const CUtensorMap &tmap_out, const uint8_t *codes
 // *result once the wait ran out and the abort flag was raised).
 cudaError_t launch_wait_selftest(uint64_t timeout_ns, int *result, cudaStream_t stream);
 
+// Set the text mxq_last_cuda_error() returns on this thread.
+void set_last_error(const char *msg);
+
 // Device address of the status word on the current device (nullptr on failure).
 unsigned int *status_word();
 
