@@ -66,6 +66,10 @@ def lib():
         L.mxq_oracle_dequantize.restype = I
         L.mxq_oracle_group_error.argtypes = [P, I64, I64, P, P, P, P, I]
         L.mxq_oracle_group_error.restype = I
+        L.mxq_oracle_givens.argtypes = [I, I, P, P]
+        L.mxq_oracle_givens.restype = None
+        L.mxq_oracle_rotation_search.argtypes = [P, I64, I64, P, I, I, P, P, P, P, I]
+        L.mxq_oracle_rotation_search.restype = I
         L.mxq_oracle_bf16_to_double.argtypes = [P, P, I64]
         L.mxq_oracle_bf16_to_double.restype = None
         L.mxq_oracle_double_to_bf16.argtypes = [P, P, I64]
@@ -221,6 +225,35 @@ def group_error(x_bits: np.ndarray, rhat_bits: np.ndarray, lam: Optional[np.ndar
     if rc:
         raise ValueError("oracle group_error: bad shape")
     return err, float(mean[0])
+
+
+def givens(a: int, n_angle: int):
+    c = ctypes.c_double()
+    s = ctypes.c_double()
+    lib().mxq_oracle_givens(int(a), int(n_angle), ctypes.byref(c), ctypes.byref(s))
+    return c.value, s.value
+
+
+def rotation_search(x_bits: np.ndarray, lam: Optional[np.ndarray] = None, max_steps: int = 128,
+                    n_angle: int = 32, threads: int = 1) -> dict:
+    """The outlier-aware greedy Givens search (DuQuant++ write-up, §3.2).
+
+    Returns R (float64 [32, 32]), its bf16 rounding, the worst group, the number of
+    steps taken, the per-step trace of (d, j, angle) and the L-inf norm before each step.
+    """
+    x_bits = _c(x_bits, np.uint16)
+    rows, cols = x_bits.shape
+    lam32 = None if lam is None else _c(lam, np.float32)
+    R = np.zeros((GROUP, GROUP), np.float64)
+    trace = np.zeros((max(max_steps, 1), 3), np.int32)
+    linf = np.zeros(max_steps + 1, np.float64)
+    group = np.zeros(1, np.int64)
+    n = lib().mxq_oracle_rotation_search(_ptr(x_bits), rows, cols, _ptr(lam32), int(max_steps), int(n_angle),
+                                         _ptr(R), _ptr(group), _ptr(trace), _ptr(linf), threads)
+    if n < 0:
+        raise ValueError("oracle rotation_search: bad argument")
+    return {"R": R, "rhat_bits": f64_to_bf16_bits(R), "group": int(group[0]), "steps": n, "trace": trace[:n],
+            "linf": linf[:n + 1]}
 
 
 def unpack_codes(codes: np.ndarray) -> np.ndarray:

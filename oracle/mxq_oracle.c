@@ -397,6 +397,151 @@ int mxq_oracle_group_error(const uint16_t *X, int64_t rows, int64_t cols, const 
     return 0;
 }
 
+/* ------------------------------------------------------- offline rotation search */
+
+/* The Givens angle grid.  The write-up's §3.2 does not give the angle of each
+ * candidate rotation.  Here angle a (0 <= a < 2n, skipping t = 0) is
+ * t = tan(theta/2) = (a' - n)/n, with a' = a < n ? a : a + 1, and
+ * c = (1 - t^2)/(1 + t^2), s = 2t/(1 + t^2): plain IEEE double operations, so any
+ * implementation that follows them gets the same bits. */
+void mxq_oracle_givens(int a, int n, double *c, double *s)
+{
+    int ap = a < n ? a : a + 1;
+    double t = (double)(ap - n) / (double)n;
+    double t2 = t * t;
+    double den = 1.0 + t2;
+    *c = (1.0 - t2) / den;
+    *s = (2.0 * t) / den;
+}
+
+/* The outlier-aware rotation search of the write-up's §3.2, step by step.
+ *   1. Locate the worst group: among the cols/32 channel groups, the [rows, 32]
+ *      block of X / Lambda with the largest L-infinity norm (the first on ties).
+ *   2. Start from R = I (32 x 32).
+ *   3. Up to K steps:
+ *      a. d = the column of the block holding its largest |value| (first on ties);
+ *      b. for every other column j and every grid angle, the Givens rotation
+ *         G(d, j): column d -> c*x_d - s*x_j, column j -> s*x_d + c*x_j;
+ *      c. evaluate the L-infinity norm of the rotated block;
+ *      d. keep the (j, angle) that lowers it most (the first on ties); stop if
+ *         none lowers it;
+ *      e. R <- R * G;
+ *      f. block <- block * G.
+ *   4. R is shared by every group (§3.2 step 4).
+ * Rotations act on the right (X * R), the side the online step uses (§3.3).
+ * R_out: 32 x 32 double, row-major [k][n].  group_out (optional): the worst group.
+ * trace (optional): per step d, j, a.
+ * linf (optional, K + 1 entries): the block's L-infinity norm before each step.
+ * Returns the number of steps taken, or -1 on a bad argument. */
+int mxq_oracle_rotation_search(const uint16_t *X, int64_t rows, int64_t cols, const float *lam, int K,
+                               int n_angle, double *R_out, int64_t *group_out, int *trace, double *linf,
+                               int nthreads)
+{
+    if (rows <= 0 || cols <= 0 || cols % GROUP || K < 0 || n_angle < 1) return -1;
+    int64_t G = cols / GROUP;
+    /* 1. the worst group */
+    int64_t gw = 0;
+    double best = -1.0;
+    for (int64_t g = 0; g < G; ++g) {
+        double m = 0.0;
+        for (int64_t r = 0; r < rows; ++r)
+            for (int k = 0; k < GROUP; ++k) {
+                double v = bf16_to_double(X[r * cols + g * GROUP + k]);
+                if (lam) v = v / (double)lam[g * GROUP + k];
+                if (fabs(v) > m) m = fabs(v);
+            }
+        if (m > best) {
+            best = m;
+            gw = g;
+        }
+    }
+    double *B = (double *)malloc(sizeof(double) * (size_t)(rows * GROUP));
+    if (!B) return -1;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int k = 0; k < GROUP; ++k) {
+            double v = bf16_to_double(X[r * cols + gw * GROUP + k]);
+            if (lam) v = v / (double)lam[gw * GROUP + k];
+            B[r * GROUP + k] = v;
+        }
+    /* 2. R = I */
+    double R[GROUP * GROUP];
+    for (int i = 0; i < GROUP * GROUP; ++i) R[i] = (i / GROUP == i % GROUP) ? 1.0 : 0.0;
+    double colmax[GROUP];
+    int steps = 0;
+    int n_cand = 2 * n_angle;
+    double *cand = (double *)malloc(sizeof(double) * GROUP * (size_t)n_cand);
+    if (!cand) {
+        free(B);
+        return -1;
+    }
+    for (int step = 0;; ++step) {
+        for (int k = 0; k < GROUP; ++k) colmax[k] = 0.0;
+        for (int64_t r = 0; r < rows; ++r)
+            for (int k = 0; k < GROUP; ++k)
+                if (fabs(B[r * GROUP + k]) > colmax[k]) colmax[k] = fabs(B[r * GROUP + k]);
+        /* a. the column of the largest value */
+        int d = 0;
+        for (int k = 1; k < GROUP; ++k)
+            if (colmax[k] > colmax[d]) d = k;
+        double cur = colmax[d];
+        if (linf) linf[step] = cur;
+        if (step == K) break;
+        /* b, c. every candidate's L-infinity norm */
+#pragma omp parallel for schedule(static) num_threads(nthreads > 0 ? nthreads : 1)
+        for (int ci = 0; ci < GROUP * n_cand; ++ci) {
+            int j = ci / n_cand, a = ci % n_cand;
+            if (j == d) {
+                cand[ci] = INFINITY;
+                continue;
+            }
+            double c, s;
+            mxq_oracle_givens(a, n_angle, &c, &s);
+            double m = 0.0;
+            for (int k = 0; k < GROUP; ++k)
+                if (k != d && k != j && colmax[k] > m) m = colmax[k];
+            for (int64_t r = 0; r < rows; ++r) {
+                double xd = B[r * GROUP + d], xj = B[r * GROUP + j];
+                double u = c * xd - s * xj;
+                double w = s * xd + c * xj;
+                if (fabs(u) > m) m = fabs(u);
+                if (fabs(w) > m) m = fabs(w);
+            }
+            cand[ci] = m;
+        }
+        /* d. the largest decrease */
+        int bi = -1;
+        for (int ci = 0; ci < GROUP * n_cand; ++ci)
+            if (cand[ci] < cur && (bi < 0 || cand[ci] < cand[bi])) bi = ci;
+        if (bi < 0) break;
+        int j = bi / n_cand, a = bi % n_cand;
+        double c, s;
+        mxq_oracle_givens(a, n_angle, &c, &s);
+        /* e. R <- R * G */
+        for (int r = 0; r < GROUP; ++r) {
+            double rd = R[r * GROUP + d], rj = R[r * GROUP + j];
+            R[r * GROUP + d] = c * rd - s * rj;
+            R[r * GROUP + j] = s * rd + c * rj;
+        }
+        /* f. block <- block * G */
+        for (int64_t r = 0; r < rows; ++r) {
+            double xd = B[r * GROUP + d], xj = B[r * GROUP + j];
+            B[r * GROUP + d] = c * xd - s * xj;
+            B[r * GROUP + j] = s * xd + c * xj;
+        }
+        if (trace) {
+            trace[3 * step] = d;
+            trace[3 * step + 1] = j;
+            trace[3 * step + 2] = a;
+        }
+        ++steps;
+    }
+    memcpy(R_out, R, sizeof R);
+    if (group_out) *group_out = gw;
+    free(cand);
+    free(B);
+    return steps;
+}
+
 /* Exposed for the pins: exact bf16 <-> double conversions. */
 void mxq_oracle_bf16_to_double(const uint16_t *b, double *d, int64_t n)
 {
