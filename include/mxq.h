@@ -179,6 +179,56 @@ mxq_status mxq_quant_error_noalloc(const void *X_bf16, int64_t rows, int64_t col
                                    void *stream);
 
 /*
+ * The outlier-aware rotation search that builds R̂ offline (DuQuant++ write-up,
+ * §3.2; its pitfalls section asks for the search on the smoothed activations
+ * X / Λ, and its implementation notes for double precision).  Steps:
+ *   1. the worst group: among the cols/32 channel groups, the [rows, 32] block
+ *      of X / Λ with the largest max |value| (the first on ties);
+ *   2. R = I;
+ *   3. up to max_steps greedy steps.  Each step:
+ *      - takes d, the first column of the block holding its largest |value|;
+ *      - tries, for every other column j and every grid angle, the Givens
+ *        rotation G(d, j) that maps column d to c x_d - s x_j and column j to
+ *        s x_d + c x_j;
+ *      - keeps the rotation that gives the smallest max |value| of block * G
+ *        (the first in (j, angle) order on ties);
+ *      - stops if no candidate is strictly below the current max;
+ *      - sets R <- R G and block <- block * G.
+ * The write-up leaves the angle open.  Here the grid has 2 * n_angle angles,
+ * angle a at t = tan(θ/2) = (a' - n_angle) / n_angle with a' = a for
+ * a < n_angle and a + 1 otherwise (t runs over [-1, 1] without 0).  Then
+ * c = (1 - t²)/(1 + t²) and s = 2t/(1 + t²), each a plain IEEE double expression.
+ * Every value a decision depends on is one IEEE double operation, and every
+ * reduction is a max, so the result is the same bits as a sequential double
+ * evaluation of these steps.
+ *
+ * All pointers are device memory of the current device; the work is queued on
+ * `stream` (2 * max_steps + 6 kernel launches, no host synchronisation).
+ *   X_bf16          in   [rows, cols] bf16 row-major, 16-byte aligned; rows >= 1,
+ *                        cols >= 32 and a multiple of 32
+ *   Lambda_or_null  in   [cols] fp32 per-channel divisor, or NULL for none
+ *   max_steps       in   K, 0..65536 (the write-up uses 128)
+ *   n_angle         in   1..128; 2 * n_angle angles are tried per column pair
+ *   R_out           out  [32][32] double row-major [k][n], 8-byte aligned: the rotation
+ *   Rhat_bf16_out_or_null  out  [32][32] bf16, R rounded to nearest even, 2-byte aligned
+ *   trace_out_or_null      out  [max_steps][3] int32 (d, j, angle) per step taken
+ *   linf_out_or_null       out  [max_steps + 1] double: the block's max |value|
+ *                        before each step, and after the last one taken
+ *   steps_out_or_null      out  one int32: the number of steps taken
+ *   group_out_or_null      out  one int64: the worst group's index
+ *   workspace       in   mxq_rotation_search_workspace_bytes(rows, cols, n_angle)
+ *                        bytes, 256-byte aligned, caller-owned, overwritten
+ * Entries of trace and linf beyond the steps taken are left untouched.
+ * Errors: MXQ_ERR_INVALID_ARG for a bad size, a host pointer, a misaligned or
+ * too-small buffer, or outputs that overlap X, Λ, each other or the workspace.
+ */
+size_t mxq_rotation_search_workspace_bytes(int64_t rows, int64_t cols, int n_angle);
+mxq_status mxq_rotation_search(const void *X_bf16, int64_t rows, int64_t cols, const float *Lambda_or_null,
+                               int max_steps, int n_angle, double *R_out, void *Rhat_bf16_out_or_null,
+                               int32_t *trace_out_or_null, double *linf_out_or_null, int32_t *steps_out_or_null,
+                               int64_t *group_out_or_null, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Synchronise `stream` and then read and clear the device status word.
  * Returns MXQ_ERR_CUDA if the stream reported an error and MXQ_ERR_TIMEOUT if
  * a kernel's bounded wait ran out since the last check; otherwise MXQ_OK.

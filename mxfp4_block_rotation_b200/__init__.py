@@ -70,6 +70,10 @@ def lib() -> ctypes.CDLL:
         L.mxq_quant_error.restype = I
         L.mxq_quant_error_noalloc.argtypes = [P, I64, I64, P, P, P, P, P]
         L.mxq_quant_error_noalloc.restype = I
+        L.mxq_rotation_search_workspace_bytes.argtypes = [I64, I64, I]
+        L.mxq_rotation_search_workspace_bytes.restype = ctypes.c_size_t
+        L.mxq_rotation_search.argtypes = [P, I64, I64, P, I, I, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+        L.mxq_rotation_search.restype = I
         L.mxq_sync_check.argtypes = [P]
         L.mxq_sync_check.restype = I
         L.mxq_status_string.argtypes = [I]
@@ -215,6 +219,45 @@ def quant_error(x: torch.Tensor, rhat: torch.Tensor, lam: Optional[torch.Tensor]
                                _ptr(workspace), workspace.numel(), _stream(dev, stream))
     _check(st, "mxq_quant_error")
     return err, mean
+
+
+def rotation_search(x: torch.Tensor, lam: Optional[torch.Tensor] = None, *, max_steps: int = 128,
+                    n_angle: int = 32, workspace: Optional[torch.Tensor] = None, stream=None) -> dict:
+    """The outlier-aware greedy Givens search for the shared rotation (DuQuant++ write-up, §3.2).
+
+    Returns device tensors: R (float64 [32, 32]), rhat (R in bf16, the hot path's input),
+    trace (int32 [max_steps, 3]: d, j, angle per step; rows past `steps` unwritten),
+    linf (float64 [max_steps + 1]), steps (int32 0-d) and group (int64 0-d).
+    `workspace` (uint8, device) is allocated here when not given.  Nothing is synchronised.
+    """
+    if x.dim() != 2:
+        raise ValueError("x must be 2-D [rows, cols]")
+    dev = x.device
+    if dev.type != "cuda":
+        raise ValueError("x must be a CUDA tensor (this library has no CPU path)")
+    _need(x, "x", torch.bfloat16, dev)
+    if lam is not None:
+        _need(lam, "lam", torch.float32, dev)
+        if tuple(lam.shape) != (x.shape[1],):
+            raise ValueError("lam must be [cols]")
+    rows, cols = x.shape
+    need = int(lib().mxq_rotation_search_workspace_bytes(rows, cols, int(n_angle)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _need(workspace, "workspace", torch.uint8, dev)
+    out = {
+        "R": torch.empty((32, 32), dtype=torch.float64, device=dev),
+        "rhat": torch.empty((32, 32), dtype=torch.bfloat16, device=dev),
+        "trace": torch.zeros((max(int(max_steps), 1), 3), dtype=torch.int32, device=dev),
+        "linf": torch.zeros(int(max_steps) + 1, dtype=torch.float64, device=dev),
+        "steps": torch.empty((), dtype=torch.int32, device=dev),
+        "group": torch.empty((), dtype=torch.int64, device=dev),
+    }
+    st = lib().mxq_rotation_search(_ptr(x), rows, cols, _ptr(lam), int(max_steps), int(n_angle), _ptr(out["R"]),
+                                   _ptr(out["rhat"]), _ptr(out["trace"]), _ptr(out["linf"]), _ptr(out["steps"]),
+                                   _ptr(out["group"]), _ptr(workspace), workspace.numel(), _stream(dev, stream))
+    _check(st, "mxq_rotation_search")
+    return out
 
 
 def selftest_bounded_wait(timeout_ms: int = 50, device=None, stream=None) -> int:

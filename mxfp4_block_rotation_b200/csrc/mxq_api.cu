@@ -405,6 +405,81 @@ mxq_status mxq_quant_error(const void *X_bf16, int64_t rows, int64_t cols, const
     return MXQ_OK;
 }
 
+size_t mxq_rotation_search_workspace_bytes(int64_t rows, int64_t cols, int n_angle)
+{
+    if (check_shape(rows, cols) != MXQ_OK || rows < 1 || cols < 32 || n_angle < 1 || n_angle > 128) return 0;
+    return mxq::rotation_search_workspace(rows, cols, n_angle);
+}
+
+mxq_status mxq_rotation_search(const void *X_bf16, int64_t rows, int64_t cols, const float *Lambda_or_null,
+                               int max_steps, int n_angle, double *R_out, void *Rhat_bf16_out_or_null,
+                               int32_t *trace_out_or_null, double *linf_out_or_null, int32_t *steps_out_or_null,
+                               int64_t *group_out_or_null, void *workspace, size_t workspace_bytes, void *stream)
+{
+    mxq_status st = check_shape(rows, cols);
+    if (st != MXQ_OK) return st;
+    if (rows < 1 || cols < 32) return bad("the search needs at least one row and one group");
+    if (max_steps < 0 || max_steps > 65536) return bad("max_steps must be in 0..65536");
+    if (n_angle < 1 || n_angle > 128) return bad("n_angle must be in 1..128");
+    if (!X_bf16 || !R_out) return bad("null pointer");
+    if (!aligned(X_bf16, 16)) return bad("X must be 16-byte aligned");
+    if (Lambda_or_null && !aligned(Lambda_or_null, 4)) return bad("Lambda must be 4-byte aligned");
+    if (!aligned(R_out, 8)) return bad("R_out must be 8-byte aligned");
+    if (Rhat_bf16_out_or_null && !aligned(Rhat_bf16_out_or_null, 2)) return bad("Rhat_out must be 2-byte aligned");
+    if (trace_out_or_null && !aligned(trace_out_or_null, 4)) return bad("trace must be 4-byte aligned");
+    if (linf_out_or_null && !aligned(linf_out_or_null, 8)) return bad("linf must be 8-byte aligned");
+    if (steps_out_or_null && !aligned(steps_out_or_null, 4)) return bad("steps_out must be 4-byte aligned");
+    if (group_out_or_null && !aligned(group_out_or_null, 8)) return bad("group_out must be 8-byte aligned");
+    const size_t need = mxq_rotation_search_workspace_bytes(rows, cols, n_angle);
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < need)
+        return bad("workspace missing, not 256-byte aligned or smaller than mxq_rotation_search_workspace_bytes()");
+    const uint64_t nx = static_cast<uint64_t>(rows) * cols * 2, nl = Lambda_or_null ? static_cast<uint64_t>(cols) * 4 : 0;
+    const void *ins[2] = {X_bf16, Lambda_or_null};
+    const uint64_t nins[2] = {nx, nl};
+    void *outs[7] = {R_out, Rhat_bf16_out_or_null, trace_out_or_null, linf_out_or_null, steps_out_or_null,
+                     group_out_or_null, workspace};
+    const uint64_t nouts[7] = {32 * 32 * 8,
+                               Rhat_bf16_out_or_null ? 32 * 32 * 2u : 0u,
+                               trace_out_or_null ? static_cast<uint64_t>(max_steps) * 12 : 0u,
+                               linf_out_or_null ? static_cast<uint64_t>(max_steps + 1) * 8 : 0u,
+                               steps_out_or_null ? 4u : 0u,
+                               group_out_or_null ? 8u : 0u,
+                               need};
+    for (int o = 0; o < 7; ++o) {
+        for (int i = 0; i < 2; ++i)
+            if (overlaps(outs[o], nouts[o], ins[i], nins[i])) return bad("an output overlaps an input");
+        for (int o2 = o + 1; o2 < 7; ++o2)
+            if (overlaps(outs[o], nouts[o], outs[o2], nouts[o2])) return bad("outputs overlap");
+    }
+    int dev = 0, sms = 0;
+    if ((st = current_device(&dev, &sms)) != MXQ_OK) return st;
+    if ((st = check_buffer(X_bf16, nx, dev)) != MXQ_OK) return st;
+    if (Lambda_or_null && (st = check_buffer(Lambda_or_null, nl, dev)) != MXQ_OK) return st;
+    for (int o = 0; o < 7; ++o)
+        if (outs[o] && nouts[o] && (st = check_buffer(outs[o], nouts[o], dev)) != MXQ_OK) return st;
+
+    mxq::SearchArgs a{};
+    a.X = X_bf16;
+    a.lambda = Lambda_or_null;
+    a.rows = rows;
+    a.cols = cols;
+    a.max_steps = max_steps;
+    a.n_angle = n_angle;
+    a.R = R_out;
+    a.rhat = static_cast<uint16_t *>(Rhat_bf16_out_or_null);
+    a.trace = trace_out_or_null;
+    a.linf = linf_out_or_null;
+    a.steps = steps_out_or_null;
+    a.group = group_out_or_null;
+    a.workspace = workspace;
+    const cudaError_t e = mxq::launch_rotation_search(a, sms, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) {
+        note_cuda(e, "launch rotation-search kernels");
+        return MXQ_ERR_CUDA;
+    }
+    return MXQ_OK;
+}
+
 mxq_status mxq_sync_check(void *stream)
 {
     unsigned int status = 0;

@@ -60,6 +60,26 @@ cudaError_t launch_dequant_rot(const CUtensorMap &tmap_out, const uint8_t *codes
                                int64_t cols, const uint16_t *rhat, const float *lambda, int num_sms,
                                cudaStream_t stream);
 
+// The outlier-aware rotation search (all pointers device memory; see mxq.h).
+struct SearchArgs {
+    const void *X;             // bf16 [rows, cols], 16-byte aligned
+    const float *lambda;       // fp32 [cols] or nullptr
+    int64_t rows;
+    int64_t cols;
+    int max_steps;             // K
+    int n_angle;               // the Givens grid has 2 * n_angle angles
+    double *R;                 // [32][32] result, row-major [k][n]
+    uint16_t *rhat;            // bf16 [32][32] or nullptr
+    int32_t *trace;            // [max_steps][3] (d, j, angle) or nullptr
+    double *linf;              // [max_steps + 1] or nullptr
+    int32_t *steps;            // steps taken, or nullptr
+    int64_t *group;            // the worst group, or nullptr
+    void *workspace;           // rotation_search_workspace() bytes, 256-byte aligned
+};
+size_t rotation_search_workspace(int64_t rows, int64_t cols, int n_angle);
+cudaError_t launch_rotation_search(const SearchArgs &args, int num_sms, cudaStream_t stream);
+int rotation_search_launches(int max_steps);
+
 // Diagnostic kernel: a bounded wait on a barrier nothing completes (writes 2 to
 // *result once the wait ran out and the abort flag was raised).
 cudaError_t launch_wait_selftest(uint64_t timeout_ns, int *result, cudaStream_t stream);

@@ -90,3 +90,34 @@ def test_binding_refuses_cpu_tensors():
     r = torch.eye(32, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         mxq.smooth_rotate_quantize(x, r)
+
+
+def _search(L, x, rows, cols, lam, K, n, R, rhat=None, trace=None, linf=None, steps=None, group=None, ws=None,
+            wsb=1 << 30):
+    return L.mxq_rotation_search(P(x), rows, cols, P(lam), K, n, P(R), P(rhat), P(trace), P(linf), P(steps),
+                                 P(group), P(ws), wsb, None)
+
+
+def test_rotation_search_rejects_bad_arguments(L):
+    a = 0x100000
+    ws = 0x40000000
+    assert L.mxq_rotation_search_workspace_bytes(4, 64, 32) >= 512 + 32 * 64 * 8 + 4 * 32 * 8
+    assert L.mxq_rotation_search_workspace_bytes(0, 64, 32) == 0
+    assert L.mxq_rotation_search_workspace_bytes(4, 64, 0) == 0
+    assert _search(L, a, 0, 64, None, 8, 32, a * 3, ws=ws) == INVALID          # no rows
+    assert _search(L, a, 4, 0, None, 8, 32, a * 3, ws=ws) == INVALID           # no groups
+    assert _search(L, a, 4, 48, None, 8, 32, a * 3, ws=ws) == INVALID          # cols not a multiple of 32
+    assert _search(L, a, 4, 64, None, -1, 32, a * 3, ws=ws) == INVALID         # negative K
+    assert _search(L, a, 4, 64, None, 65537, 32, a * 3, ws=ws) == INVALID      # K too large
+    assert _search(L, a, 4, 64, None, 8, 0, a * 3, ws=ws) == INVALID           # empty angle grid
+    assert _search(L, a, 4, 64, None, 8, 129, a * 3, ws=ws) == INVALID
+    assert _search(L, None, 4, 64, None, 8, 32, a * 3, ws=ws) == INVALID       # null X
+    assert _search(L, a, 4, 64, None, 8, 32, None, ws=ws) == INVALID           # null R
+    assert _search(L, a + 8, 4, 64, None, 8, 32, a * 3, ws=ws) == INVALID      # X not 16-B aligned
+    assert _search(L, a, 4, 64, None, 8, 32, a * 3 + 4, ws=ws) == INVALID      # R not 8-B aligned
+    assert _search(L, a, 4, 64, None, 8, 32, a * 3, ws=ws + 128) == INVALID    # workspace not 256-B aligned
+    assert _search(L, a, 4, 64, None, 8, 32, a * 3, ws=ws, wsb=64) == INVALID  # workspace too small
+    assert _search(L, a, 4, 64, None, 8, 32, a * 3, ws=None) == INVALID        # no workspace
+    assert _search(L, a, 4, 64, None, 8, 32, a + 64, ws=ws) == INVALID         # R overlaps X
+    assert _search(L, a, 4, 64, None, 8, 32, a * 3, linf=a * 3 + 8192 - 8, ws=ws) == INVALID  # linf overlaps R
+    assert L.mxq_last_cuda_error().startswith(b"invalid argument")
