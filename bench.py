@@ -384,6 +384,17 @@ def run_extras(mxq, w, xs, rhat, outs, dev, stream, k=300):
         assert st == 0
     row("quant_error_per_group_and_mean", _timed(qerr, k, stream, dev), rows * cols * 2.0 + rows * (cols // 32) * 4.0,
         "per-group ||Q(y)-y||/||y|| (fp32 out) and its mean: reads X, writes 4 B per group")
+    # the offline rotation search on the same activations, smoothed: K = 128 steps, 64 angles per pair
+    sws = torch.empty(mxq.lib().mxq_rotation_search_workspace_bytes(rows, cols, 32), dtype=torch.uint8, device=dev)
+    found = {}
+
+    def search(i):
+        found["out"] = mxq.rotation_search(xs[i & 1], lam, max_steps=128, n_angle=32, workspace=sws, stream=stream)
+    ms = _timed(search, 10, stream, dev)
+    res["rotation_search_K128"] = {
+        "what": "greedy Givens search for R^ on X / Lambda (worst group by column maxima, 128 steps, 64 angles)",
+        "ms": ms, "steps": int(found["out"]["steps"]), "launches": 2 * 128 + 6,
+        "bound": "latency: two dependent launches per step"}
     mxq.sync_check()
     return res
 

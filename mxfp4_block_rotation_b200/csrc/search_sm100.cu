@@ -24,16 +24,21 @@
 // same steps.
 //
 // Kernels, in stream order (no kernel waits on another inside the GPU):
-//   init     zero the column maxima, the search state and the candidate table; R = I
+//   init     zero the column maxima, the search state and the two candidate tables; R = I
 //   colmax   per column of X, the largest |x| (bf16 magnitude bits, NaN skipped)
 //   pick     per group, max_k colmax_k / |Λ_k|; the first group with the largest
 //   gather   the worst group's block, divided by Λ, column-major in double; its column maxima
 //   cand     (per step) for every j != d and every angle, the rotated block's
-//            max |value| over columns d and j, by row chunks, combined with atomicMax
-//   select   (per step) the best candidate; update R, the block's two columns and
-//            their maxima; record the trace; clear the candidate table
+//            max |value| over columns d and j, by row chunks (rows that cannot
+//            hold the max left out), combined with atomicMax
+//   select   (per step, one block per row range) the best candidate, found by
+//            every block; each block rotates its rows of the two columns; block 0
+//            updates R and the trace; the last block to finish sets the two new
+//            column maxima.  The candidate tables alternate by step parity, so
+//            the next step's table is cleared while this one is read.
 //   finish   R in bf16; the step count and the group
 #include <cuda_bf16.h>
+#include <math_constants.h>
 
 #include "mxq_internal.h"
 
@@ -43,7 +48,8 @@ namespace {
 constexpr int kGroup = 32;
 constexpr int kCandThreads = 256;
 constexpr int kCandChunk = 1024;      // rows per cand CTA
-constexpr int kSelectThreads = 512;
+constexpr int kSelectThreads = 256;
+constexpr int kPickThreads = 512;
 constexpr int kSelectWarps = kSelectThreads / 32;
 constexpr int kColmaxThreads = 256;
 
@@ -52,9 +58,11 @@ constexpr int kColmaxThreads = 256;
 // as numbers, so atomicMax on the bits is a max of the values.
 struct SearchState {
     unsigned long long colmax[kGroup];
+    unsigned long long nm[2];     // the two rotated columns' new maxima, during a select
     long long group;
     int done;
     int steps;
+    unsigned int ticket;          // blocks of the current select that have finished
 };
 static_assert(sizeof(SearchState) <= 512, "search state must fit its slot");
 
@@ -92,7 +100,9 @@ __global__ void __launch_bounds__(1024)
     for (int64_t i = t0; i < n_cand; i += stride) cand[i] = 0ull;
     for (int64_t i = t0; i < kGroup * kGroup; i += stride) R[i] = (i / kGroup == i % kGroup) ? 1.0 : 0.0;
     if (t0 < kGroup) st->colmax[t0] = 0ull;
+    if (t0 < 2) st->nm[t0] = 0ull;
     if (t0 == 0) {
+        st->ticket = 0u;
         st->group = 0;
         st->done = 0;
         st->steps = 0;
@@ -149,13 +159,13 @@ __global__ void __launch_bounds__(kColmaxThreads)
 // max_r (|x_r| / |Λ|) = (max_r |x_r|) / |Λ| exactly: one division per column.
 // A NaN quotient (0/0, inf/inf, NaN Λ) is skipped, as it would be element by
 // element.
-__global__ void __launch_bounds__(kSelectThreads)
+__global__ void __launch_bounds__(kPickThreads)
     search_pick_kernel(const unsigned int *__restrict__ colmax_x, const float *__restrict__ lam, int64_t n_groups,
                        SearchState *st)
 {
     double best = -1.0;
     long long bg = 0;
-    for (int64_t g = threadIdx.x; g < n_groups; g += kSelectThreads) {
+    for (int64_t g = threadIdx.x; g < n_groups; g += kPickThreads) {
         double m = 0.0;
         for (int k = 0; k < kGroup; ++k) {
             const unsigned int mb = colmax_x[g * kGroup + k];
@@ -169,8 +179,8 @@ __global__ void __launch_bounds__(kSelectThreads)
         }
     }
     // larger value wins; equal values: the smaller group
-    __shared__ double sv[kSelectThreads / 32];
-    __shared__ long long sg[kSelectThreads / 32];
+    __shared__ double sv[kPickThreads / 32];
+    __shared__ long long sg[kPickThreads / 32];
     for (int o = 16; o >= 1; o >>= 1) {
         const double ov = __shfl_xor_sync(0xffffffffu, best, o);
         const long long og = __shfl_xor_sync(0xffffffffu, bg, o);
@@ -186,8 +196,8 @@ __global__ void __launch_bounds__(kSelectThreads)
     }
     __syncthreads();
     if (warp == 0) {
-        best = lane < kSelectWarps ? sv[lane] : -1.0;
-        bg = lane < kSelectWarps ? sg[lane] : 0;
+        best = lane < (kPickThreads / 32) ? sv[lane] : -1.0;
+        bg = lane < (kPickThreads / 32) ? sg[lane] : 0;
         for (int o = 16; o >= 1; o >>= 1) {
             const double ov = __shfl_xor_sync(0xffffffffu, best, o);
             const long long og = __shfl_xor_sync(0xffffffffu, bg, o);
@@ -224,42 +234,97 @@ __global__ void __launch_bounds__(256)
     if (m > 0.0) atomicMax(&st->colmax[lane], double_to_bits(m));
 }
 
+// Block-wide max of non-negative, non-NaN doubles (every thread gets it).
+template <int kThreads>
+__device__ __forceinline__ double block_max(double m, double *red)
+{
+    for (int o = 16; o >= 1; o >>= 1) {
+        const double om = __shfl_xor_sync(0xffffffffu, m, o);
+        if (om > m) m = om;
+    }
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    __syncthreads();
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+    m = lane < kThreads / 32 ? red[lane] : 0.0;
+    for (int o = 16; o >= 1; o >>= 1) {
+        const double om = __shfl_xor_sync(0xffffffffu, m, o);
+        if (om > m) m = om;
+    }
+    return m;
+}
+
 // One greedy step's candidates.  Block (x, y): rows [x*kCandChunk, ...) of the
-// block, partner column j = y.  Columns d and j of those rows are staged in
-// shared memory; warp w evaluates angles w, w + 8, ...; each lane a strided
-// subset of the rows.  For one (j, angle) the largest |rotated value| of the
-// two columns goes to cand[j * n_cand_j + angle] by atomicMax on the bits.
-// The other 30 columns do not change under G(d, j): the select kernel adds
-// their maxima.
+// block, partner column j = y.
+// A row r can be left out when it cannot hold any candidate's max:
+//   - its rotated pair (u, w) is bounded by b_r = fl(|x_d| + |x_j|).  Rounding
+//     is monotone and |c|, |s| <= 1, so |fl(fl(c x_d) - fl(s x_j))| <= b_r, and
+//     the same holds for w;
+//   - at the row r* with the largest b, for every angle,
+//     max(|u|, |w|) >= sqrt((x_d² + x_j²) / 2) >= b_r* / 2, less a few ulps;
+//   - so a row with b_r < 0.499 b_r* never holds a candidate's max, and the max
+//     over the rows kept is the max over all rows, bit for bit.
+// With an infinite b_r* nothing is left out, because an infinite pair can
+// rotate to NaN.  The rows kept are packed in shared memory.  Warp w evaluates
+// angles w, w + 8, ... over them.  The largest |rotated value| of the two
+// columns goes to cand[j * 2n + angle] by atomicMax on the bits.  The other 30
+// columns do not change under G(d, j); the select kernel adds their maxima.
 __global__ void __launch_bounds__(kCandThreads)
     search_cand_kernel(const double *__restrict__ B, int64_t rows, int n_angle, const SearchState *st,
                        unsigned long long *cand)
 {
+    constexpr int kPer = kCandChunk / kCandThreads;
     __shared__ double sx[2][kCandChunk];
     __shared__ double cm[kGroup];
+    __shared__ double red[kCandThreads / 32];
+    __shared__ int n_kept;
     if (st->done) return;
     if (threadIdx.x < kGroup) cm[threadIdx.x] = bits_to_double(st->colmax[threadIdx.x]);
+    if (threadIdx.x == 0) n_kept = 0;
     __syncthreads();
     const int d = first_argmax32(cm);
     const int j = blockIdx.y;
     if (j == d) return;
     const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kCandChunk;
     const int n = static_cast<int>(rows - r0 < kCandChunk ? rows - r0 : kCandChunk);
-    for (int i = threadIdx.x; i < n; i += kCandThreads) {
-        sx[0][i] = B[d * rows + r0 + i];
-        sx[1][i] = B[j * rows + r0 + i];
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    double xd[kPer], xj[kPer], b[kPer];
+    double bmax = 0.0;
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+        const int i = threadIdx.x + u * kCandThreads;
+        xd[u] = i < n ? B[d * rows + r0 + i] : 0.0;
+        xj[u] = i < n ? B[j * rows + r0 + i] : 0.0;
+        b[u] = __dadd_rn(fabs(xd[u]), fabs(xj[u]));
+        if (b[u] > bmax) bmax = b[u];
+    }
+    bmax = block_max<kCandThreads>(bmax, red);
+    const double thr = bmax == CUDART_INF ? 0.0 : __dmul_rn(bmax, 0.4990234375);
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+        const int i = threadIdx.x + u * kCandThreads;
+        const bool keep = i < n && b[u] >= thr;
+        const unsigned int ballot = __ballot_sync(0xffffffffu, keep);
+        int base = 0;
+        if (lane == 0 && ballot) base = atomicAdd(&n_kept, __popc(ballot));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if (keep) {
+            const int pos = base + __popc(ballot & ((1u << lane) - 1u));
+            sx[0][pos] = xd[u];
+            sx[1][pos] = xj[u];
+        }
     }
     __syncthreads();
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int nk = n_kept;
     const int n_cand_j = 2 * n_angle;
     for (int a = warp; a < n_cand_j; a += kCandThreads / 32) {
         double c, s;
         givens_cs(a, n_angle, c, s);
         double m = 0.0;
-        for (int i = lane; i < n; i += 32) {
-            const double xd = sx[0][i], xj = sx[1][i];
-            const double u = __dsub_rn(__dmul_rn(c, xd), __dmul_rn(s, xj));
-            const double w = __dadd_rn(__dmul_rn(s, xd), __dmul_rn(c, xj));
+        for (int i = lane; i < nk; i += 32) {
+            const double x0 = sx[0][i], x1 = sx[1][i];
+            const double u = __dsub_rn(__dmul_rn(c, x0), __dmul_rn(s, x1));
+            const double w = __dadd_rn(__dmul_rn(s, x0), __dmul_rn(c, x1));
             const double au = fabs(u), aw = fabs(w);
             if (au > m) m = au;
             if (aw > m) m = aw;
@@ -272,50 +337,48 @@ __global__ void __launch_bounds__(kCandThreads)
     }
 }
 
-// Block-wide max of non-negative, non-NaN doubles over a kSelectThreads block
-// (all threads get it).
-__device__ __forceinline__ double block_max(double m, double *red)
-{
-    for (int o = 16; o >= 1; o >>= 1) {
-        const double om = __shfl_xor_sync(0xffffffffu, m, o);
-        if (om > m) m = om;
-    }
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    __syncthreads();
-    if (lane == 0) red[warp] = m;
-    __syncthreads();
-    m = lane < kSelectWarps ? red[lane] : 0.0;
-    for (int o = 16; o >= 1; o >>= 1) {
-        const double om = __shfl_xor_sync(0xffffffffu, m, o);
-        if (om > m) m = om;
-    }
-    return m;
-}
-
 // Step `step` of the search, after its cand kernel (or, at step == K, only the
-// final L-infinity norm).  One block of kSelectThreads threads.
-//   cur = the block's L-infinity norm (the largest column maximum), column d its first holder;
-//   every candidate's norm is max(its cand entry, the maxima of the 30 other columns);
-//   the first candidate with the smallest norm below cur wins; if none, the search stops;
-//   R <- R G and B <- B G on columns d and j, their maxima recomputed; the table cleared.
+// final L-infinity norm).  Every block takes the same decision from the same
+// data:
+//   - cur = the block's L-infinity norm (the largest column maximum), column d
+//     its first holder;
+//   - a candidate's norm is max(its cand entry, the maxima of the 30 other columns);
+//   - the first candidate with the smallest norm below cur wins; with none, the
+//     search stops.
+// Each block then applies B <- B G to its own rows of columns d and j and adds
+// their maxima to st->nm by atomicMax.  Block 0 applies R <- R G and records
+// the trace.  The last block to finish (a ticket counter; nothing waits) moves
+// the two new maxima into st->colmax.  The next step's candidate table is
+// cleared here: nobody reads it during this kernel.
 __global__ void __launch_bounds__(kSelectThreads)
-    search_select_kernel(double *__restrict__ B, int64_t rows, int n_angle, int step, int K, SearchState *st,
-                         unsigned long long *cand, double *__restrict__ R, int32_t *trace, double *linf)
+    search_select_kernel(double *__restrict__ B, int64_t rows, int64_t rows_per_block, int n_angle, int step, int K,
+                         SearchState *st, const unsigned long long *__restrict__ cand, unsigned long long *cand_next,
+                         double *__restrict__ R, int32_t *trace, double *linf)
 {
     __shared__ double cm[kGroup];
-    __shared__ double red[kSelectThreads / 32];
-    __shared__ double sv[kSelectThreads / 32];
-    __shared__ int sc[kSelectThreads / 32];
+    __shared__ double other[kGroup];
+    __shared__ double red[kSelectWarps];
+    __shared__ double sv[kSelectWarps];
+    __shared__ int sc[kSelectWarps];
     if (st->done) return;
+    const bool lead = blockIdx.x == 0 && threadIdx.x == 0;
     if (threadIdx.x < kGroup) cm[threadIdx.x] = bits_to_double(st->colmax[threadIdx.x]);
     __syncthreads();
     const int d = first_argmax32(cm);
     const double cur = cm[d];
-    if (threadIdx.x == 0 && linf) linf[step] = cur;
+    if (lead && linf) linf[step] = cur;
     if (step == K) {
-        if (threadIdx.x == 0) st->steps = K;
+        if (lead) st->steps = K;
         return;
     }
+    if (threadIdx.x < kGroup) {
+        const int j = threadIdx.x;
+        double v = 0.0;
+        for (int k = 0; k < kGroup; ++k)
+            if (k != d && k != j && cm[k] > v) v = cm[k];
+        other[j] = v;
+    }
+    __syncthreads();
     const int n_cand_j = 2 * n_angle;
     const int n_cand = kGroup * n_cand_j;
     double bv = 0.0;
@@ -323,9 +386,7 @@ __global__ void __launch_bounds__(kSelectThreads)
     for (int ci = threadIdx.x; ci < n_cand; ci += kSelectThreads) {
         const int j = ci / n_cand_j;
         if (j == d) continue;
-        double v = 0.0;
-        for (int k = 0; k < kGroup; ++k)
-            if (k != d && k != j && cm[k] > v) v = cm[k];
+        double v = other[j];
         const double cv = bits_to_double(cand[ci]);
         if (cv > v) v = cv;
         if (v < cur && (bc < 0 || v < bv)) {
@@ -358,11 +419,10 @@ __global__ void __launch_bounds__(kSelectThreads)
             bc = oc;
         }
     }
-    // every thread now holds the same (bv, bc); the table is read: clear it for the next step
-    __syncthreads();
-    for (int ci = threadIdx.x; ci < n_cand; ci += kSelectThreads) cand[ci] = 0ull;
+    for (int i = blockIdx.x * kSelectThreads + threadIdx.x; i < n_cand; i += gridDim.x * kSelectThreads)
+        cand_next[i] = 0ull;
     if (bc < 0) {
-        if (threadIdx.x == 0) {
+        if (lead) {
             st->done = 1;
             st->steps = step;
         }
@@ -371,16 +431,23 @@ __global__ void __launch_bounds__(kSelectThreads)
     const int j = bc / n_cand_j, a = bc % n_cand_j;
     double c, s;
     givens_cs(a, n_angle, c, s);
-    if (threadIdx.x < kGroup) {
+    if (blockIdx.x == 0 && threadIdx.x < kGroup) {
         double *row = R + threadIdx.x * kGroup;
         const double rd = row[d], rj = row[j];
         row[d] = __dsub_rn(__dmul_rn(c, rd), __dmul_rn(s, rj));
         row[j] = __dadd_rn(__dmul_rn(s, rd), __dmul_rn(c, rj));
     }
+    if (lead && trace) {
+        trace[3 * step] = d;
+        trace[3 * step + 1] = j;
+        trace[3 * step + 2] = a;
+    }
     double *bd = B + d * rows;
     double *bj = B + j * rows;
+    const int64_t lo = static_cast<int64_t>(blockIdx.x) * rows_per_block;
+    const int64_t hi = lo + rows_per_block < rows ? lo + rows_per_block : rows;
     double md = 0.0, mj = 0.0;
-    for (int64_t r = threadIdx.x; r < rows; r += kSelectThreads) {
+    for (int64_t r = lo + threadIdx.x; r < hi; r += kSelectThreads) {
         const double xd = bd[r], xj = bj[r];
         const double u = __dsub_rn(__dmul_rn(c, xd), __dmul_rn(s, xj));
         const double w = __dadd_rn(__dmul_rn(s, xd), __dmul_rn(c, xj));
@@ -390,16 +457,18 @@ __global__ void __launch_bounds__(kSelectThreads)
         if (au > md) md = au;
         if (aw > mj) mj = aw;
     }
-    md = block_max(md, red);
-    mj = block_max(mj, red);
+    md = block_max<kSelectThreads>(md, red);
+    mj = block_max<kSelectThreads>(mj, red);
     if (threadIdx.x == 0) {
-        st->colmax[d] = double_to_bits(md);
-        st->colmax[j] = double_to_bits(mj);
-        st->steps = step + 1;
-        if (trace) {
-            trace[3 * step] = d;
-            trace[3 * step + 1] = j;
-            trace[3 * step + 2] = a;
+        if (md > 0.0) atomicMax(&st->nm[0], double_to_bits(md));
+        if (mj > 0.0) atomicMax(&st->nm[1], double_to_bits(mj));
+        __threadfence();
+        if (atomicAdd(&st->ticket, 1u) == gridDim.x - 1) {
+            __threadfence();
+            st->colmax[d] = atomicExch(&st->nm[0], 0ull);
+            st->colmax[j] = atomicExch(&st->nm[1], 0ull);
+            st->ticket = 0u;
+            st->steps = step + 1;
         }
     }
 }
@@ -430,7 +499,7 @@ SearchLayout search_layout(int64_t rows, int64_t cols, int n_angle)
 {
     SearchLayout L{};
     L.cand = 512;
-    L.colmax_x = L.cand + align256(static_cast<int64_t>(kGroup) * 2 * n_angle * 8);
+    L.colmax_x = L.cand + align256(2 * static_cast<int64_t>(kGroup) * 2 * n_angle * 8);   // two tables
     L.block = L.colmax_x + align256(cols * 4);
     L.total = L.block + rows * kGroup * 8;
     return L;
@@ -453,7 +522,7 @@ cudaError_t launch_rotation_search(const SearchArgs &a, int num_sms, cudaStream_
     double *B = reinterpret_cast<double *>(ws + L.block);
     const int n_cand = kGroup * 2 * a.n_angle;
 
-    search_init_kernel<<<num_sms, 1024, 0, stream>>>(colmax_x, a.cols, st, cand, n_cand, a.R);
+    search_init_kernel<<<num_sms, 1024, 0, stream>>>(colmax_x, a.cols, st, cand, 2 * n_cand, a.R);
     const int64_t nvec = a.cols / 8;
     const int64_t gx = (nvec + kColmaxThreads - 1) / kColmaxThreads;
     int64_t gy = (static_cast<int64_t>(num_sms) * 4 + gx - 1) / gx;
@@ -462,19 +531,24 @@ cudaError_t launch_rotation_search(const SearchArgs &a, int num_sms, cudaStream_
     if (gy < 1) gy = 1;
     search_colmax_kernel<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)), kColmaxThreads, 0, stream>>>(
         static_cast<const uint4 *>(a.X), a.rows, a.cols, colmax_x);
-    search_pick_kernel<<<1, kSelectThreads, 0, stream>>>(colmax_x, a.lambda, a.cols / kGroup, st);
+    search_pick_kernel<<<1, kPickThreads, 0, stream>>>(colmax_x, a.lambda, a.cols / kGroup, st);
     int64_t gb = (a.rows + 7) / 8;
     if (gb > static_cast<int64_t>(num_sms) * 4) gb = static_cast<int64_t>(num_sms) * 4;
     search_gather_kernel<<<static_cast<unsigned>(gb), 256, 0, stream>>>(static_cast<const uint16_t *>(a.X), a.rows,
                                                                         a.cols, a.lambda, st, B);
     const unsigned chunks = static_cast<unsigned>((a.rows + kCandChunk - 1) / kCandChunk);
+    int64_t sel_blocks = (a.rows + 2 * kSelectThreads - 1) / (2 * kSelectThreads);
+    if (sel_blocks > 2 * static_cast<int64_t>(num_sms)) sel_blocks = 2 * static_cast<int64_t>(num_sms);
+    const int64_t rows_per_block = (a.rows + sel_blocks - 1) / sel_blocks;
     for (int step = 0; step < a.max_steps; ++step) {
-        search_cand_kernel<<<dim3(chunks, kGroup), kCandThreads, 0, stream>>>(B, a.rows, a.n_angle, st, cand);
-        search_select_kernel<<<1, kSelectThreads, 0, stream>>>(B, a.rows, a.n_angle, step, a.max_steps, st, cand,
-                                                               a.R, a.trace, a.linf);
+        unsigned long long *tab = cand + (step & 1) * n_cand;
+        unsigned long long *next = cand + ((step + 1) & 1) * n_cand;
+        search_cand_kernel<<<dim3(chunks, kGroup), kCandThreads, 0, stream>>>(B, a.rows, a.n_angle, st, tab);
+        search_select_kernel<<<static_cast<unsigned>(sel_blocks), kSelectThreads, 0, stream>>>(
+            B, a.rows, rows_per_block, a.n_angle, step, a.max_steps, st, tab, next, a.R, a.trace, a.linf);
     }
-    search_select_kernel<<<1, kSelectThreads, 0, stream>>>(B, a.rows, a.n_angle, a.max_steps, a.max_steps, st, cand,
-                                                           a.R, a.trace, a.linf);
+    search_select_kernel<<<1, kSelectThreads, 0, stream>>>(B, a.rows, a.rows, a.n_angle, a.max_steps, a.max_steps,
+                                                           st, cand, cand + n_cand, a.R, a.trace, a.linf);
     search_finish_kernel<<<1, kGroup * kGroup, 0, stream>>>(a.R, st, a.rhat, a.steps, a.group);
     return cudaGetLastError();
 }
