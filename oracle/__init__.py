@@ -61,6 +61,8 @@ def lib():
         L.mxq_oracle_quantize.argtypes = [P, I64, I64, P, P, P, P, P, P, I]
         L.mxq_oracle_quantize.restype = I
         L.mxq_oracle_smooth_rotate_quantize.argtypes = [P, I64, I64, P, P, P, P, P, P, P, P, P, I]
+        L.mxq_oracle_block_rotate_quantize.argtypes = [P, I64, I64, I, P, P, P, P, P, P, P, P, P, I]
+        L.mxq_oracle_block_rotate_quantize.restype = I
         L.mxq_oracle_smooth_rotate_quantize.restype = I
         L.mxq_oracle_dequantize.argtypes = [P, P, I64, I64, P, P, P, P, I]
         L.mxq_oracle_dequantize.restype = I
@@ -190,6 +192,31 @@ def smooth_rotate_quantize(x_bits: np.ndarray, rhat_bits: np.ndarray, lam: Optio
         _ptr(g("y")), _ptr(g("eflags")), _ptr(g("alt")), _ptr(g("gflags")), _ptr(g("alt_scales")), threads)
     if rc:
         raise ValueError("oracle: bad shape")
+    return out
+
+
+def block_rotate_quantize(x_bits: np.ndarray, r_bits: np.ndarray, lam: Optional[np.ndarray] = None,
+                          want_y: bool = False, flags: bool = False, threads: int = 1) -> dict:
+    """Rotation blocks of B = r_bits.shape[0] columns, MXFP4 groups of 32 (the §4.3 block-size variants)."""
+    x_bits = _c(x_bits, np.uint16)
+    r_bits = _c(r_bits, np.uint16)
+    blk = r_bits.shape[0]
+    assert r_bits.shape == (blk, blk)
+    rows, cols = x_bits.shape
+    G = cols // GROUP
+    lam32 = None if lam is None else _c(lam, np.float32)
+    out = {"codes": np.zeros((rows, cols // 2), np.uint8), "scales": np.zeros((rows, G), np.uint8)}
+    if want_y:
+        out["y"] = np.zeros((rows, cols), np.float64)
+    if flags:
+        out.update(eflags=np.zeros((rows, cols), np.uint8), alt=np.zeros((rows, cols), np.uint8),
+                   gflags=np.zeros((rows, G), np.uint8), alt_scales=np.zeros((rows, G), np.uint8))
+    g = out.get
+    rc = lib().mxq_oracle_block_rotate_quantize(
+        _ptr(x_bits), rows, cols, blk, _ptr(r_bits), _ptr(lam32), _ptr(out["codes"]), _ptr(out["scales"]),
+        _ptr(g("y")), _ptr(g("eflags")), _ptr(g("alt")), _ptr(g("gflags")), _ptr(g("alt_scales")), threads)
+    if rc:
+        raise ValueError("oracle: bad shape or block size")
     return out
 
 

@@ -305,6 +305,69 @@ int mxq_oracle_smooth_rotate_quantize(const uint16_t *X, int64_t rows, int64_t c
     return 0;
 }
 
+/* The rotation-block-size variant of the write-up's §4.3 ablation: blocks of
+ * B = 16, 32, 64 or 128 columns are rotated by one shared B x B matrix, and
+ * the MXFP4 groups stay at 32 columns.  For each row and each block of B
+ * columns:
+ *   1. x = the block's bf16 values in double, divided by Λ per channel;
+ *   2. y = x * R_B (R_B bf16 [B][B], row-major [k][n]);
+ *   3. every 32 consecutive columns of y (in the row) form one MXFP4 group,
+ *      quantised as in mxq_oracle_smooth_rotate_quantize.
+ * Outputs and flags have the layouts of mxq_oracle_smooth_rotate_quantize.
+ * cols must be a multiple of both B and 32. */
+int mxq_oracle_block_rotate_quantize(const uint16_t *X, int64_t rows, int64_t cols, int blk,
+                                     const uint16_t *Rb, const float *lam, uint8_t *codes,
+                                     uint8_t *scales, double *Y, uint8_t *eflags, uint8_t *alt,
+                                     uint8_t *gflags, uint8_t *alt_scales, int nthreads)
+{
+    if (rows < 0 || cols < 0 || cols % GROUP || blk < 1 || blk > 128 || cols % blk) return 1;
+    int64_t G = cols / GROUP;
+    double *R = (double *)malloc(sizeof(double) * (size_t)(blk * blk));
+    if (!R) return 1;
+    for (int i = 0; i < blk * blk; ++i) R[i] = bf16_to_double(Rb[i]);
+    int rc = 0;
+#pragma omp parallel num_threads(nthreads > 0 ? nthreads : 1)
+    {
+        double *yrow = (double *)malloc(sizeof(double) * (size_t)cols);
+        double *x = (double *)malloc(sizeof(double) * (size_t)blk);
+        if (!yrow || !x) {
+#pragma omp atomic write
+            rc = 1;
+        } else {
+#pragma omp for schedule(dynamic, 4)
+            for (int64_t r = 0; r < rows; ++r) {
+                /* steps 1-2, block by block */
+                for (int64_t b0 = 0; b0 < cols; b0 += blk) {
+                    for (int k = 0; k < blk; ++k) {
+                        x[k] = bf16_to_double(X[r * cols + b0 + k]);
+                        if (lam) x[k] = x[k] / (double)lam[b0 + k];
+                    }
+                    for (int n = 0; n < blk; ++n) {
+                        double acc = 0.0;
+                        for (int k = 0; k < blk; ++k) acc += x[k] * R[k * blk + n];
+                        yrow[b0 + n] = acc;
+                    }
+                }
+                if (Y) memcpy(Y + r * cols, yrow, sizeof(double) * (size_t)cols);
+                /* step 3: 32-column groups of the rotated row */
+                for (int64_t g = 0; g < G; ++g) {
+                    uint8_t c[GROUP];
+                    int64_t e0 = r * cols + g * GROUP;
+                    quantize_group(yrow + g * GROUP, c, scales + r * G + g, eflags ? eflags + e0 : NULL,
+                                   alt ? alt + e0 : NULL, gflags ? gflags + r * G + g : NULL,
+                                   alt_scales ? alt_scales + r * G + g : NULL);
+                    for (int i = 0; i < GROUP / 2; ++i)
+                        codes[e0 / 2 + i] = (uint8_t)(c[2 * i] | (c[2 * i + 1] << 4));
+                }
+            }
+        }
+        free(yrow);
+        free(x);
+    }
+    free(R);
+    return rc;
+}
+
 /* Dequantise: v = E2M1(code) * 2^(byte-127).  With R (bf16 [k][n]) the
  * rotation is undone, x_k = sum_n v_n R[k][n], and with lam the smoothing too,
  * x_k *= lam[k].  The exact double result is rounded once to bf16.  out_f64
