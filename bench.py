@@ -384,6 +384,16 @@ def run_extras(mxq, w, xs, rhat, outs, dev, stream, k=300):
         assert st == 0
     row("quant_error_per_group_and_mean", _timed(qerr, k, stream, dev), rows * cols * 2.0 + rows * (cols // 32) * 4.0,
         "per-group ||Q(y)-y||/||y|| (fp32 out) and its mean: reads X, writes 4 B per group")
+    # the rotation-block-size variants on the same X (no smoothing): B = 16, 64, 128
+    for blk in (16, 64, 128):
+        rblk = synth.rhat_tensor(synth.haar_orthogonal(300 + blk, n=blk)).to(dev)
+
+        def quant_blk(i, rblk=rblk):
+            c, s = outs[i & 1]
+            mxq.rotate_quantize_block(xs[i & 1], rblk, codes=c, scales=s, stream=stream)
+        row(f"rotate_quantize_block{blk}", _timed(quant_blk, k, stream, dev), algorithmic_bytes(rows, cols),
+            f"rotation blocks of {blk} columns, MXFP4 groups of 32 "
+            f"({'rotate_flat_kernel with diag(R16, R16)' if blk == 16 else 'rotate_block_kernel'})")
     # the offline rotation search on the same activations, smoothed: K = 128 steps, 64 angles per pair
     sws = torch.empty(mxq.lib().mxq_rotation_search_workspace_bytes(rows, cols, 32), dtype=torch.uint8, device=dev)
     found = {}

@@ -107,6 +107,31 @@ mxq_status mxq_smooth_rotate_f32(const void *X_bf16, int64_t rows, int64_t cols,
                                  float *out_f32, void *stream);
 
 /*
+ * Rotation-block-size variants (DuQuant++ write-up, §4.3: rotation blocks of
+ * B = 16, 32, 64 or 128 channels, B = 32 found best).  The MXFP4 groups stay
+ * at 32 columns.  Each row is cut into cols/B blocks; block x becomes
+ * y = (x / Λ) · R_B, with one shared B×B matrix R_B.  Every 32 consecutive
+ * columns of y are then quantised exactly as mxq_smooth_rotate_quantize does.
+ * B = 32 is mxq_smooth_rotate_quantize itself.  B = 16 runs on the same kernels
+ * with the block-diagonal diag(R_16, R_16).  B = 64 and 128 run on a kernel
+ * whose MMA is B wide and B deep.
+ *
+ *   block           16, 32, 64 or 128; cols must be a multiple of max(block, 32)
+ *   R_bf16          in   [block][block] bf16 row-major [k][n], 2-byte aligned
+ *   Lambda_or_null  in   [cols] fp32, for block 16 or 32 only (NULL for 64, 128)
+ *   other arguments, layouts and errors as mxq_smooth_rotate_quantize /
+ *   mxq_smooth_rotate_f32; a block width outside the list, cols not a multiple
+ *   of it, or Λ with block 64/128 return MXQ_ERR_INVALID_ARG.
+ */
+mxq_status mxq_rotate_quantize_block(const void *X_bf16, int64_t rows, int64_t cols, int block,
+                                     const void *R_bf16, const float *Lambda_or_null,
+                                     uint8_t *out_codes_u8_packed, uint8_t *out_scales_e8m0,
+                                     void *stream);
+mxq_status mxq_rotate_block_f32(const void *X_bf16, int64_t rows, int64_t cols, int block,
+                                const void *R_bf16, const float *Lambda_or_null, float *out_f32,
+                                void *stream);
+
+/*
  * MXFP4 dequantise: the fake-quant "simulator" of the write-up's §5.1 item 5.
  * Each value is v = E2M1(code) * 2^(byte - 127), with byte 0xFF giving NaN.
  *

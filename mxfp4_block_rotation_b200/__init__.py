@@ -60,6 +60,10 @@ def lib() -> ctypes.CDLL:
         L.mxq_smooth_rotate_quantize.restype = I
         L.mxq_smooth_rotate_f32.argtypes = [P, I64, I64, P, P, P, P]
         L.mxq_smooth_rotate_f32.restype = I
+        L.mxq_rotate_quantize_block.argtypes = [P, I64, I64, I, P, P, P, P, P]
+        L.mxq_rotate_quantize_block.restype = I
+        L.mxq_rotate_block_f32.argtypes = [P, I64, I64, I, P, P, P, P]
+        L.mxq_rotate_block_f32.restype = I
         L.mxq_dequantize.argtypes = [P, P, I64, I64, P, P, P, P]
         L.mxq_dequantize.restype = I
         L.mxq_selftest_bounded_wait.argtypes = [ctypes.c_uint32, P, P]
@@ -172,6 +176,54 @@ def smooth_rotate_f32(x: torch.Tensor, rhat: torch.Tensor, lam: Optional[torch.T
     st = lib().mxq_smooth_rotate_f32(_ptr(x), rows, cols, _ptr(rhat), _ptr(lam), _ptr(out),
                                      _stream(dev, stream))
     _check(st, "mxq_smooth_rotate_f32")
+    return out
+
+
+def _block_inputs(x, r, lam):
+    if x.dim() != 2:
+        raise ValueError("x must be 2-D [rows, cols]")
+    dev = x.device
+    if dev.type != "cuda":
+        raise ValueError("x must be a CUDA tensor (this library has no CPU path)")
+    _need(x, "x", torch.bfloat16, dev)
+    _need(r, "r", torch.bfloat16, dev)
+    if r.dim() != 2 or r.shape[0] != r.shape[1]:
+        raise ValueError("r must be square [block, block]")
+    if lam is not None:
+        _need(lam, "lam", torch.float32, dev)
+        if tuple(lam.shape) != (x.shape[1],):
+            raise ValueError("lam must be [cols]")
+    return dev, int(r.shape[0])
+
+
+def rotate_quantize_block(x: torch.Tensor, r: torch.Tensor, lam: Optional[torch.Tensor] = None, *,
+                          codes: Optional[torch.Tensor] = None, scales: Optional[torch.Tensor] = None,
+                          stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """MXFP4 of X · Λ⁻¹ rotated in blocks of B = r.shape[0] columns (16, 32, 64 or 128), 32-column groups."""
+    dev, blk = _block_inputs(x, r, lam)
+    rows, cols = x.shape
+    if codes is None:
+        codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+    if scales is None:
+        scales = torch.empty((rows, cols // 32), dtype=torch.uint8, device=dev)
+    _need(codes, "codes", torch.uint8, dev)
+    _need(scales, "scales", torch.uint8, dev)
+    st = lib().mxq_rotate_quantize_block(_ptr(x), rows, cols, blk, _ptr(r), _ptr(lam), _ptr(codes), _ptr(scales),
+                                         _stream(dev, stream))
+    _check(st, "mxq_rotate_quantize_block")
+    return codes, scales
+
+
+def rotate_block_f32(x: torch.Tensor, r: torch.Tensor, lam: Optional[torch.Tensor] = None, *,
+                     out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """X · Λ⁻¹ rotated in blocks of B = r.shape[0] columns, in fp32 [rows, cols]."""
+    dev, blk = _block_inputs(x, r, lam)
+    rows, cols = x.shape
+    if out is None:
+        out = torch.empty((rows, cols), dtype=torch.float32, device=dev)
+    _need(out, "out", torch.float32, dev)
+    st = lib().mxq_rotate_block_f32(_ptr(x), rows, cols, blk, _ptr(r), _ptr(lam), _ptr(out), _stream(dev, stream))
+    _check(st, "mxq_rotate_block_f32")
     return out
 
 

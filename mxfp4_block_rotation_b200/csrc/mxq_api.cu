@@ -185,6 +185,26 @@ mxq_status make_tmap_groups(CUtensorMap *map, const void *X, int64_t rows, int64
     return MXQ_OK;
 }
 
+// A bf16 [rows, cols] matrix viewed as [rows*cols/blk, blk]: one row per rotation block
+// (blk = 64 or 128), loaded in 128-byte K-atoms of 64 columns, 16384/blk rows per box
+// (32 KB of X per stage).
+mxq_status make_tmap_blocks(CUtensorMap *map, const void *X, int64_t rows, int64_t cols, int blk)
+{
+    const Driver &d = driver();
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(blk), static_cast<cuuint64_t>(rows) * static_cast<cuuint64_t>(cols / blk)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(blk) * 2};
+    cuuint32_t box[2] = {64, static_cast<cuuint32_t>(16384 / blk)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = d.encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(X), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        note_cu(r, "cuTensorMapEncodeTiled(blocks)");
+        return MXQ_ERR_CUDA;
+    }
+    return MXQ_OK;
+}
+
 mxq_status make_tmap_x(CUtensorMap *map, const void *X, int64_t rows, int64_t cols)
 {
     const Driver &d = driver();
@@ -203,12 +223,16 @@ mxq_status make_tmap_x(CUtensorMap *map, const void *X, int64_t rows, int64_t co
 }
 
 // Common front half of the two rotate entry points.
+// blk: the rotation block width (32 for the main path; 16, 64 or 128 for the variants).
 mxq_status rotate_common(const void *X, int64_t rows, int64_t cols, const void *R, const float *lam,
                          void *out0, uint64_t out0_bytes, uint64_t out0_align, void *out1,
-                         uint64_t out1_bytes, mxq::RotOut mode, void *stream)
+                         uint64_t out1_bytes, mxq::RotOut mode, void *stream, int blk = 32)
 {
     mxq_status st = check_shape(rows, cols);
     if (st != MXQ_OK) return st;
+    if (blk != 16 && blk != 32 && blk != 64 && blk != 128) return bad("block must be 16, 32, 64 or 128");
+    if (cols % blk) return bad("cols must be a multiple of the block width");
+    if (lam && blk > 32) return bad("Lambda is supported with blocks of 16 or 32 columns only");
     if (rows == 0 || cols == 0) return MXQ_OK;   // nothing is read or written
     if (!X || !R || !out0 || (mode == mxq::RotOut::Quant && !out1)) return bad("null pointer");
     if (!aligned(X, 16)) return bad("X must be 16-byte aligned");
@@ -216,8 +240,9 @@ mxq_status rotate_common(const void *X, int64_t rows, int64_t cols, const void *
     if (lam && !aligned(lam, 4)) return bad("Lambda must be 4-byte aligned");
     if (!aligned(out0, out0_align)) return bad("output must be 16-byte aligned");
     const uint64_t nx = static_cast<uint64_t>(rows) * cols * 2, nl = lam ? static_cast<uint64_t>(cols) * 4 : 0;
+    const uint64_t nr = static_cast<uint64_t>(blk) * blk * 2;
     const void *ins[3] = {X, R, lam};
-    const uint64_t nins[3] = {nx, 32 * 32 * 2, nl};
+    const uint64_t nins[3] = {nx, nr, nl};
     for (int i = 0; i < 3; ++i) {
         if (overlaps(out0, out0_bytes, ins[i], nins[i]) || (out1 && overlaps(out1, out1_bytes, ins[i], nins[i])))
             return bad("an output overlaps an input");
@@ -227,14 +252,16 @@ mxq_status rotate_common(const void *X, int64_t rows, int64_t cols, const void *
     int dev = 0, sms = 0;
     if ((st = current_device(&dev, &sms)) != MXQ_OK) return st;
     if ((st = check_buffer(X, nx, dev)) != MXQ_OK) return st;
-    if ((st = check_buffer(R, 32 * 32 * 2, dev)) != MXQ_OK) return st;
+    if ((st = check_buffer(R, nr, dev)) != MXQ_OK) return st;
     if (lam && (st = check_buffer(lam, nl, dev)) != MXQ_OK) return st;
     if ((st = check_buffer(out0, out0_bytes, dev)) != MXQ_OK) return st;
     if (out1 && (st = check_buffer(out1, out1_bytes, dev)) != MXQ_OK) return st;
 
-    alignas(64) CUtensorMap map_a;   // X as [n_groups, 32] (no smoothing) or [rows, cols]
+    alignas(64) CUtensorMap map_a;   // X as [n_groups, 32] (no smoothing), [n_blocks, blk] or [rows, cols]
     alignas(64) CUtensorMap map_c;   // the packed codes (smoothing, quantise mode)
-    if (lam == nullptr) {
+    if (blk > 32) {
+        if ((st = make_tmap_blocks(&map_a, X, rows, cols, blk)) != MXQ_OK) return st;
+    } else if (lam == nullptr) {
         if ((st = make_tmap_groups(&map_a, X, rows, cols)) != MXQ_OK) return st;
     } else {
         if ((st = make_tmap_x(&map_a, X, rows, cols)) != MXQ_OK) return st;
@@ -246,6 +273,7 @@ mxq_status rotate_common(const void *X, int64_t rows, int64_t cols, const void *
     }
     mxq::RotArgs args{};
     args.rhat = static_cast<const uint16_t *>(R);
+    args.rblk = blk == 16 ? 16 : 32;
     args.lambda = lam;
     args.rows = rows;
     args.cols = cols;
@@ -255,9 +283,10 @@ mxq_status rotate_common(const void *X, int64_t rows, int64_t cols, const void *
     } else {
         args.y = static_cast<float *>(out0);
     }
-    cudaError_t e = lam == nullptr
-                        ? mxq::launch_rotate_flat(map_a, args, mode, sms, static_cast<cudaStream_t>(stream))
-                        : mxq::launch_rotate_cols(map_a, map_c, args, mode, sms, static_cast<cudaStream_t>(stream));
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = blk > 32           ? mxq::launch_rotate_block(map_a, args, blk, mode, sms, s)
+                    : lam == nullptr ? mxq::launch_rotate_flat(map_a, args, mode, sms, s)
+                                     : mxq::launch_rotate_cols(map_a, map_c, args, mode, sms, s);
     if (e != cudaSuccess) {
         note_cuda(e, "launch rotate kernel");
         return MXQ_ERR_CUDA;
@@ -289,6 +318,24 @@ mxq_status mxq_smooth_rotate_f32(const void *X_bf16, int64_t rows, int64_t cols,
     const uint64_t ny = rows > 0 && cols > 0 ? static_cast<uint64_t>(rows) * cols * 4 : 0;
     return rotate_common(X_bf16, rows, cols, Rhat_bf16, Lambda_or_null, out_f32, ny, 16, nullptr, 0,
                          mxq::RotOut::F32, stream);
+}
+
+mxq_status mxq_rotate_quantize_block(const void *X_bf16, int64_t rows, int64_t cols, int block, const void *R_bf16,
+                                     const float *Lambda_or_null, uint8_t *out_codes_u8_packed,
+                                     uint8_t *out_scales_e8m0, void *stream)
+{
+    const uint64_t nc = rows > 0 && cols > 0 ? static_cast<uint64_t>(rows) * cols / 2 : 0;
+    const uint64_t ns = rows > 0 && cols > 0 ? static_cast<uint64_t>(rows) * (cols / 32) : 0;
+    return rotate_common(X_bf16, rows, cols, R_bf16, Lambda_or_null, out_codes_u8_packed, nc, 16, out_scales_e8m0,
+                         ns, mxq::RotOut::Quant, stream, block);
+}
+
+mxq_status mxq_rotate_block_f32(const void *X_bf16, int64_t rows, int64_t cols, int block, const void *R_bf16,
+                                const float *Lambda_or_null, float *out_f32, void *stream)
+{
+    const uint64_t ny = rows > 0 && cols > 0 ? static_cast<uint64_t>(rows) * cols * 4 : 0;
+    return rotate_common(X_bf16, rows, cols, R_bf16, Lambda_or_null, out_f32, ny, 16, nullptr, 0,
+                         mxq::RotOut::F32, stream, block);
 }
 
 mxq_status mxq_dequantize(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t cols,

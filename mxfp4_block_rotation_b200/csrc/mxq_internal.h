@@ -19,7 +19,8 @@ enum : unsigned int {
 enum class RotOut { Quant, F32, Err };
 
 struct RotArgs {
-    const uint16_t *rhat;      // bf16 [32][32], row-major [k][n]
+    const uint16_t *rhat;      // bf16 [32][32], row-major [k][n]; [16][16] when rblk == 16
+    int rblk;                  // 16: R^ is diag(R16, R16) built from a 16x16 input; otherwise 32
     const float *lambda;       // fp32 [cols] or nullptr
     uint8_t *codes;            // [rows, cols/2]   (Quant)
     uint8_t *scales;           // [rows, cols/32]  (Quant)
@@ -40,6 +41,12 @@ cudaError_t launch_rotate_flat(const CUtensorMap &tmap_groups, const RotArgs &ar
 // codes as [rows, cols/2] uint8 (box {64, 128}, 64-byte swizzle; Quant mode only).
 cudaError_t launch_rotate_cols(const CUtensorMap &tmap_x, const CUtensorMap &tmap_codes, const RotArgs &args,
                                RotOut mode, int num_sms, cudaStream_t stream);
+
+// Rotate -> MXFP4 with rotation blocks of blk = 64 or 128 columns (no smoothing).
+// `tmap_blocks` views X as [rows*cols/blk, blk] bf16 (box {64, 16384/blk}, 128-byte
+// swizzle); args.rhat is bf16 [blk][blk].
+cudaError_t launch_rotate_block(const CUtensorMap &tmap_blocks, const RotArgs &args, int blk, RotOut mode,
+                                int num_sms, cudaStream_t stream);
 
 // Number of per-warp partial sums the Err mode writes (one double each).
 int64_t rotate_flat_partials(int64_t rows, int64_t cols);

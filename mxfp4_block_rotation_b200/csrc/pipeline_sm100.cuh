@@ -61,6 +61,14 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
     }
 }
 
+// Element [k][n] of the 32x32 rotation, as bf16 bits: the matrix itself, or for
+// rotation blocks of 16 columns the block-diagonal diag(R16, R16) of a 16x16 input.
+__device__ __forceinline__ uint16_t rhat_at(const RotArgs &a, int k, int n)
+{
+    if (a.rblk == 16) return ((k ^ n) & 16) ? static_cast<uint16_t>(0) : a.rhat[(k & 15) * 16 + (n & 15)];
+    return a.rhat[k * 32 + n];
+}
+
 // Byte offset of 16-byte chunk c of row r inside a 128-byte-swizzled atom.
 __device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t c)
 {

@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(kColThreads, 1)
         constexpr int kB = kColBuildWarps * 32;
         for (int i = bt; i < 32 * 32; i += kB) {
             const int k = i >> 5, n = i & 31;
-            rt[n * 32 + k] = __bfloat162float(__ushort_as_bfloat16(args.rhat[i]));
+            rt[n * 32 + k] = __bfloat162float(__ushort_as_bfloat16(rhat_at(args, k, n)));
         }
         ptx::named_bar_sync(3, kB);
         int built0 = -1, built1 = -1;   // column tile whose B_g each slot holds

@@ -108,8 +108,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int k = c * 8 + 2 * e;
-                w[e] = static_cast<uint32_t>(args.rhat[k * 32 + n]) |
-                       (static_cast<uint32_t>(args.rhat[(k + 1) * 32 + n]) << 16);
+                w[e] = static_cast<uint32_t>(rhat_at(args, k, n)) |
+                       (static_cast<uint32_t>(rhat_at(args, k + 1, n)) << 16);
             }
             *reinterpret_cast<uint4 *>(bmat + sw128(n, c)) = make_uint4(w[0], w[1], w[2], w[3]);
         }

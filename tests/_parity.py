@@ -18,10 +18,14 @@ import numpy as np
 import oracle
 
 
-def check_quant(x_bits, rhat_bits, lam, gpu_codes, gpu_scales, threads=None, exact=False):
-    """Compare GPU codes/scales for the rows of x_bits; returns a dict of counts (raises on failure)."""
+def check_quant(x_bits, rhat_bits, lam, gpu_codes, gpu_scales, threads=None, exact=False, ref=None):
+    """Compare GPU codes/scales for the rows of x_bits; returns a dict of counts (raises on failure).
+
+    `ref` is the oracle's output (with y and flags) when the caller has it already, e.g. from
+    another oracle entry point; otherwise the main path's oracle is run here."""
     threads = threads or oracle.default_threads()
-    ref = oracle.smooth_rotate_quantize(x_bits, rhat_bits, lam, want_y=True, flags=True, threads=threads)
+    if ref is None:
+        ref = oracle.smooth_rotate_quantize(x_bits, rhat_bits, lam, want_y=True, flags=True, threads=threads)
     rows, cols = x_bits.shape
     G = cols // 32
     gpu_codes = np.asarray(gpu_codes, np.uint8)

@@ -121,3 +121,22 @@ def test_rotation_search_rejects_bad_arguments(L):
     assert _search(L, a, 4, 64, None, 8, 32, a + 64, ws=ws) == INVALID         # R overlaps X
     assert _search(L, a, 4, 64, None, 8, 32, a * 3, linf=a * 3 + 8192 - 8, ws=ws) == INVALID  # linf overlaps R
     assert L.mxq_last_cuda_error().startswith(b"invalid argument")
+
+
+def test_block_variant_rejects_bad_arguments(L):
+    a = 0x100000
+
+    def q(rows, cols, blk, lam=None, codes=a * 2, x=a):
+        return L.mxq_rotate_quantize_block(P(x), rows, cols, blk, P(a * 5), P(lam), P(codes), P(a * 3), None)
+
+    assert q(4, 128, 48) == INVALID                     # not a supported block width
+    assert q(4, 128, 256) == INVALID
+    assert q(4, 96, 64) == INVALID                      # cols not a multiple of the block
+    assert q(4, 192, 128) == INVALID
+    assert q(4, 128, 64, lam=a * 7) == INVALID          # Λ with a block wider than a group
+    assert q(4, 128, 128, lam=a * 7) == INVALID
+    assert q(4, 128, 64, x=a + 8) == INVALID            # X not 16-B aligned
+    assert q(4, 128, 64, codes=a + 16) == INVALID       # codes overlap X
+    assert L.mxq_last_cuda_error().startswith(b"invalid argument")
+    assert q(0, 128, 128) == 0 and q(4, 0, 64) == 0     # empty: nothing to do
+    assert L.mxq_rotate_block_f32(P(a), 4, 96, 64, P(a * 5), None, P(a * 2), None) == INVALID
