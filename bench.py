@@ -285,7 +285,8 @@ def run_mine(args):
 
     # end to end through the public API: pinned host X -> device -> kernel -> codes/scales back to host
     e2e = None if args.no_e2e else run_e2e(mxq, w, rhat, dev, stream, args, dist)
-    extras = None if (args.no_extras or world > 1) else run_extras(mxq, w, xs, rhat, outs, dev, stream)
+    extras = None if (args.no_extras or world > 1) else run_extras(mxq, w, xs, rhat, outs, dev, stream,
+                                                                    k=max(1, args.extras_steps))
 
     if rank == 0:
         peak, peak_kind = hbm_peak()
@@ -400,7 +401,7 @@ def run_extras(mxq, w, xs, rhat, outs, dev, stream, k=300):
 
     def search(i):
         found["out"] = mxq.rotation_search(xs[i & 1], lam, max_steps=128, n_angle=32, workspace=sws, stream=stream)
-    ms = _timed(search, 10, stream, dev)
+    ms = _timed(search, max(1, min(10, k)), stream, dev)
     res["rotation_search_K128"] = {
         "what": "greedy Givens search for R^ on X / Lambda (worst group by column maxima, 128 steps, 64 angles)",
         "ms": ms, "steps": int(found["out"]["steps"]), "launches": 2 * 128 + 6,
@@ -456,6 +457,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg (profiling runs)")
     ap.add_argument("--no-extras", action="store_true", help="skip timing the smoothing and dequantize rows")
+    ap.add_argument("--extras-steps", type=int, default=300,
+                    help="timed launches per extra row (the search row times min(10, this) runs)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
