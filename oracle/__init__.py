@@ -61,6 +61,10 @@ def lib():
         L.mxq_oracle_quantize.argtypes = [P, I64, I64, P, P, P, P, P, P, I]
         L.mxq_oracle_quantize.restype = I
         L.mxq_oracle_smooth_rotate_quantize.argtypes = [P, I64, I64, P, P, P, P, P, P, P, P, P, I]
+        L.mxq_oracle_weight_rotate_quantize.argtypes = [P, I64, I64, P, P, P, P, P, P, P, P, P, I]
+        L.mxq_oracle_weight_rotate_quantize.restype = I
+        L.mxq_oracle_mxfp4_gemm.argtypes = [P, P, P, P, I64, I64, I64, P, I]
+        L.mxq_oracle_mxfp4_gemm.restype = I
         L.mxq_oracle_block_rotate_quantize.argtypes = [P, I64, I64, I, P, P, P, P, P, P, P, P, P, I]
         L.mxq_oracle_block_rotate_quantize.restype = I
         L.mxq_oracle_smooth_rotate_quantize.restype = I
@@ -193,6 +197,44 @@ def smooth_rotate_quantize(x_bits: np.ndarray, rhat_bits: np.ndarray, lam: Optio
     if rc:
         raise ValueError("oracle: bad shape")
     return out
+
+
+def weight_rotate_quantize(wt_bits: np.ndarray, rhat_bits: np.ndarray, lam: Optional[np.ndarray] = None,
+                           want_y: bool = False, flags: bool = False, threads: int = 1) -> dict:
+    """MXFP4 of the absorbed weights: each row of Wt = W^T times Λ, then R̂ per group (§3.3)."""
+    wt_bits = _c(wt_bits, np.uint16)
+    rhat_bits = _c(rhat_bits, np.uint16)
+    rows, cols = wt_bits.shape
+    G = cols // GROUP
+    lam32 = None if lam is None else _c(lam, np.float32)
+    out = {"codes": np.zeros((rows, cols // 2), np.uint8), "scales": np.zeros((rows, G), np.uint8)}
+    if want_y:
+        out["y"] = np.zeros((rows, cols), np.float64)
+    if flags:
+        out.update(eflags=np.zeros((rows, cols), np.uint8), alt=np.zeros((rows, cols), np.uint8),
+                   gflags=np.zeros((rows, G), np.uint8), alt_scales=np.zeros((rows, G), np.uint8))
+    g = out.get
+    rc = lib().mxq_oracle_weight_rotate_quantize(
+        _ptr(wt_bits), rows, cols, _ptr(rhat_bits), _ptr(lam32), _ptr(out["codes"]), _ptr(out["scales"]),
+        _ptr(g("y")), _ptr(g("eflags")), _ptr(g("alt")), _ptr(g("gflags")), _ptr(g("alt_scales")), threads)
+    if rc:
+        raise ValueError("oracle: bad shape")
+    return out
+
+
+def mxfp4_gemm(a_codes: np.ndarray, a_scales: np.ndarray, b_codes: np.ndarray, b_scales: np.ndarray,
+               threads: int = 1) -> np.ndarray:
+    """Y[m, n] = sum_k deq(A)[m, k] deq(B)[n, k] in double (both operands K-major MXFP4)."""
+    a_codes, a_scales = _c(a_codes, np.uint8), _c(a_scales, np.uint8)
+    b_codes, b_scales = _c(b_codes, np.uint8), _c(b_scales, np.uint8)
+    M, K = a_codes.shape[0], a_codes.shape[1] * 2
+    N = b_codes.shape[0]
+    assert b_codes.shape[1] * 2 == K and a_scales.shape == (M, K // GROUP) and b_scales.shape == (N, K // GROUP)
+    y = np.zeros((M, N), np.float64)
+    if lib().mxq_oracle_mxfp4_gemm(_ptr(a_codes), _ptr(a_scales), _ptr(b_codes), _ptr(b_scales), M, N, K, _ptr(y),
+                                   threads):
+        raise ValueError("oracle mxfp4_gemm: bad shape")
+    return y
 
 
 def block_rotate_quantize(x_bits: np.ndarray, r_bits: np.ndarray, lam: Optional[np.ndarray] = None,

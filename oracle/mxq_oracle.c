@@ -266,11 +266,13 @@ int mxq_oracle_quantize(const double *Y, int64_t rows, int64_t cols, uint8_t *co
 
 /* The whole path from bf16 inputs, one row at a time (no full-size double
  * buffers): X bf16 [rows, cols], R bf16 [32][32] row-major [k][n], lam fp32
- * [cols] or NULL.  Y (double [rows, cols]) and the flag outputs may be NULL. */
-int mxq_oracle_smooth_rotate_quantize(const uint16_t *X, int64_t rows, int64_t cols,
-                                      const uint16_t *Rb, const float *lam, uint8_t *codes,
-                                      uint8_t *scales, double *Y, uint8_t *eflags, uint8_t *alt,
-                                      uint8_t *gflags, uint8_t *alt_scales, int nthreads)
+ * [cols] or NULL.  Y (double [rows, cols]) and the flag outputs may be NULL.
+ * lam_mul = 0 divides by lam (the activations, X·Λ⁻¹); 1 multiplies (the
+ * weights' side of §3.3's absorption, Wᵀ·Λ). */
+static int rotate_quantize_rows(const uint16_t *X, int64_t rows, int64_t cols, const uint16_t *Rb,
+                                const float *lam, int lam_mul, uint8_t *codes, uint8_t *scales,
+                                double *Y, uint8_t *eflags, uint8_t *alt, uint8_t *gflags,
+                                uint8_t *alt_scales, int nthreads)
 {
     if (rows < 0 || cols < 0 || cols % GROUP) return 1;
     int64_t G = cols / GROUP;
@@ -282,10 +284,11 @@ int mxq_oracle_smooth_rotate_quantize(const uint16_t *X, int64_t rows, int64_t c
             double x[GROUP], y[GROUP];
             uint8_t c[GROUP];
             int64_t e0 = r * cols + g * GROUP;
-            /* step 1-2: exact bf16 -> double, then the per-channel division */
+            /* step 1-2: exact bf16 -> double, then the per-channel division
+             * (or, for weights, multiplication) */
             for (int k = 0; k < GROUP; ++k) {
                 x[k] = bf16_to_double(X[e0 + k]);
-                if (lam) x[k] = x[k] / (double)lam[g * GROUP + k];
+                if (lam) x[k] = lam_mul ? x[k] * (double)lam[g * GROUP + k] : x[k] / (double)lam[g * GROUP + k];
             }
             /* step 3: y = x * R^ */
             for (int n = 0; n < GROUP; ++n) {
@@ -302,6 +305,68 @@ int mxq_oracle_smooth_rotate_quantize(const uint16_t *X, int64_t rows, int64_t c
                 codes[e0 / 2 + i] = (uint8_t)(c[2 * i] | (c[2 * i + 1] << 4));
         }
     }
+    return 0;
+}
+
+int mxq_oracle_smooth_rotate_quantize(const uint16_t *X, int64_t rows, int64_t cols,
+                                      const uint16_t *Rb, const float *lam, uint8_t *codes,
+                                      uint8_t *scales, double *Y, uint8_t *eflags, uint8_t *alt,
+                                      uint8_t *gflags, uint8_t *alt_scales, int nthreads)
+{
+    return rotate_quantize_rows(X, rows, cols, Rb, lam, 0, codes, scales, Y, eflags, alt, gflags,
+                                alt_scales, nthreads);
+}
+
+/* The weights' side of the write-up's §3.3 (Ŵ = R̂ᵀ·Λ·W, absorbed offline):
+ * with W stored transposed, Wt = Wᵀ [n_out, k_in], each row of Ŵᵀ = (Wt row · Λ)
+ * · R̂ per 32-column group, then MXFP4 along k_in like the activations. */
+int mxq_oracle_weight_rotate_quantize(const uint16_t *Wt, int64_t rows, int64_t cols,
+                                      const uint16_t *Rb, const float *lam, uint8_t *codes,
+                                      uint8_t *scales, double *Y, uint8_t *eflags, uint8_t *alt,
+                                      uint8_t *gflags, uint8_t *alt_scales, int nthreads)
+{
+    return rotate_quantize_rows(Wt, rows, cols, Rb, lam, 1, codes, scales, Y, eflags, alt, gflags,
+                                alt_scales, nthreads);
+}
+
+/* The consumer GEMM on MXFP4 operands (the write-up's §3.3 inference step on
+ * Blackwell's native MXFP4 tensor cores, §1/§5.4): both operands K-major, codes
+ * packed two per byte (even k in the low nibble), one E8M0 scale per 32 k.
+ *   Y[m][n] = sum_k deq(A)[m][k] * deq(B)[n][k],  deq = E2M1 value * 2^(byte - 127)
+ * in double, k ascending.  A: codes [M, K/2], scales [M, K/32]; B: codes [N, K/2],
+ * scales [N, K/32]; Y: double [M, N].  A 0xFF scale makes its products NaN. */
+int mxq_oracle_mxfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, const uint8_t *b_codes,
+                          const uint8_t *b_scales, int64_t M, int64_t N, int64_t K, double *Y,
+                          int nthreads)
+{
+    if (M < 0 || N < 0 || K < 0 || K % GROUP) return 1;
+    int64_t G = K / GROUP;
+    double *bd = (double *)malloc(sizeof(double) * (size_t)(N * K > 0 ? N * K : 1));
+    if (!bd) return 1;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) {
+            int code = (b_codes[n * (K / 2) + k / 2] >> (4 * (k & 1))) & 0xF;
+            bd[n * K + k] = mxq_oracle_e2m1_value(code) * mxq_oracle_e8m0_value(b_scales[n * G + k / GROUP]);
+        }
+#pragma omp parallel num_threads(nthreads > 0 ? nthreads : 1)
+    {
+        double *ad = (double *)malloc(sizeof(double) * (size_t)(K > 0 ? K : 1));
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t m = 0; m < M; ++m) {
+            if (!ad) continue;
+            for (int64_t k = 0; k < K; ++k) {
+                int code = (a_codes[m * (K / 2) + k / 2] >> (4 * (k & 1))) & 0xF;
+                ad[k] = mxq_oracle_e2m1_value(code) * mxq_oracle_e8m0_value(a_scales[m * G + k / GROUP]);
+            }
+            for (int64_t n = 0; n < N; ++n) {
+                double acc = 0.0;
+                for (int64_t k = 0; k < K; ++k) acc += ad[k] * bd[n * K + k];
+                Y[m * N + n] = acc;
+            }
+        }
+        free(ad);
+    }
+    free(bd);
     return 0;
 }
 
