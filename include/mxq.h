@@ -86,8 +86,8 @@ typedef enum {
  *   stream              in   cudaStream_t
  *
  * The rotation runs on the tensor cores.  X is the exact bf16 A operand and
- * R^ (or, with Lambda, diag(1/Lambda)·R^ split into a bf16 high part and a
- * bf16 low part) is the B operand, with fp32 accumulation.  The scale and the
+ * R^ (or, with Lambda, diag(1/Lambda)·R^ split into three bf16 parts: high,
+ * middle and low) is the B operand, with fp32 accumulation.  The scale and the
  * codes are then decided on those fp32 values.
  */
 mxq_status mxq_smooth_rotate_quantize(const void *X_bf16, int64_t rows, int64_t cols,
@@ -105,6 +105,58 @@ mxq_status mxq_smooth_rotate_quantize(const void *X_bf16, int64_t rows, int64_t 
 mxq_status mxq_smooth_rotate_f32(const void *X_bf16, int64_t rows, int64_t cols,
                                  const void *Rhat_bf16, const float *Lambda_or_null,
                                  float *out_f32, void *stream);
+
+/*
+ * The weights' side of the absorption (DuQuant++ write-up, §3.3: Ŵ = R̂ᵀ·Λ·W,
+ * done offline so that X̂·Ŵ = X·W).  With W stored transposed, Wt = Wᵀ
+ * [rows = n_out, cols = k_in] bf16, each row becomes (row · Λ) · R̂ per
+ * 32-column group: the same computation as mxq_smooth_rotate_quantize with Λ
+ * multiplying instead of dividing.  The result is quantised to MXFP4 along
+ * k_in, in the layout mxq_mxfp4_gemm takes as its B operand.
+ *   arguments, layouts and errors as mxq_smooth_rotate_quantize (Λ may be NULL:
+ *   then it is identical to mxq_smooth_rotate_quantize without Λ).
+ */
+mxq_status mxq_weight_rotate_quantize(const void *Wt_bf16, int64_t rows, int64_t cols,
+                                      const void *Rhat_bf16, const float *Lambda_or_null,
+                                      uint8_t *out_codes_u8_packed, uint8_t *out_scales_e8m0,
+                                      void *stream);
+
+/*
+ * Row-major E8M0 scales [rows, K/32] (the quantisers' layout) -> the layout
+ * Blackwell's block-scaled MMA reads scale factors in.  The output is 512-byte
+ * atoms, one per 128 rows × 4 k-blocks, ordered by row block and then k-block.
+ * Inside an atom, the scale of row r (0..127) and k-block j (0..3) is byte
+ * 16·(r % 32) + 4·(r / 32) + j.  Rows and k-blocks past the matrix are 0.  A
+ * lane of the MMA's scale loader thus finds its four 32-bit scale words in one
+ * contiguous 16-byte line.  This is layout work only: the same bytes, moved.
+ *   scales  in   [rows, K/32] bytes;  K a multiple of 32
+ *   out     out  mxq_scales_mma_bytes(rows, K) bytes, 16-byte aligned
+ */
+size_t mxq_scales_mma_bytes(int64_t rows, int64_t K);
+mxq_status mxq_scales_to_mma_layout(const uint8_t *scales, int64_t rows, int64_t K, uint8_t *out, void *stream);
+
+/*
+ * The MXFP4 × MXFP4 consumer GEMM on the block-scaled tensor cores (the
+ * write-up's §3.3 inference step; §1 and §5.4 name Blackwell's native MXFP4):
+ *   Y[m][n] = Σ_k deq(A)[m][k] · deq(B)[n][k],  deq = E2M1 code · 2^(E8M0 byte − 127)
+ * A is the activations (mxq_smooth_rotate_quantize's output), B the absorbed
+ * weights (mxq_weight_rotate_quantize's output), both K-major: codes two per
+ * byte (even k in the low nibble), one scale per 32 k, the scales converted by
+ * mxq_scales_to_mma_layout.  The tensor cores accumulate in fp32.
+ *   a_codes       in   [M, K/2] bytes, 16-byte aligned
+ *   a_scales_mma  in   mxq_scales_mma_bytes(M, K) bytes, 16-byte aligned
+ *   b_codes       in   [N, K/2] bytes, 16-byte aligned
+ *   b_scales_mma  in   mxq_scales_mma_bytes(N, K) bytes, 16-byte aligned
+ *   K                  a multiple of 32; M, N, K < 2^31
+ *   out           out  [M, N] row-major, fp32 (out_bf16 = 0) or bf16 rounded to
+ *                      nearest even (out_bf16 = 1), 16-byte aligned; K = 0 writes zeros
+ *   A 0xFF scale byte (NaN) makes the products it scales NaN.
+ * Errors: MXQ_ERR_INVALID_ARG for a bad size or alignment, a host pointer or an
+ * output that overlaps an input.
+ */
+mxq_status mxq_mxfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales_mma, const uint8_t *b_codes,
+                          const uint8_t *b_scales_mma, int64_t M, int64_t N, int64_t K, void *out,
+                          int out_bf16, void *stream);
 
 /*
  * Rotation-block-size variants (DuQuant++ write-up, §4.3: rotation blocks of

@@ -64,6 +64,14 @@ def lib() -> ctypes.CDLL:
         L.mxq_rotate_quantize_block.restype = I
         L.mxq_rotate_block_f32.argtypes = [P, I64, I64, I, P, P, P, P]
         L.mxq_rotate_block_f32.restype = I
+        L.mxq_weight_rotate_quantize.argtypes = [P, I64, I64, P, P, P, P, P]
+        L.mxq_weight_rotate_quantize.restype = I
+        L.mxq_mxfp4_gemm.argtypes = [P, P, P, P, I64, I64, I64, P, I, P]
+        L.mxq_scales_mma_bytes.argtypes = [I64, I64]
+        L.mxq_scales_mma_bytes.restype = ctypes.c_size_t
+        L.mxq_scales_to_mma_layout.argtypes = [P, I64, I64, P, P]
+        L.mxq_scales_to_mma_layout.restype = I
+        L.mxq_mxfp4_gemm.restype = I
         L.mxq_dequantize.argtypes = [P, P, I64, I64, P, P, P, P]
         L.mxq_dequantize.restype = I
         L.mxq_selftest_bounded_wait.argtypes = [ctypes.c_uint32, P, P]
@@ -176,6 +184,79 @@ def smooth_rotate_f32(x: torch.Tensor, rhat: torch.Tensor, lam: Optional[torch.T
     st = lib().mxq_smooth_rotate_f32(_ptr(x), rows, cols, _ptr(rhat), _ptr(lam), _ptr(out),
                                      _stream(dev, stream))
     _check(st, "mxq_smooth_rotate_f32")
+    return out
+
+
+def weight_rotate_quantize(wt: torch.Tensor, rhat: torch.Tensor, lam: Optional[torch.Tensor] = None, *,
+                           codes: Optional[torch.Tensor] = None, scales: Optional[torch.Tensor] = None,
+                           stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """MXFP4(Wᵀ · Λ · R̂): the absorbed weights, W given transposed as wt [n_out, k_in] bf16."""
+    dev = _inputs(wt, rhat, lam)
+    rows, cols = wt.shape
+    if codes is None:
+        codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+    if scales is None:
+        scales = torch.empty((rows, cols // 32), dtype=torch.uint8, device=dev)
+    _need(codes, "codes", torch.uint8, dev)
+    _need(scales, "scales", torch.uint8, dev)
+    st = lib().mxq_weight_rotate_quantize(_ptr(wt), rows, cols, _ptr(rhat), _ptr(lam), _ptr(codes), _ptr(scales),
+                                          _stream(dev, stream))
+    _check(st, "mxq_weight_rotate_quantize")
+    return codes, scales
+
+
+def scales_to_mma_layout(scales: torch.Tensor, *, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Row-major E8M0 scales [rows, K/32] -> the block-scaled MMA's 512-byte atoms (flat uint8)."""
+    dev = scales.device
+    if dev.type != "cuda":
+        raise ValueError("scales must be a CUDA tensor (this library has no CPU path)")
+    _need(scales, "scales", torch.uint8, dev)
+    rows, G = scales.shape
+    n = int(lib().mxq_scales_mma_bytes(rows, G * 32))
+    if out is None:
+        out = torch.empty(n, dtype=torch.uint8, device=dev)
+    _need(out, "out", torch.uint8, dev)
+    if out.numel() < n:
+        raise ValueError(f"out needs {n} bytes")
+    st = lib().mxq_scales_to_mma_layout(_ptr(scales), rows, G * 32, _ptr(out), _stream(dev, stream))
+    _check(st, "mxq_scales_to_mma_layout")
+    return out
+
+
+def mxfp4_gemm(a_codes: torch.Tensor, a_scales: torch.Tensor, b_codes: torch.Tensor, b_scales: torch.Tensor, *,
+               out_dtype: torch.dtype = torch.float32, out: Optional[torch.Tensor] = None,
+               stream=None) -> torch.Tensor:
+    """Y = deq(A) · deq(B)ᵀ on the block-scaled tensor cores; A [M, K/2] codes, B [N, K/2] codes.
+
+    Scales may be row-major ([M, K/32], [N, K/32]: converted here by the layout kernel) or
+    already in the MMA layout (flat uint8 of mxq_scales_mma_bytes)."""
+    dev = a_codes.device
+    if dev.type != "cuda":
+        raise ValueError("operands must be CUDA tensors (this library has no CPU path)")
+    for t, name in ((a_codes, "a_codes"), (a_scales, "a_scales"), (b_codes, "b_codes"), (b_scales, "b_scales")):
+        _need(t, name, torch.uint8, dev)
+    M, K = a_codes.shape[0], a_codes.shape[1] * 2
+    N = b_codes.shape[0]
+    if b_codes.shape[1] * 2 != K:
+        raise ValueError("operand shapes disagree")
+    if a_scales.dim() == 2:
+        if tuple(a_scales.shape) != (M, K // 32):
+            raise ValueError("a_scales must be [M, K/32]")
+        a_scales = scales_to_mma_layout(a_scales, stream=stream) if M and K else a_scales
+    if b_scales.dim() == 2:
+        if tuple(b_scales.shape) != (N, K // 32):
+            raise ValueError("b_scales must be [N, K/32]")
+        b_scales = scales_to_mma_layout(b_scales, stream=stream) if N and K else b_scales
+    if out is not None:
+        out_dtype = out.dtype
+    if out_dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("out_dtype must be float32 or bfloat16")
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=dev)
+    _need(out, "out", out_dtype, dev)
+    st = lib().mxq_mxfp4_gemm(_ptr(a_codes), _ptr(a_scales), _ptr(b_codes), _ptr(b_scales), M, N, K, _ptr(out),
+                              int(out_dtype == torch.bfloat16), _stream(dev, stream))
+    _check(st, "mxq_mxfp4_gemm")
     return out
 
 

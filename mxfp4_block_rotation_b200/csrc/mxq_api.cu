@@ -205,6 +205,25 @@ mxq_status make_tmap_blocks(CUtensorMap *map, const void *X, int64_t rows, int64
     return MXQ_OK;
 }
 
+// MXFP4 codes [rows, K/2] bytes as a GEMM operand: boxes of 128 bytes (256 k) x box_rows
+// rows, 128-byte swizzle, zero fill past the edges.
+mxq_status make_tmap_operand(CUtensorMap *map, const void *codes, int64_t rows, int64_t K, uint32_t box_rows)
+{
+    const Driver &d = driver();
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
+    cuuint32_t box[2] = {128, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = d.encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(codes), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        note_cu(r, "cuTensorMapEncodeTiled(gemm operand)");
+        return MXQ_ERR_CUDA;
+    }
+    return MXQ_OK;
+}
+
 mxq_status make_tmap_x(CUtensorMap *map, const void *X, int64_t rows, int64_t cols)
 {
     const Driver &d = driver();
@@ -226,7 +245,7 @@ mxq_status make_tmap_x(CUtensorMap *map, const void *X, int64_t rows, int64_t co
 // blk: the rotation block width (32 for the main path; 16, 64 or 128 for the variants).
 mxq_status rotate_common(const void *X, int64_t rows, int64_t cols, const void *R, const float *lam,
                          void *out0, uint64_t out0_bytes, uint64_t out0_align, void *out1,
-                         uint64_t out1_bytes, mxq::RotOut mode, void *stream, int blk = 32)
+                         uint64_t out1_bytes, mxq::RotOut mode, void *stream, int blk = 32, int lam_mul = 0)
 {
     mxq_status st = check_shape(rows, cols);
     if (st != MXQ_OK) return st;
@@ -274,6 +293,7 @@ mxq_status rotate_common(const void *X, int64_t rows, int64_t cols, const void *
     mxq::RotArgs args{};
     args.rhat = static_cast<const uint16_t *>(R);
     args.rblk = blk == 16 ? 16 : 32;
+    args.lam_mul = lam_mul;
     args.lambda = lam;
     args.rows = rows;
     args.cols = cols;
@@ -336,6 +356,105 @@ mxq_status mxq_rotate_block_f32(const void *X_bf16, int64_t rows, int64_t cols, 
     const uint64_t ny = rows > 0 && cols > 0 ? static_cast<uint64_t>(rows) * cols * 4 : 0;
     return rotate_common(X_bf16, rows, cols, R_bf16, Lambda_or_null, out_f32, ny, 16, nullptr, 0,
                          mxq::RotOut::F32, stream, block);
+}
+
+mxq_status mxq_weight_rotate_quantize(const void *Wt_bf16, int64_t rows, int64_t cols, const void *Rhat_bf16,
+                                      const float *Lambda_or_null, uint8_t *out_codes_u8_packed,
+                                      uint8_t *out_scales_e8m0, void *stream)
+{
+    const uint64_t nc = rows > 0 && cols > 0 ? static_cast<uint64_t>(rows) * cols / 2 : 0;
+    const uint64_t ns = rows > 0 && cols > 0 ? static_cast<uint64_t>(rows) * (cols / 32) : 0;
+    return rotate_common(Wt_bf16, rows, cols, Rhat_bf16, Lambda_or_null, out_codes_u8_packed, nc, 16,
+                         out_scales_e8m0, ns, mxq::RotOut::Quant, stream, 32, 1);
+}
+
+size_t mxq_scales_mma_bytes(int64_t rows, int64_t K)
+{
+    if (rows <= 0 || K <= 0 || K % 32) return 0;
+    return static_cast<size_t>((rows + 127) / 128) * static_cast<size_t>((K / 32 + 3) / 4) * 512;
+}
+
+mxq_status mxq_scales_to_mma_layout(const uint8_t *scales, int64_t rows, int64_t K, uint8_t *out, void *stream)
+{
+    if (rows < 0 || K < 0 || K % 32) return bad("rows >= 0 and K a multiple of 32 required");
+    if (rows >= (int64_t(1) << 31) || K >= (int64_t(1) << 31)) return bad("rows and K must be < 2^31");
+    if (rows == 0 || K == 0) return MXQ_OK;
+    if (!scales || !out) return bad("null pointer");
+    if (!aligned(out, 16)) return bad("out must be 16-byte aligned");
+    const uint64_t ns = static_cast<uint64_t>(rows) * (K / 32), no = mxq_scales_mma_bytes(rows, K);
+    if (overlaps(out, no, scales, ns)) return bad("the output overlaps the input");
+    int dev = 0, sms = 0;
+    mxq_status st;
+    if ((st = current_device(&dev, &sms)) != MXQ_OK) return st;
+    if ((st = check_buffer(scales, ns, dev)) != MXQ_OK) return st;
+    if ((st = check_buffer(out, no, dev)) != MXQ_OK) return st;
+    const cudaError_t e = mxq::launch_scales_to_mma(scales, rows, K / 32, out, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) {
+        note_cuda(e, "launch scale layout kernel");
+        return MXQ_ERR_CUDA;
+    }
+    return MXQ_OK;
+}
+
+mxq_status mxq_mxfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales_mma, const uint8_t *b_codes,
+                          const uint8_t *b_scales_mma, int64_t M, int64_t N, int64_t K, void *out, int out_bf16,
+                          void *stream)
+{
+    const uint8_t *a_scales = a_scales_mma, *b_scales = b_scales_mma;
+    if (M < 0 || N < 0 || K < 0) return bad("negative size");
+    if (K % 32) return bad("K must be a multiple of 32");
+    if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
+        return bad("M, N and K must be < 2^31");
+    if (out_bf16 != 0 && out_bf16 != 1) return bad("out_bf16 must be 0 (fp32) or 1 (bf16)");
+    if (M == 0 || N == 0) return MXQ_OK;
+    const uint64_t ny = static_cast<uint64_t>(M) * N * (out_bf16 ? 2 : 4);
+    if (!out) return bad("null pointer");
+    if (!aligned(out, 16)) return bad("out must be 16-byte aligned");
+    int dev = 0, sms = 0;
+    mxq_status st = MXQ_OK;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (K == 0) {   // an empty sum: Y = 0
+        if ((st = current_device(&dev, &sms)) != MXQ_OK) return st;
+        if ((st = check_buffer(out, ny, dev)) != MXQ_OK) return st;
+        const cudaError_t e = cudaMemsetAsync(out, 0, ny, s);
+        if (e != cudaSuccess) {
+            note_cuda(e, "cudaMemsetAsync");
+            return MXQ_ERR_CUDA;
+        }
+        return MXQ_OK;
+    }
+    if (!a_codes || !a_scales || !b_codes || !b_scales) return bad("null pointer");
+    if (!aligned(a_codes, 16) || !aligned(b_codes, 16)) return bad("codes must be 16-byte aligned");
+    if (!aligned(a_scales, 16) || !aligned(b_scales, 16)) return bad("scale atoms must be 16-byte aligned");
+    const uint64_t nca = static_cast<uint64_t>(M) * (K / 2), nsa = mxq_scales_mma_bytes(M, K);
+    const uint64_t ncb = static_cast<uint64_t>(N) * (K / 2), nsb = mxq_scales_mma_bytes(N, K);
+    const void *ins[4] = {a_codes, a_scales, b_codes, b_scales};
+    const uint64_t nins[4] = {nca, nsa, ncb, nsb};
+    for (int i = 0; i < 4; ++i)
+        if (overlaps(out, ny, ins[i], nins[i])) return bad("the output overlaps an input");
+    if ((st = current_device(&dev, &sms)) != MXQ_OK) return st;
+    for (int i = 0; i < 4; ++i)
+        if ((st = check_buffer(ins[i], nins[i], dev)) != MXQ_OK) return st;
+    if ((st = check_buffer(out, ny, dev)) != MXQ_OK) return st;
+    alignas(64) CUtensorMap map_a, map_b;
+    if ((st = make_tmap_operand(&map_a, a_codes, M, K, 128)) != MXQ_OK) return st;
+    if ((st = make_tmap_operand(&map_b, b_codes, N, K, 256)) != MXQ_OK) return st;
+    mxq::GemmArgs g{};
+    g.a_sf = a_scales;
+    g.b_sf = b_scales;
+    g.cb_n = (K / 32 + 3) / 4;
+    g.rb_b = (N + 127) / 128;
+    g.y = out;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.out_bf16 = out_bf16;
+    const cudaError_t e = mxq::launch_mxfp4_gemm(map_a, map_b, g, sms, s);
+    if (e != cudaSuccess) {
+        note_cuda(e, "launch MXFP4 GEMM kernel");
+        return MXQ_ERR_CUDA;
+    }
+    return MXQ_OK;
 }
 
 mxq_status mxq_dequantize(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t cols,

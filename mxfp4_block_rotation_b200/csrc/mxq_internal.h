@@ -21,6 +21,7 @@ enum class RotOut { Quant, F32, Err };
 struct RotArgs {
     const uint16_t *rhat;      // bf16 [32][32], row-major [k][n]; [16][16] when rblk == 16
     int rblk;                  // 16: R^ is diag(R16, R16) built from a 16x16 input; otherwise 32
+    int lam_mul;               // 1: multiply by lambda (the weights' side); 0: divide (activations)
     const float *lambda;       // fp32 [cols] or nullptr
     uint8_t *codes;            // [rows, cols/2]   (Quant)
     uint8_t *scales;           // [rows, cols/32]  (Quant)
@@ -47,6 +48,25 @@ cudaError_t launch_rotate_cols(const CUtensorMap &tmap_x, const CUtensorMap &tma
 // swizzle); args.rhat is bf16 [blk][blk].
 cudaError_t launch_rotate_block(const CUtensorMap &tmap_blocks, const RotArgs &args, int blk, RotOut mode,
                                 int num_sms, cudaStream_t stream);
+
+// The MXFP4 x MXFP4 consumer GEMM: Y[M, N] = deq(A)[M, K] * deq(B)[N, K]^T.  `tmap_a` /
+// `tmap_b` view the codes as uint8 [M, K/2] / [N, K/2] (boxes {128, 128} / {128, 256},
+// 128-byte swizzle).
+struct GemmArgs {
+    const uint8_t *a_sf;       // A's scales as 512-byte MMA atoms [ceil(M/128)][cb_n], 16-byte aligned
+    const uint8_t *b_sf;       // B's scales as atoms [rb_b = ceil(N/128)][cb_n]
+    int64_t cb_n;              // atoms per row block: ceil(K/128)
+    int64_t rb_b;
+    void *y;                   // [M, N] fp32 or bf16, row-major, 16-byte aligned
+    int64_t M, N, K;
+    int out_bf16;
+};
+cudaError_t launch_mxfp4_gemm(const CUtensorMap &tmap_a, const CUtensorMap &tmap_b, const GemmArgs &args,
+                              int num_sms, cudaStream_t stream);
+
+// Row-major E8M0 scales [rows, G] -> the block-scaled MMA's 512-byte atoms (128 rows x 4
+// k-blocks; row r, k-block j at byte 16 (r % 32) + 4 (r / 32) + j; padding 0).
+cudaError_t launch_scales_to_mma(const uint8_t *scales, int64_t rows, int64_t G, uint8_t *out, cudaStream_t stream);
 
 // Number of per-warp partial sums the Err mode writes (one double each).
 int64_t rotate_flat_partials(int64_t rows, int64_t cols);

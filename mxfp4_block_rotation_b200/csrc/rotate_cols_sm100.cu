@@ -169,6 +169,7 @@ __global__ void __launch_bounds__(kColThreads, 1)
         // Builders: R^ in fp32, transposed to [n][k]; then per tile 1/Lambda of its 128
         // channels (a reciprocal plus its FMA residual, so R*(1/Lambda) is good to about
         // an ulp), then the four B_g = diag(1/Lambda_g) R^ split three ways into bf16.
+        // The weights' side (lam_mul) uses Lambda itself: B_g = diag(Lambda_g) R^.
         const int bt = threadIdx.x - kBuildWarp0 * 32;   // 0..127
         constexpr int kB = kColBuildWarps * 32;
         for (int i = bt; i < 32 * 32; i += kB) {
@@ -198,8 +199,12 @@ __global__ void __launch_bounds__(kColThreads, 1)
                     float ih = 0.0f, il = 0.0f;
                     if (ch < cols) {
                         const float lam = args.lambda[ch];
-                        ih = __frcp_rn(lam);
-                        il = __fmul_rn(__fmaf_rn(-lam, ih, 1.0f), ih);   // 1/lam - ih, to working precision
+                        if (args.lam_mul) {
+                            ih = lam;   // the weights' side: R * Lambda, one rounding
+                        } else {
+                            ih = __frcp_rn(lam);
+                            il = __fmul_rn(__fmaf_rn(-lam, ih, 1.0f), ih);   // 1/lam - ih, to working precision
+                        }
                     }
                     inv[bt] = make_float2(ih, il);
                 }

@@ -63,6 +63,8 @@ def lib():
         L.mxq_oracle_smooth_rotate_quantize.argtypes = [P, I64, I64, P, P, P, P, P, P, P, P, P, I]
         L.mxq_oracle_weight_rotate_quantize.argtypes = [P, I64, I64, P, P, P, P, P, P, P, P, P, I]
         L.mxq_oracle_weight_rotate_quantize.restype = I
+        L.mxq_oracle_scales_to_mma.argtypes = [P, I64, I64, P]
+        L.mxq_oracle_scales_to_mma.restype = I
         L.mxq_oracle_mxfp4_gemm.argtypes = [P, P, P, P, I64, I64, I64, P, I]
         L.mxq_oracle_mxfp4_gemm.restype = I
         L.mxq_oracle_block_rotate_quantize.argtypes = [P, I64, I64, I, P, P, P, P, P, P, P, P, P, I]
@@ -219,6 +221,16 @@ def weight_rotate_quantize(wt_bits: np.ndarray, rhat_bits: np.ndarray, lam: Opti
         _ptr(g("y")), _ptr(g("eflags")), _ptr(g("alt")), _ptr(g("gflags")), _ptr(g("alt_scales")), threads)
     if rc:
         raise ValueError("oracle: bad shape")
+    return out
+
+
+def scales_to_mma(scales: np.ndarray) -> np.ndarray:
+    """Row-major E8M0 scales [rows, G] -> the block-scaled MMA's 512-byte atoms (flat uint8)."""
+    scales = _c(scales, np.uint8)
+    rows, G = scales.shape
+    out = np.zeros(((rows + 127) // 128) * ((G + 3) // 4) * 512, np.uint8)
+    if lib().mxq_oracle_scales_to_mma(_ptr(scales), rows, G, _ptr(out)):
+        raise ValueError("oracle scales_to_mma: bad shape")
     return out
 
 

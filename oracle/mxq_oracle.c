@@ -370,6 +370,26 @@ int mxq_oracle_mxfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, const
     return 0;
 }
 
+/* Row-major E8M0 scales [rows, G] (G = K/32) in the layout Blackwell's
+ * block-scaled MMA reads them in: 512-byte atoms, one per 128 rows x 4
+ * k-blocks, atoms ordered by row block then k-block; inside an atom the scale
+ * of row r (0..127) and k-block j (0..3) is byte 16 * (r % 32) + 4 * (r / 32) + j.
+ * Rows and k-blocks past the matrix are 0.  out: ceil(rows/128) * ceil(G/4) * 512 bytes. */
+int mxq_oracle_scales_to_mma(const uint8_t *scales, int64_t rows, int64_t G, uint8_t *out)
+{
+    if (rows < 0 || G < 0) return 1;
+    int64_t RB = (rows + 127) / 128, CB = (G + 3) / 4;
+    for (int64_t rb = 0; rb < RB; ++rb)
+        for (int64_t cb = 0; cb < CB; ++cb)
+            for (int r = 0; r < 128; ++r)
+                for (int j = 0; j < 4; ++j) {
+                    int64_t row = rb * 128 + r, kb = cb * 4 + j;
+                    uint8_t v = (row < rows && kb < G) ? scales[row * G + kb] : 0;
+                    out[(rb * CB + cb) * 512 + 16 * (r % 32) + 4 * (r / 32) + j] = v;
+                }
+    return 0;
+}
+
 /* The rotation-block-size variant of the write-up's §4.3 ablation: blocks of
  * B = 16, 32, 64 or 128 columns are rotated by one shared B x B matrix, and
  * the MXFP4 groups stay at 32 columns.  For each row and each block of B

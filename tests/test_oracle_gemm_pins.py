@@ -109,3 +109,23 @@ def test_quantised_product_approximates_the_full_product():
     y = oracle.mxfp4_gemm(qa["codes"], qa["scales"], qb["codes"], qb["scales"])
     want = _f64(x) @ _f64(wt).T
     assert np.linalg.norm(y - want) / np.linalg.norm(want) < 0.25
+
+
+def test_scale_atoms_hold_every_scale_once():
+    # every scale lands at the byte the atom formula names, and everything else is 0
+    rng = np.random.default_rng(9)
+    rows, G = 300, 13                      # ragged in both: 3 row blocks, 4 k-block groups
+    sc = rng.integers(1, 255, (rows, G), dtype=np.uint8)
+    out = oracle.scales_to_mma(sc)
+    CB = (G + 3) // 4
+    assert out.size == 3 * CB * 512
+    seen = np.zeros(out.size, bool)
+    for r in range(rows):
+        for kb in range(G):
+            off = ((r // 128) * CB + kb // 4) * 512 + 16 * (r % 32) + 4 * ((r % 128) // 32) + kb % 4
+            assert out[off] == sc[r, kb]
+            seen[off] = True
+    assert not out[~seen].any()
+    # one 16-byte row of an atom: four words, one per 32-row slice, each the row's 4 k-blocks
+    atom = out[:512].reshape(32, 4, 4)
+    assert np.array_equal(atom[5, 2], sc[64 + 5, 0:4])
