@@ -73,6 +73,15 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def _bf16_peak_tflops() -> float:
+    """Measured dense bf16 burst TFLOP/s (MEASURED_PEAKS.json), else the recipe's fallback 1590."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except (OSError, KeyError, ValueError):
+        return 1590.0
+
+
 def recorded_traffic():
     """DRAM bytes per launch from the committed ncu summary, if the kernel source is unchanged."""
     try:
@@ -395,6 +404,37 @@ def run_extras(mxq, w, xs, rhat, outs, dev, stream, k=300):
         row(f"rotate_quantize_block{blk}", _timed(quant_blk, k, stream, dev), algorithmic_bytes(rows, cols),
             f"rotation blocks of {blk} columns, MXFP4 groups of 32 "
             f"({'rotate_flat_kernel with diag(R16, R16)' if blk == 16 else 'rotate_block_kernel'})")
+    # the consumer GEMM of the down-projection: MXFP4(X R) [8192 x 14336] times the absorbed weight
+    # MXFP4(W^T R) [4096 x 14336] (synthetic N(0, 1/K) weight), bf16 out, on the block-scaled tensor cores
+    n_out = 4096
+    wt = synth.random_bf16(n_out, cols, seed=77, scale=1.0 / cols ** 0.5).to(dev)
+    cb, sb = mxq.weight_rotate_quantize(wt, rhat, None, stream=stream)
+    ca, sa = outs[0]
+    sfa = mxq.scales_to_mma_layout(sa, stream=stream)
+    sfb = mxq.scales_to_mma_layout(sb, stream=stream)
+    y = torch.empty((rows, n_out), dtype=torch.bfloat16, device=dev)
+    flops = 2.0 * rows * n_out * cols
+    fp4_peak = _bf16_peak_tflops() * 4.0
+
+    def gemm(i):
+        mxq.mxfp4_gemm(ca, sfa, cb, sfb, out=y, stream=stream)
+    ms = _timed(gemm, max(1, min(50, k)), stream, dev)
+    res["mxfp4_gemm_downproj"] = {
+        "what": f"Y[{rows}x{n_out}] = MXFP4(X R) MXFP4(W^T R)^T, K = {cols}, bf16 out (mxfp4_gemm_kernel)",
+        "ms": ms, "TFLOP/s": flops / (ms * 1e-3) / 1e12, "peak_TFLOP/s": fp4_peak,
+        "frac_of_fp4_peak": flops / (ms * 1e-3) / 1e12 / fp4_peak,
+        "peak_source": "measured bf16 burst (MEASURED_PEAKS.json bf16_tflops) x 4, the nominal fp4/bf16 ratio"}
+
+    def layer(i):
+        c, s = outs[i & 1]
+        mxq.smooth_rotate_quantize(xs[i & 1], rhat, None, codes=c, scales=s, stream=stream)
+        mxq.scales_to_mma_layout(s, out=sfa, stream=stream)
+        mxq.mxfp4_gemm(c, sfa, cb, sfb, out=y, stream=stream)
+    ms = _timed(layer, max(1, min(50, k)), stream, dev)
+    res["downproj_layer_quantize_plus_gemm"] = {
+        "what": "the whole layer: rotate+quantise X, scale layout, MXFP4 GEMM (3 launches)", "ms": ms,
+        "TFLOP/s": flops / (ms * 1e-3) / 1e12}
+    del wt, cb, sb, sfa, sfb, y
     # the offline rotation search on the same activations, smoothed: K = 128 steps, 64 angles per pair
     sws = torch.empty(mxq.lib().mxq_rotation_search_workspace_bytes(rows, cols, 32), dtype=torch.uint8, device=dev)
     found = {}
