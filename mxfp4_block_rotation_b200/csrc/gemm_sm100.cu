@@ -13,7 +13,7 @@
 //   warps 0-3  epilogue: TMEM -> registers -> fp32 or bf16 stores (warp w reads lane quarter w)
 //   warp 4     TMA producer: per stage, 256 k of A (128 rows x 128 B) and B (256 rows x 128 B),
 //              128-byte swizzle, zero fill past the matrix edges, plus the stage's scale atoms
-//              (bulk copies of 512-byte atoms: 2 for A, 2 x 2 for B) on the same barrier
+//              (bulk copies of 512-byte atoms: 2 for A, 2 x 2 for B) on a barrier of their own
 //   warp 5     TMEM owner and MMA issuer: four tcgen05.mma kind::mxf4 block32 of K = 64 per
 //              stage, M = 128, N = 256, fp32 accumulator in TMEM columns 0-255
 //   warps 6-9  scale movers: the stage's atoms from shared memory into TMEM with tcgen05.st,
@@ -104,7 +104,8 @@ static_assert(kGAccCols + kGStages * kGSfCols <= 512, "TMEM budget");
 static_assert(kGSmem <= 232448, "shared memory budget");
 
 struct GemmBars {
-    uint64_t full[kGStages];      // TMA bytes of a stage landed
+    uint64_t full[kGStages];      // TMA bytes of a stage's operands landed
+    uint64_t sf_in[kGStages];     // the stage's scale atoms landed in shared memory
     uint64_t sf_full[kGStages];   // the stage's scales are in TMEM (4 loader warps)
     uint64_t empty[kGStages];     // the stage's MMAs are done (smem and scale columns free)
     uint64_t acc_full;            // the tile's accumulator is complete
@@ -161,6 +162,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < kGStages; ++s) {
             ptx::mbar_init(ptx::smem_addr(&bars->full[s]), 1);
+            ptx::mbar_init(ptx::smem_addr(&bars->sf_in[s]), 1);
             ptx::mbar_init(ptx::smem_addr(&bars->sf_full[s]), 4);
             ptx::mbar_init(ptx::smem_addr(&bars->empty[s]), 1);
         }
@@ -203,21 +205,26 @@ __global__ void __launch_bounds__(kGThreads, 1)
                     const uint32_t n_at = cb0 + 1 < args.cb_n ? 2u : 1u;
                     const int64_t rb0 = 2 * static_cast<int64_t>(tn);
                     const uint32_t n_rb = rb0 + 1 < args.rb_b ? 2u : 1u;
-                    ptx::mbar_arrive_expect_tx(full, kGAStage + kGBStage + n_at * 512u * (1u + n_rb));
-                    ptx::tma_load_2d(dst, &tmap_a, kt * 128, tm * kGM, full, pol);
-                    ptx::tma_load_2d(dst + kGAStage, &tmap_b, kt * 128, tn * kGN, full, pol);
+                    // the scale atoms first, on their own barrier: the scale warps can move them
+                    // into TMEM while the operand tiles are still in flight
+                    const uint32_t sfb = ptx::smem_addr(&bars->sf_in[s]);
+                    ptx::mbar_arrive_expect_tx(sfb, n_at * 512u * (1u + n_rb));
                     const uint32_t sf = dst + kGAStage + kGBStage;
-                    bulk_load(sf, args.a_sf + (static_cast<int64_t>(tm) * args.cb_n + cb0) * 512, n_at * 512u, full,
+                    bulk_load(sf, args.a_sf + (static_cast<int64_t>(tm) * args.cb_n + cb0) * 512, n_at * 512u, sfb,
                               pol);
                     for (uint32_t h = 0; h < n_rb; ++h)
                         bulk_load(sf + 1024u + h * 1024u, args.b_sf + ((rb0 + h) * args.cb_n + cb0) * 512,
-                                  n_at * 512u, full, pol);
+                                  n_at * 512u, sfb, pol);
+                    ptx::mbar_arrive_expect_tx(full, kGAStage + kGBStage);
+                    ptx::tma_load_2d(dst, &tmap_a, kt * 128, tm * kGM, full, pol);
+                    ptx::tma_load_2d(dst + kGAStage, &tmap_b, kt * 128, tn * kGN, full, pol);
                 }
             }
             // let the last copy into each stage land before the CTA can exit
             for (int s = 0; s < kGStages && s < it; ++s) {
                 const int last = it - 1 - ((it - 1 - s) % kGStages);
                 wait_bar(&bars->full[s], (last / kGStages) & 1, nullptr, status);
+                wait_bar(&bars->sf_in[s], (last / kGStages) & 1, nullptr, status);
             }
         }
     } else if (warp >= kGSfWarp0) {
@@ -228,10 +235,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
             const int64_t rb0 = 2 * (t % tiles_n);
             for (int kt = 0; kt < kt_n; ++kt, ++it) {
                 const int s = it % kGStages;
-                // full[s] covers the atoms; it can only complete after the stage's previous
-                // MMAs freed it, so the scale columns of slot s are free too
+                // sf_in[s] is armed only after the stage's previous MMAs freed it, so the scale
+                // columns of slot s are free too
                 int w_ok = 0;
-                if (lane == 0) w_ok = wait_bar(&bars->full[s], (it / kGStages) & 1, abort, status);
+                if (lane == 0) w_ok = wait_bar(&bars->sf_in[s], (it / kGStages) & 1, abort, status);
                 if (!__shfl_sync(0xffffffffu, w_ok, 0)) {
                     ok = false;
                     break;
