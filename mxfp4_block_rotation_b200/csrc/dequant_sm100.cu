@@ -17,6 +17,7 @@
 #include <cuda_bf16.h>
 
 #include "pipeline_sm100.cuh"
+#include "sm100_bulk.cuh"
 
 namespace mxq {
 namespace {
@@ -76,35 +77,50 @@ using namespace pipe;
 // ---------------------------------------------------------------- undo the transform
 //
 // out = (v * R^T) * Lambda, v = E2M1(code) * 2^e.
-// The same flat group-major pipeline as rotate_flat_kernel, run backwards.  Four
-// decoder warps turn each stage's 512 groups of codes into bf16 values in
-// shared memory: the MMA's A tile, 64-byte swizzle.  The values are exact in
-// bf16: two significant bits times a power of two.  The MMA computes
-// D[g][k] = sum_n v[g][n] * R^[k][n], so B is R^ as stored (row k, contiguous n
-// = K-major).  The epilogue multiplies by Lambda_k and rounds to bf16.
+// The same flat group-major pipeline as rotate_flat_kernel, run backwards.
+//   warp 13     TMA: bulk-copies each stage's codes (512 groups x 16 B = 8 KB, contiguous)
+//               into a 4-deep shared-memory ring
+//   warps 4-11  decoders (two per scheduler): each lane takes one group per pass, reads its 16 code bytes
+//               from the ring, decodes them with byte permutes (no table, so no bank
+//               conflicts), scales by 2^e and writes the MMA's A tile (bf16, 64-byte
+//               swizzle).  The values are exact in bf16: two significant bits times a
+//               power of two.  The scale bytes are fetched before the stage's waits.
+//   warp 12     MMA: D[g][k] = sum_n v[g][n] * R^[k][n], so B is R^ as stored (row k,
+//               contiguous n = K-major)
+//   warps 0-3   epilogue, one per TMEM lane quarter, every stage: times Lambda_k, bf16,
+//               per-warp 2 KB TMA stores
 
-constexpr int kDqDecWarp0 = 8;
-constexpr int kDqDecWarps = 4;
+// The warp split depends on the smoothing: without Lambda the decoders are the
+// critical path (4 epilogue warps, 8 decoders measured best: 86 us against 104 us);
+// with Lambda the epilogue is (8 epilogue warps in two groups taking alternate
+// stages, 4 decoders).  Both use 14 warps.
+template <bool kLambda>
+struct DqSplit {
+    static constexpr int kEpi = kLambda ? 8 : 4;
+    static constexpr int kDec0 = kEpi;
+    static constexpr int kDec = 12 - kEpi;
+};
 constexpr int kDqMmaWarp = 12;
-constexpr int kDqThreads = (kDqMmaWarp + 1) * 32;   // 416
+constexpr int kDqTmaWarp = 13;
+constexpr int kDqThreads = (kDqTmaWarp + 1) * 32;   // 448
 constexpr int kDqStages = 3;
 constexpr int kDqStageGroups = 512;                 // 4 MMAs of 128 groups
 constexpr int kDqStageBytes = kDqStageGroups * 64;
+constexpr int kDqCStages = 3;                       // codes ring
+constexpr int kDqCodeBytes = kDqStageGroups * 16;   // 8 KB of codes per stage
 constexpr int kDqAcc = 4;
 constexpr int kDqAccCols = 128;
 constexpr int kDqOutBuf = 32 * 64;                 // one epilogue warp's 32 output groups (2 KB)
-constexpr int kDqOutBytes = kEpiWarps * 2 * kDqOutBuf;   // double-buffered per epilogue warp
-constexpr int kDqLamBytes = kEpiWarps * 32 * 128;   // per epilogue warp: Lambda of its 32 groups
-constexpr int kDqSmemBytes = kDqStages * kDqStageBytes + kBMatBytes + 1024 + kDqOutBytes + kDqLamBytes + 512 + 1024;
-
-__device__ __forceinline__ uint32_t e2m1_bf16(uint32_t code)
+constexpr int kDqOutBufs = 2;                      // staging buffers per epilogue warp
+__host__ __device__ constexpr int dq_out_bytes(int epi) { return epi * kDqOutBufs * kDqOutBuf; }
+__host__ __device__ constexpr int dq_lam_bytes(int epi) { return epi * 2 * 32 * 128; }   // per warp: Lambda of 32 groups, double-buffered
+__host__ __device__ constexpr int dq_smem_bytes(int epi)
 {
-    // magnitudes {0, 0.5, 1, 1.5, 2, 3, 4, 6}: code 1 is E2M1's subnormal 0.5; codes
-    // 2..7 are 2^(e-1) * (1 + m/2) with e = code >> 1, m = code & 1
-    const uint32_t m = code & 7u;
-    const uint32_t mag = m == 0u ? 0u : (m == 1u ? 0x3F00u : ((126u + (m >> 1)) << 7) | ((m & 1u) << 6));
-    return mag | ((code & 8u) << 12);
+    return kDqStages * kDqStageBytes + kBMatBytes + kDqCStages * kDqCodeBytes + dq_out_bytes(epi) + dq_lam_bytes(epi) +
+           512 + 128 + 1024;
 }
+static_assert(dq_smem_bytes(8) <= 232448 && dq_smem_bytes(4) <= 232448, "shared memory budget");
+static_assert(kEpiWarps / 2 == 4, "acc_empty completes with four arrivals: one epilogue warp per lane quarter");
 
 __device__ __forceinline__ uint32_t hmul2_bits(uint32_t a, __nv_bfloat162 s)
 {
@@ -124,22 +140,48 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *stages = align_1k(smem_raw);
     uint8_t *bmat = stages + kDqStages * kDqStageBytes;
-    uint32_t *lut = reinterpret_cast<uint32_t *>(bmat + kBMatBytes);   // code byte -> bf16x2
-    uint8_t *outbuf = bmat + kBMatBytes + 1024;                          // epilogue staging
-    uint8_t *lambuf = outbuf + kDqOutBytes;                              // epilogue Lambda rows
-    Bars *bars = reinterpret_cast<Bars *>(lambuf + kDqLamBytes);
+    uint8_t *cring = bmat + kBMatBytes;                                  // codes ring
+    using W = DqSplit<kLambda>;
+    uint8_t *outbuf = cring + kDqCStages * kDqCodeBytes;                 // epilogue staging
+    uint8_t *lambuf = outbuf + dq_out_bytes(W::kEpi);                    // epilogue Lambda rows
+    Bars *bars = reinterpret_cast<Bars *>(lambuf + dq_lam_bytes(W::kEpi));
+    uint64_t *c_full = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(bars) + 512);
+    uint64_t *c_empty = c_full + kDqCStages;
     volatile int *abort = &bars->abort;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int n_chunks = static_cast<int>((n_groups + kDqStageGroups - 1) / kDqStageGroups);
 
+    if (threadIdx.x == 0) {   // the codes ring's barriers (kernel_setup fences every init)
+        for (int s = 0; s < kDqCStages; ++s) {
+            ptx::mbar_init(ptx::smem_addr(&c_full[s]), 1);
+            ptx::mbar_init(ptx::smem_addr(&c_empty[s]), W::kDec);
+        }
+    }
     const uint32_t tmem_base = kernel_setup(
-        bars, SetupCfg{kDqStages, kDqAcc, kDqDecWarps * 32, kDqDecWarps * 32, kDqMmaWarp}, &tmap_out, nullptr);
+        bars, SetupCfg{kDqStages, kDqAcc, W::kDec * 32, W::kDec * 32, kDqMmaWarp}, &tmap_out, nullptr);
 
-    if (warp >= kDqDecWarp0 && warp < kDqDecWarp0 + kDqDecWarps) {
-        const int dt = threadIdx.x - kDqDecWarp0 * 32;   // 0..127
-        for (int i = dt; i < 256; i += kDqDecWarps * 32)
-            lut[i] = e2m1_bf16(static_cast<uint32_t>(i) & 15u) | (e2m1_bf16(static_cast<uint32_t>(i) >> 4) << 16);
+    if (warp == kDqTmaWarp) {
+        if (lane == 0) {
+            const uint64_t pol = ptx::policy_evict_first();
+            int it = 0;
+            for (int c = blockIdx.x; c < n_chunks; c += gridDim.x, ++it) {
+                const int cs = it % kDqCStages;
+                if (!wait_bar(&c_empty[cs], ((it / kDqCStages) & 1) ^ 1, abort, status)) break;
+                const int64_t g0 = static_cast<int64_t>(c) * kDqStageGroups;
+                const int64_t n = n_groups - g0 < kDqStageGroups ? n_groups - g0 : kDqStageGroups;
+                const uint32_t bar = ptx::smem_addr(&c_full[cs]);
+                ptx::mbar_arrive_expect_tx(bar, static_cast<uint32_t>(n) * 16u);
+                ptx::bulk_load(ptx::smem_addr(cring + cs * kDqCodeBytes), codes + g0, static_cast<uint32_t>(n) * 16u,
+                               bar, pol);
+            }
+            for (int cs = 0; cs < kDqCStages && cs < it; ++cs) {   // the last copies land before exit
+                const int last = it - 1 - ((it - 1 - cs) % kDqCStages);
+                wait_bar(&c_full[cs], (last / kDqCStages) & 1, nullptr, status);
+            }
+        }
+    } else if (warp >= W::kDec0 && warp < W::kDec0 + W::kDec) {
+        const int dt = threadIdx.x - W::kDec0 * 32;   // 0 .. 32 kDec - 1
         // B: row k holds R^[k][0..31] (bf16) in the first 64 B of a 128-byte-swizzled row
         if (dt < 32 * 4) {
             const int k = dt >> 2, c = dt & 3;
@@ -148,28 +190,43 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         }
         ptx::fence_proxy_async_smem();
         ptx::mbar_arrive(ptx::smem_addr(&bars->b_full[0]));
-        ptx::named_bar_sync(3, kDqDecWarps * 32);   // the table is complete
+        constexpr int kPer = kDqStageGroups / (W::kDec * 32);   // groups per lane per stage
         int it = 0;
         for (int c = blockIdx.x; c < n_chunks; c += gridDim.x, ++it) {
-            const int s = it % kDqStages;
+            const int s = it % kDqStages, cs = it % kDqCStages;
+            const int64_t g0 = static_cast<int64_t>(c) * kDqStageGroups;
+            uint32_t sb[kPer];   // scale bytes, in flight while this warp waits
+#pragma unroll
+            for (int i = 0; i < kPer; ++i) {
+                const int64_t g = g0 + dt + i * W::kDec * 32;
+                sb[i] = g < n_groups ? static_cast<uint32_t>(__ldg(scales + g)) : 0u;
+            }
             int ok = 0;
-            if (lane == 0) ok = wait_bar(&bars->empty[s], ((it / kDqStages) & 1) ^ 1, abort, status);
+            if (lane == 0)
+                ok = wait_bar(&c_full[cs], (it / kDqCStages) & 1, abort, status) &&
+                     wait_bar(&bars->empty[s], ((it / kDqStages) & 1) ^ 1, abort, status);
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
             const uint32_t st = ptx::smem_addr(stages + s * kDqStageBytes);
+            const uint32_t cr = ptx::smem_addr(cring + cs * kDqCodeBytes);
 #pragma unroll
-            for (int i = 0; i < kDqStageGroups / (kDqDecWarps * 32); ++i) {
-                const int r = dt + i * kDqDecWarps * 32;   // group row within the stage
-                const int64_t g = static_cast<int64_t>(c) * kDqStageGroups + r;
+            for (int i = 0; i < kPer; ++i) {
+                const int r = dt + i * W::kDec * 32;   // group row within the stage
                 uint32_t w[16];
-                if (g < n_groups) {
-                    const uint4 cw = __ldcs(codes + g);
-                    const uint32_t byte = __ldg(scales + g);
-                    const uint32_t sb = byte == 0xFFu ? 0x7FC0u : (byte == 0u ? 0x0040u : (byte << 7));
-                    const __nv_bfloat162 s2 = __halves2bfloat162(__ushort_as_bfloat16(static_cast<unsigned short>(sb)),
-                                                                 __ushort_as_bfloat16(static_cast<unsigned short>(sb)));
+                if (g0 + r < n_groups) {
+                    const uint4 cw = ptx::ld_shared_v4(cr + r * 16);
+                    const uint32_t byte = sb[i];
+                    const uint32_t sbits = byte == 0xFFu ? 0x7FC0u : (byte == 0u ? 0x0040u : (byte << 7));
+                    const __nv_bfloat162 s2 =
+                        __halves2bfloat162(__ushort_as_bfloat16(static_cast<unsigned short>(sbits)),
+                                           __ushort_as_bfloat16(static_cast<unsigned short>(sbits)));
                     const uint32_t cws[4] = {cw.x, cw.y, cw.z, cw.w};
 #pragma unroll
-                    for (int b = 0; b < 16; ++b) w[b] = hmul2_bits(lut[(cws[b >> 2] >> (8 * (b & 3))) & 0xFFu], s2);
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t v[4];
+                        ptx::e2m1x8_to_bf16(cws[q], v);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) w[4 * q + e] = hmul2_bits(v[e], s2);
+                    }
                 } else {
 #pragma unroll
                     for (int b = 0; b < 16; ++b) w[b] = 0u;
@@ -180,6 +237,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                     ptx::st_shared_v4(st + r * 64 + ((q ^ ((r >> 1) & 3)) << 4), w[4 * q], w[4 * q + 1],
                                       w[4 * q + 2], w[4 * q + 3]);
             }
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(ptx::smem_addr(&c_empty[cs]));   // this warp's reads of the ring are done
             ptx::fence_proxy_async_smem();
             ptx::mbar_arrive(ptx::smem_addr(&bars->full[s]));
         }
@@ -209,17 +268,17 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             }
             drain_mmas(bars, status);
         }
-    } else if (warp < kEpiWarps) {
+    } else if (warp < W::kEpi) {
         // Each warp stages its 32 groups' outputs (2 KB, 64-byte swizzle) and writes them
         // with one TMA bulk tensor store: 2 KB contiguous instead of 16-byte pieces.
-        const int q = warp & 3;
-        const int ewg = warp >> 2;
-        const uint32_t obuf0 = ptx::smem_addr(outbuf + warp * 2 * kDqOutBuf);
+        const int q = warp & 3;     // TMEM lane quarter
+        const int ewg = warp >> 2;  // with 8 epilogue warps, the two groups take alternate stages
+        const uint32_t obuf0 = ptx::smem_addr(outbuf + warp * kDqOutBufs * kDqOutBuf);
         const bool lam_vec = kLambda && ((reinterpret_cast<uintptr_t>(lambda) & 15) == 0);
-        float *lrows = reinterpret_cast<float *>(lambuf + warp * 32 * 128);   // 32 rows x 32 channels
+        float *lrows2 = reinterpret_cast<float *>(lambuf + warp * 2 * 32 * 128);   // 2 x (32 rows x 32 channels)
         int it = 0, nstore = 0;
         for (int c = blockIdx.x; c < n_chunks; c += gridDim.x, ++it) {
-            if ((it & 1) != ewg) continue;
+            if (W::kEpi == 8 && (it & 1) != ewg) continue;
             const int a = it % kDqAcc;
             int ok = 0;
             if (lane == 0) ok = wait_bar(&bars->acc_full[a], (it / kDqAcc) & 1, abort, status);
@@ -227,35 +286,58 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             ptx::tc_fence_after();
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * kDqAccCols;
             const int64_t g_warp = static_cast<int64_t>(c) * kDqStageGroups + q * 32;
-            // (one register buffer: with 13 warps an SMSP holds four, so 128 registers a thread)
+            // Lambda of the 32 groups of MMA j: rows (g % G) of Lambda viewed as [G][32],
+            // copied into buffer (j & 1) with 16-byte chunks XOR-swizzled by row (8 lanes per
+            // 128-byte row).  With a 16-byte-aligned Lambda the copies are asynchronous and the
+            // next MMA's rows are in flight while this one is processed.
+            // Column groups are taken mod G by subtraction (at most one step once G >= 128): a
+            // division per stage instead of nine per fetch.
+            const int Gi = static_cast<int>(G);
+            const int col_warp = kLambda ? static_cast<int>(g_warp % G) : 0;
+            auto fetch_lambda = [&](int j) {
+                int col0 = col_warp + j * 128;
+                while (col0 >= Gi) col0 -= Gi;
+                float *dst_rows = lrows2 + (j & 1) * 32 * 32;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int r = 4 * i + (lane >> 3), cc = lane & 7;
+                    int cg = col0 + r;
+                    while (cg >= Gi) cg -= Gi;
+                    const float *src = lambda + static_cast<int64_t>(cg) * 32 + cc * 4;
+                    float *dst = dst_rows + r * 32 + ((cc ^ (r & 7)) << 2);
+                    if (lam_vec) {
+                        ptx::cp_async16(ptx::smem_addr(dst), src);
+                    } else {
+                        dst[0] = __ldg(src);
+                        dst[1] = __ldg(src + 1);
+                        dst[2] = __ldg(src + 2);
+                        dst[3] = __ldg(src + 3);
+                    }
+                }
+                ptx::cp_async_commit();
+            };
+            if constexpr (kLambda) {
+                __syncwarp();   // the previous stage's reads of both buffers are done
+                fetch_lambda(0);
+            }
+            // (one register buffer: with 14 warps an SMSP holds four, so 128 registers a thread)
 #pragma unroll 1
             for (int j = 0; j < 4; ++j) {
                 uint32_t cur[32];
                 ptx::tmem_ld_32cols(t_row + j * 32, cur);
-                ptx::tmem_wait_ld();
                 const int64_t g0 = g_warp + j * 128;   // this warp's first group of MMA j
-                // Lambda of the 32 groups' channels: fetched with coalesced loads (8 lanes per
-                // 128-byte row) into this warp's rows, 16-byte chunks XOR-swizzled by row.
+                const float *lrows = lrows2 + (j & 1) * 32 * 32;
                 if constexpr (kLambda) {
-                    __syncwarp();
-                    const int col0 = static_cast<int>(g0 % G);   // column group of this warp's first group
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int r = 4 * i + (lane >> 3), cc = lane & 7;
-                        const float *src = lambda + static_cast<int64_t>((col0 + r) % static_cast<int>(G)) * 32 + cc * 4;
-                        float4 l4;
-                        if (lam_vec) {
-                            l4 = __ldg(reinterpret_cast<const float4 *>(src));
-                        } else {
-                            l4.x = __ldg(src);
-                            l4.y = __ldg(src + 1);
-                            l4.z = __ldg(src + 2);
-                            l4.w = __ldg(src + 3);
-                        }
-                        *reinterpret_cast<float4 *>(lrows + r * 32 + ((cc ^ (r & 7)) << 2)) = l4;
+                    if (j + 1 < 4) {
+                        __syncwarp();   // every lane is done reading buffer (j + 1) & 1 (MMA j - 1)
+                        fetch_lambda(j + 1);
+                        ptx::cp_async_wait<1>();   // MMA j's rows have landed
+                    } else {
+                        ptx::cp_async_wait<0>();
                     }
                     __syncwarp();
                 }
+                ptx::tmem_wait_ld();
                 // times Lambda_k (channels of this group), then round to bf16 pairs
                 uint32_t o[16];
 #pragma unroll
@@ -272,9 +354,9 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                     o[2 * k4 + 1] = static_cast<uint32_t>(__bfloat16_as_ushort(__low2bfloat16(p1))) |
                                     (static_cast<uint32_t>(__bfloat16_as_ushort(__high2bfloat16(p1))) << 16);
                 }
-                const uint32_t buf = obuf0 + (nstore & 1) * kDqOutBuf;
-                // the buffer's previous store (two stores ago) must have been read
-                if (lane == 0) ptx::bulk_wait_group_read1();
+                const uint32_t buf = obuf0 + (nstore % kDqOutBufs) * kDqOutBuf;
+                // the buffer's previous store (kDqOutBufs stores ago) must have been read
+                if (lane == 0) ptx::bulk_wait_group_read<kDqOutBufs - 1>();
                 __syncwarp();
 #pragma unroll
                 for (int v = 0; v < 4; ++v)
@@ -297,7 +379,6 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     kernel_teardown(tmem_base, kDqMmaWarp);
 }
 
-static_assert(kDqSmemBytes <= 232448, "shared memory budget");
 
 }  // namespace
 
@@ -313,9 +394,9 @@ cudaError_t launch_dequant_rot(const CUtensorMap &tmap_out, const uint8_t *codes
     unsigned int *status = status_word();
     if (!status) return cudaErrorInvalidSymbol;
     const uint4 *c4 = reinterpret_cast<const uint4 *>(codes);
-    return lambda ? launch_pdl(dequant_rot_kernel<true>, grid, kDqThreads, kDqSmemBytes, stream, tmap_out, c4, scales,
+    return lambda ? launch_pdl(dequant_rot_kernel<true>, grid, kDqThreads, dq_smem_bytes(8), stream, tmap_out, c4, scales,
                                n_groups, G, rhat, lambda, status)
-                  : launch_pdl(dequant_rot_kernel<false>, grid, kDqThreads, kDqSmemBytes, stream, tmap_out, c4, scales,
+                  : launch_pdl(dequant_rot_kernel<false>, grid, kDqThreads, dq_smem_bytes(4), stream, tmap_out, c4, scales,
                                n_groups, G, rhat, lambda, status);
 }
 

@@ -26,6 +26,7 @@
 // chosen by the top two bits of the scale address and the descriptor's scale ids.
 // Every wait is bounded (2 s) and raises the status word; nothing waits on another CTA.
 #include "pipeline_sm100.cuh"
+#include "sm100_bulk.cuh"
 
 namespace mxq {
 namespace {
@@ -121,23 +122,6 @@ static_assert(sizeof(GemmBars) <= 1024, "barrier block");
 __device__ __forceinline__ uint32_t sfa_col(int s) { return kGAccCols + s * kGSfaCols; }
 __device__ __forceinline__ uint32_t sfb_col(int s) { return kGAccCols + kGStages * kGSfaCols + s * kGSfbCols; }
 
-// Untiled bulk copy global -> shared (16-byte aligned, a multiple of 16 bytes), completing
-// on an mbarrier's transaction count.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar, uint64_t pol)
-{
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
-        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar), "l"(pol)
-        : "memory");
-}
-
-__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr)
-{
-    uint4 v;
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-    return v;
-}
-
 __device__ __forceinline__ uint64_t policy_evict_last()
 {
     uint64_t pol;
@@ -210,10 +194,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
                     const uint32_t sfb = ptx::smem_addr(&bars->sf_in[s]);
                     ptx::mbar_arrive_expect_tx(sfb, n_at * 512u * (1u + n_rb));
                     const uint32_t sf = dst + kGAStage + kGBStage;
-                    bulk_load(sf, args.a_sf + (static_cast<int64_t>(tm) * args.cb_n + cb0) * 512, n_at * 512u, sfb,
+                    ptx::bulk_load(sf, args.a_sf + (static_cast<int64_t>(tm) * args.cb_n + cb0) * 512, n_at * 512u, sfb,
                               pol);
                     for (uint32_t h = 0; h < n_rb; ++h)
-                        bulk_load(sf + 1024u + h * 1024u, args.b_sf + ((rb0 + h) * args.cb_n + cb0) * 512,
+                        ptx::bulk_load(sf + 1024u + h * 1024u, args.b_sf + ((rb0 + h) * args.cb_n + cb0) * 512,
                                   n_at * 512u, sfb, pol);
                     ptx::mbar_arrive_expect_tx(full, kGAStage + kGBStage);
                     ptx::tma_load_2d(dst, &tmap_a, kt * 128, tm * kGM, full, pol);
@@ -248,7 +232,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
                     const bool cv = 2 * static_cast<int64_t>(kt) + c < args.cb_n;
-                    const uint4 va = cv ? ld_shared_v4(sf + c * 512) : make_uint4(0, 0, 0, 0);
+                    const uint4 va = cv ? ptx::ld_shared_v4(sf + c * 512) : make_uint4(0, 0, 0, 0);
                     wa[4 * c] = va.x;
                     wa[4 * c + 1] = va.y;
                     wa[4 * c + 2] = va.z;
@@ -256,7 +240,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const bool v = cv && rb0 + h < args.rb_b;
-                        const uint4 vb = v ? ld_shared_v4(sf + 1024 + h * 1024 + c * 512) : make_uint4(0, 0, 0, 0);
+                        const uint4 vb = v ? ptx::ld_shared_v4(sf + 1024 + h * 1024 + c * 512) : make_uint4(0, 0, 0, 0);
                         wb[8 * c + 4 * h] = vb.x;
                         wb[8 * c + 4 * h + 1] = vb.y;
                         wb[8 * c + 4 * h + 2] = vb.z;
