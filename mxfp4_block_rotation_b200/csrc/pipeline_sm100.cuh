@@ -7,6 +7,7 @@
 #include <cuda_bf16.h>
 
 #include "mxq_internal.h"
+#include "sm100_bulk.cuh"
 #include "sm100_ptx.cuh"
 
 namespace mxq {
@@ -117,19 +118,6 @@ __device__ __forceinline__ uint32_t quantize_group(const uint32_t (&r)[32], uint
     return byte;
 }
 
-// E2M1 value of u (|u| < 8): round to nearest, ties to the even code, saturate at
-// 6, sign kept.  The grid step is 0.5 below 2, 1 below 4 and 2 above, and on each
-// stretch "even code" is "even multiple of the step", so rint (ties to even)
-// applied to u/step gives the same value the E2M1 conversion encodes.
-__device__ __forceinline__ float e2m1_round(float u)
-{
-    const float a = fabsf(u);
-    const float step = a < 2.0f ? 0.5f : (a < 4.0f ? 1.0f : 2.0f);
-    const float inv = a < 2.0f ? 2.0f : (a < 4.0f ? 1.0f : 0.5f);
-    const float q = fminf(__fmul_rn(rintf(__fmul_rn(a, inv)), step), 6.0f);
-    return copysignf(q, u);
-}
-
 // MXFP4 of one group as in quantize_group, plus its normalised quantisation error
 // ||Q(y) - y||_2 / ||y||_2.  With u = y * 2^-e the power of two cancels:
 // error = ||Q(u) - u|| / ||u||, where Q(u) is u's E2M1 value.  An all-zero group
@@ -159,12 +147,27 @@ __device__ __forceinline__ uint32_t quantize_group_err(const uint32_t (&r)[32], 
     for (int q = 0; q < 4; ++q)
         w[q] = ptx::cvt_e2m1x8(u[8 * q], u[8 * q + 1], u[8 * q + 2], u[8 * q + 3], u[8 * q + 4], u[8 * q + 5],
                                u[8 * q + 6], u[8 * q + 7]);
+    // |Q(u)| straight from the codes just produced: byte permutes pick the bf16 bits of each
+    // code's magnitude {0, .5, 1, 1.5, 2, 3, 4, 6} (code 8q + k is nibble k of w[q]); Q(u) has
+    // u's sign, so |Q(u) - u| = ||u| - |Q(u)||.
     float num[4] = {0.0f, 0.0f, 0.0f, 0.0f}, den[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        const float d = __fsub_rn(e2m1_round(u[i]), u[i]);
-        num[i & 3] = __fmaf_rn(d, d, num[i & 3]);
-        den[i & 3] = __fmaf_rn(u[i], u[i], den[i & 3]);
+    for (int q = 0; q < 4; ++q) {
+        const uint32_t m = w[q] & 0x77777777u;
+        const uint32_t h0 = ptx::prmt(0x3F3F3F00u, 0x40404040u, m & 0xFFFFu);
+        const uint32_t l0 = ptx::prmt(0xC0800000u, 0xC0804000u, m & 0xFFFFu);
+        const uint32_t h1 = ptx::prmt(0x3F3F3F00u, 0x40404040u, m >> 16);
+        const uint32_t l1 = ptx::prmt(0xC0800000u, 0xC0804000u, m >> 16);
+        const uint32_t p[4] = {ptx::prmt(l0, h0, 0x5140u), ptx::prmt(l0, h0, 0x7362u), ptx::prmt(l1, h1, 0x5140u),
+                               ptx::prmt(l1, h1, 0x7362u)};
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int i = 8 * q + k;
+            const float qm = __uint_as_float((k & 1) ? (p[k >> 1] & 0xFFFF0000u) : (p[k >> 1] << 16));
+            const float d = __fsub_rn(fabsf(u[i]), qm);
+            num[i & 3] = __fmaf_rn(d, d, num[i & 3]);
+            den[i & 3] = __fmaf_rn(u[i], u[i], den[i & 3]);
+        }
     }
     const float n = (num[0] + num[1]) + (num[2] + num[3]);
     const float d = (den[0] + den[1]) + (den[2] + den[3]);
