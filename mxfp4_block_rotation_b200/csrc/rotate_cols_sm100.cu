@@ -12,8 +12,10 @@
 // an ulp.  Each B_g is then split three ways into bf16, high + middle + low
 // (three MMAs into one accumulator, ~24 bits of B).  X stays the exact bf16 A
 // operand, so the smoothing adds only ~2^-25 relative error on top of fp32
-// accumulation.  Codes go through a shared-memory staging tile (64-byte swizzle)
-// and one TMA bulk tensor store per tile (64 contiguous bytes per row).
+// accumulation.  Each epilogue warp stages its 32 rows of codes in shared memory
+// (64-byte swizzle, two buffers so that one store can be in flight while the next
+// tile is quantised) and writes them with its own TMA bulk tensor store (64
+// contiguous bytes per row); no warp waits for another.
 #include "pipeline_sm100.cuh"
 
 namespace mxq {
@@ -26,13 +28,13 @@ constexpr int kColAcc = 4;                                    // accumulator sta
 constexpr int kColAccCols = 128;
 constexpr int kColStageBytes = kTileM * kTileCols * 2;        // 32 KB of bf16 per stage
 constexpr int kColBoxBytes = kColStageBytes / 2;              // one TMA box: 128 rows x 128 B
-constexpr int kCodeTileBytes = kTileM * kColTileG * 16;       // 128 rows x 64 B of packed codes
 // A tile's B slot holds, per group j, an atom [hi | mid] at j*4 KB and the low
 // parts of groups 2p and 2p+1 side by side in the atom at 16 KB + p*4 KB.
 constexpr int kBLoOffset = kColTileG * kBMatBytes;
 constexpr int kBSlotBytes = kBLoOffset + (kColTileG / 2) * kBMatBytes;   // 24 KB
 constexpr int kColStages = 4;
-constexpr int kColStageOffset = 2 * kCodeTileBytes;           // code staging tiles first
+constexpr int kWarpCodeBytes = 32 * kColTileG * 16;           // one epilogue warp's 32 rows of codes (2 KB)
+constexpr int kColStageOffset = kEpiWarps * 2 * kWarpCodeBytes;   // code staging first: 2 buffers per epilogue warp
 constexpr int kColBOffset = kColStageOffset + kColStages * kColStageBytes;
 constexpr int kColRtOffset = kColBOffset + 2 * kBSlotBytes;
 constexpr int kColInvOffset = kColRtOffset + 32 * 32 * 4;     // per slot: 1/Lambda of the tile's 128 channels
@@ -88,7 +90,7 @@ __global__ void __launch_bounds__(kColThreads, 1)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align_1k(smem_raw);
-    uint8_t *code_tiles = smem;                       // one staging tile per epilogue warp group
+    uint8_t *code_tiles = smem;                       // two 2 KB staging buffers per epilogue warp
     uint8_t *stages = smem + kColStageOffset;
     uint8_t *bmat = smem + kColBOffset;
     float *rt = reinterpret_cast<float *>(smem + kColRtOffset);   // R^ as fp32, [n][k]
@@ -141,22 +143,24 @@ __global__ void __launch_bounds__(kColThreads, 1)
                 if (!wait_bar(&bars->acc_empty[a], ((it / kColAcc) & 1) ^ 1, abort, status)) break;
                 if (sub == 0 && !wait_bar(&bars->b_full[slot], (ui >> 1) & 1, abort, status)) break;
                 ptx::tc_fence_after();
-                const uint32_t a_base = ptx::smem_addr(stages + s * kColStageBytes);
-                const uint32_t b_base = b_base0 + slot * kBSlotBytes;
+                // Descriptors built once per tile; each MMA adds a compile-time offset to the
+                // start-address field (16-byte units; addresses stay below 256 KB, so no carry).
+                const uint64_t ad0 = ptx::smem_desc_sw128(ptx::smem_addr(stages + s * kColStageBytes));
+                const uint64_t bd0 = ptx::smem_desc_sw128(b_base0 + slot * kBSlotBytes);
                 const uint32_t d_base = tmem_base + static_cast<uint32_t>(a * kColAccCols);
 #pragma unroll
                 for (int j = 0; j < kColTileG; ++j) {
-                    const uint32_t a_j = a_base + (j >> 1) * kColBoxBytes + (j & 1) * 64;
                     const uint32_t d_j = d_base + j * 32;
 #pragma unroll
                     for (int kh = 0; kh < 2; ++kh) {
-                        const uint64_t ad = ptx::smem_desc_sw128(a_j + kh * 32);
+                        const uint64_t ad = ad0 + ((((j >> 1) * kColBoxBytes + (j & 1) * 64 + kh * 32)) >> 4);
+                        constexpr uint32_t kLo0 = kBLoOffset;
+                        const uint32_t hi_off = j * kBMatBytes + kh * 32;
+                        const uint32_t lo_off = kLo0 + (j >> 1) * kBMatBytes + (j & 1) * 64 + kh * 32;
                         // smallest part first; the first MMA of the group overwrites D
-                        const uint32_t b_hi = b_base + j * kBMatBytes + kh * 32;
-                        const uint32_t b_lo = b_base + kBLoOffset + (j >> 1) * kBMatBytes + (j & 1) * 64 + kh * 32;
-                        ptx::mma_bf16(d_j, ad, ptx::smem_desc_sw128(b_lo), idesc, kh);
-                        ptx::mma_bf16(d_j, ad, ptx::smem_desc_sw128(b_hi + 64), idesc, 1);
-                        ptx::mma_bf16(d_j, ad, ptx::smem_desc_sw128(b_hi), idesc, 1);
+                        ptx::mma_bf16(d_j, ad, bd0 + (lo_off >> 4), idesc, kh);
+                        ptx::mma_bf16(d_j, ad, bd0 + ((hi_off + 64) >> 4), idesc, 1);
+                        ptx::mma_bf16(d_j, ad, bd0 + (hi_off >> 4), idesc, 1);
                     }
                 }
                 ptx::mma_commit(ptx::smem_addr(&bars->empty[s]));
@@ -248,26 +252,24 @@ __global__ void __launch_bounds__(kColThreads, 1)
         const int q = warp & 3;
         const int ewg = warp >> 2;
         const bool scale_vec = (G % 4 == 0) && ((reinterpret_cast<uintptr_t>(args.scales) & 3) == 0);
-        const uint32_t ctile_smem = ptx::smem_addr(code_tiles + ewg * kCodeTileBytes);
-        const bool leader = q == 0 && lane == 0;   // issues this warp group's code stores
+        // Each warp stages its own 32 rows' codes (32 x 64 B, two buffers) and stores them
+        // with its own TMA store, so the warps of a group never wait for one another.
+        const uint32_t wbuf0 = ptx::smem_addr(code_tiles + warp * 2 * kWarpCodeBytes);
+        int n_st = 0;
         for (int it = ewg; it < sched.n_tiles; it += 2) {
             const int a = it % kColAcc;
-            // The leader alone waits (bounded) and hands the verdict to its warp group through a
-            // named barrier, so the four warps leave the loop together or not at all.
-            volatile int *ok_slot = &bars->eg_ok[ewg][(it >> 1) & 1];
-            if (leader) {
-                int ok = wait_bar(&bars->acc_full[a], (it / kColAcc) & 1, abort, status);
-                // the staging tile must have been read by this group's previous store
-                if constexpr (kMode == RotOut::Quant) ptx::bulk_wait_group_read0();
-                *ok_slot = ok;
+            int ok = 0;
+            if (lane == 0) {
+                ok = wait_bar(&bars->acc_full[a], (it / kColAcc) & 1, abort, status);
+                // this warp's next staging buffer must have been read by the store that used it
+                if constexpr (kMode == RotOut::Quant) ptx::bulk_wait_group_read1();
             }
-            __syncwarp();
-            ptx::named_bar_sync(1 + ewg, 128);
-            if (!*ok_slot) break;
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
             ptx::tc_fence_after();
             int ui, sub, len;
             sched.at(it, ui, sub, len);
             const int ctile = sched.ct_of_unit(ui), rtile = sched.rt0_of_unit(ui) + sub;
+            const uint32_t wbuf = wbuf0 + (n_st & 1) * kWarpCodeBytes;
             const int r_local = q * 32 + lane;
             const int64_t row = static_cast<int64_t>(rtile) * kTileM + r_local;
             const bool row_ok = row < rows;
@@ -303,8 +305,8 @@ __global__ void __launch_bounds__(kColThreads, 1)
                     uint32_t w[4];
                     const uint32_t byte = quantize_group(cur, w);
                     // 64-byte swizzle: 16-byte chunk j of row r sits at chunk j ^ ((r >> 1) & 3)
-                    const uint32_t chunk = static_cast<uint32_t>(j) ^ ((static_cast<uint32_t>(r_local) >> 1) & 3u);
-                    ptx::st_shared_v4(ctile_smem + r_local * 64 + chunk * 16, w[0], w[1], w[2], w[3]);
+                    const uint32_t chunk = static_cast<uint32_t>(j) ^ ((static_cast<uint32_t>(lane) >> 1) & 3u);
+                    ptx::st_shared_v4(wbuf + lane * 64 + chunk * 16, w[0], w[1], w[2], w[3]);
                     if (scale_vec)
                         sc_word |= byte << (8 * j);
                     else if (g < G && row_ok)
@@ -323,18 +325,18 @@ __global__ void __launch_bounds__(kColThreads, 1)
                 if (scale_vec && row_ok)
                     *reinterpret_cast<uint32_t *>(args.scales + row * G + static_cast<int64_t>(ctile) * kColTileG) =
                         sc_word;
-                // staging tile complete -> one bulk store (rows/columns past the tensor are clipped)
+                // this warp's 32 rows complete -> one bulk store (rows/columns past the tensor are clipped)
                 ptx::fence_proxy_async_smem();
                 __syncwarp();
-                ptx::named_bar_sync(1 + ewg, 128);
-                if (leader) {
-                    ptx::tma_store_2d(&tmap_codes, ctile * (kTileCols / 2), rtile * kTileM, ctile_smem);
+                if (lane == 0) {
+                    ptx::tma_store_2d(&tmap_codes, ctile * (kTileCols / 2), rtile * kTileM + q * 32, wbuf);
                     ptx::bulk_commit_group();
                 }
+                ++n_st;
             }
         }
         if constexpr (kMode == RotOut::Quant) {
-            if (leader) ptx::bulk_wait_group0();   // stores done before the CTA's shared memory goes
+            if (lane == 0) ptx::bulk_wait_group0();   // stores done before the CTA's shared memory goes
         }
     }
     kernel_teardown(tmem_base, kMmaWarp);
