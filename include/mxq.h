@@ -240,10 +240,12 @@ mxq_status mxq_quant_error(const void *X_bf16, int64_t rows, int64_t cols, const
  * The function itself allocates nothing.
  *
  *   arguments        as mxq_quant_error, without workspace/workspace_bytes
- *   limit            131072 partial sums: at most 16,777,216 groups of 32
- *                    (rows * cols <= 536,870,912; with Lambda, rows and cols
- *                    count as rounded up to multiples of 128).  Larger inputs
- *                    return MXQ_ERR_INVALID_ARG and mxq_last_cuda_error() says why
+ *   limit            131072 partial sums.  Without Lambda: at most 16,777,216
+ *                    groups of 32 (rows * cols <= 536,870,912).  With Lambda:
+ *                    one sum per 32 rows x 64 columns, so rows * cols <=
+ *                    268,435,456 with rows rounded up to a multiple of 128 and
+ *                    cols to a multiple of 64.  Larger inputs return
+ *                    MXQ_ERR_INVALID_ARG and mxq_last_cuda_error() says why
  *   first call       on each device, the first call looks up the array's device
  *                    address (cudaGetSymbolAddress) with that device current;
  *                    make that first call before any stream capture

@@ -8,9 +8,10 @@
 //     synchronisation.
 // For them, mxq_quant_error_noalloc keeps the per-warp partial sums that
 // mxq_quant_error needs in a fixed array of device memory that belongs to this
-// library.  The array is 1 MiB of doubles: 131072 partial sums, enough for
-// 131072 * 128 = 16,777,216 groups of 32 values (536,870,912 elements).  Larger
-// inputs are rejected.
+// library.  The array is 1 MiB of doubles: 131072 partial sums.  Without the
+// smoothing that covers 131072 * 128 = 16,777,216 groups of 32 values
+// (536,870,912 elements); with it, one sum covers 32 rows x 64 columns, so half
+// as many elements.  Larger inputs are rejected.
 //
 // Every GPU that loads the library holds the array until the process exits.
 // All calls share it.  Each call writes every slot it later reads, so nothing
@@ -66,7 +67,7 @@ extern "C" mxq_status mxq_quant_error_noalloc(const void *X_bf16, int64_t rows, 
         char msg[200];
         std::snprintf(msg, sizeof msg,
                       "invalid argument: %lld x %lld needs %zu bytes of scratch; mxq_quant_error_noalloc has %zu "
-                      "(at most 16777216 groups of 32)",
+                      "(at most 16777216 groups of 32, half that with Lambda)",
                       static_cast<long long>(rows), static_cast<long long>(cols), need, sizeof(g_noalloc_partials));
         mxq::set_last_error(msg);
         return MXQ_ERR_INVALID_ARG;

@@ -4,18 +4,21 @@
 // SmoothQuant scale: X_hat = X * Lambda^-1 * R^ (§3.1, §3.3), quantised to MXFP4 as
 // in §2.1.  The B operand depends on the channel group, B_g = diag(1/Lambda_g)·R^,
 // so an MMA must hold one column group over 128 token rows.  A tile is 128 rows x
-// 128 columns (4 groups), loaded as two 128-byte-swizzled TMA boxes.
+// 64 columns (2 groups): one 128-byte-swizzled TMA box.
 //
 // Warp roles as in the flat kernel, with four builder warps (10-13).  Per unit
-// (4 row blocks of one column tile) they make the tile's four B_g in fp32: a
+// (4 row blocks of one column tile) they make the tile's two B_g in fp32: a
 // reciprocal per channel plus its FMA residual, so R*(1/Lambda) is good to about
-// an ulp.  Each B_g is then split three ways into bf16, high + middle + low
-// (three MMAs into one accumulator, ~24 bits of B).  X stays the exact bf16 A
-// operand, so the smoothing adds only ~2^-25 relative error on top of fp32
-// accumulation.  Each epilogue warp stages its 32 rows of codes in shared memory
-// (64-byte swizzle, two buffers so that one store can be in flight while the next
-// tile is quantised) and writes them with its own TMA bulk tensor store (64
-// contiguous bytes per row); no warp waits for another.
+// an ulp.  Each B_g is split three ways into bf16, high + middle + low (~24 bits
+// of B).  The three parts are stacked along N: one group's B is 96 rows (n of the
+// high part, then the middle, then the low) x 32 k, so a K = 16 step is ONE MMA
+// with N = 96 instead of three with N = 32; the small MMAs' fixed cost in the
+// tensor pipe, not HBM, bounded the three-MMA form.  The epilogue adds the three
+// 32-column partial results, (low + middle) + high, in fp32.  X stays the exact
+// bf16 A operand, so the smoothing adds only ~2^-25 relative error on top of
+// fp32 accumulation.  Each epilogue warp stages its 32 rows of codes (32 x 32 B,
+// two buffers so that one store can be in flight) and writes them with its own
+// TMA bulk tensor store; no warp waits for another.
 #include "pipeline_sm100.cuh"
 
 namespace mxq {
@@ -23,25 +26,28 @@ namespace {
 
 using namespace pipe;
 
-constexpr int kColTileG = 4;                                  // groups per tile
-constexpr int kColAcc = 4;                                    // accumulator stages of 128 columns
-constexpr int kColAccCols = 128;
-constexpr int kColStageBytes = kTileM * kTileCols * 2;        // 32 KB of bf16 per stage
-constexpr int kColBoxBytes = kColStageBytes / 2;              // one TMA box: 128 rows x 128 B
-// A tile's B slot holds, per group j, an atom [hi | mid] at j*4 KB and the low
-// parts of groups 2p and 2p+1 side by side in the atom at 16 KB + p*4 KB.
-constexpr int kBLoOffset = kColTileG * kBMatBytes;
-constexpr int kBSlotBytes = kBLoOffset + (kColTileG / 2) * kBMatBytes;   // 24 KB
-constexpr int kColStages = 4;
-constexpr int kWarpCodeBytes = 32 * kColTileG * 16;           // one epilogue warp's 32 rows of codes (2 KB)
+constexpr int kColTileCols = 64;                              // columns per tile
+constexpr int kColTileG = kColTileCols / 32;                  // groups per tile
+constexpr int kColParts = 3;                                  // bf16 parts of B, stacked along N
+constexpr int kColN = 32 * kColParts;                         // MMA N per group: 96
+constexpr int kColAcc = 2;                                    // accumulator stages
+constexpr int kColAccCols = kColTileG * kColN;                // 192 TMEM columns per stage
+constexpr int kColStageBytes = kTileM * kColTileCols * 2;     // 16 KB of bf16 per stage: one TMA box
+constexpr int kBGroupBytes = kColN * 64;                      // one group's B: 96 rows x 64 B, 64-byte swizzle
+constexpr int kBSlotBytes = kColTileG * kBGroupBytes;         // 12 KB
+constexpr int kColStages = 6;
+constexpr int kWarpCodeBytes = 32 * kColTileG * 16;           // one epilogue warp's 32 rows of codes (1 KB)
 constexpr int kColStageOffset = kEpiWarps * 2 * kWarpCodeBytes;   // code staging first: 2 buffers per epilogue warp
 constexpr int kColBOffset = kColStageOffset + kColStages * kColStageBytes;
 constexpr int kColRtOffset = kColBOffset + 2 * kBSlotBytes;
-constexpr int kColInvOffset = kColRtOffset + 32 * 32 * 4;     // per slot: 1/Lambda of the tile's 128 channels
-constexpr int kColBarOffset = kColInvOffset + 2 * kTileCols * 8;
+constexpr int kColInvOffset = kColRtOffset + 32 * 32 * 4;     // per slot: 1/Lambda of the tile's channels
+constexpr int kColBarOffset = kColInvOffset + 2 * kColTileCols * 8;
 constexpr int kColSmemBytes = kColBarOffset + 512 + 1024;
 constexpr int kColBuildWarps = 4;                             // warps 10-13
 constexpr int kColThreads = (kEpiWarps + 2 + kColBuildWarps) * 32;   // 448
+static_assert(kColStages <= kMaxStages && kColAcc * kColAccCols <= 512 && kColStageOffset % 1024 == 0 &&
+                  kColBOffset % 1024 == 0 && kBGroupBytes % 512 == 0,
+              "smoothing kernel layout");
 
 // Tile order of the smoothing kernel.  A unit is kUnitRows consecutive row
 // blocks of one column tile, so one B_g build serves kUnitRows tiles.  Units are
@@ -103,7 +109,7 @@ __global__ void __launch_bounds__(kColThreads, 1)
     const int64_t rows = args.rows;
     const int64_t cols = args.cols;
     const int64_t G = cols / 32;
-    const int n_ct = static_cast<int>((cols + kTileCols - 1) / kTileCols);
+    const int n_ct = static_cast<int>((cols + kColTileCols - 1) / kColTileCols);
     const int n_rt = static_cast<int>((rows + kTileM - 1) / kTileM);
     const UnitSched sched(n_ct, n_rt, blockIdx.x, gridDim.x);
 
@@ -124,14 +130,13 @@ __global__ void __launch_bounds__(kColThreads, 1)
                 const uint32_t full = ptx::smem_addr(&bars->full[s]);
                 const uint32_t dst = ptx::smem_addr(stages + s * kColStageBytes);
                 ptx::mbar_arrive_expect_tx(full, kColStageBytes);
-                ptx::tma_load_2d(dst, &tmap_x, ctile * kTileCols, rtile * kTileM, full, pol);
-                ptx::tma_load_2d(dst + kColBoxBytes, &tmap_x, ctile * kTileCols + 64, rtile * kTileM, full, pol);
+                ptx::tma_load_2d(dst, &tmap_x, ctile * kColTileCols, rtile * kTileM, full, pol);
             }
             drain_loads(bars, kColStages, it, status);
         }
     } else if (warp == kMmaWarp) {
         if (lane == 0) {
-            constexpr uint32_t idesc = ptx::idesc_bf16_f32(128, 32);
+            constexpr uint32_t idesc = ptx::idesc_bf16_f32(128, kColN);
             const uint32_t b_base0 = ptx::smem_addr(bmat);
             for (int it = 0; it < sched.n_tiles; ++it) {
                 const int s = it % kColStages;
@@ -146,22 +151,14 @@ __global__ void __launch_bounds__(kColThreads, 1)
                 // Descriptors built once per tile; each MMA adds a compile-time offset to the
                 // start-address field (16-byte units; addresses stay below 256 KB, so no carry).
                 const uint64_t ad0 = ptx::smem_desc_sw128(ptx::smem_addr(stages + s * kColStageBytes));
-                const uint64_t bd0 = ptx::smem_desc_sw128(b_base0 + slot * kBSlotBytes);
+                const uint64_t bd0 = ptx::smem_desc_sw64(b_base0 + slot * kBSlotBytes);
                 const uint32_t d_base = tmem_base + static_cast<uint32_t>(a * kColAccCols);
 #pragma unroll
                 for (int j = 0; j < kColTileG; ++j) {
-                    const uint32_t d_j = d_base + j * 32;
 #pragma unroll
-                    for (int kh = 0; kh < 2; ++kh) {
-                        const uint64_t ad = ad0 + ((((j >> 1) * kColBoxBytes + (j & 1) * 64 + kh * 32)) >> 4);
-                        constexpr uint32_t kLo0 = kBLoOffset;
-                        const uint32_t hi_off = j * kBMatBytes + kh * 32;
-                        const uint32_t lo_off = kLo0 + (j >> 1) * kBMatBytes + (j & 1) * 64 + kh * 32;
-                        // smallest part first; the first MMA of the group overwrites D
-                        ptx::mma_bf16(d_j, ad, bd0 + (lo_off >> 4), idesc, kh);
-                        ptx::mma_bf16(d_j, ad, bd0 + ((hi_off + 64) >> 4), idesc, 1);
-                        ptx::mma_bf16(d_j, ad, bd0 + (hi_off >> 4), idesc, 1);
-                    }
+                    for (int kh = 0; kh < 2; ++kh)
+                        ptx::mma_bf16(d_base + j * kColN, ad0 + ((j * 64 + kh * 32) >> 4),
+                                      bd0 + ((j * kBGroupBytes + kh * 32) >> 4), idesc, kh);
                 }
                 ptx::mma_commit(ptx::smem_addr(&bars->empty[s]));
                 ptx::mma_commit(ptx::smem_addr(&bars->acc_full[a]));
@@ -170,9 +167,9 @@ __global__ void __launch_bounds__(kColThreads, 1)
             drain_mmas(bars, status);
         }
     } else if (warp >= kBuildWarp0) {
-        // Builders: R^ in fp32, transposed to [n][k]; then per tile 1/Lambda of its 128
+        // Builders: R^ in fp32, transposed to [n][k]; then per tile 1/Lambda of its 64
         // channels (a reciprocal plus its FMA residual, so R*(1/Lambda) is good to about
-        // an ulp), then the four B_g = diag(1/Lambda_g) R^ split three ways into bf16.
+        // an ulp), then the two B_g = diag(1/Lambda_g) R^ split three ways into bf16.
         // The weights' side (lam_mul) uses Lambda itself: B_g = diag(Lambda_g) R^.
         const int bt = threadIdx.x - kBuildWarp0 * 32;   // 0..127
         constexpr int kB = kColBuildWarps * 32;
@@ -196,9 +193,9 @@ __global__ void __launch_bounds__(kColThreads, 1)
                     built1 = ct;
                 else
                     built0 = ct;
-                const int64_t ch_tile = static_cast<int64_t>(ct) * kTileCols;
-                float2 *inv = inv_tab + slot * kTileCols;
-                {
+                const int64_t ch_tile = static_cast<int64_t>(ct) * kColTileCols;
+                float2 *inv = inv_tab + slot * kColTileCols;
+                if (bt < kColTileCols) {
                     const int64_t ch = ch_tile + bt;
                     float ih = 0.0f, il = 0.0f;
                     if (ch < cols) {
@@ -214,7 +211,9 @@ __global__ void __launch_bounds__(kColThreads, 1)
                 }
                 ptx::named_bar_sync(3, kB);
                 uint8_t *bs = bmat + slot * kBSlotBytes;
-                // 4 groups x 32 rows (n) x 4 chunks of 8 k = 512 chunk tasks.
+                // 2 groups x 32 rows (n) x 4 chunks of 8 k = 256 chunk tasks.  Part p of row n
+                // goes to B row p * 32 + n (64-byte swizzle: 16-byte chunk c of row r sits at
+                // chunk c ^ ((r >> 1) & 3)).
                 for (int task = bt; task < kColTileG * 32 * 4; task += kB) {
                     const int j = task >> 7, n = (task >> 2) & 31, c = task & 3;
                     uint32_t hw[4], mw[4], lw[4];
@@ -237,12 +236,14 @@ __global__ void __launch_bounds__(kColThreads, 1)
                         mw[e] = pack_bf16x2(m[0], m[1]);
                         lw[e] = pack_bf16x2(l[0], l[1]);
                     }
-                    uint8_t *bm = bs + j * kBMatBytes;
-                    uint8_t *bl = bs + kBLoOffset + (j >> 1) * kBMatBytes;
-                    *reinterpret_cast<uint4 *>(bm + sw128(n, c)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-                    *reinterpret_cast<uint4 *>(bm + sw128(n, c + 4)) = make_uint4(mw[0], mw[1], mw[2], mw[3]);
-                    *reinterpret_cast<uint4 *>(bl + sw128(n, c + 4 * (j & 1))) =
-                        make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                    uint8_t *bg = bs + j * kBGroupBytes;
+                    const uint32_t rows3[3] = {static_cast<uint32_t>(n), static_cast<uint32_t>(32 + n),
+                                               static_cast<uint32_t>(64 + n)};
+                    const uint4 v3[3] = {make_uint4(hw[0], hw[1], hw[2], hw[3]), make_uint4(mw[0], mw[1], mw[2], mw[3]),
+                                         make_uint4(lw[0], lw[1], lw[2], lw[3])};
+#pragma unroll
+                    for (int pp = 0; pp < 3; ++pp)
+                        *reinterpret_cast<uint4 *>(bg + rows3[pp] * 64 + ((c ^ ((rows3[pp] >> 1) & 3u)) << 4)) = v3[pp];
                 }
                 ptx::fence_proxy_async_smem();
             }
@@ -251,9 +252,9 @@ __global__ void __launch_bounds__(kColThreads, 1)
     } else {
         const int q = warp & 3;
         const int ewg = warp >> 2;
-        const bool scale_vec = (G % 4 == 0) && ((reinterpret_cast<uintptr_t>(args.scales) & 3) == 0);
-        // Each warp stages its own 32 rows' codes (32 x 64 B, two buffers) and stores them
-        // with its own TMA store, so the warps of a group never wait for one another.
+        const bool scale_vec = (G % 2 == 0) && ((reinterpret_cast<uintptr_t>(args.scales) & 1) == 0);
+        // Each warp stages its own 32 rows' codes (32 rows x 32 B, plain layout, two buffers)
+        // and stores them with its own TMA store, so the warps of a group never wait for one another.
         const uint32_t wbuf0 = ptx::smem_addr(code_tiles + warp * 2 * kWarpCodeBytes);
         int n_st = 0;
         for (int it = ewg; it < sched.n_tiles; it += 2) {
@@ -276,14 +277,22 @@ __global__ void __launch_bounds__(kColThreads, 1)
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * kColAccCols;
             uint32_t sc_word = 0;
             double err_acc = 0.0;   // Err mode: this row's groups of the tile, in order
-            uint32_t ra[32], rb[32];
-            ptx::tmem_ld_32cols(t_row, ra);
-            ptx::tmem_wait_ld();
 #pragma unroll
             for (int j = 0; j < kColTileG; ++j) {
-                uint32_t(&cur)[32] = (j & 1) ? rb : ra;
-                uint32_t(&nxt)[32] = (j & 1) ? ra : rb;
-                if (j + 1 < kColTileG) ptx::tmem_ld_32cols(t_row + (j + 1) * 32, nxt);
+                // the group's value = (low + middle) + high: the three 32-column partials
+                uint32_t cur[32], part[32];
+                const uint32_t tg = t_row + j * kColN;
+                ptx::tmem_ld_32cols(tg + 64, cur);    // low
+                ptx::tmem_ld_32cols(tg + 32, part);   // middle
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    cur[i] = __float_as_uint(__fadd_rn(__uint_as_float(cur[i]), __uint_as_float(part[i])));
+                ptx::tmem_ld_32cols(tg, part);        // high
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    cur[i] = __float_as_uint(__fadd_rn(__uint_as_float(cur[i]), __uint_as_float(part[i])));
                 const int64_t g = static_cast<int64_t>(ctile) * kColTileG + j;
                 if constexpr (kMode == RotOut::F32) {
                     if (g < G && row_ok) {
@@ -304,15 +313,12 @@ __global__ void __launch_bounds__(kColThreads, 1)
                 } else {
                     uint32_t w[4];
                     const uint32_t byte = quantize_group(cur, w);
-                    // 64-byte swizzle: 16-byte chunk j of row r sits at chunk j ^ ((r >> 1) & 3)
-                    const uint32_t chunk = static_cast<uint32_t>(j) ^ ((static_cast<uint32_t>(lane) >> 1) & 3u);
-                    ptx::st_shared_v4(wbuf + lane * 64 + chunk * 16, w[0], w[1], w[2], w[3]);
+                    ptx::st_shared_v4(wbuf + lane * (kColTileG * 16) + j * 16, w[0], w[1], w[2], w[3]);
                     if (scale_vec)
                         sc_word |= byte << (8 * j);
                     else if (g < G && row_ok)
                         args.scales[row * G + g] = static_cast<uint8_t>(byte);
                 }
-                if (j + 1 < kColTileG) ptx::tmem_wait_ld();
             }
             ptx::tc_fence_before();
             __syncwarp();
@@ -323,13 +329,13 @@ __global__ void __launch_bounds__(kColThreads, 1)
             }
             if constexpr (kMode == RotOut::Quant) {
                 if (scale_vec && row_ok)
-                    *reinterpret_cast<uint32_t *>(args.scales + row * G + static_cast<int64_t>(ctile) * kColTileG) =
-                        sc_word;
+                    *reinterpret_cast<uint16_t *>(args.scales + row * G + static_cast<int64_t>(ctile) * kColTileG) =
+                        static_cast<uint16_t>(sc_word);
                 // this warp's 32 rows complete -> one bulk store (rows/columns past the tensor are clipped)
                 ptx::fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    ptx::tma_store_2d(&tmap_codes, ctile * (kTileCols / 2), rtile * kTileM + q * 32, wbuf);
+                    ptx::tma_store_2d(&tmap_codes, ctile * (kColTileCols / 2), rtile * kTileM + q * 32, wbuf);
                     ptx::bulk_commit_group();
                 }
                 ++n_st;
@@ -349,7 +355,7 @@ static_assert(kColSmemBytes <= 232448, "shared memory budget");
 cudaError_t launch_rotate_cols(const CUtensorMap &tmap_x, const CUtensorMap &tmap_codes, const RotArgs &args,
                                RotOut mode, int num_sms, cudaStream_t stream)
 {
-    const int64_t n_tiles = ((args.rows + kTileM - 1) / kTileM) * ((args.cols + kTileCols - 1) / kTileCols);
+    const int64_t n_tiles = ((args.rows + kTileM - 1) / kTileM) * ((args.cols + kColTileCols - 1) / kColTileCols);
     if (n_tiles <= 0) return cudaSuccess;
     const int grid = static_cast<int>(n_tiles < num_sms ? n_tiles : num_sms);
     unsigned int *status = status_word();
@@ -366,7 +372,7 @@ cudaError_t launch_rotate_cols(const CUtensorMap &tmap_x, const CUtensorMap &tma
 
 int64_t rotate_cols_partials(int64_t rows, int64_t cols)
 {
-    return ((rows + kTileM - 1) / kTileM) * ((cols + kTileCols - 1) / kTileCols) * 4;
+    return ((rows + kTileM - 1) / kTileM) * ((cols + kColTileCols - 1) / kColTileCols) * 4;
 }
 
 }  // namespace mxq
