@@ -347,3 +347,20 @@ def test_quant_error_deterministic_and_workspace_checked():
     with pytest.raises(mxq.MxqError) as ei:
         mxq.quant_error(x, r, workspace=small)
     assert ei.value.status == 1
+
+
+def test_row_chunks_equal_one_call():
+    # the rows are independent: quantising row slices (as the pipelined end-to-end leg of the
+    # bench does) gives the same bits as one call over the whole matrix
+    w = synth.make_config(2, rows=1000, cols=1024)
+    x = w.x.to(DEV)
+    rhat = w.rhat.to(DEV)
+    lam = synth.smoothing_scale(w.x).to(DEV)
+    for lm in (None, lam):
+        c, s = mxq.smooth_rotate_quantize(x, rhat, lm)
+        c2 = torch.empty_like(c)
+        s2 = torch.empty_like(s)
+        for lo, hi in ((0, 125), (125, 512), (512, 1000)):
+            mxq.smooth_rotate_quantize(x[lo:hi], rhat, lm, codes=c2[lo:hi], scales=s2[lo:hi])
+        mxq.sync_check()
+        assert torch.equal(c, c2) and torch.equal(s, s2)
