@@ -63,6 +63,14 @@ def lib():
         L.mxq_oracle_smooth_rotate_quantize.argtypes = [P, I64, I64, P, P, P, P, P, P, P, P, P, I]
         L.mxq_oracle_weight_rotate_quantize.argtypes = [P, I64, I64, P, P, P, P, P, P, P, P, P, I]
         L.mxq_oracle_weight_rotate_quantize.restype = I
+        L.mxq_oracle_e4m3_value.argtypes = [I]
+        L.mxq_oracle_e4m3_value.restype = ctypes.c_double
+        L.mxq_oracle_e4m3_code.argtypes = [ctypes.c_double]
+        L.mxq_oracle_e4m3_code.restype = I
+        L.mxq_oracle_nvfp4_block_at.argtypes = [P, I, ctypes.c_float, P, P, P]
+        L.mxq_oracle_nvfp4_block_at.restype = I
+        L.mxq_oracle_nvfp4_quantize.argtypes = [P, I64, I64, P, P, ctypes.c_float, P, P, P, P, P, P, P, I]
+        L.mxq_oracle_nvfp4_quantize.restype = I
         L.mxq_oracle_scales_to_mma.argtypes = [P, I64, I64, P]
         L.mxq_oracle_scales_to_mma.restype = I
         L.mxq_oracle_mxfp4_gemm.argtypes = [P, P, P, P, I64, I64, I64, P, I]
@@ -219,6 +227,47 @@ def weight_rotate_quantize(wt_bits: np.ndarray, rhat_bits: np.ndarray, lam: Opti
     rc = lib().mxq_oracle_weight_rotate_quantize(
         _ptr(wt_bits), rows, cols, _ptr(rhat_bits), _ptr(lam32), _ptr(out["codes"]), _ptr(out["scales"]),
         _ptr(g("y")), _ptr(g("eflags")), _ptr(g("alt")), _ptr(g("gflags")), _ptr(g("alt_scales")), threads)
+    if rc:
+        raise ValueError("oracle: bad shape")
+    return out
+
+
+def e4m3_value(code: int) -> float:
+    return lib().mxq_oracle_e4m3_value(int(code))
+
+
+def e4m3_code(v: float) -> int:
+    return lib().mxq_oracle_e4m3_code(float(v))
+
+
+def nvfp4_block_at(y16, sb: int, s_t: float):
+    """Codes (+ flags, alternatives) of one 16-value block under E4M3 scale byte sb."""
+    y = _c(np.asarray(y16, np.float64), np.float64)
+    codes = np.zeros(16, np.uint8)
+    flags = np.zeros(16, np.uint8)
+    alt = np.zeros(16, np.uint8)
+    lib().mxq_oracle_nvfp4_block_at(_ptr(y), int(sb), float(s_t), _ptr(codes), _ptr(flags), _ptr(alt))
+    return codes, flags, alt
+
+
+def nvfp4_quantize(x_bits: np.ndarray, rhat_bits: np.ndarray, lam: Optional[np.ndarray], s_t: float,
+                   want_y: bool = False, flags: bool = False, threads: int = 1) -> dict:
+    """NVFP4 of X·Λ⁻¹·R̂ (blocks of 16, E4M3 block scales, fp32 tensor scale s_t)."""
+    x_bits = _c(x_bits, np.uint16)
+    rhat_bits = _c(rhat_bits, np.uint16)
+    rows, cols = x_bits.shape
+    NB = cols // 16
+    lam32 = None if lam is None else _c(lam, np.float32)
+    out = {"codes": np.zeros((rows, cols // 2), np.uint8), "scales": np.zeros((rows, NB), np.uint8)}
+    if want_y:
+        out["y"] = np.zeros((rows, cols), np.float64)
+    if flags:
+        out.update(eflags=np.zeros((rows, cols), np.uint8), alt=np.zeros((rows, cols), np.uint8),
+                   bflags=np.zeros((rows, NB), np.uint8), alt_scales=np.zeros((rows, NB), np.uint8))
+    g = out.get
+    rc = lib().mxq_oracle_nvfp4_quantize(
+        _ptr(x_bits), rows, cols, _ptr(rhat_bits), _ptr(lam32), float(s_t), _ptr(out["codes"]), _ptr(out["scales"]),
+        _ptr(g("y")), _ptr(g("eflags")), _ptr(g("alt")), _ptr(g("bflags")), _ptr(g("alt_scales")), threads)
     if rc:
         raise ValueError("oracle: bad shape")
     return out

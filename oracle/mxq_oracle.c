@@ -370,6 +370,159 @@ int mxq_oracle_mxfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, const
     return 0;
 }
 
+/* --------------------------------------------------------------- NVFP4 variant */
+
+/* The write-up's §5.3 names NVFP4 as another block-scaled format the method
+ * suits; it gives no rule for it.  The reading taken is the public NVFP4 format:
+ * blocks of 16 E2M1 values, one E4M3 scale per block and one fp32 scale s_t per
+ * tensor, supplied by the caller.  Every decision is made in fp32 with this
+ * sequence of correctly rounded single-precision operations:
+ *   r_t = 1 / (6 * s_t)                         once per tensor
+ *   v   = amax(block) * r_t;  s_b = E4M3(v)     round to nearest even, saturating at 448
+ *   s   = s_b * s_t;          r   = 1 / s       (s == 0: all codes 0)
+ *   u_n = y_n * r;            code_n = E2M1(u_n) as for MXFP4
+ * A block holding NaN or Inf gets scale byte 0x7F (E4M3 NaN) and codes 0.     */
+
+/* Value of an E4M3 code (OCP FP8, the variant without infinities: sign bit 7,
+ * exponent bits 6-3 with bias 7, mantissa bits 2-0; exponent 0 is subnormal,
+ * 0x7F and 0xFF are NaN, the largest value is 448). */
+double mxq_oracle_e4m3_value(int code)
+{
+    int sgn = (code >> 7) & 1, e = (code >> 3) & 15, m = code & 7;
+    if (e == 15 && m == 7) return NAN;
+    double v = e == 0 ? ldexp(m / 8.0, -6) : ldexp(1.0 + m / 8.0, e - 7);
+    return sgn ? -v : v;
+}
+
+/* Nearest non-negative E4M3 code of v >= 0 by search over every code: ties go
+ * to the even code, values past 448 to 448 (its nearest code), NaN to 0x7F. */
+int mxq_oracle_e4m3_code(double v)
+{
+    if (isnan(v)) return 0x7F;
+    int best = 0;
+    double bd = fabs(v);
+    for (int c = 1; c <= 0x7E; ++c) {
+        double d = fabs(v - mxq_oracle_e4m3_value(c));
+        if (d < bd || (d == bd && (c & 1) == 0)) {
+            best = c;
+            bd = d;
+        }
+    }
+    return best;
+}
+
+/* Codes of one 16-value block (values already fp32) under scale byte sb, with the
+ * same element boundary flags as the MXFP4 quantiser. */
+int mxq_oracle_nvfp4_block_at(const double *y, int sb, float s_t, uint8_t *codes, uint8_t *flags, uint8_t *alt)
+{
+    float s = (float)mxq_oracle_e4m3_value(sb) * s_t;
+    int zero = sb == 0x7F || sb == 0xFF || s == 0.0f;
+    float r = zero ? 0.0f : 1.0f / s;
+    for (int n = 0; n < 16; ++n) {
+        double u = zero ? 0.0 : (double)((float)y[n] * r);
+        int c = zero ? 0 : mxq_oracle_e2m1_code(u);
+        codes[n] = (uint8_t)c;
+        if (flags || alt) {
+            double a = fabs(u);
+            int f = 0, other = c;
+            for (int m = 0; m < 8 && !zero; ++m) {
+                if (fabs(a - MID[m]) < 1e-3 * STEP[m]) {
+                    f = 1;
+                    if (m == 0) {
+                        other = c ^ 8;
+                    } else {
+                        int lo = m - 1, hi = m, mag = c & 7;
+                        other = (c & 8) | (mag == lo ? hi : lo);
+                    }
+                }
+            }
+            if (flags) flags[n] = (uint8_t)f;
+            if (alt) alt[n] = (uint8_t)other;
+        }
+    }
+    return 0;
+}
+
+/* X bf16 [rows, cols] -> y = (X / lam) * R per 32-column group (R bf16 [32][32], as
+ * mxq_oracle_smooth_rotate_quantize) -> NVFP4 of every 16 columns of y.
+ * codes [rows, cols/2] (even column in the low nibble); scales [rows, cols/16] E4M3;
+ * Y, eflags/alt [rows, cols], bflags/alt_scales [rows, cols/16] may be NULL.
+ * A block is flagged when v lies within 2.5e-4 (relative) of an E4M3 rounding midpoint;
+ * alt_scales then holds the code on the other side. */
+int mxq_oracle_nvfp4_quantize(const uint16_t *X, int64_t rows, int64_t cols, const uint16_t *Rb, const float *lam,
+                              float s_t, uint8_t *codes, uint8_t *scales, double *Y, uint8_t *eflags, uint8_t *alt,
+                              uint8_t *bflags, uint8_t *alt_scales, int nthreads)
+{
+    if (rows < 0 || cols < 0 || cols % GROUP) return 1;
+    int64_t G = cols / GROUP, NB = cols / 16;
+    double R[GROUP * GROUP];
+    for (int i = 0; i < GROUP * GROUP; ++i) R[i] = bf16_to_double(Rb[i]);
+    const float d6 = 6.0f * s_t;
+    const float r_t = 1.0f / d6;
+#pragma omp parallel for schedule(dynamic, 4) num_threads(nthreads > 0 ? nthreads : 1)
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t g = 0; g < G; ++g) {
+            double x[GROUP], y[GROUP];
+            int64_t e0 = r * cols + g * GROUP;
+            for (int k = 0; k < GROUP; ++k) {
+                x[k] = bf16_to_double(X[e0 + k]);
+                if (lam) x[k] = x[k] / (double)lam[g * GROUP + k];
+            }
+            for (int n = 0; n < GROUP; ++n) {
+                double acc = 0.0;
+                for (int k = 0; k < GROUP; ++k) acc += x[k] * R[k * GROUP + n];
+                if (Y) Y[e0 + n] = acc;
+                y[n] = (double)(float)acc;          /* the decision precision: fp32 */
+            }
+            for (int h = 0; h < 2; ++h) {
+                const double *yb = y + 16 * h;
+                int64_t b = r * NB + g * 2 + h, eb = e0 + 16 * h;
+                uint8_t c[16];
+                float amax = 0.0f;
+                int bad = 0;
+                for (int n = 0; n < 16; ++n) {
+                    if (isnan(yb[n]) || isinf(yb[n])) bad = 1;
+                    float a = fabsf((float)yb[n]);
+                    if (a > amax) amax = a;
+                }
+                int sb;
+                if (bad) {
+                    sb = 0x7F;
+                    for (int n = 0; n < 16; ++n) {
+                        c[n] = 0;
+                        if (eflags) eflags[eb + n] = 0;
+                        if (alt) alt[eb + n] = 0;
+                    }
+                } else {
+                    float v = amax * r_t;
+                    sb = mxq_oracle_e4m3_code((double)v);
+                    mxq_oracle_nvfp4_block_at(yb, sb, s_t, c, eflags ? eflags + eb : NULL, alt ? alt + eb : NULL);
+                }
+                scales[b] = (uint8_t)sb;
+                if (bflags || alt_scales) {
+                    int f = 0, other = sb;
+                    if (!bad) {
+                        double v = (double)(amax * r_t), sv = mxq_oracle_e4m3_value(sb);
+                        for (int dc = -1; dc <= 1; dc += 2) {
+                            int cn = sb + dc;
+                            if (cn < 0 || cn > 0x7E) continue;
+                            double mid = 0.5 * (sv + mxq_oracle_e4m3_value(cn));
+                            if (fabs(v - mid) < 2.5e-4 * mid) {
+                                f = 1;
+                                other = cn;
+                            }
+                        }
+                    }
+                    if (bflags) bflags[b] = (uint8_t)f;
+                    if (alt_scales) alt_scales[b] = (uint8_t)other;
+                }
+                for (int i = 0; i < 8; ++i) codes[eb / 2 + i] = (uint8_t)(c[2 * i] | (c[2 * i + 1] << 4));
+            }
+        }
+    }
+    return 0;
+}
+
 /* Row-major E8M0 scales [rows, G] (G = K/32) in the layout Blackwell's
  * block-scaled MMA reads them in: 512-byte atoms, one per 128 rows x 4
  * k-blocks, atoms ordered by row block then k-block; inside an atom the scale
