@@ -122,6 +122,31 @@ mxq_status mxq_weight_rotate_quantize(const void *Wt_bf16, int64_t rows, int64_t
                                       void *stream);
 
 /*
+ * The same rotation quantised to NVFP4 instead of MXFP4 (DuQuant++ write-up,
+ * §5.3, names NVFP4 as another block-scaled format the method suits; it gives
+ * no rule for it, so the public NVFP4 format is the one taken).  Each 32-value
+ * group of Y = X * Lambda^-1 * R^ is quantised as two blocks of 16 values.
+ * There is one E4M3 scale per block and one fp32 tensor scale s_t, which the
+ * caller supplies in device memory.  Every decision is made in fp32:
+ *   r_t = 1 / (6 s_t);  v = amax(block) * r_t;  s_b = E4M3(v), round to nearest
+ *   even, saturating at 448;  s = s_b * s_t;  code_n = E2M1(y_n * (1 / s)) as for MXFP4.
+ * A block holding NaN or Inf gets scale 0x7F (E4M3 NaN) and codes 0, and so
+ * does a block whose scale is NaN or 0.  With s_t = amax(Y) / (6 * 448), every
+ * block scale covers its block.
+ *
+ *   X_bf16, rows, cols, Rhat_bf16, Lambda_or_null   as mxq_smooth_rotate_quantize
+ *   tensor_scale_f32    in   fp32 [1] in device memory, 4-byte aligned; read by the kernel
+ *   out_codes_u8_packed out  uint8 [rows, cols/2], 16-byte aligned (even column in the low nibble)
+ *   out_scales_e4m3     out  uint8 [rows, cols/16], 2-byte aligned
+ *   stream              in   cudaStream_t
+ * Errors as mxq_smooth_rotate_quantize; a NULL tensor scale is MXQ_ERR_INVALID_ARG.
+ */
+mxq_status mxq_smooth_rotate_quantize_nvfp4(const void *X_bf16, int64_t rows, int64_t cols,
+                                            const void *Rhat_bf16, const float *Lambda_or_null,
+                                            const float *tensor_scale_f32, uint8_t *out_codes_u8_packed,
+                                            uint8_t *out_scales_e4m3, void *stream);
+
+/*
  * Row-major E8M0 scales [rows, K/32] (the quantisers' layout) -> the layout
  * Blackwell's block-scaled MMA reads scale factors in.  The output is 512-byte
  * atoms, one per 128 rows × 4 k-blocks, ordered by row block and then k-block.

@@ -22,8 +22,9 @@ from typing import Optional, Tuple
 import torch
 
 __all__ = [
-    "MxqError", "smooth_rotate_quantize", "smooth_rotate_f32", "dequantize", "sync_check",
-    "selftest_bounded_wait", "quant_error",
+    "MxqError", "smooth_rotate_quantize", "smooth_rotate_quantize_nvfp4", "smooth_rotate_f32",
+    "weight_rotate_quantize", "rotate_quantize_block", "rotate_block_f32", "scales_to_mma_layout",
+    "mxfp4_gemm", "dequantize", "quant_error", "rotation_search", "sync_check", "selftest_bounded_wait",
     "status_string", "version", "lib", "LIB_PATH", "HEADER_PATH", "declared_symbols",
 ]
 
@@ -66,6 +67,8 @@ def lib() -> ctypes.CDLL:
         L.mxq_rotate_block_f32.restype = I
         L.mxq_weight_rotate_quantize.argtypes = [P, I64, I64, P, P, P, P, P]
         L.mxq_weight_rotate_quantize.restype = I
+        L.mxq_smooth_rotate_quantize_nvfp4.argtypes = [P, I64, I64, P, P, P, P, P, P]
+        L.mxq_smooth_rotate_quantize_nvfp4.restype = I
         L.mxq_mxfp4_gemm.argtypes = [P, P, P, P, I64, I64, I64, P, I, P]
         L.mxq_scales_mma_bytes.argtypes = [I64, I64]
         L.mxq_scales_mma_bytes.restype = ctypes.c_size_t
@@ -170,6 +173,30 @@ def smooth_rotate_quantize(x: torch.Tensor, rhat: torch.Tensor, lam: Optional[to
     st = lib().mxq_smooth_rotate_quantize(_ptr(x), rows, cols, _ptr(rhat), _ptr(lam), _ptr(codes),
                                           _ptr(scales), _stream(dev, stream))
     _check(st, "mxq_smooth_rotate_quantize")
+    return codes, scales
+
+
+def smooth_rotate_quantize_nvfp4(x: torch.Tensor, rhat: torch.Tensor, tensor_scale: torch.Tensor,
+                                 lam: Optional[torch.Tensor] = None, *, codes: Optional[torch.Tensor] = None,
+                                 scales: Optional[torch.Tensor] = None,
+                                 stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """NVFP4(X · Λ⁻¹ · R̂) -> (codes uint8 [rows, cols/2], E4M3 scales uint8 [rows, cols/16]).
+
+    tensor_scale: fp32 [1] on the device (the per-tensor scale s_t)."""
+    dev = _inputs(x, rhat, lam)
+    _need(tensor_scale, "tensor_scale", torch.float32, dev)
+    if tensor_scale.numel() != 1:
+        raise ValueError("tensor_scale must hold one float")
+    rows, cols = x.shape
+    if codes is None:
+        codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+    if scales is None:
+        scales = torch.empty((rows, cols // 16), dtype=torch.uint8, device=dev)
+    _need(codes, "codes", torch.uint8, dev)
+    _need(scales, "scales", torch.uint8, dev)
+    st = lib().mxq_smooth_rotate_quantize_nvfp4(_ptr(x), rows, cols, _ptr(rhat), _ptr(lam), _ptr(tensor_scale),
+                                                _ptr(codes), _ptr(scales), _stream(dev, stream))
+    _check(st, "mxq_smooth_rotate_quantize_nvfp4")
     return codes, scales
 
 

@@ -246,24 +246,32 @@ mxq_status make_tmap_x(CUtensorMap *map, const void *X, int64_t rows, int64_t co
 // blk: the rotation block width (32 for the main path; 16, 64 or 128 for the variants).
 mxq_status rotate_common(const void *X, int64_t rows, int64_t cols, const void *R, const float *lam,
                          void *out0, uint64_t out0_bytes, uint64_t out0_align, void *out1,
-                         uint64_t out1_bytes, mxq::RotOut mode, void *stream, int blk = 32, int lam_mul = 0)
+                         uint64_t out1_bytes, mxq::RotOut mode, void *stream, int blk = 32, int lam_mul = 0,
+                         const float *nv_scale = nullptr)
 {
+    const bool quant = mode == mxq::RotOut::Quant || mode == mxq::RotOut::QuantNv;
     mxq_status st = check_shape(rows, cols);
     if (st != MXQ_OK) return st;
     if (blk != 16 && blk != 32 && blk != 64 && blk != 128) return bad("block must be 16, 32, 64 or 128");
     if (cols % blk) return bad("cols must be a multiple of the block width");
     if (lam && blk > 32) return bad("Lambda is supported with blocks of 16 or 32 columns only");
     if (rows == 0 || cols == 0) return MXQ_OK;   // nothing is read or written
-    if (!X || !R || !out0 || (mode == mxq::RotOut::Quant && !out1)) return bad("null pointer");
+    if (!X || !R || !out0 || (quant && !out1)) return bad("null pointer");
+    if (mode == mxq::RotOut::QuantNv) {
+        if (blk != 32) return bad("NVFP4 takes a 32x32 Rhat");
+        if (!nv_scale) return bad("null pointer");
+        if (!aligned(nv_scale, 4)) return bad("tensor scale must be 4-byte aligned");
+        if (!aligned(out1, 2)) return bad("NVFP4 scales must be 2-byte aligned");
+    }
     if (!aligned(X, 16)) return bad("X must be 16-byte aligned");
     if (!aligned(R, 2)) return bad("Rhat must be 2-byte aligned");
     if (lam && !aligned(lam, 4)) return bad("Lambda must be 4-byte aligned");
     if (!aligned(out0, out0_align)) return bad("output must be 16-byte aligned");
     const uint64_t nx = static_cast<uint64_t>(rows) * cols * 2, nl = lam ? static_cast<uint64_t>(cols) * 4 : 0;
     const uint64_t nr = static_cast<uint64_t>(blk) * blk * 2;
-    const void *ins[3] = {X, R, lam};
-    const uint64_t nins[3] = {nx, nr, nl};
-    for (int i = 0; i < 3; ++i) {
+    const void *ins[4] = {X, R, lam, nv_scale};
+    const uint64_t nins[4] = {nx, nr, nl, nv_scale ? 4u : 0u};
+    for (int i = 0; i < 4; ++i) {
         if (overlaps(out0, out0_bytes, ins[i], nins[i]) || (out1 && overlaps(out1, out1_bytes, ins[i], nins[i])))
             return bad("an output overlaps an input");
     }
@@ -274,6 +282,7 @@ mxq_status rotate_common(const void *X, int64_t rows, int64_t cols, const void *
     if ((st = check_buffer(X, nx, dev)) != MXQ_OK) return st;
     if ((st = check_buffer(R, nr, dev)) != MXQ_OK) return st;
     if (lam && (st = check_buffer(lam, nl, dev)) != MXQ_OK) return st;
+    if (nv_scale && (st = check_buffer(nv_scale, 4, dev)) != MXQ_OK) return st;
     if ((st = check_buffer(out0, out0_bytes, dev)) != MXQ_OK) return st;
     if (out1 && (st = check_buffer(out1, out1_bytes, dev)) != MXQ_OK) return st;
 
@@ -285,7 +294,7 @@ mxq_status rotate_common(const void *X, int64_t rows, int64_t cols, const void *
         if ((st = make_tmap_groups(&map_a, X, rows, cols)) != MXQ_OK) return st;
     } else {
         if ((st = make_tmap_x(&map_a, X, rows, cols)) != MXQ_OK) return st;
-        if (mode == mxq::RotOut::Quant) {
+        if (quant) {
             if ((st = make_tmap_codes(&map_c, out0, rows, cols)) != MXQ_OK) return st;
         } else {
             map_c = map_a;   // unused by the fp32 variant
@@ -295,10 +304,11 @@ mxq_status rotate_common(const void *X, int64_t rows, int64_t cols, const void *
     args.rhat = static_cast<const uint16_t *>(R);
     args.rblk = blk == 16 ? 16 : 32;
     args.lam_mul = lam_mul;
+    args.nv_scale = nv_scale;
     args.lambda = lam;
     args.rows = rows;
     args.cols = cols;
-    if (mode == mxq::RotOut::Quant) {
+    if (quant) {
         args.codes = static_cast<uint8_t *>(out0);
         args.scales = static_cast<uint8_t *>(out1);
     } else {
@@ -367,6 +377,16 @@ mxq_status mxq_weight_rotate_quantize(const void *Wt_bf16, int64_t rows, int64_t
     const uint64_t ns = rows > 0 && cols > 0 ? static_cast<uint64_t>(rows) * (cols / 32) : 0;
     return rotate_common(Wt_bf16, rows, cols, Rhat_bf16, Lambda_or_null, out_codes_u8_packed, nc, 16,
                          out_scales_e8m0, ns, mxq::RotOut::Quant, stream, 32, 1);
+}
+
+mxq_status mxq_smooth_rotate_quantize_nvfp4(const void *X_bf16, int64_t rows, int64_t cols, const void *Rhat_bf16,
+                                             const float *Lambda_or_null, const float *tensor_scale_f32,
+                                             uint8_t *out_codes_u8_packed, uint8_t *out_scales_e4m3, void *stream)
+{
+    const uint64_t nc = rows > 0 && cols > 0 ? static_cast<uint64_t>(rows) * cols / 2 : 0;
+    const uint64_t ns = rows > 0 && cols > 0 ? static_cast<uint64_t>(rows) * (cols / 16) : 0;
+    return rotate_common(X_bf16, rows, cols, Rhat_bf16, Lambda_or_null, out_codes_u8_packed, nc, 16,
+                         out_scales_e4m3, ns, mxq::RotOut::QuantNv, stream, 32, 0, tensor_scale_f32);
 }
 
 size_t mxq_scales_mma_bytes(int64_t rows, int64_t K)

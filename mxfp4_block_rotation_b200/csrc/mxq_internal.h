@@ -14,14 +14,15 @@ enum : unsigned int {
 };
 
 // Output mode of the fused rotate kernels: packed codes + scales, the rotated
-// fp32 values, or the per-group MXFP4 quantisation error (plus per-warp partial
-// sums for its mean).
-enum class RotOut { Quant, F32, Err };
+// fp32 values, the per-group MXFP4 quantisation error (plus per-warp partial
+// sums for its mean), or NVFP4 (codes + one E4M3 scale per 16 values).
+enum class RotOut { Quant, F32, Err, QuantNv };
 
 struct RotArgs {
     const uint16_t *rhat;      // bf16 [32][32], row-major [k][n]; [16][16] when rblk == 16
     int rblk;                  // 16: R^ is diag(R16, R16) built from a 16x16 input; otherwise 32
     int lam_mul;               // 1: multiply by lambda (the weights' side); 0: divide (activations)
+    const float *nv_scale;     // QuantNv: the fp32 tensor scale s_t (device, one float)
     const float *lambda;       // fp32 [cols] or nullptr
     uint8_t *codes;            // [rows, cols/2]   (Quant)
     uint8_t *scales;           // [rows, cols/32]  (Quant)

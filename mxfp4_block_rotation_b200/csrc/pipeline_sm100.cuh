@@ -175,6 +175,57 @@ __device__ __forceinline__ uint32_t quantize_group_err(const uint32_t (&r)[32], 
     return byte;
 }
 
+// NVFP4 of one 32-value group = two 16-value blocks (the public NVFP4 format; decided
+// in fp32 as r_t = 1 / (6 s_t), v = amax * r_t, s_b = E4M3(v) round to nearest even
+// saturating at 448, s = s_b * s_t, u = y * (1 / s), E2M1(u)).  Writes the 32 codes
+// packed as quantize_group does and returns the two E4M3 scale bytes (block 0 in the
+// low byte).  A block holding NaN or Inf gets 0x7F (E4M3 NaN) and codes 0; a zero
+// scale gives codes 0.
+__device__ __forceinline__ uint32_t quantize_group_nv(const uint32_t (&r)[32], uint32_t (&w)[4], float r_t, float s_t)
+{
+    float amax[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        float m[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            m[i] = ptx::fmax_nan(fabsf(__uint_as_float(r[16 * h + 2 * i])), fabsf(__uint_as_float(r[16 * h + 2 * i + 1])));
+#pragma unroll
+        for (int step = 4; step >= 1; step >>= 1)
+#pragma unroll
+            for (int i = 0; i < step; ++i) m[i] = ptx::fmax_nan(m[i], m[i + step]);
+        amax[h] = m[0];
+    }
+    uint32_t sb2;   // the two E4M3 bytes, block 0 low
+    {
+        const float v0 = __fmul_rn(amax[0], r_t), v1 = __fmul_rn(amax[1], r_t);
+        uint16_t d;
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(v1), "f"(v0));
+        sb2 = d;
+    }
+    uint32_t out = 0;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const bool bad = ((__float_as_uint(amax[h]) >> 23) & 0xFFu) == 0xFFu;
+        const uint32_t b = bad ? 0x7Fu : ((sb2 >> (8 * h)) & 0xFFu);
+        out |= b << (8 * h);
+        // E4M3 -> fp32 (exact): exponent e (bias 7), 3 mantissa bits; e = 0 is subnormal m * 2^-9
+        const uint32_t e = (b >> 3) & 15u, mm = b & 7u;
+        const float sbv = e ? __uint_as_float(((e + 120u) << 23) | (mm << 20)) : __fmul_rn(static_cast<float>(mm), 0x1p-9f);
+        const float s = __fmul_rn(sbv, s_t);
+        const bool zero = b == 0x7Fu || s == 0.0f;   // NaN scale (bad block, or v = 0 * inf)
+        const float rr = zero ? 0.0f : __frcp_rn(s);
+        float u[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) u[i] = zero ? 0.0f : __fmul_rn(__uint_as_float(r[16 * h + i]), rr);
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+            w[2 * h + q] = ptx::cvt_e2m1x8(u[8 * q], u[8 * q + 1], u[8 * q + 2], u[8 * q + 3], u[8 * q + 4],
+                                           u[8 * q + 5], u[8 * q + 6], u[8 * q + 7]);
+    }
+    return out;
+}
+
 // Sum over the warp in a fixed shuffle order (deterministic); the result is in lane 0.
 __device__ __forceinline__ double warp_sum(double v)
 {

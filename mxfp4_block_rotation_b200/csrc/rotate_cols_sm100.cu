@@ -94,6 +94,7 @@ __global__ void __launch_bounds__(kColThreads, 1)
     rotate_cols_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_codes,
                        const RotArgs args, unsigned int *status)
 {
+    constexpr bool kCodes = kMode == RotOut::Quant || kMode == RotOut::QuantNv;   // codes via staging + TMA
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align_1k(smem_raw);
     uint8_t *code_tiles = smem;                       // two 2 KB staging buffers per epilogue warp
@@ -115,7 +116,7 @@ __global__ void __launch_bounds__(kColThreads, 1)
 
     const uint32_t tmem_base =
         kernel_setup(bars, SetupCfg{kColStages, kColAcc, 1, kColBuildWarps * 32, kMmaWarp}, &tmap_x,
-                     kMode == RotOut::Quant ? &tmap_codes : nullptr);
+                     kCodes ? &tmap_codes : nullptr);
 
     if (warp == kTmaWarp) {
         if (lane == 0) {
@@ -252,7 +253,15 @@ __global__ void __launch_bounds__(kColThreads, 1)
     } else {
         const int q = warp & 3;
         const int ewg = warp >> 2;
+        // NVFP4: the tensor scale s_t and r_t = 1 / (6 s_t), once per thread
+        float nv_st = 0.0f, nv_rt = 0.0f;
+        if constexpr (kMode == RotOut::QuantNv) {
+            nv_st = *args.nv_scale;
+            nv_rt = __frcp_rn(__fmul_rn(6.0f, nv_st));
+        }
         const bool scale_vec = (G % 2 == 0) && ((reinterpret_cast<uintptr_t>(args.scales) & 1) == 0);
+        // NVFP4 scales are 2 bytes per group: a tile's 4 bytes go as one word when aligned
+        const bool nv_vec = (G % 2 == 0) && ((reinterpret_cast<uintptr_t>(args.scales) & 3) == 0);
         // Each warp stages its own 32 rows' codes (32 rows x 32 B, plain layout, two buffers)
         // and stores them with its own TMA store, so the warps of a group never wait for one another.
         const uint32_t wbuf0 = ptx::smem_addr(code_tiles + warp * 2 * kWarpCodeBytes);
@@ -263,7 +272,7 @@ __global__ void __launch_bounds__(kColThreads, 1)
             if (lane == 0) {
                 ok = wait_bar(&bars->acc_full[a], (it / kColAcc) & 1, abort, status);
                 // this warp's next staging buffer must have been read by the store that used it
-                if constexpr (kMode == RotOut::Quant) ptx::bulk_wait_group_read1();
+                if constexpr (kCodes) ptx::bulk_wait_group_read1();
             }
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
             ptx::tc_fence_after();
@@ -310,6 +319,14 @@ __global__ void __launch_bounds__(kColThreads, 1)
                         if (args.err) args.err[row * G + g] = e;
                         err_acc += static_cast<double>(e);
                     }
+                } else if constexpr (kMode == RotOut::QuantNv) {
+                    uint32_t w[4];
+                    const uint32_t bytes = quantize_group_nv(cur, w, nv_rt, nv_st);
+                    ptx::st_shared_v4(wbuf + lane * (kColTileG * 16) + j * 16, w[0], w[1], w[2], w[3]);
+                    if (nv_vec)
+                        sc_word |= bytes << (16 * j);
+                    else if (g < G && row_ok)
+                        reinterpret_cast<uint16_t *>(args.scales)[row * G + g] = static_cast<uint16_t>(bytes);
                 } else {
                     uint32_t w[4];
                     const uint32_t byte = quantize_group(cur, w);
@@ -327,10 +344,15 @@ __global__ void __launch_bounds__(kColThreads, 1)
                 const double sum = warp_sum(err_acc);
                 if (lane == 0) args.partials[(static_cast<int64_t>(rtile) * n_ct + ctile) * 4 + q] = sum;
             }
-            if constexpr (kMode == RotOut::Quant) {
-                if (scale_vec && row_ok)
+            if constexpr (kCodes) {
+                if constexpr (kMode == RotOut::QuantNv) {
+                    // two groups x two E4M3 bytes: 4 bytes at group 2 ctile of the row
+                    if (nv_vec && row_ok)
+                        reinterpret_cast<uint32_t *>(args.scales)[(row * G) / 2 + ctile] = sc_word;
+                } else if (scale_vec && row_ok) {
                     *reinterpret_cast<uint16_t *>(args.scales + row * G + static_cast<int64_t>(ctile) * kColTileG) =
                         static_cast<uint16_t>(sc_word);
+                }
                 // this warp's 32 rows complete -> one bulk store (rows/columns past the tensor are clipped)
                 ptx::fence_proxy_async_smem();
                 __syncwarp();
@@ -341,7 +363,7 @@ __global__ void __launch_bounds__(kColThreads, 1)
                 ++n_st;
             }
         }
-        if constexpr (kMode == RotOut::Quant) {
+        if constexpr (kCodes) {
             if (lane == 0) ptx::bulk_wait_group0();   // stores done before the CTA's shared memory goes
         }
     }
@@ -365,6 +387,9 @@ cudaError_t launch_rotate_cols(const CUtensorMap &tmap_x, const CUtensorMap &tma
                           tmap_codes, args, status);
     if (mode == RotOut::Err)
         return launch_pdl(rotate_cols_kernel<RotOut::Err>, grid, kColThreads, kColSmemBytes, stream, tmap_x,
+                          tmap_codes, args, status);
+    if (mode == RotOut::QuantNv)
+        return launch_pdl(rotate_cols_kernel<RotOut::QuantNv>, grid, kColThreads, kColSmemBytes, stream, tmap_x,
                           tmap_codes, args, status);
     return launch_pdl(rotate_cols_kernel<RotOut::F32>, grid, kColThreads, kColSmemBytes, stream, tmap_x, tmap_codes,
                       args, status);

@@ -118,6 +118,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         const int q = warp & 3;       // TMEM lane quarter this warp may access
         const int ewg = warp >> 2;    // which half of the stages this warp group takes
+        // NVFP4: the tensor scale s_t and r_t = 1 / (6 s_t), once per thread
+        float nv_st = 0.0f, nv_rt = 0.0f;
+        if constexpr (kMode == RotOut::QuantNv) {
+            nv_st = *args.nv_scale;
+            nv_rt = __frcp_rn(__fmul_rn(6.0f, nv_st));
+        }
         int it = 0;
         for (int c = blockIdx.x; c < n_chunks; c += gridDim.x, ++it) {
             if ((it & 1) != ewg) continue;
@@ -153,6 +159,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         quantize_group_err(cur, w, e);
                         if (args.err) args.err[g] = e;
                         err_acc += static_cast<double>(e);
+                    } else if constexpr (kMode == RotOut::QuantNv) {
+                        uint32_t w[4];
+                        const uint32_t bytes = quantize_group_nv(cur, w, nv_rt, nv_st);
+                        ptx::st_global_v4(args.codes + g * 16, w[0], w[1], w[2], w[3]);
+                        reinterpret_cast<uint16_t *>(args.scales)[g] = static_cast<uint16_t>(bytes);
                     } else {
                         uint32_t w[4];
                         const uint32_t byte = quantize_group(cur, w);
@@ -193,6 +204,9 @@ cudaError_t launch_rotate_flat(const CUtensorMap &tmap_groups, const RotArgs &ar
     if (mode == RotOut::Err)
         return launch_pdl(rotate_flat_kernel<RotOut::Err>, grid, kThreads, kFlatSmemBytes, stream, tmap_groups, args,
                           status);
+    if (mode == RotOut::QuantNv)
+        return launch_pdl(rotate_flat_kernel<RotOut::QuantNv>, grid, kThreads, kFlatSmemBytes, stream, tmap_groups,
+                          args, status);
     return launch_pdl(rotate_flat_kernel<RotOut::F32>, grid, kThreads, kFlatSmemBytes, stream, tmap_groups, args,
                       status);
 }

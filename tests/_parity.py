@@ -88,3 +88,47 @@ def check_f32(y_oracle, y_gpu, rel=2e-3):
         r, c = np.argwhere(bad)[0]
         raise AssertionError(f"fp32 rotated value off at ({r},{c}): gpu {y_gpu[r, c]!r} oracle {y_oracle[r, c]!r}")
     return float((err / np.maximum(tol, 1e-300)).max()) * rel
+
+
+def check_nvfp4(x_bits, rhat_bits, lam, s_t, gpu_codes, gpu_scales, exact=False, threads=None):
+    """NVFP4 variant of check_quant: blocks of 16 with E4M3 scales (the oracle's NVFP4 reading).
+
+    A block scale may differ only where the oracle flags v = amax * r_t as within 2.5e-4 of an
+    E4M3 rounding midpoint and the GPU took the code on the other side; such a block's codes are
+    then checked against the oracle under the GPU's scale.  Codes may differ only inside the
+    E2M1 rounding band, to the neighbouring code; the total is at most 1e-5 of the elements."""
+    threads = threads or oracle.default_threads()
+    ref = oracle.nvfp4_quantize(x_bits, rhat_bits, lam, s_t, want_y=True, flags=True, threads=threads)
+    rows, cols = x_bits.shape
+    gpu_codes = np.asarray(gpu_codes, np.uint8)
+    gpu_scales = np.asarray(gpu_scales, np.uint8)
+    assert gpu_codes.shape == ref["codes"].shape and gpu_scales.shape == ref["scales"].shape
+    sc_diff = gpu_scales != ref["scales"]
+    bad_sc = sc_diff & ~((ref["bflags"] == 1) & (gpu_scales == ref["alt_scales"]))
+    if bad_sc.any():
+        r, b = np.argwhere(bad_sc)[0]
+        raise AssertionError(f"E4M3 scale mismatch outside the band at row {r} block {b}: gpu "
+                             f"{gpu_scales[r, b]:#x} oracle {ref['scales'][r, b]:#x} "
+                             f"(y={ref['y'][r, 16 * b:16 * b + 16]})")
+    gc = oracle.unpack_codes(gpu_codes)
+    rc = oracle.unpack_codes(ref["codes"])
+    diff = (gc != rc) & np.repeat(~sc_diff, 16, axis=1)
+    bad = diff & ~((ref["eflags"] == 1) & (gc == ref["alt"]))
+    if bad.any():
+        r, c = np.argwhere(bad)[0]
+        raise AssertionError(f"NVFP4 code mismatch outside the band at row {r} col {c}: gpu {gc[r, c]:#x} "
+                             f"oracle {rc[r, c]:#x} alt {ref['alt'][r, c]:#x} y={ref['y'][r, c]!r} "
+                             f"scale={ref['scales'][r, c // 16]:#x}")
+    n_alt = 0
+    for r, b in np.argwhere(sc_diff):
+        n_alt += 1
+        codes, flags, alt = oracle.nvfp4_block_at(ref["y"][r, 16 * b:16 * b + 16], int(gpu_scales[r, b]), s_t)
+        got = gc[r, 16 * b:16 * b + 16]
+        if not ((got == codes) | ((flags == 1) & (got == alt))).all():
+            raise AssertionError(f"block at row {r} block {b} under the neighbouring scale does not match")
+    n_excused = int(diff.sum()) + 16 * n_alt
+    if exact:
+        assert n_excused == 0, f"{int(diff.sum())} code and {n_alt} scale differences where exact was required"
+    assert n_excused <= 1e-5 * rows * cols, f"{n_excused} boundary differences > 1e-5 of {rows * cols}"
+    return {"elements": rows * cols, "code_boundary_diffs": int(diff.sum()), "scale_boundary_diffs": n_alt,
+            "ref": ref}

@@ -140,3 +140,19 @@ def test_block_variant_rejects_bad_arguments(L):
     assert L.mxq_last_cuda_error().startswith(b"invalid argument")
     assert q(0, 128, 128) == 0 and q(4, 0, 64) == 0     # empty: nothing to do
     assert L.mxq_rotate_block_f32(P(a), 4, 96, 64, P(a * 5), None, P(a * 2), None) == INVALID
+
+
+def test_nvfp4_rejects_bad_arguments(L):
+    a = 0x100000
+
+    def nv(x, rows, cols, r, lam, st, codes, scales):
+        return L.mxq_smooth_rotate_quantize_nvfp4(P(x), rows, cols, P(r), P(lam), P(st), P(codes), P(scales), None)
+
+    assert nv(a, 0, 64, a * 5, None, None, None, None) == 0                      # nothing to do
+    assert nv(a, 4, 48, a * 5, None, a * 7, a * 2, a * 3) == INVALID            # cols not a multiple of 32
+    assert nv(a, 4, 64, a * 5, None, None, a * 2, a * 3) == INVALID             # no tensor scale
+    assert nv(a, 4, 64, a * 5, None, a * 7 + 2, a * 2, a * 3) == INVALID        # tensor scale not 4-B aligned
+    assert nv(a, 4, 64, a * 5, None, a * 7, a * 2, a * 3 + 1) == INVALID        # scales at an odd address
+    assert nv(a, 4, 64, a * 5, None, a * 7, a * 2, None) == INVALID             # no scales
+    assert nv(a, 4, 64, a * 5, None, a * 2 + 4, a * 2, a * 3) == INVALID        # tensor scale inside the codes
+    assert L.mxq_last_cuda_error().startswith(b"invalid argument")
