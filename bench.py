@@ -404,6 +404,18 @@ def run_extras(mxq, w, xs, rhat, outs, dev, stream, k=300):
         row(f"rotate_quantize_block{blk}", _timed(quant_blk, k, stream, dev), algorithmic_bytes(rows, cols),
             f"rotation blocks of {blk} columns, MXFP4 groups of 32 "
             f"({'rotate_flat_kernel with diag(R16, R16)' if blk == 16 else 'rotate_block_kernel'})")
+    # the NVFP4 variant (16-value blocks, E4M3 block scales, an fp32 tensor scale on the device)
+    nv_scales = [torch.empty((rows, cols // 16), dtype=torch.uint8, device=dev) for _ in range(2)]
+    s_t = torch.tensor([float(w.x.abs().max().float()) * 32 ** 0.5 / (6 * 448)], dtype=torch.float32, device=dev)
+    nv_bytes = rows * cols * (2.0 + 0.5 + 1.0 / 16.0) + 32 * 32 * 2 + 4
+    for name, lam_nv, kern in (("nvfp4_rotate_quantize", None, "rotate_flat_kernel"),
+                               ("nvfp4_rotate_quantize_with_lambda", lam, "rotate_cols_kernel")):
+        def quant_nv(i, lam_nv=lam_nv):
+            mxq.smooth_rotate_quantize_nvfp4(xs[i & 1], rhat, s_t, lam_nv, codes=outs[i & 1][0],
+                                             scales=nv_scales[i & 1], stream=stream)
+        row(name, _timed(quant_nv, k, stream, dev), nv_bytes + (4 * cols if lam_nv is not None else 0),
+            f"NVFP4: blocks of 16, E4M3 scales [rows, cols/16], fp32 tensor scale ({kern})")
+    del nv_scales
     # the consumer GEMM of the down-projection: MXFP4(X R) [8192 x 14336] times the absorbed weight
     # MXFP4(W^T R) [4096 x 14336] (synthetic N(0, 1/K) weight), bf16 out, on the block-scaled tensor cores
     n_out = 4096
