@@ -327,9 +327,15 @@ def run_mine(args):
             threads = host_cores()
             gbs, n_el, sec = oracle_rate(synth.bf16_bits(w.x), synth.bf16_bits(w.rhat), args.cpu_seconds,
                                          threads)
+            # the same at one thread (a fifth of the time budget), for the per-core rate
+            gbs1, n_el1, sec1 = oracle_rate(synth.bf16_bits(w.x), synth.bf16_bits(w.rhat),
+                                            max(1.0, args.cpu_seconds / 5), 1)
             line["cpu_baseline"] = {"value": gbs, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                    "elements_per_s": n_el / sec,
                                     "sample": f"{n_el} elements (leading rows of the workload, whole "
-                                              f"passes repeated) in {sec:.1f} s of oracle time"}
+                                              f"passes repeated) in {sec:.1f} s of oracle time",
+                                    "one_thread": {"value": gbs1, "unit": UNIT, "elements_per_s": n_el1 / sec1,
+                                                   "sample": f"{n_el1} elements in {sec1:.1f} s"}}
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()
@@ -458,6 +464,28 @@ def run_extras(mxq, w, xs, rhat, outs, dev, stream, k=300):
         "what": "greedy Givens search for R^ on X / Lambda (worst group by column maxima, 128 steps, 64 angles)",
         "ms": ms, "steps": int(found["out"]["steps"]), "launches": 2 * 128 + 6,
         "bound": "latency: two dependent launches per step"}
+    # §4.1 / Figure 1 on the synthetic activations: the mean per-group MXFP4 error under the identity,
+    # a random-sign Hadamard, a random orthogonal R and the searched R (on X / Lambda: the searched
+    # R's own target) -- the write-up's comparison, on the down-proj and QKV-input shapes
+    fig1 = {}
+    qkv = synth.make_config(2)
+    for name, xw in (("down_proj", xs[0]), ("qkv_input", qkv.x.to(dev))):
+        lam_w = synth.smoothing_scale(w.x if name == "down_proj" else qkv.x).to(dev)
+        mats = {"identity": synth.rhat_tensor(np.eye(32)).to(dev),
+                "hadamard_random_signs": synth.rhat_tensor(synth.hadamard_rhat(5)).to(dev),
+                "random_orthogonal": synth.rhat_tensor(synth.haar_orthogonal(6)).to(dev)}
+        fig1[name] = {}
+        for key, lam_k in (("no_smoothing", None), ("smoothed", lam_w)):
+            # the searched R is found on the very input it rotates (X, or X / Lambda)
+            mats["searched_K128"] = mxq.rotation_search(xw, lam_k, max_steps=128, n_angle=32, stream=stream)["rhat"]
+            fig1[name][key] = {}
+            for rn, rm in mats.items():
+                _, mean = mxq.quant_error(xw, rm, lam_k, per_group=False, stream=stream)
+                fig1[name][key][rn] = float(mean.item())
+        del xw
+    res["figure1_mean_group_error"] = {
+        "what": "mean over groups of ||Q(y) - y|| / ||y|| (MXFP4), y = X Lambda^-1 R; the searched R is found "
+                "on the same X (or X / Lambda), K = 128, 64 angles", **fig1}
     mxq.sync_check()
     return res
 

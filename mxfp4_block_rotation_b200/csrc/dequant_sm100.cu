@@ -6,8 +6,9 @@
 // (two significant bits, fp32's exponent range), so the output is exact; a
 // scale byte 0xFF gives NaN and values past bf16's range give +-Inf.
 //
-// One thread per 8 outputs: it loads 4 code bytes and its group's scale byte
-// and looks each code byte up in a 256-entry shared-memory table.  The table
+// A thread takes 8 outputs at a time (four such chunks per pass, their loads
+// issued together): it loads 4 code bytes and the group's scale byte and looks
+// each code byte up in a 256-entry shared-memory table.  The table
 // holds the bf16 pair of the byte's two E2M1 values (low nibble = even column).
 // One packed bf16x2 multiply by 2^e then gives two outputs at once.  The warp
 // reads 128 contiguous code bytes and writes 512 contiguous output bytes.
@@ -23,6 +24,7 @@ namespace mxq {
 namespace {
 
 constexpr int kPlainThreads = 256;
+constexpr int kPlainUnroll = 4;   // chunks per thread per pass
 
 // bf16 bit pattern of the E2M1 value of a 4-bit code (bit 3 = sign).
 __device__ __forceinline__ uint32_t e2m1_bf16_bits(uint32_t code)
@@ -57,18 +59,36 @@ __global__ void __launch_bounds__(kPlainThreads)
         lut[i] = e2m1_bf16_bits(static_cast<uint32_t>(i) & 15u) | (e2m1_bf16_bits(static_cast<uint32_t>(i) >> 4) << 16);
     __syncthreads();
     const int64_t stride = static_cast<int64_t>(gridDim.x) * kPlainThreads;
-    for (int64_t t = static_cast<int64_t>(blockIdx.x) * kPlainThreads + threadIdx.x; t < n_chunks; t += stride) {
-        const uint32_t c = __ldcs(codes4 + t);                       // 8 codes
-        const __nv_bfloat162 s2 = e8m0_bf16x2(__ldg(scales + (t >> 2)));   // 4 chunks per group
-        uint32_t o[4];
+    // kPlainUnroll chunks per pass, all loads issued before any use: the code reads are
+    // small (4 B a lane), so several must be in flight per thread to cover DRAM latency
+    for (int64_t t0 = static_cast<int64_t>(blockIdx.x) * kPlainThreads + threadIdx.x; t0 < n_chunks;
+         t0 += stride * kPlainUnroll) {
+        uint32_t c[kPlainUnroll], sb[kPlainUnroll];
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            const uint32_t pair = lut[(c >> (8 * b)) & 0xFFu];
-            __nv_bfloat162 v = __halves2bfloat162(__ushort_as_bfloat16(static_cast<unsigned short>(pair & 0xFFFFu)),
-                                                  __ushort_as_bfloat16(static_cast<unsigned short>(pair >> 16)));
-            o[b] = bf162_bits(__hmul2(v, s2));   // exact: a power-of-two scaling of a 2-bit significand
+        for (int u = 0; u < kPlainUnroll; ++u) {
+            const int64_t t = t0 + u * stride;
+            c[u] = 0u;
+            sb[u] = 0u;
+            if (t < n_chunks) {
+                c[u] = __ldcs(codes4 + t);                 // 8 codes
+                sb[u] = __ldg(scales + (t >> 2));          // 4 chunks per group
+            }
         }
-        __stcs(out + t, make_uint4(o[0], o[1], o[2], o[3]));
+#pragma unroll
+        for (int u = 0; u < kPlainUnroll; ++u) {
+            const int64_t t = t0 + u * stride;
+            if (t >= n_chunks) break;
+            const __nv_bfloat162 s2 = e8m0_bf16x2(sb[u]);
+            uint32_t o[4];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const uint32_t pair = lut[(c[u] >> (8 * b)) & 0xFFu];
+                __nv_bfloat162 v = __halves2bfloat162(__ushort_as_bfloat16(static_cast<unsigned short>(pair & 0xFFFFu)),
+                                                      __ushort_as_bfloat16(static_cast<unsigned short>(pair >> 16)));
+                o[b] = bf162_bits(__hmul2(v, s2));   // exact: a power-of-two scaling of a 2-bit significand
+            }
+            __stcs(out + t, make_uint4(o[0], o[1], o[2], o[3]));
+        }
     }
 }
 
