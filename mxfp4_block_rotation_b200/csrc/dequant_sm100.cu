@@ -99,7 +99,7 @@ using namespace pipe;
 // out = (v * R^T) * Lambda, v = E2M1(code) * 2^e.
 // The same flat group-major pipeline as rotate_flat_kernel, run backwards.
 //   warp 13     TMA: bulk-copies each stage's codes (512 groups x 16 B = 8 KB, contiguous)
-//               into a 4-deep shared-memory ring
+//               into a 3-deep shared-memory ring
 //   warps 4-11  decoders (two per scheduler): each lane takes one group per pass, reads its 16 code bytes
 //               from the ring, decodes them with byte permutes (no table, so no bank
 //               conflicts), scales by 2^e and writes the MMA's A tile (bf16, 64-byte
@@ -110,13 +110,18 @@ using namespace pipe;
 //   warps 0-3   epilogue, one per TMEM lane quarter, every stage: times Lambda_k, bf16,
 //               per-warp 2 KB TMA stores
 
-// The warp split depends on the smoothing: without Lambda the decoders are the
-// critical path (4 epilogue warps, 8 decoders measured best: 86 us against 104 us);
-// with Lambda the epilogue is (8 epilogue warps in two groups taking alternate
-// stages, 4 decoders).  Both use 14 warps.
-template <bool kLambda>
+// Lambda reaches the epilogue in one of two ways.  When all of it fits 64 KB (cols <=
+// 16384) and is 16-byte aligned it is copied into shared memory once per CTA; each
+// lane then reads its group's 32 channels from there (the group's row in Lambda
+// viewed as [G][32] is its index mod G).  Otherwise each epilogue warp fetches the
+// Lambda rows of its 32 groups per MMA into a double buffer (the rows of one
+// 128-group MMA hold 128 consecutive column groups, so this is 128 B per group from
+// L2).  The warp split: 4 epilogue warps and 8 decoders, except with per-warp
+// fetches, whose epilogue is the critical path (8 epilogue warps in two groups
+// taking alternate stages, 4 decoders).  All use 14 warps.
+template <int kLam>
 struct DqSplit {
-    static constexpr int kEpi = kLambda ? 8 : 4;
+    static constexpr int kEpi = kLam == 1 ? 8 : 4;
     static constexpr int kDec0 = kEpi;
     static constexpr int kDec = 12 - kEpi;
 };
@@ -131,15 +136,21 @@ constexpr int kDqCodeBytes = kDqStageGroups * 16;   // 8 KB of codes per stage
 constexpr int kDqAcc = 4;
 constexpr int kDqAccCols = 128;
 constexpr int kDqOutBuf = 32 * 64;                 // one epilogue warp's 32 output groups (2 KB)
-constexpr int kDqOutBufs = 2;                      // staging buffers per epilogue warp
+constexpr int kDqOutBufs = 2;                      // staging buffers per epilogue warp (4 measured no faster)
 __host__ __device__ constexpr int dq_out_bytes(int epi) { return epi * kDqOutBufs * kDqOutBuf; }
-__host__ __device__ constexpr int dq_lam_bytes(int epi) { return epi * 2 * 32 * 128; }   // per warp: Lambda of 32 groups, double-buffered
-__host__ __device__ constexpr int dq_smem_bytes(int epi)
+// Lambda space: per warp, the rows of 32 groups double-buffered; or the whole resident table
+__host__ __device__ constexpr int dq_lam_bytes(int epi, int lam)
 {
-    return kDqStages * kDqStageBytes + kBMatBytes + kDqCStages * kDqCodeBytes + dq_out_bytes(epi) + dq_lam_bytes(epi) +
+    return lam == 2 ? 512 * 128 : (lam == 1 ? epi * 2 * 32 * 128 : 0);
+}
+__host__ __device__ constexpr int dq_smem_bytes(int epi, int lam)
+{
+    return kDqStages * kDqStageBytes + kBMatBytes + kDqCStages * kDqCodeBytes + dq_out_bytes(epi) + dq_lam_bytes(epi, lam) +
            512 + 128 + 1024;
 }
-static_assert(dq_smem_bytes(8) <= 232448 && dq_smem_bytes(4) <= 232448, "shared memory budget");
+static_assert(dq_smem_bytes(DqSplit<0>::kEpi, 0) <= 232448 && dq_smem_bytes(DqSplit<1>::kEpi, 1) <= 232448 &&
+                  dq_smem_bytes(DqSplit<2>::kEpi, 2) <= 232448,
+              "shared memory budget");
 static_assert(kEpiWarps / 2 == 4, "acc_empty completes with four arrivals: one epilogue warp per lane quarter");
 
 __device__ __forceinline__ uint32_t hmul2_bits(uint32_t a, __nv_bfloat162 s)
@@ -151,7 +162,10 @@ __device__ __forceinline__ uint32_t hmul2_bits(uint32_t a, __nv_bfloat162 s)
            (static_cast<uint32_t>(__bfloat16_as_ushort(__high2bfloat16(r))) << 16);
 }
 
-template <bool kLambda>
+// kLam: 0 no Lambda; 1 Lambda rows fetched per warp and MMA (any width); 2 all of Lambda
+// resident in shared memory for the whole kernel (G <= kDqLamTableRows, 16-byte aligned).
+constexpr int kDqLamTableRows = 512;   // 64 KB: cols <= 16384
+template <int kLam>
 __global__ void __launch_bounds__(kDqThreads, 1)
     dequant_rot_kernel(const __grid_constant__ CUtensorMap tmap_out, const uint4 *__restrict__ codes,
                        const uint8_t *__restrict__ scales, int64_t n_groups, int64_t G,
@@ -161,10 +175,11 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     uint8_t *stages = align_1k(smem_raw);
     uint8_t *bmat = stages + kDqStages * kDqStageBytes;
     uint8_t *cring = bmat + kBMatBytes;                                  // codes ring
-    using W = DqSplit<kLambda>;
+    constexpr bool kLambda = kLam != 0;
+    using W = DqSplit<kLam>;
     uint8_t *outbuf = cring + kDqCStages * kDqCodeBytes;                 // epilogue staging
     uint8_t *lambuf = outbuf + dq_out_bytes(W::kEpi);                    // epilogue Lambda rows
-    Bars *bars = reinterpret_cast<Bars *>(lambuf + dq_lam_bytes(W::kEpi));
+    Bars *bars = reinterpret_cast<Bars *>(lambuf + dq_lam_bytes(W::kEpi, kLam));
     uint64_t *c_full = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(bars) + 512);
     uint64_t *c_empty = c_full + kDqCStages;
     volatile int *abort = &bars->abort;
@@ -296,6 +311,18 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         const uint32_t obuf0 = ptx::smem_addr(outbuf + warp * kDqOutBufs * kDqOutBuf);
         const bool lam_vec = kLambda && ((reinterpret_cast<uintptr_t>(lambda) & 15) == 0);
         float *lrows2 = reinterpret_cast<float *>(lambuf + warp * 2 * 32 * 128);   // 2 x (32 rows x 32 channels)
+        const int Gi = static_cast<int>(G);
+        if constexpr (kLam == 2) {
+            // Lambda as [G][32] once, 16-byte chunk c of row r at chunk c ^ (r & 7): the lanes of
+            // a warp read consecutive rows (mod G), so a float4 read takes the minimum 4 wavefronts
+            for (int i = threadIdx.x; i < Gi * 8; i += W::kEpi * 32) {
+                const int r = i >> 3, cc = i & 7;
+                ptx::cp_async16(ptx::smem_addr(lambuf + r * 128 + ((cc ^ (r & 7)) << 4)), lambda + r * 32 + cc * 4);
+            }
+            ptx::cp_async_commit();
+            ptx::cp_async_wait<0>();
+            ptx::named_bar_sync(1, W::kEpi * 32);
+        }
         int it = 0, nstore = 0;
         for (int c = blockIdx.x; c < n_chunks; c += gridDim.x, ++it) {
             if (W::kEpi == 8 && (it & 1) != ewg) continue;
@@ -312,8 +339,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             // next MMA's rows are in flight while this one is processed.
             // Column groups are taken mod G by subtraction (at most one step once G >= 128): a
             // division per stage instead of nine per fetch.
-            const int Gi = static_cast<int>(G);
-            const int col_warp = kLambda ? static_cast<int>(g_warp % G) : 0;
+            const int col_warp = kLam == 1 ? static_cast<int>(g_warp % G) : 0;
+            const int row_lane = kLam == 2 ? static_cast<int>((g_warp + lane) % G) : 0;   // Lambda row of MMA 0
             auto fetch_lambda = [&](int j) {
                 int col0 = col_warp + j * 128;
                 while (col0 >= Gi) col0 -= Gi;
@@ -336,7 +363,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                 }
                 ptx::cp_async_commit();
             };
-            if constexpr (kLambda) {
+            if constexpr (kLam == 1) {
                 __syncwarp();   // the previous stage's reads of both buffers are done
                 fetch_lambda(0);
             }
@@ -347,7 +374,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                 ptx::tmem_ld_32cols(t_row + j * 32, cur);
                 const int64_t g0 = g_warp + j * 128;   // this warp's first group of MMA j
                 const float *lrows = lrows2 + (j & 1) * 32 * 32;
-                if constexpr (kLambda) {
+                if constexpr (kLam == 1) {
                     if (j + 1 < 4) {
                         __syncwarp();   // every lane is done reading buffer (j + 1) & 1 (MMA j - 1)
                         fetch_lambda(j + 1);
@@ -357,14 +384,18 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                     }
                     __syncwarp();
                 }
+                const int rj = kLam == 2 ? (row_lane + j * 128) % Gi : 0;   // this lane's Lambda row
+                const float *ltab = reinterpret_cast<const float *>(lambuf) + rj * 32;
                 ptx::tmem_wait_ld();
                 // times Lambda_k (channels of this group), then round to bf16 pairs
                 uint32_t o[16];
 #pragma unroll
                 for (int k4 = 0; k4 < 8; ++k4) {
                     float4 l4 = make_float4(1.0f, 1.0f, 1.0f, 1.0f);
-                    if constexpr (kLambda)
+                    if constexpr (kLam == 1)
                         l4 = *reinterpret_cast<const float4 *>(lrows + lane * 32 + ((k4 ^ (lane & 7)) << 2));
+                    else if constexpr (kLam == 2)
+                        l4 = *reinterpret_cast<const float4 *>(ltab + ((k4 ^ (rj & 7)) << 2));
                     const __nv_bfloat162 p0 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(cur[4 * k4]), l4.x),
                                                                     __fmul_rn(__uint_as_float(cur[4 * k4 + 1]), l4.y));
                     const __nv_bfloat162 p1 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(cur[4 * k4 + 2]), l4.z),
@@ -414,10 +445,16 @@ cudaError_t launch_dequant_rot(const CUtensorMap &tmap_out, const uint8_t *codes
     unsigned int *status = status_word();
     if (!status) return cudaErrorInvalidSymbol;
     const uint4 *c4 = reinterpret_cast<const uint4 *>(codes);
-    return lambda ? launch_pdl(dequant_rot_kernel<true>, grid, kDqThreads, dq_smem_bytes(8), stream, tmap_out, c4, scales,
-                               n_groups, G, rhat, lambda, status)
-                  : launch_pdl(dequant_rot_kernel<false>, grid, kDqThreads, dq_smem_bytes(4), stream, tmap_out, c4, scales,
-                               n_groups, G, rhat, lambda, status);
+    if (!lambda)
+        return launch_pdl(dequant_rot_kernel<0>, grid, kDqThreads, dq_smem_bytes(DqSplit<0>::kEpi, 0), stream, tmap_out, c4, scales,
+                          n_groups, G, rhat, lambda, status);
+    // all of Lambda fits the per-warp buffers' space (and can be copied in 16-byte pieces): keep it resident
+    if (G <= kDqLamTableRows && (reinterpret_cast<uintptr_t>(lambda) & 15) == 0)
+        return launch_pdl(dequant_rot_kernel<2>, grid, kDqThreads, dq_smem_bytes(DqSplit<2>::kEpi, 2), stream, tmap_out,
+                          c4, scales,
+                          n_groups, G, rhat, lambda, status);
+    return launch_pdl(dequant_rot_kernel<1>, grid, kDqThreads, dq_smem_bytes(DqSplit<1>::kEpi, 1), stream, tmap_out, c4, scales,
+                      n_groups, G, rhat, lambda, status);
 }
 
 cudaError_t launch_dequant_plain(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t cols,

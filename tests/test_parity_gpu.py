@@ -238,16 +238,24 @@ def test_dequant_plain_bit_exact():
     assert np.array_equal(ref[~ref_nan], got[~got_nan])
 
 
-@pytest.mark.parametrize("with_lambda", [False, True])
-def test_dequant_inverse_rotation(with_lambda):
-    rows, cols = 300, 2048
+# Lambda kinds: resident in shared memory (16-byte aligned, G <= 512), or fetched per warp
+# (G > 512, or Lambda only 4-byte aligned); a few groups per row make the row index wrap often
+@pytest.mark.parametrize("rows,cols,lam_kind", [(300, 2048, None), (300, 2048, "aligned"), (300, 2048, "offset"),
+                                                (40, 16416, "aligned"), (37, 16384, "aligned"), (129, 96, "aligned"),
+                                                (129, 96, "offset")])
+def test_dequant_inverse_rotation(rows, cols, lam_kind):
     codes, scales = _synthetic_codes(rows, cols, seed=4)
     r = synth.rhat_tensor(synth.haar_orthogonal(14))
-    lam = synth.random_lambda(cols, seed=5) if with_lambda else None
+    lam = synth.random_lambda(cols, seed=5) if lam_kind else None
     ref_bits, ref64 = oracle.dequantize(codes, scales, cols, _bits(r), None if lam is None else lam.numpy(),
                                         want_f64=True)
-    got = mxq.dequantize(torch.from_numpy(codes).to(DEV), torch.from_numpy(scales).to(DEV), r.to(DEV),
-                         None if lam is None else lam.to(DEV))
+    lam_dev = None
+    if lam_kind == "aligned":
+        lam_dev = lam.to(DEV)
+    elif lam_kind == "offset":
+        lam_dev = torch.cat([torch.zeros(1), lam]).to(DEV)[1:]   # 4-byte but not 16-byte aligned
+        assert lam_dev.data_ptr() % 16 != 0
+    got = mxq.dequantize(torch.from_numpy(codes).to(DEV), torch.from_numpy(scales).to(DEV), r.to(DEV), lam_dev)
     got64 = oracle.bf16_bits_to_f64(synth.bf16_bits(got.cpu()))
     # bound: one bf16 ulp of the exact value plus fp32 accumulation error of 32 terms
     v = oracle.bf16_bits_to_f64(oracle.dequantize(codes, scales, cols))
