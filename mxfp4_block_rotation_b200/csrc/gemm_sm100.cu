@@ -7,24 +7,35 @@
 //   Y[m][n] = sum_k deq(A)[m][k] * deq(B)[n][k],   deq = E2M1 code * 2^(E8M0 byte - 127)
 // A = the activations' codes [M, K/2] and scales [M, K/32]; B = the absorbed
 // weights, stored transposed ([N, K/2], [N, K/32]), so both are K-major, exactly
-// as the quantiser writes them.
+// as the quantiser writes them.  The scales come in the MMA's atom layout (512-byte
+// atoms of 128 rows x 4 k-blocks; row r's word at byte 16 (r % 32) + 4 (r / 32)).
 //
-// One persistent CTA per SM takes 128 x 256 output tiles.  Warp roles (320 threads):
-//   warps 0-3  epilogue: TMEM -> registers -> fp32 or bf16 stores (warp w reads lane quarter w)
-//   warp 4     TMA producer: per stage, 256 k of A (128 rows x 128 B) and B (256 rows x 128 B),
-//              128-byte swizzle, zero fill past the matrix edges, plus the stage's scale atoms
-//              (bulk copies of 512-byte atoms: 2 for A, 2 x 2 for B) on a barrier of their own
-//   warp 5     TMEM owner and MMA issuer: four tcgen05.mma kind::mxf4 block32 of K = 64 per
-//              stage, M = 128, N = 256, fp32 accumulator in TMEM columns 0-255
-//   warps 6-9  scale movers: the stage's atoms from shared memory into TMEM with tcgen05.st,
-//              in the layout the block-scaled MMA reads: the scales of row r, k-blocks
-//              4c..4c+3, form one 32-bit word in lane r % 32 (of every lane quarter) and column
-//              base + 4c + r / 32 (A; 8c + r / 32 for the 256 rows of B).  An atom (128 rows x
-//              4 k-blocks, row r's word at byte 16 (r % 32) + 4 (r / 32)) holds, in lane l's 16
-//              bytes, exactly the four words lane l stores.
+// CTA pairs (clusters of two, tcgen05 cta_group::2) share each 256 x 256 output tile:
+// CTA r holds rows 128 r .. 128 r + 127 of the tile's A and rows (n) 128 r .. 128 r + 127
+// of its B in shared memory, and its TMEM holds its 128 output rows x all 256 columns
+// plus its own scales (A: its rows; B: all 256).  The even CTA issues one M = 256,
+// N = 256, K = 64 MMA per step that reads both CTAs' tiles, so each CTA brings in only
+// half of B: 35 KB per 256-k stage (A 16 KB + B 16 KB + scale atoms 3 KB) against 51 KB
+// for a 128 x 256 tile on one CTA.  The mainloop is bound by the bytes in flight per SM
+// (six stages fill shared memory), so fewer bytes per stage is what pays.  Warp roles
+// (224 threads per CTA):
+//   warps 0-3  epilogue (both CTAs): TMEM lanes 32w.. -> fp32 or bf16 stores, then an
+//              arrival on the even CTA's acc_empty
+//   warp 4     TMA (both CTAs): per stage its A rows, its half of B, its A row block's
+//              scale atoms and both of B's row blocks' atoms, all counted on the even
+//              CTA's full[s] (tensor copies with cta_group::2, no cluster multicast)
+//   warp 5     TMEM owner (both CTAs) and, in the even CTA, the MMA issuer: four
+//              kind::mxf4 block32 MMAs per stage, fp32 accumulator in TMEM columns 0-255;
+//              it commits each stage to both CTAs' empty[s] and each tile to acc_full
+//   warp 6     scale copies (even CTA): tcgen05.cp of the stage's atoms into both CTAs'
+//              TMEM (32x128b, replicated over the four lane quarters), committed to
+//              sf_ready[s].  Issued from their own warp the copies run ahead of the MMAs;
+//              issued by the MMA thread before each stage's MMAs they cost a quarter of
+//              the time.
 // A K = 64 MMA takes two scales per row: bytes 0-1 (first half of a 128-k word) or 2-3,
 // chosen by the top two bits of the scale address and the descriptor's scale ids.
-// Every wait is bounded (2 s) and raises the status word; nothing waits on another CTA.
+// Every wait on a barrier is bounded (2 s) and raises the status word; the two CTAs
+// of a pair meet at the hardware cluster barrier only at start and end.
 #include "pipeline_sm100.cuh"
 #include "sm100_bulk.cuh"
 
@@ -34,42 +45,6 @@ namespace {
 using namespace pipe;
 
 // ------------------------------------------------------------------ PTX used only here
-
-// D (+)= A * B with per-32-k E8M0 scales (MXFP4 operands in shared memory, scales in TMEM).
-__device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                         uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %6, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
-        :
-        : "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
-        : "memory");
-}
-
-// Eight / sixteen 32-bit registers of each lane into consecutive TMEM columns of its lane.
-__device__ __forceinline__ void tmem_st_8cols(uint32_t taddr, const uint32_t (&r)[8])
-{
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
-                 :
-                 : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
-                   "r"(r[7])
-                 : "memory");
-}
-
-__device__ __forceinline__ void tmem_st_16cols(uint32_t taddr, const uint32_t (&r)[16])
-{
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-        "%14, %15, %16};"
-        :
-        : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-          "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-        : "memory");
-}
-
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Instruction descriptor, kind::mxf4 block-scaled: E2M1 A and B (format 1), UE8M0 scales,
 // both K-major, M = 128, N = 256, K = 64; scale ids (the byte pair inside a scale word) added per MMA.
@@ -82,45 +57,97 @@ __host__ __device__ constexpr uint32_t idesc_mxf4(int m, int n)
            | (static_cast<uint32_t>(m >> 4) << 24);   // M / 16
 }
 
-// ------------------------------------------------------------------ tiling
+__device__ __forceinline__ uint32_t cluster_ctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
 
-constexpr int kGM = 128;                      // tile rows (M)
-constexpr int kGN = 256;                      // tile columns (N)
-constexpr int kGK = 256;                      // k per stage (128 bytes of codes per row)
-constexpr int kGStages = 4;
-constexpr int kGAStage = kGM * 128;           // 16 KB
-constexpr int kGBStage = kGN * 128;           // 32 KB
-constexpr int kGSfStage = 3 * 1024;           // scale atoms: A 2 x 512 B, B 2 row blocks x 2 x 512 B
-constexpr int kGStageBytes = kGAStage + kGBStage + kGSfStage;   // 51 KB, a multiple of 1 KB
-constexpr int kGThreads = 10 * 32;
-constexpr int kGTmaWarp = 4;
-constexpr int kGMmaWarp = 5;
-constexpr int kGSfWarp0 = 6;
-constexpr int kGAccCols = kGN;                // fp32 accumulator: TMEM columns 0..255
-constexpr int kGSfaCols = 2 * (kGM / 32);     // per stage: two 128-k words x 4 row blocks
-constexpr int kGSfbCols = 2 * (kGN / 32);     // per stage: two 128-k words x 8 row blocks
-constexpr int kGSfCols = kGSfaCols + kGSfbCols;
-constexpr int kGSmem = kGStages * kGStageBytes + 1024 + 1024;
-static_assert(kGAccCols + kGStages * kGSfCols <= 512, "TMEM budget");
-static_assert(kGSmem <= 232448, "shared memory budget");
+// The shared::cluster address of the same variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
 
-struct GemmBars {
-    uint64_t full[kGStages];      // TMA bytes of a stage's operands landed
-    uint64_t sf_in[kGStages];     // the stage's scale atoms landed in shared memory
-    uint64_t sf_full[kGStages];   // the stage's scales are in TMEM (4 loader warps)
-    uint64_t empty[kGStages];     // the stage's MMAs are done (smem and scale columns free)
-    uint64_t acc_full;            // the tile's accumulator is complete
-    uint64_t acc_empty;           // the epilogue has read the accumulator (4 warps)
-    uint64_t drain;
-    uint32_t tmem_base;
-    int abort;
-};
-static_assert(sizeof(GemmBars) <= 1024, "barrier block");
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
 
-// TMEM columns of stage s's scales: all A words first, then all B words, so every
-// tcgen05.st starts on a multiple of its width.
-__device__ __forceinline__ uint32_t sfa_col(int s) { return kGAccCols + s * kGSfaCols; }
-__device__ __forceinline__ uint32_t sfb_col(int s) { return kGAccCols + kGStages * kGSfaCols + s * kGSfbCols; }
+// A tile of this CTA's operand into its own shared memory; the bytes count on the
+// mbarrier at bar_cluster (the even CTA's).  No cluster multicast.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, int32_t x, int32_t y,
+                                                 uint32_t bar_cluster, uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cluster), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_mxf4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+        :
+        : "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive on the mbarrier at bar_cluster (either CTA's) once the pair MMAs issued so far are done.
+__device__ __forceinline__ void commit_pair(uint32_t bar_cluster)
+{
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar_cluster)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_slot, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_slot), "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair()
+{
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// tcgen05.cp of one 512-byte scale atom (32 rows of 16 B) into TMEM, four columns from
+// taddr, replicated over the four lane quarters, in both CTAs of the pair (each from its
+// own shared memory at the same offset).
+__device__ __forceinline__ void tmem_cp_atom_pair(uint32_t taddr, uint64_t sdesc)
+{
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Shared-memory descriptor of a scale atom for tcgen05.cp: no swizzle, 8-row core
+// matrices of 16-byte rows, 128 B apart (stride byte offset); one core matrix along K.
+__device__ __forceinline__ uint64_t smem_desc_atom(uint32_t saddr)
+{
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFF);   // start address, 16-B units
+    d |= static_cast<uint64_t>(128 >> 4) << 16;           // leading byte offset (one core matrix: unused)
+    d |= static_cast<uint64_t>(128 >> 4) << 32;           // stride byte offset: next 8 rows
+    d |= static_cast<uint64_t>(1) << 46;                  // descriptor version (sm100)
+    return d;                                             // layout 0: no swizzle
+}
 
 __device__ __forceinline__ uint64_t policy_evict_last()
 {
@@ -129,231 +156,264 @@ __device__ __forceinline__ uint64_t policy_evict_last()
     return pol;
 }
 
-__global__ void __launch_bounds__(kGThreads, 1)
+// 32 accumulator columns of one output row (col0 < N) as bf16 or fp32: 16-byte stores
+// when the row's chunk is whole and aligned, element stores at the right edge.
+__device__ __forceinline__ void store_row_chunk(const GemmArgs &args, int64_t row, int64_t col0, const uint32_t (&cur)[32],
+                                                bool vec)
+{
+    if (args.out_bf16) {
+        uint16_t *dst = static_cast<uint16_t *>(args.y) + row * args.N + col0;
+        if (vec && col0 + 32 <= args.N) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    w[e] = pack_bf16x2(__float2bfloat16_rn(__uint_as_float(cur[8 * i + 2 * e])),
+                                       __float2bfloat16_rn(__uint_as_float(cur[8 * i + 2 * e + 1])));
+                ptx::st_global_v4(dst + 8 * i, w[0], w[1], w[2], w[3]);
+            }
+        } else {
+            for (int i = 0; i < 32 && col0 + i < args.N; ++i)
+                dst[i] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(cur[i])));
+        }
+    } else {
+        float *dst = static_cast<float *>(args.y) + row * args.N + col0;
+        if (vec && col0 + 32 <= args.N) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                ptx::st_global_v4(dst + 4 * i, cur[4 * i], cur[4 * i + 1], cur[4 * i + 2], cur[4 * i + 3]);
+        } else {
+            for (int i = 0; i < 32 && col0 + i < args.N; ++i) dst[i] = __uint_as_float(cur[i]);
+        }
+    }
+}
+
+constexpr int kGK = 256;                      // k per stage (128 bytes of codes per row)
+constexpr int kGTmaWarp = 4;
+constexpr int kGMmaWarp = 5;
+constexpr int kGAccCols = 256;                // fp32 accumulator: TMEM columns 0..255
+
+constexpr int kPM = 256;                      // pair tile rows (128 per CTA)
+constexpr int kPN = 256;                      // pair tile columns
+constexpr int kPStages = 6;
+constexpr int kPAStage = 128 * 128;           // this CTA's 128 rows x 256 k: 16 KB
+constexpr int kPBStage = 128 * 128;           // this CTA's half of B: 16 KB
+constexpr int kPSfStage = 3 * 1024;           // A: 2 atoms of its row block; B: 2 row blocks x 2 atoms
+constexpr int kPStageBytes = kPAStage + kPBStage + kPSfStage;   // 35 KB
+constexpr int kPTx = 2 * kPStageBytes;        // bytes a stage brings into the pair
+constexpr int kPSmem = kPStages * kPStageBytes + 1024 + 1024;
+constexpr int kPThreads = 7 * 32;             // warps 0-3 epilogue, 4 TMA, 5 MMA, 6 scale copies
+constexpr int kPCpWarp = 6;
+constexpr int kPSfaCols = 2 * (128 / 32);     // per stage: two 128-k words x 4 row blocks
+constexpr int kPSfbCols = 2 * (kPN / 32);     // two 128-k words x 8 row blocks
+static_assert(kGAccCols + kPStages * (kPSfaCols + kPSfbCols) <= 512, "TMEM budget (pairs)");
+static_assert(kPSmem <= 232448, "shared memory budget (pairs)");
+
+struct PairBars {
+    uint64_t full[kPStages];      // even CTA: both CTAs' operand and scale bytes of a stage landed
+    uint64_t empty[kPStages];     // the stage's pair MMAs are done (from the even CTA's commit)
+    uint64_t sf_ready[kPStages];  // even CTA: the stage's scales have been copied into both CTAs' TMEM
+    uint64_t acc_full;            // the tile's accumulator is complete (from the even CTA's commit)
+    uint64_t acc_empty;           // even CTA: both CTAs' epilogues have read the accumulator (8 warps)
+    uint64_t drain;
+    uint64_t cp_drain;
+    uint32_t tmem_base;
+    int abort;
+};
+static_assert(sizeof(PairBars) <= 1024, "barrier block (pairs)");
+
+__device__ __forceinline__ uint32_t psfa_col(int s) { return kGAccCols + s * kPSfaCols; }
+__device__ __forceinline__ uint32_t psfb_col(int s) { return kGAccCols + kPStages * kPSfaCols + s * kPSfbCols; }
+
+__global__ void __launch_bounds__(kPThreads, 1)
     mxfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                      const GemmArgs args, unsigned int *status)
+                           const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
+                           const GemmArgs args, unsigned int *status)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *stages = align_1k(smem_raw);
-    GemmBars *bars = reinterpret_cast<GemmBars *>(stages + kGStages * kGStageBytes);
+    PairBars *bars = reinterpret_cast<PairBars *>(stages + kPStages * kPStageBytes);
     volatile int *abort = &bars->abort;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int64_t tiles_n = (args.N + kGN - 1) / kGN;
-    const int64_t n_tiles = ((args.M + kGM - 1) / kGM) * tiles_n;
+    const uint32_t rank = cluster_ctarank();   // 0: the even CTA, which issues the MMAs
+    const int64_t pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+    const int64_t tiles_n = (args.N + kPN - 1) / kPN;
+    const int64_t n_tiles = ((args.M + kPM - 1) / kPM) * tiles_n;
     const int kt_n = static_cast<int>((args.K + kGK - 1) / kGK);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kGStages; ++s) {
+        for (int s = 0; s < kPStages; ++s) {
             ptx::mbar_init(ptx::smem_addr(&bars->full[s]), 1);
-            ptx::mbar_init(ptx::smem_addr(&bars->sf_in[s]), 1);
-            ptx::mbar_init(ptx::smem_addr(&bars->sf_full[s]), 4);
             ptx::mbar_init(ptx::smem_addr(&bars->empty[s]), 1);
+            ptx::mbar_init(ptx::smem_addr(&bars->sf_ready[s]), 1);
         }
         ptx::mbar_init(ptx::smem_addr(&bars->acc_full), 1);
-        ptx::mbar_init(ptx::smem_addr(&bars->acc_empty), 4);
+        ptx::mbar_init(ptx::smem_addr(&bars->acc_empty), 8);
         ptx::mbar_init(ptx::smem_addr(&bars->drain), 1);
+        ptx::mbar_init(ptx::smem_addr(&bars->cp_drain), 1);
         bars->abort = 0;
         ptx::fence_mbar_init();
         ptx::prefetch_tmap(&tmap_a);
         ptx::prefetch_tmap(&tmap_b);
+        ptx::prefetch_tmap(&tmap_sfa);
+        ptx::prefetch_tmap(&tmap_sfb);
     }
     if (warp == kGMmaWarp) {
-        ptx::tmem_alloc(ptx::smem_addr(&bars->tmem_base), kTmemCols);
-        ptx::tmem_relinquish();
+        tmem_alloc_pair(ptx::smem_addr(&bars->tmem_base), kTmemCols);
+        tmem_relinquish_pair();
     }
     ptx::griddep_launch_dependents();
     ptx::tc_fence_before();
     __syncthreads();
+    cluster_sync();   // both CTAs' barriers exist before either signals the other's
     ptx::tc_fence_after();
     const uint32_t tmem_base = bars->tmem_base;
     ptx::griddep_wait();
 
     if (warp == kGTmaWarp) {
         if (lane == 0) {
-            const uint64_t pol = policy_evict_last();   // A and B tiles are re-read by other CTAs
+            const uint64_t pol = policy_evict_last();   // A and B tiles are re-read by other pairs
             int it = 0;
             bool ok = true;
-            for (int64_t t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
-                const int tm = static_cast<int>(t / tiles_n), tn = static_cast<int>(t % tiles_n);
+            for (int64_t t = pair; ok && t < n_tiles; t += n_pairs) {
+                const int tm2 = static_cast<int>(t / tiles_n), tn = static_cast<int>(t % tiles_n);
                 for (int kt = 0; kt < kt_n; ++kt, ++it) {
-                    const int s = it % kGStages;
-                    if (!wait_bar(&bars->empty[s], ((it / kGStages) & 1) ^ 1, abort, status)) {
+                    const int s = it % kPStages;
+                    if (!wait_bar(&bars->empty[s], ((it / kPStages) & 1) ^ 1, abort, status)) {
                         ok = false;
                         break;
                     }
-                    const uint32_t full = ptx::smem_addr(&bars->full[s]);
-                    const uint32_t dst = ptx::smem_addr(stages + s * kGStageBytes);
-                    // scale atoms of k-blocks 8kt..8kt+7: two atoms, or one at an odd-sized K tail
-                    const int64_t cb0 = 2 * static_cast<int64_t>(kt);
-                    const uint32_t n_at = cb0 + 1 < args.cb_n ? 2u : 1u;
-                    const int64_t rb0 = 2 * static_cast<int64_t>(tn);
-                    const uint32_t n_rb = rb0 + 1 < args.rb_b ? 2u : 1u;
-                    // the scale atoms first, on their own barrier: the scale warps can move them
-                    // into TMEM while the operand tiles are still in flight
-                    const uint32_t sfb = ptx::smem_addr(&bars->sf_in[s]);
-                    ptx::mbar_arrive_expect_tx(sfb, n_at * 512u * (1u + n_rb));
-                    const uint32_t sf = dst + kGAStage + kGBStage;
-                    ptx::bulk_load(sf, args.a_sf + (static_cast<int64_t>(tm) * args.cb_n + cb0) * 512, n_at * 512u, sfb,
-                              pol);
-                    for (uint32_t h = 0; h < n_rb; ++h)
-                        ptx::bulk_load(sf + 1024u + h * 1024u, args.b_sf + ((rb0 + h) * args.cb_n + cb0) * 512,
-                                  n_at * 512u, sfb, pol);
-                    ptx::mbar_arrive_expect_tx(full, kGAStage + kGBStage);
-                    ptx::tma_load_2d(dst, &tmap_a, kt * 128, tm * kGM, full, pol);
-                    ptx::tma_load_2d(dst + kGAStage, &tmap_b, kt * 128, tn * kGN, full, pol);
+                    const uint32_t dst = ptx::smem_addr(stages + s * kPStageBytes);
+                    const uint32_t full0 = mapa(ptx::smem_addr(&bars->full[s]), 0);
+                    if (rank == 0) ptx::mbar_arrive_expect_tx(ptx::smem_addr(&bars->full[s]), kPTx);
+                    // this CTA's A rows and half of B; its A row block's scale atoms and the atoms of
+                    // both of B's row blocks (zero past the matrices' edges)
+                    tma_load_2d_pair(dst, &tmap_a, kt * 128, tm2 * kPM + static_cast<int>(rank) * 128, full0, pol);
+                    tma_load_2d_pair(dst + kPAStage, &tmap_b, kt * 128, tn * kPN + static_cast<int>(rank) * 128, full0,
+                                     pol);
+                    tma_load_2d_pair(dst + kPAStage + kPBStage, &tmap_sfa, kt * 256, 2 * tm2 + static_cast<int>(rank),
+                                     full0, pol);
+                    tma_load_2d_pair(dst + kPAStage + kPBStage + 1024, &tmap_sfb, kt * 256, 2 * tn, full0, pol);
                 }
             }
-            // let the last copy into each stage land before the CTA can exit
-            for (int s = 0; s < kGStages && s < it; ++s) {
-                const int last = it - 1 - ((it - 1 - s) % kGStages);
-                wait_bar(&bars->full[s], (last / kGStages) & 1, nullptr, status);
-                wait_bar(&bars->sf_in[s], (last / kGStages) & 1, nullptr, status);
-            }
-        }
-    } else if (warp >= kGSfWarp0) {
-        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        int it = 0;
-        bool ok = true;
-        for (int64_t t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
-            const int64_t rb0 = 2 * (t % tiles_n);
-            for (int kt = 0; kt < kt_n; ++kt, ++it) {
-                const int s = it % kGStages;
-                // sf_in[s] is armed only after the stage's previous MMAs freed it, so the scale
-                // columns of slot s are free too
-                int w_ok = 0;
-                if (lane == 0) w_ok = wait_bar(&bars->sf_in[s], (it / kGStages) & 1, abort, status);
-                if (!__shfl_sync(0xffffffffu, w_ok, 0)) {
-                    ok = false;
-                    break;
+            // the last copies into each stage land before the CTA can exit (the even CTA's
+            // full[s] counts both CTAs' bytes; the cluster barrier at the end covers the odd CTA)
+            if (rank == 0) {
+                for (int s = 0; s < kPStages && s < it; ++s) {
+                    const int last = it - 1 - ((it - 1 - s) % kPStages);
+                    wait_bar(&bars->full[s], (last / kPStages) & 1, nullptr, status);
                 }
-                const uint32_t sf = ptx::smem_addr(stages + s * kGStageBytes + kGAStage + kGBStage) + 16u * lane;
-                uint32_t wa[8], wb[16];
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    const bool cv = 2 * static_cast<int64_t>(kt) + c < args.cb_n;
-                    const uint4 va = cv ? ptx::ld_shared_v4(sf + c * 512) : make_uint4(0, 0, 0, 0);
-                    wa[4 * c] = va.x;
-                    wa[4 * c + 1] = va.y;
-                    wa[4 * c + 2] = va.z;
-                    wa[4 * c + 3] = va.w;
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const bool v = cv && rb0 + h < args.rb_b;
-                        const uint4 vb = v ? ptx::ld_shared_v4(sf + 1024 + h * 1024 + c * 512) : make_uint4(0, 0, 0, 0);
-                        wb[8 * c + 4 * h] = vb.x;
-                        wb[8 * c + 4 * h + 1] = vb.y;
-                        wb[8 * c + 4 * h + 2] = vb.z;
-                        wb[8 * c + 4 * h + 3] = vb.w;
-                    }
-                }
-                tmem_st_8cols(tmem_base + lane_base + sfa_col(s), wa);
-                tmem_st_16cols(tmem_base + lane_base + sfb_col(s), wb);
-                tmem_wait_st();
-                ptx::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(ptx::smem_addr(&bars->sf_full[s]));
             }
         }
     } else if (warp == kGMmaWarp) {
-        if (lane == 0) {
-            constexpr uint32_t idesc0 = idesc_mxf4(kGM, kGN);
+        if (lane == 0 && rank == 0) {
+            constexpr uint32_t idesc0 = idesc_mxf4(kPM, kPN);
             int it = 0, tile_i = 0;
             bool ok = true;
-            for (int64_t t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++tile_i) {
+            for (int64_t t = pair; ok && t < n_tiles; t += n_pairs, ++tile_i) {
                 if (!wait_bar(&bars->acc_empty, (tile_i & 1) ^ 1, abort, status)) break;
                 ptx::tc_fence_after();
                 for (int kt = 0; kt < kt_n; ++kt, ++it) {
-                    const int s = it % kGStages;
-                    const uint32_t par = (it / kGStages) & 1;
-                    if (!wait_bar(&bars->full[s], par, abort, status) ||
-                        !wait_bar(&bars->sf_full[s], par, abort, status)) {
+                    const int s = it % kPStages;
+                    // full[s] then sf_ready[s] (the copy warp's copies of the stage's scales done)
+                    if (!wait_bar(&bars->full[s], (it / kPStages) & 1, abort, status) ||
+                        !wait_bar(&bars->sf_ready[s], (it / kPStages) & 1, abort, status)) {
                         ok = false;
                         break;
                     }
                     ptx::tc_fence_after();
-                    const uint32_t a_base = ptx::smem_addr(stages + s * kGStageBytes);
-                    const uint32_t b_base = a_base + kGAStage;
+                    const uint32_t a_base = ptx::smem_addr(stages + s * kPStageBytes);
+                    const uint32_t b_base = a_base + kPAStage;
 #pragma unroll
                     for (int j = 0; j < kGK / 64; ++j) {
-                        const uint32_t c = j >> 1, byte = 2u * (j & 1);   // 128-k word, byte pair in it
-                        const uint32_t sfa = (tmem_base + sfa_col(s) + 4 * c) | (byte << 30);
-                        const uint32_t sfb = (tmem_base + sfb_col(s) + 8 * c) | (byte << 30);
+                        const uint32_t c = j >> 1, byte = 2u * (j & 1);
+                        const uint32_t sfa = (tmem_base + psfa_col(s) + 4 * c) | (byte << 30);
+                        const uint32_t sfb = (tmem_base + psfb_col(s) + 8 * c) | (byte << 30);
                         const uint32_t idesc = idesc0 | (byte << 29) | (byte << 4);
-                        mma_mxf4(tmem_base, ptx::smem_desc_sw128(a_base + j * 32), ptx::smem_desc_sw128(b_base + j * 32),
-                                 idesc, sfa, sfb, static_cast<uint32_t>(kt | j));
+                        mma_mxf4_pair(tmem_base, ptx::smem_desc_sw128(a_base + j * 32),
+                                      ptx::smem_desc_sw128(b_base + j * 32), idesc, sfa, sfb,
+                                      static_cast<uint32_t>(kt | j));
                     }
-                    ptx::mma_commit(ptx::smem_addr(&bars->empty[s]));
+                    const uint32_t e = ptx::smem_addr(&bars->empty[s]);
+                    commit_pair(mapa(e, 0));
+                    commit_pair(mapa(e, 1));
                 }
                 if (!ok) break;
-                ptx::mma_commit(ptx::smem_addr(&bars->acc_full));
+                const uint32_t af = ptx::smem_addr(&bars->acc_full);
+                commit_pair(mapa(af, 0));
+                commit_pair(mapa(af, 1));
             }
-            ptx::mma_commit(ptx::smem_addr(&bars->drain));
+            commit_pair(mapa(ptx::smem_addr(&bars->drain), 0));
             wait_bar(&bars->drain, 0, nullptr, status);
         }
-    } else {
-        // epilogue: warp w reads TMEM lanes 32w..32w+31 = tile rows 32w..32w+31
+    } else if (warp == kPCpWarp) {
+        // the stages' scale atoms into both CTAs' TMEM, ahead of the MMAs that read them.  A
+        // stage's columns are free once its bytes are back: the producer reloads a stage only
+        // after the MMAs that read its previous contents (and scales) completed.
+        if (lane == 0 && rank == 0) {
+            int it = 0;
+            bool ok = true;
+            for (int64_t t = pair; ok && t < n_tiles; t += n_pairs) {
+                for (int kt = 0; kt < kt_n; ++kt, ++it) {
+                    const int s = it % kPStages;
+                    if (!wait_bar(&bars->full[s], (it / kPStages) & 1, abort, status)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    const uint32_t sf_base = ptx::smem_addr(stages + s * kPStageBytes) + kPAStage + kPBStage;
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        tmem_cp_atom_pair(tmem_base + psfa_col(s) + 4 * c, smem_desc_atom(sf_base + c * 512));
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)
+                            tmem_cp_atom_pair(tmem_base + psfb_col(s) + 8 * c + 4 * h,
+                                              smem_desc_atom(sf_base + 1024 + h * 1024 + c * 512));
+                    }
+                    commit_pair(mapa(ptx::smem_addr(&bars->sf_ready[s]), 0));
+                }
+            }
+            commit_pair(mapa(ptx::smem_addr(&bars->cp_drain), 0));   // no copy in flight at exit
+            wait_bar(&bars->cp_drain, 0, nullptr, status);
+        }
+    } else if (warp < 4) {
+        // epilogue: warp w reads TMEM lanes 32w..32w+31 = this CTA's rows 32w..32w+31 of the tile
         const uint32_t t_row = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
         const bool vec = args.out_bf16 ? (args.N % 8 == 0) : (args.N % 4 == 0);
+        const uint32_t acc_empty0 = mapa(ptx::smem_addr(&bars->acc_empty), 0);
         int tile_i = 0;
-        for (int64_t t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tile_i) {
+        for (int64_t t = pair; t < n_tiles; t += n_pairs, ++tile_i) {
             int w_ok = 0;
             if (lane == 0) w_ok = wait_bar(&bars->acc_full, tile_i & 1, abort, status);
             if (!__shfl_sync(0xffffffffu, w_ok, 0)) break;
             ptx::tc_fence_after();
-            const int64_t row = (t / tiles_n) * kGM + warp * 32 + lane;
-            const int64_t col_tile = (t % tiles_n) * kGN;
+            const int64_t row = (t / tiles_n) * kPM + static_cast<int64_t>(rank) * 128 + warp * 32 + lane;
+            const int64_t col_tile = (t % tiles_n) * kPN;
             uint32_t ra[32], rb[32];
             ptx::tmem_ld_32cols(t_row, ra);
             ptx::tmem_wait_ld();
 #pragma unroll
-            for (int cb = 0; cb < kGN / 32; ++cb) {
+            for (int cb = 0; cb < kPN / 32; ++cb) {
                 uint32_t(&cur)[32] = (cb & 1) ? rb : ra;
                 uint32_t(&nxt)[32] = (cb & 1) ? ra : rb;
-                if (cb + 1 < kGN / 32) ptx::tmem_ld_32cols(t_row + (cb + 1) * 32, nxt);
+                if (cb + 1 < kPN / 32) ptx::tmem_ld_32cols(t_row + (cb + 1) * 32, nxt);
                 const int64_t col0 = col_tile + cb * 32;
-                if (row < args.M && col0 < args.N) {
-                    if (args.out_bf16) {
-                        uint16_t *dst = static_cast<uint16_t *>(args.y) + row * args.N + col0;
-                        if (vec && col0 + 32 <= args.N) {
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                uint32_t w[4];
-#pragma unroll
-                                for (int e = 0; e < 4; ++e)
-                                    w[e] = pack_bf16x2(__float2bfloat16_rn(__uint_as_float(cur[8 * i + 2 * e])),
-                                                       __float2bfloat16_rn(__uint_as_float(cur[8 * i + 2 * e + 1])));
-                                ptx::st_global_v4(dst + 8 * i, w[0], w[1], w[2], w[3]);
-                            }
-                        } else {
-                            for (int i = 0; i < 32 && col0 + i < args.N; ++i)
-                                dst[i] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(cur[i])));
-                        }
-                    } else {
-                        float *dst = static_cast<float *>(args.y) + row * args.N + col0;
-                        if (vec && col0 + 32 <= args.N) {
-#pragma unroll
-                            for (int i = 0; i < 8; ++i)
-                                ptx::st_global_v4(dst + 4 * i, cur[4 * i], cur[4 * i + 1], cur[4 * i + 2],
-                                                  cur[4 * i + 3]);
-                        } else {
-                            for (int i = 0; i < 32 && col0 + i < args.N; ++i) dst[i] = __uint_as_float(cur[i]);
-                        }
-                    }
-                }
-                if (cb + 1 < kGN / 32) ptx::tmem_wait_ld();
+                if (row < args.M && col0 < args.N) store_row_chunk(args, row, col0, cur, vec);
+                if (cb + 1 < kPN / 32) ptx::tmem_wait_ld();
             }
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(ptx::smem_addr(&bars->acc_empty));
+            if (lane == 0) mbar_arrive_cluster(acc_empty0);
         }
     }
     ptx::tc_fence_before();
     __syncthreads();
+    cluster_sync();   // neither CTA leaves while the other may still touch its barriers, smem or TMEM
     if (warp == kGMmaWarp) {
-        __syncwarp();
         ptx::tc_fence_after();
-        ptx::tmem_dealloc(tmem_base, kTmemCols);
+        tmem_dealloc_pair(tmem_base, kTmemCols);
     }
 }
 
@@ -396,15 +456,32 @@ cudaError_t launch_scales_to_mma(const uint8_t *scales, int64_t rows, int64_t G,
     return cudaGetLastError();
 }
 
-cudaError_t launch_mxfp4_gemm(const CUtensorMap &tmap_a, const CUtensorMap &tmap_b, const GemmArgs &args,
-                              int num_sms, cudaStream_t stream)
+cudaError_t launch_mxfp4_gemm(const CUtensorMap &tmap_a, const CUtensorMap &tmap_b, const CUtensorMap &tmap_sfa,
+                              const CUtensorMap &tmap_sfb, const GemmArgs &args, int num_sms, cudaStream_t stream)
 {
-    const int64_t n_tiles = ((args.M + kGM - 1) / kGM) * ((args.N + kGN - 1) / kGN);
-    if (n_tiles <= 0 || args.K <= 0) return cudaSuccess;
-    const int grid = static_cast<int>(n_tiles < num_sms ? n_tiles : num_sms);
     unsigned int *status = status_word();
     if (!status) return cudaErrorInvalidSymbol;
-    return launch_pdl(mxfp4_gemm_kernel, grid, kGThreads, kGSmem, stream, tmap_a, tmap_b, args, status);
+    // clusters of two CTAs, one pair per two SMs, persistent over the 256 x 256 tiles
+    const int64_t n_tiles = ((args.M + kPM - 1) / kPM) * ((args.N + kPN - 1) / kPN);
+    if (n_tiles <= 0 || args.K <= 0) return cudaSuccess;
+    const int64_t pairs = n_tiles < num_sms / 2 ? n_tiles : num_sms / 2;
+    cudaError_t e = cudaFuncSetAttribute(mxfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+    cfg.blockDim = dim3(kPThreads);
+    cfg.dynamicSmemBytes = kPSmem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, mxfp4_gemm_kernel, tmap_a, tmap_b, tmap_sfa, tmap_sfb, args, status);
 }
 
 }  // namespace mxq

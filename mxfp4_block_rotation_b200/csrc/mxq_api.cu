@@ -225,6 +225,25 @@ mxq_status make_tmap_operand(CUtensorMap *map, const void *codes, int64_t rows, 
     return MXQ_OK;
 }
 
+// Scale atoms [row blocks][cb_n] x 512 B viewed as uint32 [row blocks][cb_n * 128]:
+// boxes of two atoms (256 words) x box_rows row blocks, no swizzle, zero fill past the edges.
+mxq_status make_tmap_sf(CUtensorMap *map, const void *atoms, int64_t row_blocks, int64_t cb_n, uint32_t box_rows)
+{
+    const Driver &d = driver();
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cb_n * 128), static_cast<cuuint64_t>(row_blocks)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cb_n * 512)};
+    cuuint32_t box[2] = {256, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = d.encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void *>(atoms), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        note_cu(r, "cuTensorMapEncodeTiled(scale atoms)");
+        return MXQ_ERR_CUDA;
+    }
+    return MXQ_OK;
+}
+
 mxq_status make_tmap_x(CUtensorMap *map, const void *X, int64_t rows, int64_t cols)
 {
     const Driver &d = driver();
@@ -457,20 +476,19 @@ mxq_status mxq_mxfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales_mma, c
     for (int i = 0; i < 4; ++i)
         if ((st = check_buffer(ins[i], nins[i], dev)) != MXQ_OK) return st;
     if ((st = check_buffer(out, ny, dev)) != MXQ_OK) return st;
-    alignas(64) CUtensorMap map_a, map_b;
+    alignas(64) CUtensorMap map_a, map_b, map_sfa, map_sfb;
     if ((st = make_tmap_operand(&map_a, a_codes, M, K, 128)) != MXQ_OK) return st;
-    if ((st = make_tmap_operand(&map_b, b_codes, N, K, 256)) != MXQ_OK) return st;
+    if ((st = make_tmap_operand(&map_b, b_codes, N, K, 128)) != MXQ_OK) return st;   // a CTA's half of B
+    const int64_t cb_n = (K / 32 + 3) / 4;
+    if ((st = make_tmap_sf(&map_sfa, a_scales, (M + 127) / 128, cb_n, 1)) != MXQ_OK) return st;
+    if ((st = make_tmap_sf(&map_sfb, b_scales, (N + 127) / 128, cb_n, 2)) != MXQ_OK) return st;
     mxq::GemmArgs g{};
-    g.a_sf = a_scales;
-    g.b_sf = b_scales;
-    g.cb_n = (K / 32 + 3) / 4;
-    g.rb_b = (N + 127) / 128;
     g.y = out;
     g.M = M;
     g.N = N;
     g.K = K;
     g.out_bf16 = out_bf16;
-    const cudaError_t e = mxq::launch_mxfp4_gemm(map_a, map_b, g, sms, s);
+    const cudaError_t e = mxq::launch_mxfp4_gemm(map_a, map_b, map_sfa, map_sfb, g, sms, s);
     if (e != cudaSuccess) {
         note_cuda(e, "launch MXFP4 GEMM kernel");
         return MXQ_ERR_CUDA;

@@ -55,16 +55,15 @@ cudaError_t launch_rotate_block(const CUtensorMap &tmap_blocks, const RotArgs &a
 // `tmap_b` view the codes as uint8 [M, K/2] / [N, K/2] (boxes {128, 128} / {128, 256},
 // 128-byte swizzle).
 struct GemmArgs {
-    const uint8_t *a_sf;       // A's scales as 512-byte MMA atoms [ceil(M/128)][cb_n], 16-byte aligned
-    const uint8_t *b_sf;       // B's scales as atoms [rb_b = ceil(N/128)][cb_n]
-    int64_t cb_n;              // atoms per row block: ceil(K/128)
-    int64_t rb_b;
     void *y;                   // [M, N] fp32 or bf16, row-major, 16-byte aligned
     int64_t M, N, K;
     int out_bf16;
 };
-cudaError_t launch_mxfp4_gemm(const CUtensorMap &tmap_a, const CUtensorMap &tmap_b, const GemmArgs &args,
-                              int num_sms, cudaStream_t stream);
+// The GEMM runs on CTA pairs (cta_group::2, 256 x 256 tiles): tmap_a / tmap_b in boxes of
+// 128 rows x 128 B; tmap_sfa / tmap_sfb: the scale atoms as uint32 [row blocks][cb_n * 128],
+// boxes of 256 (two atoms) x 1 row block (A) or 2 (B).
+cudaError_t launch_mxfp4_gemm(const CUtensorMap &tmap_a, const CUtensorMap &tmap_b, const CUtensorMap &tmap_sfa,
+                              const CUtensorMap &tmap_sfb, const GemmArgs &args, int num_sms, cudaStream_t stream);
 
 // Row-major E8M0 scales [rows, G] -> the block-scaled MMA's 512-byte atoms (128 rows x 4
 // k-blocks; row r, k-block j at byte 16 (r % 32) + 4 (r / 32) + j; padding 0).
