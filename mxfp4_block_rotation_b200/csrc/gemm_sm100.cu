@@ -23,7 +23,7 @@
 //              arrival on the even CTA's acc_empty
 //   warp 4     TMA (both CTAs): per stage its A rows, its half of B, its A row block's
 //              scale atoms and both of B's row blocks' atoms, all counted on the even
-//              CTA's full[s] (tensor copies with cta_group::2, no cluster multicast)
+//              CTA's full[s] (tensor copies with cta_group::2, each into its own CTA only)
 //   warp 5     TMEM owner (both CTAs) and, in the even CTA, the MMA issuer: four
 //              kind::mxf4 block32 MMAs per stage, fp32 accumulator in TMEM columns 0-255;
 //              it commits each stage to both CTAs' empty[s] and each tile to acc_full
@@ -78,7 +78,7 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
 }
 
 // A tile of this CTA's operand into its own shared memory; the bytes count on the
-// mbarrier at bar_cluster (the even CTA's).  No cluster multicast.
+// mbarrier at bar_cluster (the even CTA's).  The data lands in this CTA only.
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, int32_t x, int32_t y,
                                                  uint32_t bar_cluster, uint64_t policy)
 {
