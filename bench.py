@@ -543,6 +543,32 @@ def run_e2e(mxq, w, rhat, dev, stream, args, dist):
             "pipeline": f"{n_chunks} row chunks over three streams (H2D, kernel, D2H)"}
 
 
+def run_gemm_only(args):
+    """The consumer GEMM alone at a chosen shape (small cases for ncu captures)."""
+    import mxfp4_block_rotation_b200 as mxq
+    M, N, K = (int(v) for v in args.gemm_only.split(","))
+    dev = torch.device("cuda:0")
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    a = torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device=dev, generator=g)
+    b = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device=dev, generator=g)
+    sfa = mxq.scales_to_mma_layout(torch.randint(120, 134, (M, K // 32), dtype=torch.uint8, device=dev, generator=g))
+    sfb = mxq.scales_to_mma_layout(torch.randint(120, 134, (N, K // 32), dtype=torch.uint8, device=dev, generator=g))
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    for _ in range(3):
+        mxq.mxfp4_gemm(a, sfa, b, sfb, out=y)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        mxq.mxfp4_gemm(a, sfa, b, sfb, out=y)
+    e1.record()
+    torch.cuda.synchronize(dev)
+    mxq.sync_check()
+    ms = e0.elapsed_time(e1) / max(args.steps, 1)
+    print(json.dumps({"gemm": [M, N, K], "ms": ms, "TFLOP/s": 2.0 * M * N * K / (ms * 1e-3) / 1e12}), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -556,9 +582,14 @@ def main(argv=None):
     ap.add_argument("--no-extras", action="store_true", help="skip timing the smoothing and dequantize rows")
     ap.add_argument("--extras-steps", type=int, default=300,
                     help="timed launches per extra row (the search row times min(10, this) runs)")
+    ap.add_argument("--gemm-only", metavar="M,N,K",
+                    help="profiling aid: run only the MXFP4 GEMM, 3 + --steps launches on random operands of this "
+                         "shape (bf16 out), print its time and exit")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
+    if args.gemm_only:
+        return run_gemm_only(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_mine(args)

@@ -140,37 +140,41 @@ __device__ __forceinline__ uint32_t quantize_group_err(const uint32_t (&r)[32], 
     }
     const uint32_t byte = E > 2u ? E - 2u : 0u;
     const float s = __uint_as_float((254u - byte) << 23);   // 2^-e
-    float u[32];
+    // the arithmetic on pairs of values (sm_100's packed fp32 instructions): u = y * 2^-e exactly
+    float2 u[16];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) u[i] = __fmul_rn(__uint_as_float(r[i]), s);
+    for (int i = 0; i < 16; ++i)
+        u[i] = __fmul2_rn(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), make_float2(s, s));
 #pragma unroll
     for (int q = 0; q < 4; ++q)
-        w[q] = ptx::cvt_e2m1x8(u[8 * q], u[8 * q + 1], u[8 * q + 2], u[8 * q + 3], u[8 * q + 4], u[8 * q + 5],
-                               u[8 * q + 6], u[8 * q + 7]);
-    // |Q(u)| straight from the codes just produced: byte permutes pick the bf16 bits of each
-    // code's magnitude {0, .5, 1, 1.5, 2, 3, 4, 6} (code 8q + k is nibble k of w[q]); Q(u) has
-    // u's sign, so |Q(u) - u| = ||u| - |Q(u)||.
-    float num[4] = {0.0f, 0.0f, 0.0f, 0.0f}, den[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        w[q] = ptx::cvt_e2m1x8(u[4 * q].x, u[4 * q].y, u[4 * q + 1].x, u[4 * q + 1].y, u[4 * q + 2].x, u[4 * q + 2].y,
+                               u[4 * q + 3].x, u[4 * q + 3].y);
+    // -|Q(u)| straight from the codes just produced: byte permutes pick the bf16 bits of each
+    // code's magnitude {0, .5, 1, 1.5, 2, 3, 4, 6} (code 8q + k is nibble k of w[q]), with the
+    // sign bit set; Q(u) has u's sign, so |Q(u) - u| = ||u| - |Q(u)||.
+    float2 num[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+    float2 den[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-        const uint32_t m = w[q] & 0x77777777u;
-        const uint32_t h0 = ptx::prmt(0x3F3F3F00u, 0x40404040u, m & 0xFFFFu);
-        const uint32_t l0 = ptx::prmt(0xC0800000u, 0xC0804000u, m & 0xFFFFu);
-        const uint32_t h1 = ptx::prmt(0x3F3F3F00u, 0x40404040u, m >> 16);
-        const uint32_t l1 = ptx::prmt(0xC0800000u, 0xC0804000u, m >> 16);
+        const uint32_t mg = w[q] & 0x77777777u;
+        const uint32_t h0 = ptx::prmt(0xBFBFBF80u, 0xC0C0C0C0u, mg & 0xFFFFu);
+        const uint32_t l0 = ptx::prmt(0xC0800000u, 0xC0804000u, mg & 0xFFFFu);
+        const uint32_t h1 = ptx::prmt(0xBFBFBF80u, 0xC0C0C0C0u, mg >> 16);
+        const uint32_t l1 = ptx::prmt(0xC0800000u, 0xC0804000u, mg >> 16);
         const uint32_t p[4] = {ptx::prmt(l0, h0, 0x5140u), ptx::prmt(l0, h0, 0x7362u), ptx::prmt(l1, h1, 0x5140u),
                                ptx::prmt(l1, h1, 0x7362u)};
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const int i = 8 * q + k;
-            const float qm = __uint_as_float((k & 1) ? (p[k >> 1] & 0xFFFF0000u) : (p[k >> 1] << 16));
-            const float d = __fsub_rn(fabsf(u[i]), qm);
-            num[i & 3] = __fmaf_rn(d, d, num[i & 3]);
-            den[i & 3] = __fmaf_rn(u[i], u[i], den[i & 3]);
+        for (int k2 = 0; k2 < 4; ++k2) {
+            const int i = 4 * q + k2;   // the pair (2i, 2i + 1): nibbles 2 k2, 2 k2 + 1 of w[q]
+            const float2 nq = make_float2(__uint_as_float(p[k2] << 16), __uint_as_float(p[k2] & 0xFFFF0000u));
+            const float2 a = make_float2(fabsf(u[i].x), fabsf(u[i].y));
+            const float2 d = __fadd2_rn(a, nq);
+            num[i & 1] = __ffma2_rn(d, d, num[i & 1]);
+            den[i & 1] = __ffma2_rn(u[i], u[i], den[i & 1]);
         }
     }
-    const float n = (num[0] + num[1]) + (num[2] + num[3]);
-    const float d = (den[0] + den[1]) + (den[2] + den[3]);
+    const float n = (num[0].x + num[1].x) + (num[0].y + num[1].y);
+    const float d = (den[0].x + den[1].x) + (den[0].y + den[1].y);
     err = d > 0.0f ? __fsqrt_rn(__fdiv_rn(n, d)) : 0.0f;
     return byte;
 }

@@ -39,8 +39,22 @@ constexpr int kFlatAcc = (512 / kFlatAccCols) < kMaxAcc ? (512 / kFlatAccCols) :
 constexpr int kFlatSmemBytes = kFlatStages * kFlatStageBytes + kBMatBytes + 512 + 1024;
 static_assert(kFlatBoxes >= 1 && kFlatStageGroups % kFlatBoxGroups == 0 && kFlatStages <= kMaxStages, "flat tiling");
 
+// Warp roles per output mode.  The error mode's epilogue (quantise, decode, two sums per
+// group) is the longest, so it runs four groups of four epilogue warps, each taking every
+// fourth stage (one accumulator stage each); the others run two groups.
 template <RotOut kMode>
-__global__ void __launch_bounds__(kThreads, 1)
+struct FlatRoles {
+    static constexpr int kGroups = (kMode == RotOut::Err || kMode == RotOut::QuantNv) ? 4 : 2;
+    static constexpr int kEpi = 4 * kGroups;
+    static constexpr int kTma = kEpi;
+    static constexpr int kMma = kEpi + 1;
+    static constexpr int kBuild0 = kEpi + 2;
+    static constexpr int kThreadsF = (kEpi + 2 + kBuildWarps) * 32;
+};
+static_assert(kFlatAcc % FlatRoles<RotOut::Err>::kGroups == 0, "one accumulator stage per epilogue group");
+
+template <RotOut kMode>
+__global__ void __launch_bounds__(FlatRoles<kMode>::kThreadsF, 1)
     rotate_flat_kernel(const __grid_constant__ CUtensorMap tmap_g, const RotArgs args, unsigned int *status)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -48,15 +62,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *bmat = stages + kFlatStages * kFlatStageBytes;
     Bars *bars = reinterpret_cast<Bars *>(bmat + kBMatBytes);
     volatile int *abort = &bars->abort;
+    using Ro = FlatRoles<kMode>;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int64_t n_groups = args.rows * (args.cols / 32);
     const int n_chunks = static_cast<int>((n_groups + kFlatStageGroups - 1) / kFlatStageGroups);
 
     const uint32_t tmem_base =
-        kernel_setup(bars, SetupCfg{kFlatStages, kFlatAcc, 1, kBuildWarps * 32, kMmaWarp}, &tmap_g, nullptr);
+        kernel_setup(bars, SetupCfg{kFlatStages, kFlatAcc, 1, kBuildWarps * 32, Ro::kMma}, &tmap_g, nullptr);
 
-    if (warp == kTmaWarp) {
+    if (warp == Ro::kTma) {
         if (lane == 0) {
             const uint64_t pol = ptx::policy_evict_first();
             int it = 0;
@@ -73,7 +88,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             drain_loads(bars, kFlatStages, it, status);
         }
-    } else if (warp == kMmaWarp) {
+    } else if (warp == Ro::kMma) {
         if (lane == 0) {
             constexpr uint32_t idesc = ptx::idesc_bf16_f32(128, 32);
             const uint32_t b_base = ptx::smem_addr(bmat);
@@ -99,9 +114,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             drain_mmas(bars, status);
         }
-    } else if (warp >= kBuildWarp0) {
+    } else if (warp >= Ro::kBuild0) {
         // B = R^ in K-major form: row n holds R^[0..31][n] (bf16, first 64 B of a 128-B row).
-        const int bt = threadIdx.x - kBuildWarp0 * 32;
+        const int bt = threadIdx.x - Ro::kBuild0 * 32;
         for (int t = bt; t < 32 * 4; t += kBuildWarps * 32) {
             const int n = t >> 2, c = t & 3;
             uint32_t w[4];
@@ -117,7 +132,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::mbar_arrive(ptx::smem_addr(&bars->b_full[0]));
     } else {
         const int q = warp & 3;       // TMEM lane quarter this warp may access
-        const int ewg = warp >> 2;    // which half of the stages this warp group takes
+        const int ewg = warp >> 2;    // which of the stages (every kGroups-th) this warp group takes
         // NVFP4: the tensor scale s_t and r_t = 1 / (6 s_t), once per thread
         float nv_st = 0.0f, nv_rt = 0.0f;
         if constexpr (kMode == RotOut::QuantNv) {
@@ -126,7 +141,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         int it = 0;
         for (int c = blockIdx.x; c < n_chunks; c += gridDim.x, ++it) {
-            if ((it & 1) != ewg) continue;
+            if ((it % Ro::kGroups) != ewg) continue;
             const int a = it % kFlatAcc;
             int ok = 0;
             if (lane == 0) ok = wait_bar(&bars->acc_full[a], (it / kFlatAcc) & 1, abort, status);
@@ -182,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     }
-    kernel_teardown(tmem_base, kMmaWarp);
+    kernel_teardown(tmem_base, Ro::kMma);
 }
 
 static_assert(kFlatSmemBytes <= 232448, "shared memory budget");
@@ -199,15 +214,15 @@ cudaError_t launch_rotate_flat(const CUtensorMap &tmap_groups, const RotArgs &ar
     unsigned int *status = status_word();
     if (!status) return cudaErrorInvalidSymbol;
     if (mode == RotOut::Quant)
-        return launch_pdl(rotate_flat_kernel<RotOut::Quant>, grid, kThreads, kFlatSmemBytes, stream, tmap_groups,
+        return launch_pdl(rotate_flat_kernel<RotOut::Quant>, grid, FlatRoles<RotOut::Quant>::kThreadsF, kFlatSmemBytes, stream, tmap_groups,
                           args, status);
     if (mode == RotOut::Err)
-        return launch_pdl(rotate_flat_kernel<RotOut::Err>, grid, kThreads, kFlatSmemBytes, stream, tmap_groups, args,
+        return launch_pdl(rotate_flat_kernel<RotOut::Err>, grid, FlatRoles<RotOut::Err>::kThreadsF, kFlatSmemBytes, stream, tmap_groups, args,
                           status);
     if (mode == RotOut::QuantNv)
-        return launch_pdl(rotate_flat_kernel<RotOut::QuantNv>, grid, kThreads, kFlatSmemBytes, stream, tmap_groups,
+        return launch_pdl(rotate_flat_kernel<RotOut::QuantNv>, grid, FlatRoles<RotOut::QuantNv>::kThreadsF, kFlatSmemBytes, stream, tmap_groups,
                           args, status);
-    return launch_pdl(rotate_flat_kernel<RotOut::F32>, grid, kThreads, kFlatSmemBytes, stream, tmap_groups, args,
+    return launch_pdl(rotate_flat_kernel<RotOut::F32>, grid, FlatRoles<RotOut::F32>::kThreadsF, kFlatSmemBytes, stream, tmap_groups, args,
                       status);
 }
 
