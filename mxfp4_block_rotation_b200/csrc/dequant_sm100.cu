@@ -194,7 +194,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         }
     }
     const uint32_t tmem_base = kernel_setup(
-        bars, SetupCfg{kDqStages, kDqAcc, W::kDec * 32, W::kDec * 32, kDqMmaWarp}, &tmap_out, nullptr);
+        bars, SetupCfg{kDqStages, kDqAcc, W::kDec, W::kDec * 32, kDqMmaWarp}, &tmap_out, nullptr);
 
     if (warp == kDqTmaWarp) {
         if (lane == 0) {
@@ -274,8 +274,9 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             }
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(ptx::smem_addr(&c_empty[cs]));   // this warp's reads of the ring are done
-            ptx::fence_proxy_async_smem();
-            ptx::mbar_arrive(ptx::smem_addr(&bars->full[s]));
+            ptx::fence_proxy_async_smem();   // each lane's A writes, then one arrival per warp
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(ptx::smem_addr(&bars->full[s]));
         }
     } else if (warp == kDqMmaWarp) {
         if (lane == 0) {
