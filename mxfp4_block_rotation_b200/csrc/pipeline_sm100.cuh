@@ -108,13 +108,14 @@ __device__ __forceinline__ uint32_t quantize_group(const uint32_t (&r)[32], uint
     }
     const uint32_t byte = E > 2u ? E - 2u : 0u;
     const float s = __uint_as_float((254u - byte) << 23);   // 2^-e
-    float u[32];
+    float2 u[16];   // u = y * 2^-e, exact, on pairs (sm_100's packed fp32 multiply)
 #pragma unroll
-    for (int i = 0; i < 32; ++i) u[i] = __fmul_rn(__uint_as_float(r[i]), s);
+    for (int i = 0; i < 16; ++i)
+        u[i] = __fmul2_rn(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), make_float2(s, s));
 #pragma unroll
     for (int q = 0; q < 4; ++q)
-        w[q] = ptx::cvt_e2m1x8(u[8 * q], u[8 * q + 1], u[8 * q + 2], u[8 * q + 3], u[8 * q + 4], u[8 * q + 5],
-                               u[8 * q + 6], u[8 * q + 7]);
+        w[q] = ptx::cvt_e2m1x8(u[4 * q].x, u[4 * q].y, u[4 * q + 1].x, u[4 * q + 1].y, u[4 * q + 2].x, u[4 * q + 2].y,
+                               u[4 * q + 3].x, u[4 * q + 3].y);
     return byte;
 }
 

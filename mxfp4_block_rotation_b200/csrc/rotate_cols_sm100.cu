@@ -89,6 +89,18 @@ struct UnitSched {
     __device__ int rt0_of_unit(int ui) const { return ((cta + ui * grid) / n_ct) * kUnitRows; }
 };
 
+// cur += part, element-wise in fp32 (round to nearest), two at a time with the packed add.
+__device__ __forceinline__ void add_pairs(uint32_t (&cur)[32], const uint32_t (&part)[32])
+{
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float2 v = __fadd2_rn(make_float2(__uint_as_float(cur[2 * i]), __uint_as_float(cur[2 * i + 1])),
+                                    make_float2(__uint_as_float(part[2 * i]), __uint_as_float(part[2 * i + 1])));
+        cur[2 * i] = __float_as_uint(v.x);
+        cur[2 * i + 1] = __float_as_uint(v.y);
+    }
+}
+
 template <RotOut kMode>
 __global__ void __launch_bounds__(kColThreads, 1)
     rotate_cols_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_codes,
@@ -294,14 +306,10 @@ __global__ void __launch_bounds__(kColThreads, 1)
                 ptx::tmem_ld_32cols(tg + 64, cur);    // low
                 ptx::tmem_ld_32cols(tg + 32, part);   // middle
                 ptx::tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    cur[i] = __float_as_uint(__fadd_rn(__uint_as_float(cur[i]), __uint_as_float(part[i])));
+                add_pairs(cur, part);
                 ptx::tmem_ld_32cols(tg, part);        // high
                 ptx::tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    cur[i] = __float_as_uint(__fadd_rn(__uint_as_float(cur[i]), __uint_as_float(part[i])));
+                add_pairs(cur, part);
                 const int64_t g = static_cast<int64_t>(ctile) * kColTileG + j;
                 if constexpr (kMode == RotOut::F32) {
                     if (g < G && row_ok) {
