@@ -301,15 +301,14 @@ __global__ void __launch_bounds__(kColThreads, 1)
 #pragma unroll
             for (int j = 0; j < kColTileG; ++j) {
                 // the group's value = (low + middle) + high: the three 32-column partials
-                uint32_t cur[32], part[32];
+                uint32_t cur[32], part[32], hi[32];
                 const uint32_t tg = t_row + j * kColN;
                 ptx::tmem_ld_32cols(tg + 64, cur);    // low
                 ptx::tmem_ld_32cols(tg + 32, part);   // middle
+                ptx::tmem_ld_32cols(tg, hi);          // high: all three loads in flight, one wait
                 ptx::tmem_wait_ld();
                 add_pairs(cur, part);
-                ptx::tmem_ld_32cols(tg, part);        // high
-                ptx::tmem_wait_ld();
-                add_pairs(cur, part);
+                add_pairs(cur, hi);
                 const int64_t g = static_cast<int64_t>(ctile) * kColTileG + j;
                 if constexpr (kMode == RotOut::F32) {
                     if (g < G && row_ok) {
