@@ -61,6 +61,16 @@ def test_gemm_matches_oracle(M, N, K):
     _check_gemm(a, sa, b, sb)
 
 
+def test_gemm_several_tiles_per_pair():
+    # 9 x 9 = 81 tiles of 256 x 256 on at most 74 CTA pairs: some pairs take a second tile, so
+    # the accumulator's empty/full phases turn over; ragged M and N edges, K not a multiple of 256
+    M, N, K = 2300, 2250, 800
+    rng = np.random.default_rng(11)
+    a, sa = _rand_mx(rng, M, K)
+    b, sb = _rand_mx(rng, N, K)
+    _check_gemm(a, sa, b, sb)
+
+
 @pytest.mark.parametrize("M,N,K", [(128, 256, 512), (200, 300, 2048)])
 def test_gemm_exact_with_unit_scales(M, N, K):
     # scale 2^0: every product is a multiple of 1/4 below 36, every partial sum an exact fp32
