@@ -308,6 +308,12 @@ __global__ void __launch_bounds__(kColThreads, 1)
                 ptx::tmem_ld_32cols(tg, hi);          // high: all three loads in flight, one wait
                 ptx::tmem_wait_ld();
                 add_pairs(cur, part);
+                if (j == kColTileG - 1) {
+                    // the tile's last TMEM reads have landed: free the accumulator stage now
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(ptx::smem_addr(&bars->acc_empty[a]));
+                }
                 add_pairs(cur, hi);
                 const int64_t g = static_cast<int64_t>(ctile) * kColTileG + j;
                 if constexpr (kMode == RotOut::F32) {
@@ -344,9 +350,6 @@ __global__ void __launch_bounds__(kColThreads, 1)
                         args.scales[row * G + g] = static_cast<uint8_t>(byte);
                 }
             }
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(ptx::smem_addr(&bars->acc_empty[a]));
             if constexpr (kMode == RotOut::Err) {
                 const double sum = warp_sum(err_acc);
                 if (lane == 0) args.partials[(static_cast<int64_t>(rtile) * n_ct + ctile) * 4 + q] = sum;
