@@ -38,60 +38,97 @@ def build(force: bool = False) -> str:
 _lib = None
 
 
+def build_variant(mutant: int) -> str:
+    """Compile the oracle with planted mistake `mutant` (see the C file's list) into
+    ``oracle/_mutants/`` -- for the pin-sensitivity test only; returns the library path."""
+    out_dir = os.path.join(_HERE, "_mutants")
+    os.makedirs(out_dir, exist_ok=True)
+    path = os.path.join(out_dir, f"libmxq_oracle_m{int(mutant)}.so")
+    if not os.path.exists(path) or os.path.getmtime(path) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=c11", "-fno-fast-math", "-ffp-contract=off", "-fopenmp", f"-DMXQ_MUTANT={int(mutant)}",
+               "-shared", "-fPIC", "-o", path + ".tmp", _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(path + ".tmp", path)
+    return path
+
+
+class use_library:
+    """Context manager: every oracle call inside uses the library at `path` (test infrastructure)."""
+
+    def __init__(self, path: str):
+        self.path = path
+        self.saved = None
+
+    def __enter__(self):
+        global _lib
+        self.saved = lib()
+        _lib = _bind(ctypes.CDLL(self.path))
+        return _lib
+
+    def __exit__(self, *exc):
+        global _lib
+        _lib = self.saved
+        return False
+
+
 def lib():
     global _lib
     if _lib is None:
         build()
-        L = ctypes.CDLL(_LIB)
-        P = ctypes.c_void_p
-        I64 = ctypes.c_int64
-        I = ctypes.c_int
-        L.mxq_oracle_e2m1_code.argtypes = [ctypes.c_double]
-        L.mxq_oracle_e2m1_code.restype = I
-        L.mxq_oracle_e2m1_value.argtypes = [I]
-        L.mxq_oracle_e2m1_value.restype = ctypes.c_double
-        L.mxq_oracle_e8m0_byte.argtypes = [ctypes.c_double]
-        L.mxq_oracle_e8m0_byte.restype = I
-        L.mxq_oracle_e8m0_value.argtypes = [I]
-        L.mxq_oracle_e8m0_value.restype = ctypes.c_double
-        L.mxq_oracle_quantize_group_at.argtypes = [P, I, P, P, P]
-        L.mxq_oracle_quantize_group_at.restype = I
-        L.mxq_oracle_rotate_f64.argtypes = [P, I64, I64, P, P, P, I]
-        L.mxq_oracle_rotate_f64.restype = I
-        L.mxq_oracle_quantize.argtypes = [P, I64, I64, P, P, P, P, P, P, I]
-        L.mxq_oracle_quantize.restype = I
-        L.mxq_oracle_smooth_rotate_quantize.argtypes = [P, I64, I64, P, P, P, P, P, P, P, P, P, I]
-        L.mxq_oracle_weight_rotate_quantize.argtypes = [P, I64, I64, P, P, P, P, P, P, P, P, P, I]
-        L.mxq_oracle_weight_rotate_quantize.restype = I
-        L.mxq_oracle_e4m3_value.argtypes = [I]
-        L.mxq_oracle_e4m3_value.restype = ctypes.c_double
-        L.mxq_oracle_e4m3_code.argtypes = [ctypes.c_double]
-        L.mxq_oracle_e4m3_code.restype = I
-        L.mxq_oracle_nvfp4_block_at.argtypes = [P, I, ctypes.c_float, P, P, P]
-        L.mxq_oracle_nvfp4_block_at.restype = I
-        L.mxq_oracle_nvfp4_quantize.argtypes = [P, I64, I64, P, P, ctypes.c_float, P, P, P, P, P, P, P, I]
-        L.mxq_oracle_nvfp4_quantize.restype = I
-        L.mxq_oracle_scales_to_mma.argtypes = [P, I64, I64, P]
-        L.mxq_oracle_scales_to_mma.restype = I
-        L.mxq_oracle_mxfp4_gemm.argtypes = [P, P, P, P, I64, I64, I64, P, I]
-        L.mxq_oracle_mxfp4_gemm.restype = I
-        L.mxq_oracle_block_rotate_quantize.argtypes = [P, I64, I64, I, P, P, P, P, P, P, P, P, P, I]
-        L.mxq_oracle_block_rotate_quantize.restype = I
-        L.mxq_oracle_smooth_rotate_quantize.restype = I
-        L.mxq_oracle_dequantize.argtypes = [P, P, I64, I64, P, P, P, P, I]
-        L.mxq_oracle_dequantize.restype = I
-        L.mxq_oracle_group_error.argtypes = [P, I64, I64, P, P, P, P, I]
-        L.mxq_oracle_group_error.restype = I
-        L.mxq_oracle_givens.argtypes = [I, I, P, P]
-        L.mxq_oracle_givens.restype = None
-        L.mxq_oracle_rotation_search.argtypes = [P, I64, I64, P, I, I, P, P, P, P, I]
-        L.mxq_oracle_rotation_search.restype = I
-        L.mxq_oracle_bf16_to_double.argtypes = [P, P, I64]
-        L.mxq_oracle_bf16_to_double.restype = None
-        L.mxq_oracle_double_to_bf16.argtypes = [P, P, I64]
-        L.mxq_oracle_double_to_bf16.restype = None
-        _lib = L
+        _lib = _bind(ctypes.CDLL(_LIB))
     return _lib
+
+
+def _bind(L):
+    """Declare every entry point's argument and result types on a loaded oracle library."""
+    P = ctypes.c_void_p
+    I64 = ctypes.c_int64
+    I = ctypes.c_int
+    L.mxq_oracle_e2m1_code.argtypes = [ctypes.c_double]
+    L.mxq_oracle_e2m1_code.restype = I
+    L.mxq_oracle_e2m1_value.argtypes = [I]
+    L.mxq_oracle_e2m1_value.restype = ctypes.c_double
+    L.mxq_oracle_e8m0_byte.argtypes = [ctypes.c_double]
+    L.mxq_oracle_e8m0_byte.restype = I
+    L.mxq_oracle_e8m0_value.argtypes = [I]
+    L.mxq_oracle_e8m0_value.restype = ctypes.c_double
+    L.mxq_oracle_quantize_group_at.argtypes = [P, I, P, P, P]
+    L.mxq_oracle_quantize_group_at.restype = I
+    L.mxq_oracle_rotate_f64.argtypes = [P, I64, I64, P, P, P, I]
+    L.mxq_oracle_rotate_f64.restype = I
+    L.mxq_oracle_quantize.argtypes = [P, I64, I64, P, P, P, P, P, P, I]
+    L.mxq_oracle_quantize.restype = I
+    L.mxq_oracle_smooth_rotate_quantize.argtypes = [P, I64, I64, P, P, P, P, P, P, P, P, P, I]
+    L.mxq_oracle_weight_rotate_quantize.argtypes = [P, I64, I64, P, P, P, P, P, P, P, P, P, I]
+    L.mxq_oracle_weight_rotate_quantize.restype = I
+    L.mxq_oracle_e4m3_value.argtypes = [I]
+    L.mxq_oracle_e4m3_value.restype = ctypes.c_double
+    L.mxq_oracle_e4m3_code.argtypes = [ctypes.c_double]
+    L.mxq_oracle_e4m3_code.restype = I
+    L.mxq_oracle_nvfp4_block_at.argtypes = [P, I, ctypes.c_float, P, P, P]
+    L.mxq_oracle_nvfp4_block_at.restype = I
+    L.mxq_oracle_nvfp4_quantize.argtypes = [P, I64, I64, P, P, ctypes.c_float, P, P, P, P, P, P, P, I]
+    L.mxq_oracle_nvfp4_quantize.restype = I
+    L.mxq_oracle_scales_to_mma.argtypes = [P, I64, I64, P]
+    L.mxq_oracle_scales_to_mma.restype = I
+    L.mxq_oracle_mxfp4_gemm.argtypes = [P, P, P, P, I64, I64, I64, P, I]
+    L.mxq_oracle_mxfp4_gemm.restype = I
+    L.mxq_oracle_block_rotate_quantize.argtypes = [P, I64, I64, I, P, P, P, P, P, P, P, P, P, I]
+    L.mxq_oracle_block_rotate_quantize.restype = I
+    L.mxq_oracle_smooth_rotate_quantize.restype = I
+    L.mxq_oracle_dequantize.argtypes = [P, P, I64, I64, P, P, P, P, I]
+    L.mxq_oracle_dequantize.restype = I
+    L.mxq_oracle_group_error.argtypes = [P, I64, I64, P, P, P, P, I]
+    L.mxq_oracle_group_error.restype = I
+    L.mxq_oracle_givens.argtypes = [I, I, P, P]
+    L.mxq_oracle_givens.restype = None
+    L.mxq_oracle_rotation_search.argtypes = [P, I64, I64, P, I, I, P, P, P, P, I]
+    L.mxq_oracle_rotation_search.restype = I
+    L.mxq_oracle_bf16_to_double.argtypes = [P, P, I64]
+    L.mxq_oracle_bf16_to_double.restype = None
+    L.mxq_oracle_double_to_bf16.argtypes = [P, P, I64]
+    L.mxq_oracle_double_to_bf16.restype = None
+    return L
 
 
 def _ptr(a: Optional[np.ndarray]):

@@ -39,6 +39,31 @@
 
 #define GROUP 32
 
+/* Planted mistakes: test infrastructure for the pins themselves.  A normal build
+ * has MXQ_MUTANT 0 and none of them.  The pin-sensitivity test builds this file
+ * with -DMXQ_MUTANT=k and checks that at least one pin fails for every k:
+ *    1  E8M0 exponent floor(log2 amax) - 1 instead of - 2
+ *    2  E2M1 ties away from zero instead of to the even code
+ *    3  no saturation: |u| >= 7 wraps to code 0
+ *    4  the sign of negative values dropped
+ *    5  the rotation transposed (R[n][k] instead of R[k][n])
+ *    6  Lambda multiplies the activations instead of dividing them
+ *    7  nibble order swapped (odd column in the low nibble)
+ *    8  scale and codes decided on the double values, not on fp32
+ *    9  a NaN/Inf group gets scale byte 0 instead of 0xFF
+ *   10  an E8M0 byte's value taken as 2^(byte - 126)
+ *   11  the rotation sums only 31 of the 32 terms
+ *   12  the search updates R <- G R instead of R <- R G
+ *   13  the inverse rotation of the dequantiser uses R instead of R^T
+ *   14  NVFP4: r_t = 1 / s_t (the 6 dropped)
+ *   15  an all-zero group gets scale byte 127 instead of 0 */
+#ifndef MXQ_MUTANT
+#define MXQ_MUTANT 0
+#endif
+#define PLANTED(k) (MXQ_MUTANT == (k))
+/* R^[k][n] of a row-major 32x32 matrix (transposed under planted mistake 5) */
+#define RKN(R, k, n) (PLANTED(5) ? (R)[(n) * GROUP + (k)] : (R)[(k) * GROUP + (n)])
+
 /* ---------------------------------------------------------------- formats */
 
 /* bf16 bit pattern -> double (exact: bf16 is the top half of an IEEE single). */
@@ -83,18 +108,20 @@ static const double STEP[8] = {0.5, 0.5, 0.5, 0.5, 0.5, 1.0, 1.0, 2.0};
  * saturate above 6, keep the sign.  Returns the 4-bit code. */
 int mxq_oracle_e2m1_code(double u)
 {
-    int neg = signbit(u) ? 1 : 0;
+    int neg = (signbit(u) && !PLANTED(4)) ? 1 : 0;
     double a = fabs(u);
     int best = 0;
     if (isnan(u)) return 0;
-    if (a >= E2M1_MAG[7]) {
+    if (PLANTED(3) && a >= 7.0) {
+        best = 0;
+    } else if (a >= E2M1_MAG[7]) {
         best = 7;
     } else {
         double bestd = a;                   /* distance to magnitude 0 */
         for (int c = 1; c < 8; ++c) {
             double d = fabs(a - E2M1_MAG[c]);
             /* strictly nearer wins; an exact tie goes to the even code */
-            if (d < bestd || (d == bestd && (c & 1) == 0)) {
+            if (d < bestd || (d == bestd && (PLANTED(2) || (c & 1) == 0))) {
                 best = c;
                 bestd = d;
             }
@@ -115,10 +142,10 @@ double mxq_oracle_e2m1_value(int code)
 int mxq_oracle_e8m0_byte(double amax)
 {
     if (isnan(amax) || isinf(amax)) return 0xFF;
-    if (amax == 0.0) return 0;
+    if (amax == 0.0) return PLANTED(15) ? 127 : 0;
     int ex;
     frexp(amax, &ex);                       /* floor(log2 amax) = ex - 1 */
-    int e = (ex - 1) - 2;
+    int e = (ex - 1) - (PLANTED(1) ? 1 : 2);
     if (e < -127) e = -127;
     if (e > 127) e = 127;
     return e + 127;
@@ -128,7 +155,7 @@ int mxq_oracle_e8m0_byte(double amax)
 double mxq_oracle_e8m0_value(int byte)
 {
     if (byte == 0xFF) return NAN;
-    return ldexp(1.0, byte - 127);
+    return ldexp(1.0, byte - (PLANTED(10) ? 126 : 127));
 }
 
 /* ------------------------------------------------------ one group, step by step */
@@ -183,12 +210,12 @@ static void quantize_group(const double *yin, uint8_t *codes_unpacked, uint8_t *
     double amax = 0.0;
     int bad = 0;
     for (int n = 0; n < GROUP; ++n) {
-        y[n] = (double)(float)yin[n];       /* the decision precision: fp32 */
+        y[n] = PLANTED(8) ? yin[n] : (double)(float)yin[n];   /* the decision precision: fp32 */
         if (isnan(y[n]) || isinf(y[n])) bad = 1;
         double a = fabs(y[n]);
         if (a > amax) amax = a;
     }
-    int byte = bad ? 0xFF : mxq_oracle_e8m0_byte(amax);
+    int byte = bad ? (PLANTED(9) ? 0 : 0xFF) : mxq_oracle_e8m0_byte(amax);
     *byte_out = (uint8_t)byte;
     mxq_oracle_quantize_group_at(y, byte, codes_unpacked, eflags, alt);
 
@@ -227,11 +254,11 @@ int mxq_oracle_rotate_f64(const double *X, int64_t rows, int64_t cols, const dou
             double x[GROUP];
             for (int k = 0; k < GROUP; ++k) {
                 x[k] = X[r * cols + g * GROUP + k];
-                if (lam) x[k] = x[k] / lam[g * GROUP + k];
+                if (lam) x[k] = PLANTED(6) ? x[k] * lam[g * GROUP + k] : x[k] / lam[g * GROUP + k];
             }
             for (int n = 0; n < GROUP; ++n) {
                 double acc = 0.0;
-                for (int k = 0; k < GROUP; ++k) acc += x[k] * R[k * GROUP + n];
+                for (int k = 0; k < GROUP - (PLANTED(11) ? 1 : 0); ++k) acc += x[k] * RKN(R, k, n);
                 Y[r * cols + g * GROUP + n] = acc;
             }
         }
@@ -258,7 +285,8 @@ int mxq_oracle_quantize(const double *Y, int64_t rows, int64_t cols, uint8_t *co
                            alt ? alt + e0 : NULL, gflags ? gflags + r * G + g : NULL,
                            alt_scales ? alt_scales + r * G + g : NULL);
             for (int i = 0; i < GROUP / 2; ++i)
-                codes[e0 / 2 + i] = (uint8_t)(c[2 * i] | (c[2 * i + 1] << 4));
+                codes[e0 / 2 + i] = PLANTED(7) ? (uint8_t)(c[2 * i + 1] | (c[2 * i] << 4))
+                                               : (uint8_t)(c[2 * i] | (c[2 * i + 1] << 4));
         }
     }
     return 0;
@@ -288,12 +316,12 @@ static int rotate_quantize_rows(const uint16_t *X, int64_t rows, int64_t cols, c
              * (or, for weights, multiplication) */
             for (int k = 0; k < GROUP; ++k) {
                 x[k] = bf16_to_double(X[e0 + k]);
-                if (lam) x[k] = lam_mul ? x[k] * (double)lam[g * GROUP + k] : x[k] / (double)lam[g * GROUP + k];
+                if (lam) x[k] = (lam_mul || PLANTED(6)) ? x[k] * (double)lam[g * GROUP + k] : x[k] / (double)lam[g * GROUP + k];
             }
             /* step 3: y = x * R^ */
             for (int n = 0; n < GROUP; ++n) {
                 double acc = 0.0;
-                for (int k = 0; k < GROUP; ++k) acc += x[k] * R[k * GROUP + n];
+                for (int k = 0; k < GROUP - (PLANTED(11) ? 1 : 0); ++k) acc += x[k] * RKN(R, k, n);
                 y[n] = acc;
                 if (Y) Y[e0 + n] = acc;
             }
@@ -302,7 +330,8 @@ static int rotate_quantize_rows(const uint16_t *X, int64_t rows, int64_t cols, c
                            alt ? alt + e0 : NULL, gflags ? gflags + r * G + g : NULL,
                            alt_scales ? alt_scales + r * G + g : NULL);
             for (int i = 0; i < GROUP / 2; ++i)
-                codes[e0 / 2 + i] = (uint8_t)(c[2 * i] | (c[2 * i + 1] << 4));
+                codes[e0 / 2 + i] = PLANTED(7) ? (uint8_t)(c[2 * i + 1] | (c[2 * i] << 4))
+                                               : (uint8_t)(c[2 * i] | (c[2 * i + 1] << 4));
         }
     }
     return 0;
@@ -457,7 +486,7 @@ int mxq_oracle_nvfp4_quantize(const uint16_t *X, int64_t rows, int64_t cols, con
     int64_t G = cols / GROUP, NB = cols / 16;
     double R[GROUP * GROUP];
     for (int i = 0; i < GROUP * GROUP; ++i) R[i] = bf16_to_double(Rb[i]);
-    const float d6 = 6.0f * s_t;
+    const float d6 = PLANTED(14) ? s_t : 6.0f * s_t;
     const float r_t = 1.0f / d6;
 #pragma omp parallel for schedule(dynamic, 4) num_threads(nthreads > 0 ? nthreads : 1)
     for (int64_t r = 0; r < rows; ++r) {
@@ -633,7 +662,7 @@ int mxq_oracle_dequantize(const uint8_t *codes, const uint8_t *scales, int64_t r
             for (int k = 0; k < GROUP; ++k) {
                 if (Rb) {
                     double acc = 0.0;
-                    for (int n = 0; n < GROUP; ++n) acc += v[n] * R[k * GROUP + n];
+                    for (int n = 0; n < GROUP; ++n) acc += v[n] * (PLANTED(13) ? R[n * GROUP + k] : R[k * GROUP + n]);
                     x[k] = acc;
                 } else {
                     x[k] = v[k];
@@ -819,6 +848,12 @@ int mxq_oracle_rotation_search(const uint16_t *X, int64_t rows, int64_t cols, co
         mxq_oracle_givens(a, n_angle, &c, &s);
         /* e. R <- R * G */
         for (int r = 0; r < GROUP; ++r) {
+            if (PLANTED(12)) {   /* G * R: rows d and j instead of columns */
+                double rd = R[d * GROUP + r], rj = R[j * GROUP + r];
+                R[d * GROUP + r] = c * rd - s * rj;
+                R[j * GROUP + r] = s * rd + c * rj;
+                continue;
+            }
             double rd = R[r * GROUP + d], rj = R[r * GROUP + j];
             R[r * GROUP + d] = c * rd - s * rj;
             R[r * GROUP + j] = s * rd + c * rj;
