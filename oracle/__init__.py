@@ -112,6 +112,8 @@ def _bind(L):
     L.mxq_oracle_scales_to_mma.argtypes = [P, I64, I64, P]
     L.mxq_oracle_scales_to_mma.restype = I
     L.mxq_oracle_mxfp4_gemm.argtypes = [P, P, P, P, I64, I64, I64, P, I]
+    L.mxq_oracle_nvfp4_gemm.argtypes = [P, P, ctypes.c_float, P, P, ctypes.c_float, I64, I64, I64, P, I]
+    L.mxq_oracle_nvfp4_gemm.restype = I
     L.mxq_oracle_mxfp4_gemm.restype = I
     L.mxq_oracle_block_rotate_quantize.argtypes = [P, I64, I64, I, P, P, P, P, P, P, P, P, P, I]
     L.mxq_oracle_block_rotate_quantize.restype = I
@@ -332,6 +334,21 @@ def mxfp4_gemm(a_codes: np.ndarray, a_scales: np.ndarray, b_codes: np.ndarray, b
     if lib().mxq_oracle_mxfp4_gemm(_ptr(a_codes), _ptr(a_scales), _ptr(b_codes), _ptr(b_scales), M, N, K, _ptr(y),
                                    threads):
         raise ValueError("oracle mxfp4_gemm: bad shape")
+    return y
+
+
+def nvfp4_gemm(a_codes: np.ndarray, a_scales: np.ndarray, a_tscale: float, b_codes: np.ndarray,
+               b_scales: np.ndarray, b_tscale: float, threads: int = 1) -> np.ndarray:
+    """Y[m, n] = sum_k deq(A)[m, k] deq(B)[n, k] in double, NVFP4 operands (E4M3 per 16 k, fp32 tensor scales)."""
+    a_codes, a_scales = _c(a_codes, np.uint8), _c(a_scales, np.uint8)
+    b_codes, b_scales = _c(b_codes, np.uint8), _c(b_scales, np.uint8)
+    M, K = a_codes.shape[0], a_codes.shape[1] * 2
+    N = b_codes.shape[0]
+    assert b_codes.shape[1] * 2 == K and a_scales.shape == (M, K // 16) and b_scales.shape == (N, K // 16)
+    y = np.zeros((M, N), np.float64)
+    if lib().mxq_oracle_nvfp4_gemm(_ptr(a_codes), _ptr(a_scales), float(a_tscale), _ptr(b_codes), _ptr(b_scales),
+                                   float(b_tscale), M, N, K, _ptr(y), threads):
+        raise ValueError("oracle nvfp4_gemm: bad shape")
     return y
 
 

@@ -552,6 +552,51 @@ int mxq_oracle_nvfp4_quantize(const uint16_t *X, int64_t rows, int64_t cols, con
     return 0;
 }
 
+/* The consumer GEMM on NVFP4 operands (the NVFP4 reading of the write-up's
+ * §5.3, fed to the block-scaled tensor cores of §1/§5.4): both operands K-major,
+ * codes packed two per byte (even k in the low nibble), one E4M3 scale per 16 k
+ * and one fp32 tensor scale per operand:
+ *   Y[m][n] = sum_k deq(A)[m][k] * deq(B)[n][k],
+ *   deq = E2M1 value * E4M3 value of the block's scale * tensor scale,
+ * in double, k ascending.  A: codes [M, K/2], scales [M, K/16]; B: codes [N, K/2],
+ * scales [N, K/16]; Y: double [M, N].  A NaN scale (0x7F, 0xFF) makes its products NaN. */
+int mxq_oracle_nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, float a_tscale, const uint8_t *b_codes,
+                          const uint8_t *b_scales, float b_tscale, int64_t M, int64_t N, int64_t K, double *Y,
+                          int nthreads)
+{
+    if (M < 0 || N < 0 || K < 0 || K % GROUP) return 1;
+    int64_t NB = K / 16;
+    double *bd = (double *)malloc(sizeof(double) * (size_t)(N * K > 0 ? N * K : 1));
+    if (!bd) return 1;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) {
+            int code = (b_codes[n * (K / 2) + k / 2] >> (4 * (k & 1))) & 0xF;
+            bd[n * K + k] = mxq_oracle_e2m1_value(code) * mxq_oracle_e4m3_value(b_scales[n * NB + k / 16]) *
+                            (double)b_tscale;
+        }
+#pragma omp parallel num_threads(nthreads > 0 ? nthreads : 1)
+    {
+        double *ad = (double *)malloc(sizeof(double) * (size_t)(K > 0 ? K : 1));
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t m = 0; m < M; ++m) {
+            if (!ad) continue;
+            for (int64_t k = 0; k < K; ++k) {
+                int code = (a_codes[m * (K / 2) + k / 2] >> (4 * (k & 1))) & 0xF;
+                ad[k] = mxq_oracle_e2m1_value(code) * mxq_oracle_e4m3_value(a_scales[m * NB + k / 16]) *
+                        (double)a_tscale;
+            }
+            for (int64_t n = 0; n < N; ++n) {
+                double acc = 0.0;
+                for (int64_t k = 0; k < K; ++k) acc += ad[k] * bd[n * K + k];
+                Y[m * N + n] = acc;
+            }
+        }
+        free(ad);
+    }
+    free(bd);
+    return 0;
+}
+
 /* Row-major E8M0 scales [rows, G] (G = K/32) in the layout Blackwell's
  * block-scaled MMA reads them in: 512-byte atoms, one per 128 rows x 4
  * k-blocks, atoms ordered by row block then k-block; inside an atom the scale

@@ -129,3 +129,76 @@ def test_scale_atoms_hold_every_scale_once():
     # one 16-byte row of an atom: four words, one per 32-row slice, each the row's 4 k-blocks
     atom = out[:512].reshape(32, 4, 4)
     assert np.array_equal(atom[5, 2], sc[64 + 5, 0:4])
+
+
+# ---------------------------------------------------------------- the NVFP4 consumer GEMM
+
+def _decode_e4m3(b):
+    """E4M3 (OCP, no infinities): sign bit 7, exponent bits 6-3 (bias 7), mantissa bits 2-0;
+    exponent 0 is subnormal m/8 * 2^-6; 0x7F and 0xFF are NaN."""
+    b = b.astype(np.int64)
+    s, e, m = (b >> 7) & 1, (b >> 3) & 15, b & 7
+    mag = np.where(e == 0, (m / 8.0) * 2.0 ** -6, (1.0 + m / 8.0) * 2.0 ** (e - 7))
+    mag = np.where((e == 15) & (m == 7), np.nan, mag)
+    return np.where(s == 1, -mag, mag)
+
+
+def _decode_nv(codes, scales, tscale):
+    rows = codes.shape[0]
+    c = np.empty((rows, codes.shape[1] * 2), np.int64)
+    c[:, 0::2] = codes & 0xF
+    c[:, 1::2] = codes >> 4
+    s, e, m = (c >> 3) & 1, (c >> 1) & 3, c & 1
+    mag = np.where(e == 0, 0.5 * m, (1.0 + 0.5 * m) * 2.0 ** (e - 1))
+    v = np.where(s == 1, -mag, mag)
+    return v * np.repeat(_decode_e4m3(scales), 16, axis=1) * float(np.float32(tscale))
+
+
+def _rand_nv(rng, rows, k):
+    # E4M3 scale codes in [0x20, 0x48]: normal values 2^-3 .. 2^2
+    return (rng.integers(0, 256, (rows, k // 2), dtype=np.uint8),
+            rng.integers(0x20, 0x48, (rows, k // 16), dtype=np.uint8))
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 1, 32), (5, 7, 64), (33, 20, 320)])
+def test_nvfp4_gemm_is_the_decoded_matmul(M, N, K):
+    rng = np.random.default_rng(M * 100 + N + K)
+    a, sa = _rand_nv(rng, M, K)
+    b, sb = _rand_nv(rng, N, K)
+    ta, tb = 0.37, 1.9
+    y = oracle.nvfp4_gemm(a, sa, ta, b, sb, tb)
+    ref = _decode_nv(a, sa, ta) @ _decode_nv(b, sb, tb).T
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+
+
+def test_nvfp4_gemm_scales_and_nan():
+    rng = np.random.default_rng(5)
+    a, sa = _rand_nv(rng, 3, 64)
+    b, sb = _rand_nv(rng, 4, 64)
+    y = oracle.nvfp4_gemm(a, sa, 1.0, b, sb, 1.0)
+    # an E4M3 exponent step (+8 on a normal code) doubles that block's contribution: here every
+    # block of row 0 of A at once, so the whole row doubles
+    sa2 = sa.copy()
+    sa2[0] += 8
+    assert np.array_equal(oracle.nvfp4_gemm(a, sa2, 1.0, b, sb, 1.0)[0], 2 * y[0])
+    # the tensor scales multiply the result
+    assert np.allclose(oracle.nvfp4_gemm(a, sa, 4.0, b, sb, 0.5), 2.0 * y, rtol=0, atol=0)
+    # a NaN block scale (0x7F) poisons its row; 0xFF too
+    sa3 = sa.copy()
+    sa3[1, 2] = 0x7F
+    sa3[2, 0] = 0xFF
+    y3 = oracle.nvfp4_gemm(a, sa3, 1.0, b, sb, 1.0)
+    assert np.isnan(y3[1]).all() and np.isnan(y3[2]).all() and np.array_equal(y3[0], y[0])
+    # the scale of block 1 (k = 16..31) acts on those k only: zero the codes of k < 16 and of
+    # k >= 32, then doubling block 1's scale doubles the product and changing block 0's does nothing
+    a4 = a.copy()
+    a4[:, :8] = 0
+    a4[:, 16:] = 0
+    y4 = oracle.nvfp4_gemm(a4, sa, 1.0, b, sb, 1.0)
+    sa4 = sa.copy()
+    sa4[:, 1] += 8
+    sa4[:, 0] += 8
+    assert np.array_equal(oracle.nvfp4_gemm(a4, sa4, 1.0, b, sb, 1.0), 2 * y4)
+    sa5 = sa.copy()
+    sa5[:, 0] += 8
+    assert np.array_equal(oracle.nvfp4_gemm(a4, sa5, 1.0, b, sb, 1.0), y4)
