@@ -443,6 +443,25 @@ def run_extras(mxq, w, xs, rhat, outs, dev, stream, k=300):
         "frac_of_fp4_peak": flops / (ms * 1e-3) / 1e12 / fp4_peak,
         "peak_source": "measured bf16 burst (MEASURED_PEAKS.json bf16_tflops) x 4, the nominal fp4/bf16 ratio"}
 
+    # the NVFP4 consumer GEMM on the same shape: operands quantised by the NVFP4 path (tensor
+    # scales from the bound amax <= sqrt(32) max|x|), E4M3 scales per 16 k
+    ts_a = torch.tensor([float(w.x.abs().max().float()) * 32 ** 0.5 / (6 * 448)], dtype=torch.float32, device=dev)
+    ts_b = torch.tensor([float(wt.abs().max().float()) * 32 ** 0.5 / (6 * 448)], dtype=torch.float32, device=dev)
+    nca, nsa = mxq.smooth_rotate_quantize_nvfp4(xs[0], rhat, ts_a, stream=stream)
+    ncb, nsb = mxq.smooth_rotate_quantize_nvfp4(wt, rhat, ts_b, stream=stream)
+    nsfa = mxq.nvfp4_scales_to_mma_layout(nsa, stream=stream)
+    nsfb = mxq.nvfp4_scales_to_mma_layout(nsb, stream=stream)
+
+    def gemm_nv(i):
+        mxq.nvfp4_gemm(nca, nsfa, ts_a, ncb, nsfb, ts_b, out=y, stream=stream)
+    ms = _timed(gemm_nv, max(1, min(50, k)), stream, dev)
+    res["nvfp4_gemm_downproj"] = {
+        "what": f"Y[{rows}x{n_out}] = NVFP4(X R) NVFP4(W^T R)^T, K = {cols}, bf16 out (mxfp4_gemm_kernel<NVFP4>)",
+        "ms": ms, "TFLOP/s": flops / (ms * 1e-3) / 1e12, "peak_TFLOP/s": fp4_peak,
+        "frac_of_fp4_peak": flops / (ms * 1e-3) / 1e12 / fp4_peak,
+        "peak_source": "measured bf16 burst (MEASURED_PEAKS.json bf16_tflops) x 4, the nominal fp4/bf16 ratio"}
+    del nca, nsa, ncb, nsb, nsfa, nsfb
+
     def layer(i):
         c, s = outs[i & 1]
         mxq.smooth_rotate_quantize(xs[i & 1], rhat, None, codes=c, scales=s, stream=stream)

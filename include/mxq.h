@@ -184,6 +184,29 @@ mxq_status mxq_mxfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales_mma, c
                           int out_bf16, void *stream);
 
 /*
+ * The NVFP4 × NVFP4 consumer GEMM (the NVFP4 reading of the write-up's §5.3 on
+ * the same block-scaled tensor cores): operands as mxq_smooth_rotate_quantize_nvfp4
+ * writes them, one E4M3 scale per 16 k and one fp32 tensor scale per operand:
+ *   Y[m][n] = Σ_k deq(A)[m][k] · deq(B)[n][k],
+ *   deq = E2M1 code · E4M3 block scale · tensor scale
+ * The tensor cores accumulate Σ code·scale·code·scale in fp32; the product of
+ * the two tensor scales (fp32) then multiplies every output.
+ *   a_codes, b_codes     in   [M, K/2], [N, K/2] bytes, 16-byte aligned
+ *   a_scales_mma, ...    in   mxq_nvfp4_scales_mma_bytes(rows, K) bytes, 16-byte aligned:
+ *                             the [rows, K/16] E4M3 scales through mxq_nvfp4_scales_to_mma_layout
+ *                             (the same 512-byte atoms, each holding 64 k of 128 rows)
+ *   a_tensor_scale, ...  in   one fp32 each, device memory, 4-byte aligned; read by the kernel
+ *   K, out, out_bf16, errors as mxq_mxfp4_gemm.  A NaN scale (0x7F or 0xFF) makes the
+ *   products it scales NaN.
+ */
+size_t mxq_nvfp4_scales_mma_bytes(int64_t rows, int64_t K);
+mxq_status mxq_nvfp4_scales_to_mma_layout(const uint8_t *scales, int64_t rows, int64_t K, uint8_t *out,
+                                          void *stream);
+mxq_status mxq_nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales_mma, const float *a_tensor_scale,
+                          const uint8_t *b_codes, const uint8_t *b_scales_mma, const float *b_tensor_scale,
+                          int64_t M, int64_t N, int64_t K, void *out, int out_bf16, void *stream);
+
+/*
  * Rotation-block-size variants (DuQuant++ write-up, §4.3: rotation blocks of
  * B = 16, 32, 64 or 128 channels, B = 32 found best).  The MXFP4 groups stay
  * at 32 columns.  Each row is cut into cols/B blocks; block x becomes

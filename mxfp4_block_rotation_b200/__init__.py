@@ -24,7 +24,7 @@ import torch
 __all__ = [
     "MxqError", "smooth_rotate_quantize", "smooth_rotate_quantize_nvfp4", "smooth_rotate_f32",
     "weight_rotate_quantize", "rotate_quantize_block", "rotate_block_f32", "scales_to_mma_layout",
-    "mxfp4_gemm", "dequantize", "quant_error", "rotation_search", "sync_check", "selftest_bounded_wait",
+    "mxfp4_gemm", "nvfp4_scales_to_mma_layout", "nvfp4_gemm", "dequantize", "quant_error", "rotation_search", "sync_check", "selftest_bounded_wait",
     "status_string", "version", "lib", "LIB_PATH", "HEADER_PATH", "declared_symbols",
 ]
 
@@ -73,6 +73,12 @@ def lib() -> ctypes.CDLL:
         L.mxq_scales_mma_bytes.argtypes = [I64, I64]
         L.mxq_scales_mma_bytes.restype = ctypes.c_size_t
         L.mxq_scales_to_mma_layout.argtypes = [P, I64, I64, P, P]
+        L.mxq_nvfp4_scales_mma_bytes.argtypes = [I64, I64]
+        L.mxq_nvfp4_scales_mma_bytes.restype = ctypes.c_size_t
+        L.mxq_nvfp4_scales_to_mma_layout.argtypes = [P, I64, I64, P, P]
+        L.mxq_nvfp4_scales_to_mma_layout.restype = I
+        L.mxq_nvfp4_gemm.argtypes = [P, P, P, P, P, P, I64, I64, I64, P, I, P]
+        L.mxq_nvfp4_gemm.restype = I
         L.mxq_scales_to_mma_layout.restype = I
         L.mxq_mxfp4_gemm.restype = I
         L.mxq_dequantize.argtypes = [P, P, I64, I64, P, P, P, P]
@@ -284,6 +290,65 @@ def mxfp4_gemm(a_codes: torch.Tensor, a_scales: torch.Tensor, b_codes: torch.Ten
     st = lib().mxq_mxfp4_gemm(_ptr(a_codes), _ptr(a_scales), _ptr(b_codes), _ptr(b_scales), M, N, K, _ptr(out),
                               int(out_dtype == torch.bfloat16), _stream(dev, stream))
     _check(st, "mxq_mxfp4_gemm")
+    return out
+
+
+def nvfp4_scales_to_mma_layout(scales: torch.Tensor, *, out: Optional[torch.Tensor] = None,
+                               stream=None) -> torch.Tensor:
+    """Row-major E4M3 scales [rows, K/16] -> the block-scaled MMA's 512-byte atoms (flat uint8)."""
+    dev = scales.device
+    if dev.type != "cuda":
+        raise ValueError("scales must be a CUDA tensor (this library has no CPU path)")
+    _need(scales, "scales", torch.uint8, dev)
+    rows, nb = scales.shape
+    n = int(lib().mxq_nvfp4_scales_mma_bytes(rows, nb * 16))
+    if out is None:
+        out = torch.empty(n, dtype=torch.uint8, device=dev)
+    _need(out, "out", torch.uint8, dev)
+    if out.numel() < n:
+        raise ValueError(f"out needs {n} bytes")
+    st = lib().mxq_nvfp4_scales_to_mma_layout(_ptr(scales), rows, nb * 16, _ptr(out), _stream(dev, stream))
+    _check(st, "mxq_nvfp4_scales_to_mma_layout")
+    return out
+
+
+def nvfp4_gemm(a_codes: torch.Tensor, a_scales: torch.Tensor, a_tscale: torch.Tensor, b_codes: torch.Tensor,
+               b_scales: torch.Tensor, b_tscale: torch.Tensor, *, out_dtype: torch.dtype = torch.float32,
+               out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Y = deq(A) · deq(B)ᵀ for NVFP4 operands (E4M3 per 16 k; fp32 tensor scales a_tscale, b_tscale of
+    one element each, on the device).  Scales row-major ([rows, K/16]) or already in the MMA layout."""
+    dev = a_codes.device
+    if dev.type != "cuda":
+        raise ValueError("operands must be CUDA tensors (this library has no CPU path)")
+    for t, name in ((a_codes, "a_codes"), (a_scales, "a_scales"), (b_codes, "b_codes"), (b_scales, "b_scales")):
+        _need(t, name, torch.uint8, dev)
+    for t, name in ((a_tscale, "a_tscale"), (b_tscale, "b_tscale")):
+        _need(t, name, torch.float32, dev)
+        if t.numel() != 1:
+            raise ValueError(f"{name} must hold one float")
+    M, K = a_codes.shape[0], a_codes.shape[1] * 2
+    N = b_codes.shape[0]
+    if b_codes.shape[1] * 2 != K:
+        raise ValueError("operand shapes disagree")
+    if a_scales.dim() == 2:
+        if tuple(a_scales.shape) != (M, K // 16):
+            raise ValueError("a_scales must be [M, K/16]")
+        a_scales = nvfp4_scales_to_mma_layout(a_scales, stream=stream) if M and K else a_scales
+    if b_scales.dim() == 2:
+        if tuple(b_scales.shape) != (N, K // 16):
+            raise ValueError("b_scales must be [N, K/16]")
+        b_scales = nvfp4_scales_to_mma_layout(b_scales, stream=stream) if N and K else b_scales
+    if out is not None:
+        out_dtype = out.dtype
+    if out_dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("out_dtype must be float32 or bfloat16")
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=dev)
+    _need(out, "out", out_dtype, dev)
+    st = lib().mxq_nvfp4_gemm(_ptr(a_codes), _ptr(a_scales), _ptr(a_tscale), _ptr(b_codes), _ptr(b_scales),
+                              _ptr(b_tscale), M, N, K, _ptr(out), int(out_dtype == torch.bfloat16),
+                              _stream(dev, stream))
+    _check(st, "mxq_nvfp4_gemm")
     return out
 
 

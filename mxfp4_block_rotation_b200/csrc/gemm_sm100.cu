@@ -48,12 +48,12 @@ using namespace pipe;
 
 // Instruction descriptor, kind::mxf4 block-scaled: E2M1 A and B (format 1), UE8M0 scales,
 // both K-major, M = 128, N = 256, K = 64; scale ids (the byte pair inside a scale word) added per MMA.
-__host__ __device__ constexpr uint32_t idesc_mxf4(int m, int n)
+__host__ __device__ constexpr uint32_t idesc_mxf4(int m, int n, bool e8m0 = true)
 {
     return (1u << 7)                                  // A format: E2M1
            | (1u << 10)                               // B format: E2M1
            | (static_cast<uint32_t>(n >> 3) << 17)    // N / 8
-           | (1u << 23)                               // scale format: UE8M0
+           | ((e8m0 ? 1u : 0u) << 23)                 // scale format: UE8M0 (MXFP4) or UE4M3 (NVFP4)
            | (static_cast<uint32_t>(m >> 4) << 24);   // M / 16
 }
 
@@ -96,6 +96,20 @@ __device__ __forceinline__ void mma_mxf4_pair(uint32_t d_tmem, uint64_t a_desc, 
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %6, 0;\n\t"
         "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+        :
+        : "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+        : "memory");
+}
+
+// The same with NVFP4 operands: E2M1 codes, one E4M3 scale per 16 k (a K = 64 MMA takes the
+// four scales of a 32-bit TMEM word).
+__device__ __forceinline__ void mma_nvf4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
         :
         : "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
         : "memory");
@@ -196,26 +210,37 @@ constexpr int kGAccCols = 256;                // fp32 accumulator: TMEM columns 
 
 constexpr int kPM = 256;                      // pair tile rows (128 per CTA)
 constexpr int kPN = 256;                      // pair tile columns
-constexpr int kPStages = 6;
 constexpr int kPAStage = 128 * 128;           // this CTA's 128 rows x 256 k: 16 KB
 constexpr int kPBStage = 128 * 128;           // this CTA's half of B: 16 KB
-constexpr int kPSfStage = 3 * 1024;           // A: 2 atoms of its row block; B: 2 row blocks x 2 atoms
-constexpr int kPStageBytes = kPAStage + kPBStage + kPSfStage;   // 35 KB
-constexpr int kPTx = 2 * kPStageBytes;        // bytes a stage brings into the pair
-constexpr int kPSmem = kPStages * kPStageBytes + 1024 + 1024;
 constexpr int kPThreads = 7 * 32;             // warps 0-3 epilogue, 4 TMA, 5 MMA, 6 scale copies
 constexpr int kPCpWarp = 6;
-constexpr int kPSfaCols = 2 * (128 / 32);     // per stage: two 128-k words x 4 row blocks
-constexpr int kPSfbCols = 2 * (kPN / 32);     // two 128-k words x 8 row blocks
-static_assert(kGAccCols + kPStages * (kPSfaCols + kPSfbCols) <= 512, "TMEM budget (pairs)");
-static_assert(kPSmem <= 232448, "shared memory budget (pairs)");
+constexpr int kPMaxStages = 6;
+
+// Per format: MXFP4 scales cover 32 k (a 512-byte atom = 128 rows x 128 k), NVFP4 scales 16 k
+// (an atom = 128 rows x 64 k), so a 256-k stage holds 2 or 4 atoms per 128-row block.
+template <bool kNv>
+struct PairCfg {
+    static constexpr int kAtoms = kNv ? 4 : 2;                       // atoms per stage per row block
+    static constexpr int kStages = kNv ? 5 : 6;
+    static constexpr int kSfStage = 3 * kAtoms * 512;                 // A: its row block; B: two row blocks
+    static constexpr int kStageBytes = kPAStage + kPBStage + kSfStage;   // 35 KB or 38 KB
+    static constexpr int kTx = 2 * kStageBytes;                      // bytes a stage brings into the pair
+    static constexpr int kSmem = kStages * kStageBytes + 1024 + 1024;
+    static constexpr int kSfaCols = 4 * kAtoms;                       // scale words x 4 row blocks
+    static constexpr int kSfbCols = 8 * kAtoms;                       // x 8 row blocks
+    static_assert(kStages <= kPMaxStages, "barrier arrays");
+    static_assert(kGAccCols + kStages * (kSfaCols + kSfbCols) <= 512, "TMEM budget (pairs)");
+    static_assert(kSmem <= 232448, "shared memory budget (pairs)");
+    __device__ static uint32_t sfa_col(int s) { return kGAccCols + s * kSfaCols; }
+    __device__ static uint32_t sfb_col(int s) { return kGAccCols + kStages * kSfaCols + s * kSfbCols; }
+};
 
 struct PairBars {
-    uint64_t full[kPStages];      // even CTA: both CTAs' operand and scale bytes of a stage landed
-    uint64_t empty[kPStages];     // the stage's pair MMAs are done (from the even CTA's commit)
-    uint64_t sf_ready[kPStages];  // even CTA: the stage's scales have been copied into both CTAs' TMEM
-    uint64_t acc_full;            // the tile's accumulator is complete (from the even CTA's commit)
-    uint64_t acc_empty;           // even CTA: both CTAs' epilogues have read the accumulator (8 warps)
+    uint64_t full[kPMaxStages];      // even CTA: both CTAs' operand and scale bytes of a stage landed
+    uint64_t empty[kPMaxStages];     // the stage's pair MMAs are done (from the even CTA's commit)
+    uint64_t sf_ready[kPMaxStages];  // even CTA: the stage's scales have been copied into both CTAs' TMEM
+    uint64_t acc_full;               // the tile's accumulator is complete (from the even CTA's commit)
+    uint64_t acc_empty;              // even CTA: both CTAs' epilogues have read the accumulator (8 warps)
     uint64_t drain;
     uint64_t cp_drain;
     uint32_t tmem_base;
@@ -223,14 +248,15 @@ struct PairBars {
 };
 static_assert(sizeof(PairBars) <= 1024, "barrier block (pairs)");
 
-__device__ __forceinline__ uint32_t psfa_col(int s) { return kGAccCols + s * kPSfaCols; }
-__device__ __forceinline__ uint32_t psfb_col(int s) { return kGAccCols + kPStages * kPSfaCols + s * kPSfbCols; }
-
+template <bool kNv>
 __global__ void __launch_bounds__(kPThreads, 1)
     mxfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                           const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
-                           const GemmArgs args, unsigned int *status)
+                      const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
+                      const GemmArgs args, unsigned int *status)
 {
+    using C = PairCfg<kNv>;
+    constexpr int kPStages = C::kStages;
+    constexpr int kPStageBytes = C::kStageBytes;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *stages = align_1k(smem_raw);
     PairBars *bars = reinterpret_cast<PairBars *>(stages + kPStages * kPStageBytes);
@@ -287,15 +313,20 @@ __global__ void __launch_bounds__(kPThreads, 1)
                     }
                     const uint32_t dst = ptx::smem_addr(stages + s * kPStageBytes);
                     const uint32_t full0 = mapa(ptx::smem_addr(&bars->full[s]), 0);
-                    if (rank == 0) ptx::mbar_arrive_expect_tx(ptx::smem_addr(&bars->full[s]), kPTx);
+                    if (rank == 0) ptx::mbar_arrive_expect_tx(ptx::smem_addr(&bars->full[s]), C::kTx);
                     // this CTA's A rows and half of B; its A row block's scale atoms and the atoms of
                     // both of B's row blocks (zero past the matrices' edges)
                     tma_load_2d_pair(dst, &tmap_a, kt * 128, tm2 * kPM + static_cast<int>(rank) * 128, full0, pol);
                     tma_load_2d_pair(dst + kPAStage, &tmap_b, kt * 128, tn * kPN + static_cast<int>(rank) * 128, full0,
                                      pol);
-                    tma_load_2d_pair(dst + kPAStage + kPBStage, &tmap_sfa, kt * 256, 2 * tm2 + static_cast<int>(rank),
-                                     full0, pol);
-                    tma_load_2d_pair(dst + kPAStage + kPBStage + 1024, &tmap_sfb, kt * 256, 2 * tn, full0, pol);
+                    // scale atoms in boxes of two (256 words); NVFP4 has four per stage
+                    const uint32_t sfd = dst + kPAStage + kPBStage;
+#pragma unroll
+                    for (int h2 = 0; h2 < C::kAtoms / 2; ++h2) {
+                        const int x = kt * C::kAtoms * 128 + h2 * 256;
+                        tma_load_2d_pair(sfd + h2 * 1024, &tmap_sfa, x, 2 * tm2 + static_cast<int>(rank), full0, pol);
+                        tma_load_2d_pair(sfd + C::kAtoms * 512 + h2 * 2048, &tmap_sfb, x, 2 * tn, full0, pol);
+                    }
                 }
             }
             // the last copies into each stage land before the CTA can exit (the even CTA's
@@ -309,7 +340,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
         }
     } else if (warp == kGMmaWarp) {
         if (lane == 0 && rank == 0) {
-            constexpr uint32_t idesc0 = idesc_mxf4(kPM, kPN);
+            constexpr uint32_t idesc0 = idesc_mxf4(kPM, kPN, !kNv);
             int it = 0, tile_i = 0;
             bool ok = true;
             for (int64_t t = pair; ok && t < n_tiles; t += n_pairs, ++tile_i) {
@@ -328,13 +359,17 @@ __global__ void __launch_bounds__(kPThreads, 1)
                     const uint32_t b_base = a_base + kPAStage;
 #pragma unroll
                     for (int j = 0; j < kGK / 64; ++j) {
-                        const uint32_t c = j >> 1, byte = 2u * (j & 1);
-                        const uint32_t sfa = (tmem_base + psfa_col(s) + 4 * c) | (byte << 30);
-                        const uint32_t sfb = (tmem_base + psfb_col(s) + 8 * c) | (byte << 30);
+                        // MXFP4: a word holds the scales of 128 k, the MMA takes bytes 0-1 or 2-3;
+                        // NVFP4: a word holds the four scales of 64 k, one word per MMA
+                        const uint32_t c = kNv ? j : j >> 1, byte = kNv ? 0u : 2u * (j & 1);
+                        const uint32_t sfa = (tmem_base + C::sfa_col(s) + 4 * c) | (byte << 30);
+                        const uint32_t sfb = (tmem_base + C::sfb_col(s) + 8 * c) | (byte << 30);
                         const uint32_t idesc = idesc0 | (byte << 29) | (byte << 4);
-                        mma_mxf4_pair(tmem_base, ptx::smem_desc_sw128(a_base + j * 32),
-                                      ptx::smem_desc_sw128(b_base + j * 32), idesc, sfa, sfb,
-                                      static_cast<uint32_t>(kt | j));
+                        const uint64_t ad = ptx::smem_desc_sw128(a_base + j * 32), bd = ptx::smem_desc_sw128(b_base + j * 32);
+                        if constexpr (kNv)
+                            mma_nvf4_pair(tmem_base, ad, bd, idesc, sfa, sfb, static_cast<uint32_t>(kt | j));
+                        else
+                            mma_mxf4_pair(tmem_base, ad, bd, idesc, sfa, sfb, static_cast<uint32_t>(kt | j));
                     }
                     const uint32_t e = ptx::smem_addr(&bars->empty[s]);
                     commit_pair(mapa(e, 0));
@@ -364,13 +399,16 @@ __global__ void __launch_bounds__(kPThreads, 1)
                     }
                     ptx::tc_fence_after();
                     const uint32_t sf_base = ptx::smem_addr(stages + s * kPStageBytes) + kPAStage + kPBStage;
+                    // A's atoms c at sf_base + 512 c; B's (row block h, atom c) in boxes of two
+                    // atoms by two row blocks: sf_base + 512 kAtoms + 2048 (c / 2) + 1024 h + 512 (c % 2)
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        tmem_cp_atom_pair(tmem_base + psfa_col(s) + 4 * c, smem_desc_atom(sf_base + c * 512));
+                    for (int c = 0; c < C::kAtoms; ++c) {
+                        tmem_cp_atom_pair(tmem_base + C::sfa_col(s) + 4 * c, smem_desc_atom(sf_base + c * 512));
 #pragma unroll
                         for (int h = 0; h < 2; ++h)
-                            tmem_cp_atom_pair(tmem_base + psfb_col(s) + 8 * c + 4 * h,
-                                              smem_desc_atom(sf_base + 1024 + h * 1024 + c * 512));
+                            tmem_cp_atom_pair(tmem_base + C::sfb_col(s) + 8 * c + 4 * h,
+                                              smem_desc_atom(sf_base + C::kAtoms * 512 + (c / 2) * 2048 + h * 1024 +
+                                                             (c % 2) * 512));
                     }
                     commit_pair(mapa(ptx::smem_addr(&bars->sf_ready[s]), 0));
                 }
@@ -383,6 +421,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
         const uint32_t t_row = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
         const bool vec = args.out_bf16 ? (args.N % 8 == 0) : (args.N % 4 == 0);
         const uint32_t acc_empty0 = mapa(ptx::smem_addr(&bars->acc_empty), 0);
+        // NVFP4: the product of the two tensor scales multiplies every output
+        const float alpha = kNv ? __fmul_rn(*args.a_tscale, *args.b_tscale) : 1.0f;
         int tile_i = 0;
         for (int64_t t = pair; t < n_tiles; t += n_pairs, ++tile_i) {
             int w_ok = 0;
@@ -400,6 +440,10 @@ __global__ void __launch_bounds__(kPThreads, 1)
                 uint32_t(&nxt)[32] = (cb & 1) ? ra : rb;
                 if (cb + 1 < kPN / 32) ptx::tmem_ld_32cols(t_row + (cb + 1) * 32, nxt);
                 const int64_t col0 = col_tile + cb * 32;
+                if constexpr (kNv) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) cur[i] = __float_as_uint(__fmul_rn(__uint_as_float(cur[i]), alpha));
+                }
                 if (row < args.M && col0 < args.N) store_row_chunk(args, row, col0, cur, vec);
                 if (cb + 1 < kPN / 32) ptx::tmem_wait_ld();
             }
@@ -456,8 +500,11 @@ cudaError_t launch_scales_to_mma(const uint8_t *scales, int64_t rows, int64_t G,
     return cudaGetLastError();
 }
 
-cudaError_t launch_mxfp4_gemm(const CUtensorMap &tmap_a, const CUtensorMap &tmap_b, const CUtensorMap &tmap_sfa,
-                              const CUtensorMap &tmap_sfb, const GemmArgs &args, int num_sms, cudaStream_t stream)
+namespace {
+
+template <bool kNv>
+cudaError_t launch_pairs(const CUtensorMap &tmap_a, const CUtensorMap &tmap_b, const CUtensorMap &tmap_sfa,
+                         const CUtensorMap &tmap_sfb, const GemmArgs &args, int num_sms, cudaStream_t stream)
 {
     unsigned int *status = status_word();
     if (!status) return cudaErrorInvalidSymbol;
@@ -465,7 +512,8 @@ cudaError_t launch_mxfp4_gemm(const CUtensorMap &tmap_a, const CUtensorMap &tmap
     const int64_t n_tiles = ((args.M + kPM - 1) / kPM) * ((args.N + kPN - 1) / kPN);
     if (n_tiles <= 0 || args.K <= 0) return cudaSuccess;
     const int64_t pairs = n_tiles < num_sms / 2 ? n_tiles : num_sms / 2;
-    cudaError_t e = cudaFuncSetAttribute(mxfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmem);
+    constexpr int smem = PairCfg<kNv>::kSmem;
+    cudaError_t e = cudaFuncSetAttribute(mxfp4_gemm_kernel<kNv>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -477,11 +525,20 @@ cudaError_t launch_mxfp4_gemm(const CUtensorMap &tmap_a, const CUtensorMap &tmap
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
     cfg.blockDim = dim3(kPThreads);
-    cfg.dynamicSmemBytes = kPSmem;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, mxfp4_gemm_kernel, tmap_a, tmap_b, tmap_sfa, tmap_sfb, args, status);
+    return cudaLaunchKernelEx(&cfg, mxfp4_gemm_kernel<kNv>, tmap_a, tmap_b, tmap_sfa, tmap_sfb, args, status);
+}
+
+}  // namespace
+
+cudaError_t launch_mxfp4_gemm(const CUtensorMap &tmap_a, const CUtensorMap &tmap_b, const CUtensorMap &tmap_sfa,
+                              const CUtensorMap &tmap_sfb, const GemmArgs &args, int num_sms, cudaStream_t stream)
+{
+    return args.nvfp4 ? launch_pairs<true>(tmap_a, tmap_b, tmap_sfa, tmap_sfb, args, num_sms, stream)
+                      : launch_pairs<false>(tmap_a, tmap_b, tmap_sfa, tmap_sfb, args, num_sms, stream);
 }
 
 }  // namespace mxq

@@ -436,11 +436,11 @@ mxq_status mxq_scales_to_mma_layout(const uint8_t *scales, int64_t rows, int64_t
     return MXQ_OK;
 }
 
-mxq_status mxq_mxfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales_mma, const uint8_t *b_codes,
-                          const uint8_t *b_scales_mma, int64_t M, int64_t N, int64_t K, void *out, int out_bf16,
-                          void *stream)
+// MXFP4 (nv = 0) or NVFP4 (nv = 1, with the tensor scales) GEMM: validation and launch.
+static mxq_status gemm_common(const uint8_t *a_codes, const uint8_t *a_scales, const uint8_t *b_codes,
+                              const uint8_t *b_scales, int64_t M, int64_t N, int64_t K, void *out, int out_bf16,
+                              void *stream, int nv, const float *a_tscale, const float *b_tscale)
 {
-    const uint8_t *a_scales = a_scales_mma, *b_scales = b_scales_mma;
     if (M < 0 || N < 0 || K < 0) return bad("negative size");
     if (K % 32) return bad("K must be a multiple of 32");
     if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
@@ -464,22 +464,26 @@ mxq_status mxq_mxfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales_mma, c
         return MXQ_OK;
     }
     if (!a_codes || !a_scales || !b_codes || !b_scales) return bad("null pointer");
+    if (nv && (!a_tscale || !b_tscale)) return bad("null pointer");
     if (!aligned(a_codes, 16) || !aligned(b_codes, 16)) return bad("codes must be 16-byte aligned");
     if (!aligned(a_scales, 16) || !aligned(b_scales, 16)) return bad("scale atoms must be 16-byte aligned");
-    const uint64_t nca = static_cast<uint64_t>(M) * (K / 2), nsa = mxq_scales_mma_bytes(M, K);
-    const uint64_t ncb = static_cast<uint64_t>(N) * (K / 2), nsb = mxq_scales_mma_bytes(N, K);
-    const void *ins[4] = {a_codes, a_scales, b_codes, b_scales};
-    const uint64_t nins[4] = {nca, nsa, ncb, nsb};
-    for (int i = 0; i < 4; ++i)
-        if (overlaps(out, ny, ins[i], nins[i])) return bad("the output overlaps an input");
+    if (nv && (!aligned(a_tscale, 4) || !aligned(b_tscale, 4))) return bad("tensor scales must be 4-byte aligned");
+    const uint64_t nca = static_cast<uint64_t>(M) * (K / 2), ncb = static_cast<uint64_t>(N) * (K / 2);
+    const uint64_t nsa = nv ? mxq_nvfp4_scales_mma_bytes(M, K) : mxq_scales_mma_bytes(M, K);
+    const uint64_t nsb = nv ? mxq_nvfp4_scales_mma_bytes(N, K) : mxq_scales_mma_bytes(N, K);
+    const void *ins[6] = {a_codes, a_scales, b_codes, b_scales, a_tscale, b_tscale};
+    const uint64_t nins[6] = {nca, nsa, ncb, nsb, nv ? 4u : 0u, nv ? 4u : 0u};
+    for (int i = 0; i < 6; ++i)
+        if (ins[i] && overlaps(out, ny, ins[i], nins[i])) return bad("the output overlaps an input");
     if ((st = current_device(&dev, &sms)) != MXQ_OK) return st;
-    for (int i = 0; i < 4; ++i)
-        if ((st = check_buffer(ins[i], nins[i], dev)) != MXQ_OK) return st;
+    for (int i = 0; i < 6; ++i)
+        if (ins[i] && nins[i] && (st = check_buffer(ins[i], nins[i], dev)) != MXQ_OK) return st;
     if ((st = check_buffer(out, ny, dev)) != MXQ_OK) return st;
     alignas(64) CUtensorMap map_a, map_b, map_sfa, map_sfb;
     if ((st = make_tmap_operand(&map_a, a_codes, M, K, 128)) != MXQ_OK) return st;
     if ((st = make_tmap_operand(&map_b, b_codes, N, K, 128)) != MXQ_OK) return st;   // a CTA's half of B
-    const int64_t cb_n = (K / 32 + 3) / 4;
+    // scale atoms per 128-row block: one per 128 k (MXFP4) or per 64 k (NVFP4)
+    const int64_t cb_n = nv ? (K / 16 + 3) / 4 : (K / 32 + 3) / 4;
     if ((st = make_tmap_sf(&map_sfa, a_scales, (M + 127) / 128, cb_n, 1)) != MXQ_OK) return st;
     if ((st = make_tmap_sf(&map_sfb, b_scales, (N + 127) / 128, cb_n, 2)) != MXQ_OK) return st;
     mxq::GemmArgs g{};
@@ -488,12 +492,60 @@ mxq_status mxq_mxfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales_mma, c
     g.N = N;
     g.K = K;
     g.out_bf16 = out_bf16;
+    g.nvfp4 = nv;
+    g.a_tscale = a_tscale;
+    g.b_tscale = b_tscale;
     const cudaError_t e = mxq::launch_mxfp4_gemm(map_a, map_b, map_sfa, map_sfb, g, sms, s);
     if (e != cudaSuccess) {
-        note_cuda(e, "launch MXFP4 GEMM kernel");
+        note_cuda(e, nv ? "launch NVFP4 GEMM kernel" : "launch MXFP4 GEMM kernel");
         return MXQ_ERR_CUDA;
     }
     return MXQ_OK;
+}
+
+mxq_status mxq_mxfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales_mma, const uint8_t *b_codes,
+                          const uint8_t *b_scales_mma, int64_t M, int64_t N, int64_t K, void *out, int out_bf16,
+                          void *stream)
+{
+    return gemm_common(a_codes, a_scales_mma, b_codes, b_scales_mma, M, N, K, out, out_bf16, stream, 0, nullptr,
+                       nullptr);
+}
+
+size_t mxq_nvfp4_scales_mma_bytes(int64_t rows, int64_t K)
+{
+    if (rows <= 0 || K <= 0 || K % 32) return 0;
+    return static_cast<size_t>((rows + 127) / 128) * static_cast<size_t>((K / 16 + 3) / 4) * 512;
+}
+
+mxq_status mxq_nvfp4_scales_to_mma_layout(const uint8_t *scales, int64_t rows, int64_t K, uint8_t *out, void *stream)
+{
+    if (rows < 0 || K < 0 || K % 32) return bad("rows >= 0 and K a multiple of 32 required");
+    if (rows >= (int64_t(1) << 31) || K >= (int64_t(1) << 31)) return bad("rows and K must be < 2^31");
+    if (rows == 0 || K == 0) return MXQ_OK;
+    if (!scales || !out) return bad("null pointer");
+    if (!aligned(out, 16)) return bad("out must be 16-byte aligned");
+    const uint64_t ns = static_cast<uint64_t>(rows) * (K / 16), no = mxq_nvfp4_scales_mma_bytes(rows, K);
+    if (overlaps(out, no, scales, ns)) return bad("the output overlaps the input");
+    int dev = 0, sms = 0;
+    mxq_status st;
+    if ((st = current_device(&dev, &sms)) != MXQ_OK) return st;
+    if ((st = check_buffer(scales, ns, dev)) != MXQ_OK) return st;
+    if ((st = check_buffer(out, no, dev)) != MXQ_OK) return st;
+    // the same 512-byte atoms, four scale columns each: here a column is 16 k
+    const cudaError_t e = mxq::launch_scales_to_mma(scales, rows, K / 16, out, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) {
+        note_cuda(e, "launch scale layout kernel");
+        return MXQ_ERR_CUDA;
+    }
+    return MXQ_OK;
+}
+
+mxq_status mxq_nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales_mma, const float *a_tensor_scale,
+                          const uint8_t *b_codes, const uint8_t *b_scales_mma, const float *b_tensor_scale, int64_t M,
+                          int64_t N, int64_t K, void *out, int out_bf16, void *stream)
+{
+    return gemm_common(a_codes, a_scales_mma, b_codes, b_scales_mma, M, N, K, out, out_bf16, stream, 1,
+                       a_tensor_scale, b_tensor_scale);
 }
 
 mxq_status mxq_dequantize(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t cols,

@@ -58,6 +58,9 @@ struct GemmArgs {
     void *y;                   // [M, N] fp32 or bf16, row-major, 16-byte aligned
     int64_t M, N, K;
     int out_bf16;
+    int nvfp4;                 // 0: MXFP4 (E8M0 per 32 k); 1: NVFP4 (E4M3 per 16 k, times the tensor scales)
+    const float *a_tscale;     // NVFP4: the operands' fp32 tensor scales (device, one float each)
+    const float *b_tscale;
 };
 // The GEMM runs on CTA pairs (cta_group::2, 256 x 256 tiles): tmap_a / tmap_b in boxes of
 // 128 rows x 128 B; tmap_sfa / tmap_sfb: the scale atoms as uint32 [row blocks][cb_n * 128],

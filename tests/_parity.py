@@ -18,6 +18,22 @@ import numpy as np
 import oracle
 
 
+def unpack(codes):
+    """[rows, cols/2] packed bytes -> [rows, cols] 4-bit codes (even column = low nibble).  The
+    tests' own helper: GPU outputs are never fed to the oracle, not even to unpack them."""
+    codes = np.asarray(codes, np.uint8)
+    out = np.empty(codes.shape[:-1] + (codes.shape[-1] * 2,), np.uint8)
+    out[..., 0::2] = codes & 15
+    out[..., 1::2] = codes >> 4
+    return out
+
+
+def bf16_to_f64(bits):
+    """bf16 bit patterns (uint16) -> float64, exactly (bf16 is the top half of an fp32)."""
+    b = np.asarray(bits).astype(np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)
+
+
 def check_quant(x_bits, rhat_bits, lam, gpu_codes, gpu_scales, threads=None, exact=False, ref=None):
     """Compare GPU codes/scales for the rows of x_bits; returns a dict of counts (raises on failure).
 
@@ -41,8 +57,8 @@ def check_quant(x_bits, rhat_bits, lam, gpu_codes, gpu_scales, threads=None, exa
                              f"gpu {gpu_scales[r, g]:#x} oracle {ref['scales'][r, g]:#x} "
                              f"(y={ref['y'][r, 32 * g:32 * g + 32]})")
 
-    gc = oracle.unpack_codes(gpu_codes)
-    rc = oracle.unpack_codes(ref["codes"])
+    gc = unpack(gpu_codes)
+    rc = unpack(ref["codes"])
     same_scale = np.repeat(~sc_diff, 32, axis=1)
     diff = (gc != rc) & same_scale
     excused = (ref["eflags"] == 1) & (gc == ref["alt"])
@@ -60,7 +76,8 @@ def check_quant(x_bits, rhat_bits, lam, gpu_codes, gpu_scales, threads=None, exa
     for r, g in np.argwhere(sc_diff):
         n_alt_groups += 1
         y32 = ref["y"][r, 32 * g:32 * g + 32].astype(np.float32).astype(np.float64)
-        codes, flags, alt = oracle.quantize_group_at(y32, int(gpu_scales[r, g]))
+        # (the GPU's scale equals the oracle's alternative here: the oracle's value is the input)
+        codes, flags, alt = oracle.quantize_group_at(y32, int(ref["alt_scales"][r, g]))
         got = gc[r, 32 * g:32 * g + 32]
         ok = (got == codes) | ((flags == 1) & (got == alt))
         if not ok.all():
@@ -110,8 +127,8 @@ def check_nvfp4(x_bits, rhat_bits, lam, s_t, gpu_codes, gpu_scales, exact=False,
         raise AssertionError(f"E4M3 scale mismatch outside the band at row {r} block {b}: gpu "
                              f"{gpu_scales[r, b]:#x} oracle {ref['scales'][r, b]:#x} "
                              f"(y={ref['y'][r, 16 * b:16 * b + 16]})")
-    gc = oracle.unpack_codes(gpu_codes)
-    rc = oracle.unpack_codes(ref["codes"])
+    gc = unpack(gpu_codes)
+    rc = unpack(ref["codes"])
     diff = (gc != rc) & np.repeat(~sc_diff, 16, axis=1)
     bad = diff & ~((ref["eflags"] == 1) & (gc == ref["alt"]))
     if bad.any():
@@ -122,7 +139,8 @@ def check_nvfp4(x_bits, rhat_bits, lam, s_t, gpu_codes, gpu_scales, exact=False,
     n_alt = 0
     for r, b in np.argwhere(sc_diff):
         n_alt += 1
-        codes, flags, alt = oracle.nvfp4_block_at(ref["y"][r, 16 * b:16 * b + 16], int(gpu_scales[r, b]), s_t)
+        # (the GPU's scale equals the oracle's alternative here: the oracle's value is the input)
+        codes, flags, alt = oracle.nvfp4_block_at(ref["y"][r, 16 * b:16 * b + 16], int(ref["alt_scales"][r, b]), s_t)
         got = gc[r, 16 * b:16 * b + 16]
         if not ((got == codes) | ((flags == 1) & (got == alt))).all():
             raise AssertionError(f"block at row {r} block {b} under the neighbouring scale does not match")

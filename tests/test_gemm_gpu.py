@@ -125,8 +125,10 @@ def test_weight_side_matches_oracle(use_lam):
 def test_chain_downproj_full_size():
     # The layer end to end on the 8192 x 14336 down-projection activations and a synthetic
     # 4096 x 14336 weight (N(0, 1/K)): X -> MXFP4(X Λ⁻¹ R̂), Wᵀ -> MXFP4(Wᵀ Λ R̂), then the GEMM.
-    # Sampled rows of Y against the oracle GEMM of the GPU's own operands, and the weight codes
-    # against the oracle's weight quantiser on sampled rows.
+    #  - both GPU quantisers against the oracle's (parity rule) on sampled rows;
+    #  - the GPU GEMM on the oracle's operands (uploaded) against the oracle GEMM of them;
+    #  - the GPU chain (its own operands) equals that GEMM bit for bit wherever its operands
+    #    equal the oracle's.  The oracle never takes GPU output.
     w = synth.make_config(3)
     K, N = w.cols, 4096
     wt = synth.random_bf16(N, K, seed=77, scale=1.0 / np.sqrt(K))
@@ -134,23 +136,36 @@ def test_chain_downproj_full_size():
     rhat = w.rhat.to(DEV)
     ca, sa = mxq.smooth_rotate_quantize(w.x.to(DEV), rhat, lam.to(DEV))
     cb, sb = mxq.weight_rotate_quantize(wt.to(DEV), rhat, lam.to(DEV))
-    y = mxq.mxfp4_gemm(ca, sa, cb, sb)
+    y_chain = mxq.mxfp4_gemm(ca, sa, cb, sb)
     mxq.sync_check()
-    rows_s = synth.sample_rows(w.rows, 48, seed=8100, must=w.outlier_rows)
-    idx = torch.from_numpy(rows_s).to(DEV)
-    a_s, sa_s = ca.index_select(0, idx).cpu().numpy(), sa.index_select(0, idx).cpu().numpy()
-    b_np, sb_np = cb.cpu().numpy(), sb.cpu().numpy()
     th = oracle.default_threads()
-    ref = oracle.mxfp4_gemm(a_s, sa_s, b_np, sb_np, threads=th)
-    mag = oracle.mxfp4_gemm(_abs_codes(a_s), sa_s, _abs_codes(b_np), sb_np, threads=th)
-    got = y.index_select(0, idx).cpu().numpy().astype(np.float64)
-    assert (np.abs(got - ref) <= 1e-5 * mag).all()
+    rows_s = synth.sample_rows(w.rows, 48, seed=8100, must=w.outlier_rows)
+    idx = torch.from_numpy(rows_s)
+    xs = synth.bf16_bits(w.x[idx])
+    qa = oracle.smooth_rotate_quantize(xs, synth.bf16_bits(w.rhat), lam.numpy(), want_y=True, flags=True, threads=th)
+    qb = oracle.weight_rotate_quantize(synth.bf16_bits(wt), synth.bf16_bits(w.rhat), lam.numpy(), want_y=True,
+                                       flags=True, threads=th)
+    ga, gsa = ca.index_select(0, idx.to(DEV)).cpu().numpy(), sa.index_select(0, idx.to(DEV)).cpu().numpy()
+    gb, gsb = cb.cpu().numpy(), sb.cpu().numpy()
+    _parity.check_quant(xs, None, None, ga, gsa, ref=qa)
     wrows = synth.sample_rows(N, 64, seed=8200)
-    wb = synth.bf16_bits(wt[torch.from_numpy(wrows)])
-    refw = oracle.weight_rotate_quantize(wb, synth.bf16_bits(w.rhat), lam.numpy(), want_y=True, flags=True,
-                                         threads=th)
-    _parity.check_quant(wb, None, None, cb.index_select(0, torch.from_numpy(wrows).to(DEV)).cpu().numpy(),
-                        sb.index_select(0, torch.from_numpy(wrows).to(DEV)).cpu().numpy(), ref=refw)
+    _parity.check_quant(synth.bf16_bits(wt[torch.from_numpy(wrows)]), None, None, gb[wrows], gsb[wrows],
+                        ref={k: v[wrows] for k, v in qb.items()})
+    # the GEMM on the oracle's operands
+    ops = [torch.from_numpy(np.ascontiguousarray(v)).to(DEV) for v in (qa["codes"], qa["scales"], qb["codes"],
+                                                                       qb["scales"])]
+    y_o = mxq.mxfp4_gemm(*ops)
+    mxq.sync_check()
+    ref = oracle.mxfp4_gemm(qa["codes"], qa["scales"], qb["codes"], qb["scales"], threads=th)
+    mag = oracle.mxfp4_gemm(_abs_codes(qa["codes"]), qa["scales"], _abs_codes(qb["codes"]), qb["scales"], threads=th)
+    got = y_o.cpu().numpy().astype(np.float64)
+    assert (np.abs(got - ref) <= 1e-5 * mag).all()
+    # the chain where its operands are the oracle's
+    row_ok = (ga == qa["codes"]).all(1) & (gsa == qa["scales"]).all(1)
+    col_ok = (gb == qb["codes"]).all(1) & (gsb == qb["scales"]).all(1)
+    assert row_ok.mean() > 0.5 and col_ok.mean() > 0.5
+    chain = y_chain.index_select(0, idx.to(DEV)).cpu().numpy()
+    assert np.array_equal(chain[row_ok][:, col_ok], y_o.cpu().numpy()[row_ok][:, col_ok])
 
 
 @pytest.mark.parametrize("rows,K", [(1, 32), (300, 416), (128, 4096), (4096, 14336)])
@@ -160,3 +175,115 @@ def test_scale_layout_matches_oracle(rows, K):
     got = mxq.scales_to_mma_layout(torch.from_numpy(sc).to(DEV))
     mxq.sync_check()
     assert np.array_equal(got.cpu().numpy(), oracle.scales_to_mma(sc))
+
+
+# ---------------------------------------------------------------- the NVFP4 consumer GEMM
+
+def _rand_nv(rng, rows, K):
+    # E4M3 scale codes in [0x20, 0x48): normal values 2^-3 .. 2^2
+    return (rng.integers(0, 256, (rows, K // 2), dtype=np.uint8),
+            rng.integers(0x20, 0x48, (rows, K // 16), dtype=np.uint8))
+
+
+def _gpu_nv(a, sa, ta, b, sb, tb, out_dtype=torch.float32):
+    t = [torch.from_numpy(np.ascontiguousarray(v)).to(DEV) for v in (a, sa, b, sb)]
+    ts = [torch.tensor([v], dtype=torch.float32, device=DEV) for v in (ta, tb)]
+    y = mxq.nvfp4_gemm(t[0], t[1], ts[0], t[2], t[3], ts[1], out_dtype=out_dtype)
+    mxq.sync_check()
+    return y.float().cpu().numpy().astype(np.float64)
+
+
+def _check_nv(a, sa, ta, b, sb, tb, exact=False, rel=1e-5):
+    th = oracle.default_threads()
+    ref = oracle.nvfp4_gemm(a, sa, ta, b, sb, tb, threads=th)
+    mag = oracle.nvfp4_gemm(_abs_codes(a), sa, abs(ta), _abs_codes(b), sb, abs(tb), threads=th)
+    got = _gpu_nv(a, sa, ta, b, sb, tb)
+    if exact:
+        assert np.array_equal(got, ref)
+    else:
+        bad = ~(np.abs(got - ref) <= rel * mag)
+        assert not bad.any(), f"{bad.sum()} elements off; first at {np.argwhere(bad)[0]}"
+    gb = _gpu_nv(a, sa, ta, b, sb, tb, torch.bfloat16)
+    assert (np.abs(gb - ref) <= rel * mag + 2.0 ** -8 * np.abs(ref)).all()
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (1, 1, 32), (129, 257, 288), (300, 520, 1024), (64, 1000, 96),
+                                   (2300, 2250, 800)])
+def test_nvfp4_gemm_matches_oracle(M, N, K):
+    rng = np.random.default_rng(M + 3 * N + 17 * K)
+    a, sa = _rand_nv(rng, M, K)
+    b, sb = _rand_nv(rng, N, K)
+    _check_nv(a, sa, 0.37, b, sb, 1.9)
+
+
+def test_nvfp4_gemm_exact_with_unit_scales():
+    rng = np.random.default_rng(2)
+    M, N, K = 200, 300, 2048
+    a = rng.integers(0, 256, (M, K // 2), dtype=np.uint8)
+    b = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    one = 0x38   # E4M3 1.0
+    _check_nv(a, np.full((M, K // 16), one, np.uint8), 1.0, b, np.full((N, K // 16), one, np.uint8), 1.0, exact=True)
+
+
+def test_nvfp4_gemm_nan_scale_and_bad_arguments():
+    rng = np.random.default_rng(3)
+    a, sa = _rand_nv(rng, 8, 64)
+    b, sb = _rand_nv(rng, 8, 64)
+    sa[1, 2] = 0x7F
+    got = _gpu_nv(a, sa, 1.0, b, sb, 1.0)
+    assert np.isnan(got[1]).all() and not np.isnan(np.delete(got, 1, axis=0)).any()
+    t = [torch.from_numpy(v).to(DEV) for v in (a, sa, b, sb)]
+    one = torch.ones(1, dtype=torch.float32, device=DEV)
+    with pytest.raises(ValueError):
+        mxq.nvfp4_gemm(t[0], t[1], torch.ones(2, dtype=torch.float32, device=DEV), t[2], t[3], one)
+    # a tensor scale in host memory is refused before any launch
+    sfa = mxq.nvfp4_scales_to_mma_layout(t[1])
+    sfb = mxq.nvfp4_scales_to_mma_layout(t[3])
+    y = torch.empty((8, 8), dtype=torch.float32, device=DEV)
+    host = torch.ones(1, dtype=torch.float32)
+    rc = mxq.lib().mxq_nvfp4_gemm(t[0].data_ptr(), sfa.data_ptr(), host.data_ptr(), t[2].data_ptr(), sfb.data_ptr(),
+                                  one.data_ptr(), 8, 8, 64, y.data_ptr(), 0, None)
+    assert rc == 1
+
+
+def test_nvfp4_chain():
+    # NVFP4(X R̂) and NVFP4(Wᵀ R̂) by the GPU quantiser, against the oracle's; the GPU GEMM on the
+    # oracle's operands against the oracle GEMM; the GPU chain equals it where its operands do
+    rows, K, N = 1024, 4096, 512
+    w = synth.make_config(2, rows=rows, cols=K)
+    wt = synth.random_bf16(N, K, seed=78, scale=1.0 / np.sqrt(K))
+    th = oracle.default_threads()
+    xb, wb, rb = synth.bf16_bits(w.x), synth.bf16_bits(wt), synth.bf16_bits(w.rhat)
+    ya = oracle.nvfp4_quantize(xb, rb, None, 1.0, want_y=True, threads=th)["y"]
+    yb = oracle.nvfp4_quantize(wb, rb, None, 1.0, want_y=True, threads=th)["y"]
+    ta = float(np.float32(np.abs(ya).max() / (6 * 448)))
+    tb = float(np.float32(np.abs(yb).max() / (6 * 448)))
+    qa = oracle.nvfp4_quantize(xb, rb, None, ta, want_y=True, flags=True, threads=th)
+    qb = oracle.nvfp4_quantize(wb, rb, None, tb, want_y=True, flags=True, threads=th)
+    tta = torch.tensor([ta], dtype=torch.float32, device=DEV)
+    ttb = torch.tensor([tb], dtype=torch.float32, device=DEV)
+    ca, sa = mxq.smooth_rotate_quantize_nvfp4(w.x.to(DEV), w.rhat.to(DEV), tta)
+    cb, sb = mxq.smooth_rotate_quantize_nvfp4(wt.to(DEV), w.rhat.to(DEV), ttb)
+    y_chain = mxq.nvfp4_gemm(ca, sa, tta, cb, sb, ttb)
+    mxq.sync_check()
+    ga, gsa, gb, gsb = (v.cpu().numpy() for v in (ca, sa, cb, sb))
+    _parity.check_nvfp4(xb, rb, None, ta, ga, gsa)
+    _parity.check_nvfp4(wb, rb, None, tb, gb, gsb)
+    ops = [torch.from_numpy(v).to(DEV) for v in (qa["codes"], qa["scales"], qb["codes"], qb["scales"])]
+    y_o = mxq.nvfp4_gemm(ops[0], ops[1], tta, ops[2], ops[3], ttb)
+    mxq.sync_check()
+    ref = oracle.nvfp4_gemm(qa["codes"], qa["scales"], ta, qb["codes"], qb["scales"], tb, threads=th)
+    mag = oracle.nvfp4_gemm(_abs_codes(qa["codes"]), qa["scales"], ta, _abs_codes(qb["codes"]), qb["scales"], tb,
+                            threads=th)
+    assert (np.abs(y_o.cpu().numpy().astype(np.float64) - ref) <= 1e-5 * mag).all()
+    row_ok = (ga == qa["codes"]).all(1) & (gsa == qa["scales"]).all(1)
+    col_ok = (gb == qb["codes"]).all(1) & (gsb == qb["scales"]).all(1)
+    assert row_ok.mean() > 0.5 and col_ok.mean() > 0.5
+    assert np.array_equal(y_chain.cpu().numpy()[row_ok][:, col_ok], y_o.cpu().numpy()[row_ok][:, col_ok])
+    # and the layer approximates X Wᵀ (R̂ orthogonal): relative Frobenius error of NVFP4 x NVFP4
+    xw = synth.bf16_bits(w.x).astype(np.uint32)
+    xf = (xw << 16).view(np.float32).astype(np.float64)
+    wf = (synth.bf16_bits(wt).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    exact = xf @ wf.T
+    rel = np.linalg.norm(y_chain.cpu().numpy() - exact) / np.linalg.norm(exact)
+    assert rel < 0.25

@@ -232,8 +232,8 @@ def test_dequant_plain_bit_exact():
     ref = oracle.dequantize(codes, scales, cols)
     got = mxq.dequantize(torch.from_numpy(codes).to(DEV), torch.from_numpy(scales).to(DEV))
     got = synth.bf16_bits(got.cpu())
-    ref_nan = np.isnan(oracle.bf16_bits_to_f64(ref))
-    got_nan = np.isnan(oracle.bf16_bits_to_f64(got))
+    ref_nan = np.isnan(_parity.bf16_to_f64(ref))
+    got_nan = np.isnan(_parity.bf16_to_f64(got))
     assert np.array_equal(ref_nan, got_nan)
     assert np.array_equal(ref[~ref_nan], got[~got_nan])
 
@@ -256,17 +256,17 @@ def test_dequant_inverse_rotation(rows, cols, lam_kind):
         lam_dev = torch.cat([torch.zeros(1), lam]).to(DEV)[1:]   # 4-byte but not 16-byte aligned
         assert lam_dev.data_ptr() % 16 != 0
     got = mxq.dequantize(torch.from_numpy(codes).to(DEV), torch.from_numpy(scales).to(DEV), r.to(DEV), lam_dev)
-    got64 = oracle.bf16_bits_to_f64(synth.bf16_bits(got.cpu()))
+    got64 = _parity.bf16_to_f64(synth.bf16_bits(got.cpu()))
     # bound: one bf16 ulp of the exact value plus fp32 accumulation error of 32 terms
-    v = oracle.bf16_bits_to_f64(oracle.dequantize(codes, scales, cols))
-    rr = oracle.bf16_bits_to_f64(_bits(r))
+    v = _parity.bf16_to_f64(oracle.dequantize(codes, scales, cols))
+    rr = _parity.bf16_to_f64(_bits(r))
     s_abs = (np.abs(v).reshape(rows, cols // 32, 32) @ np.abs(rr).T).reshape(rows, cols)
     if lam is not None:
         s_abs = s_abs * lam.numpy()[None, :]
     tol = 2.0 ** -7 * np.abs(ref64) + 2.0 ** -18 * s_abs
     assert (np.abs(got64 - ref64) <= tol).all()
     # most outputs round to the same bf16 as the exact value
-    assert (got64 == oracle.bf16_bits_to_f64(ref_bits)).mean() > 0.99
+    assert (got64 == _parity.bf16_to_f64(ref_bits)).mean() > 0.99
 
 
 # ---------------------------------------------------------------- full-size configurations
@@ -300,24 +300,24 @@ def test_full_config5_with_round_trip():
     back = mxq.dequantize(codes, scales, rd, ld)
     mxq.sync_check()
     idx = torch.from_numpy(rows_s).to(DEV)
-    got = oracle.bf16_bits_to_f64(synth.bf16_bits(back.index_select(0, idx).cpu()))
+    got = _parity.bf16_to_f64(synth.bf16_bits(back.index_select(0, idx).cpu()))
     ref = res["ref"]
     ref_back_bits, ref_back = oracle.dequantize(ref["codes"], ref["scales"], w.cols, _bits(w.rhat),
                                                 w.lam.numpy(), want_f64=True)
     # compare where the GPU's codes and scales equal the oracle's (elsewhere a boundary tie differs)
     gc = codes.index_select(0, idx).cpu().numpy()
     gs = scales.index_select(0, idx).cpu().numpy()
-    same = (oracle.unpack_codes(gc) == oracle.unpack_codes(ref["codes"])).reshape(len(rows_s), -1, 32).all(2)
+    same = (_parity.unpack(gc) == _parity.unpack(ref["codes"])).reshape(len(rows_s), -1, 32).all(2)
     same &= gs == ref["scales"]
     mask = np.repeat(same, 32, axis=1)
-    v = oracle.bf16_bits_to_f64(oracle.dequantize(ref["codes"], ref["scales"], w.cols))
-    rr = oracle.bf16_bits_to_f64(_bits(w.rhat))
+    v = _parity.bf16_to_f64(oracle.dequantize(ref["codes"], ref["scales"], w.cols))
+    rr = _parity.bf16_to_f64(_bits(w.rhat))
     s_abs = (np.abs(v).reshape(len(rows_s), -1, 32) @ np.abs(rr).T).reshape(len(rows_s), -1)
     s_abs *= w.lam.numpy()[None, :]
     tol = 2.0 ** -7 * np.abs(ref_back) + 2.0 ** -18 * s_abs
     assert (np.abs(got - ref_back)[mask] <= tol[mask]).all()
     # round trip error relative to the input, per group: the MXFP4 error budget of an orthogonal map
-    x = oracle.bf16_bits_to_f64(synth.bf16_bits(w.x[torch.from_numpy(rows_s)]))
+    x = _parity.bf16_to_f64(synth.bf16_bits(w.x[torch.from_numpy(rows_s)]))
     rel = np.linalg.norm((got - x).reshape(len(rows_s), -1, 32), axis=2) / \
         np.maximum(np.linalg.norm(x.reshape(len(rows_s), -1, 32), axis=2), 1e-30)
     assert np.median(rel) < 0.2
