@@ -24,7 +24,8 @@ import torch
 __all__ = [
     "MxqError", "smooth_rotate_quantize", "smooth_rotate_quantize_nvfp4", "smooth_rotate_f32",
     "weight_rotate_quantize", "rotate_quantize_block", "rotate_block_f32", "scales_to_mma_layout",
-    "mxfp4_gemm", "nvfp4_scales_to_mma_layout", "nvfp4_gemm", "dequantize", "quant_error", "rotation_search", "sync_check", "selftest_bounded_wait",
+    "mxfp4_gemm", "nvfp4_scales_to_mma_layout", "nvfp4_gemm", "dequantize", "quant_error", "rotation_search",
+    "sync_check", "selftest_bounded_wait",
     "status_string", "version", "lib", "LIB_PATH", "HEADER_PATH", "declared_symbols",
 ]
 
