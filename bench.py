@@ -394,7 +394,8 @@ def run_extras(mxq, w, xs, rhat, outs, dev, stream, k=300):
 
     def qerr(i):
         import ctypes
-        st = mxq.lib().mxq_quant_error(ctypes.c_void_p(xs[i & 1].data_ptr()), rows, cols, ctypes.c_void_p(rhat.data_ptr()),
+        st = mxq.lib().mxq_quant_error(ctypes.c_void_p(xs[i & 1].data_ptr()), rows, cols,
+                                       ctypes.c_void_p(rhat.data_ptr()),
                                        None, ctypes.c_void_p(errs.data_ptr()), ctypes.c_void_p(mean.data_ptr()),
                                        ctypes.c_void_p(ws.data_ptr()), ws.numel(), ctypes.c_void_p(stream.cuda_stream))
         assert st == 0

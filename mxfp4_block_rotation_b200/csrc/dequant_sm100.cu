@@ -145,8 +145,8 @@ __host__ __device__ constexpr int dq_lam_bytes(int epi, int lam)
 }
 __host__ __device__ constexpr int dq_smem_bytes(int epi, int lam)
 {
-    return kDqStages * kDqStageBytes + kBMatBytes + kDqCStages * kDqCodeBytes + dq_out_bytes(epi) + dq_lam_bytes(epi, lam) +
-           512 + 128 + 1024;
+    return kDqStages * kDqStageBytes + kBMatBytes + kDqCStages * kDqCodeBytes + dq_out_bytes(epi) +
+           dq_lam_bytes(epi, lam) + 512 + 128 + 1024;
 }
 static_assert(dq_smem_bytes(DqSplit<0>::kEpi, 0) <= 232448 && dq_smem_bytes(DqSplit<1>::kEpi, 1) <= 232448 &&
                   dq_smem_bytes(DqSplit<2>::kEpi, 2) <= 232448,
@@ -447,15 +447,14 @@ cudaError_t launch_dequant_rot(const CUtensorMap &tmap_out, const uint8_t *codes
     if (!status) return cudaErrorInvalidSymbol;
     const uint4 *c4 = reinterpret_cast<const uint4 *>(codes);
     if (!lambda)
-        return launch_pdl(dequant_rot_kernel<0>, grid, kDqThreads, dq_smem_bytes(DqSplit<0>::kEpi, 0), stream, tmap_out, c4, scales,
-                          n_groups, G, rhat, lambda, status);
+        return launch_pdl(dequant_rot_kernel<0>, grid, kDqThreads, dq_smem_bytes(DqSplit<0>::kEpi, 0), stream,
+                          tmap_out, c4, scales, n_groups, G, rhat, lambda, status);
     // all of Lambda fits the per-warp buffers' space (and can be copied in 16-byte pieces): keep it resident
     if (G <= kDqLamTableRows && (reinterpret_cast<uintptr_t>(lambda) & 15) == 0)
-        return launch_pdl(dequant_rot_kernel<2>, grid, kDqThreads, dq_smem_bytes(DqSplit<2>::kEpi, 2), stream, tmap_out,
-                          c4, scales,
-                          n_groups, G, rhat, lambda, status);
-    return launch_pdl(dequant_rot_kernel<1>, grid, kDqThreads, dq_smem_bytes(DqSplit<1>::kEpi, 1), stream, tmap_out, c4, scales,
-                      n_groups, G, rhat, lambda, status);
+        return launch_pdl(dequant_rot_kernel<2>, grid, kDqThreads, dq_smem_bytes(DqSplit<2>::kEpi, 2), stream,
+                          tmap_out, c4, scales, n_groups, G, rhat, lambda, status);
+    return launch_pdl(dequant_rot_kernel<1>, grid, kDqThreads, dq_smem_bytes(DqSplit<1>::kEpi, 1), stream,
+                      tmap_out, c4, scales, n_groups, G, rhat, lambda, status);
 }
 
 cudaError_t launch_dequant_plain(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t cols,
@@ -466,8 +465,8 @@ cudaError_t launch_dequant_plain(const uint8_t *codes, const uint8_t *scales, in
     const int64_t want = (n_chunks + kPlainThreads - 1) / kPlainThreads;
     const int64_t cap = static_cast<int64_t>(num_sms) * 8;
     const int grid = static_cast<int>(want < cap ? want : cap);
-    dequant_plain_kernel<<<grid, kPlainThreads, 0, stream>>>(reinterpret_cast<const uint32_t *>(codes), scales, n_chunks,
-                                                        reinterpret_cast<uint4 *>(out));
+    dequant_plain_kernel<<<grid, kPlainThreads, 0, stream>>>(reinterpret_cast<const uint32_t *>(codes), scales,
+                                                             n_chunks, reinterpret_cast<uint4 *>(out));
     return cudaGetLastError();
 }
 

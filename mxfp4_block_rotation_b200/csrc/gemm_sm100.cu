@@ -172,8 +172,8 @@ __device__ __forceinline__ uint64_t policy_evict_last()
 
 // 32 accumulator columns of one output row (col0 < N) as bf16 or fp32: 16-byte stores
 // when the row's chunk is whole and aligned, element stores at the right edge.
-__device__ __forceinline__ void store_row_chunk(const GemmArgs &args, int64_t row, int64_t col0, const uint32_t (&cur)[32],
-                                                bool vec)
+__device__ __forceinline__ void store_row_chunk(const GemmArgs &args, int64_t row, int64_t col0,
+                                                const uint32_t (&cur)[32], bool vec)
 {
     if (args.out_bf16) {
         uint16_t *dst = static_cast<uint16_t *>(args.y) + row * args.N + col0;
@@ -365,7 +365,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
                         const uint32_t sfa = (tmem_base + C::sfa_col(s) + 4 * c) | (byte << 30);
                         const uint32_t sfb = (tmem_base + C::sfb_col(s) + 8 * c) | (byte << 30);
                         const uint32_t idesc = idesc0 | (byte << 29) | (byte << 4);
-                        const uint64_t ad = ptx::smem_desc_sw128(a_base + j * 32), bd = ptx::smem_desc_sw128(b_base + j * 32);
+                        const uint64_t ad = ptx::smem_desc_sw128(a_base + j * 32);
+                        const uint64_t bd = ptx::smem_desc_sw128(b_base + j * 32);
                         if constexpr (kNv)
                             mma_nvf4_pair(tmem_base, ad, bd, idesc, sfa, sfb, static_cast<uint32_t>(kt | j));
                         else

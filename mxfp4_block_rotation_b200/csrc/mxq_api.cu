@@ -192,7 +192,8 @@ mxq_status make_tmap_groups(CUtensorMap *map, const void *X, int64_t rows, int64
 mxq_status make_tmap_blocks(CUtensorMap *map, const void *X, int64_t rows, int64_t cols, int blk)
 {
     const Driver &d = driver();
-    cuuint64_t dims[2] = {static_cast<cuuint64_t>(blk), static_cast<cuuint64_t>(rows) * static_cast<cuuint64_t>(cols / blk)};
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(blk),
+                          static_cast<cuuint64_t>(rows) * static_cast<cuuint64_t>(cols / blk)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(blk) * 2};
     cuuint32_t box[2] = {64, static_cast<cuuint32_t>(16384 / blk)};
     cuuint32_t estr[2] = {1, 1};
@@ -578,8 +579,9 @@ mxq_status mxq_dequantize(const uint8_t *codes, const uint8_t *scales, int64_t r
     if (Rhat_bf16_or_null) {
         alignas(64) CUtensorMap map_out;
         if ((st = make_tmap_groups(&map_out, out_bf16, rows, cols, 32)) != MXQ_OK) return st;
-        e = mxq::launch_dequant_rot(map_out, codes, scales, rows, cols, static_cast<const uint16_t *>(Rhat_bf16_or_null),
-                                    Lambda_or_null, sms, static_cast<cudaStream_t>(stream));
+        e = mxq::launch_dequant_rot(map_out, codes, scales, rows, cols,
+                                    static_cast<const uint16_t *>(Rhat_bf16_or_null), Lambda_or_null, sms,
+                                    static_cast<cudaStream_t>(stream));
     } else {
         e = mxq::launch_dequant_plain(codes, scales, rows, cols, static_cast<uint16_t *>(out_bf16), sms,
                                       static_cast<cudaStream_t>(stream));
@@ -610,11 +612,13 @@ mxq_status mxq_quant_error(const void *X_bf16, int64_t rows, int64_t cols, const
     if (!aligned(X_bf16, 16)) return bad("X must be 16-byte aligned");
     if (!aligned(Rhat_bf16, 2)) return bad("Rhat must be 2-byte aligned");
     if (Lambda_or_null && !aligned(Lambda_or_null, 4)) return bad("Lambda must be 4-byte aligned");
-    if (out_group_err_or_null && !aligned(out_group_err_or_null, 4)) return bad("per-group errors must be 4-byte aligned");
+    if (out_group_err_or_null && !aligned(out_group_err_or_null, 4))
+        return bad("per-group errors must be 4-byte aligned");
     const size_t need = mxq_quant_error_workspace_bytes(rows, cols, Lambda_or_null != nullptr);
     if (!workspace || !aligned(workspace, 8) || workspace_bytes < need)
         return bad("workspace missing, not 8-byte aligned or smaller than mxq_quant_error_workspace_bytes()");
-    const uint64_t nx = static_cast<uint64_t>(rows) * cols * 2, nl = Lambda_or_null ? static_cast<uint64_t>(cols) * 4 : 0;
+    const uint64_t nx = static_cast<uint64_t>(rows) * cols * 2;
+    const uint64_t nl = Lambda_or_null ? static_cast<uint64_t>(cols) * 4 : 0;
     const uint64_t ne = out_group_err_or_null ? static_cast<uint64_t>(rows) * (cols / 32) * 4 : 0;
     const void *ins[3] = {X_bf16, Rhat_bf16, Lambda_or_null};
     const uint64_t nins[3] = {nx, 32 * 32 * 2, nl};
@@ -690,7 +694,8 @@ mxq_status mxq_rotation_search(const void *X_bf16, int64_t rows, int64_t cols, c
     const size_t need = mxq_rotation_search_workspace_bytes(rows, cols, n_angle);
     if (!workspace || !aligned(workspace, 256) || workspace_bytes < need)
         return bad("workspace missing, not 256-byte aligned or smaller than mxq_rotation_search_workspace_bytes()");
-    const uint64_t nx = static_cast<uint64_t>(rows) * cols * 2, nl = Lambda_or_null ? static_cast<uint64_t>(cols) * 4 : 0;
+    const uint64_t nx = static_cast<uint64_t>(rows) * cols * 2;
+    const uint64_t nl = Lambda_or_null ? static_cast<uint64_t>(cols) * 4 : 0;
     const void *ins[2] = {X_bf16, Lambda_or_null};
     const uint64_t nins[2] = {nx, nl};
     void *outs[7] = {R_out, Rhat_bf16_out_or_null, trace_out_or_null, linf_out_or_null, steps_out_or_null,

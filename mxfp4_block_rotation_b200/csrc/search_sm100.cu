@@ -66,8 +66,14 @@ struct SearchState {
 };
 static_assert(sizeof(SearchState) <= 512, "search state must fit its slot");
 
-__device__ __forceinline__ double bits_to_double(unsigned long long b) { return __longlong_as_double(static_cast<long long>(b)); }
-__device__ __forceinline__ unsigned long long double_to_bits(double v) { return static_cast<unsigned long long>(__double_as_longlong(v)); }
+__device__ __forceinline__ double bits_to_double(unsigned long long b)
+{
+    return __longlong_as_double(static_cast<long long>(b));
+}
+__device__ __forceinline__ unsigned long long double_to_bits(double v)
+{
+    return static_cast<unsigned long long>(__double_as_longlong(v));
+}
 
 // Givens grid: angle a of 2n, t = (a' - n) / n with a' = a (a < n) or a + 1,
 // c = (1 - t^2) / (1 + t^2), s = 2t / (1 + t^2).

@@ -45,8 +45,8 @@ def build_variant(mutant: int) -> str:
     os.makedirs(out_dir, exist_ok=True)
     path = os.path.join(out_dir, f"libmxq_oracle_m{int(mutant)}.so")
     if not os.path.exists(path) or os.path.getmtime(path) < os.path.getmtime(_SRC):
-        cmd = ["gcc", "-O2", "-std=c11", "-fno-fast-math", "-ffp-contract=off", "-fopenmp", f"-DMXQ_MUTANT={int(mutant)}",
-               "-shared", "-fPIC", "-o", path + ".tmp", _SRC, "-lm"]
+        cmd = ["gcc", "-O2", "-std=c11", "-fno-fast-math", "-ffp-contract=off", "-fopenmp",
+               f"-DMXQ_MUTANT={int(mutant)}", "-shared", "-fPIC", "-o", path + ".tmp", _SRC, "-lm"]
         subprocess.run(cmd, check=True)
         os.replace(path + ".tmp", path)
     return path
