@@ -383,24 +383,36 @@ def run_extras(mxq, w, xs, rhat, outs, dev, stream, k=300):
         mxq.dequantize(c, s, out=deq[i & 1], stream=stream)
     row("dequantize", _timed(dq_plain, k, stream, dev), deq_bytes, "codes + scales -> bf16 (rotated domain)")
 
+    def dq_rot(i):
+        c, s = outs[i & 1]
+        mxq.dequantize(c, s, rhat, out=deq[i & 1], stream=stream)
+    row("dequantize_inverse_rotation", _timed(dq_rot, k, stream, dev), deq_bytes, "codes + scales -> v * R^T -> bf16")
+
     def dq_inv(i):
         c, s = outs[i & 1]
         mxq.dequantize(c, s, rhat, lam, out=deq[i & 1], stream=stream)
     row("dequantize_inverse_rotation_and_smoothing", _timed(dq_inv, k, stream, dev), deq_bytes + 4 * cols,
         "codes + scales -> (v * R^T) * Lambda -> bf16")
-    ws = torch.empty(mxq.lib().mxq_quant_error_workspace_bytes(rows, cols, 0), dtype=torch.uint8, device=dev)
     errs = torch.empty((rows, cols // 32), dtype=torch.float32, device=dev)
     mean = torch.empty((), dtype=torch.float64, device=dev)
+    for lam_q in (None, lam):
+        ws = torch.empty(mxq.lib().mxq_quant_error_workspace_bytes(rows, cols, int(lam_q is not None)),
+                         dtype=torch.uint8, device=dev)
 
-    def qerr(i):
-        import ctypes
-        st = mxq.lib().mxq_quant_error(ctypes.c_void_p(xs[i & 1].data_ptr()), rows, cols,
-                                       ctypes.c_void_p(rhat.data_ptr()),
-                                       None, ctypes.c_void_p(errs.data_ptr()), ctypes.c_void_p(mean.data_ptr()),
-                                       ctypes.c_void_p(ws.data_ptr()), ws.numel(), ctypes.c_void_p(stream.cuda_stream))
-        assert st == 0
-    row("quant_error_per_group_and_mean", _timed(qerr, k, stream, dev), rows * cols * 2.0 + rows * (cols // 32) * 4.0,
-        "per-group ||Q(y)-y||/||y|| (fp32 out) and its mean: reads X, writes 4 B per group")
+        def qerr(i, lam_q=lam_q, ws=ws):
+            import ctypes
+            st = mxq.lib().mxq_quant_error(ctypes.c_void_p(xs[i & 1].data_ptr()), rows, cols,
+                                           ctypes.c_void_p(rhat.data_ptr()),
+                                           None if lam_q is None else ctypes.c_void_p(lam_q.data_ptr()),
+                                           ctypes.c_void_p(errs.data_ptr()), ctypes.c_void_p(mean.data_ptr()),
+                                           ctypes.c_void_p(ws.data_ptr()), ws.numel(),
+                                           ctypes.c_void_p(stream.cuda_stream))
+            assert st == 0
+        lam_bytes = 0.0 if lam_q is None else 4.0 * cols
+        row("quant_error_per_group_and_mean" + ("" if lam_q is None else "_with_lambda"),
+            _timed(qerr, k, stream, dev), rows * cols * 2.0 + rows * (cols // 32) * 4.0 + lam_bytes,
+            "per-group ||Q(y)-y||/||y|| (fp32 out) and its mean: reads X, writes 4 B per group" +
+            ("" if lam_q is None else "; y = X Lambda^-1 R (rotate_cols_kernel<Err>)"))
     # the rotation-block-size variants on the same X (no smoothing): B = 16, 64, 128
     for blk in (16, 64, 128):
         rblk = synth.rhat_tensor(synth.haar_orthogonal(300 + blk, n=blk)).to(dev)

@@ -14,23 +14,49 @@ namespace mxq {
 namespace {
 
 constexpr int kMeanThreads = 1024;
+constexpr int kMeanUnroll = 8;   // loads in flight per thread
 
+// Fixed-order sum of 32 lanes' values (the same tree every run); lane 0 holds it.
+__device__ __forceinline__ double warp_tree_sum(double v)
+{
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) v += __shfl_down_sync(0xffffffffu, v, off);
+    return v;
+}
+
+// One block.  Thread t adds the elements t + kMeanThreads * (kMeanUnroll * r + u) into
+// accumulator u, so each warp load reads 256 contiguous bytes and kMeanUnroll loads per
+// thread are in flight together; the accumulators, the lanes and the warps are then
+// combined in a fixed order.  The partial sums were just written and sit in L2, so the
+// kernel is bound by L2 latency: about n / (kMeanThreads * kMeanUnroll) round trips.
 __global__ void __launch_bounds__(kMeanThreads)
     error_mean_kernel(const double *__restrict__ partials, int64_t n, int64_t n_groups, double *__restrict__ out)
 {
-    __shared__ double red[kMeanThreads];
-    const int64_t per = (n + kMeanThreads - 1) / kMeanThreads;
-    const int64_t lo = static_cast<int64_t>(threadIdx.x) * per;
-    const int64_t hi = lo + per < n ? lo + per : n;
-    double s = 0.0;
-    for (int64_t i = lo; i < hi; ++i) s += partials[i];
-    red[threadIdx.x] = s;
-    __syncthreads();
-    for (int step = kMeanThreads / 2; step >= 1; step >>= 1) {
-        if (static_cast<int>(threadIdx.x) < step) red[threadIdx.x] += red[threadIdx.x + step];
-        __syncthreads();
+    __shared__ double red[kMeanThreads / 32];
+    double acc[kMeanUnroll];
+#pragma unroll
+    for (int u = 0; u < kMeanUnroll; ++u) acc[u] = 0.0;
+    constexpr int64_t kStep = static_cast<int64_t>(kMeanThreads) * kMeanUnroll;
+    for (int64_t base = threadIdx.x; base < n; base += kStep) {
+        double v[kMeanUnroll];
+#pragma unroll
+        for (int u = 0; u < kMeanUnroll; ++u) {
+            const int64_t i = base + static_cast<int64_t>(u) * kMeanThreads;
+            v[u] = i < n ? partials[i] : 0.0;
+        }
+#pragma unroll
+        for (int u = 0; u < kMeanUnroll; ++u) acc[u] += v[u];
     }
-    if (threadIdx.x == 0) *out = red[0] / static_cast<double>(n_groups);
+    double s = acc[0];
+#pragma unroll
+    for (int u = 1; u < kMeanUnroll; ++u) s += acc[u];
+    s = warp_tree_sum(s);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        s = warp_tree_sum(red[threadIdx.x]);
+        if (threadIdx.x == 0) *out = s / static_cast<double>(n_groups);
+    }
 }
 
 }  // namespace
