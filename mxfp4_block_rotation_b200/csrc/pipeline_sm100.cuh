@@ -194,7 +194,8 @@ __device__ __forceinline__ uint32_t quantize_group_nv(const uint32_t (&r)[32], u
         float m[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-            m[i] = ptx::fmax_nan(fabsf(__uint_as_float(r[16 * h + 2 * i])), fabsf(__uint_as_float(r[16 * h + 2 * i + 1])));
+            m[i] = ptx::fmax_nan(fabsf(__uint_as_float(r[16 * h + 2 * i])),
+                                 fabsf(__uint_as_float(r[16 * h + 2 * i + 1])));
 #pragma unroll
         for (int step = 4; step >= 1; step >>= 1)
 #pragma unroll
@@ -216,17 +217,23 @@ __device__ __forceinline__ uint32_t quantize_group_nv(const uint32_t (&r)[32], u
         out |= b << (8 * h);
         // E4M3 -> fp32 (exact): exponent e (bias 7), 3 mantissa bits; e = 0 is subnormal m * 2^-9
         const uint32_t e = (b >> 3) & 15u, mm = b & 7u;
-        const float sbv = e ? __uint_as_float(((e + 120u) << 23) | (mm << 20)) : __fmul_rn(static_cast<float>(mm), 0x1p-9f);
+        const float sbv =
+            e ? __uint_as_float(((e + 120u) << 23) | (mm << 20)) : __fmul_rn(static_cast<float>(mm), 0x1p-9f);
         const float s = __fmul_rn(sbv, s_t);
         const bool zero = b == 0x7Fu || s == 0.0f;   // NaN scale (bad block, or v = 0 * inf)
         const float rr = zero ? 0.0f : __frcp_rn(s);
-        float u[16];
+        // u = y * (1/s), two elements per packed multiply; a zero block's codes are all 0
+        float2 u[8];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) u[i] = zero ? 0.0f : __fmul_rn(__uint_as_float(r[16 * h + i]), rr);
+        for (int i = 0; i < 8; ++i)
+            u[i] = __fmul2_rn(make_float2(__uint_as_float(r[16 * h + 2 * i]), __uint_as_float(r[16 * h + 2 * i + 1])),
+                              make_float2(rr, rr));
 #pragma unroll
-        for (int q = 0; q < 2; ++q)
-            w[2 * h + q] = ptx::cvt_e2m1x8(u[8 * q], u[8 * q + 1], u[8 * q + 2], u[8 * q + 3], u[8 * q + 4],
-                                           u[8 * q + 5], u[8 * q + 6], u[8 * q + 7]);
+        for (int q = 0; q < 2; ++q) {
+            const uint32_t c = ptx::cvt_e2m1x8(u[4 * q].x, u[4 * q].y, u[4 * q + 1].x, u[4 * q + 1].y, u[4 * q + 2].x,
+                                               u[4 * q + 2].y, u[4 * q + 3].x, u[4 * q + 3].y);
+            w[2 * h + q] = zero ? 0u : c;
+        }
     }
     return out;
 }

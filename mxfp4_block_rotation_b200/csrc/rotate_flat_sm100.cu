@@ -214,16 +214,16 @@ cudaError_t launch_rotate_flat(const CUtensorMap &tmap_groups, const RotArgs &ar
     unsigned int *status = status_word();
     if (!status) return cudaErrorInvalidSymbol;
     if (mode == RotOut::Quant)
-        return launch_pdl(rotate_flat_kernel<RotOut::Quant>, grid, FlatRoles<RotOut::Quant>::kThreadsF, kFlatSmemBytes, stream, tmap_groups,
-                          args, status);
+        return launch_pdl(rotate_flat_kernel<RotOut::Quant>, grid, FlatRoles<RotOut::Quant>::kThreadsF, kFlatSmemBytes,
+                          stream, tmap_groups, args, status);
     if (mode == RotOut::Err)
-        return launch_pdl(rotate_flat_kernel<RotOut::Err>, grid, FlatRoles<RotOut::Err>::kThreadsF, kFlatSmemBytes, stream, tmap_groups, args,
-                          status);
+        return launch_pdl(rotate_flat_kernel<RotOut::Err>, grid, FlatRoles<RotOut::Err>::kThreadsF, kFlatSmemBytes,
+                          stream, tmap_groups, args, status);
     if (mode == RotOut::QuantNv)
-        return launch_pdl(rotate_flat_kernel<RotOut::QuantNv>, grid, FlatRoles<RotOut::QuantNv>::kThreadsF, kFlatSmemBytes, stream, tmap_groups,
-                          args, status);
-    return launch_pdl(rotate_flat_kernel<RotOut::F32>, grid, FlatRoles<RotOut::F32>::kThreadsF, kFlatSmemBytes, stream, tmap_groups, args,
-                      status);
+        return launch_pdl(rotate_flat_kernel<RotOut::QuantNv>, grid, FlatRoles<RotOut::QuantNv>::kThreadsF,
+                          kFlatSmemBytes, stream, tmap_groups, args, status);
+    return launch_pdl(rotate_flat_kernel<RotOut::F32>, grid, FlatRoles<RotOut::F32>::kThreadsF, kFlatSmemBytes, stream,
+                      tmap_groups, args, status);
 }
 
 int64_t rotate_flat_partials(int64_t rows, int64_t cols)
