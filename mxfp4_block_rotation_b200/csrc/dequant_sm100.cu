@@ -388,23 +388,22 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                 const int rj = kLam == 2 ? (row_lane + j * 128) % Gi : 0;   // this lane's Lambda row
                 const float *ltab = reinterpret_cast<const float *>(lambuf) + rj * 32;
                 ptx::tmem_wait_ld();
-                // times Lambda_k (channels of this group), then round to bf16 pairs
+                // times Lambda_k (channels of this group, two per packed multiply), then round to
+                // bf16 pairs; without Lambda the fp32 values are rounded as they are
                 uint32_t o[16];
 #pragma unroll
                 for (int k4 = 0; k4 < 8; ++k4) {
-                    float4 l4 = make_float4(1.0f, 1.0f, 1.0f, 1.0f);
-                    if constexpr (kLam == 1)
-                        l4 = *reinterpret_cast<const float4 *>(lrows + lane * 32 + ((k4 ^ (lane & 7)) << 2));
-                    else if constexpr (kLam == 2)
-                        l4 = *reinterpret_cast<const float4 *>(ltab + ((k4 ^ (rj & 7)) << 2));
-                    const __nv_bfloat162 p0 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(cur[4 * k4]), l4.x),
-                                                                    __fmul_rn(__uint_as_float(cur[4 * k4 + 1]), l4.y));
-                    const __nv_bfloat162 p1 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(cur[4 * k4 + 2]), l4.z),
-                                                                    __fmul_rn(__uint_as_float(cur[4 * k4 + 3]), l4.w));
-                    o[2 * k4] = static_cast<uint32_t>(__bfloat16_as_ushort(__low2bfloat16(p0))) |
-                                (static_cast<uint32_t>(__bfloat16_as_ushort(__high2bfloat16(p0))) << 16);
-                    o[2 * k4 + 1] = static_cast<uint32_t>(__bfloat16_as_ushort(__low2bfloat16(p1))) |
-                                    (static_cast<uint32_t>(__bfloat16_as_ushort(__high2bfloat16(p1))) << 16);
+                    float2 v0 = make_float2(__uint_as_float(cur[4 * k4]), __uint_as_float(cur[4 * k4 + 1]));
+                    float2 v1 = make_float2(__uint_as_float(cur[4 * k4 + 2]), __uint_as_float(cur[4 * k4 + 3]));
+                    if constexpr (kLambda) {
+                        const float4 l4 =
+                            kLam == 1 ? *reinterpret_cast<const float4 *>(lrows + lane * 32 + ((k4 ^ (lane & 7)) << 2))
+                                      : *reinterpret_cast<const float4 *>(ltab + ((k4 ^ (rj & 7)) << 2));
+                        v0 = __fmul2_rn(v0, make_float2(l4.x, l4.y));
+                        v1 = __fmul2_rn(v1, make_float2(l4.z, l4.w));
+                    }
+                    o[2 * k4] = bf162_bits(__floats2bfloat162_rn(v0.x, v0.y));
+                    o[2 * k4 + 1] = bf162_bits(__floats2bfloat162_rn(v1.x, v1.y));
                 }
                 const uint32_t buf = obuf0 + (nstore % kDqOutBufs) * kDqOutBuf;
                 // the buffer's previous store (kDqOutBufs stores ago) must have been read
