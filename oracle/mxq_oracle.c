@@ -56,7 +56,14 @@
  *   12  the search updates R <- G R instead of R <- R G
  *   13  the inverse rotation of the dequantiser uses R instead of R^T
  *   14  NVFP4: r_t = 1 / s_t (the 6 dropped)
- *   15  an all-zero group gets scale byte 127 instead of 0 */
+ *   15  an all-zero group gets scale byte 127 instead of 0
+ *   16  the MXFP4 GEMM ignores B's E8M0 scales
+ *   17  the NVFP4 GEMM drops B's tensor scale
+ *   18  E4M3 ties go to the odd code
+ *   19  the group error without its square root (a ratio of squared norms)
+ *   20  the B x B block rotation transposed
+ *   21  scale atoms with the roles of r % 32 and r / 32 swapped
+ *   22  the dequantiser divides by Lambda instead of multiplying */
 #ifndef MXQ_MUTANT
 #define MXQ_MUTANT 0
 #endif
@@ -375,7 +382,8 @@ int mxq_oracle_mxfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, const
     for (int64_t n = 0; n < N; ++n)
         for (int64_t k = 0; k < K; ++k) {
             int code = (b_codes[n * (K / 2) + k / 2] >> (4 * (k & 1))) & 0xF;
-            bd[n * K + k] = mxq_oracle_e2m1_value(code) * mxq_oracle_e8m0_value(b_scales[n * G + k / GROUP]);
+            bd[n * K + k] = mxq_oracle_e2m1_value(code) *
+                            (PLANTED(16) ? 1.0 : mxq_oracle_e8m0_value(b_scales[n * G + k / GROUP]));
         }
 #pragma omp parallel num_threads(nthreads > 0 ? nthreads : 1)
     {
@@ -432,7 +440,7 @@ int mxq_oracle_e4m3_code(double v)
     double bd = fabs(v);
     for (int c = 1; c <= 0x7E; ++c) {
         double d = fabs(v - mxq_oracle_e4m3_value(c));
-        if (d < bd || (d == bd && (c & 1) == 0)) {
+        if (d < bd || (d == bd && (c & 1) == (PLANTED(18) ? 1 : 0))) {
             best = c;
             bd = d;
         }
@@ -572,7 +580,7 @@ int mxq_oracle_nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, float
         for (int64_t k = 0; k < K; ++k) {
             int code = (b_codes[n * (K / 2) + k / 2] >> (4 * (k & 1))) & 0xF;
             bd[n * K + k] = mxq_oracle_e2m1_value(code) * mxq_oracle_e4m3_value(b_scales[n * NB + k / 16]) *
-                            (double)b_tscale;
+                            (PLANTED(17) ? 1.0 : (double)b_tscale);
         }
 #pragma omp parallel num_threads(nthreads > 0 ? nthreads : 1)
     {
@@ -612,7 +620,8 @@ int mxq_oracle_scales_to_mma(const uint8_t *scales, int64_t rows, int64_t G, uin
                 for (int j = 0; j < 4; ++j) {
                     int64_t row = rb * 128 + r, kb = cb * 4 + j;
                     uint8_t v = (row < rows && kb < G) ? scales[row * G + kb] : 0;
-                    out[(rb * CB + cb) * 512 + 16 * (r % 32) + 4 * (r / 32) + j] = v;
+                    int64_t at = PLANTED(21) ? 16 * (r / 32) + 4 * (r % 32) + j : 16 * (r % 32) + 4 * (r / 32) + j;
+                    out[(rb * CB + cb) * 512 + at] = v;
                 }
     return 0;
 }
@@ -656,7 +665,7 @@ int mxq_oracle_block_rotate_quantize(const uint16_t *X, int64_t rows, int64_t co
                     }
                     for (int n = 0; n < blk; ++n) {
                         double acc = 0.0;
-                        for (int k = 0; k < blk; ++k) acc += x[k] * R[k * blk + n];
+                        for (int k = 0; k < blk; ++k) acc += x[k] * (PLANTED(20) ? R[n * blk + k] : R[k * blk + n]);
                         yrow[b0 + n] = acc;
                     }
                 }
@@ -712,7 +721,7 @@ int mxq_oracle_dequantize(const uint8_t *codes, const uint8_t *scales, int64_t r
                 } else {
                     x[k] = v[k];
                 }
-                if (lam) x[k] = x[k] * (double)lam[g * GROUP + k];
+                if (lam) x[k] = PLANTED(22) ? x[k] / (double)lam[g * GROUP + k] : x[k] * (double)lam[g * GROUP + k];
                 out[e0 + k] = double_to_bf16(x[k]);
                 if (out_f64) out_f64[e0 + k] = x[k];
             }
@@ -761,7 +770,7 @@ int mxq_oracle_group_error(const uint16_t *X, int64_t rows, int64_t cols, const 
             }
             double e;
             if (byte == 0xFF) e = NAN;
-            else e = den > 0.0 ? sqrt(num / den) : 0.0;
+            else e = den > 0.0 ? (PLANTED(19) ? num / den : sqrt(num / den)) : 0.0;
             e_all[r * G + g] = e;
         }
     }

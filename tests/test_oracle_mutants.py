@@ -19,7 +19,7 @@ from tests import test_oracle_nvfp4_pins as nvfp4_pins
 from tests import test_oracle_pins as pins
 from tests import test_oracle_search_pins as search_pins
 
-N_MUTANTS = 15
+N_MUTANTS = 22
 
 
 def _calls():
