@@ -8,7 +8,7 @@
 // groups in a fixed order and leaves one partial sum per (stage or tile, warp)
 // in a caller-provided workspace.  This kernel adds the partial sums, again in
 // a fixed order, so the mean is the same on every run and for any grid size.
-#include "mxq_internal.h"
+#include "pipeline_sm100.cuh"
 
 namespace mxq {
 namespace {
@@ -29,10 +29,14 @@ __device__ __forceinline__ double warp_tree_sum(double v)
 // thread are in flight together; the accumulators, the lanes and the warps are then
 // combined in a fixed order.  The partial sums were just written and sit in L2, so the
 // kernel is bound by L2 latency: about n / (kMeanThreads * kMeanUnroll) round trips.
+// It is launched as a programmatic dependent of the rotate kernel, so its launch
+// overlaps that kernel's tail; griddepcontrol.wait then holds it until every partial
+// sum is written and visible.
 __global__ void __launch_bounds__(kMeanThreads)
     error_mean_kernel(const double *__restrict__ partials, int64_t n, int64_t n_groups, double *__restrict__ out)
 {
     __shared__ double red[kMeanThreads / 32];
+    ptx::griddep_wait();
     double acc[kMeanUnroll];
 #pragma unroll
     for (int u = 0; u < kMeanUnroll; ++u) acc[u] = 0.0;
@@ -64,8 +68,7 @@ __global__ void __launch_bounds__(kMeanThreads)
 cudaError_t launch_error_mean(const double *partials, int64_t n_partials, int64_t n_groups, double *out,
                               cudaStream_t stream)
 {
-    error_mean_kernel<<<1, kMeanThreads, 0, stream>>>(partials, n_partials, n_groups, out);
-    return cudaGetLastError();
+    return pipe::launch_pdl(error_mean_kernel, 1, kMeanThreads, 0, stream, partials, n_partials, n_groups, out);
 }
 
 }  // namespace mxq
