@@ -156,3 +156,56 @@ def test_nvfp4_rejects_bad_arguments(L):
     assert nv(a, 4, 64, a * 5, None, a * 7, a * 2, None) == INVALID             # no scales
     assert nv(a, 4, 64, a * 5, None, a * 2 + 4, a * 2, a * 3) == INVALID        # tensor scale inside the codes
     assert L.mxq_last_cuda_error().startswith(b"invalid argument")
+
+
+def test_gemm_and_scale_layout_reject_bad_arguments(L):
+    """The consumer GEMMs and the scale-atom layouts: sizes, nulls, alignment and overlaps
+    are refused on the host (nothing here reaches a device query)."""
+    a = 0x100000
+    M, N, K = 256, 256, 512
+    nca = M * K // 2
+    # atom arrays: one 512-byte atom per 128 rows x 4 scale columns
+    assert L.mxq_scales_mma_bytes(256, 512) == 2 * 4 * 512
+    assert L.mxq_scales_mma_bytes(129, 160) == 2 * 2 * 512
+    assert L.mxq_nvfp4_scales_mma_bytes(256, 512) == 2 * 8 * 512
+    assert L.mxq_nvfp4_scales_mma_bytes(1, 32) == 512
+    for f in (L.mxq_scales_mma_bytes, L.mxq_nvfp4_scales_mma_bytes):
+        assert f(0, 64) == 0 and f(4, 0) == 0 and f(4, 48) == 0 and f(-1, 64) == 0
+
+    def mx(ac, asf, bc, bsf, m, n, k, y, bf16=0):
+        return L.mxq_mxfp4_gemm(P(ac), P(asf), P(bc), P(bsf), m, n, k, P(y), bf16, None)
+
+    def nv(ac, asf, ta, bc, bsf, tb, m, n, k, y, bf16=0):
+        return L.mxq_nvfp4_gemm(P(ac), P(asf), P(ta), P(bc), P(bsf), P(tb), m, n, k, P(y), bf16, None)
+
+    ok = (a, a * 2, a * 3, a * 4)
+    y = a * 64
+    assert mx(*ok, -1, N, K, y) == INVALID                       # negative size
+    assert mx(*ok, M, N, 48, y) == INVALID                       # K not a multiple of 32
+    assert mx(*ok, 1 << 31, N, K, y) == INVALID                  # past the 32-bit tile indices
+    assert mx(*ok, M, N, K, y, bf16=2) == INVALID                # output type flag
+    assert mx(*ok, 0, N, K, None) == 0 and mx(*ok, M, 0, K, None) == 0   # nothing to compute
+    assert mx(*ok, M, N, K, None) == INVALID                     # no output
+    assert mx(*ok, M, N, K, y + 8) == INVALID                    # output not 16-byte aligned
+    assert mx(None, a * 2, a * 3, a * 4, M, N, K, y) == INVALID  # no A codes
+    assert mx(a, a * 2, a * 3, None, M, N, K, y) == INVALID      # no B scales
+    assert mx(a + 8, a * 2, a * 3, a * 4, M, N, K, y) == INVALID # codes not 16-byte aligned
+    assert mx(a, a * 2 + 4, a * 3, a * 4, M, N, K, y) == INVALID # scale atoms not 16-byte aligned
+    assert mx(*ok, M, N, K, a + nca - 16) == INVALID             # output overlaps A's codes
+    assert L.mxq_last_cuda_error().startswith(b"invalid argument")
+
+    okn = (a, a * 2, a * 5, a * 3, a * 4, a * 6)
+    assert nv(*okn, M, N, 40, y) == INVALID                      # K not a multiple of 32
+    assert nv(a, a * 2, None, a * 3, a * 4, a * 6, M, N, K, y) == INVALID       # no A tensor scale
+    assert nv(a, a * 2, a * 5, a * 3, a * 4, a * 6 + 2, M, N, K, y) == INVALID  # tensor scale not 4-byte aligned
+    assert nv(*okn, M, N, K, a * 5) == INVALID                   # output overlaps a tensor scale
+    assert nv(*okn, 0, N, K, None) == 0
+
+    for lay in (L.mxq_scales_to_mma_layout, L.mxq_nvfp4_scales_to_mma_layout):
+        assert lay(P(a), -1, 64, P(a * 2), None) == INVALID     # negative rows
+        assert lay(P(a), 4, 48, P(a * 2), None) == INVALID      # K not a multiple of 32
+        assert lay(P(a), 0, 64, None, None) == 0                 # nothing to lay out
+        assert lay(None, 4, 64, P(a * 2), None) == INVALID      # no input
+        assert lay(P(a), 4, 64, P(a * 2 + 8), None) == INVALID  # output not 16-byte aligned
+        assert lay(P(a), 4, 64, P(a - 16), None) == INVALID     # output overlaps the scales
+        assert L.mxq_last_cuda_error().startswith(b"invalid argument")
