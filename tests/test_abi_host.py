@@ -209,3 +209,41 @@ def test_gemm_and_scale_layout_reject_bad_arguments(L):
         assert lay(P(a), 4, 64, P(a * 2 + 8), None) == INVALID  # output not 16-byte aligned
         assert lay(P(a), 4, 64, P(a - 16), None) == INVALID     # output overlaps the scales
         assert L.mxq_last_cuda_error().startswith(b"invalid argument")
+
+
+def test_quant_error_and_weight_side_reject_bad_arguments(L):
+    """The error metric and the weights' quantiser: the host-side checks, and the
+    workspace size the error metric asks for (one double per partial sum)."""
+    a = 0x100000
+    # one partial sum per 512 groups and lane quarter without Lambda; per 128 x 64 tile and
+    # lane quarter with it
+    assert L.mxq_quant_error_workspace_bytes(4, 64, 0) == 4 * 8
+    assert L.mxq_quant_error_workspace_bytes(300, 4096, 0) == 75 * 4 * 8
+    assert L.mxq_quant_error_workspace_bytes(300, 4096, 1) == 3 * 64 * 4 * 8
+    assert L.mxq_quant_error_workspace_bytes(0, 64, 0) == 0 and L.mxq_quant_error_workspace_bytes(4, 48, 1) == 0
+
+    def qe(x, rows, cols, r, lam, err, mean, ws, wsb):
+        return L.mxq_quant_error(P(x), rows, cols, P(r), P(lam), P(err), P(mean), P(ws), wsb, None)
+
+    ws, wsb = a * 9, 1 << 20
+    assert qe(a, 4, 48, a * 5, None, None, a * 3, ws, wsb) == INVALID           # cols not a multiple of 32
+    assert qe(a, 4, 64, a * 5, None, None, None, ws, wsb) == INVALID            # no mean
+    assert qe(a, 4, 64, a * 5, None, None, a * 3 + 4, ws, wsb) == INVALID       # mean not 8-byte aligned
+    assert qe(a, 0, 64, a * 5, None, None, a * 3, ws, wsb) == INVALID           # the mean of nothing
+    assert qe(None, 4, 64, a * 5, None, None, a * 3, ws, wsb) == INVALID        # no X
+    assert qe(a + 8, 4, 64, a * 5, None, None, a * 3, ws, wsb) == INVALID       # X not 16-byte aligned
+    assert qe(a, 4, 64, a * 5, None, a * 2 + 2, a * 3, ws, wsb) == INVALID      # errors not 4-byte aligned
+    assert qe(a, 4, 64, a * 5, None, None, a * 3, None, wsb) == INVALID         # no workspace
+    assert qe(a, 4, 64, a * 5, None, None, a * 3, ws, 31) == INVALID            # workspace too small
+    assert qe(a, 4, 64, a * 5, None, None, a * 3, ws + 4, wsb) == INVALID       # workspace not 8-byte aligned
+    assert qe(a, 4, 64, a * 5, None, None, a + 64, ws, wsb) == INVALID          # mean inside X
+    assert qe(a, 4, 64, a * 5, None, None, a * 3, a * 3, wsb) == INVALID        # workspace holds the mean
+    assert L.mxq_last_cuda_error().startswith(b"invalid argument")
+
+    def wq(w, rows, cols, r, lam, codes, scales):
+        return L.mxq_weight_rotate_quantize(P(w), rows, cols, P(r), P(lam), P(codes), P(scales), None)
+
+    assert wq(a, 4, 48, a * 5, None, a * 2, a * 3) == INVALID                   # cols not a multiple of 32
+    assert wq(a, 4, 64, a * 5, a * 7 + 2, a * 2, a * 3) == INVALID              # Lambda not 4-byte aligned
+    assert wq(a, 4, 64, a * 5, None, a + 16, a * 3) == INVALID                  # codes overlap W
+    assert wq(a, 0, 64, a * 5, None, a * 2, a * 3) == 0                         # nothing to do
