@@ -611,7 +611,8 @@ def main(argv=None):
                     help="oracle seconds: the cpu_baseline sample (rank 0, N=1) and each --impl reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg (profiling runs)")
-    ap.add_argument("--no-extras", action="store_true", help="skip timing the smoothing and dequantize rows")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip other_rows: the other rows of the path, the GEMMs, the search and the error comparison")
     ap.add_argument("--extras-steps", type=int, default=300,
                     help="timed launches per extra row (the search row times min(10, this) runs)")
     ap.add_argument("--gemm-only", metavar="M,N,K",
