@@ -278,7 +278,7 @@ mxq_status mxq_quant_error(const void *X_bf16, int64_t rows, int64_t cols, const
 
 /*
  * mxq_quant_error without a workspace, for callers that cannot allocate device
- * memory (no counterpart in the paper; it only changes where scratch lives).
+ * memory (no counterpart in the write-up; it only changes where scratch lives).
  * Such callers include a plug-in handed only input and output pointers, a
  * process whose framework already holds the GPU's free memory (cudaMalloc
  * would fail), and a latency-critical path that cannot take cudaMalloc's
