@@ -35,8 +35,11 @@
  *
  * Common rules for every entry point below.
  *   Memory.  All pointers are device memory owned by the caller (for example
- *     from PyTorch).  The library allocates nothing, keeps no per-call state
- *     and may be called from several host threads.
+ *     from PyTorch).  The library allocates nothing and may be called from
+ *     several host threads.  Between calls it keeps only host-side caches that
+ *     cannot change a result: per host thread, the TMA descriptors of the last
+ *     few calls (keyed by everything a descriptor is encoded from), and per
+ *     device, the SM count and the kernels whose shared-memory opt-in is set.
  *   Streams.  `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Work is queued on it asynchronously; the call returns right
  *     after the launch.
@@ -270,6 +273,10 @@ mxq_status mxq_dequantize(const uint8_t *codes, const uint8_t *scales, int64_t r
  *   workspace               in/out  device scratch for per-warp partial sums, 8-byte
  *                                aligned, at least mxq_quant_error_workspace_bytes()
  *                                bytes; caller-owned, overwritten, no state kept
+ *
+ * If a bounded wait runs out (the device status word then holds MXQ_ERR_TIMEOUT,
+ * which mxq_sync_check reports), some partial sums are never written, so the mean
+ * is written as NaN rather than summed from stale scratch.
  */
 size_t mxq_quant_error_workspace_bytes(int64_t rows, int64_t cols, int with_lambda);
 mxq_status mxq_quant_error(const void *X_bf16, int64_t rows, int64_t cols, const void *Rhat_bf16,
@@ -294,12 +301,18 @@ mxq_status mxq_quant_error(const void *X_bf16, int64_t rows, int64_t cols, const
  *                    268,435,456 with rows rounded up to a multiple of 128 and
  *                    cols to a multiple of 64.  Larger inputs return
  *                    MXQ_ERR_INVALID_ARG and mxq_last_cuda_error() says why
- *   first call       on each device, the first call looks up the array's device
- *                    address (cudaGetSymbolAddress) with that device current;
- *                    make that first call before any stream capture
+ *   set-up           every call looks up the array's device address
+ *                    (cudaGetSymbolAddress) with the current device, so the
+ *                    address stays right after a device reset; the first call on
+ *                    a device also loads the library's device code there, so make
+ *                    that first call before any stream capture
  *   sharing          all calls use the same array; each call writes every slot
  *                    it reads, so nothing carries over.  Calls whose GPU work
  *                    overlaps (different streams, no ordering) race on it.
+ *   timeout          if a kernel's bounded wait runs out (mxq_sync_check then
+ *                    returns MXQ_ERR_TIMEOUT), some slots of that call are never
+ *                    written; the mean kernel sees the status word and writes NaN
+ *                    (the same holds for mxq_quant_error's workspace)
  */
 mxq_status mxq_quant_error_noalloc(const void *X_bf16, int64_t rows, int64_t cols, const void *Rhat_bf16,
                                    const float *Lambda_or_null, float *out_group_err_or_null, double *out_mean,

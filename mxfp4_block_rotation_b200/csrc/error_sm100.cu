@@ -31,12 +31,18 @@ __device__ __forceinline__ double warp_tree_sum(double v)
 // kernel is bound by L2 latency: about n / (kMeanThreads * kMeanUnroll) round trips.
 // It is launched as a programmatic dependent of the rotate kernel, so its launch
 // overlaps that kernel's tail; griddepcontrol.wait then holds it until every partial
-// sum is written and visible.
+// sum is written and visible.  A rotate kernel whose bounded wait ran out leaves some
+// partial sums unwritten and the timeout bit in the status word; the mean is then NaN.
 __global__ void __launch_bounds__(kMeanThreads)
-    error_mean_kernel(const double *__restrict__ partials, int64_t n, int64_t n_groups, double *__restrict__ out)
+    error_mean_kernel(const double *__restrict__ partials, int64_t n, int64_t n_groups, double *__restrict__ out,
+                      const unsigned int *status)
 {
     __shared__ double red[kMeanThreads / 32];
     ptx::griddep_wait();
+    if (*reinterpret_cast<const volatile unsigned int *>(status) & kStatusTimeout) {
+        if (threadIdx.x == 0) *out = __longlong_as_double(0x7FF8000000000000ll);
+        return;
+    }
     double acc[kMeanUnroll];
 #pragma unroll
     for (int u = 0; u < kMeanUnroll; ++u) acc[u] = 0.0;
@@ -68,7 +74,10 @@ __global__ void __launch_bounds__(kMeanThreads)
 cudaError_t launch_error_mean(const double *partials, int64_t n_partials, int64_t n_groups, double *out,
                               cudaStream_t stream)
 {
-    return pipe::launch_pdl(error_mean_kernel, 1, kMeanThreads, 0, stream, partials, n_partials, n_groups, out);
+    unsigned int *status = status_word();
+    if (!status) return cudaErrorInvalidSymbol;
+    return pipe::launch_pdl(error_mean_kernel, 1, kMeanThreads, 0, stream, partials, n_partials, n_groups, out,
+                            static_cast<const unsigned int *>(status));
 }
 
 }  // namespace mxq

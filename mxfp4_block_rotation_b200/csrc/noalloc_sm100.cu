@@ -15,10 +15,11 @@
 //
 // Every GPU that loads the library holds the array until the process exits.
 // All calls share it.  Each call writes every slot it later reads, so nothing
-// needs clearing between calls.  Two calls whose work overlaps on the GPU race
-// on the array, so the caller must order them (one stream, or events).
+// needs clearing between calls; the one exception is a kernel whose bounded wait
+// runs out, whose missing slots make the mean kernel write NaN instead (it reads
+// the status word).  Two calls whose work overlaps on the GPU race on the array,
+// so the caller must order them (one stream, or events).
 #include <cstdio>
-#include <mutex>
 
 #include "../../include/mxq.h"
 #include "mxq_internal.h"
@@ -29,30 +30,22 @@ constexpr int64_t kNoAllocPartials = 131072;   // doubles in the array (1 MiB)
 
 static __device__ __align__(256) double g_noalloc_partials[kNoAllocPartials];
 
-std::mutex g_noalloc_mu;
-double *g_noalloc_ptr[64] = {};
-
 // The array's device address on the current device.  Host code may not use the
 // symbol itself as a pointer (on the host it names a stand-in object, not device
-// memory), so the address is looked up with cudaGetSymbolAddress.  That happens
-// once per device, on the first call with that device current.
+// memory), so the address is looked up with cudaGetSymbolAddress, with the device
+// current, on every call.  Nothing is kept between calls, so the address stays right
+// even after a device reset has reloaded the module and moved the array.
 mxq_status noalloc_scratch(double **out)
 {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MXQ_ERR_CUDA;
-    std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
-        void *p = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_partials);
-        if (e != cudaSuccess || p == nullptr) {
-            char msg[160];
-            std::snprintf(msg, sizeof msg, "cudaGetSymbolAddress of the no-alloc scratch: %s", cudaGetErrorString(e));
-            mxq::set_last_error(msg);
-            return MXQ_ERR_CUDA;
-        }
-        g_noalloc_ptr[dev] = static_cast<double *>(p);
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_partials);
+    if (e != cudaSuccess || p == nullptr) {
+        char msg[160];
+        std::snprintf(msg, sizeof msg, "cudaGetSymbolAddress of the no-alloc scratch: %s", cudaGetErrorString(e));
+        mxq::set_last_error(msg);
+        return MXQ_ERR_CUDA;
     }
-    *out = g_noalloc_ptr[dev];
+    *out = static_cast<double *>(p);
     return MXQ_OK;
 }
 

@@ -247,3 +247,21 @@ def test_quant_error_and_weight_side_reject_bad_arguments(L):
     assert wq(a, 4, 64, a * 5, a * 7 + 2, a * 2, a * 3) == INVALID              # Lambda not 4-byte aligned
     assert wq(a, 4, 64, a * 5, None, a + 16, a * 3) == INVALID                  # codes overlap W
     assert wq(a, 0, 64, a * 5, None, a * 2, a * 3) == 0                         # nothing to do
+
+
+def test_noalloc_refuses_one_past_either_limit_before_any_cuda_call(L):
+    """mxq_quant_error_noalloc's fixed array holds 131072 partial sums.  Without Lambda one sum
+    covers 128 groups (four per 512-group stage), so 16,777,217 groups is one group too many.
+    With Lambda one sum covers a warp's 32 rows of a 128 x 64 tile, four per tile, so 32,769
+    tiles is one too many, even when the elements would fit: 129 rows round up to two row
+    tiles.  Both are refused from the sizes alone, so no device is needed."""
+    a = 0x100000
+    assert L.mxq_quant_error_workspace_bytes(1, 16777216 * 32, 0) == 131072 * 8
+    assert L.mxq_quant_error_workspace_bytes(1, 16777217 * 32, 0) > 131072 * 8
+    st = L.mxq_quant_error_noalloc(P(a), 1, 16777217 * 32, P(a), None, None, P(a), None)
+    assert st == INVALID and b"scratch" in L.mxq_last_cuda_error()
+    cols = 16385 * 64 - 32   # rounds up to 16385 column tiles; 2 row tiles -> 32,770 tiles
+    assert 129 * cols < 16777216 * 16   # fewer elements than the with-Lambda bound
+    assert L.mxq_quant_error_workspace_bytes(129, cols, 1) > 131072 * 8
+    st = L.mxq_quant_error_noalloc(P(a), 129, cols, P(a), P(a), None, P(a), None)
+    assert st == INVALID and b"scratch" in L.mxq_last_cuda_error()

@@ -57,7 +57,29 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     r = synth.rhat_tensor(np.eye(32)).to(DEV)
     mean = torch.zeros((), dtype=torch.float64, device=DEV)
     L = mxq.lib()
-    # 65536 x 8256 is 16,908,288 groups: one stage past the 16,777,216 the array covers (nothing is launched)
+    # 65536 x 8256 is 16,908,288 groups: 131,072 groups (256 stages of 512) past the 16,777,216
+    # the array covers; refused before anything is launched
     st = L.mxq_quant_error_noalloc(_ptr(x), 65536, 8256, _ptr(r), None, None, _ptr(mean),
                                    P(torch.cuda.current_stream().cuda_stream))
     assert st == 1 and b"scratch" in L.mxq_last_cuda_error()
+
+
+@pytest.mark.parametrize("rows,cols,with_lam", [(65536, 8192, False), (16384, 16384, True)])
+def test_noalloc_exactly_at_its_limit(rows, cols, with_lam):
+    """The largest inputs the array covers: 65536 x 8192 is exactly 16,777,216 groups of 32;
+    with Lambda, 16384 x 16384 is exactly 128 row tiles x 256 column tiles = 32,768 tiles of
+    four partial sums.  Both must run and agree with the workspace entry point."""
+    g = torch.Generator(device=DEV)
+    g.manual_seed(rows + cols)
+    x = torch.randn((rows, cols), generator=g, device=DEV, dtype=torch.float32).to(torch.bfloat16)
+    r = synth.rhat_tensor(synth.haar_orthogonal(11)).to(DEV)
+    lam = synth.random_lambda(cols, seed=12).to(DEV) if with_lam else None
+    L = mxq.lib()
+    assert L.mxq_quant_error_workspace_bytes(rows, cols, int(with_lam)) == 131072 * 8
+    ref_err, ref_mean = mxq.quant_error(x, r, lam)
+    err = torch.full((rows, cols // 32), float("nan"), dtype=torch.float32, device=DEV)
+    mean = torch.full((), float("nan"), dtype=torch.float64, device=DEV)
+    assert _noalloc(x, r, lam, err, mean) == 0, L.mxq_last_cuda_error()
+    mxq.sync_check()
+    assert torch.equal(err, ref_err)   # the same kernel on the same input: the same bits
+    assert abs(mean.item() - ref_mean.item()) <= 1e-12 * abs(ref_mean.item())
