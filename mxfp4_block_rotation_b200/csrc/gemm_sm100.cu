@@ -514,7 +514,8 @@ cudaError_t launch_pairs(const CUtensorMap &tmap_a, const CUtensorMap &tmap_b, c
     if (n_tiles <= 0 || args.K <= 0) return cudaSuccess;
     const int64_t pairs = n_tiles < num_sms / 2 ? n_tiles : num_sms / 2;
     constexpr int smem = PairCfg<kNv>::kSmem;
-    cudaError_t e = cudaFuncSetAttribute(mxfp4_gemm_kernel<kNv>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    const void *fn = reinterpret_cast<const void *>(mxfp4_gemm_kernel<kNv>);
+    cudaError_t e = smem_optin(fn, smem, false);
     if (e != cudaSuccess) return e;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -530,6 +531,10 @@ cudaError_t launch_pairs(const CUtensorMap &tmap_a, const CUtensorMap &tmap_b, c
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
+    e = cudaLaunchKernelEx(&cfg, mxfp4_gemm_kernel<kNv>, tmap_a, tmap_b, tmap_sfa, tmap_sfb, args, status);
+    if (e == cudaSuccess) return e;
+    (void)cudaGetLastError();   // refused: set the opt-in again (a device reset clears it) and retry once
+    if ((e = smem_optin(fn, smem, true)) != cudaSuccess) return e;
     return cudaLaunchKernelEx(&cfg, mxfp4_gemm_kernel<kNv>, tmap_a, tmap_b, tmap_sfa, tmap_sfb, args, status);
 }
 

@@ -4,7 +4,9 @@
 // the GPU: sizes, alignment, device residency and extent of every buffer,
 // overlap of outputs with inputs.  It then builds the TMA descriptor over X
 // and launches the kernels on the caller's stream.  It allocates no device
-// memory and keeps no per-call state.
+// memory.  The only state kept across calls is a per-thread cache of encoded TMA
+// descriptors (keyed by everything a descriptor is encoded from) and, per device,
+// the SM count and which kernels have their shared-memory opt-in set.
 #include <cudaTypedefs.h>
 
 #include <atomic>
@@ -150,8 +152,55 @@ mxq_status check_shape(int64_t rows, int64_t cols)
     return MXQ_OK;
 }
 
+// Encoded tensor maps of recent calls, per host thread.  A map is a pure function of
+// what it is encoded from (its kind, base address, extents and box), so a call that
+// repeats those reuses the encoded map instead of encoding it again: repeated calls on
+// the same buffers then skip cuTensorMapEncodeTiled.  Eight slots, replaced in turn.
+struct TmapKey {
+    int kind;
+    const void *p;
+    int64_t a, b;
+    uint32_t box;
+    bool operator==(const TmapKey &o) const
+    {
+        return kind == o.kind && p == o.p && a == o.a && b == o.b && box == o.box;
+    }
+};
+struct TmapSlot {
+    alignas(64) CUtensorMap map;
+    TmapKey key;
+    bool used;
+};
+constexpr int kTmapSlots = 8;
+thread_local TmapSlot g_tmaps[kTmapSlots];
+thread_local int g_tmap_next = 0;
+
+bool tmap_lookup(const TmapKey &key, CUtensorMap *map)
+{
+    for (int i = 0; i < kTmapSlots; ++i) {
+        if (g_tmaps[i].used && g_tmaps[i].key == key) {
+            *map = g_tmaps[i].map;
+            return true;
+        }
+    }
+    return false;
+}
+
+void tmap_store(const TmapKey &key, const CUtensorMap &map)
+{
+    TmapSlot &slot = g_tmaps[g_tmap_next];
+    g_tmap_next = (g_tmap_next + 1) % kTmapSlots;
+    slot.map = map;
+    slot.key = key;
+    slot.used = true;
+}
+
+enum TmapKind { kMapCodes = 1, kMapGroups, kMapBlocks, kMapOperand, kMapSf, kMapX };
+
 mxq_status make_tmap_codes(CUtensorMap *map, void *codes, int64_t rows, int64_t cols)
 {
+    const TmapKey key{kMapCodes, codes, rows, cols, 0};
+    if (tmap_lookup(key, map)) return MXQ_OK;
     const Driver &d = driver();
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols / 2), static_cast<cuuint64_t>(rows)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols / 2)};
@@ -165,12 +214,15 @@ mxq_status make_tmap_codes(CUtensorMap *map, void *codes, int64_t rows, int64_t 
         note_cu(r, "cuTensorMapEncodeTiled(codes)");
         return MXQ_ERR_CUDA;
     }
+    tmap_store(key, *map);
     return MXQ_OK;
 }
 
 // A bf16 [rows, cols] matrix viewed as [rows*cols/32, 32]: one 64-byte row per group.
 mxq_status make_tmap_groups(CUtensorMap *map, const void *X, int64_t rows, int64_t cols, uint32_t box_rows = 256)
 {
+    const TmapKey key{kMapGroups, X, rows, cols, box_rows};
+    if (tmap_lookup(key, map)) return MXQ_OK;
     const Driver &d = driver();
     cuuint64_t dims[2] = {32, static_cast<cuuint64_t>(rows) * static_cast<cuuint64_t>(cols / 32)};
     cuuint64_t strides[1] = {64};
@@ -183,6 +235,7 @@ mxq_status make_tmap_groups(CUtensorMap *map, const void *X, int64_t rows, int64
         note_cu(r, "cuTensorMapEncodeTiled(groups)");
         return MXQ_ERR_CUDA;
     }
+    tmap_store(key, *map);
     return MXQ_OK;
 }
 
@@ -191,6 +244,8 @@ mxq_status make_tmap_groups(CUtensorMap *map, const void *X, int64_t rows, int64
 // (32 KB of X per stage).
 mxq_status make_tmap_blocks(CUtensorMap *map, const void *X, int64_t rows, int64_t cols, int blk)
 {
+    const TmapKey key{kMapBlocks, X, rows, cols, static_cast<uint32_t>(blk)};
+    if (tmap_lookup(key, map)) return MXQ_OK;
     const Driver &d = driver();
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(blk),
                           static_cast<cuuint64_t>(rows) * static_cast<cuuint64_t>(cols / blk)};
@@ -204,6 +259,7 @@ mxq_status make_tmap_blocks(CUtensorMap *map, const void *X, int64_t rows, int64
         note_cu(r, "cuTensorMapEncodeTiled(blocks)");
         return MXQ_ERR_CUDA;
     }
+    tmap_store(key, *map);
     return MXQ_OK;
 }
 
@@ -211,6 +267,8 @@ mxq_status make_tmap_blocks(CUtensorMap *map, const void *X, int64_t rows, int64
 // rows, 128-byte swizzle, zero fill past the edges.
 mxq_status make_tmap_operand(CUtensorMap *map, const void *codes, int64_t rows, int64_t K, uint32_t box_rows)
 {
+    const TmapKey key{kMapOperand, codes, rows, K, box_rows};
+    if (tmap_lookup(key, map)) return MXQ_OK;
     const Driver &d = driver();
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
@@ -223,6 +281,7 @@ mxq_status make_tmap_operand(CUtensorMap *map, const void *codes, int64_t rows, 
         note_cu(r, "cuTensorMapEncodeTiled(gemm operand)");
         return MXQ_ERR_CUDA;
     }
+    tmap_store(key, *map);
     return MXQ_OK;
 }
 
@@ -230,6 +289,8 @@ mxq_status make_tmap_operand(CUtensorMap *map, const void *codes, int64_t rows, 
 // boxes of two atoms (256 words) x box_rows row blocks, no swizzle, zero fill past the edges.
 mxq_status make_tmap_sf(CUtensorMap *map, const void *atoms, int64_t row_blocks, int64_t cb_n, uint32_t box_rows)
 {
+    const TmapKey key{kMapSf, atoms, row_blocks, cb_n, box_rows};
+    if (tmap_lookup(key, map)) return MXQ_OK;
     const Driver &d = driver();
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(cb_n * 128), static_cast<cuuint64_t>(row_blocks)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(cb_n * 512)};
@@ -242,11 +303,14 @@ mxq_status make_tmap_sf(CUtensorMap *map, const void *atoms, int64_t row_blocks,
         note_cu(r, "cuTensorMapEncodeTiled(scale atoms)");
         return MXQ_ERR_CUDA;
     }
+    tmap_store(key, *map);
     return MXQ_OK;
 }
 
 mxq_status make_tmap_x(CUtensorMap *map, const void *X, int64_t rows, int64_t cols)
 {
+    const TmapKey key{kMapX, X, rows, cols, 0};
+    if (tmap_lookup(key, map)) return MXQ_OK;
     const Driver &d = driver();
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
@@ -259,6 +323,7 @@ mxq_status make_tmap_x(CUtensorMap *map, const void *X, int64_t rows, int64_t co
         note_cu(r, "cuTensorMapEncodeTiled");
         return MXQ_ERR_CUDA;
     }
+    tmap_store(key, *map);
     return MXQ_OK;
 }
 

@@ -118,8 +118,13 @@ cudaError_t launch_wait_selftest(uint64_t timeout_ns, int *result, cudaStream_t 
 // Set the text mxq_last_cuda_error() returns on this thread.
 void set_last_error(const char *msg);
 
-// Device address of the status word on the current device (nullptr on failure).
+// Device address of the status word on the current device (nullptr on failure).  It is
+// looked up on every call, so it stays right after a device reset moves the module.
 unsigned int *status_word();
+
+// Opt `func` in to `smem` bytes of dynamic shared memory on the current device.  The
+// runtime call is made once per (kernel, device, size); force makes it again.
+cudaError_t smem_optin(const void *func, int smem, bool force);
 
 // Read-and-clear of the device status word, stream ordered.
 cudaError_t read_and_clear_status(unsigned int *host_status, cudaStream_t stream);

@@ -325,10 +325,14 @@ __device__ __forceinline__ void kernel_teardown(uint32_t tmem_base, int mma_warp
 // Launch with programmatic stream serialisation: the grid may start while the
 // previous kernel in the stream drains (the kernels order their global accesses
 // with griddepcontrol.wait).
+// The dynamic shared-memory opt-in is set once per (kernel, device) (smem_optin); a
+// launch the runtime refuses is retried once after setting it again, which covers a
+// device reset having cleared it.
 template <typename Kern, typename... Args>
 cudaError_t launch_pdl(Kern kern, int grid, int block, int smem, cudaStream_t stream, Args... args)
 {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    const void *fn = reinterpret_cast<const void *>(kern);
+    cudaError_t e = smem_optin(fn, smem, false);
     if (e != cudaSuccess) return e;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -340,6 +344,10 @@ cudaError_t launch_pdl(Kern kern, int grid, int block, int smem, cudaStream_t st
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, args...);
+    if (e == cudaSuccess || smem <= 48 * 1024) return e;
+    (void)cudaGetLastError();
+    if ((e = smem_optin(fn, smem, true)) != cudaSuccess) return e;
     return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 

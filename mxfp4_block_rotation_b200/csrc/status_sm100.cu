@@ -33,22 +33,41 @@ __global__ void bounded_wait_selftest(uint64_t timeout_ns, int *result, unsigned
     ptx::mbar_arrive(ptx::smem_addr(&bar));   // complete the phase before exit
 }
 
-std::mutex g_status_mu;
-unsigned int *g_status_ptr[64] = {};
+// (kernel, device, bytes) triples whose shared-memory opt-in has been set.
+struct OptIn {
+    const void *func;
+    int dev;
+    int smem;
+};
+std::mutex g_optin_mu;
+OptIn g_optin[256];
+int g_n_optin = 0;
 
 }  // namespace
 
 unsigned int *status_word()
 {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+    return static_cast<unsigned int *>(p);
+}
+
+cudaError_t smem_optin(const void *func, int smem, bool force)
+{
+    if (smem <= 48 * 1024) return cudaSuccess;   // below the default limit no opt-in is needed
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    std::lock_guard<std::mutex> lock(g_status_mu);
-    if (!g_status_ptr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
-        g_status_ptr[dev] = static_cast<unsigned int *>(p);
-    }
-    return g_status_ptr[dev];
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(g_optin_mu);
+    int slot = -1;
+    for (int i = 0; i < g_n_optin; ++i)
+        if (g_optin[i].func == func && g_optin[i].dev == dev) slot = i;
+    if (slot >= 0 && g_optin[slot].smem >= smem && !force) return cudaSuccess;
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    if (slot < 0 && g_n_optin < 256) slot = g_n_optin++;
+    if (slot >= 0) g_optin[slot] = OptIn{func, dev, smem};
+    return cudaSuccess;
 }
 
 cudaError_t launch_wait_selftest(uint64_t timeout_ns, int *result, cudaStream_t stream)
