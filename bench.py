@@ -46,19 +46,33 @@ UNIT = "GB/s"
 WORKLOAD = ("down-proj input 8192x14336 bf16 (Student-t(3), 8 tokens x 4 channels of 1e3-1e4 outliers), "
             "random orthogonal 32x32 R, no smoothing -> MXFP4 codes + E8M0 scales")
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_SOURCES = ["mxfp4_block_rotation_b200/csrc/rotate_flat_sm100.cu",
-                  "mxfp4_block_rotation_b200/csrc/pipeline_sm100.cuh",
-                  "mxfp4_block_rotation_b200/csrc/sm100_ptx.cuh"]
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "rotate_flat_kernel_downproj_traffic.json")
+_CSRC = "mxfp4_block_rotation_b200/csrc/"
+_COMMON = [_CSRC + "pipeline_sm100.cuh", _CSRC + "sm100_ptx.cuh", _CSRC + "sm100_bulk.cuh",
+           _CSRC + "mxq_internal.h"]
+# The device code each timed kernel is built from: a DRAM-traffic record under profiles/ is
+# reported only while the hash of these files matches the one it was taken with.
+KERNEL_SOURCES = {
+    "rotate_flat": [_CSRC + "rotate_flat_sm100.cu"] + _COMMON,
+    "rotate_cols": [_CSRC + "rotate_cols_sm100.cu"] + _COMMON,
+    "dequant_rot": [_CSRC + "dequant_sm100.cu"] + _COMMON,
+}
+# profiles/traffic_<row>.json: ncu's dram__bytes_read.sum + dram__bytes_write.sum of one launch
+TRAFFIC_KERNEL = {
+    "qkv_o_proj_input_8192x4096": "rotate_flat",
+    "down_proj_input_8192x14336": "rotate_flat",
+    "large_prefill_65536x8192_hadamard": "rotate_flat",
+    "smoothing_32768x14336_quantize": "rotate_cols",
+    "smoothing_32768x14336_dequantize_round_trip": "dequant_rot",
+}
 
 
 def algorithmic_bytes(rows: int, cols: int) -> float:
     return rows * cols * BYTES_PER_ELEM
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(kernel: str = "rotate_flat") -> str:
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES:
+    for p in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, p), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
@@ -82,14 +96,15 @@ def _bf16_peak_tflops() -> float:
         return 1590.0
 
 
-def recorded_traffic():
-    """DRAM bytes per launch from the committed ncu summary, if the kernel source is unchanged."""
+def recorded_traffic(row: str = "down_proj_input_8192x14336"):
+    """DRAM bytes per launch of a row's kernel from its committed ncu record, or None when there
+    is no record or the kernel's source has changed since it was taken."""
     try:
-        with open(TRAFFIC_FILE) as f:
+        with open(os.path.join(ROOT, "profiles", f"traffic_{row}.json")) as f:
             rec = json.load(f)
     except (OSError, ValueError):
         return None
-    if rec.get("kernel_source_sha256") != kernel_source_hash():
+    if rec.get("kernel_source_sha256") != kernel_source_hash(TRAFFIC_KERNEL[row]):
         return None
     return rec.get("dram_bytes_per_launch")
 
@@ -263,30 +278,33 @@ def run_mine(args):
         c, s = outs[i & 1]
         mxq.smooth_rotate_quantize(xs[i & 1], rhat, None, codes=c, scales=s, stream=stream)
 
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize(dev)
-    mxq.sync_check()
-
     # Timed region: K back-to-back launches on one stream, bracketed by two events (no
     # events between launches, so programmatic dependent launch can overlap each
     # launch's set-up with the previous one's tail).  The kernel's average launch
-    # duration is therefore the region's time / K.
+    # duration is therefore the region's time / K.  The clock sampler starts before the
+    # warm-up, so the GPU does not sit idle between the warm-up and the timed region.
     k = args.steps
     t_begin = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clocks:
+        for i in range(args.warmup):
+            step(i)
+        torch.cuda.synchronize(dev)
+        mxq.sync_check()
         if dist is not None:
             dist.barrier()
         torch.cuda.synchronize(dev)
         t_begin.record(stream)
+        h0 = time.perf_counter()
         for i in range(k):
             step(i)
+        h1 = time.perf_counter()
         t_end.record(stream)
         torch.cuda.synchronize(dev)
         if dist is not None:
             dist.barrier()
     mxq.sync_check()
+    host_us_per_call = (h1 - h0) / k * 1e6
     total_ms = max_over_ranks([t_begin.elapsed_time(t_end)], dist, dev)[0]
     kern_avg_ms = total_ms / k
     ms_per_step = total_ms / k
@@ -296,6 +314,9 @@ def run_mine(args):
     e2e = None if args.no_e2e else run_e2e(mxq, w, rhat, dev, stream, args, dist)
     extras = None if (args.no_extras or world > 1) else run_extras(mxq, w, xs, rhat, outs, dev, stream,
                                                                     k=max(1, args.extras_steps))
+    del xs, outs
+    per_config = None if (args.no_configs or world > 1) else run_configs(mxq, dev, stream,
+                                                                         k=max(1, args.extras_steps))
 
     if rank == 0:
         peak, peak_kind = hbm_peak()
@@ -317,8 +338,11 @@ def run_mine(args):
                          "kernel": "rotate_flat_kernel<Quant> (no smoothing)", "kernel_ms": kern_avg_ms},
             "e2e": e2e,
             "gpu_launches": k,
+            "host_submit_us_per_call": host_us_per_call,
             "clocks": clocks.summary(),
         }
+        if per_config is not None:
+            line["per_config"] = per_config
         if extras is not None:
             line["other_rows"] = extras
         if world == 1 and not args.no_cpu_baseline:
@@ -522,6 +546,100 @@ def run_extras(mxq, w, xs, rhat, outs, dev, stream, k=300):
     return res
 
 
+L2_BYTES = 126 * 2 ** 20
+
+
+def _sets_for(set_bytes: float) -> int:
+    """Input/output sets to rotate so that a launch never finds its buffers in L2: the sets
+    together hold at least three times the L2 capacity (at least two sets)."""
+    return max(2, -(-int(3 * L2_BYTES) // int(set_bytes)))
+
+
+# The workloads of the write-up's layer inputs (§4.1 / Figure 1: QKV-in, O-in and Down-in), each
+# timed as its own row: (config, what the launch does, kernel)
+CONFIG_ROWS = {
+    "qkv_o_proj_input_8192x4096": (2, "quantize", "rotate_flat_kernel<Quant>"),
+    "down_proj_input_8192x14336": (3, "quantize", "rotate_flat_kernel<Quant>"),
+    "large_prefill_65536x8192_hadamard": (4, "quantize", "rotate_flat_kernel<Quant>"),
+    "smoothing_32768x14336_quantize": (5, "quantize", "rotate_cols_kernel<Quant>"),
+    "smoothing_32768x14336_dequantize_round_trip": (5, "dequantize", "dequant_rot_kernel<2>"),
+}
+
+
+def _config_row(mxq, name, w, dev, stream, k, codes_scales=None):
+    """One CONFIG_ROWS row, K back-to-back launches on rotating sets; returns (row, codes, scales)."""
+    cfg, what, kern = CONFIG_ROWS[name]
+    rows, cols = w.rows, w.cols
+    peak, _ = hbm_peak()
+    rhat = w.rhat.to(dev)
+    lam = None if w.lam is None else w.lam.to(dev)
+    lam_bytes = 0 if lam is None else 4 * cols
+    if what == "quantize":
+        n_bytes = algorithmic_bytes(rows, cols) + lam_bytes
+        n_sets = _sets_for(n_bytes)
+        x0 = w.x.to(dev)
+        xs = [x0] + [x0.clone() for _ in range(n_sets - 1)]
+        outs = [(torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev),
+                 torch.empty((rows, cols // 32), dtype=torch.uint8, device=dev)) for _ in range(n_sets)]
+
+        def fn(i):
+            c, s = outs[i % n_sets]
+            mxq.smooth_rotate_quantize(xs[i % n_sets], rhat, lam, codes=c, scales=s, stream=stream)
+        keep = outs[0]
+    else:
+        c0, s0 = codes_scales
+        n_bytes = rows * cols * (0.5 + 1.0 / 32.0 + 2.0) + lam_bytes
+        n_sets = _sets_for(n_bytes)
+        ins = [(c0, s0)] + [(c0.clone(), s0.clone()) for _ in range(n_sets - 1)]
+        outs = [torch.empty((rows, cols), dtype=torch.bfloat16, device=dev) for _ in range(n_sets)]
+
+        def fn(i):
+            c, s = ins[i % n_sets]
+            mxq.dequantize(c, s, rhat, lam, out=outs[i % n_sets], stream=stream)
+        keep = None
+    ms = _timed(fn, k, stream, dev)
+    mxq.sync_check()
+    gbs = n_bytes / (ms * 1e-3) / 1e9
+    row = {"config": cfg, "shape": [rows, cols], "what": what, "kernel": kern, "ms": ms, "GB/s": gbs,
+           "frac_of_hbm_peak": gbs / peak, "elements_per_s": rows * cols / (ms * 1e-3),
+           "bytes_per_launch": n_bytes, "traffic": recorded_traffic(name), "lambda": lam is not None,
+           "launches": k,
+           "l2": f"{n_sets} input/output sets rotated ({n_bytes / 1e6:.0f} MB each; L2 126 MB)"}
+    return row, keep
+
+
+def run_configs(mxq, dev, stream, k=300):
+    """Every workload's own row (CONFIG_ROWS), each against the HBM roofline."""
+    res = {}
+    for cfg in (2, 3, 4, 5):
+        w = synth.make_config(cfg)
+        keep = None
+        for name, (c, what, _) in CONFIG_ROWS.items():
+            if c != cfg:
+                continue
+            res[name], got = _config_row(mxq, name, w, dev, stream, k, keep)
+            keep = got if got is not None else keep
+        del w, keep
+        torch.cuda.empty_cache()
+    return res
+
+
+def run_row_only(args):
+    """Profiling aid: one CONFIG_ROWS row alone, --warmup + --steps launches, then its time."""
+    import mxfp4_block_rotation_b200 as mxq
+    dev = torch.device("cuda:0")
+    stream = torch.cuda.current_stream(dev)
+    cfg, what, _ = CONFIG_ROWS[args.row]
+    w = synth.make_config(cfg)
+    keep = None
+    if what == "dequantize":
+        keep = mxq.smooth_rotate_quantize(w.x.to(dev), w.rhat.to(dev), None if w.lam is None else w.lam.to(dev),
+                                          stream=stream)
+    row, _ = _config_row(mxq, args.row, w, dev, stream, max(1, args.steps), keep)
+    print(json.dumps({args.row: row}), flush=True)
+    return 0
+
+
 def run_e2e(mxq, w, rhat, dev, stream, args, dist):
     rows, cols = w.rows, w.cols
     x_host = w.x.pin_memory()
@@ -615,6 +733,11 @@ def main(argv=None):
                     help="skip other_rows: the other rows of the path, the GEMMs, the search and the error comparison")
     ap.add_argument("--extras-steps", type=int, default=300,
                     help="timed launches per extra row (the search row times min(10, this) runs)")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip per_config: the other workloads' rows (QKV/O-proj, large prefill, smoothing)")
+    ap.add_argument("--row", choices=sorted(CONFIG_ROWS),
+                    help="profiling aid: run only this per_config row, --steps launches after 5 warm-up "
+                         "launches, print its time and exit")
     ap.add_argument("--gemm-only", metavar="M,N,K",
                     help="profiling aid: run only the MXFP4 GEMM, 3 + --steps launches on random operands of this "
                          "shape (bf16 out), print its time and exit")
@@ -623,6 +746,8 @@ def main(argv=None):
         raise SystemExit("--warmup must be >= 3")
     if args.gemm_only:
         return run_gemm_only(args)
+    if args.row:
+        return run_row_only(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_mine(args)

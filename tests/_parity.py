@@ -34,11 +34,14 @@ def bf16_to_f64(bits):
     return b.view(np.float32).astype(np.float64)
 
 
-def check_quant(x_bits, rhat_bits, lam, gpu_codes, gpu_scales, threads=None, exact=False, ref=None):
+def check_quant(x_bits, rhat_bits, lam, gpu_codes, gpu_scales, threads=None, exact=False, ref=None,
+                max_frac=1e-5):
     """Compare GPU codes/scales for the rows of x_bits; returns a dict of counts (raises on failure).
 
     `ref` is the oracle's output (with y and flags) when the caller has it already, e.g. from
-    another oracle entry point; otherwise the main path's oracle is run here."""
+    another oracle entry point; otherwise the main path's oracle is run here.  `max_frac` bounds
+    the boundary differences as a fraction of these rows' elements; a caller checking a matrix in
+    row chunks passes None and applies the bound to the totals."""
     threads = threads or oracle.default_threads()
     if ref is None:
         ref = oracle.smooth_rotate_quantize(x_bits, rhat_bits, lam, want_y=True, flags=True, threads=threads)
@@ -86,7 +89,8 @@ def check_quant(x_bits, rhat_bits, lam, gpu_codes, gpu_scales, threads=None, exa
     n_excused = n_code_diff + 32 * n_alt_groups
     if exact:
         assert n_excused == 0, f"{n_code_diff} code and {n_alt_groups} scale differences where exact was required"
-    assert n_excused <= 1e-5 * n_elems, f"{n_excused} boundary differences > 1e-5 of {n_elems}"
+    if max_frac is not None:
+        assert n_excused <= max_frac * n_elems, f"{n_excused} boundary differences > {max_frac} of {n_elems}"
     return {"elements": n_elems, "code_boundary_diffs": n_code_diff, "scale_boundary_diffs": n_alt_groups,
             "y": ref["y"], "ref": ref}
 
@@ -150,3 +154,54 @@ def check_nvfp4(x_bits, rhat_bits, lam, s_t, gpu_codes, gpu_scales, exact=False,
     assert n_excused <= 1e-5 * rows * cols, f"{n_excused} boundary differences > 1e-5 of {rows * cols}"
     return {"elements": rows * cols, "code_boundary_diffs": int(diff.sum()), "scale_boundary_diffs": n_alt,
             "ref": ref}
+
+
+def bf16_rne_bits(t):
+    """float64 -> bf16 bit patterns, rounded once to nearest even (no detour through fp32, so no
+    double rounding).  Finite values only; bf16 subnormals are rounded on their own grid."""
+    t = np.asarray(t, np.float64)
+    assert np.isfinite(t).all()
+    m, e = np.frexp(t)                                   # t = m 2^e, 0.5 <= |m| < 1
+    e = np.maximum(e, -125)                              # below 2^-126 the grid is fixed: 2^-133
+    q = np.rint(np.ldexp(m, 8 + (np.frexp(t)[1] - e)))   # 8 significant bits (fewer when subnormal)
+    v = np.ldexp(q, e - 8)                               # exact in double and in fp32
+    bits = (v.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    return bits
+
+
+def _bf16_order(bits):
+    """bf16 bit patterns -> integers in the order of their values (-0 and +0 adjacent)."""
+    b = np.asarray(bits, np.uint16).astype(np.int32)
+    return np.where(b & 0x8000, -(b & 0x7FFF) - 1, b)
+
+
+def check_dequant_inverse(codes, scales, cols, rhat_bits, lam, gpu_bits, ref=None):
+    """Inverse dequantiser (v R^T, then times Lambda) against the exact value rounded once to
+    bf16 (the oracle's definition).  The kernel computes in fp32: 32 exact products summed on
+    the tensor cores, then one multiply by Lambda, then the rounding to bf16.  Its fp32 value is
+    within A = 2^-18 sum_n |v_n||R[k][n]| Lambda_k + 2^-23 |x| of the exact x (sum of 32 terms:
+    at most 31 roundings of 2^-24 of the running sum, doubled for margin; the Lambda multiply and
+    the accumulator's last rounding).  So an output must be the correctly rounded bf16, except
+    where [x - A, x + A] holds a bf16 rounding midpoint: there either rounding is right.  Returns
+    the number of outputs that differ from the correctly rounded value (all of them at such
+    midpoints); raises on any other difference."""
+    if ref is None:
+        ref = oracle.dequantize(codes, scales, cols, rhat_bits, lam, want_f64=True)
+    ref_bits, ref64 = ref
+    rows = ref_bits.shape[0]
+    v = bf16_to_f64(oracle.dequantize(codes, scales, cols))
+    rr = bf16_to_f64(rhat_bits)
+    s_abs = (np.abs(v).reshape(rows, cols // 32, 32) @ np.abs(rr).T).reshape(rows, cols)
+    if lam is not None:
+        s_abs = s_abs * np.asarray(lam, np.float64)[None, :]
+    acc = 2.0 ** -18 * s_abs + 2.0 ** -23 * np.abs(ref64)
+    lo = _bf16_order(bf16_rne_bits(ref64 - acc))
+    hi = _bf16_order(bf16_rne_bits(ref64 + acc))
+    got = _bf16_order(gpu_bits)
+    bad = (got < lo) | (got > hi)
+    if bad.any():
+        r, c = np.argwhere(bad)[0]
+        raise AssertionError(f"inverse dequantise at ({r},{c}): gpu {bf16_to_f64(gpu_bits)[r, c]!r}, exact "
+                             f"{ref64[r, c]!r} (correctly rounded {bf16_to_f64(ref_bits)[r, c]!r}), fp32 bound "
+                             f"{acc[r, c]!r}")
+    return int((np.asarray(gpu_bits, np.uint16) != ref_bits).sum())

@@ -23,13 +23,25 @@ def test_reference_arm_json_line():
     assert line["config"]["rows"] == 8192 and line["config"]["cols"] == 14336
 
 
-def test_algorithmic_bytes_and_traffic_record():
+def test_algorithmic_bytes_and_traffic_records():
     assert bench.algorithmic_bytes(8192, 14336) == 297271296.0
-    rec = json.load(open(bench.TRAFFIC_FILE))
-    assert rec["algorithmic_bytes_per_launch"] == 297271296.0
-    # the recorded traffic is reported only while the kernel source is unchanged
-    t = bench.recorded_traffic()
-    assert t is None or abs(t - rec["dram_bytes_per_launch"]) < 1
+    for row, kern in bench.TRAFFIC_KERNEL.items():
+        assert row in bench.CONFIG_ROWS and kern in bench.KERNEL_SOURCES
+        path = os.path.join(ROOT, "profiles", f"traffic_{row}.json")
+        if not os.path.exists(path):
+            assert bench.recorded_traffic(row) is None
+            continue
+        rec = json.load(open(path))
+        assert rec["dram_bytes_per_launch"] == rec["dram_bytes_read"] + rec["dram_bytes_write"]
+        # the recorded traffic is reported only while the kernel source is unchanged
+        t = bench.recorded_traffic(row)
+        assert t is None or abs(t - rec["dram_bytes_per_launch"]) < 1
+
+
+def test_rotating_sets_exceed_l2():
+    for set_bytes in (85e6, 297e6, 1.19e9, 1.36e9):
+        n = bench._sets_for(set_bytes)
+        assert n >= 2 and n * set_bytes >= 3 * bench.L2_BYTES
 
 
 def test_peak_source():

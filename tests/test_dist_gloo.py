@@ -53,7 +53,7 @@ def _worker(rank, world, port, out):
 
 def test_two_rank_max_and_sharding():
     world, port = 2, _free_port()
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()   # no fork of this (threaded) process
     mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
     assert out[0][0] == out[1][0] == [15.0, 2.0]
     import numpy as np
