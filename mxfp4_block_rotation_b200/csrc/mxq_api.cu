@@ -204,11 +204,12 @@ mxq_status make_tmap_codes(CUtensorMap *map, void *codes, int64_t rows, int64_t 
     const Driver &d = driver();
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols / 2), static_cast<cuuint64_t>(rows)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols / 2)};
-    // one epilogue warp's store: 32 rows x 32 bytes (the codes of a 64-column tile), plain layout
+    // one epilogue warp's store: 32 rows x 32 bytes (the codes of a 64-column tile), 32-byte swizzle
+    // (16-byte chunk c of row r staged at chunk c ^ ((r >> 2) & 1), so the staging stores are conflict free)
     cuuint32_t box[2] = {32, 32};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = d.encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, codes, dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
                           CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
         note_cu(r, "cuTensorMapEncodeTiled(codes)");

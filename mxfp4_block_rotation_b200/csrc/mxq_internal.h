@@ -41,7 +41,7 @@ cudaError_t launch_rotate_flat(const CUtensorMap &tmap_groups, const RotArgs &ar
 // Fused smooth -> rotate -> MXFP4 (args.lambda non-null).  `tmap_x` views X as
 // [rows, cols] bf16 (box {64, 128}, 128-byte swizzle); `tmap_codes` the packed
 // codes as [rows, cols/2] uint8 (box {32, 32}: one epilogue warp's rows of a 64-column
-// tile, no swizzle; Quant mode only).
+// tile, 32-byte swizzle; Quant mode only).
 cudaError_t launch_rotate_cols(const CUtensorMap &tmap_x, const CUtensorMap &tmap_codes, const RotArgs &args,
                                RotOut mode, int num_sms, cudaStream_t stream);
 

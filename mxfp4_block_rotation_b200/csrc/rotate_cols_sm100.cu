@@ -10,15 +10,24 @@
 // (4 row blocks of one column tile) they make the tile's two B_g in fp32: a
 // reciprocal per channel plus its FMA residual, so R*(1/Lambda) is good to about
 // an ulp.  Each B_g is split three ways into bf16, high + middle + low (~24 bits
-// of B).  The three parts are stacked along N: one group's B is 96 rows (n of the
-// high part, then the middle, then the low) x 32 k, so a K = 16 step is ONE MMA
-// with N = 96 instead of three with N = 32; the small MMAs' fixed cost in the
-// tensor pipe, not HBM, bounded the three-MMA form.  The epilogue adds the three
-// 32-column partial results, (low + middle) + high, in fp32.  X stays the exact
-// bf16 A operand, so the smoothing adds only ~2^-25 relative error on top of
-// fp32 accumulation.  Each epilogue warp stages its 32 rows of codes (32 x 32 B,
-// two buffers so that one store can be in flight) and writes them with its own
-// TMA bulk tensor store; no warp waits for another.
+// of B).  A builder thread owns one column n of R^ and one k-chunk of 8 for the
+// whole kernel, so its R^ values stay in registers; a warp shares the k-chunk, so
+// its reads of 1/Lambda are broadcasts and its stores hit distinct banks.  The three
+// parts are stacked along N: one group's B is 96 rows (n of the high part, then
+// the middle, then the low) x 32 k, so a K = 16 step is ONE MMA with N = 96.  An
+// MMA's cost follows the bytes it reads from shared memory (A once, B's 96 rows),
+// so one N = 96 MMA per step is cheaper than three N = 32 MMAs, each reading A.
+// The epilogue adds the three 32-column partial results, (low + middle) + high,
+// in fp32.  X stays the exact bf16 A operand, so the smoothing adds only ~2^-25
+// relative error on top of fp32 accumulation.  Each epilogue warp stages its 32
+// rows of codes (32 x 32 B, 32-byte swizzle so that the staging stores are
+// conflict free; two buffers so that one store can be in flight) and writes them
+// with its own TMA bulk tensor store; no warp waits for another.
+//
+// The MMA thread is the pipeline's critical path, so it does only waits, the MMAs
+// and one commit per tile.  The tile order advances by additions (no division per
+// tile), and the epilogue's leader, which sees each tile's MMAs complete, hands its
+// shared-memory stage back to the TMA producer.
 #include "pipeline_sm100.cuh"
 
 namespace mxq {
@@ -39,23 +48,22 @@ constexpr int kColStages = 6;
 constexpr int kWarpCodeBytes = 32 * kColTileG * 16;           // one epilogue warp's 32 rows of codes (1 KB)
 constexpr int kColStageOffset = kEpiWarps * 2 * kWarpCodeBytes;   // code staging first: 2 buffers per epilogue warp
 constexpr int kColBOffset = kColStageOffset + kColStages * kColStageBytes;
-constexpr int kColRtOffset = kColBOffset + 2 * kBSlotBytes;
-constexpr int kColInvOffset = kColRtOffset + 32 * 32 * 4;     // per slot: 1/Lambda of the tile's channels
+constexpr int kColInvOffset = kColBOffset + 2 * kBSlotBytes;   // per slot: 1/Lambda of the tile's channels
 constexpr int kColBarOffset = kColInvOffset + 2 * kColTileCols * 8;
 constexpr int kColSmemBytes = kColBarOffset + 512 + 1024;
 constexpr int kColBuildWarps = 4;                             // warps 10-13
 constexpr int kColThreads = (kEpiWarps + 2 + kColBuildWarps) * 32;   // 448
-static_assert(kColStages <= kMaxStages && kColAcc * kColAccCols <= 512 && kColStageOffset % 1024 == 0 &&
-                  kColBOffset % 1024 == 0 && kBGroupBytes % 512 == 0,
-              "smoothing kernel layout");
+static_assert(kColStages <= kMaxStages && kColStages % 2 == 0 && kColAcc == 2 && kColAcc * kColAccCols <= 512 &&
+                  kColStageOffset % 1024 == 0 && kColBOffset % 1024 == 0 && kBGroupBytes % 512 == 0 &&
+                  kColInvOffset % 16 == 0,
+              "smoothing kernel layout (an epilogue group takes every other tile, so every other stage)");
 
 // Tile order of the smoothing kernel.  A unit is kUnitRows consecutive row
 // blocks of one column tile, so one B_g build serves kUnitRows tiles.  Units are
 // numbered band-major (u = band * n_ct + ct) and dealt round robin to the CTAs.
 // At any moment the CTAs' units therefore cover whole rows of a couple of row
 // bands, which DRAM reads well.  Only the last band can be shorter than
-// kUnitRows, and a CTA meets it only in its last units, so a CTA's it-th tile
-// has a closed form.
+// kUnitRows, and a CTA meets it only in its last units (from unit k_full on).
 constexpr int kUnitRows = 4;
 
 struct UnitSched {
@@ -71,22 +79,41 @@ struct UnitSched {
         k_full = k < n_units_cta ? k : n_units_cta;
         n_tiles = k_full * kUnitRows + (n_units_cta - k_full) * r_last;
     }
-    // The it-th tile of this CTA: its unit's ordinal ui, the position in the unit and the unit's length.
-    __device__ void at(int it, int &ui, int &sub, int &len) const
+};
+
+// A CTA's tiles in order, advanced by additions only: the unit's column tile ct and
+// first row tile rt0, the position sub inside the unit and the unit's length.  Unit
+// ui + 1 is unit ui moved by grid in the band-major numbering, i.e. by grid % n_ct
+// column tiles and grid / n_ct bands, with a carry into the band.
+struct TileCursor {
+    int sub, len, ui, ct, rt0;
+    int n_ct, step_ct, step_rt, k_full, r_last;
+    __device__ explicit TileCursor(const UnitSched &s)
+        : sub(0), ui(0), n_ct(s.n_ct), step_ct(s.grid % s.n_ct), step_rt((s.grid / s.n_ct) * kUnitRows),
+          k_full(s.k_full), r_last(s.r_last)
     {
-        if (it < k_full * kUnitRows) {
-            ui = it / kUnitRows;
-            sub = it % kUnitRows;
-            len = kUnitRows;
-        } else {
-            const int t = it - k_full * kUnitRows;
-            ui = k_full + t / r_last;
-            sub = t % r_last;
-            len = r_last;
-        }
+        ct = s.cta % s.n_ct;
+        rt0 = (s.cta / s.n_ct) * kUnitRows;
+        len = k_full > 0 ? kUnitRows : r_last;
     }
-    __device__ int ct_of_unit(int ui) const { return (cta + ui * grid) % n_ct; }
-    __device__ int rt0_of_unit(int ui) const { return ((cta + ui * grid) / n_ct) * kUnitRows; }
+    __device__ int rtile() const { return rt0 + sub; }
+    // Step to the next unit (the builders walk units, not tiles).
+    __device__ void next_unit()
+    {
+        sub = 0;
+        ++ui;
+        ct += step_ct;
+        rt0 += step_rt;
+        if (ct >= n_ct) {
+            ct -= n_ct;
+            rt0 += kUnitRows;
+        }
+        len = ui < k_full ? kUnitRows : r_last;
+    }
+    __device__ void next()
+    {
+        if (++sub == len) next_unit();
+    }
 };
 
 // cur += part, element-wise in fp32 (round to nearest), two at a time with the packed add.
@@ -112,7 +139,6 @@ __global__ void __launch_bounds__(kColThreads, 1)
     uint8_t *code_tiles = smem;                       // two 2 KB staging buffers per epilogue warp
     uint8_t *stages = smem + kColStageOffset;
     uint8_t *bmat = smem + kColBOffset;
-    float *rt = reinterpret_cast<float *>(smem + kColRtOffset);   // R^ as fp32, [n][k]
     float2 *inv_tab = reinterpret_cast<float2 *>(smem + kColInvOffset);   // [slot][channel] (1/L, residual)
     Bars *bars = reinterpret_cast<Bars *>(smem + kColBarOffset);
     volatile int *abort = &bars->abort;
@@ -133,17 +159,19 @@ __global__ void __launch_bounds__(kColThreads, 1)
     if (warp == kTmaWarp) {
         if (lane == 0) {
             const uint64_t pol = ptx::policy_evict_first();
-            int it = 0;
-            for (; it < sched.n_tiles; ++it) {
-                const int s = it % kColStages;
-                if (!wait_bar(&bars->empty[s], ((it / kColStages) & 1) ^ 1, abort, status)) break;
-                int ui, sub, len;
-                sched.at(it, ui, sub, len);
-                const int ctile = sched.ct_of_unit(ui), rtile = sched.rt0_of_unit(ui) + sub;
+            TileCursor cur(sched);
+            int it = 0, s = 0, ph = 1;
+            for (; it < sched.n_tiles; ++it, cur.next()) {
+                // stage s is free once the epilogue has seen the MMAs that read it complete
+                if (!wait_bar(&bars->empty[s], ph, abort, status)) break;
                 const uint32_t full = ptx::smem_addr(&bars->full[s]);
                 const uint32_t dst = ptx::smem_addr(stages + s * kColStageBytes);
                 ptx::mbar_arrive_expect_tx(full, kColStageBytes);
-                ptx::tma_load_2d(dst, &tmap_x, ctile * kColTileCols, rtile * kTileM, full, pol);
+                ptx::tma_load_2d(dst, &tmap_x, cur.ct * kColTileCols, cur.rtile() * kTileM, full, pol);
+                if (++s == kColStages) {
+                    s = 0;
+                    ph ^= 1;
+                }
             }
             drain_loads(bars, kColStages, it, status);
         }
@@ -151,15 +179,14 @@ __global__ void __launch_bounds__(kColThreads, 1)
         if (lane == 0) {
             constexpr uint32_t idesc = ptx::idesc_bf16_f32(128, kColN);
             const uint32_t b_base0 = ptx::smem_addr(bmat);
-            for (int it = 0; it < sched.n_tiles; ++it) {
-                const int s = it % kColStages;
-                const int a = it % kColAcc;
-                int ui, sub, len;
-                sched.at(it, ui, sub, len);
-                const int slot = ui & 1;
-                if (!wait_bar(&bars->full[s], (it / kColStages) & 1, abort, status)) break;
-                if (!wait_bar(&bars->acc_empty[a], ((it / kColAcc) & 1) ^ 1, abort, status)) break;
-                if (sub == 0 && !wait_bar(&bars->b_full[slot], (ui >> 1) & 1, abort, status)) break;
+            TileCursor cur(sched);
+            int s = 0, s_ph = 0;
+            for (int it = 0; it < sched.n_tiles; ++it, cur.next()) {
+                const int a = it & (kColAcc - 1);
+                const int slot = cur.ui & 1;
+                if (!wait_bar(&bars->full[s], s_ph, abort, status)) break;
+                if (!wait_bar(&bars->acc_empty[a], ((it >> 1) & 1) ^ 1, abort, status)) break;
+                if (cur.sub == 0 && !wait_bar(&bars->b_full[slot], (cur.ui >> 1) & 1, abort, status)) break;
                 ptx::tc_fence_after();
                 // Descriptors built once per tile; each MMA adds a compile-time offset to the
                 // start-address field (16-byte units; addresses stay below 256 KB, so no carry).
@@ -173,26 +200,33 @@ __global__ void __launch_bounds__(kColThreads, 1)
                         ptx::mma_bf16(d_base + j * kColN, ad0 + ((j * 64 + kh * 32) >> 4),
                                       bd0 + ((j * kBGroupBytes + kh * 32) >> 4), idesc, kh);
                 }
-                ptx::mma_commit(ptx::smem_addr(&bars->empty[s]));
+                // one commit: the epilogue learns of the tile and frees its shared-memory stage
                 ptx::mma_commit(ptx::smem_addr(&bars->acc_full[a]));
-                if (sub == len - 1) ptx::mma_commit(ptx::smem_addr(&bars->b_empty[slot]));
+                if (cur.sub == cur.len - 1) ptx::mma_commit(ptx::smem_addr(&bars->b_empty[slot]));
+                if (++s == kColStages) {
+                    s = 0;
+                    s_ph ^= 1;
+                }
             }
             drain_mmas(bars, status);
         }
     } else if (warp >= kBuildWarp0) {
-        // Builders: R^ in fp32, transposed to [n][k]; then per tile 1/Lambda of its 64
-        // channels (a reciprocal plus its FMA residual, so R*(1/Lambda) is good to about
-        // an ulp), then the two B_g = diag(1/Lambda_g) R^ split three ways into bf16.
-        // The weights' side (lam_mul) uses Lambda itself: B_g = diag(Lambda_g) R^.
+        // Builders: thread bt owns column n = bt % 32 of R^ and the k-chunk c = bt / 32 (k = 8c..8c+7)
+        // for both groups of every tile, so its eight R^ values live in registers.  Per unit: 1/Lambda
+        // of the tile's 64 channels (a reciprocal plus its FMA residual, so R*(1/Lambda) is good to
+        // about an ulp) into shared memory, then per group the eight entries of B_g = diag(1/Lambda_g) R^
+        // split three ways into bf16, stored to B rows n, 32 + n and 64 + n (16-byte chunk c; 64-byte
+        // swizzle: chunk c of row r sits at chunk c ^ ((r >> 1) & 3)).  The weights' side (lam_mul)
+        // uses Lambda itself: B_g = diag(Lambda_g) R^.
         const int bt = threadIdx.x - kBuildWarp0 * 32;   // 0..127
         constexpr int kB = kColBuildWarps * 32;
-        for (int i = bt; i < 32 * 32; i += kB) {
-            const int k = i >> 5, n = i & 31;
-            rt[n * 32 + k] = __bfloat162float(__ushort_as_bfloat16(rhat_at(args, k, n)));
-        }
-        ptx::named_bar_sync(3, kB);
+        const int bn = bt & 31, bc = bt >> 5;
+        float rr[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) rr[e] = __bfloat162float(__ushort_as_bfloat16(rhat_at(args, bc * 8 + e, bn)));
+        TileCursor cur(sched);
         int built0 = -1, built1 = -1;   // column tile whose B_g each slot holds
-        for (int ui = 0; ui < sched.n_units_cta; ++ui) {
+        for (int ui = 0; ui < sched.n_units_cta; ++ui, cur.next_unit()) {
             const int slot = ui & 1;
             // one thread waits (bounded) for the slot; the verdict goes to all builders
             // (the flag alternates per unit, so a slow reader never sees the next unit's value)
@@ -200,7 +234,7 @@ __global__ void __launch_bounds__(kColThreads, 1)
             __syncwarp();
             ptx::named_bar_sync(3, kB);
             if (!*reinterpret_cast<volatile int *>(&bars->bl_ok[ui & 1])) break;
-            const int ct = sched.ct_of_unit(ui);
+            const int ct = cur.ct;
             if ((slot ? built1 : built0) != ct) {
                 if (slot)
                     built1 = ct;
@@ -224,39 +258,37 @@ __global__ void __launch_bounds__(kColThreads, 1)
                 }
                 ptx::named_bar_sync(3, kB);
                 uint8_t *bs = bmat + slot * kBSlotBytes;
-                // 2 groups x 32 rows (n) x 4 chunks of 8 k = 256 chunk tasks.  Part p of row n
-                // goes to B row p * 32 + n (64-byte swizzle: 16-byte chunk c of row r sits at
-                // chunk c ^ ((r >> 1) & 3)).
-                for (int task = bt; task < kColTileG * 32 * 4; task += kB) {
-                    const int j = task >> 7, n = (task >> 2) & 31, c = task & 3;
+#pragma unroll
+                for (int j = 0; j < kColTileG; ++j) {
+                    const float4 *iv4 = reinterpret_cast<const float4 *>(inv + j * 32 + bc * 8);
                     uint32_t hw[4], mw[4], lw[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
+                    for (int e2 = 0; e2 < 4; ++e2) {
+                        const float4 iv = iv4[e2];   // (1/L, residual) of k = 8c + 2 e2 and 8c + 2 e2 + 1
                         __nv_bfloat16 h[2], m[2], l[2];
 #pragma unroll
                         for (int u = 0; u < 2; ++u) {
-                            const int k = c * 8 + 2 * e + u;
-                            const float2 iv = inv[j * 32 + k];
-                            const float r = rt[n * 32 + k];
-                            const float val = __fmaf_rn(r, iv.x, __fmul_rn(r, iv.y));   // R / Lambda
+                            const float r = rr[2 * e2 + u];
+                            const float val = __fmaf_rn(r, u ? iv.z : iv.x, __fmul_rn(r, u ? iv.w : iv.y));   // R / Lambda
                             // val = hi + mid + lo to ~24 bits; each residual is exact in fp32
                             h[u] = __float2bfloat16_rn(val);
                             const float r1 = val - __bfloat162float(h[u]);
                             m[u] = __float2bfloat16_rn(r1);
                             l[u] = __float2bfloat16_rn(r1 - __bfloat162float(m[u]));
                         }
-                        hw[e] = pack_bf16x2(h[0], h[1]);
-                        mw[e] = pack_bf16x2(m[0], m[1]);
-                        lw[e] = pack_bf16x2(l[0], l[1]);
+                        hw[e2] = pack_bf16x2(h[0], h[1]);
+                        mw[e2] = pack_bf16x2(m[0], m[1]);
+                        lw[e2] = pack_bf16x2(l[0], l[1]);
                     }
                     uint8_t *bg = bs + j * kBGroupBytes;
-                    const uint32_t rows3[3] = {static_cast<uint32_t>(n), static_cast<uint32_t>(32 + n),
-                                               static_cast<uint32_t>(64 + n)};
                     const uint4 v3[3] = {make_uint4(hw[0], hw[1], hw[2], hw[3]), make_uint4(mw[0], mw[1], mw[2], mw[3]),
                                          make_uint4(lw[0], lw[1], lw[2], lw[3])};
 #pragma unroll
-                    for (int pp = 0; pp < 3; ++pp)
-                        *reinterpret_cast<uint4 *>(bg + rows3[pp] * 64 + ((c ^ ((rows3[pp] >> 1) & 3u)) << 4)) = v3[pp];
+                    for (int pp = 0; pp < 3; ++pp) {
+                        const uint32_t row = static_cast<uint32_t>(pp * 32 + bn);
+                        *reinterpret_cast<uint4 *>(bg + row * 64 + ((static_cast<uint32_t>(bc) ^ ((row >> 1) & 3u)) << 4)) =
+                            v3[pp];
+                    }
                 }
                 ptx::fence_proxy_async_smem();
             }
@@ -274,23 +306,28 @@ __global__ void __launch_bounds__(kColThreads, 1)
         const bool scale_vec = (G % 2 == 0) && ((reinterpret_cast<uintptr_t>(args.scales) & 1) == 0);
         // NVFP4 scales are 2 bytes per group: a tile's 4 bytes go as one word when aligned
         const bool nv_vec = (G % 2 == 0) && ((reinterpret_cast<uintptr_t>(args.scales) & 3) == 0);
-        // Each warp stages its own 32 rows' codes (32 rows x 32 B, plain layout, two buffers)
+        // Each warp stages its own 32 rows' codes (32 rows x 32 B, 32-byte swizzle, two buffers)
         // and stores them with its own TMA store, so the warps of a group never wait for one another.
         const uint32_t wbuf0 = ptx::smem_addr(code_tiles + warp * 2 * kWarpCodeBytes);
         int n_st = 0;
-        for (int it = ewg; it < sched.n_tiles; it += 2) {
-            const int a = it % kColAcc;
+        TileCursor cur(sched);
+        if (ewg) cur.next();
+        // this group's tiles are it = ewg, ewg + 2, ...; tile it used stage it % kColStages
+        int s = ewg;
+        for (int it = ewg; it < sched.n_tiles; it += 2, cur.next(), cur.next()) {
+            const int a = it & (kColAcc - 1);
             int ok = 0;
             if (lane == 0) {
-                ok = wait_bar(&bars->acc_full[a], (it / kColAcc) & 1, abort, status);
+                ok = wait_bar(&bars->acc_full[a], (it >> 1) & 1, abort, status);
+                // the tile's MMAs are complete, so its shared-memory stage can be refilled
+                if (ok && q == 0) ptx::mbar_arrive(ptx::smem_addr(&bars->empty[s]));
                 // this warp's next staging buffer must have been read by the store that used it
                 if constexpr (kCodes) ptx::bulk_wait_group_read1();
             }
+            if ((s += 2) >= kColStages) s -= kColStages;
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
             ptx::tc_fence_after();
-            int ui, sub, len;
-            sched.at(it, ui, sub, len);
-            const int ctile = sched.ct_of_unit(ui), rtile = sched.rt0_of_unit(ui) + sub;
+            const int ctile = cur.ct, rtile = cur.rtile();
             const uint32_t wbuf = wbuf0 + (n_st & 1) * kWarpCodeBytes;
             const int r_local = q * 32 + lane;
             const int64_t row = static_cast<int64_t>(rtile) * kTileM + r_local;
@@ -335,7 +372,8 @@ __global__ void __launch_bounds__(kColThreads, 1)
                 } else if constexpr (kMode == RotOut::QuantNv) {
                     uint32_t w[4];
                     const uint32_t bytes = quantize_group_nv(cur, w, nv_rt, nv_st);
-                    ptx::st_shared_v4(wbuf + lane * (kColTileG * 16) + j * 16, w[0], w[1], w[2], w[3]);
+                    // 32-byte swizzle: chunk j of row lane sits at chunk j ^ ((lane >> 2) & 1)
+                    ptx::st_shared_v4(wbuf + lane * 32 + ((j ^ ((lane >> 2) & 1)) << 4), w[0], w[1], w[2], w[3]);
                     if (nv_vec)
                         sc_word |= bytes << (16 * j);
                     else if (g < G && row_ok)
@@ -343,7 +381,7 @@ __global__ void __launch_bounds__(kColThreads, 1)
                 } else {
                     uint32_t w[4];
                     const uint32_t byte = quantize_group(cur, w);
-                    ptx::st_shared_v4(wbuf + lane * (kColTileG * 16) + j * 16, w[0], w[1], w[2], w[3]);
+                    ptx::st_shared_v4(wbuf + lane * 32 + ((j ^ ((lane >> 2) & 1)) << 4), w[0], w[1], w[2], w[3]);
                     if (scale_vec)
                         sc_word |= byte << (8 * j);
                     else if (g < G && row_ok)
