@@ -98,17 +98,21 @@ using namespace pipe;
 //
 // out = (v * R^T) * Lambda, v = E2M1(code) * 2^e.
 // The same flat group-major pipeline as rotate_flat_kernel, run backwards.
-//   warp 13     TMA: bulk-copies each stage's codes (512 groups x 16 B = 8 KB, contiguous)
-//               into a 3-deep shared-memory ring
-//   warps 4-11  decoders (two per scheduler): each lane takes one group per pass, reads its 16 code bytes
-//               from the ring, decodes them with byte permutes (no table, so no bank
-//               conflicts), scales by 2^e and writes the MMA's A tile (bf16, 64-byte
-//               swizzle).  The values are exact in bf16: two significant bits times a
-//               power of two.  The scale bytes are fetched before the stage's waits.
-//   warp 12     MMA: D[g][k] = sum_n v[g][n] * R^[k][n], so B is R^ as stored (row k,
+//   TMA warp    bulk-copies each stage's codes (512 groups x 16 B = 8 KB, contiguous) and,
+//               when the copy can be 16-byte aligned, the stage's 512 scale bytes into a
+//               3-deep shared-memory ring (a scale byte fetched from global memory just
+//               before its use would expose a DRAM round trip every stage)
+//   decoders    eight warps, two per scheduler: each lane takes one group per pass,
+//               reads its 16 code bytes and its scale byte from the ring, decodes them with
+//               byte permutes (no table, so no bank conflicts), scales by 2^e and writes the
+//               MMA's A tile (bf16, 64-byte swizzle).  The values are exact in bf16: two
+//               significant bits times a power of two.
+//   MMA warp    D[g][k] = sum_n v[g][n] * R^[k][n], so B is R^ as stored (row k,
 //               contiguous n = K-major)
-//   warps 0-3   epilogue, one per TMEM lane quarter, every stage: times Lambda_k, bf16,
-//               per-warp 2 KB TMA stores
+//   epilogue    eight warps in two groups of four (one warp per TMEM lane quarter), the
+//               groups taking alternate stages: times Lambda_k, bf16, per-warp 2 KB TMA
+//               stores.  Four warps, one per lane quarter, left the epilogue the critical
+//               path.
 
 // Lambda reaches the epilogue in one of two ways.  When all of it fits 64 KB (cols <=
 // 16384) and is 16-byte aligned it is copied into shared memory once per CTA; each
@@ -116,23 +120,24 @@ using namespace pipe;
 // viewed as [G][32] is its index mod G).  Otherwise each epilogue warp fetches the
 // Lambda rows of its 32 groups per MMA into a double buffer (the rows of one
 // 128-group MMA hold 128 consecutive column groups, so this is 128 B per group from
-// L2).  The warp split: 4 epilogue warps and 8 decoders, except with per-warp
-// fetches, whose epilogue is the critical path (8 epilogue warps in two groups
-// taking alternate stages, 4 decoders).  All use 14 warps.
+// L2).  The warp split: 8 epilogue warps and 8 decoders (18 warps with the MMA and TMA
+// warps), except with per-warp fetches, whose registers allow 8 epilogue warps and 4
+// decoders (14 warps).
 template <int kLam>
 struct DqSplit {
-    static constexpr int kEpi = kLam == 1 ? 8 : 4;
+    static constexpr int kEpi = 8;
     static constexpr int kDec0 = kEpi;
-    static constexpr int kDec = 12 - kEpi;
+    static constexpr int kDec = kLam == 1 ? 4 : 8;
+    static constexpr int kMma = kDec0 + kDec;
+    static constexpr int kTma = kMma + 1;
+    static constexpr int kThreads = (kTma + 1) * 32;
 };
-constexpr int kDqMmaWarp = 12;
-constexpr int kDqTmaWarp = 13;
-constexpr int kDqThreads = (kDqTmaWarp + 1) * 32;   // 448
 constexpr int kDqStages = 3;
 constexpr int kDqStageGroups = 512;                 // 4 MMAs of 128 groups
 constexpr int kDqStageBytes = kDqStageGroups * 64;
 constexpr int kDqCStages = 3;                       // codes ring
 constexpr int kDqCodeBytes = kDqStageGroups * 16;   // 8 KB of codes per stage
+constexpr int kDqCSlotBytes = kDqCodeBytes + kDqStageGroups;   // a ring slot: the codes, then the scale bytes
 constexpr int kDqAcc = 4;
 constexpr int kDqAccCols = 128;
 constexpr int kDqOutBuf = 32 * 64;                 // one epilogue warp's 32 output groups (2 KB)
@@ -145,7 +150,7 @@ __host__ __device__ constexpr int dq_lam_bytes(int epi, int lam)
 }
 __host__ __device__ constexpr int dq_smem_bytes(int epi, int lam)
 {
-    return kDqStages * kDqStageBytes + kBMatBytes + kDqCStages * kDqCodeBytes + dq_out_bytes(epi) +
+    return kDqStages * kDqStageBytes + kBMatBytes + kDqCStages * kDqCSlotBytes + dq_out_bytes(epi) +
            dq_lam_bytes(epi, lam) + 512 + 128 + 1024;
 }
 static_assert(dq_smem_bytes(DqSplit<0>::kEpi, 0) <= 232448 && dq_smem_bytes(DqSplit<1>::kEpi, 1) <= 232448 &&
@@ -166,7 +171,7 @@ __device__ __forceinline__ uint32_t hmul2_bits(uint32_t a, __nv_bfloat162 s)
 // resident in shared memory for the whole kernel (G <= kDqLamTableRows, 16-byte aligned).
 constexpr int kDqLamTableRows = 512;   // 64 KB: cols <= 16384
 template <int kLam>
-__global__ void __launch_bounds__(kDqThreads, 1)
+__global__ void __launch_bounds__(DqSplit<kLam>::kThreads, 1)
     dequant_rot_kernel(const __grid_constant__ CUtensorMap tmap_out, const uint4 *__restrict__ codes,
                        const uint8_t *__restrict__ scales, int64_t n_groups, int64_t G,
                        const uint16_t *__restrict__ rhat, const float *__restrict__ lambda, unsigned int *status)
@@ -177,7 +182,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     uint8_t *cring = bmat + kBMatBytes;                                  // codes ring
     constexpr bool kLambda = kLam != 0;
     using W = DqSplit<kLam>;
-    uint8_t *outbuf = cring + kDqCStages * kDqCodeBytes;                 // epilogue staging
+    uint8_t *outbuf = cring + kDqCStages * kDqCSlotBytes;                 // epilogue staging
     uint8_t *lambuf = outbuf + dq_out_bytes(W::kEpi);                    // epilogue Lambda rows
     Bars *bars = reinterpret_cast<Bars *>(lambuf + dq_lam_bytes(W::kEpi, kLam));
     uint64_t *c_full = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(bars) + 512);
@@ -194,9 +199,9 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         }
     }
     const uint32_t tmem_base = kernel_setup(
-        bars, SetupCfg{kDqStages, kDqAcc, W::kDec, W::kDec * 32, kDqMmaWarp}, &tmap_out, nullptr);
+        bars, SetupCfg{kDqStages, kDqAcc, W::kDec, W::kDec * 32, W::kMma}, &tmap_out, nullptr);
 
-    if (warp == kDqTmaWarp) {
+    if (warp == W::kTma) {
         if (lane == 0) {
             const uint64_t pol = ptx::policy_evict_first();
             int it = 0;
@@ -206,9 +211,14 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                 const int64_t g0 = static_cast<int64_t>(c) * kDqStageGroups;
                 const int64_t n = n_groups - g0 < kDqStageGroups ? n_groups - g0 : kDqStageGroups;
                 const uint32_t bar = ptx::smem_addr(&c_full[cs]);
-                ptx::mbar_arrive_expect_tx(bar, static_cast<uint32_t>(n) * 16u);
-                ptx::bulk_load(ptx::smem_addr(cring + cs * kDqCodeBytes), codes + g0, static_cast<uint32_t>(n) * 16u,
+                // the stage's scale bytes ride along when that copy can be 16-byte aligned
+                const bool sc_bulk = ((reinterpret_cast<uintptr_t>(scales + g0) & 15) == 0) && (n % 16) == 0;
+                ptx::mbar_arrive_expect_tx(bar, static_cast<uint32_t>(n) * (sc_bulk ? 17u : 16u));
+                ptx::bulk_load(ptx::smem_addr(cring + cs * kDqCSlotBytes), codes + g0, static_cast<uint32_t>(n) * 16u,
                                bar, pol);
+                if (sc_bulk)
+                    ptx::bulk_load(ptx::smem_addr(cring + cs * kDqCSlotBytes + kDqCodeBytes), scales + g0,
+                                   static_cast<uint32_t>(n), bar, pol);
             }
             for (int cs = 0; cs < kDqCStages && cs < it; ++cs) {   // the last copies land before exit
                 const int last = it - 1 - ((it - 1 - cs) % kDqCStages);
@@ -230,11 +240,17 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         for (int c = blockIdx.x; c < n_chunks; c += gridDim.x, ++it) {
             const int s = it % kDqStages, cs = it % kDqCStages;
             const int64_t g0 = static_cast<int64_t>(c) * kDqStageGroups;
-            uint32_t sb[kPer];   // scale bytes, in flight while this warp waits
+            // the scale bytes: from the ring when the TMA warp copied them (the same test it
+            // made), otherwise fetched now, in flight while this warp waits
+            const int64_t n_st = n_groups - g0 < kDqStageGroups ? n_groups - g0 : kDqStageGroups;
+            const bool sc_bulk = ((reinterpret_cast<uintptr_t>(scales + g0) & 15) == 0) && (n_st % 16) == 0;
+            uint32_t sb[kPer];
+            if (!sc_bulk) {
 #pragma unroll
-            for (int i = 0; i < kPer; ++i) {
-                const int64_t g = g0 + dt + i * W::kDec * 32;
-                sb[i] = g < n_groups ? static_cast<uint32_t>(__ldg(scales + g)) : 0u;
+                for (int i = 0; i < kPer; ++i) {
+                    const int64_t g = g0 + dt + i * W::kDec * 32;
+                    sb[i] = g < n_groups ? static_cast<uint32_t>(__ldg(scales + g)) : 0u;
+                }
             }
             int ok = 0;
             if (lane == 0)
@@ -242,7 +258,11 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                      wait_bar(&bars->empty[s], ((it / kDqStages) & 1) ^ 1, abort, status);
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
             const uint32_t st = ptx::smem_addr(stages + s * kDqStageBytes);
-            const uint32_t cr = ptx::smem_addr(cring + cs * kDqCodeBytes);
+            const uint32_t cr = ptx::smem_addr(cring + cs * kDqCSlotBytes);
+            if (sc_bulk) {
+#pragma unroll
+                for (int i = 0; i < kPer; ++i) sb[i] = ptx::ld_shared_u8(cr + kDqCodeBytes + dt + i * W::kDec * 32);
+            }
 #pragma unroll
             for (int i = 0; i < kPer; ++i) {
                 const int r = dt + i * W::kDec * 32;   // group row within the stage
@@ -278,7 +298,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(ptx::smem_addr(&bars->full[s]));
         }
-    } else if (warp == kDqMmaWarp) {
+    } else if (warp == W::kMma) {
         if (lane == 0) {
             constexpr uint32_t idesc = ptx::idesc_bf16_f32(128, 32);
             const uint32_t b_base = ptx::smem_addr(bmat);
@@ -368,11 +388,21 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                 __syncwarp();   // the previous stage's reads of both buffers are done
                 fetch_lambda(0);
             }
-            // (one register buffer: with 14 warps an SMSP holds four, so 128 registers a thread)
-#pragma unroll 1
+            // Two register buffers: MMA j + 1's TMEM rows are in flight while MMA j's are converted
+            // and stored (with Lambda fetched per warp, one buffer: that form's registers are full).
+            uint32_t rbuf[2][32];
+            if constexpr (kLam != 1) {
+                ptx::tmem_ld_32cols(t_row, rbuf[0]);
+                ptx::tmem_wait_ld();
+            }
+#pragma unroll
             for (int j = 0; j < 4; ++j) {
-                uint32_t cur[32];
-                ptx::tmem_ld_32cols(t_row + j * 32, cur);
+                uint32_t(&cur)[32] = rbuf[j & 1];
+                if constexpr (kLam != 1) {
+                    if (j + 1 < 4) ptx::tmem_ld_32cols(t_row + (j + 1) * 32, rbuf[(j + 1) & 1]);
+                } else {
+                    ptx::tmem_ld_32cols(t_row + j * 32, cur);
+                }
                 const int64_t g0 = g_warp + j * 128;   // this warp's first group of MMA j
                 const float *lrows = lrows2 + (j & 1) * 32 * 32;
                 if constexpr (kLam == 1) {
@@ -387,7 +417,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                 }
                 const int rj = kLam == 2 ? (row_lane + j * 128) % Gi : 0;   // this lane's Lambda row
                 const float *ltab = reinterpret_cast<const float *>(lambuf) + rj * 32;
-                ptx::tmem_wait_ld();
+                if constexpr (kLam == 1) ptx::tmem_wait_ld();
                 // times Lambda_k (channels of this group, two per packed multiply), then round to
                 // bf16 pairs; without Lambda the fp32 values are rounded as they are
                 uint32_t o[16];
@@ -420,6 +450,9 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                     ptx::bulk_commit_group();
                 }
                 ++nstore;
+                if constexpr (kLam != 1) {
+                    if (j + 1 < 4) ptx::tmem_wait_ld();   // MMA j + 1's rows, for the next pass
+                }
             }
             ptx::tc_fence_before();
             __syncwarp();
@@ -427,7 +460,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         }
         if (lane == 0) ptx::bulk_wait_group0();   // stores done before the CTA's shared memory goes
     }
-    kernel_teardown(tmem_base, kDqMmaWarp);
+    kernel_teardown(tmem_base, W::kMma);
 }
 
 
@@ -446,13 +479,13 @@ cudaError_t launch_dequant_rot(const CUtensorMap &tmap_out, const uint8_t *codes
     if (!status) return cudaErrorInvalidSymbol;
     const uint4 *c4 = reinterpret_cast<const uint4 *>(codes);
     if (!lambda)
-        return launch_pdl(dequant_rot_kernel<0>, grid, kDqThreads, dq_smem_bytes(DqSplit<0>::kEpi, 0), stream,
+        return launch_pdl(dequant_rot_kernel<0>, grid, DqSplit<0>::kThreads, dq_smem_bytes(DqSplit<0>::kEpi, 0), stream,
                           tmap_out, c4, scales, n_groups, G, rhat, lambda, status);
     // all of Lambda fits the per-warp buffers' space (and can be copied in 16-byte pieces): keep it resident
     if (G <= kDqLamTableRows && (reinterpret_cast<uintptr_t>(lambda) & 15) == 0)
-        return launch_pdl(dequant_rot_kernel<2>, grid, kDqThreads, dq_smem_bytes(DqSplit<2>::kEpi, 2), stream,
+        return launch_pdl(dequant_rot_kernel<2>, grid, DqSplit<2>::kThreads, dq_smem_bytes(DqSplit<2>::kEpi, 2), stream,
                           tmap_out, c4, scales, n_groups, G, rhat, lambda, status);
-    return launch_pdl(dequant_rot_kernel<1>, grid, kDqThreads, dq_smem_bytes(DqSplit<1>::kEpi, 1), stream,
+    return launch_pdl(dequant_rot_kernel<1>, grid, DqSplit<1>::kThreads, dq_smem_bytes(DqSplit<1>::kEpi, 1), stream,
                       tmap_out, c4, scales, n_groups, G, rhat, lambda, status);
 }
 
