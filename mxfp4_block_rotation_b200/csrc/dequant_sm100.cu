@@ -103,10 +103,12 @@ using namespace pipe;
 //               3-deep shared-memory ring (a scale byte fetched from global memory just
 //               before its use would expose a DRAM round trip every stage)
 //   decoders    eight warps, two per scheduler: each lane takes one group per pass,
-//               reads its 16 code bytes and its scale byte from the ring, decodes them with
-//               byte permutes (no table, so no bank conflicts), scales by 2^e and writes the
-//               MMA's A tile (bf16, 64-byte swizzle).  The values are exact in bf16: two
-//               significant bits times a power of two.
+//               reads its 16 code bytes (and, with Lambda, its scale byte) from the ring,
+//               decodes them with byte permutes (no table, so no bank conflicts), with Lambda
+//               scales them by 2^e, and writes the MMA's A tile (bf16, 64-byte swizzle).  The
+//               values are exact in bf16: two significant bits times a power of two.  Without
+//               Lambda the epilogue applies 2^e to the fp32 sums instead (exact, the same
+//               values), which moves work off the decoders, that form's critical path.
 //   MMA warp    D[g][k] = sum_n v[g][n] * R^[k][n], so B is R^ as stored (row k,
 //               contiguous n = K-major)
 //   epilogue    eight warps in two groups of four (one warp per TMEM lane quarter), the
@@ -211,8 +213,10 @@ __global__ void __launch_bounds__(DqSplit<kLam>::kThreads, 1)
                 const int64_t g0 = static_cast<int64_t>(c) * kDqStageGroups;
                 const int64_t n = n_groups - g0 < kDqStageGroups ? n_groups - g0 : kDqStageGroups;
                 const uint32_t bar = ptx::smem_addr(&c_full[cs]);
-                // the stage's scale bytes ride along when that copy can be 16-byte aligned
-                const bool sc_bulk = ((reinterpret_cast<uintptr_t>(scales + g0) & 15) == 0) && (n % 16) == 0;
+                // the stage's scale bytes ride along when that copy can be 16-byte aligned (without
+                // Lambda the epilogue applies the scales and fetches them itself)
+                const bool sc_bulk =
+                    kLambda && ((reinterpret_cast<uintptr_t>(scales + g0) & 15) == 0) && (n % 16) == 0;
                 ptx::mbar_arrive_expect_tx(bar, static_cast<uint32_t>(n) * (sc_bulk ? 17u : 16u));
                 ptx::bulk_load(ptx::smem_addr(cring + cs * kDqCSlotBytes), codes + g0, static_cast<uint32_t>(n) * 16u,
                                bar, pol);
@@ -243,9 +247,10 @@ __global__ void __launch_bounds__(DqSplit<kLam>::kThreads, 1)
             // the scale bytes: from the ring when the TMA warp copied them (the same test it
             // made), otherwise fetched now, in flight while this warp waits
             const int64_t n_st = n_groups - g0 < kDqStageGroups ? n_groups - g0 : kDqStageGroups;
-            const bool sc_bulk = ((reinterpret_cast<uintptr_t>(scales + g0) & 15) == 0) && (n_st % 16) == 0;
-            uint32_t sb[kPer];
-            if (!sc_bulk) {
+            const bool sc_bulk =
+                kLambda && ((reinterpret_cast<uintptr_t>(scales + g0) & 15) == 0) && (n_st % 16) == 0;
+            uint32_t sb[kPer] = {};
+            if (kLambda && !sc_bulk) {
 #pragma unroll
                 for (int i = 0; i < kPer; ++i) {
                     const int64_t g = g0 + dt + i * W::kDec * 32;
@@ -279,8 +284,11 @@ __global__ void __launch_bounds__(DqSplit<kLam>::kThreads, 1)
                     for (int q = 0; q < 4; ++q) {
                         uint32_t v[4];
                         ptx::e2m1x8_to_bf16(cws[q], v);
+                        // without Lambda the E2M1 values go in as they are and the epilogue
+                        // multiplies the fp32 result by 2^e (the decoders are that form's
+                        // critical path, the epilogue has room); with Lambda the decoders scale
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) w[4 * q + e] = hmul2_bits(v[e], s2);
+                        for (int e = 0; e < 4; ++e) w[4 * q + e] = kLambda ? hmul2_bits(v[e], s2) : v[e];
                     }
                 } else {
 #pragma unroll
@@ -348,6 +356,15 @@ __global__ void __launch_bounds__(DqSplit<kLam>::kThreads, 1)
         for (int c = blockIdx.x; c < n_chunks; c += gridDim.x, ++it) {
             if (W::kEpi == 8 && (it & 1) != ewg) continue;
             const int a = it % kDqAcc;
+            // without Lambda: this lane's group's scale byte for each of the stage's four MMAs,
+            // in flight while the warp waits
+            uint32_t esc[4] = {127u, 127u, 127u, 127u};
+            if constexpr (!kLambda) {
+                const int64_t gl = static_cast<int64_t>(c) * kDqStageGroups + q * 32 + lane;
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (gl + j * 128 < n_groups) esc[j] = __ldg(scales + gl + j * 128);
+            }
             int ok = 0;
             if (lane == 0) ok = wait_bar(&bars->acc_full[a], (it / kDqAcc) & 1, abort, status);
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
@@ -421,10 +438,20 @@ __global__ void __launch_bounds__(DqSplit<kLam>::kThreads, 1)
                 // times Lambda_k (channels of this group, two per packed multiply), then round to
                 // bf16 pairs; without Lambda the fp32 values are rounded as they are
                 uint32_t o[16];
+                // 2^(byte - 127) as fp32 (byte 0 is the subnormal 2^-127, 0xFF is NaN): the sums
+                // of exact products times a power of two, the same fp32 values as summing the
+                // scaled products
+                const uint32_t eb = esc[j];
+                const float esf = __uint_as_float(eb == 0xFFu ? 0x7FC00000u : (eb == 0u ? 0x00400000u : (eb << 23)));
+                const float2 es2 = make_float2(esf, esf);
 #pragma unroll
                 for (int k4 = 0; k4 < 8; ++k4) {
                     float2 v0 = make_float2(__uint_as_float(cur[4 * k4]), __uint_as_float(cur[4 * k4 + 1]));
                     float2 v1 = make_float2(__uint_as_float(cur[4 * k4 + 2]), __uint_as_float(cur[4 * k4 + 3]));
+                    if constexpr (!kLambda) {
+                        v0 = __fmul2_rn(v0, es2);
+                        v1 = __fmul2_rn(v1, es2);
+                    }
                     if constexpr (kLambda) {
                         const float4 l4 =
                             kLam == 1 ? *reinterpret_cast<const float4 *>(lrows + lane * 32 + ((k4 ^ (lane & 7)) << 2))
