@@ -630,7 +630,7 @@ def run_row_only(args):
     dev = torch.device("cuda:0")
     stream = torch.cuda.current_stream(dev)
     cfg, what, _ = CONFIG_ROWS[args.row]
-    w = synth.make_config(cfg)
+    w = synth.make_config(cfg, rows=args.row_rows)   # the row's recipe, optionally cut to fewer rows
     keep = None
     if what == "dequantize":
         keep = mxq.smooth_rotate_quantize(w.x.to(dev), w.rhat.to(dev), None if w.lam is None else w.lam.to(dev),
@@ -738,6 +738,8 @@ def main(argv=None):
     ap.add_argument("--row", choices=sorted(CONFIG_ROWS),
                     help="profiling aid: run only this per_config row, --steps launches after 5 warm-up "
                          "launches, print its time and exit")
+    ap.add_argument("--row-rows", type=int, default=None,
+                    help="with --row: the same recipe with this many rows (smaller cases for full ncu captures)")
     ap.add_argument("--gemm-only", metavar="M,N,K",
                     help="profiling aid: run only the MXFP4 GEMM, 3 + --steps launches on random operands of this "
                          "shape (bf16 out), print its time and exit")

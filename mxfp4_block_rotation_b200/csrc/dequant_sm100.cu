@@ -352,8 +352,21 @@ __global__ void __launch_bounds__(DqSplit<kLam>::kThreads, 1)
             ptx::cp_async_wait<0>();
             ptx::named_bar_sync(1, W::kEpi * 32);
         }
+        // Lambda rows by additions (no division per stage): the row of group g is g mod G, and
+        // this lane's group (this warp's first, with per-warp fetches) advances by
+        // kDqStageGroups x gridDim.x per CTA stage and by 128 per MMA.
+        const int step_c = kLambda ? static_cast<int>((static_cast<int64_t>(kDqStageGroups) * gridDim.x) % G) : 0;
+        const int step_j = kLambda ? static_cast<int>(128 % G) : 0;
+        int row_c = kLambda ? static_cast<int>((static_cast<int64_t>(blockIdx.x) * kDqStageGroups + q * 32 +
+                                                (kLam == 2 ? lane : 0)) % G)
+                            : 0;
         int it = 0, nstore = 0;
         for (int c = blockIdx.x; c < n_chunks; c += gridDim.x, ++it) {
+            const int row_stage = row_c;   // Lambda row of this stage's MMA 0 (lane's, or warp's first)
+            if constexpr (kLambda) {
+                row_c += step_c;
+                if (row_c >= Gi) row_c -= Gi;
+            }
             if (W::kEpi == 8 && (it & 1) != ewg) continue;
             const int a = it % kDqAcc;
             // without Lambda: this lane's group's scale byte for each of the stage's four MMAs,
@@ -377,11 +390,14 @@ __global__ void __launch_bounds__(DqSplit<kLam>::kThreads, 1)
             // next MMA's rows are in flight while this one is processed.
             // Column groups are taken mod G by subtraction (at most one step once G >= 128): a
             // division per stage instead of nine per fetch.
-            const int col_warp = kLam == 1 ? static_cast<int>(g_warp % G) : 0;
-            const int row_lane = kLam == 2 ? static_cast<int>((g_warp + lane) % G) : 0;   // Lambda row of MMA 0
+            const int col_warp = kLam == 1 ? row_stage : 0;
+            int rj = kLam == 2 ? row_stage : 0;   // this lane's Lambda row for MMA j, advanced per MMA
             auto fetch_lambda = [&](int j) {
-                int col0 = col_warp + j * 128;
-                while (col0 >= Gi) col0 -= Gi;
+                int col0 = col_warp;
+                for (int t = 0; t < j; ++t) {
+                    col0 += step_j;
+                    if (col0 >= Gi) col0 -= Gi;
+                }
                 float *dst_rows = lrows2 + (j & 1) * 32 * 32;
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
@@ -432,7 +448,6 @@ __global__ void __launch_bounds__(DqSplit<kLam>::kThreads, 1)
                     }
                     __syncwarp();
                 }
-                const int rj = kLam == 2 ? (row_lane + j * 128) % Gi : 0;   // this lane's Lambda row
                 const float *ltab = reinterpret_cast<const float *>(lambuf) + rj * 32;
                 if constexpr (kLam == 1) ptx::tmem_wait_ld();
                 // times Lambda_k (channels of this group, two per packed multiply), then round to
@@ -479,6 +494,10 @@ __global__ void __launch_bounds__(DqSplit<kLam>::kThreads, 1)
                 ++nstore;
                 if constexpr (kLam != 1) {
                     if (j + 1 < 4) ptx::tmem_wait_ld();   // MMA j + 1's rows, for the next pass
+                }
+                if constexpr (kLam == 2) {
+                    rj += step_j;
+                    if (rj >= Gi) rj -= Gi;
                 }
             }
             ptx::tc_fence_before();
