@@ -19,7 +19,7 @@ LIB = os.path.join(HERE, "libmxq.so")
 SOURCES = ["mxq_api.cu", "rotate_flat_sm100.cu", "rotate_cols_sm100.cu", "dequant_sm100.cu", "status_sm100.cu",
            "error_sm100.cu", "noalloc_sm100.cu", "search_sm100.cu", "rotate_block_sm100.cu",
            "gemm_sm100.cu"]
-HEADERS = ["mxq_internal.h", "sm100_ptx.cuh", "sm100_bulk.cuh", "pipeline_sm100.cuh",
+HEADERS = ["mxq_internal.h", "sm100_ptx.cuh", "sm100_bulk.cuh", "pipeline_sm100.cuh", "tile_order.cuh",
            os.path.join("..", "..", "include", "mxq.h")]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2"]
