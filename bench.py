@@ -53,7 +53,7 @@ _COMMON = [_CSRC + "pipeline_sm100.cuh", _CSRC + "sm100_ptx.cuh", _CSRC + "sm100
 # reported only while the hash of these files matches the one it was taken with.
 KERNEL_SOURCES = {
     "rotate_flat": [_CSRC + "rotate_flat_sm100.cu"] + _COMMON,
-    "rotate_cols": [_CSRC + "rotate_cols_sm100.cu"] + _COMMON,
+    "rotate_cols": [_CSRC + "rotate_cols_sm100.cu", _CSRC + "tile_order.cuh"] + _COMMON,
     "dequant_rot": [_CSRC + "dequant_sm100.cu"] + _COMMON,
 }
 # profiles/traffic_<row>.json: ncu's dram__bytes_read.sum + dram__bytes_write.sum of one launch
@@ -694,7 +694,8 @@ def run_e2e(mxq, w, rhat, dev, stream, args, dist):
 
 
 def run_gemm_only(args):
-    """The consumer GEMM alone at a chosen shape (small cases for ncu captures)."""
+    """The consumer GEMM alone at a chosen shape (small cases for ncu captures): MXFP4, or NVFP4
+    with --gemm-nvfp4 (E4M3 block scales in [0x30, 0x40), tensor scales 0.5 and 0.25)."""
     import mxfp4_block_rotation_b200 as mxq
     M, N, K = (int(v) for v in args.gemm_only.split(","))
     dev = torch.device("cuda:0")
@@ -702,20 +703,37 @@ def run_gemm_only(args):
     g.manual_seed(0)
     a = torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device=dev, generator=g)
     b = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device=dev, generator=g)
-    sfa = mxq.scales_to_mma_layout(torch.randint(120, 134, (M, K // 32), dtype=torch.uint8, device=dev, generator=g))
-    sfb = mxq.scales_to_mma_layout(torch.randint(120, 134, (N, K // 32), dtype=torch.uint8, device=dev, generator=g))
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    if args.gemm_nvfp4:
+        sfa = mxq.nvfp4_scales_to_mma_layout(
+            torch.randint(0x30, 0x40, (M, K // 16), dtype=torch.uint8, device=dev, generator=g))
+        sfb = mxq.nvfp4_scales_to_mma_layout(
+            torch.randint(0x30, 0x40, (N, K // 16), dtype=torch.uint8, device=dev, generator=g))
+        ta = torch.tensor([0.5], device=dev)
+        tb = torch.tensor([0.25], device=dev)
+
+        def gemm():
+            mxq.nvfp4_gemm(a, sfa, ta, b, sfb, tb, out=y)
+    else:
+        sfa = mxq.scales_to_mma_layout(
+            torch.randint(120, 134, (M, K // 32), dtype=torch.uint8, device=dev, generator=g))
+        sfb = mxq.scales_to_mma_layout(
+            torch.randint(120, 134, (N, K // 32), dtype=torch.uint8, device=dev, generator=g))
+
+        def gemm():
+            mxq.mxfp4_gemm(a, sfa, b, sfb, out=y)
     for _ in range(3):
-        mxq.mxfp4_gemm(a, sfa, b, sfb, out=y)
+        gemm()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(args.steps):
-        mxq.mxfp4_gemm(a, sfa, b, sfb, out=y)
+        gemm()
     e1.record()
     torch.cuda.synchronize(dev)
     mxq.sync_check()
     ms = e0.elapsed_time(e1) / max(args.steps, 1)
-    print(json.dumps({"gemm": [M, N, K], "ms": ms, "TFLOP/s": 2.0 * M * N * K / (ms * 1e-3) / 1e12}), flush=True)
+    print(json.dumps({"gemm": [M, N, K], "format": "nvfp4" if args.gemm_nvfp4 else "mxfp4", "ms": ms,
+                      "TFLOP/s": 2.0 * M * N * K / (ms * 1e-3) / 1e12}), flush=True)
     return 0
 
 
@@ -743,6 +761,7 @@ def main(argv=None):
     ap.add_argument("--gemm-only", metavar="M,N,K",
                     help="profiling aid: run only the MXFP4 GEMM, 3 + --steps launches on random operands of this "
                          "shape (bf16 out), print its time and exit")
+    ap.add_argument("--gemm-nvfp4", action="store_true", help="with --gemm-only: the NVFP4 GEMM instead")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -1,5 +1,5 @@
-// tile_order.cuh -- the tile order of the column-tiled kernels (rotate_cols_sm100.cu,
-// dequant_cols_sm100.cu): tiles of 128 rows x one column tile, walked in units of
+// tile_order.cuh -- the tile order of the column-tiled smoothing kernel
+// (rotate_cols_sm100.cu): tiles of 128 rows x one column tile, walked in units of
 // kUnitRows row blocks of one column tile, so that one build of the column tile's B
 // operand serves a whole unit.
 #pragma once
