@@ -508,7 +508,18 @@ def run_extras(mxq, w, xs, rhat, outs, dev, stream, k=300):
     res["downproj_layer_quantize_plus_gemm"] = {
         "what": "the whole layer: rotate+quantise X, scale layout, MXFP4 GEMM (3 launches)", "ms": ms,
         "TFLOP/s": flops / (ms * 1e-3) / 1e12}
-    del wt, cb, sb, sfa, sfb, y
+    # the same layer with the quantiser writing its scales in the MMA layout (2 launches)
+    sfa2 = [torch.empty_like(sfa) for _ in range(2)]
+
+    def layer_fused(i):
+        c = outs[i & 1][0]
+        mxq.smooth_rotate_quantize_mma(xs[i & 1], rhat, None, codes=c, sf=sfa2[i & 1], stream=stream)
+        mxq.mxfp4_gemm(c, sfa2[i & 1], cb, sfb, out=y, stream=stream)
+    ms = _timed(layer_fused, max(1, min(50, k)), stream, dev)
+    res["downproj_layer_fused_scales_plus_gemm"] = {
+        "what": "the whole layer with the quantiser writing MMA-layout scales, then the MXFP4 GEMM (2 launches)",
+        "ms": ms, "TFLOP/s": flops / (ms * 1e-3) / 1e12}
+    del wt, cb, sb, sfa, sfb, y, sfa2
     # the offline rotation search on the same activations, smoothed: K = 128 steps, 64 angles per pair
     sws = torch.empty(mxq.lib().mxq_rotation_search_workspace_bytes(rows, cols, 32), dtype=torch.uint8, device=dev)
     found = {}

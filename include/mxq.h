@@ -99,6 +99,27 @@ mxq_status mxq_smooth_rotate_quantize(const void *X_bf16, int64_t rows, int64_t 
                                       void *stream);
 
 /*
+ * mxq_smooth_rotate_quantize with the scales written straight into the layout
+ * the block-scaled MMA reads them in (DuQuant++ write-up §3.3: the rotated
+ * activations feed the MXFP4 linear; §1 and §5.4: Blackwell's native MXFP4
+ * tensor cores), so mxq_mxfp4_gemm takes them with no layout pass between.
+ * The codes and the scale bytes are the same as mxq_smooth_rotate_quantize's;
+ * out_scales_mma holds exactly what mxq_scales_to_mma_layout makes of its
+ * scales, padding included (rows past the matrix in the last 128-row block and
+ * k-blocks past cols/32 read 0: the call zeroes the buffer first when the
+ * shape has such padding, so the kernel itself writes only the scales).
+ *
+ *   X_bf16, rows, cols, Rhat_bf16, Lambda_or_null, out_codes_u8_packed, stream
+ *                       as mxq_smooth_rotate_quantize
+ *   out_scales_mma      out  mxq_scales_mma_bytes(rows, cols) bytes, 16-byte aligned
+ * Errors as mxq_smooth_rotate_quantize.
+ */
+mxq_status mxq_smooth_rotate_quantize_mma(const void *X_bf16, int64_t rows, int64_t cols,
+                                          const void *Rhat_bf16, const float *Lambda_or_null,
+                                          uint8_t *out_codes_u8_packed, uint8_t *out_scales_mma,
+                                          void *stream);
+
+/*
  * Same inputs as mxq_smooth_rotate_quantize.  Writes the rotated fp32 values
  * Y = X * Lambda^-1 * R^ (§3.3) instead of quantising them.  It checks the
  * intermediate precision; the quantiser decides on these same values.

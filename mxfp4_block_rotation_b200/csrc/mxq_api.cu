@@ -335,7 +335,7 @@ mxq_status rotate_common(const void *X, int64_t rows, int64_t cols, const void *
                          uint64_t out1_bytes, mxq::RotOut mode, void *stream, int blk = 32, int lam_mul = 0,
                          const float *nv_scale = nullptr)
 {
-    const bool quant = mode == mxq::RotOut::Quant || mode == mxq::RotOut::QuantNv;
+    const bool quant = mode == mxq::RotOut::Quant || mode == mxq::RotOut::QuantNv || mode == mxq::RotOut::QuantMma;
     mxq_status st = check_shape(rows, cols);
     if (st != MXQ_OK) return st;
     if (blk != 16 && blk != 32 && blk != 64 && blk != 128) return bad("block must be 16, 32, 64 or 128");
@@ -349,6 +349,7 @@ mxq_status rotate_common(const void *X, int64_t rows, int64_t cols, const void *
         if (!aligned(nv_scale, 4)) return bad("tensor scale must be 4-byte aligned");
         if (!aligned(out1, 2)) return bad("NVFP4 scales must be 2-byte aligned");
     }
+    if (mode == mxq::RotOut::QuantMma && !aligned(out1, 16)) return bad("MMA-layout scales must be 16-byte aligned");
     if (!aligned(X, 16)) return bad("X must be 16-byte aligned");
     if (!aligned(R, 2)) return bad("Rhat must be 2-byte aligned");
     if (lam && !aligned(lam, 4)) return bad("Lambda must be 4-byte aligned");
@@ -394,13 +395,26 @@ mxq_status rotate_common(const void *X, int64_t rows, int64_t cols, const void *
     args.lambda = lam;
     args.rows = rows;
     args.cols = cols;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (quant) {
         args.codes = static_cast<uint8_t *>(out0);
-        args.scales = static_cast<uint8_t *>(out1);
+        if (mode == mxq::RotOut::QuantMma) {
+            args.sf_mma = static_cast<uint8_t *>(out1);
+            // the kernels write every scale of the matrix; the atoms' rows past it (rows not a
+            // multiple of 128) and groups past it (cols/32 not a multiple of 4) must read 0
+            if (rows % 128 || (cols / 32) % 4) {
+                const cudaError_t me = cudaMemsetAsync(out1, 0, out1_bytes, s);
+                if (me != cudaSuccess) {
+                    note_cuda(me, "cudaMemsetAsync(MMA-layout scales)");
+                    return MXQ_ERR_CUDA;
+                }
+            }
+        } else {
+            args.scales = static_cast<uint8_t *>(out1);
+        }
     } else {
         args.y = static_cast<float *>(out0);
     }
-    const cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = blk > 32           ? mxq::launch_rotate_block(map_a, args, blk, mode, sms, s)
                     : lam == nullptr ? mxq::launch_rotate_flat(map_a, args, mode, sms, s)
                                      : mxq::launch_rotate_cols(map_a, map_c, args, mode, sms, s);
@@ -427,6 +441,16 @@ mxq_status mxq_smooth_rotate_quantize(const void *X_bf16, int64_t rows, int64_t 
     const uint64_t ns = rows > 0 && cols > 0 ? static_cast<uint64_t>(rows) * (cols / 32) : 0;
     return rotate_common(X_bf16, rows, cols, Rhat_bf16, Lambda_or_null, out_codes_u8_packed, nc, 16,
                          out_scales_e8m0, ns, mxq::RotOut::Quant, stream);
+}
+
+mxq_status mxq_smooth_rotate_quantize_mma(const void *X_bf16, int64_t rows, int64_t cols, const void *Rhat_bf16,
+                                          const float *Lambda_or_null, uint8_t *out_codes_u8_packed,
+                                          uint8_t *out_scales_mma, void *stream)
+{
+    const uint64_t nc = rows > 0 && cols > 0 ? static_cast<uint64_t>(rows) * cols / 2 : 0;
+    const uint64_t ns = rows > 0 && cols > 0 && cols % 32 == 0 ? mxq_scales_mma_bytes(rows, cols) : 0;
+    return rotate_common(X_bf16, rows, cols, Rhat_bf16, Lambda_or_null, out_codes_u8_packed, nc, 16,
+                         out_scales_mma, ns, mxq::RotOut::QuantMma, stream);
 }
 
 mxq_status mxq_smooth_rotate_f32(const void *X_bf16, int64_t rows, int64_t cols, const void *Rhat_bf16,

@@ -16,7 +16,10 @@ enum : unsigned int {
 // Output mode of the fused rotate kernels: packed codes + scales, the rotated
 // fp32 values, the per-group MXFP4 quantisation error (plus per-warp partial
 // sums for its mean), or NVFP4 (codes + one E4M3 scale per 16 values).
-enum class RotOut { Quant, F32, Err, QuantNv };
+// Quant: MXFP4 codes and row-major scales; QuantMma: the same codes with the scales in
+// the block-scaled MMA's atom layout (args.sf_mma); F32: the rotated values; Err: the
+// per-group quantisation error; QuantNv: NVFP4.
+enum class RotOut { Quant, F32, Err, QuantNv, QuantMma };
 
 struct RotArgs {
     const uint16_t *rhat;      // bf16 [32][32], row-major [k][n]; [16][16] when rblk == 16
@@ -26,6 +29,8 @@ struct RotArgs {
     const float *lambda;       // fp32 [cols] or nullptr
     uint8_t *codes;            // [rows, cols/2]   (Quant)
     uint8_t *scales;           // [rows, cols/32]  (Quant)
+    uint8_t *sf_mma;           // QuantMma: the scales in the block-scaled MMA's atom layout
+                               // (mxq_scales_to_mma_layout's output)
     float *y;                  // [rows, cols]     (F32)
     float *err;                // [rows, cols/32]  (Err; may be null)
     double *partials;          // per-warp error sums (Err): see rotate_*_partials()

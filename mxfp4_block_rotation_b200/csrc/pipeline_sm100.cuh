@@ -119,6 +119,15 @@ __device__ __forceinline__ uint32_t quantize_group(const uint32_t (&r)[32], uint
     return byte;
 }
 
+// Byte offset of the E8M0 scale of row r, group g in the block-scaled MMA's scale layout:
+// 512-byte atoms of 128 rows x 4 groups, ordered by row block and then group block
+// (kb4 = ceil(G / 4) atoms per row block); inside an atom, row r and group g sit at byte
+// 16 (r % 32) + 4 ((r / 32) % 4) + g % 4.
+__device__ __forceinline__ int64_t sf_mma_offset(int64_t r, int64_t g, int64_t kb4)
+{
+    return ((r >> 7) * kb4 + (g >> 2)) * 512 + ((r & 31) << 4) + (((r >> 5) & 3) << 2) + (g & 3);
+}
+
 // MXFP4 of one group as in quantize_group, plus its normalised quantisation error
 // ||Q(y) - y||_2 / ||y||_2.  With u = y * 2^-e the power of two cancels:
 // error = ||Q(u) - u|| / ||u||, where Q(u) is u's E2M1 value.  An all-zero group

@@ -76,7 +76,7 @@ __global__ void __launch_bounds__(kColThreads, 1)
     rotate_cols_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_codes,
                        const RotArgs args, unsigned int *status)
 {
-    constexpr bool kCodes = kMode == RotOut::Quant || kMode == RotOut::QuantNv;   // codes via staging + TMA
+    constexpr bool kCodes = kMode == RotOut::Quant || kMode == RotOut::QuantNv || kMode == RotOut::QuantMma;   // codes via staging + TMA
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align_1k(smem_raw);
     uint8_t *code_tiles = smem;                       // two 2 KB staging buffers per epilogue warp
@@ -325,7 +325,7 @@ __global__ void __launch_bounds__(kColThreads, 1)
                     uint32_t w[4];
                     const uint32_t byte = quantize_group(cur, w);
                     ptx::st_shared_v4(wbuf + lane * 32 + ((j ^ ((lane >> 2) & 1)) << 4), w[0], w[1], w[2], w[3]);
-                    if (scale_vec)
+                    if (kMode == RotOut::QuantMma || scale_vec)
                         sc_word |= byte << (8 * j);
                     else if (g < G && row_ok)
                         args.scales[row * G + g] = static_cast<uint8_t>(byte);
@@ -340,6 +340,17 @@ __global__ void __launch_bounds__(kColThreads, 1)
                     // two groups x two E4M3 bytes: 4 bytes at group 2 ctile of the row
                     if (nv_vec && row_ok)
                         reinterpret_cast<uint32_t *>(args.scales)[(row * G) / 2 + ctile] = sc_word;
+                } else if constexpr (kMode == RotOut::QuantMma) {
+                    // the tile's groups 2 ctile and 2 ctile + 1 share one 4-byte word of the atom
+                    // (from an even byte): one 16-bit store, or one byte for a last odd group
+                    if (row_ok) {
+                        const int64_t g0 = static_cast<int64_t>(ctile) * kColTileG;
+                        uint8_t *dst = args.sf_mma + sf_mma_offset(row, g0, (G + 3) >> 2);
+                        if (g0 + 1 < G)
+                            *reinterpret_cast<uint16_t *>(dst) = static_cast<uint16_t>(sc_word);
+                        else
+                            *dst = static_cast<uint8_t>(sc_word);
+                    }
                 } else if (scale_vec && row_ok) {
                     *reinterpret_cast<uint16_t *>(args.scales + row * G + static_cast<int64_t>(ctile) * kColTileG) =
                         static_cast<uint16_t>(sc_word);
@@ -375,6 +386,9 @@ cudaError_t launch_rotate_cols(const CUtensorMap &tmap_x, const CUtensorMap &tma
     if (!status) return cudaErrorInvalidSymbol;
     if (mode == RotOut::Quant)
         return launch_pdl(rotate_cols_kernel<RotOut::Quant>, grid, kColThreads, kColSmemBytes, stream, tmap_x,
+                          tmap_codes, args, status);
+    if (mode == RotOut::QuantMma)
+        return launch_pdl(rotate_cols_kernel<RotOut::QuantMma>, grid, kColThreads, kColSmemBytes, stream, tmap_x,
                           tmap_codes, args, status);
     if (mode == RotOut::Err)
         return launch_pdl(rotate_cols_kernel<RotOut::Err>, grid, kColThreads, kColSmemBytes, stream, tmap_x,

@@ -150,6 +150,14 @@ __global__ void __launch_bounds__(FlatRoles<kMode>::kThreadsF, 1)
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * kFlatAccCols;
             const int64_t g_lane = static_cast<int64_t>(c) * kFlatStageGroups + q * 32 + lane;
             double err_acc = 0.0;   // Err mode: this lane's groups, in order
+            // QuantMma: the lane's row and group from one division per stage, then advanced by
+            // 128 groups per MMA with additions (at most one wrap when G >= 128)
+            [[maybe_unused]] const int64_t G = args.cols / 32;
+            [[maybe_unused]] int64_t sf_r = 0, sf_g = 0;
+            if constexpr (kMode == RotOut::QuantMma) {
+                sf_r = g_lane / G;
+                sf_g = g_lane - sf_r * G;
+            }
             // The TMEM load of MMA j+1 is in flight while group j is quantised; fully
             // unrolled so both register buffers stay put.
             uint32_t ra[32], rb[32];
@@ -183,7 +191,17 @@ __global__ void __launch_bounds__(FlatRoles<kMode>::kThreadsF, 1)
                         uint32_t w[4];
                         const uint32_t byte = quantize_group(cur, w);
                         ptx::st_global_v4(args.codes + g * 16, w[0], w[1], w[2], w[3]);
-                        args.scales[g] = static_cast<uint8_t>(byte);
+                        if constexpr (kMode == RotOut::QuantMma)
+                            args.sf_mma[sf_mma_offset(sf_r, sf_g, (G + 3) >> 2)] = static_cast<uint8_t>(byte);
+                        else
+                            args.scales[g] = static_cast<uint8_t>(byte);
+                    }
+                }
+                if constexpr (kMode == RotOut::QuantMma) {
+                    sf_g += 128;
+                    while (sf_g >= G) {
+                        sf_g -= G;
+                        ++sf_r;
                     }
                 }
                 if (j + 1 < kFlatMmas) ptx::tmem_wait_ld();
@@ -216,6 +234,9 @@ cudaError_t launch_rotate_flat(const CUtensorMap &tmap_groups, const RotArgs &ar
     if (mode == RotOut::Quant)
         return launch_pdl(rotate_flat_kernel<RotOut::Quant>, grid, FlatRoles<RotOut::Quant>::kThreadsF, kFlatSmemBytes,
                           stream, tmap_groups, args, status);
+    if (mode == RotOut::QuantMma)
+        return launch_pdl(rotate_flat_kernel<RotOut::QuantMma>, grid, FlatRoles<RotOut::QuantMma>::kThreadsF,
+                          kFlatSmemBytes, stream, tmap_groups, args, status);
     if (mode == RotOut::Err)
         return launch_pdl(rotate_flat_kernel<RotOut::Err>, grid, FlatRoles<RotOut::Err>::kThreadsF, kFlatSmemBytes,
                           stream, tmap_groups, args, status);

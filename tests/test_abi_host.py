@@ -62,6 +62,9 @@ def test_rejects_null_and_misaligned(L):
     assert _q(L, a, 4, 64, a * 5, a * 7 + 2, a * 2, a * 3) == INVALID       # Lambda not 4-B aligned
     assert _q(L, a, 4, 64, a * 5, None, a * 2 + 4, a * 3) == INVALID        # codes not 16-B aligned
     assert L.mxq_smooth_rotate_f32(P(a), 4, 64, P(a * 5), None, P(a * 2 + 8), None) == INVALID
+    # scales in the MMA layout: a null or not 16-byte-aligned buffer
+    assert L.mxq_smooth_rotate_quantize_mma(P(a), 4, 64, P(a * 5), None, P(a * 2), None, None) == INVALID
+    assert L.mxq_smooth_rotate_quantize_mma(P(a), 4, 64, P(a * 5), None, P(a * 2), P(a * 3 + 4), None) == INVALID
     # dequantize: Lambda without R^, misaligned output
     assert L.mxq_dequantize(P(a), P(a * 2), 4, 64, None, P(a * 3), P(a * 4), None) == INVALID
     assert L.mxq_dequantize(P(a), P(a * 2), 4, 64, None, None, P(a * 4 + 2), None) == INVALID

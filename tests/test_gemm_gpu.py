@@ -177,6 +177,49 @@ def test_scale_layout_matches_oracle(rows, K):
     assert np.array_equal(got.cpu().numpy(), oracle.scales_to_mma(sc))
 
 
+@pytest.mark.parametrize("rows,cols,use_lam", [(300, 2048, False), (300, 2048, True), (129, 96, False),
+                                               (129, 96, True), (37, 16416, False), (40, 16416, True),
+                                               (256, 4096, False)])
+def test_quantize_with_mma_scales(rows, cols, use_lam):
+    # The quantiser writing its scales straight into the MMA layout.  The buffer is poisoned
+    # first, so every byte must be written: the scales where the oracle's layout function puts
+    # the row-major call's scales, and 0 in the padding (rows past a multiple of 128, groups
+    # past a multiple of 4).  The codes equal the row-major call's, and both calls' output
+    # meets the quantiser's parity rule against the oracle.  Shapes cover the flat kernel
+    # (no Lambda, G < 128 and odd G) and the column-tiled one (a last tile of one group).
+    x = synth.random_bf16(rows, cols, seed=rows * 7 + cols, scale=1.0)
+    rhat = synth.rhat_tensor(synth.haar_orthogonal(rows + 1))
+    lam = synth.random_lambda(cols, seed=rows) if use_lam else None
+    xd, rd, ld = x.to(DEV), rhat.to(DEV), None if lam is None else lam.to(DEV)
+    c0, s0 = mxq.smooth_rotate_quantize(xd, rd, ld)
+    n = int(mxq.lib().mxq_scales_mma_bytes(rows, cols))
+    sf = torch.full((n,), 0xAB, dtype=torch.uint8, device=DEV)
+    c1, sf1 = mxq.smooth_rotate_quantize_mma(xd, rd, ld, sf=sf)
+    mxq.sync_check()
+    assert torch.equal(c1, c0)
+    s0n = s0.cpu().numpy()
+    assert np.array_equal(sf1.cpu().numpy(), oracle.scales_to_mma(s0n))
+    _parity.check_quant(synth.bf16_bits(x), synth.bf16_bits(rhat), None if lam is None else lam.numpy(),
+                        c1.cpu().numpy(), s0n)
+
+
+def test_gemm_on_mma_scales_equals_layout_pass():
+    # The layer without the layout pass gives the same output bits as with it.
+    rows, cols, n_out = 300, 1024, 520
+    x = synth.random_bf16(rows, cols, seed=5, scale=1.0)
+    wt = synth.random_bf16(n_out, cols, seed=6, scale=1.0 / np.sqrt(cols))
+    rhat = synth.rhat_tensor(synth.haar_orthogonal(12)).to(DEV)
+    lam = synth.random_lambda(cols, seed=13).to(DEV)
+    cb, sb = mxq.weight_rotate_quantize(wt.to(DEV), rhat, lam)
+    for lam_a in (None, lam):
+        c0, s0 = mxq.smooth_rotate_quantize(x.to(DEV), rhat, lam_a)
+        c1, sf1 = mxq.smooth_rotate_quantize_mma(x.to(DEV), rhat, lam_a)
+        y0 = mxq.mxfp4_gemm(c0, mxq.scales_to_mma_layout(s0), cb, sb)
+        y1 = mxq.mxfp4_gemm(c1, sf1, cb, sb)
+        mxq.sync_check()
+        assert torch.equal(y0, y1)
+
+
 # ---------------------------------------------------------------- the NVFP4 consumer GEMM
 
 def _rand_nv(rng, rows, K):
