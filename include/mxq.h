@@ -224,6 +224,21 @@ mxq_status mxq_mxfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales_mma, c
  *   products it scales NaN.
  */
 size_t mxq_nvfp4_scales_mma_bytes(int64_t rows, int64_t K);
+
+/*
+ * mxq_smooth_rotate_quantize_nvfp4 with the E4M3 scales written straight into
+ * the layout mxq_nvfp4_gemm reads (what mxq_nvfp4_scales_to_mma_layout makes of
+ * the row-major scales, padding included; zeroed first only when the shape has
+ * padding), so the NVFP4 GEMM takes them with no layout pass between.
+ *   X_bf16, rows, cols, Rhat_bf16, Lambda_or_null, tensor_scale_f32,
+ *   out_codes_u8_packed, stream   as mxq_smooth_rotate_quantize_nvfp4
+ *   out_scales_mma      out  mxq_nvfp4_scales_mma_bytes(rows, cols) bytes, 16-byte aligned
+ * Errors as mxq_smooth_rotate_quantize_nvfp4.
+ */
+mxq_status mxq_smooth_rotate_quantize_nvfp4_mma(const void *X_bf16, int64_t rows, int64_t cols,
+                                                const void *Rhat_bf16, const float *Lambda_or_null,
+                                                const float *tensor_scale_f32, uint8_t *out_codes_u8_packed,
+                                                uint8_t *out_scales_mma, void *stream);
 mxq_status mxq_nvfp4_scales_to_mma_layout(const uint8_t *scales, int64_t rows, int64_t K, uint8_t *out,
                                           void *stream);
 mxq_status mxq_nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales_mma, const float *a_tensor_scale,

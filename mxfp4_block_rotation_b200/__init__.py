@@ -23,7 +23,7 @@ import torch
 
 __all__ = [
     "MxqError", "smooth_rotate_quantize", "smooth_rotate_quantize_mma", "smooth_rotate_quantize_nvfp4",
-    "smooth_rotate_f32",
+    "smooth_rotate_quantize_nvfp4_mma", "smooth_rotate_f32",
     "weight_rotate_quantize", "rotate_quantize_block", "rotate_block_f32", "scales_to_mma_layout",
     "mxfp4_gemm", "nvfp4_scales_to_mma_layout", "nvfp4_gemm", "dequantize", "quant_error", "rotation_search",
     "sync_check", "selftest_bounded_wait",
@@ -63,6 +63,8 @@ def lib() -> ctypes.CDLL:
         L.mxq_smooth_rotate_quantize.restype = I
         L.mxq_smooth_rotate_quantize_mma.argtypes = [P, I64, I64, P, P, P, P, P]
         L.mxq_smooth_rotate_quantize_mma.restype = I
+        L.mxq_smooth_rotate_quantize_nvfp4_mma.argtypes = [P, I64, I64, P, P, P, P, P, P]
+        L.mxq_smooth_rotate_quantize_nvfp4_mma.restype = I
         L.mxq_smooth_rotate_f32.argtypes = [P, I64, I64, P, P, P, P]
         L.mxq_smooth_rotate_f32.restype = I
         L.mxq_rotate_quantize_block.argtypes = [P, I64, I64, I, P, P, P, P, P]
@@ -205,6 +207,32 @@ def smooth_rotate_quantize_mma(x: torch.Tensor, rhat: torch.Tensor, lam: Optiona
     st = lib().mxq_smooth_rotate_quantize_mma(_ptr(x), rows, cols, _ptr(rhat), _ptr(lam), _ptr(codes), _ptr(sf),
                                               _stream(dev, stream))
     _check(st, "mxq_smooth_rotate_quantize_mma")
+    return codes, sf
+
+
+def smooth_rotate_quantize_nvfp4_mma(x: torch.Tensor, rhat: torch.Tensor, tensor_scale: torch.Tensor,
+                                     lam: Optional[torch.Tensor] = None, *, codes: Optional[torch.Tensor] = None,
+                                     sf: Optional[torch.Tensor] = None,
+                                     stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """NVFP4(X · Λ⁻¹ · R̂) -> (codes uint8 [rows, cols/2], E4M3 scales in the block-scaled MMA layout:
+    flat uint8 of mxq_nvfp4_scales_mma_bytes(rows, cols)), ready for nvfp4_gemm with no layout pass."""
+    dev = _inputs(x, rhat, lam)
+    _need(tensor_scale, "tensor_scale", torch.float32, dev)
+    if tensor_scale.numel() != 1:
+        raise ValueError("tensor_scale must hold one float")
+    rows, cols = x.shape
+    n = int(lib().mxq_nvfp4_scales_mma_bytes(rows, cols))
+    if codes is None:
+        codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+    if sf is None:
+        sf = torch.empty(n, dtype=torch.uint8, device=dev)
+    _need(codes, "codes", torch.uint8, dev)
+    _need(sf, "sf", torch.uint8, dev)
+    if sf.numel() < n:
+        raise ValueError(f"sf needs {n} bytes")
+    st = lib().mxq_smooth_rotate_quantize_nvfp4_mma(_ptr(x), rows, cols, _ptr(rhat), _ptr(lam), _ptr(tensor_scale),
+                                                    _ptr(codes), _ptr(sf), _stream(dev, stream))
+    _check(st, "mxq_smooth_rotate_quantize_nvfp4_mma")
     return codes, sf
 
 

@@ -335,7 +335,8 @@ mxq_status rotate_common(const void *X, int64_t rows, int64_t cols, const void *
                          uint64_t out1_bytes, mxq::RotOut mode, void *stream, int blk = 32, int lam_mul = 0,
                          const float *nv_scale = nullptr)
 {
-    const bool quant = mode == mxq::RotOut::Quant || mode == mxq::RotOut::QuantNv || mode == mxq::RotOut::QuantMma;
+    const bool quant = mode == mxq::RotOut::Quant || mxq::rot_nvfp4(mode) || mode == mxq::RotOut::QuantMma;
+    const bool sf_mma = mxq::rot_sf_mma(mode);
     mxq_status st = check_shape(rows, cols);
     if (st != MXQ_OK) return st;
     if (blk != 16 && blk != 32 && blk != 64 && blk != 128) return bad("block must be 16, 32, 64 or 128");
@@ -343,13 +344,13 @@ mxq_status rotate_common(const void *X, int64_t rows, int64_t cols, const void *
     if (lam && blk > 32) return bad("Lambda is supported with blocks of 16 or 32 columns only");
     if (rows == 0 || cols == 0) return MXQ_OK;   // nothing is read or written
     if (!X || !R || !out0 || (quant && !out1)) return bad("null pointer");
-    if (mode == mxq::RotOut::QuantNv) {
+    if (mxq::rot_nvfp4(mode)) {
         if (blk != 32) return bad("NVFP4 takes a 32x32 Rhat");
         if (!nv_scale) return bad("null pointer");
         if (!aligned(nv_scale, 4)) return bad("tensor scale must be 4-byte aligned");
         if (!aligned(out1, 2)) return bad("NVFP4 scales must be 2-byte aligned");
     }
-    if (mode == mxq::RotOut::QuantMma && !aligned(out1, 16)) return bad("MMA-layout scales must be 16-byte aligned");
+    if (sf_mma && !aligned(out1, 16)) return bad("MMA-layout scales must be 16-byte aligned");
     if (!aligned(X, 16)) return bad("X must be 16-byte aligned");
     if (!aligned(R, 2)) return bad("Rhat must be 2-byte aligned");
     if (lam && !aligned(lam, 4)) return bad("Lambda must be 4-byte aligned");
@@ -398,11 +399,13 @@ mxq_status rotate_common(const void *X, int64_t rows, int64_t cols, const void *
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (quant) {
         args.codes = static_cast<uint8_t *>(out0);
-        if (mode == mxq::RotOut::QuantMma) {
+        if (sf_mma) {
             args.sf_mma = static_cast<uint8_t *>(out1);
             // the kernels write every scale of the matrix; the atoms' rows past it (rows not a
-            // multiple of 128) and groups past it (cols/32 not a multiple of 4) must read 0
-            if (rows % 128 || (cols / 32) % 4) {
+            // multiple of 128) and scale columns past it (cols/32 for MXFP4, cols/16 for NVFP4,
+            // not a multiple of 4) must read 0
+            const int64_t sc_cols = mode == mxq::RotOut::QuantNvMma ? cols / 16 : cols / 32;
+            if (rows % 128 || sc_cols % 4) {
                 const cudaError_t me = cudaMemsetAsync(out1, 0, out1_bytes, s);
                 if (me != cudaSuccess) {
                     note_cuda(me, "cudaMemsetAsync(MMA-layout scales)");
@@ -451,6 +454,17 @@ mxq_status mxq_smooth_rotate_quantize_mma(const void *X_bf16, int64_t rows, int6
     const uint64_t ns = rows > 0 && cols > 0 && cols % 32 == 0 ? mxq_scales_mma_bytes(rows, cols) : 0;
     return rotate_common(X_bf16, rows, cols, Rhat_bf16, Lambda_or_null, out_codes_u8_packed, nc, 16,
                          out_scales_mma, ns, mxq::RotOut::QuantMma, stream);
+}
+
+mxq_status mxq_smooth_rotate_quantize_nvfp4_mma(const void *X_bf16, int64_t rows, int64_t cols,
+                                                const void *Rhat_bf16, const float *Lambda_or_null,
+                                                const float *tensor_scale_f32, uint8_t *out_codes_u8_packed,
+                                                uint8_t *out_scales_mma, void *stream)
+{
+    const uint64_t nc = rows > 0 && cols > 0 ? static_cast<uint64_t>(rows) * cols / 2 : 0;
+    const uint64_t ns = rows > 0 && cols > 0 && cols % 32 == 0 ? mxq_nvfp4_scales_mma_bytes(rows, cols) : 0;
+    return rotate_common(X_bf16, rows, cols, Rhat_bf16, Lambda_or_null, out_codes_u8_packed, nc, 16,
+                         out_scales_mma, ns, mxq::RotOut::QuantNvMma, stream, 32, 0, tensor_scale_f32);
 }
 
 mxq_status mxq_smooth_rotate_f32(const void *X_bf16, int64_t rows, int64_t cols, const void *Rhat_bf16,

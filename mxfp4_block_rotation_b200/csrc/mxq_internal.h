@@ -18,8 +18,11 @@ enum : unsigned int {
 // sums for its mean), or NVFP4 (codes + one E4M3 scale per 16 values).
 // Quant: MXFP4 codes and row-major scales; QuantMma: the same codes with the scales in
 // the block-scaled MMA's atom layout (args.sf_mma); F32: the rotated values; Err: the
-// per-group quantisation error; QuantNv: NVFP4.
-enum class RotOut { Quant, F32, Err, QuantNv, QuantMma };
+// per-group quantisation error; QuantNv: NVFP4; QuantNvMma: NVFP4 with its E4M3 scales in
+// the same atom layout (one atom column per 16-value block).
+enum class RotOut { Quant, F32, Err, QuantNv, QuantMma, QuantNvMma };
+__host__ __device__ constexpr bool rot_nvfp4(RotOut m) { return m == RotOut::QuantNv || m == RotOut::QuantNvMma; }
+__host__ __device__ constexpr bool rot_sf_mma(RotOut m) { return m == RotOut::QuantMma || m == RotOut::QuantNvMma; }
 
 struct RotArgs {
     const uint16_t *rhat;      // bf16 [32][32], row-major [k][n]; [16][16] when rblk == 16
@@ -29,8 +32,8 @@ struct RotArgs {
     const float *lambda;       // fp32 [cols] or nullptr
     uint8_t *codes;            // [rows, cols/2]   (Quant)
     uint8_t *scales;           // [rows, cols/32]  (Quant)
-    uint8_t *sf_mma;           // QuantMma: the scales in the block-scaled MMA's atom layout
-                               // (mxq_scales_to_mma_layout's output)
+    uint8_t *sf_mma;           // QuantMma, QuantNvMma: the scales in the block-scaled MMA's atom
+                               // layout (mxq_scales_to_mma_layout's or mxq_nvfp4_scales_to_mma_layout's output)
     float *y;                  // [rows, cols]     (F32)
     float *err;                // [rows, cols/32]  (Err; may be null)
     double *partials;          // per-warp error sums (Err): see rotate_*_partials()

@@ -76,7 +76,7 @@ __global__ void __launch_bounds__(kColThreads, 1)
     rotate_cols_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_codes,
                        const RotArgs args, unsigned int *status)
 {
-    constexpr bool kCodes = kMode == RotOut::Quant || kMode == RotOut::QuantNv || kMode == RotOut::QuantMma;   // codes via staging + TMA
+    constexpr bool kCodes = kMode == RotOut::Quant || rot_nvfp4(kMode) || kMode == RotOut::QuantMma;   // codes via staging + TMA
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align_1k(smem_raw);
     uint8_t *code_tiles = smem;                       // two 2 KB staging buffers per epilogue warp
@@ -242,7 +242,7 @@ __global__ void __launch_bounds__(kColThreads, 1)
         const int ewg = warp >> 2;
         // NVFP4: the tensor scale s_t and r_t = 1 / (6 s_t), once per thread
         float nv_st = 0.0f, nv_rt = 0.0f;
-        if constexpr (kMode == RotOut::QuantNv) {
+        if constexpr (rot_nvfp4(kMode)) {
             nv_st = *args.nv_scale;
             nv_rt = __frcp_rn(__fmul_rn(6.0f, nv_st));
         }
@@ -312,12 +312,12 @@ __global__ void __launch_bounds__(kColThreads, 1)
                         if (args.err) args.err[row * G + g] = e;
                         err_acc += static_cast<double>(e);
                     }
-                } else if constexpr (kMode == RotOut::QuantNv) {
+                } else if constexpr (rot_nvfp4(kMode)) {
                     uint32_t w[4];
                     const uint32_t bytes = quantize_group_nv(cur, w, nv_rt, nv_st);
                     // 32-byte swizzle: chunk j of row lane sits at chunk j ^ ((lane >> 2) & 1)
                     ptx::st_shared_v4(wbuf + lane * 32 + ((j ^ ((lane >> 2) & 1)) << 4), w[0], w[1], w[2], w[3]);
-                    if (nv_vec)
+                    if (kMode == RotOut::QuantNvMma || nv_vec)
                         sc_word |= bytes << (16 * j);
                     else if (g < G && row_ok)
                         reinterpret_cast<uint16_t *>(args.scales)[row * G + g] = static_cast<uint16_t>(bytes);
@@ -340,6 +340,17 @@ __global__ void __launch_bounds__(kColThreads, 1)
                     // two groups x two E4M3 bytes: 4 bytes at group 2 ctile of the row
                     if (nv_vec && row_ok)
                         reinterpret_cast<uint32_t *>(args.scales)[(row * G) / 2 + ctile] = sc_word;
+                } else if constexpr (kMode == RotOut::QuantNvMma) {
+                    // the tile's blocks 4 ctile .. 4 ctile + 3 fill one 4-byte word of the atom: one
+                    // 32-bit store, or 16 bits for a last odd group
+                    if (row_ok) {
+                        const int64_t g0 = static_cast<int64_t>(ctile) * kColTileG;
+                        uint8_t *dst = args.sf_mma + sf_mma_offset(row, 2 * g0, (2 * G + 3) >> 2);
+                        if (g0 + 1 < G)
+                            *reinterpret_cast<uint32_t *>(dst) = sc_word;
+                        else
+                            *reinterpret_cast<uint16_t *>(dst) = static_cast<uint16_t>(sc_word);
+                    }
                 } else if constexpr (kMode == RotOut::QuantMma) {
                     // the tile's groups 2 ctile and 2 ctile + 1 share one 4-byte word of the atom
                     // (from an even byte): one 16-bit store, or one byte for a last odd group
@@ -389,6 +400,9 @@ cudaError_t launch_rotate_cols(const CUtensorMap &tmap_x, const CUtensorMap &tma
                           tmap_codes, args, status);
     if (mode == RotOut::QuantMma)
         return launch_pdl(rotate_cols_kernel<RotOut::QuantMma>, grid, kColThreads, kColSmemBytes, stream, tmap_x,
+                          tmap_codes, args, status);
+    if (mode == RotOut::QuantNvMma)
+        return launch_pdl(rotate_cols_kernel<RotOut::QuantNvMma>, grid, kColThreads, kColSmemBytes, stream, tmap_x,
                           tmap_codes, args, status);
     if (mode == RotOut::Err)
         return launch_pdl(rotate_cols_kernel<RotOut::Err>, grid, kColThreads, kColSmemBytes, stream, tmap_x,

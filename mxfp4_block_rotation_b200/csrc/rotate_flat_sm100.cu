@@ -44,7 +44,7 @@ static_assert(kFlatBoxes >= 1 && kFlatStageGroups % kFlatBoxGroups == 0 && kFlat
 // fourth stage (one accumulator stage each); the others run two groups.
 template <RotOut kMode>
 struct FlatRoles {
-    static constexpr int kGroups = (kMode == RotOut::Err || kMode == RotOut::QuantNv) ? 4 : 2;
+    static constexpr int kGroups = (kMode == RotOut::Err || rot_nvfp4(kMode)) ? 4 : 2;
     static constexpr int kEpi = 4 * kGroups;
     static constexpr int kTma = kEpi;
     static constexpr int kMma = kEpi + 1;
@@ -135,7 +135,7 @@ __global__ void __launch_bounds__(FlatRoles<kMode>::kThreadsF, 1)
         const int ewg = warp >> 2;    // which of the stages (every kGroups-th) this warp group takes
         // NVFP4: the tensor scale s_t and r_t = 1 / (6 s_t), once per thread
         float nv_st = 0.0f, nv_rt = 0.0f;
-        if constexpr (kMode == RotOut::QuantNv) {
+        if constexpr (rot_nvfp4(kMode)) {
             nv_st = *args.nv_scale;
             nv_rt = __frcp_rn(__fmul_rn(6.0f, nv_st));
         }
@@ -150,11 +150,11 @@ __global__ void __launch_bounds__(FlatRoles<kMode>::kThreadsF, 1)
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * kFlatAccCols;
             const int64_t g_lane = static_cast<int64_t>(c) * kFlatStageGroups + q * 32 + lane;
             double err_acc = 0.0;   // Err mode: this lane's groups, in order
-            // QuantMma: the lane's row and group from one division per stage, then advanced by
-            // 128 groups per MMA with additions (at most one wrap when G >= 128)
+            // scales in the MMA layout: the lane's row and group from one division per stage,
+            // then advanced by 128 groups per MMA with additions (at most one wrap when G >= 128)
             [[maybe_unused]] const int64_t G = args.cols / 32;
             [[maybe_unused]] int64_t sf_r = 0, sf_g = 0;
-            if constexpr (kMode == RotOut::QuantMma) {
+            if constexpr (rot_sf_mma(kMode)) {
                 sf_r = g_lane / G;
                 sf_g = g_lane - sf_r * G;
             }
@@ -182,11 +182,15 @@ __global__ void __launch_bounds__(FlatRoles<kMode>::kThreadsF, 1)
                         quantize_group_err(cur, w, e);
                         if (args.err) args.err[g] = e;
                         err_acc += static_cast<double>(e);
-                    } else if constexpr (kMode == RotOut::QuantNv) {
+                    } else if constexpr (rot_nvfp4(kMode)) {
                         uint32_t w[4];
                         const uint32_t bytes = quantize_group_nv(cur, w, nv_rt, nv_st);
                         ptx::st_global_v4(args.codes + g * 16, w[0], w[1], w[2], w[3]);
-                        reinterpret_cast<uint16_t *>(args.scales)[g] = static_cast<uint16_t>(bytes);
+                        if constexpr (kMode == RotOut::QuantNvMma)   // blocks 2g, 2g + 1: one aligned 16-bit word
+                            *reinterpret_cast<uint16_t *>(args.sf_mma + sf_mma_offset(sf_r, 2 * sf_g, (2 * G + 3) >> 2)) =
+                                static_cast<uint16_t>(bytes);
+                        else
+                            reinterpret_cast<uint16_t *>(args.scales)[g] = static_cast<uint16_t>(bytes);
                     } else {
                         uint32_t w[4];
                         const uint32_t byte = quantize_group(cur, w);
@@ -197,7 +201,7 @@ __global__ void __launch_bounds__(FlatRoles<kMode>::kThreadsF, 1)
                             args.scales[g] = static_cast<uint8_t>(byte);
                     }
                 }
-                if constexpr (kMode == RotOut::QuantMma) {
+                if constexpr (rot_sf_mma(kMode)) {
                     sf_g += 128;
                     while (sf_g >= G) {
                         sf_g -= G;
@@ -236,6 +240,9 @@ cudaError_t launch_rotate_flat(const CUtensorMap &tmap_groups, const RotArgs &ar
                           stream, tmap_groups, args, status);
     if (mode == RotOut::QuantMma)
         return launch_pdl(rotate_flat_kernel<RotOut::QuantMma>, grid, FlatRoles<RotOut::QuantMma>::kThreadsF,
+                          kFlatSmemBytes, stream, tmap_groups, args, status);
+    if (mode == RotOut::QuantNvMma)
+        return launch_pdl(rotate_flat_kernel<RotOut::QuantNvMma>, grid, FlatRoles<RotOut::QuantNvMma>::kThreadsF,
                           kFlatSmemBytes, stream, tmap_groups, args, status);
     if (mode == RotOut::Err)
         return launch_pdl(rotate_flat_kernel<RotOut::Err>, grid, FlatRoles<RotOut::Err>::kThreadsF, kFlatSmemBytes,

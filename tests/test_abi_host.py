@@ -65,6 +65,10 @@ def test_rejects_null_and_misaligned(L):
     # scales in the MMA layout: a null or not 16-byte-aligned buffer
     assert L.mxq_smooth_rotate_quantize_mma(P(a), 4, 64, P(a * 5), None, P(a * 2), None, None) == INVALID
     assert L.mxq_smooth_rotate_quantize_mma(P(a), 4, 64, P(a * 5), None, P(a * 2), P(a * 3 + 4), None) == INVALID
+    assert L.mxq_smooth_rotate_quantize_nvfp4_mma(P(a), 4, 64, P(a * 5), None, P(a * 6), P(a * 2), P(a * 3 + 2),
+                                                  None) == INVALID
+    assert L.mxq_smooth_rotate_quantize_nvfp4_mma(P(a), 4, 64, P(a * 5), None, None, P(a * 2), P(a * 3),
+                                                  None) == INVALID   # no tensor scale
     # dequantize: Lambda without R^, misaligned output
     assert L.mxq_dequantize(P(a), P(a * 2), 4, 64, None, P(a * 3), P(a * 4), None) == INVALID
     assert L.mxq_dequantize(P(a), P(a * 2), 4, 64, None, None, P(a * 4 + 2), None) == INVALID

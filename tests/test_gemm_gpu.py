@@ -203,6 +203,30 @@ def test_quantize_with_mma_scales(rows, cols, use_lam):
                         c1.cpu().numpy(), s0n)
 
 
+@pytest.mark.parametrize("rows,cols,use_lam", [(300, 2048, False), (300, 2048, True), (129, 96, False),
+                                               (129, 96, True), (37, 16416, False), (40, 16416, True)])
+def test_nvfp4_quantize_with_mma_scales(rows, cols, use_lam):
+    # NVFP4 with its E4M3 scales written straight into the MMA layout: as for MXFP4, on a
+    # poisoned buffer, against the oracle's layout of the row-major call's scales (the same
+    # atoms over [rows, cols/16]), codes equal, both against the oracle's NVFP4 quantiser.
+    x = synth.random_bf16(rows, cols, seed=rows * 5 + cols, scale=1.0)
+    rhat = synth.rhat_tensor(synth.haar_orthogonal(rows + 2))
+    lam = synth.random_lambda(cols, seed=rows + 1) if use_lam else None
+    xd, rd, ld = x.to(DEV), rhat.to(DEV), None if lam is None else lam.to(DEV)
+    s_t = float(np.float32(float(x.abs().max().float()) * 32 ** 0.5 * (20.0 if use_lam else 1.0) / (6 * 448)))
+    ts = torch.tensor([s_t], dtype=torch.float32, device=DEV)
+    c0, s0 = mxq.smooth_rotate_quantize_nvfp4(xd, rd, ts, ld)
+    n = int(mxq.lib().mxq_nvfp4_scales_mma_bytes(rows, cols))
+    sf = torch.full((n,), 0xAB, dtype=torch.uint8, device=DEV)
+    c1, sf1 = mxq.smooth_rotate_quantize_nvfp4_mma(xd, rd, ts, ld, sf=sf)
+    mxq.sync_check()
+    assert torch.equal(c1, c0)
+    s0n = s0.cpu().numpy()
+    assert np.array_equal(sf1.cpu().numpy(), oracle.scales_to_mma(s0n))
+    _parity.check_nvfp4(synth.bf16_bits(x), synth.bf16_bits(rhat), None if lam is None else lam.numpy(), s_t,
+                        c1.cpu().numpy(), s0n)
+
+
 def test_gemm_on_mma_scales_equals_layout_pass():
     # The layer without the layout pass gives the same output bits as with it.
     rows, cols, n_out = 300, 1024, 520
@@ -218,6 +242,16 @@ def test_gemm_on_mma_scales_equals_layout_pass():
         y1 = mxq.mxfp4_gemm(c1, sf1, cb, sb)
         mxq.sync_check()
         assert torch.equal(y0, y1)
+    # NVFP4: the same with E4M3 scales and tensor scales
+    ts_a = torch.tensor([float(x.abs().max().float()) * 32 ** 0.5 / (6 * 448)], dtype=torch.float32, device=DEV)
+    ts_b = torch.tensor([float(wt.abs().max().float()) * 32 ** 0.5 / (6 * 448)], dtype=torch.float32, device=DEV)
+    ncb, nsb = mxq.smooth_rotate_quantize_nvfp4(wt.to(DEV), rhat, ts_b)
+    nc0, ns0 = mxq.smooth_rotate_quantize_nvfp4(x.to(DEV), rhat, ts_a)
+    nc1, nsf1 = mxq.smooth_rotate_quantize_nvfp4_mma(x.to(DEV), rhat, ts_a)
+    y0 = mxq.nvfp4_gemm(nc0, ns0, ts_a, ncb, nsb, ts_b)
+    y1 = mxq.nvfp4_gemm(nc1, nsf1, ts_a, ncb, nsb, ts_b)
+    mxq.sync_check()
+    assert torch.equal(y0, y1)
 
 
 # ---------------------------------------------------------------- the NVFP4 consumer GEMM
