@@ -179,7 +179,8 @@ def test_scale_layout_matches_oracle(rows, K):
 
 @pytest.mark.parametrize("rows,cols,use_lam", [(300, 2048, False), (300, 2048, True), (129, 96, False),
                                                (129, 96, True), (37, 16416, False), (40, 16416, True),
-                                               (256, 4096, False)])
+                                               (256, 4096, False), (1, 32, False), (1, 32, True),
+                                               (128, 128, True)])
 def test_quantize_with_mma_scales(rows, cols, use_lam):
     # The quantiser writing its scales straight into the MMA layout.  The buffer is poisoned
     # first, so every byte must be written: the scales where the oracle's layout function puts
@@ -204,7 +205,8 @@ def test_quantize_with_mma_scales(rows, cols, use_lam):
 
 
 @pytest.mark.parametrize("rows,cols,use_lam", [(300, 2048, False), (300, 2048, True), (129, 96, False),
-                                               (129, 96, True), (37, 16416, False), (40, 16416, True)])
+                                               (129, 96, True), (37, 16416, False), (40, 16416, True),
+                                               (1, 32, False), (1, 32, True)])
 def test_nvfp4_quantize_with_mma_scales(rows, cols, use_lam):
     # NVFP4 with its E4M3 scales written straight into the MMA layout: as for MXFP4, on a
     # poisoned buffer, against the oracle's layout of the row-major call's scales (the same
