@@ -497,7 +497,31 @@ def run_extras(mxq, w, xs, rhat, outs, dev, stream, k=300):
         "ms": ms, "TFLOP/s": flops / (ms * 1e-3) / 1e12, "peak_TFLOP/s": fp4_peak,
         "frac_of_fp4_peak": flops / (ms * 1e-3) / 1e12 / fp4_peak,
         "peak_source": "measured bf16 burst (MEASURED_PEAKS.json bf16_tflops) x 4, the nominal fp4/bf16 ratio"}
-    del nca, nsa, ncb, nsb, nsfa, nsfb
+    # the NVFP4 layer: quantise X (tensor scale on the device), lay out its scales, GEMM; and with
+    # the quantiser writing its E4M3 scales straight into the MMA layout
+    nv_codes = [torch.empty_like(nca) for _ in range(2)]
+    nv_rows = [torch.empty_like(nsa) for _ in range(2)]
+    nv_sf = [torch.empty_like(nsfa) for _ in range(2)]
+
+    def layer_nv(i):
+        mxq.smooth_rotate_quantize_nvfp4(xs[i & 1], rhat, ts_a, codes=nv_codes[i & 1], scales=nv_rows[i & 1],
+                                         stream=stream)
+        mxq.nvfp4_scales_to_mma_layout(nv_rows[i & 1], out=nv_sf[i & 1], stream=stream)
+        mxq.nvfp4_gemm(nv_codes[i & 1], nv_sf[i & 1], ts_a, ncb, nsfb, ts_b, out=y, stream=stream)
+    ms = _timed(layer_nv, max(1, min(50, k)), stream, dev)
+    res["nvfp4_layer_quantize_plus_gemm"] = {
+        "what": "the NVFP4 layer: rotate+quantise X, scale layout, NVFP4 GEMM (3 launches)", "ms": ms,
+        "TFLOP/s": flops / (ms * 1e-3) / 1e12}
+
+    def layer_nv_fused(i):
+        mxq.smooth_rotate_quantize_nvfp4_mma(xs[i & 1], rhat, ts_a, codes=nv_codes[i & 1], sf=nv_sf[i & 1],
+                                             stream=stream)
+        mxq.nvfp4_gemm(nv_codes[i & 1], nv_sf[i & 1], ts_a, ncb, nsfb, ts_b, out=y, stream=stream)
+    ms = _timed(layer_nv_fused, max(1, min(50, k)), stream, dev)
+    res["nvfp4_layer_fused_scales_plus_gemm"] = {
+        "what": "the NVFP4 layer with the quantiser writing MMA-layout E4M3 scales, then the GEMM (2 launches)",
+        "ms": ms, "TFLOP/s": flops / (ms * 1e-3) / 1e12}
+    del nca, nsa, ncb, nsb, nsfa, nsfb, nv_codes, nv_rows, nv_sf
 
     def layer(i):
         c, s = outs[i & 1]
